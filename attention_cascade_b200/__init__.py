@@ -1,0 +1,284 @@
+"""Python binding of libjev.so (include/jev.h): argument marshalling only.
+
+Every function here has the name of the C entry point it calls.  Tensors are
+torch CUDA tensors (PyTorch supplies device memory and the current stream);
+all computation happens in the library's CUDA kernels.  If the library has not
+been built this module raises at import time: there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+from typing import Optional
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libjev.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m attention_cascade_b200._build` "
+                      "(nvcc, sm_100a) — there is no non-CUDA fallback")
+
+_lib = C.CDLL(LIB_PATH)
+
+JEV_F32, JEV_BF16 = 0, 1
+JEV_DEV_BAD_SEQLENS, JEV_DEV_BAD_HEAD_MAP, JEV_DEV_BAD_TREE, JEV_DEV_WAIT_TIMEOUT, JEV_DEV_BAD_WINDOW = 1, 2, 4, 8, 16
+STATUS_NAMES = {0: "JEV_OK", 1: "JEV_ERR_INVALID_ARG", 2: "JEV_ERR_UNSUPPORTED", 3: "JEV_ERR_WORKSPACE",
+                4: "JEV_ERR_CUDA", 5: "JEV_ERR_DEVICE", 6: "JEV_ERR_CAPACITY"}
+
+
+class JevError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = _lib.jev_last_error().decode(errors="replace")
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}: {msg}")
+
+
+class jev_attn_desc(C.Structure):
+    _fields_ = [("B", C.c_int32), ("Lp", C.c_int32), ("Hq", C.c_int32), ("Hkv", C.c_int32), ("d", C.c_int32),
+                ("T_total", C.c_int32), ("dtype", C.c_int32), ("rope_theta", C.c_float),
+                ("softmax_scale", C.c_float), ("pos_offset", C.c_int32), ("num_splits", C.c_int32)]
+
+
+class jev_readout_desc(C.Structure):
+    _fields_ = [("n_sets", C.c_int32), ("n_cands", C.c_int32), ("n_pairs", C.c_int32), ("R", C.c_int32),
+                ("H", C.c_int32), ("V", C.c_int32), ("dtype", C.c_int32)]
+
+
+_vp, _i32, _sz = C.c_void_p, C.c_int32, C.c_size_t
+_lib.jev_last_error.restype = C.c_char_p
+_lib.jev_prefix_suffix_attn_workspace.argtypes = [C.POINTER(jev_attn_desc)]
+_lib.jev_prefix_suffix_attn_workspace.restype = _sz
+_lib.jev_prefix_suffix_attn.argtypes = [C.POINTER(jev_attn_desc)] + [_vp] * 10 + [_sz, _vp]
+_lib.jev_candidate_readout.argtypes = [C.POINTER(jev_readout_desc)] + [_vp] * 10
+_lib.jev_tree_build.argtypes = [_i32, _vp, _vp, _i32, _i32, _i32] + [_vp] * 7
+_lib.jev_tree_readout_plan.argtypes = [_i32, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp]
+_lib.jev_tree_attn_workspace.argtypes = [C.POINTER(jev_attn_desc), _i32]
+_lib.jev_tree_attn_workspace.restype = _sz
+_lib.jev_tree_attn.argtypes = [C.POINTER(jev_attn_desc), _i32] + [_vp] * 12 + [_sz, _vp]
+_lib.jev_rope_inplace.argtypes = [_vp, _i32, _i32, _i32, _i32, C.c_float, _i32, _vp]
+_lib.jev_workspace_init.argtypes = [_vp, _sz, _vp]
+_lib.jev_check_device_status.argtypes = [_vp, _sz, _vp, C.POINTER(_i32)]
+_lib.jev_profile_enable.argtypes = [_i32]
+_lib.jev_profile_read.argtypes = [_i32, C.c_char_p, _vp, _vp, _i32]
+_lib.jev_profile_read.restype = _i32
+_lib.jev_launch_count.restype = C.c_int64
+for _f in ("jev_prefix_suffix_attn", "jev_candidate_readout", "jev_tree_build", "jev_tree_readout_plan",
+           "jev_tree_attn", "jev_rope_inplace", "jev_workspace_init", "jev_check_device_status",
+           "jev_profile_enable"):
+    getattr(_lib, _f).restype = C.c_int
+
+
+def _check(st: int, where: str):
+    if st != 0:
+        raise JevError(st, where)
+
+
+def _p(t: Optional[torch.Tensor]):
+    return None if t is None else t.data_ptr()
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return JEV_BF16
+    if t.dtype == torch.float32:
+        return JEV_F32
+    raise TypeError(f"jev: tensors must be bfloat16 or float32, got {t.dtype}")
+
+
+def _dev(t: Optional[torch.Tensor], name: str, dtype=None):
+    if t is None:
+        return
+    if not t.is_cuda:
+        raise ValueError(f"jev: {name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"jev: {name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"jev: {name} must be {dtype}, got {t.dtype}")
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def make_attn_desc(B, Lp, Hq, Hkv, d, T_total, dtype_code, rope_theta=1e4, softmax_scale=0.0, pos_offset=-1,
+                   num_splits=0) -> jev_attn_desc:
+    return jev_attn_desc(int(B), int(Lp), int(Hq), int(Hkv), int(d), int(T_total), int(dtype_code),
+                         float(rope_theta), float(softmax_scale), int(pos_offset), int(num_splits))
+
+
+def jev_prefix_suffix_attn_workspace(desc: jev_attn_desc) -> int:
+    return int(_lib.jev_prefix_suffix_attn_workspace(C.byref(desc)))
+
+
+def new_workspace(nbytes: int, device, stream=None) -> torch.Tensor:
+    """A zeroed byte buffer usable as a jev workspace (256-byte aligned by torch)."""
+    ws = torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+    assert ws.data_ptr() % 256 == 0
+    return ws
+
+
+def jev_prefix_suffix_attn(q, k_pre, v_pre, k_suf, v_suf, cu_seqlens, *, head_map=None, out=None, lse=None,
+                           workspace=None, rope_theta=1e4, softmax_scale=0.0, pos_offset=-1, num_splits=0,
+                           T_total: Optional[int] = None, want_lse=True, stream=None):
+    """Shared-prefix attention for B ragged suffix branches; returns (out, lse)."""
+    dt = _dtype_code(q)
+    T, Hq, d = q.shape
+    Lp, Hkv = k_pre.shape[0], k_pre.shape[1]
+    for t, n in ((q, "q"), (k_pre, "k_pre"), (v_pre, "v_pre"), (k_suf, "k_suf"), (v_suf, "v_suf")):
+        _dev(t, n, q.dtype)
+    _dev(cu_seqlens, "cu_seqlens", torch.int32)
+    _dev(head_map, "head_map", torch.int32)
+    B = cu_seqlens.numel() - 1
+    desc = make_attn_desc(B, Lp, Hq, Hkv, d, T if T_total is None else T_total, dt, rope_theta, softmax_scale,
+                          pos_offset, num_splits)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((T, Hq), dtype=torch.float32, device=q.device)
+    _dev(out, "out", q.dtype)
+    _dev(lse, "lse", torch.float32)
+    need = jev_prefix_suffix_attn_workspace(desc)
+    if workspace is None:
+        workspace = new_workspace(need, q.device)
+    _check(_lib.jev_prefix_suffix_attn(C.byref(desc), _p(q), _p(k_pre), _p(v_pre), _p(k_suf), _p(v_suf),
+                                       _p(cu_seqlens), _p(head_map), _p(out), _p(lse), _p(workspace),
+                                       workspace.numel(), _stream(stream)), "jev_prefix_suffix_attn")
+    return out, lse
+
+
+def jev_candidate_readout(hidden, lm_head, set_offsets, pair_tok, *, cand_offsets=None, pair_row=None,
+                          logprob=None, choice=None, score=None, stream=None):
+    """Per-option log-probs and argmax over each option set; returns (logprob, choice)."""
+    dt = _dtype_code(hidden)
+    _dev(hidden, "hidden", hidden.dtype)
+    _dev(lm_head, "lm_head", hidden.dtype)
+    for t, n in ((set_offsets, "set_offsets"), (pair_tok, "pair_tok"), (cand_offsets, "cand_offsets"),
+                 (pair_row, "pair_row")):
+        _dev(t, n, torch.int32)
+    n_sets = set_offsets.numel() - 1
+    n_cands = (cand_offsets.numel() - 1) if cand_offsets is not None else pair_tok.numel()
+    desc = jev_readout_desc(n_sets, n_cands, pair_tok.numel(), hidden.shape[0], hidden.shape[1], lm_head.shape[0], dt)
+    if logprob is None:
+        logprob = torch.empty(n_cands, dtype=torch.float32, device=hidden.device)
+    if choice is None:
+        choice = torch.empty(n_sets, dtype=torch.int32, device=hidden.device)
+    _dev(logprob, "logprob", torch.float32)
+    _dev(choice, "choice", torch.int32)
+    _dev(score, "score", torch.float32)
+    _check(_lib.jev_candidate_readout(C.byref(desc), _p(hidden), _p(lm_head), _p(set_offsets), _p(cand_offsets),
+                                      _p(pair_row), _p(pair_tok), _p(logprob), _p(choice), _p(score),
+                                      _stream(stream)), "jev_candidate_readout")
+    return logprob, choice
+
+
+def jev_tree_build(seq_off: np.ndarray, toks: np.ndarray, root_len: int) -> dict:
+    """Host trie build; returns numpy int32 arrays (parent, tok_off, pos0, leaf_of, node_toks, path_row)."""
+    so = np.ascontiguousarray(seq_off, dtype=np.int32)
+    tk = np.ascontiguousarray(toks, dtype=np.int32)
+    n_cands = so.size - 1
+    total = int(so[-1]) if so.size else 0
+    cap = total + 1
+    parent = np.zeros(cap, np.int32); tok_off = np.zeros(cap + 1, np.int32); pos0 = np.zeros(cap, np.int32)
+    leaf_of = np.zeros(max(n_cands, 1), np.int32); node_toks = np.zeros(max(total, 1), np.int32)
+    path_row = np.zeros(max(total, 1), np.int32)
+    nn = C.c_int32()
+    _check(_lib.jev_tree_build(n_cands, so.ctypes.data, tk.ctypes.data if tk.size else None, int(root_len), cap,
+                               max(total, 1), parent.ctypes.data, tok_off.ctypes.data, pos0.ctypes.data,
+                               leaf_of.ctypes.data, node_toks.ctypes.data, path_row.ctypes.data, C.byref(nn)),
+           "jev_tree_build")
+    n = nn.value
+    N = int(tok_off[n])
+    return dict(n_nodes=n, parent=parent[:n].copy(), tok_off=tok_off[:n + 1].copy(), pos0=pos0[:n].copy(),
+                leaf_of=leaf_of[:n_cands].copy(), node_toks=node_toks[:N].copy(), path_row=path_row[:total].copy())
+
+
+def jev_tree_readout_plan(seq_off, toks, score_from, path_row) -> dict:
+    """Host teacher-forced readout pairs; returns numpy (cand_offsets, pair_row, pair_tok)."""
+    so = np.ascontiguousarray(seq_off, dtype=np.int32); tk = np.ascontiguousarray(toks, dtype=np.int32)
+    sf = np.ascontiguousarray(score_from, dtype=np.int32); pr = np.ascontiguousarray(path_row, dtype=np.int32)
+    n_cands = so.size - 1
+    cap = max(int(so[-1]), 1)
+    co = np.zeros(n_cands + 1, np.int32); prow = np.zeros(cap, np.int32); ptok = np.zeros(cap, np.int32)
+    n = C.c_int32()
+    _check(_lib.jev_tree_readout_plan(n_cands, so.ctypes.data, tk.ctypes.data, sf.ctypes.data, pr.ctypes.data, cap,
+                                      co.ctypes.data, prow.ctypes.data, ptok.ctypes.data, C.byref(n)),
+           "jev_tree_readout_plan")
+    return dict(cand_offsets=co, pair_row=prow[:n.value].copy(), pair_tok=ptok[:n.value].copy())
+
+
+def jev_tree_attn_workspace(desc: jev_attn_desc, n_nodes: int) -> int:
+    return int(_lib.jev_tree_attn_workspace(C.byref(desc), int(n_nodes)))
+
+
+def jev_tree_attn(parent, tok_off, pos0, q, k_root, v_root, k, v, *, head_map=None, out=None, lse=None,
+                  workspace=None, rope_theta=1e4, softmax_scale=0.0, num_splits=0, want_lse=True, stream=None):
+    """Tree attention over packed trie tokens (device parent/tok_off/pos0); returns (out, lse)."""
+    dt = _dtype_code(q)
+    N, Hq, d = q.shape
+    Lp, Hkv = k_root.shape[0], k_root.shape[1]
+    for t, n in ((q, "q"), (k_root, "k_root"), (v_root, "v_root"), (k, "k"), (v, "v")):
+        _dev(t, n, q.dtype)
+    for t, n in ((parent, "parent"), (tok_off, "tok_off"), (pos0, "pos0"), (head_map, "head_map")):
+        _dev(t, n, torch.int32)
+    n_nodes = parent.numel()
+    desc = make_attn_desc(n_nodes - 1, Lp, Hq, Hkv, d, N, dt, rope_theta, softmax_scale, -1, num_splits)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((N, Hq), dtype=torch.float32, device=q.device)
+    need = jev_tree_attn_workspace(desc, n_nodes)
+    if workspace is None:
+        workspace = new_workspace(need, q.device)
+    _check(_lib.jev_tree_attn(C.byref(desc), n_nodes, _p(parent), _p(tok_off), _p(pos0), _p(q), _p(k_root),
+                              _p(v_root), _p(k), _p(v), _p(head_map), _p(out), _p(lse), _p(workspace),
+                              workspace.numel(), _stream(stream)), "jev_tree_attn")
+    return out, lse
+
+
+def jev_rope_inplace(x: torch.Tensor, pos0: int, theta: float = 1e4, stream=None) -> torch.Tensor:
+    _dev(x, "x")
+    L, H, d = x.shape
+    _check(_lib.jev_rope_inplace(_p(x), L, H, d, int(pos0), float(theta), _dtype_code(x), _stream(stream)),
+           "jev_rope_inplace")
+    return x
+
+
+def jev_workspace_init(workspace: torch.Tensor, stream=None):
+    _check(_lib.jev_workspace_init(_p(workspace), workspace.numel(), _stream(stream)), "jev_workspace_init")
+
+
+def jev_check_device_status(workspace: torch.Tensor, stream=None) -> int:
+    """Synchronise, read and clear the status word; returns its flag bits (0 = clean)."""
+    f = C.c_int32()
+    _lib.jev_check_device_status(_p(workspace), workspace.numel(), _stream(stream), C.byref(f))
+    return f.value
+
+
+def jev_last_error() -> str:
+    return _lib.jev_last_error().decode(errors="replace")
+
+
+def jev_profile_enable(on: bool = True):
+    _lib.jev_profile_enable(int(bool(on)))
+
+
+def jev_profile_read(keep: bool = False) -> dict:
+    """{kernel name: (launches, total ms)} of the recorded launches.  With
+    keep=True the records (and their events) stay registered, so launches
+    captured in a CUDA graph can be read again after every replay."""
+    cap = 64
+    names = C.create_string_buffer(cap * 64)
+    launches = np.zeros(cap, np.int32)
+    ms = np.zeros(cap, np.float64)
+    n = _lib.jev_profile_read(cap, names, launches.ctypes.data, ms.ctypes.data, int(bool(keep)))
+    raw = names.raw
+    return {raw[64 * i:64 * i + 64].split(b"\0", 1)[0].decode(): (int(launches[i]), float(ms[i])) for i in range(min(n, cap))}
+
+
+def jev_launch_count() -> int:
+    return int(_lib.jev_launch_count())

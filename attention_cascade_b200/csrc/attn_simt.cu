@@ -1,0 +1,190 @@
+// attn_simt.cu — CUDA-core attention over [prefix split ; own suffix window]
+// for the stacked rows of one kv group.  Used for fp32 inputs, where the
+// tensor-core kernel does not apply.
+//
+// Each block holds 16 stacked rows (row m of group g is token m / G, query
+// slot m % G) and streams 32-key tiles of the prefix split through shared
+// memory; one warp owns four rows, a lane owns one key of the tile for the
+// scores and d/32 output columns for P.V.  The online softmax runs in the
+// log2 domain.  The block that holds the last prefix split also walks the
+// suffix keys its rows may see: for a flat branch, the keys of the same branch
+// up to the row's own token; for a tree token, every non-root ancestor's keys
+// plus its own node's keys up to itself.
+#include <math_constants.h>
+
+#include "kernels.h"
+
+namespace jev {
+namespace {
+
+constexpr int kRows = 16;   // stacked rows per block
+constexpr int kKeys = 32;   // keys per tile
+constexpr int kThreads = 128;
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kThreads) attn_simt_kernel(AttnArgs a) {
+  constexpr int C = D / 32;  // output columns per lane
+  __shared__ float Qs[kRows][D];
+  __shared__ float Ks[kKeys][D + 1];
+  __shared__ float Vs[kKeys][D];
+  __shared__ int r_t[kRows], r_start[kRows], r_nanc[kRows];
+  __shared__ int2 r_anc[kRows][kMaxDepth];
+  __shared__ int s_lo, s_hi;
+
+  const int g = blockIdx.y, split = blockIdx.z;
+  const int m0 = blockIdx.x * kRows;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const T* qg = reinterpret_cast<const T*>(a.q_rot) + (size_t)g * a.M * D;
+
+  for (int e = tid; e < kRows * D; e += kThreads) {
+    int r = e / D, i = e - r * D;
+    int m = m0 + r;
+    Qs[r][i] = m < a.M ? to_f32(qg[(size_t)m * D + i]) : 0.f;
+  }
+  if (tid < kRows) {
+    int m = m0 + tid;
+    if (m < a.M) {
+      int t = m / a.G;
+      TokInfo inf = a.info[t];
+      int nanc = 0;
+      if (a.node_nanc) {
+        nanc = a.node_nanc[inf.node];
+        if (nanc < 0) t = -1;  // malformed tree: row sees no suffix keys and is not written
+        for (int k = 0; k < nanc; ++k) r_anc[tid][k] = a.node_anc[(size_t)inf.node * kMaxDepth + k];
+      }
+      r_t[tid] = t;
+      r_start[tid] = inf.seg_start;
+      r_nanc[tid] = nanc > 0 ? nanc : 0;
+    } else {
+      r_t[tid] = -1;
+      r_start[tid] = 0;
+      r_nanc[tid] = 0;
+    }
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int lo = INT_MAX, hi = -1;
+    for (int r = 0; r < kRows; ++r) {
+      if (r_t[r] < 0) continue;
+      int start = r_nanc[r] > 0 ? min(r_anc[r][0].x, r_start[r]) : r_start[r];
+      lo = min(lo, start);
+      hi = max(hi, r_t[r]);
+    }
+    s_lo = lo;
+    s_hi = hi;
+  }
+
+  float m_r[4], l_r[4], acc[4][C];
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    m_r[r] = -CUDART_INF_F;
+    l_r[r] = 0.f;
+#pragma unroll
+    for (int c = 0; c < C; ++c) acc[r][c] = 0.f;
+  }
+
+  // one 32-key tile: keys [kb, kb + n) of K/V with row stride Hkv*D
+  auto tile = [&](const T* Kg, const T* Vg, int kb, int n, bool suffix) {
+    __syncthreads();
+    for (int e = tid; e < kKeys * D; e += kThreads) {
+      int j = e / D, i = e - j * D;
+      bool ok = j < n;
+      size_t off = ((size_t)(kb + j) * a.Hkv) * D + i;
+      Ks[j][i] = ok ? to_f32(Kg[off]) : 0.f;
+      Vs[j][i] = ok ? to_f32(Vg[off]) : 0.f;
+    }
+    __syncthreads();
+    float p[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int rr = warp * 4 + r;
+      float s = 0.f;
+#pragma unroll 8
+      for (int i = 0; i < D; ++i) s += Qs[rr][i] * Ks[lane][i];
+      s *= a.scale_log2;
+      const int key = kb + lane;
+      bool ok = lane < n && r_t[rr] >= 0;
+      if (ok && suffix) {
+        bool vis = key >= r_start[rr] && key <= r_t[rr];
+        for (int k = 0; k < r_nanc[rr]; ++k) vis |= (key >= r_anc[rr][k].x && key < r_anc[rr][k].y);
+        ok = vis;
+      }
+      s = ok ? s : -CUDART_INF_F;
+      const float mx = warp_max(s);
+      const float m_new = fmaxf(m_r[r], mx);
+      float alpha, pv;
+      if (m_new == -CUDART_INF_F) {
+        alpha = 1.f;
+        pv = 0.f;
+      } else {
+        alpha = exp2f(m_r[r] - m_new);
+        pv = exp2f(s - m_new);
+      }
+      l_r[r] = l_r[r] * alpha + warp_sum(pv);
+      m_r[r] = m_new;
+#pragma unroll
+      for (int c = 0; c < C; ++c) acc[r][c] *= alpha;
+      p[r] = pv;
+    }
+    for (int j = 0; j < kKeys; ++j) {
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const float pj = __shfl_sync(0xffffffffu, p[r], j);
+#pragma unroll
+        for (int c = 0; c < C; ++c) acc[r][c] += pj * Vs[j][lane + 32 * c];
+      }
+    }
+  };
+
+  const T* kp = reinterpret_cast<const T*>(a.k_pre) + (size_t)g * D;
+  const T* vp = reinterpret_cast<const T*>(a.v_pre) + (size_t)g * D;
+  const int p_lo = split * a.split_len;
+  const int p_hi = min(a.Lp, p_lo + a.split_len);
+  for (int kb = p_lo; kb < p_hi; kb += kKeys) tile(kp, vp, kb, min(kKeys, p_hi - kb), false);
+  if (split == a.S - 1) {
+    __syncthreads();
+    const int lo = s_lo, hi = s_hi;
+    const T* ks = reinterpret_cast<const T*>(a.k_rot) + (size_t)g * D;
+    const T* vs = reinterpret_cast<const T*>(a.v_suf) + (size_t)g * D;
+    for (int kb = lo; kb <= hi; kb += kKeys) tile(ks, vs, kb, min(kKeys, hi + 1 - kb), true);
+  }
+
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const int rr = warp * 4 + r;
+    const int m = m0 + rr;
+    if (m >= a.M || r_t[rr] < 0) continue;
+    const float inv = l_r[r] > 0.f ? 1.f / l_r[r] : 0.f;
+    const float lse2 = l_r[r] > 0.f ? m_r[r] + log2f(l_r[r]) : -CUDART_INF_F;
+    if (a.S == 1) {
+      const int t = m / a.G;
+      const int h = min(max(a.hinv[g * a.G + (m - t * a.G)], 0), a.Hq - 1);
+      T* o = reinterpret_cast<T*>(a.out) + ((size_t)t * a.Hq + h) * D;
+#pragma unroll
+      for (int c = 0; c < C; ++c) o[lane + 32 * c] = from_f32<T>(acc[r][c] * inv);
+      if (a.lse && lane == 0) a.lse[(size_t)t * a.Hq + h] = lse2 * 0.69314718055994531f;
+    } else {
+      float* o = a.o_part + (((size_t)split * a.Hkv + g) * a.M + m) * D;
+#pragma unroll
+      for (int c = 0; c < C; ++c) o[lane + 32 * c] = acc[r][c] * inv;
+      if (lane == 0) a.l_part[((size_t)split * a.Hkv + g) * a.M + m] = lse2;
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_attn_simt(const AttnArgs& a, jev_dtype dt, cudaStream_t s) {
+  dim3 grid((a.M + kRows - 1) / kRows, a.Hkv, a.S);
+  if (a.M == 0) return cudaSuccess;
+  if (dt == JEV_BF16) {
+    if (a.d == 64) attn_simt_kernel<__nv_bfloat16, 64><<<grid, kThreads, 0, s>>>(a);
+    else attn_simt_kernel<__nv_bfloat16, 128><<<grid, kThreads, 0, s>>>(a);
+  } else {
+    if (a.d == 64) attn_simt_kernel<float, 64><<<grid, kThreads, 0, s>>>(a);
+    else attn_simt_kernel<float, 128><<<grid, kThreads, 0, s>>>(a);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace jev

@@ -1,0 +1,55 @@
+// common.cuh — small device helpers shared by the jev kernels.
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/jev.h"
+
+namespace jev {
+
+constexpr int kStatusBytes = 256;  // status word lives in the first 256 bytes of a workspace
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__device__ __forceinline__ void raise_flag(int32_t* status, int32_t bit) {
+  if (status) atomicOr(status, bit);
+}
+
+// Largest b in [0, n) with offs[b] <= t (offs non-decreasing); 0 if none.
+__device__ __forceinline__ int upper_segment(const int32_t* offs, int n, int t) {
+  int lo = 0, hi = n - 1;
+  while (lo < hi) {
+    int mid = (lo + hi + 1) >> 1;
+    if (offs[mid] <= t) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+// Per packed token: where its own segment starts and its RoPE position.
+// Tree tokens additionally carry up to kMaxAnc ancestor key ranges.
+constexpr int kMaxDepth = 8;  // non-root ancestors + own node
+
+struct TokInfo {
+  int32_t seg_start;  // first packed key of the token's own segment (branch or node)
+  int32_t pos;        // RoPE position of the token
+  int32_t node;       // tree node (flat: branch index)
+  int32_t n_anc;      // number of ancestor ranges (flat: 0)
+};
+
+}  // namespace jev

@@ -1,0 +1,485 @@
+// jev_api.cu — the C ABI declared in include/jev.h: argument checks,
+// workspace layout, split planning, kernel launches, kernel timing and the
+// host-side candidate-prefix trie.
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <unordered_map>
+#include <vector>
+
+#include "kernels.h"
+
+namespace jev {
+namespace {
+
+thread_local char g_err[512] = "";
+
+jev_status fail(jev_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof g_err, fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+// ---------------------------------------------------------------- timing
+struct Rec {
+  int name;
+  cudaEvent_t a, b;
+};
+std::mutex g_mu;
+std::atomic<bool> g_prof{false};
+std::vector<Rec> g_recs;
+std::vector<cudaEvent_t> g_pool;
+std::vector<std::string> g_names;
+std::atomic<long long> g_launches{0};
+
+int name_id(const char* n) {
+  for (size_t i = 0; i < g_names.size(); ++i)
+    if (g_names[i] == n) return (int)i;
+  g_names.emplace_back(n);
+  return (int)g_names.size() - 1;
+}
+cudaEvent_t take_event() {
+  if (!g_pool.empty()) {
+    cudaEvent_t e = g_pool.back();
+    g_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e;
+  cudaEventCreate(&e);
+  return e;
+}
+
+// Launch one kernel through `fn`, bracketed by timing events when enabled.
+template <class F>
+jev_status run(const char* name, cudaStream_t s, F&& fn) {
+  Rec r{-1, nullptr, nullptr};
+  const bool on = g_prof.load();
+  if (on) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    r.name = name_id(name);
+    r.a = take_event();
+    r.b = take_event();
+    cudaEventRecord(r.a, s);
+  }
+  cudaError_t e = fn();
+  if (on) {
+    cudaEventRecord(r.b, s);
+    std::lock_guard<std::mutex> lk(g_mu);
+    g_recs.push_back(r);
+  }
+  g_launches++;
+  if (e != cudaSuccess) return fail(JEV_ERR_CUDA, "%s launch failed: %s", name, cudaGetErrorString(e));
+  return JEV_OK;
+}
+
+// ---------------------------------------------------------------- checks
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
+size_t esize(jev_dtype dt) { return dt == JEV_BF16 ? 2 : 4; }
+
+int num_sms() {
+  static int sms = 0;
+  if (!sms) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) sms = 148;
+  }
+  return sms;
+}
+
+bool use_tc(const jev_attn_desc* d) {
+  static int forced = -1;
+  if (forced < 0) {
+    const char* e = getenv("JEV_ATTN_KERNEL");
+    forced = (e && !strcmp(e, "simt")) ? 1 : 0;
+  }
+  return !forced && d->dtype == JEV_BF16 && attn_tc_supported(d->d);
+}
+
+// Prefix split plan: split_len is a multiple of 128 keys; the number of
+// splits depends only on Lp, the stacked row count and the SM count.
+struct Plan {
+  int S, split_len, M, G;
+};
+Plan plan_of(const jev_attn_desc* d, int T) {
+  Plan p;
+  p.G = d->Hq / d->Hkv;
+  p.M = T * p.G;
+  const int ktiles = (d->Lp + 127) / 128;
+  int S = d->num_splits;
+  if (S <= 0) {
+    const int rows_per_cta = use_tc(d) ? 256 : 16;
+    const long ctas = (long)((p.M + rows_per_cta - 1) / rows_per_cta) * d->Hkv;
+    const long target = use_tc(d) ? (long)num_sms() : 4L * num_sms();
+    S = ctas > 0 ? (int)((target + ctas - 1) / ctas) : 1;
+    // keep at least 4 key tiles per split so partial traffic stays small
+    S = std::min(S, std::max(1, ktiles / 4));
+  }
+  S = std::max(1, std::min(S, std::max(1, ktiles)));
+  p.split_len = ktiles > 0 ? ((ktiles + S - 1) / S) * 128 : 128;
+  p.S = d->Lp > 0 ? (d->Lp + p.split_len - 1) / p.split_len : 1;
+  return p;
+}
+
+struct Layout {
+  size_t hinv, info, qrot, krot, opart, lpart, anc, nanc, total;
+};
+Layout layout_of(const jev_attn_desc* d, int T, const Plan& p, int n_nodes) {
+  Layout L;
+  const size_t s = esize(d->dtype);
+  size_t off = kStatusBytes;
+  L.hinv = off; off += up256((size_t)d->Hq * 4);
+  L.info = off; off += up256((size_t)T * sizeof(TokInfo));
+  L.qrot = off; off += up256((size_t)p.M * d->Hkv * d->d * s);
+  L.krot = off; off += up256((size_t)T * d->Hkv * d->d * s);
+  L.opart = off;
+  L.lpart = off;
+  if (p.S > 1) {
+    L.opart = off; off += up256((size_t)p.S * d->Hkv * p.M * d->d * 4);
+    L.lpart = off; off += up256((size_t)p.S * d->Hkv * p.M * 4);
+  }
+  L.anc = off; L.nanc = off;
+  if (n_nodes > 0) {
+    L.anc = off; off += up256((size_t)n_nodes * kMaxDepth * sizeof(int2));
+    L.nanc = off; off += up256((size_t)n_nodes * 4);
+  }
+  L.total = off;
+  return L;
+}
+
+jev_status check_desc(const jev_attn_desc* d) {
+  if (!d) return fail(JEV_ERR_INVALID_ARG, "desc is NULL");
+  if (d->B < 0 || d->Lp < 0 || d->T_total < 0) return fail(JEV_ERR_INVALID_ARG, "negative B, Lp or T_total");
+  if (d->Hq <= 0 || d->Hkv <= 0 || d->Hq % d->Hkv) return fail(JEV_ERR_INVALID_ARG, "Hq must be a positive multiple of Hkv");
+  if (d->Hq > 256) return fail(JEV_ERR_UNSUPPORTED, "Hq > 256");
+  if (d->d != 64 && d->d != 128) return fail(JEV_ERR_UNSUPPORTED, "head dim %d (supported: 64, 128)", d->d);
+  if (d->dtype != JEV_BF16 && d->dtype != JEV_F32) return fail(JEV_ERR_UNSUPPORTED, "dtype");
+  if (!(d->rope_theta > 0.f)) return fail(JEV_ERR_INVALID_ARG, "rope_theta must be > 0");
+  if (d->softmax_scale < 0.f) return fail(JEV_ERR_INVALID_ARG, "softmax_scale must be >= 0");
+  if ((long long)d->T_total * (d->Hq / d->Hkv) > (1LL << 30)) return fail(JEV_ERR_UNSUPPORTED, "too many rows");
+  return JEV_OK;
+}
+
+float scale_log2_of(const jev_attn_desc* d) {
+  const double sc = d->softmax_scale > 0.f ? (double)d->softmax_scale : 1.0 / std::sqrt((double)d->d);
+  return (float)(sc * 1.4426950408889634);
+}
+
+// Shared tail of the flat and tree entry points.
+jev_status attention_core(const jev_attn_desc* d, int T, const Plan& p, const Layout& L, char* ws,
+                          const void* q, const void* k_pre, const void* v_pre, const void* k_suf,
+                          const void* v_suf, const int32_t* offs, int n_segs, const int32_t* pos0,
+                          const int32_t* head_map, bool tree, void* out, float* lse, cudaStream_t s) {
+  int32_t* status = reinterpret_cast<int32_t*>(ws);
+  RopePackArgs r{};
+  r.q = q; r.k = k_suf;
+  r.q_rot = ws + L.qrot; r.k_rot = ws + L.krot;
+  r.info = reinterpret_cast<TokInfo*>(ws + L.info);
+  r.hinv = reinterpret_cast<int32_t*>(ws + L.hinv);
+  r.status = status;
+  r.offs = offs; r.pos0 = pos0; r.head_map = head_map;
+  r.n_segs = n_segs; r.T = T; r.Hq = d->Hq; r.Hkv = d->Hkv; r.d = d->d;
+  r.pos_offset = d->pos_offset >= 0 ? d->pos_offset : d->Lp;
+  r.theta = (double)d->rope_theta;
+  jev_status st = run("rope_pack", s, [&] { return launch_rope_pack(r, d->dtype, s); });
+  if (st) return st;
+
+  AttnArgs a{};
+  a.q_rot = r.q_rot; a.k_pre = k_pre; a.v_pre = v_pre; a.k_rot = r.k_rot; a.v_suf = v_suf;
+  a.info = r.info;
+  a.node_anc = tree ? reinterpret_cast<const int2*>(ws + L.anc) : nullptr;
+  a.node_nanc = tree ? reinterpret_cast<const int32_t*>(ws + L.nanc) : nullptr;
+  a.hinv = r.hinv;
+  a.out = out; a.lse = lse;
+  a.o_part = reinterpret_cast<float*>(ws + L.opart);
+  a.l_part = reinterpret_cast<float*>(ws + L.lpart);
+  a.status = status;
+  a.T = T; a.M = p.M; a.Lp = d->Lp; a.Hq = d->Hq; a.Hkv = d->Hkv; a.G = p.G; a.d = d->d;
+  a.S = p.S; a.split_len = p.split_len;
+  a.scale_log2 = scale_log2_of(d);
+  if (use_tc(d)) st = run("attn_tc", s, [&] { return launch_attn_tc(a, s); });
+  else st = run("attn_simt", s, [&] { return launch_attn_simt(a, d->dtype, s); });
+  if (st) return st;
+  if (p.S > 1) {
+    MergeArgs m{};
+    m.o_part = a.o_part; m.l_part = a.l_part; m.hinv = a.hinv; m.out = out; m.lse = lse;
+    m.M = p.M; m.Hq = d->Hq; m.Hkv = d->Hkv; m.G = p.G; m.d = d->d; m.S = p.S;
+    st = run("merge_splits", s, [&] { return launch_merge(m, d->dtype, s); });
+  }
+  return st;
+}
+
+// ---------------------------------------------------------------- trie (host)
+// Token-level trie in hash maps, then segments in DFS preorder.
+struct HostTrie {
+  std::vector<int32_t> tok, depth, nchild, first_child, packed, seg;
+  std::vector<std::vector<int32_t>> kids;  // children in order of creation
+  std::vector<uint8_t> ends;
+  std::unordered_map<uint64_t, int32_t> edge;  // (parent << 32 | token) -> child
+  HostTrie() { add(-1, 0); }
+  int32_t add(int32_t tk, int32_t dep) {
+    tok.push_back(tk); depth.push_back(dep); kids.emplace_back(); ends.push_back(0);
+    packed.push_back(-1); seg.push_back(-1);
+    return (int32_t)tok.size() - 1;
+  }
+  int32_t step(int32_t u, int32_t tk) {
+    const uint64_t key = ((uint64_t)(uint32_t)u << 32) | (uint32_t)tk;
+    auto it = edge.find(key);
+    if (it != edge.end()) return it->second;
+    int32_t c = add(tk, depth[u] + 1);
+    kids[u].push_back(c);
+    edge.emplace(key, c);
+    return c;
+  }
+};
+
+}  // namespace
+}  // namespace jev
+
+using namespace jev;
+
+extern "C" {
+
+const char* jev_last_error(void) { return g_err; }
+
+int64_t jev_launch_count(void) { return (int64_t)g_launches.load(); }
+
+jev_status jev_profile_enable(int32_t on) {
+  g_prof.store(on != 0);
+  return JEV_OK;
+}
+
+int32_t jev_profile_read(int32_t cap, char* names, int32_t* launches, double* ms, int32_t keep) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  std::vector<double> tot(g_names.size(), 0.0);
+  std::vector<int> cnt(g_names.size(), 0);
+  for (const Rec& r : g_recs) {
+    cudaEventSynchronize(r.b);
+    float t = 0.f;
+    cudaEventElapsedTime(&t, r.a, r.b);
+    tot[r.name] += t;
+    cnt[r.name] += 1;
+    if (!keep) {
+      g_pool.push_back(r.a);
+      g_pool.push_back(r.b);
+    }
+  }
+  if (!keep) g_recs.clear();
+  int n = 0;
+  for (size_t i = 0; i < g_names.size(); ++i) {
+    if (!cnt[i]) continue;
+    if (n < cap) {
+      if (names) {
+        strncpy(names + 64 * n, g_names[i].c_str(), 63);
+        names[64 * n + 63] = 0;
+      }
+      if (launches) launches[n] = cnt[i];
+      if (ms) ms[n] = tot[i];
+    }
+    ++n;
+  }
+  return n;
+}
+
+size_t jev_prefix_suffix_attn_workspace(const jev_attn_desc* d) {
+  if (check_desc(d) != JEV_OK) return 0;
+  Plan p = plan_of(d, d->T_total);
+  return layout_of(d, d->T_total, p, 0).total;
+}
+
+jev_status jev_workspace_init(void* ws, size_t ws_bytes, jev_stream_t stream) {
+  if (!ws || ws_bytes < (size_t)kStatusBytes) return fail(JEV_ERR_WORKSPACE, "workspace smaller than the status word");
+  cudaError_t e = cudaMemsetAsync(ws, 0, kStatusBytes, (cudaStream_t)stream);
+  if (e != cudaSuccess) return fail(JEV_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(e));
+  return JEV_OK;
+}
+
+jev_status jev_check_device_status(void* ws, size_t ws_bytes, jev_stream_t stream, int32_t* flags) {
+  if (!ws || ws_bytes < (size_t)kStatusBytes) return fail(JEV_ERR_WORKSPACE, "workspace smaller than the status word");
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return fail(JEV_ERR_CUDA, "stream sync: %s", cudaGetErrorString(e));
+  int32_t f = 0;
+  e = cudaMemcpyAsync(&f, ws, sizeof f, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(ws, 0, kStatusBytes, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return fail(JEV_ERR_CUDA, "status read: %s", cudaGetErrorString(e));
+  if (flags) *flags = f;
+  if (f) return fail(JEV_ERR_DEVICE, "device status flags 0x%x", f);
+  return JEV_OK;
+}
+
+jev_status jev_prefix_suffix_attn(const jev_attn_desc* d, const void* q, const void* k_pre, const void* v_pre,
+                                  const void* k_suf, const void* v_suf, const int32_t* cu_seqlens,
+                                  const int32_t* head_map, void* out, float* lse, void* workspace,
+                                  size_t ws_bytes, jev_stream_t stream) {
+  jev_status st = check_desc(d);
+  if (st) return st;
+  if (d->B == 0 || d->T_total == 0) return JEV_OK;
+  if (!q || !k_suf || !v_suf || !cu_seqlens || !out) return fail(JEV_ERR_INVALID_ARG, "required pointer is NULL");
+  if (d->Lp > 0 && (!k_pre || !v_pre)) return fail(JEV_ERR_INVALID_ARG, "prefix pointers are NULL with Lp > 0");
+  const void* ptrs[] = {q, k_pre, v_pre, k_suf, v_suf, out, lse};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return fail(JEV_ERR_INVALID_ARG, "tensor pointer not 16-byte aligned");
+  if (!aligned16(cu_seqlens) && ((uintptr_t)cu_seqlens & 3)) return fail(JEV_ERR_INVALID_ARG, "cu_seqlens misaligned");
+  const int T = d->T_total;
+  Plan p = plan_of(d, T);
+  Layout L = layout_of(d, T, p, 0);
+  if (!workspace || ((uintptr_t)workspace & 255)) return fail(JEV_ERR_WORKSPACE, "workspace NULL or not 256-byte aligned");
+  if (ws_bytes < L.total) return fail(JEV_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", ws_bytes, L.total);
+  return attention_core(d, T, p, L, (char*)workspace, q, k_pre, v_pre, k_suf, v_suf, cu_seqlens, d->B, nullptr,
+                        head_map, false, out, lse, (cudaStream_t)stream);
+}
+
+jev_status jev_candidate_readout(const jev_readout_desc* d, const void* hidden, const void* lm_head,
+                                 const int32_t* set_offsets, const int32_t* cand_offsets, const int32_t* pair_row,
+                                 const int32_t* pair_tok, float* logprob, int32_t* choice, float* score,
+                                 jev_stream_t stream) {
+  if (!d) return fail(JEV_ERR_INVALID_ARG, "desc is NULL");
+  if (d->n_sets < 0 || d->n_cands < 0 || d->n_pairs < 0 || d->R < 0 || d->V <= 0 || d->H <= 0)
+    return fail(JEV_ERR_INVALID_ARG, "negative or zero sizes");
+  if (d->dtype != JEV_BF16 && d->dtype != JEV_F32) return fail(JEV_ERR_UNSUPPORTED, "dtype");
+  if (d->H % 8) return fail(JEV_ERR_UNSUPPORTED, "hidden size must be a multiple of 8");
+  if (!cand_offsets && d->n_pairs != d->n_cands) return fail(JEV_ERR_INVALID_ARG, "n_pairs != n_cands without cand_offsets");
+  if (d->n_sets == 0) return JEV_OK;
+  if (!set_offsets || !choice) return fail(JEV_ERR_INVALID_ARG, "set_offsets / choice NULL");
+  if (d->n_cands > 0 && (!hidden || !lm_head || !pair_tok || !logprob))
+    return fail(JEV_ERR_INVALID_ARG, "required pointer is NULL");
+  if ((hidden && !aligned16(hidden)) || (lm_head && !aligned16(lm_head)))
+    return fail(JEV_ERR_INVALID_ARG, "hidden / lm_head not 16-byte aligned");
+  if (!pair_row && d->R < d->n_sets) return fail(JEV_ERR_INVALID_ARG, "R < n_sets with pair_row NULL");
+  ReadoutArgs a{hidden, lm_head, set_offsets, cand_offsets, pair_row, pair_tok, logprob, choice, score,
+                d->n_sets, d->n_cands, d->n_pairs, d->R, d->H, d->V};
+  return run("readout", (cudaStream_t)stream, [&] { return launch_readout(a, d->dtype, (cudaStream_t)stream); });
+}
+
+jev_status jev_rope_inplace(void* x, int32_t L, int32_t H, int32_t d, int32_t pos0, float theta, jev_dtype dt,
+                            jev_stream_t stream) {
+  if (L < 0 || H <= 0 || d <= 0 || (d & 1) || d > 256) return fail(JEV_ERR_INVALID_ARG, "bad shape");
+  if (!(theta > 0.f)) return fail(JEV_ERR_INVALID_ARG, "theta must be > 0");
+  if (L == 0) return JEV_OK;
+  if (!x) return fail(JEV_ERR_INVALID_ARG, "x is NULL");
+  return run("rope_inplace", (cudaStream_t)stream,
+             [&] { return launch_rope_inplace(x, L, H, d, pos0, (double)theta, dt, (cudaStream_t)stream); });
+}
+
+jev_status jev_tree_build(int32_t n_cands, const int32_t* seq_off, const int32_t* toks, int32_t root_len,
+                          int32_t cap_nodes, int32_t cap_toks, int32_t* parent, int32_t* tok_off, int32_t* pos0,
+                          int32_t* leaf_of, int32_t* node_toks, int32_t* path_row, int32_t* n_nodes_out) {
+  if (n_cands < 0 || !seq_off || root_len < 0 || !parent || !tok_off || !pos0 || !n_nodes_out)
+    return fail(JEV_ERR_INVALID_ARG, "bad arguments");
+  if (n_cands > 0 && (!leaf_of)) return fail(JEV_ERR_INVALID_ARG, "leaf_of is NULL");
+  if (seq_off[0] != 0) return fail(JEV_ERR_INVALID_ARG, "seq_off[0] != 0");
+  for (int c = 0; c < n_cands; ++c)
+    if (seq_off[c + 1] < seq_off[c]) return fail(JEV_ERR_INVALID_ARG, "seq_off decreases at %d", c);
+  const int total = seq_off[n_cands];
+  if (total > 0 && !toks) return fail(JEV_ERR_INVALID_ARG, "toks is NULL");
+  HostTrie tr;
+  std::vector<int32_t> end_of(n_cands), path_tn(total);
+  for (int c = 0; c < n_cands; ++c) {
+    int32_t u = 0;
+    for (int i = seq_off[c]; i < seq_off[c + 1]; ++i) path_tn[i] = u = tr.step(u, toks[i]);
+    end_of[c] = u;
+    tr.ends[u] = (u != 0);
+  }
+  if (cap_nodes < 1) return fail(JEV_ERR_CAPACITY, "cap_nodes < 1");
+  // depth-first preorder over chain heads
+  struct Item { int32_t u, par; };
+  std::vector<Item> stack;
+  for (auto it = tr.kids[0].rbegin(); it != tr.kids[0].rend(); ++it) stack.push_back({*it, 0});
+  int32_t nn = 1, cursor = 0;
+  parent[0] = -1; pos0[0] = 0; tok_off[0] = 0;
+  if (cap_nodes >= 1) tok_off[1] = 0;
+  while (!stack.empty()) {
+    Item it = stack.back();
+    stack.pop_back();
+    if (nn >= cap_nodes) return fail(JEV_ERR_CAPACITY, "more than %d nodes", cap_nodes);
+    const int32_t id = nn++;
+    parent[id] = it.par;
+    pos0[id] = root_len + tr.depth[it.u] - 1;
+    tok_off[id] = cursor;
+    int32_t u = it.u;
+    for (;;) {
+      if (cursor >= cap_toks) return fail(JEV_ERR_CAPACITY, "more than %d packed tokens", cap_toks);
+      if (node_toks) node_toks[cursor] = tr.tok[u];
+      tr.packed[u] = cursor++;
+      tr.seg[u] = id;
+      if (tr.kids[u].size() == 1 && !tr.ends[u]) u = tr.kids[u][0];
+      else break;
+    }
+    tok_off[id + 1] = cursor;
+    for (auto k = tr.kids[u].rbegin(); k != tr.kids[u].rend(); ++k) stack.push_back({*k, id});
+  }
+  for (int c = 0; c < n_cands; ++c) leaf_of[c] = end_of[c] ? tr.seg[end_of[c]] : 0;
+  if (path_row)
+    for (int i = 0; i < total; ++i) path_row[i] = tr.packed[path_tn[i]];
+  *n_nodes_out = nn;
+  return JEV_OK;
+}
+
+jev_status jev_tree_readout_plan(int32_t n_cands, const int32_t* seq_off, const int32_t* toks,
+                                 const int32_t* score_from, const int32_t* path_row, int32_t cap_pairs,
+                                 int32_t* cand_offsets, int32_t* pair_row, int32_t* pair_tok, int32_t* n_pairs) {
+  if (n_cands < 0 || !seq_off || !score_from || !path_row || !cand_offsets || !n_pairs)
+    return fail(JEV_ERR_INVALID_ARG, "bad arguments");
+  int32_t k = 0;
+  cand_offsets[0] = 0;
+  for (int c = 0; c < n_cands; ++c) {
+    const int a = seq_off[c], e = seq_off[c + 1];
+    if (score_from[c] < 1 || a + score_from[c] > e)
+      return fail(JEV_ERR_INVALID_ARG, "score_from[%d] = %d outside [1, len]", c, score_from[c]);
+    for (int i = a + score_from[c]; i < e; ++i) {
+      if (k >= cap_pairs) return fail(JEV_ERR_CAPACITY, "more than %d pairs", cap_pairs);
+      pair_row[k] = path_row[i - 1];
+      pair_tok[k] = toks[i];
+      ++k;
+    }
+    cand_offsets[c + 1] = k;
+  }
+  *n_pairs = k;
+  return JEV_OK;
+}
+
+size_t jev_tree_attn_workspace(const jev_attn_desc* d, int32_t n_nodes) {
+  if (check_desc(d) != JEV_OK || n_nodes < 1) return 0;
+  Plan p = plan_of(d, d->T_total);
+  return layout_of(d, d->T_total, p, n_nodes).total;
+}
+
+jev_status jev_tree_attn(const jev_attn_desc* d, int32_t n_nodes, const int32_t* parent, const int32_t* tok_off,
+                         const int32_t* pos0, const void* q, const void* k_root, const void* v_root, const void* k,
+                         const void* v, const int32_t* head_map, void* out, float* lse, void* workspace,
+                         size_t ws_bytes, jev_stream_t stream) {
+  jev_status st = check_desc(d);
+  if (st) return st;
+  if (n_nodes < 1) return fail(JEV_ERR_INVALID_ARG, "n_nodes < 1");
+  if (d->T_total == 0) return JEV_OK;
+  if (!parent || !tok_off || !pos0 || !q || !k || !v || !out) return fail(JEV_ERR_INVALID_ARG, "required pointer is NULL");
+  if (d->Lp > 0 && (!k_root || !v_root)) return fail(JEV_ERR_INVALID_ARG, "root pointers are NULL with Lp > 0");
+  const void* ptrs[] = {q, k_root, v_root, k, v, out, lse};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return fail(JEV_ERR_INVALID_ARG, "tensor pointer not 16-byte aligned");
+  const int T = d->T_total;
+  Plan p = plan_of(d, T);
+  Layout L = layout_of(d, T, p, n_nodes);
+  if (!workspace || ((uintptr_t)workspace & 255)) return fail(JEV_ERR_WORKSPACE, "workspace NULL or not 256-byte aligned");
+  if (ws_bytes < L.total) return fail(JEV_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", ws_bytes, L.total);
+  char* ws = (char*)workspace;
+  TreePlanArgs tp{parent, tok_off, reinterpret_cast<int2*>(ws + L.anc), reinterpret_cast<int32_t*>(ws + L.nanc),
+                  reinterpret_cast<int32_t*>(ws), n_nodes, T};
+  st = run("tree_plan", (cudaStream_t)stream, [&] { return launch_tree_plan(tp, (cudaStream_t)stream); });
+  if (st) return st;
+  return attention_core(d, T, p, L, ws, q, k_root, v_root, k, v, tok_off, n_nodes, pos0, head_map, true, out, lse,
+                        (cudaStream_t)stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,84 @@
+// kernels.h — launchers of the jev kernels (internal to the library).
+#pragma once
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace jev {
+
+// Rotate the packed suffix (or tree) tokens and lay queries out group-major:
+// q_rot[g][t*G + slot(h)][:] = RoPE(q[t][h][:]), k_rot[t][g][:] = RoPE(k[t][g][:]).
+struct RopePackArgs {
+  const void* q;           // [T, Hq, d]
+  const void* k;           // [T, Hkv, d]
+  void* q_rot;             // [Hkv, T*G, d]
+  void* k_rot;             // [T, Hkv, d]
+  TokInfo* info;           // [T]
+  int32_t* hinv;           // [Hq]: q-head of group-major slot g*G + s
+  int32_t* status;
+  const int32_t* offs;     // flat: cu_seqlens [n_segs+1]; tree: tok_off [n_segs+1]
+  const int32_t* pos0;     // tree: [n_segs] first-token positions; flat: nullptr
+  const int32_t* head_map; // [Hq] or nullptr
+  int n_segs, T, Hq, Hkv, d, pos_offset;
+  double theta;
+};
+cudaError_t launch_rope_pack(const RopePackArgs& a, jev_dtype dt, cudaStream_t s);
+
+// Per tree node, the packed key ranges of its non-root ancestors (root first).
+struct TreePlanArgs {
+  const int32_t* parent;   // [n_nodes]
+  const int32_t* tok_off;  // [n_nodes+1]
+  int2* node_anc;          // [n_nodes, kMaxDepth]
+  int32_t* node_nanc;      // [n_nodes]
+  int32_t* status;
+  int n_nodes, N;
+};
+cudaError_t launch_tree_plan(const TreePlanArgs& a, cudaStream_t s);
+
+// Attention over [prefix split s ; own suffix window] for the stacked rows of a kv group.
+struct AttnArgs {
+  const void* q_rot;        // [Hkv, M, d]
+  const void* k_pre;        // [Lp, Hkv, d]
+  const void* v_pre;        // [Lp, Hkv, d]
+  const void* k_rot;        // [T, Hkv, d]
+  const void* v_suf;        // [T, Hkv, d]
+  const TokInfo* info;      // [T]
+  const int2* node_anc;     // tree: [n_nodes, kMaxDepth]; flat: nullptr
+  const int32_t* node_nanc; // tree: [n_nodes]; flat: nullptr
+  const int32_t* hinv;      // [Hq]
+  void* out;                // [T, Hq, d] (num_splits == 1)
+  float* lse;               // [T, Hq] or nullptr
+  float* o_part;            // [S, Hkv, M, d] (num_splits > 1)
+  float* l_part;            // [S, Hkv, M] log2-domain
+  int32_t* status;
+  int T, M, Lp, Hq, Hkv, G, d, S, split_len;  // split_len: prefix keys per split (multiple of 128)
+  float scale_log2;         // softmax scale * log2(e)
+};
+cudaError_t launch_attn_simt(const AttnArgs& a, jev_dtype dt, cudaStream_t s);
+cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t s);  // bf16, d in {64,128}
+bool attn_tc_supported(int d);
+
+struct MergeArgs {
+  const float* o_part;  // [S, Hkv, M, d]
+  const float* l_part;  // [S, Hkv, M]
+  const int32_t* hinv;
+  void* out;            // [T, Hq, d]
+  float* lse;
+  int M, Hq, Hkv, G, d, S;
+};
+cudaError_t launch_merge(const MergeArgs& a, jev_dtype dt, cudaStream_t s);
+
+struct ReadoutArgs {
+  const void* hidden; const void* lm_head;
+  const int32_t* set_offsets; const int32_t* cand_offsets; const int32_t* pair_row; const int32_t* pair_tok;
+  float* logprob; int32_t* choice; float* score;
+  int n_sets, n_cands, n_pairs, R, H, V;
+};
+cudaError_t launch_readout(const ReadoutArgs& a, jev_dtype dt, cudaStream_t s);
+
+cudaError_t launch_rope_inplace(void* x, int L, int H, int d, int pos0, double theta, jev_dtype dt,
+                                cudaStream_t s);
+
+}  // namespace jev

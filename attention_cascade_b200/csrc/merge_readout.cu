@@ -1,0 +1,177 @@
+// merge_readout.cu — log-sum-exp merge of split partials, and candidate readout.
+#include <math_constants.h>
+
+#include "kernels.h"
+
+namespace jev {
+namespace {
+
+// Merge of S partial softmaxes over disjoint key sets: with per-split
+// normalised outputs O_s and log2 normalisers L_s,
+//   L = log2 sum_s 2^L_s,   O = sum_s 2^(L_s - L) O_s.
+// This is exact (no approximation): attention over a union of key sets is the
+// normaliser-weighted average of the attentions over the parts.  One warp per
+// stacked row.
+template <typename T, int D>
+__global__ void __launch_bounds__(256) merge_kernel(MergeArgs a) {
+  constexpr int C = D / 32;
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const int rows = a.Hkv * a.M;
+  if (warp >= rows) return;
+  const int g = warp / a.M, m = warp - g * a.M;
+  float mx = -CUDART_INF_F;
+  for (int s = 0; s < a.S; ++s) mx = fmaxf(mx, a.l_part[((size_t)s * a.Hkv + g) * a.M + m]);
+  float acc[C];
+#pragma unroll
+  for (int c = 0; c < C; ++c) acc[c] = 0.f;
+  float wsum = 0.f;
+  if (mx != -CUDART_INF_F) {
+    for (int s = 0; s < a.S; ++s) {
+      const size_t r = ((size_t)s * a.Hkv + g) * a.M + m;
+      const float w = exp2f(a.l_part[r] - mx);
+      wsum += w;
+      const float* o = a.o_part + r * D;
+#pragma unroll
+      for (int c = 0; c < C; ++c) acc[c] += w * o[lane + 32 * c];
+    }
+  }
+  const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+  const int t = m / a.G;
+  const int h = min(max(a.hinv[g * a.G + (m - t * a.G)], 0), a.Hq - 1);
+  T* out = reinterpret_cast<T*>(a.out) + ((size_t)t * a.Hq + h) * D;
+#pragma unroll
+  for (int c = 0; c < C; ++c) out[lane + 32 * c] = from_f32<T>(acc[c] * inv);
+  if (a.lse && lane == 0)
+    a.lse[(size_t)t * a.Hq + h] = wsum > 0.f ? (mx + log2f(wsum)) * 0.69314718055994531f : -CUDART_INF_F;
+}
+
+// dot of two length-H rows with 16-byte loads, fp32 accumulation, warp-wide
+__device__ __forceinline__ float row_dot(const __nv_bfloat16* x, const __nv_bfloat16* w, int H, int lane) {
+  const uint4* x4 = reinterpret_cast<const uint4*>(x);
+  const uint4* w4 = reinterpret_cast<const uint4*>(w);
+  float acc = 0.f;
+  for (int i = lane; i < (H >> 3); i += 32) {
+    uint4 a = __ldg(x4 + i), b = __ldg(w4 + i);
+    const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
+    const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&b);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      float2 fa = __bfloat1622float2(a2[k]), fb = __bfloat1622float2(b2[k]);
+      acc = fmaf(fa.x, fb.x, acc);
+      acc = fmaf(fa.y, fb.y, acc);
+    }
+  }
+  return acc;
+}
+__device__ __forceinline__ float row_dot(const float* x, const float* w, int H, int lane) {
+  const float4* x4 = reinterpret_cast<const float4*>(x);
+  const float4* w4 = reinterpret_cast<const float4*>(w);
+  float acc = 0.f;
+  for (int i = lane; i < (H >> 2); i += 32) {
+    float4 a = __ldg(x4 + i), b = __ldg(w4 + i);
+    acc = fmaf(a.x, b.x, acc);
+    acc = fmaf(a.y, b.y, acc);
+    acc = fmaf(a.z, b.z, acc);
+    acc = fmaf(a.w, b.w, acc);
+  }
+  return acc;
+}
+
+// One block per option set.  Warps take the set's candidates in turn; a
+// candidate's score is the sum over its (row, token) pairs of
+// hidden[row] . lm_head[token], gathered with 16-byte loads (only option rows
+// of the LM head are ever read).  Scores are parked in `logprob`, then warp 0
+// forms the set's log-sum-exp and argmax (lowest index on ties) and rewrites
+// them as log-probabilities.
+template <typename T>
+__global__ void __launch_bounds__(128) readout_kernel(ReadoutArgs a) {
+  const int s = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ca = a.set_offsets[s], ce = a.set_offsets[s + 1];
+  const T* hid = reinterpret_cast<const T*>(a.hidden);
+  const T* W = reinterpret_cast<const T*>(a.lm_head);
+  const bool set_ok = ca >= 0 && ce >= ca && ce <= a.n_cands;
+  if (set_ok) {
+    for (int c = ca + warp; c < ce; c += 4) {
+      int pa = c, pe = c + 1;
+      if (a.cand_offsets) {
+        pa = a.cand_offsets[c];
+        pe = a.cand_offsets[c + 1];
+      }
+      float z = 0.f;
+      bool bad = pa < 0 || pe < pa || pe > a.n_pairs;
+      if (!bad) {
+        for (int k = pa; k < pe; ++k) {
+          const int row = a.pair_row ? a.pair_row[k] : s;
+          const int tok = a.pair_tok[k];
+          if (row < 0 || row >= a.R || tok < 0 || tok >= a.V) {
+            bad = true;
+            continue;
+          }
+          z += row_dot(hid + (size_t)row * a.H, W + (size_t)tok * a.H, a.H, lane);
+        }
+      }
+      z = warp_sum(z);
+      if (lane == 0) {
+        const float zz = bad ? CUDART_NAN_F : z;
+        a.logprob[c] = zz;
+        if (a.score) a.score[c] = zz;
+      }
+    }
+  }
+  __syncthreads();
+  if (warp != 0) return;
+  if (!set_ok || ce == ca) {
+    if (lane == 0) a.choice[s] = -1;
+    return;
+  }
+  float mx = -CUDART_INF_F;
+  int best = -1;
+  bool any_nan = false;
+  for (int c = ca + lane; c < ce; c += 32) {
+    const float z = a.logprob[c];
+    if (isnan(z)) any_nan = true;
+    else if (best < 0 || z > mx) { mx = z; best = c; }
+  }
+  any_nan = __any_sync(0xffffffffu, any_nan);
+  // warp argmax: larger value wins, lower index breaks ties
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float om = __shfl_xor_sync(0xffffffffu, mx, o);
+    const int ob = __shfl_xor_sync(0xffffffffu, best, o);
+    if (ob >= 0 && (best < 0 || om > mx || (om == mx && ob < best))) { mx = om; best = ob; }
+  }
+  float sum = 0.f;
+  for (int c = ca + lane; c < ce; c += 32) sum += exp2f((a.logprob[c] - mx) * 1.4426950408889634f);
+  sum = warp_sum(sum);
+  const float lse = mx + log2f(sum) * 0.69314718055994531f;
+  __syncwarp();
+  for (int c = ca + lane; c < ce; c += 32) a.logprob[c] = any_nan ? CUDART_NAN_F : a.logprob[c] - lse;
+  if (lane == 0) a.choice[s] = any_nan ? -1 : best - ca;
+}
+
+}  // namespace
+
+cudaError_t launch_merge(const MergeArgs& a, jev_dtype dt, cudaStream_t s) {
+  const int rows = a.Hkv * a.M;
+  if (rows == 0) return cudaSuccess;
+  const int blocks = (rows * 32 + 255) / 256;
+  if (dt == JEV_BF16) {
+    if (a.d == 64) merge_kernel<__nv_bfloat16, 64><<<blocks, 256, 0, s>>>(a);
+    else merge_kernel<__nv_bfloat16, 128><<<blocks, 256, 0, s>>>(a);
+  } else {
+    if (a.d == 64) merge_kernel<float, 64><<<blocks, 256, 0, s>>>(a);
+    else merge_kernel<float, 128><<<blocks, 256, 0, s>>>(a);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_readout(const ReadoutArgs& a, jev_dtype dt, cudaStream_t s) {
+  if (a.n_sets == 0) return cudaSuccess;
+  if (dt == JEV_BF16) readout_kernel<__nv_bfloat16><<<a.n_sets, 128, 0, s>>>(a);
+  else readout_kernel<float><<<a.n_sets, 128, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace jev

@@ -1,0 +1,478 @@
+#!/usr/bin/env python3
+"""Throughput of the shared-prefix attention + candidate readout hot path.
+
+One step = one jev_prefix_suffix_attn (one attention layer, all heads, all
+branches) + one jev_candidate_readout over one batch of synthetic input (the
+tree workload: jev_tree_attn + readout).  The headline metric is suffix
+tokens/s.  Steps are replayed from CUDA graphs over rotating copies of the
+inputs whose total size exceeds twice the L2, so every step reads its prefix
+cache and suffix tensors from HBM.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c1] [--impl jev|reference]
+
+With N > 1 (torchrun) every rank runs an independent replica of the workload
+on its own GPU (no collective on the data path; weak scaling); the step time
+is the max over ranks.  --impl reference times the fp64 CPU oracle on the
+host cores instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "suffix tokens/s (shared-prefix attn + readout) and % of roofline, 1 B200"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+# ----------------------------------------------------------------------------- algorithmic work
+
+
+def flat_work(c) -> dict:
+    """Algorithmic FLOPs and unique bytes of one step (prefix K/V counted once)."""
+    cfg = c.cfg
+    s = 2 if cfg.dtype == synth.BF16 else 4
+    Ls = np.diff(c.cu_seqlens).astype(np.int64)
+    T = int(Ls.sum())
+    f_attn = 4 * T * cfg.Hq * cfg.Lp * cfg.d + 4 * cfg.Hq * cfg.d * int((Ls * (Ls + 1) // 2).sum())
+    n_pairs = int(c.pair_tok.size)
+    f_read = 2 * cfg.H * n_pairs
+    b_attn = s * (2 * T * cfg.Hq * cfg.d + 2 * cfg.Lp * cfg.Hkv * cfg.d + 2 * T * cfg.Hkv * cfg.d) + 4 * T * cfg.Hq
+    b_read = s * (cfg.B * cfg.H + n_pairs * cfg.H) + 8 * n_pairs + 4 * cfg.B
+    return dict(T=T, B=cfg.B, flops_attn=f_attn, flops_readout=f_read, bytes_attn=b_attn, bytes_readout=b_read)
+
+
+# ----------------------------------------------------------------------------- clocks
+
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap,utilization.gpu")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"jev_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                p = [x.strip() for x in line.split(",")]
+                if len(p) >= 10:
+                    rows.append(p)
+        os.remove(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        loaded = [r for r in rows if (num(r[9]) or 0) > 0] or rows
+        sm = [num(r[1]) for r in loaded if num(r[1]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in loaded for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": num(rows[0][2]),
+                "reasons": reasons, "samples": len(rows), "samples_under_load": len(loaded),
+                "power_w_max": max((num(r[3]) or 0) for r in rows)}
+
+
+# ----------------------------------------------------------------------------- reference arm (oracle on CPU)
+
+
+class OracleSampler:
+    """Times the fp64 oracle on bounded samples of a flat workload and scales
+    the sample times to the whole workload: attention is sampled by (token,
+    head) rows, the readout (full-vocabulary logits + log-softmax) by option
+    sets.  Workload time = rows * (time per sampled row) + sets * (time per
+    sampled set); tokens/s = suffix tokens / workload time."""
+
+    def __init__(self, cfg):
+        import oracle
+        self.oracle = oracle
+        self.cfg = cfg
+        self.c = synth.flat_case(cfg, with_lm_head=False)
+        self.W = synth.lm_head(cfg.seed, cfg.V, cfg.H, cfg.dtype, cfg.w_std)
+        self.T = self.c.T
+        self.rng = np.random.default_rng(1234)
+        self.t_rows = self.n_rows = 0
+        self.t_sets = self.n_sets = 0
+        self.cost_row = self._attn(16)[0] / 16
+        self.cost_set = self._readout(1)[0]
+        self.t_rows = self.n_rows = self.t_sets = self.n_sets = 0
+
+    def _attn(self, n):
+        c = self.c
+        rows = np.stack([self.rng.integers(0, self.T, n), self.rng.integers(0, self.cfg.Hq, n)], 1).astype(np.int32)
+        t0 = time.perf_counter()
+        self.oracle.prefix_suffix_attn(c.q, c.k_pre, c.v_pre, c.k_suf, c.v_suf, c.cu_seqlens, theta=self.cfg.theta,
+                                       rows=rows)
+        dt = time.perf_counter() - t0
+        self.t_rows += dt
+        self.n_rows += n
+        return dt, n
+
+    def _readout(self, n):
+        c = self.c
+        s0 = int(self.rng.integers(0, self.cfg.B - n + 1))
+        so = c.set_offsets[s0:s0 + n + 1] - c.set_offsets[s0]
+        toks = c.pair_tok[c.set_offsets[s0]:c.set_offsets[s0 + n]]
+        t0 = time.perf_counter()
+        self.oracle.candidate_readout(c.hidden[s0:s0 + n], self.W, so, toks, full_vocab=True)
+        dt = time.perf_counter() - t0
+        self.t_sets += dt
+        self.n_sets += n
+        return dt, n
+
+    def step(self, budget_s):
+        """One sample costing about budget_s: attention rows and readout sets
+        in proportion to their share of the whole workload's oracle time."""
+        full_attn = self.cost_row * self.T * self.cfg.Hq
+        full_read = self.cost_set * self.cfg.B
+        f_attn = full_attn / (full_attn + full_read)
+        n_rows = int(max(1, min(self.T * self.cfg.Hq, f_attn * budget_s / self.cost_row)))
+        self._attn(n_rows)
+        n_sets = int(min(self.cfg.B, (1 - f_attn) * budget_s / self.cost_set))
+        if n_sets >= 1 or self.n_sets == 0:
+            self._readout(max(1, n_sets))
+
+    def tokens_per_s(self):
+        t = (self.t_rows / self.n_rows) * self.T * self.cfg.Hq + (self.t_sets / self.n_sets) * self.cfg.B
+        return self.T / t
+
+    def describe(self):
+        return (f"{self.n_rows} (token, head) attention rows and {self.n_sets} option sets (full-vocabulary logits) "
+                f"of the workload ({self.T} tokens x {self.cfg.Hq} heads, {self.cfg.B} sets), {self.t_rows + self.t_sets:.1f} s "
+                f"of oracle time, scaled to the whole workload")
+
+
+def reference_arm(args, wl_name):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    cfg = synth.CONFIGS[wl_name]
+    if isinstance(cfg, synth.TreeConfig):
+        print(json.dumps({"impl": "reference", "unavailable": "the oracle's tree arm is timed only by the parity tests"}))
+        return
+    total_budget = float(os.environ.get("JEV_REF_TOTAL_S", "120"))
+    per_step = max(0.002, total_budget / (args.steps + args.warmup))
+    smp = OracleSampler(cfg)
+    for _ in range(args.warmup):
+        smp.step(per_step)
+    smp.t_rows = smp.n_rows = smp.t_sets = smp.n_sets = 0
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        smp.step(per_step)
+    wall = time.perf_counter() - t0
+    value = smp.tokens_per_s()
+    cores = host_cores()
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * wall / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": synth.WORKLOAD_TEXT[wl_name], "global_batch": cfg.B,
+                                            "seq_len": cfg.Lp, "parallelism": "cpu"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": "all timed steps together: " + smp.describe()},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+
+
+# ----------------------------------------------------------------------------- jev arm
+
+
+def traffic_of(kernel: str, workload: str, src_files):
+    """DRAM traffic per launch from a committed ncu summary, if the kernel's
+    sources have not changed since it was taken (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(f"{kernel}/{workload}")
+    if not e:
+        return None
+    h = hashlib.sha256()
+    for fn in src_files:
+        with open(os.path.join(ROOT, fn), "rb") as f:
+            h.update(f.read())
+    return e["bytes_per_launch"] if e.get("src_sha256") == h.hexdigest() else None
+
+
+KERNEL_SRC = {
+    "attn_tc": ["attention_cascade_b200/csrc/attn_tc.cu", "attention_cascade_b200/csrc/common.cuh"],
+    "attn_simt": ["attention_cascade_b200/csrc/attn_simt.cu", "attention_cascade_b200/csrc/common.cuh"],
+}
+
+
+def jev_arm(args, wl_name):
+    import torch
+    import torch.distributed as dist
+    import attention_cascade_b200 as jev
+    from attention_cascade_b200 import _build  # noqa: F401  (the library is loaded at import)
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    cfg = synth.CONFIGS[wl_name]
+    if isinstance(cfg, synth.TreeConfig):
+        raise SystemExit("bench.py: the tree workload is measured by the parity tests; use a flat workload")
+
+    # ---- inputs (host generation, one copy; device clones to exceed L2)
+    c = synth.flat_case(cfg, with_lm_head=False)
+    work = flat_work(c)
+    tdt = torch.bfloat16 if cfg.dtype == synth.BF16 else torch.float32
+
+    def to_dev(a):
+        if a.dtype == np.uint16:
+            return torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
+        return torch.from_numpy(a).to(dev)
+
+    W = torch.empty((cfg.V, cfg.H), dtype=tdt, device=dev)
+    for ch in range((cfg.V + synth.W_CHUNK_ROWS - 1) // synth.W_CHUNK_ROWS):
+        blk = synth.lm_head_block(cfg.seed, cfg.V, cfg.H, ch, cfg.dtype, cfg.w_std)
+        W[ch * synth.W_CHUNK_ROWS: ch * synth.W_CHUNK_ROWS + blk.shape[0]] = to_dev(blk)
+    base = dict(q=to_dev(c.q), k_pre=to_dev(c.k_pre), v_pre=to_dev(c.v_pre), k_suf=to_dev(c.k_suf),
+                v_suf=to_dev(c.v_suf), hidden=to_dev(c.hidden), pair_tok=to_dev(c.pair_tok))
+    per_copy = sum(t.numel() * t.element_size() for t in base.values())
+    ncopies = max(2, math.ceil(2 * L2_BYTES / per_copy))
+    copies = []
+    for i in range(ncopies):
+        cp = {k: v.clone() for k, v in base.items()}
+        # each copy reads different option rows of the LM head
+        cp["pair_tok"] = ((base["pair_tok"].long() + 7919 * i) % cfg.V).to(torch.int32)
+        copies.append(cp)
+    cu = to_dev(c.cu_seqlens)
+    so = to_dev(c.set_offsets)
+    T = work["T"]
+    desc = jev.make_attn_desc(cfg.B, cfg.Lp, cfg.Hq, cfg.Hkv, cfg.d, T, jev.JEV_BF16 if tdt == torch.bfloat16 else jev.JEV_F32,
+                              cfg.theta)
+    ws = jev.new_workspace(jev.jev_prefix_suffix_attn_workspace(desc), dev)
+    out = torch.empty_like(base["q"])
+    lse = torch.empty((T, cfg.Hq), dtype=torch.float32, device=dev)
+    lp = torch.empty(c.pair_tok.size, dtype=torch.float32, device=dev)
+    choice = torch.empty(cfg.B, dtype=torch.int32, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    def step(cp, s):
+        jev.jev_prefix_suffix_attn(cp["q"], cp["k_pre"], cp["v_pre"], cp["k_suf"], cp["v_suf"], cu, out=out, lse=lse,
+                                   workspace=ws, rope_theta=cfg.theta, stream=s)
+        jev.jev_candidate_readout(cp["hidden"], W, so, cp["pair_tok"], logprob=lp, choice=choice, stream=s)
+
+    # ---- graphs: one per input copy (at most one per timed step).  Kernel
+    # timing is on while they are captured, so every kernel launch in them is
+    # bracketed by CUDA event nodes on the launching stream.
+    with torch.cuda.stream(stream):
+        for i in range(3):
+            step(copies[i % ncopies], stream)
+    stream.synchronize()
+    ngraph = max(1, min(ncopies, args.steps))
+    jev.jev_profile_read()
+    jev.jev_profile_enable(True)
+    n0 = jev.jev_launch_count()
+    graphs = []
+    for cp in copies[:ngraph]:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            step(cp, torch.cuda.current_stream())
+        graphs.append(g)
+    launches_per_step = (jev.jev_launch_count() - n0) // ngraph
+    jev.jev_profile_enable(False)
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            graphs[i % ngraph].replay()
+    stream.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for i in range(args.steps):
+            graphs[i % ngraph].replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms = e0.elapsed_time(e1)
+    clk = clocks.stop()
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    assert jev.jev_check_device_status(ws, stream) == 0, "device status flags set during the bench"
+    # per-kernel durations: each graph's event nodes hold its last replay in the timed region
+    prof = jev.jev_profile_read()
+
+    # ---- end to end through the public API: pinned host inputs in, results out, every step
+    hq = {k: base[k].cpu().pin_memory() for k in ("q", "k_suf", "v_suf", "hidden", "pair_tok")}
+    h_cu = cu.cpu().pin_memory()
+    h_so = so.cpu().pin_memory()
+    d_in = {k: torch.empty_like(base[k]) for k in hq}
+    d_cu, d_so = torch.empty_like(cu), torch.empty_like(so)
+    h_lp = torch.empty(lp.shape, dtype=lp.dtype).pin_memory()
+    h_ch = torch.empty(choice.shape, dtype=choice.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in hq.values()) + h_cu.numel() * 4 + h_so.numel() * 4
+    d2h = h_lp.numel() * 4 + h_ch.numel() * 4
+    k_pre, v_pre = base["k_pre"], base["v_pre"]
+
+    def e2e_step(s):
+        for k in hq:
+            d_in[k].copy_(hq[k], non_blocking=True)
+        d_cu.copy_(h_cu, non_blocking=True)
+        d_so.copy_(h_so, non_blocking=True)
+        jev.jev_prefix_suffix_attn(d_in["q"], k_pre, v_pre, d_in["k_suf"], d_in["v_suf"], d_cu, out=out, lse=lse,
+                                   workspace=ws, rope_theta=cfg.theta, stream=s)
+        jev.jev_candidate_readout(d_in["hidden"], W, d_so, d_in["pair_tok"], logprob=lp, choice=choice, stream=s)
+        h_lp.copy_(lp, non_blocking=True)
+        h_ch.copy_(choice, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.warmup)):
+            e2e_step(stream)
+    stream.synchronize()
+    if world > 1:
+        dist.barrier()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        f0.record(stream)
+        for _ in range(args.steps):
+            e2e_step(stream)
+        f1.record(stream)
+    stream.synchronize()
+    e2e_ms = f0.elapsed_time(f1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    # ---- roofline of the dominant kernel
+    pk, src = peaks()
+    attn_name = "attn_tc" if "attn_tc" in prof else "attn_simt"
+    dom = max(prof.items(), key=lambda kv: kv[1][1])[0] if prof else attn_name
+    n_l, t_ms = prof.get(attn_name, (1, float("nan")))
+    avg_s = t_ms / 1e3 / max(n_l, 1)
+    achieved = work["flops_attn"] / avg_s / 1e12
+    peak = float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"]))
+    per_kernel = {k: {"launches": v[0], "avg_us": 1e3 * v[1] / max(v[0], 1), "share": v[1] / sum(x[1] for x in prof.values())}
+                  for k, v in prof.items()}
+    step_s = ms / 1e3 / args.steps
+    ideal = max((work["flops_attn"] + work["flops_readout"]) / (float(pk["bf16_tflops"]) * 1e12),
+                (work["bytes_attn"] + work["bytes_readout"]) / (float(pk["hbm_gbs"]) * 1e9))
+    value = world * T * args.steps / (ms / 1e3)
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16" if cfg.dtype == synth.BF16 else "f32", "data": "synthetic",
+        "config": {"workload": synth.WORKLOAD_TEXT[wl_name], "global_batch": cfg.B * world, "seq_len": cfg.Lp,
+                   "suffix_tokens_per_replica": T, "parallelism": f"replicas{world}" if world > 1 else "single",
+                   "l2": f"inputs rotate over {ncopies} device copies ({ncopies * per_copy / 2**20:.0f} MiB > 2x L2)",
+                   "timing": "CUDA graph replay per step, CUDA events on the launching stream; per-kernel times "
+                             "from event nodes around each kernel in the replayed graphs"},
+        "branches_per_s": world * cfg.B * args.steps / (ms / 1e3),
+        "clocks": clk,
+        "e2e": {"value": world * T * args.steps / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h,
+                "note": "per step: pinned H2D of suffix q/k/v, cu_seqlens, hidden rows, option sets; both C-ABI "
+                        "calls; D2H of log-probs and choices (prefix cache and LM head stay resident)"},
+        "gpu_launches": launches_per_step * args.steps,
+        "roofline": {"bound": "tensor", "kernel": attn_name, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": traffic_of(attn_name, wl_name, KERNEL_SRC[attn_name]),
+                     "peak_source": f"bf16_tflops_sustained, {src}",
+                     "frac_of_burst_peak": achieved / float(pk["bf16_tflops"]),
+                     "algorithmic_flops_per_launch": work["flops_attn"], "dominant_kernel_by_time": dom},
+        "step_roofline": {"ideal_us": ideal * 1e6, "measured_us": step_s * 1e6, "frac": ideal / step_s,
+                          "definition": "max(F / bf16 burst peak, U / HBM peak) over the whole step"},
+        "kernels": per_kernel,
+    }
+    if rank == 0 and world == 1 and os.environ.get("JEV_SKIP_CPU_BASELINE") != "1":
+        del graphs
+        budget = float(os.environ.get("JEV_CPU_BASELINE_S", "12"))
+        smp = OracleSampler(cfg)
+        t0 = time.perf_counter()
+        while time.perf_counter() - t0 < budget:
+            smp.step(min(2.0, budget / 4))
+        line["cpu_baseline"] = {"value": smp.tokens_per_s(), "unit": "tokens/s", "cores": host_cores(),
+                                "kind": "oracle", "sample": smp.describe()}
+    if rank == 0:
+        print(json.dumps(line))
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--workload", default="c1", choices=sorted(synth.CONFIGS))
+    ap.add_argument("--impl", default="jev", choices=["jev", "reference"])
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("bench.py: at least 3 warm-up steps")
+    if args.impl == "reference":
+        reference_arm(args, args.workload)
+    else:
+        jev_arm(args, args.workload)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,116 @@
+"""C-ABI checks that need no GPU: the library loads, exports every entry point
+include/jev.h declares, rejects bad arguments on the host before anything is
+enqueued, and its host-side trie / readout planning matches the oracle bit
+for bit."""
+import ctypes as C
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def jev():
+    from attention_cascade_b200 import _build
+    _build.build()
+    import attention_cascade_b200 as m
+    return m
+
+
+def _declared():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names |= set(re.findall(r"\b(jev_[a-z0-9_]+)\s*\(", src))
+    return names
+
+
+def test_exports_every_declared_symbol(jev):
+    names = _declared()
+    assert {"jev_prefix_suffix_attn", "jev_candidate_readout", "jev_tree_attn", "jev_tree_build"} <= names
+    lib = C.CDLL(jev.LIB_PATH)
+    missing = [n for n in sorted(names) if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_host_rejects_bad_arguments(jev):
+    lib = jev._lib
+    d = jev.make_attn_desc(2, 16, 4, 2, 96, 8, jev.JEV_BF16)
+    assert lib.jev_prefix_suffix_attn(C.byref(d), *([None] * 10), 0, None) == 2  # d = 96 unsupported
+    d = jev.make_attn_desc(2, 16, 6, 4, 64, 8, jev.JEV_BF16)
+    assert lib.jev_prefix_suffix_attn(C.byref(d), *([None] * 10), 0, None) == 1  # Hq % Hkv
+    d = jev.make_attn_desc(2, 16, 4, 2, 64, 8, jev.JEV_BF16)
+    assert lib.jev_prefix_suffix_attn(C.byref(d), *([None] * 10), 0, None) == 1  # NULL q
+    assert "NULL" in jev.jev_last_error()
+    fake = 1 << 20  # never dereferenced: the workspace check fails first
+    st = lib.jev_prefix_suffix_attn(C.byref(d), fake, fake, fake, fake, fake, fake, None, fake, None, fake, 64, None)
+    assert st == 3 and "workspace" in jev.jev_last_error()
+    st = lib.jev_prefix_suffix_attn(C.byref(d), fake + 2, fake, fake, fake, fake, fake, None, fake, None, fake, 1 << 30, None)
+    assert st == 1 and "aligned" in jev.jev_last_error()
+    d0 = jev.make_attn_desc(0, 16, 4, 2, 64, 0, jev.JEV_BF16)
+    assert lib.jev_prefix_suffix_attn(C.byref(d0), *([None] * 10), 0, None) == 0  # empty: no work
+    r = jev.jev_readout_desc(3, 5, 5, 3, 100, 1000, jev.JEV_BF16)  # H not a multiple of 8
+    assert lib.jev_candidate_readout(C.byref(r), *([None] * 10)) == 2
+
+
+def test_workspace_size_is_monotone(jev):
+    small = jev.jev_prefix_suffix_attn_workspace(jev.make_attn_desc(4, 256, 2, 1, 64, 64, jev.JEV_F32))
+    big = jev.jev_prefix_suffix_attn_workspace(jev.make_attn_desc(128, 4096, 28, 4, 128, 3072, jev.JEV_BF16))
+    assert 256 < small < big
+    # q_rot (bf16) for 3072 tokens x 28 heads x 128 fits in the wide workspace
+    assert big >= 3072 * 28 * 128 * 2
+
+
+def _csr(cands):
+    so = np.concatenate([[0], np.cumsum([len(c) for c in cands])]).astype(np.int32)
+    return so, np.array([t for c in cands for t in c], np.int32)
+
+
+def test_tree_build_matches_oracle_bitwise(jev):
+    rng = np.random.default_rng(7)
+    for trial in range(300):
+        n = int(rng.integers(1, 12))
+        vocab = int(rng.integers(2, 6))
+        cands = [list(rng.integers(0, vocab, int(rng.integers(0, 8)))) for _ in range(n)]
+        so, toks = _csr(cands)
+        root = int(rng.integers(0, 3000))
+        a = jev.jev_tree_build(so, toks, root)
+        b = oracle.trie_build(so, toks, root)
+        for k in ("parent", "tok_off", "pos0", "leaf_of", "node_toks", "path_row"):
+            assert np.array_equal(a[k], b[k]), (k, cands)
+        assert a["n_nodes"] == b["n_nodes"]
+
+
+def test_tree_build_on_tree_workload(jev):
+    import synth
+    tc = synth.tree_case(synth.CONFIGS["c4"], with_lm_head=False)
+    a = jev.jev_tree_build(tc.seq_off, tc.toks, tc.cfg.Lp)
+    b = oracle.trie_build(tc.seq_off, tc.toks, tc.cfg.Lp)
+    for k in ("parent", "tok_off", "pos0", "leaf_of", "node_toks", "path_row"):
+        assert np.array_equal(a[k], b[k])
+    assert a["tok_off"][-1] == tc.n_unique
+    assert a["n_nodes"] == 1 + 16 + tc.seq_off.size - 1  # root + questions + one node per option
+    plan = jev.jev_tree_readout_plan(tc.seq_off, tc.toks, tc.score_from, a["path_row"])
+    co, prow, tix = oracle.tree_readout_pairs(tc.seq_off, tc.score_from, b["path_row"], tc.set_offsets)
+    assert np.array_equal(plan["cand_offsets"], co)
+    assert np.array_equal(plan["pair_row"], prow)
+    assert np.array_equal(plan["pair_tok"], tc.toks[tix])
+
+
+def test_tree_build_capacity_and_errors(jev):
+    so, toks = _csr([[1, 2, 3], [1, 4]])
+    lib = jev._lib
+    parent = np.zeros(2, np.int32); tok_off = np.zeros(3, np.int32); pos0 = np.zeros(2, np.int32)
+    leaf = np.zeros(2, np.int32); nt = np.zeros(8, np.int32); nn = C.c_int32()
+    st = lib.jev_tree_build(2, so.ctypes.data, toks.ctypes.data, 0, 2, 8, parent.ctypes.data, tok_off.ctypes.data,
+                            pos0.ctypes.data, leaf.ctypes.data, nt.ctypes.data, None, C.byref(nn))
+    assert st == 6  # JEV_ERR_CAPACITY
+    with pytest.raises(jev.JevError):
+        jev.jev_tree_readout_plan(so, toks, np.array([0, 1], np.int32), np.zeros(5, np.int32))

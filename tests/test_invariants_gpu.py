@@ -1,0 +1,132 @@
+"""GPU invariants the pages state ("Ochevid Jev-VL 2B" model card, Evidence:
+question order, added questions and unequal tail lengths preserve answers;
+Runtime 0.2: repeated runs reproduce probabilities exactly; the answers match
+serial execution), plus split-count invariance, empty inputs and the device
+status word on malformed inputs (which must flag, never fault)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from gpu_helpers import TOL, dev, host_f64
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def jev():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import attention_cascade_b200 as m
+    return m
+
+
+def _case(lens, seed=0, dtype=synth.BF16, Lp=640, Hq=14, Hkv=2, d=128):
+    cfg = synth.FlatConfig("inv", dtype, Lp, len(lens), 1, 1, Hq, Hkv, d, 16, 32, 2, 3, seed=seed)
+    return synth.flat_case(cfg, with_lm_head=False, lengths=np.array(lens, np.int32))
+
+
+def _run(jev, c, **kw):
+    out, lse = jev.jev_prefix_suffix_attn(*(dev(x) for x in (c.q, c.k_pre, c.v_pre, c.k_suf, c.v_suf)),
+                                          dev(c.cu_seqlens), **kw)
+    torch.cuda.synchronize()
+    return out, lse
+
+
+def test_repeat_runs_are_bit_identical(jev):
+    c = _case([13, 29, 7, 40, 1])
+    a = _run(jev, c)
+    b = _run(jev, c)
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+def test_branch_order_and_insertion(jev):
+    lens = [13, 29, 7, 40, 1, 22]
+    c = _case(lens, seed=1)
+    out, lse = _run(jev, c, num_splits=2)
+    perm = [3, 0, 5, 2, 1, 4]
+    cu = c.cu_seqlens
+    idx = np.concatenate([np.arange(cu[b], cu[b + 1]) for b in perm])
+    c2 = synth.FlatCase(c.cfg, c.q[idx], c.k_pre, c.v_pre, c.k_suf[idx], c.v_suf[idx],
+                        np.concatenate([[0], np.cumsum(np.array(lens)[perm])]).astype(np.int32),
+                        c.hidden, c.set_offsets, c.pair_tok)
+    o2, l2 = _run(jev, c2, num_splits=2)
+    tol = TOL[synth.BF16]
+    assert (o2.float() - out[torch.from_numpy(idx).cuda()].float()).abs().max().item() <= tol["max_abs"] / 2
+    assert (l2 - lse[torch.from_numpy(idx).cuda()]).abs().max().item() <= 1e-3
+    # serial: each branch alone matches its rows in the batch
+    for b in range(len(lens)):
+        sl = slice(cu[b], cu[b + 1])
+        cb = synth.FlatCase(c.cfg, c.q[sl], c.k_pre, c.v_pre, c.k_suf[sl], c.v_suf[sl],
+                            np.array([0, lens[b]], np.int32), c.hidden, c.set_offsets, c.pair_tok)
+        ob, lb = _run(jev, cb, num_splits=2)
+        assert (ob.float() - out[cu[b]:cu[b + 1]].float()).abs().max().item() <= tol["max_abs"] / 2
+        assert (lb - lse[cu[b]:cu[b + 1]]).abs().max().item() <= 1e-3
+
+
+@pytest.mark.parametrize("dtype", [synth.BF16, synth.F32])
+def test_split_count_invariance(jev, dtype):
+    c = _case([31, 9, 18], seed=2, dtype=dtype, Lp=1500)
+    outs = [_run(jev, c, num_splits=s) for s in (1, 2, 5, 0)]
+    tol = 2e-2 if dtype == synth.BF16 else 1e-5
+    for o, l in outs[1:]:
+        assert (o.float() - outs[0][0].float()).abs().max().item() <= tol
+        assert (l - outs[0][1]).abs().max().item() <= (1e-3 if dtype == synth.BF16 else 1e-5)
+
+
+def test_empty_inputs(jev):
+    z = torch.zeros((0, 4, 64), dtype=torch.bfloat16, device="cuda")
+    kp = torch.zeros((16, 2, 64), dtype=torch.bfloat16, device="cuda")
+    n0 = jev.jev_launch_count()
+    out, lse = jev.jev_prefix_suffix_attn(z, kp, kp, z[:, :2], z[:, :2], torch.zeros(1, dtype=torch.int32, device="cuda"))
+    assert out.numel() == 0 and jev.jev_launch_count() == n0
+    # branches that all have an empty suffix: nothing to compute
+    out, lse = jev.jev_prefix_suffix_attn(z, kp, kp, z[:, :2], z[:, :2],
+                                          torch.zeros(4, dtype=torch.int32, device="cuda"))
+    assert jev.jev_launch_count() == n0
+
+
+def test_status_word_flags_bad_inputs_without_faulting(jev):
+    c = _case([5, 6, 7], seed=3, Lp=128)
+    q, kp, vp, ks, vs = (dev(x) for x in (c.q, c.k_pre, c.v_pre, c.k_suf, c.v_suf))
+    desc = jev.make_attn_desc(3, 128, 14, 2, 128, 18, jev.JEV_BF16)
+    ws = jev.new_workspace(jev.jev_prefix_suffix_attn_workspace(desc), "cuda")
+    bad_cu = torch.tensor([0, 9, 4, 18], dtype=torch.int32, device="cuda")  # decreasing
+    jev.jev_prefix_suffix_attn(q, kp, vp, ks, vs, bad_cu, workspace=ws)
+    assert jev.jev_check_device_status(ws) & jev.JEV_DEV_BAD_SEQLENS
+    bad_hm = torch.tensor([0] * 14, dtype=torch.int32, device="cuda")  # every head on kv 0
+    jev.jev_prefix_suffix_attn(q, kp, vp, ks, vs, dev(c.cu_seqlens), head_map=bad_hm, workspace=ws)
+    assert jev.jev_check_device_status(ws) & jev.JEV_DEV_BAD_HEAD_MAP
+    # the status word was cleared by the read; a good call leaves it clean
+    jev.jev_prefix_suffix_attn(q, kp, vp, ks, vs, dev(c.cu_seqlens), workspace=ws)
+    assert jev.jev_check_device_status(ws) == 0
+    # the context is still healthy
+    torch.cuda.synchronize()
+    assert torch.isfinite(torch.ones(4, device="cuda").sum())
+
+
+def test_tree_status_flags_deep_chain(jev):
+    # a chain of 10 single-token nodes (each candidate ends one token deeper) exceeds the depth limit of 8
+    cands = [list(range(1, k + 1)) for k in range(1, 11)]
+    so = np.concatenate([[0], np.cumsum([len(x) for x in cands])]).astype(np.int32)
+    toks = np.array([t for x in cands for t in x], np.int32)
+    t = jev.jev_tree_build(so, toks, 64)
+    assert t["n_nodes"] == 11
+    N = int(t["tok_off"][-1])
+    rng = np.random.default_rng(0)
+    mk = lambda *s: dev(synth.f32_to_bf16_bits(rng.standard_normal(s).astype(np.float32)))
+    q, k, v, kr, vr = mk(N, 4, 64), mk(N, 2, 64), mk(N, 2, 64), mk(64, 2, 64), mk(64, 2, 64)
+    desc = jev.make_attn_desc(10, 64, 4, 2, 64, N, jev.JEV_BF16)
+    ws = jev.new_workspace(jev.jev_tree_attn_workspace(desc, 11), "cuda")
+    out, lse = jev.jev_tree_attn(dev(t["parent"]), dev(t["tok_off"]), dev(t["pos0"]), q, kr, vr, k, v, workspace=ws)
+    flags = jev.jev_check_device_status(ws)
+    assert flags & jev.JEV_DEV_BAD_TREE
+    # rows of nodes within the depth limit are still correct
+    ref_o, _ = oracle.tree_attn(oracle.trie_build(so, toks, 64), synth.f32_to_bf16_bits(host_f64(q).astype(np.float32)),
+                                synth.f32_to_bf16_bits(host_f64(k).astype(np.float32)),
+                                synth.f32_to_bf16_bits(host_f64(v).astype(np.float32)),
+                                synth.f32_to_bf16_bits(host_f64(kr).astype(np.float32)),
+                                synth.f32_to_bf16_bits(host_f64(vr).astype(np.float32)))
+    ok_rows = 8  # nodes 1..8 have depth <= 8
+    assert np.abs(host_f64(out)[:ok_rows] - ref_o[:ok_rows]).max() <= TOL[synth.BF16]["max_abs"]

@@ -1,0 +1,186 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle on the
+same seeded inputs, element by element.
+
+* c0 and c1 are compared on every output element (c1 readout against the
+  oracle's full-vocabulary logits, the pages' plain definition).
+* c2 and c3 run at full size in the launch configuration bench.py times
+  (automatic split count, default kernel) and are compared on sampled rows the
+  oracle forms one by one: every branch's first and last token at every head
+  plus random rows; the readout is compared on every set.
+* Small cases cover the edges: ragged prefix tails, Lp = 0, empty and
+  one-token branches, a suffix longer than a key tile, MHA (G = 1), G = 7,
+  d = 64 and 128, explicit head maps, forced split counts, a position offset.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from gpu_helpers import NEAR_TIE, TOL, check_attn, check_readout, compact_lm_head, dev, host_f64
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def jev():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import attention_cascade_b200 as m
+    return m
+
+
+def run_flat(jev, c, **kw):
+    q, kp, vp, ks, vs = (dev(x) for x in (c.q, c.k_pre, c.v_pre, c.k_suf, c.v_suf))
+    cu = dev(c.cu_seqlens)
+    ws_kw = {}
+    if "head_map" in kw and kw["head_map"] is not None:
+        kw["head_map"] = dev(np.asarray(kw["head_map"], np.int32))
+    out, lse = jev.jev_prefix_suffix_attn(q, kp, vp, ks, vs, cu, **kw, **ws_kw)
+    torch.cuda.synchronize()
+    return host_f64(out), host_f64(lse)
+
+
+def run_readout(jev, hidden, W_dev, so, toks, **kw):
+    extra = {k: (dev(np.asarray(v, np.int32)) if v is not None else None) for k, v in kw.items()}
+    lp, ch = jev.jev_candidate_readout(dev(hidden), W_dev, dev(so), dev(toks.astype(np.int32)), **extra)
+    torch.cuda.synchronize()
+    return lp.cpu().numpy().astype(np.float64), ch.cpu().numpy()
+
+
+@pytest.mark.parametrize("name", ["c0", "c1"])
+def test_flat_config_every_element(jev, name):
+    cfg = synth.CONFIGS[name]
+    c = synth.flat_case(cfg)
+    out, lse = run_flat(jev, c, rope_theta=cfg.theta)
+    ref_o, ref_l = oracle.prefix_suffix_attn(c.q, c.k_pre, c.v_pre, c.k_suf, c.v_suf, c.cu_seqlens, theta=cfg.theta)
+    check_attn(out, lse, ref_o, ref_l, cfg.dtype, name)
+    ref = oracle.candidate_readout(c.hidden, c.W, c.set_offsets, c.pair_tok, full_vocab=True)
+    lp, ch = run_readout(jev, c.hidden, dev(c.W), c.set_offsets, c.pair_tok)
+    check_readout(lp, ch, ref, cfg.dtype, name)
+
+
+def _sample_rows(c, n_random, seed):
+    rng = np.random.default_rng(seed)
+    cu = c.cu_seqlens
+    Hq = c.cfg.Hq
+    toks = []
+    for b in range(cu.size - 1):
+        if cu[b + 1] > cu[b]:
+            toks += [cu[b], cu[b + 1] - 1]
+    rows = [(t, h) for t in sorted(set(toks)) for h in range(Hq)]
+    rows += [(int(rng.integers(0, c.T)), int(rng.integers(0, Hq))) for _ in range(n_random)]
+    return np.array(rows, np.int32)
+
+
+@pytest.mark.parametrize("name", ["c2", "c3"])
+def test_flat_config_full_size_sampled(jev, name):
+    cfg = synth.CONFIGS[name]
+    c = synth.flat_case(cfg, with_lm_head=False)
+    out, lse = run_flat(jev, c, rope_theta=cfg.theta)
+    rows = _sample_rows(c, 300, seed=7)
+    ref_o, ref_l = oracle.prefix_suffix_attn(c.q, c.k_pre, c.v_pre, c.k_suf, c.v_suf, c.cu_seqlens,
+                                             theta=cfg.theta, rows=rows)
+    check_attn(out[rows[:, 0], rows[:, 1]], lse[rows[:, 0], rows[:, 1]], ref_o, ref_l, cfg.dtype, name)
+    Wd, Wrows, inv = compact_lm_head(cfg, c.pair_tok)
+    ref = oracle.candidate_readout(c.hidden, Wrows, c.set_offsets, inv, full_vocab=False)
+    lp, ch = run_readout(jev, c.hidden, Wd, c.set_offsets, c.pair_tok)
+    check_readout(lp, ch, ref, cfg.dtype, name)
+
+
+EDGE = [
+    # dtype, Lp, lens, Hq, Hkv, d, splits, pos_offset, head_map
+    (synth.BF16, 300, [1, 7, 0, 33, 130], 8, 2, 128, 0, -1, None),
+    (synth.BF16, 0, [5, 17], 4, 4, 64, 0, -1, None),
+    (synth.BF16, 1000, [200], 14, 2, 128, 3, -1, None),
+    (synth.F32, 129, [3, 1, 2], 6, 3, 64, 0, 500, None),
+    (synth.BF16, 256, [9, 4, 12], 8, 2, 128, 2, -1, [1, 0, 0, 1, 1, 0, 1, 0]),
+    (synth.BF16, 2048, [40] * 12, 28, 4, 128, 1, -1, None),
+    (synth.BF16, 2048, [40] * 12, 28, 4, 128, 5, -1, None),
+    (synth.BF16, 384, [1] * 37, 12, 2, 64, 0, -1, None),
+    (synth.F32, 200, [70, 1, 15], 4, 2, 128, 2, -1, None),
+]
+
+
+@pytest.mark.parametrize("case", EDGE, ids=[f"e{i}" for i in range(len(EDGE))])
+def test_flat_edge_shapes(jev, case):
+    dtype, Lp, lens, Hq, Hkv, d, splits, pos_off, hm = case
+    cfg = synth.FlatConfig("edge", dtype, Lp, len(lens), 1, 1, Hq, Hkv, d, 16, 32, 2, 3, seed=sum(lens) + Lp)
+    c = synth.flat_case(cfg, with_lm_head=False, lengths=np.array(lens, np.int32))
+    out, lse = run_flat(jev, c, num_splits=splits, pos_offset=pos_off, head_map=hm)
+    ref_o, ref_l = oracle.prefix_suffix_attn(c.q, c.k_pre, c.v_pre, c.k_suf, c.v_suf, c.cu_seqlens,
+                                             pos_offset=pos_off, head_map=hm)
+    check_attn(out, lse, ref_o, ref_l, dtype, str(case[:3]))
+
+
+@pytest.mark.parametrize("dtype", [synth.BF16, synth.F32])
+def test_readout_multi_token_invalid_and_empty(jev, dtype):
+    rng = np.random.default_rng(3)
+    R, H, V = 9, 256, 3000
+    hidden = rng.standard_normal((R, H)).astype(np.float32)
+    W = (0.05 * rng.standard_normal((V, H))).astype(np.float32)
+    if dtype == synth.BF16:
+        hidden, W = synth.f32_to_bf16_bits(hidden), synth.f32_to_bf16_bits(W)
+    # 5 sets: multi-token candidates, an empty set, a set with an invalid token, a 40-candidate set
+    so = np.array([0, 3, 3, 5, 6, 46], np.int32)
+    npair = np.array([1, 2, 4, 1, 3, 1] + [1] * 40)
+    co = np.concatenate([[0], np.cumsum(npair)]).astype(np.int32)
+    P = int(co[-1])
+    prow = rng.integers(0, R, P).astype(np.int32)
+    ptok = rng.integers(0, V, P).astype(np.int32)
+    ptok[co[4]] = V + 5  # candidate 4 (set 2) invalid
+    ref = oracle.candidate_readout(hidden, W, so, ptok, cand_offsets=co, pair_row=prow)
+    lp, ch = run_readout(jev, hidden, dev(W), so, ptok, cand_offsets=co, pair_row=prow)
+    check_readout(lp, ch, ref, dtype, "multi")
+    assert ch[1] == -1 and ch[2] == -1 and np.all(np.isnan(lp[3:5]))
+
+
+def test_readout_tie_goes_to_first(jev):
+    hidden = np.ones((2, 8), np.float32)
+    W = np.zeros((4, 8), np.float32)
+    W[1] = W[3] = 0.5
+    lp, ch = run_readout(jev, hidden, dev(W), np.array([0, 2, 4], np.int32), np.array([1, 3, 3, 1], np.int32))
+    assert ch.tolist() == [0, 0]
+    np.testing.assert_allclose(lp, np.log(0.5), atol=1e-6)
+
+
+def _tree_inputs(tc, jev):
+    t = jev.jev_tree_build(tc.seq_off, tc.toks, tc.cfg.Lp)
+    return t, dict(parent=dev(t["parent"]), tok_off=dev(t["tok_off"]), pos0=dev(t["pos0"]))
+
+
+@pytest.mark.parametrize("seed,d", [(0, 64), (1, 128)])
+def test_tree_small_every_element(jev, seed, d):
+    cfg = synth.TreeConfig("t", synth.BF16, 300, 5, 9, 2, 6, 1, 5, 8, 2, d, 64, 500, seed=seed)
+    tc = synth.tree_case(cfg, with_lm_head=True)
+    t, td = _tree_inputs(tc, jev)
+    out, lse = jev.jev_tree_attn(td["parent"], td["tok_off"], td["pos0"], dev(tc.q), dev(tc.k_root), dev(tc.v_root),
+                                 dev(tc.k), dev(tc.v))
+    ref_o, ref_l = oracle.tree_attn(oracle.trie_build(tc.seq_off, tc.toks, cfg.Lp), tc.q, tc.k, tc.v,
+                                    tc.k_root, tc.v_root)
+    check_attn(host_f64(out), host_f64(lse), ref_o, ref_l, cfg.dtype, "tree")
+    plan = jev.jev_tree_readout_plan(tc.seq_off, tc.toks, tc.score_from, t["path_row"])
+    ref = oracle.candidate_readout(tc.hidden, tc.W, tc.set_offsets, plan["pair_tok"],
+                                   cand_offsets=plan["cand_offsets"], pair_row=plan["pair_row"])
+    lp, ch = run_readout(jev, tc.hidden, dev(tc.W), tc.set_offsets, plan["pair_tok"],
+                         cand_offsets=plan["cand_offsets"], pair_row=plan["pair_row"])
+    check_readout(lp, ch, ref, cfg.dtype, "tree readout")
+
+
+def test_tree_config_c4(jev):
+    cfg = synth.CONFIGS["c4"]
+    tc = synth.tree_case(cfg, with_lm_head=False)
+    t, td = _tree_inputs(tc, jev)
+    out, lse = jev.jev_tree_attn(td["parent"], td["tok_off"], td["pos0"], dev(tc.q), dev(tc.k_root), dev(tc.v_root),
+                                 dev(tc.k), dev(tc.v))
+    torch.cuda.synchronize()
+    ref_o, ref_l = oracle.tree_attn(oracle.trie_build(tc.seq_off, tc.toks, cfg.Lp), tc.q, tc.k, tc.v,
+                                    tc.k_root, tc.v_root)
+    check_attn(host_f64(out), host_f64(lse), ref_o, ref_l, cfg.dtype, "c4 tree")
+    plan = jev.jev_tree_readout_plan(tc.seq_off, tc.toks, tc.score_from, t["path_row"])
+    Wd, Wrows, inv = compact_lm_head(cfg, plan["pair_tok"])
+    ref = oracle.candidate_readout(tc.hidden, Wrows, tc.set_offsets, inv, cand_offsets=plan["cand_offsets"],
+                                   pair_row=plan["pair_row"], full_vocab=False)
+    lp, ch = run_readout(jev, tc.hidden, Wd, tc.set_offsets, plan["pair_tok"], cand_offsets=plan["cand_offsets"],
+                         pair_row=plan["pair_row"])
+    check_readout(lp, ch, ref, cfg.dtype, "c4 readout")
