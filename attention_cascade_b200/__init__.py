@@ -151,6 +151,35 @@ def jev_prefix_suffix_attn(q, k_pre, v_pre, k_suf, v_suf, cu_seqlens, *, head_ma
     return out, lse
 
 
+JEV_NOALLOC_SCRATCH_BYTES = 32 << 20
+_lib.jev_prefix_suffix_attn_noalloc.argtypes = [C.POINTER(jev_attn_desc)] + [_vp] * 11
+_lib.jev_prefix_suffix_attn_noalloc.restype = C.c_int
+
+
+def jev_prefix_suffix_attn_noalloc(q, k_pre, v_pre, k_suf, v_suf, cu_seqlens, out, lse=None, *, head_map=None,
+                                   status_flags=None, rope_theta=1e4, softmax_scale=0.0, pos_offset=-1,
+                                   num_splits=0, stream=None):
+    """The attention of jev_prefix_suffix_attn for callers that cannot allocate
+    device memory: the library's static scratch replaces the workspace, and the
+    caller passes preallocated outputs.  Calls that overlap on the GPU race on
+    that one scratch array."""
+    dt = _dtype_code(q)
+    T, Hq, d = q.shape
+    Lp, Hkv = k_pre.shape[0], k_pre.shape[1]
+    for t, n in ((q, "q"), (k_pre, "k_pre"), (v_pre, "v_pre"), (k_suf, "k_suf"), (v_suf, "v_suf"), (out, "out")):
+        _dev(t, n, q.dtype)
+    _dev(cu_seqlens, "cu_seqlens", torch.int32)
+    _dev(head_map, "head_map", torch.int32)
+    _dev(lse, "lse", torch.float32)
+    _dev(status_flags, "status_flags", torch.int32)
+    desc = make_attn_desc(cu_seqlens.numel() - 1, Lp, Hq, Hkv, d, T, dt, rope_theta, softmax_scale, pos_offset,
+                          num_splits)
+    _check(_lib.jev_prefix_suffix_attn_noalloc(C.byref(desc), _p(q), _p(k_pre), _p(v_pre), _p(k_suf), _p(v_suf),
+                                               _p(cu_seqlens), _p(head_map), _p(out), _p(lse), _p(status_flags),
+                                               _stream(stream)), "jev_prefix_suffix_attn_noalloc")
+    return out, lse
+
+
 def jev_candidate_readout(hidden, lm_head, set_offsets, pair_tok, *, cand_offsets=None, pair_row=None,
                           logprob=None, choice=None, score=None, stream=None):
     """Per-option log-probs and argmax over each option set; returns (logprob, choice)."""

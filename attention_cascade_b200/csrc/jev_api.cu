@@ -340,6 +340,80 @@ jev_status jev_prefix_suffix_attn(const jev_attn_desc* d, const void* q, const v
                         head_map, false, out, lse, (cudaStream_t)stream);
 }
 
+}  // extern "C"
+
+// ---------------------------------------------------------------- fixed scratch
+// Scratch of jev_prefix_suffix_attn_noalloc for callers that cannot allocate.
+// Host code must not use this symbol as an address: the device address of
+// each GPU's copy is looked up once per device with cudaGetSymbolAddress.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[JEV_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kMaxDevices] = {};
+
+jev_status noalloc_scratch(void** ptr) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(JEV_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= kMaxDevices) return fail(JEV_ERR_UNSUPPORTED, "device index %d", dev);
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || !p)
+      return fail(JEV_ERR_CUDA, "cudaGetSymbolAddress of the static scratch: %s", cudaGetErrorString(e));
+    g_noalloc_addr[dev] = p;
+  }
+  *ptr = g_noalloc_addr[dev];
+  return JEV_OK;
+}
+}  // namespace
+
+extern "C" {
+
+jev_status jev_prefix_suffix_attn_noalloc(const jev_attn_desc* d, const void* q, const void* k_pre,
+                                          const void* v_pre, const void* k_suf, const void* v_suf,
+                                          const int32_t* cu_seqlens, const int32_t* head_map, void* out,
+                                          float* lse, int32_t* status_flags, jev_stream_t stream) {
+  jev_status st = check_desc(d);
+  if (st) return st;
+  if (d->B == 0 || d->T_total == 0) return JEV_OK;
+  if (!q || !k_suf || !v_suf || !cu_seqlens || !out) return fail(JEV_ERR_INVALID_ARG, "required pointer is NULL");
+  if (d->Lp > 0 && (!k_pre || !v_pre)) return fail(JEV_ERR_INVALID_ARG, "prefix pointers are NULL with Lp > 0");
+  const void* ptrs[] = {q, k_pre, v_pre, k_suf, v_suf, out, lse};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return fail(JEV_ERR_INVALID_ARG, "tensor pointer not 16-byte aligned");
+  if ((uintptr_t)cu_seqlens & 3) return fail(JEV_ERR_INVALID_ARG, "cu_seqlens misaligned");
+  const int T = d->T_total;
+  jev_attn_desc dd = *d;
+  Plan p = plan_of(&dd, T);
+  Layout L = layout_of(&dd, T, p, 0);
+  if (L.total > JEV_NOALLOC_SCRATCH_BYTES && p.S > 1) {
+    dd.num_splits = 1;  // a single split needs no partials
+    p = plan_of(&dd, T);
+    L = layout_of(&dd, T, p, 0);
+  }
+  if (L.total > JEV_NOALLOC_SCRATCH_BYTES)
+    return fail(JEV_ERR_UNSUPPORTED, "problem needs %zu bytes of scratch; the static scratch holds %u bytes",
+                L.total, (unsigned)JEV_NOALLOC_SCRATCH_BYTES);
+  void* scratch = nullptr;
+  st = noalloc_scratch(&scratch);
+  if (st) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaMemsetAsync(scratch, 0, kStatusBytes, s);
+  if (e != cudaSuccess) return fail(JEV_ERR_CUDA, "clearing the status word: %s", cudaGetErrorString(e));
+  st = attention_core(&dd, T, p, L, (char*)scratch, q, k_pre, v_pre, k_suf, v_suf, cu_seqlens, dd.B, nullptr,
+                      head_map, false, out, lse, s);
+  if (st) return st;
+  if (status_flags) {
+    e = cudaMemcpyAsync(status_flags, scratch, sizeof(int32_t), cudaMemcpyDeviceToDevice, s);
+    if (e != cudaSuccess) return fail(JEV_ERR_CUDA, "copying the status word: %s", cudaGetErrorString(e));
+  }
+  return JEV_OK;
+}
+
 jev_status jev_candidate_readout(const jev_readout_desc* d, const void* hidden, const void* lm_head,
                                  const int32_t* set_offsets, const int32_t* cand_offsets, const int32_t* pair_row,
                                  const int32_t* pair_tok, float* logprob, int32_t* choice, float* score,

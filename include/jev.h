@@ -120,6 +120,47 @@ jev_status jev_prefix_suffix_attn(const jev_attn_desc* desc, const void* q, cons
                                   float* lse, void* workspace, size_t ws_bytes, jev_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
+/* Fixed-scratch variant (no allocation)                                     */
+/* ------------------------------------------------------------------------ */
+
+/* Size of the library's static device scratch used by the variant below. */
+#define JEV_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+/*
+ * jev_prefix_suffix_attn_noalloc — the same attention as
+ * jev_prefix_suffix_attn (same arguments and results) for callers that cannot
+ * hand the library a workspace: code whose device memory is owned and
+ * budgeted by a host runtime that exposes no allocator to it (a plugin inside
+ * an inference engine, a pre-planned static memory arena), or code that must
+ * not call cudaMalloc/cudaFree because those synchronise the device or are
+ * not allowed at that point.  The paper has no counterpart; this entry point
+ * exists only for such callers.
+ *
+ * Scratch comes from one file-scope device array of JEV_NOALLOC_SCRATCH_BYTES
+ * bytes that every GPU loading the library holds until the process exits.
+ * The call allocates nothing (no cudaMalloc, no cudaFree, no allocating
+ * library routine).  If the automatic split plan does not fit in the array
+ * the call falls back to a single prefix split; if that does not fit either
+ * it returns JEV_ERR_UNSUPPORTED, naming the bytes needed, before enqueuing
+ * anything.
+ *
+ * The first call on a device looks up the array's device address on that
+ * device (cudaGetSymbolAddress, with the device current) and caches it; make
+ * that first call before any stream capture.  Every call shares the one array
+ * and leaves its contents behind; the call clears the status word at its
+ * start.  Calls whose work overlaps on the GPU (different streams, or
+ * different host threads on one device) race on the array: serialise them.
+ *
+ *   status_flags  optional DEVICE int32: receives the call's status-word bits
+ *                 (JEV_DEV_*) at the end of the call, in stream order; NULL
+ *                 discards them.
+ */
+jev_status jev_prefix_suffix_attn_noalloc(const jev_attn_desc* desc, const void* q, const void* k_pre,
+                                          const void* v_pre, const void* k_suf, const void* v_suf,
+                                          const int32_t* cu_seqlens, const int32_t* head_map, void* out,
+                                          float* lse, int32_t* status_flags, jev_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
 /* Candidate readout                                                         */
 /* ------------------------------------------------------------------------ */
 
