@@ -58,23 +58,44 @@ cudaEvent_t take_event() {
   return e;
 }
 
+// Record a timing event on s; inside a stream capture the record becomes an
+// external event node that every replay of the graph re-records.
+bool record(cudaEvent_t ev, cudaStream_t s) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(s, &cs) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  const unsigned flags = cs == cudaStreamCaptureStatusActive ? cudaEventRecordExternal : cudaEventRecordDefault;
+  if (cudaEventRecordWithFlags(ev, s, flags) != cudaSuccess) {
+    cudaGetLastError();  // timing is best effort; never let it fail a launch
+    return false;
+  }
+  return true;
+}
+
 // Launch one kernel through `fn`, bracketed by timing events when enabled.
 template <class F>
 jev_status run(const char* name, cudaStream_t s, F&& fn) {
   Rec r{-1, nullptr, nullptr};
-  const bool on = g_prof.load();
+  bool on = g_prof.load();
   if (on) {
     std::lock_guard<std::mutex> lk(g_mu);
     r.name = name_id(name);
     r.a = take_event();
     r.b = take_event();
-    cudaEventRecord(r.a, s);
   }
+  if (on) on = record(r.a, s);
   cudaError_t e = fn();
-  if (on) {
-    cudaEventRecord(r.b, s);
+  if (on && e == cudaSuccess) on = record(r.b, s);
+  if (r.a) {
     std::lock_guard<std::mutex> lk(g_mu);
-    g_recs.push_back(r);
+    if (on) {
+      g_recs.push_back(r);
+    } else {
+      g_pool.push_back(r.a);
+      g_pool.push_back(r.b);
+    }
   }
   g_launches++;
   if (e != cudaSuccess) return fail(JEV_ERR_CUDA, "%s launch failed: %s", name, cudaGetErrorString(e));
@@ -116,10 +137,29 @@ Plan plan_of(const jev_attn_desc* d, int T) {
   p.M = T * p.G;
   const int ktiles = (d->Lp + 127) / 128;
   int S = d->num_splits;
-  if (S <= 0) {
-    const int rows_per_cta = use_tc(d) ? 256 : 16;
-    const long ctas = (long)((p.M + rows_per_cta - 1) / rows_per_cta) * d->Hkv;
-    const long target = use_tc(d) ? (long)num_sms() : 4L * num_sms();
+  if (S <= 0 && use_tc(d)) {
+    // Tensor-core kernel: one CTA per SM, 256 stacked rows per CTA.  Pick the
+    // split count with the least estimated time: waves of CTAs times key
+    // tiles per split (+1 for the suffix window), plus the merge's traffic of
+    // fp32 partials when split.
+    const long ctas = (long)((p.M + 255) / 256) * d->Hkv;
+    const double sms = num_sms();
+    const double unit_us = 4.0 * 256 * 128 * d->d / (1.4e15 / sms) * 1e6;
+    const double rows = (double)p.M * d->Hkv;
+    double best = 1e30;
+    S = 1;
+    for (int s = 1; s <= std::min(16, std::max(1, ktiles)); ++s) {
+      const double waves = std::ceil(ctas * s / sms);
+      double t = waves * ((ktiles + s - 1) / s + 1) * unit_us;
+      if (s > 1) t += rows * d->d * 4.0 * (2 * s + 1) / 6.5e12 * 1e6 + 3.0;
+      if (t < best * 0.97) {
+        best = t;
+        S = s;
+      }
+    }
+  } else if (S <= 0) {
+    const long ctas = (long)((p.M + 15) / 16) * d->Hkv;
+    const long target = 4L * num_sms();
     S = ctas > 0 ? (int)((target + ctas - 1) / ctas) : 1;
     // keep at least 4 key tiles per split so partial traffic stays small
     S = std::min(S, std::max(1, ktiles / 4));
@@ -263,9 +303,11 @@ int32_t jev_profile_read(int32_t cap, char* names, int32_t* launches, double* ms
   std::vector<double> tot(g_names.size(), 0.0);
   std::vector<int> cnt(g_names.size(), 0);
   for (const Rec& r : g_recs) {
-    cudaEventSynchronize(r.b);
     float t = 0.f;
-    cudaEventElapsedTime(&t, r.a, r.b);
+    if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&t, r.a, r.b) != cudaSuccess) {
+      cudaGetLastError();  // an event of a graph that was never replayed
+      continue;
+    }
     tot[r.name] += t;
     cnt[r.name] += 1;
     if (!keep) {
