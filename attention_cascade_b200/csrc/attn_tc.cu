@@ -64,7 +64,13 @@ struct Bars {
 struct Shared {
   uint32_t tmem_base;
   int abort;
+  int last;
 };
+
+// barrier over the first `count` threads of the CTA (ids 1..15; 0 is __syncthreads)
+__device__ __forceinline__ void named_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
 
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort, int32_t* status) {
   if (mbar_try_wait(bar, parity)) return true;
@@ -105,6 +111,90 @@ __device__ __forceinline__ void tile_window(const AttnArgs& a, int m0, int lane,
   hi = t1;
 }
 
+// One segment of a CTA's unit range: units [ua, ub) of work tile w.
+struct Segment {
+  int w, ua, ub;
+  int g, m0;
+  int n_pre, n;  // prefix key tiles of the segment, key tiles in total
+  int lo;        // first suffix key of the window (valid when the segment holds the suffix unit)
+  bool complete; // the segment is the whole tile: write the final output
+  int slot;      // partial slot when not complete
+};
+
+// Segments are visited by every role in the same order; each role derives
+// the same description (the window needs one warp-wide reduction).
+__device__ __forceinline__ Segment make_segment(const AttnArgs& a, int c, long long u, long long u_end, int lane) {
+  Segment sg;
+  sg.w = (int)(u / a.P);
+  const long long t0 = (long long)sg.w * a.P;
+  sg.ua = (int)(u - t0);
+  sg.ub = (int)(min(u_end, t0 + a.P) - t0);
+  sg.g = sg.w / a.n_pairs;
+  sg.m0 = (sg.w - sg.g * a.n_pairs) * 2 * kBM;
+  sg.n_pre = max(0, min(sg.ub, a.n_pre) - sg.ua);
+  int n_suf = 0;
+  sg.lo = 0;
+  if (sg.ub == a.P) {
+    int lo, hi;
+    tile_window(a, sg.m0, lane, lo, hi);
+    sg.lo = lo;
+    n_suf = lo <= hi ? (hi - lo + kBN) / kBN : 0;
+  }
+  sg.n = sg.n_pre + n_suf;
+  sg.complete = sg.ua == 0 && sg.ub == a.P;
+  sg.slot = tc_unit_begin(a, c) >= t0 ? 2 * c : 2 * c + 1;
+  return sg;
+}
+
+// Row r of split tile w: combine the normalised partials of every CTA that
+// holds a segment of the tile.  Segment of CTA c: its first segment (slot 2c)
+// when the CTA's range starts inside the tile, else its last (slot 2c + 1).
+template <int D>
+__device__ __forceinline__ void merge_row(const AttnArgs& a, int w, int r, int m, int g, int t, int h) {
+  const long long t0 = (long long)w * a.P;
+  const int c_lo = tc_cta_of(a, t0), c_hi = tc_cta_of(a, t0 + a.P - 1);
+  float mx = -CUDART_INF_F;
+  for (int c = c_lo; c <= c_hi; ++c) {
+    const int slot = tc_unit_begin(a, c) >= t0 ? 2 * c : 2 * c + 1;
+    mx = fmaxf(mx, a.l_part[(size_t)slot * 2 * kBM + r]);
+  }
+  float wsum = 0.f;
+  if (mx != -CUDART_INF_F)
+    for (int c = c_lo; c <= c_hi; ++c) {
+      const int slot = tc_unit_begin(a, c) >= t0 ? 2 * c : 2 * c + 1;
+      wsum += exp2f(a.l_part[(size_t)slot * 2 * kBM + r] - mx);
+    }
+  const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+  __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(a.out) + ((size_t)t * a.Hq + h) * D;
+#pragma unroll 1
+  for (int c0 = 0; c0 < D; c0 += 32) {
+    float acc[32];
+#pragma unroll
+    for (int k = 0; k < 32; ++k) acc[k] = 0.f;
+    if (mx != -CUDART_INF_F)
+      for (int c = c_lo; c <= c_hi; ++c) {
+        const int slot = tc_unit_begin(a, c) >= t0 ? 2 * c : 2 * c + 1;
+        const size_t row = (size_t)slot * 2 * kBM + r;
+        const float wgt = exp2f(a.l_part[row] - mx) * inv;
+        const float4* src = reinterpret_cast<const float4*>(a.o_part + row * D + c0);
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+          const float4 x = src[v];
+          acc[4 * v] += wgt * x.x;
+          acc[4 * v + 1] += wgt * x.y;
+          acc[4 * v + 2] += wgt * x.z;
+          acc[4 * v + 3] += wgt * x.w;
+        }
+      }
+    uint4* dst = reinterpret_cast<uint4*>(o + c0);
+#pragma unroll
+    for (int v = 0; v < 4; ++v)
+      dst[v] = make_uint4(pack_bf16(acc[8 * v], acc[8 * v + 1]), pack_bf16(acc[8 * v + 2], acc[8 * v + 3]),
+                          pack_bf16(acc[8 * v + 4], acc[8 * v + 5]), pack_bf16(acc[8 * v + 6], acc[8 * v + 7]));
+  }
+  if (a.lse) a.lse[(size_t)t * a.Hq + h] = wsum > 0.f ? (mx + log2f(wsum)) * 0.69314718055994531f : -CUDART_INF_F;
+}
+
 template <int D, bool TREE>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kp,
@@ -114,7 +204,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   const uint32_t sbase = smem_u32(smem);
-  Shared* sh = reinterpret_cast<Shared*>(smem + C::kOffBar + 192);
+  Shared* sh = reinterpret_cast<Shared*>(smem + C::kOffBar + 224);
   const uint32_t bar0 = sbase + C::kOffBar;
   Bars B;
   B.q_full = bar0;
@@ -125,16 +215,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   B.p_full = B.s_full + 16;
   B.o_full = B.p_full + 16;
   B.drain = B.o_full + 16;
+  const uint32_t q_empty = B.drain + 8;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.x * 2 * kBM, g = blockIdx.y, split = blockIdx.z;
-  const int p_lo = split * a.split_len;
-  const int p_hi = min(a.Lp, p_lo + a.split_len);
-  const int n_pre = p_hi > p_lo ? (p_hi - p_lo + kBN - 1) / kBN : 0;
-  const bool last = split == a.S - 1;
+  const int cta = blockIdx.x;
+  const long long u_begin = tc_unit_begin(a, cta), u_end = tc_unit_begin(a, cta + 1);
 
   if (threadIdx.x == 0) {
     mbar_init(B.q_full, 1);
+    mbar_init(q_empty, 1);
     for (int s = 0; s < C::kNS; ++s) {
       mbar_init(B.k_full + 8 * s, 1);
       mbar_init(B.v_full + 8 * s, 1);
@@ -159,86 +248,120 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = sh->tmem_base;
   volatile int* abort = &sh->abort;
 
-  int lo, hi;
-  tile_window(a, m0, lane, lo, hi);
-  const int n_suf = (last && lo <= hi) ? (hi - lo + kBN) / kBN : 0;
-  const int n = n_pre + n_suf;
-  auto key_base = [&](int j) { return j < n_pre ? p_lo + j * kBN : lo + (j - n_pre) * kBN; };
-
   if (warp == kProducerWarp) {
-    if (lane == 0) {
-      tma_prefetch_desc(&tm_q);
-      mbar_expect_tx(B.q_full, 2 * C::kQBytes);
-      for (int i = 0; i < 2; ++i)
-        for (int b = 0; b < D / 64; ++b)
-          tma_load_3d(sbase + i * C::kQBytes + b * C::kBlk, &tm_q, b * 64, m0 + i * kBM, g, B.q_full);
-      for (int j = 0; j < n; ++j) {
-        const int st = j % C::kNS, use = j / C::kNS;
-        if (j >= C::kNS && !wait_bar(B.kv_empty + 8 * st, (use - 1) & 1, abort, a.status)) break;
-        const int kb = key_base(j);
-        const CUtensorMap* mk = j < n_pre ? &tm_kp : &tm_ks;
-        const CUtensorMap* mv = j < n_pre ? &tm_vp : &tm_vs;
-        const uint32_t ks = sbase + C::kOffK + st * C::kKVBytes, vs = sbase + C::kOffV + st * C::kKVBytes;
-        mbar_expect_tx(B.k_full + 8 * st, C::kKVBytes);
-        for (int b = 0; b < D / 64; ++b) tma_load_2d(ks + b * C::kBlk, mk, g * D + b * 64, kb, B.k_full + 8 * st);
-        mbar_expect_tx(B.v_full + 8 * st, C::kKVBytes);
-        for (int b = 0; b < D / 64; ++b) tma_load_2d(vs + b * C::kBlk, mv, g * D + b * 64, kb, B.v_full + 8 * st);
+    // ---------------------------------------------------------------- TMA producer
+    long long J = 0;
+    int k = 0;
+    bool ok = true;
+    tma_prefetch_desc(&tm_q);
+    for (long long u = u_begin; ok && u < u_end; ++k) {
+      const Segment sg = make_segment(a, cta, u, u_end, lane);
+      u = (long long)sg.w * a.P + sg.ub;
+      if (lane == 0) {
+        if (k > 0 && !wait_bar(q_empty, (k - 1) & 1, abort, a.status)) ok = false;
+        if (ok) {
+          mbar_expect_tx(B.q_full, 2 * C::kQBytes);
+          for (int i = 0; i < 2; ++i)
+            for (int b = 0; b < D / 64; ++b)
+              tma_load_3d(sbase + i * C::kQBytes + b * C::kBlk, &tm_q, b * 64, sg.m0 + i * kBM, sg.g, B.q_full);
+        }
+        for (int j = 0; ok && j < sg.n; ++j) {
+          const long long JJ = J + j;
+          const int st = (int)(JJ % C::kNS);
+          const long long use = JJ / C::kNS;
+          if (JJ >= C::kNS && !wait_bar(B.kv_empty + 8 * st, (uint32_t)((use - 1) & 1), abort, a.status)) {
+            ok = false;
+            break;
+          }
+          const bool pre = j < sg.n_pre;
+          const int kb = pre ? (sg.ua + j) * kBN : sg.lo + (j - sg.n_pre) * kBN;
+          const CUtensorMap* mk = pre ? &tm_kp : &tm_ks;
+          const CUtensorMap* mv = pre ? &tm_vp : &tm_vs;
+          const uint32_t ks = sbase + C::kOffK + st * C::kKVBytes, vs = sbase + C::kOffV + st * C::kKVBytes;
+          mbar_expect_tx(B.k_full + 8 * st, C::kKVBytes);
+          for (int b = 0; b < D / 64; ++b) tma_load_2d(ks + b * C::kBlk, mk, sg.g * D + b * 64, kb, B.k_full + 8 * st);
+          mbar_expect_tx(B.v_full + 8 * st, C::kKVBytes);
+          for (int b = 0; b < D / 64; ++b) tma_load_2d(vs + b * C::kBlk, mv, sg.g * D + b * 64, kb, B.v_full + 8 * st);
+        }
       }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      J += sg.n;
     }
   } else if (warp == kMmaWarp) {
-    if (lane == 0) {
-      constexpr uint32_t id_qk = idesc_bf16(kBM, kBN, false);
-      constexpr uint32_t id_pv = idesc_bf16(kBM, D, true);
-      auto issue_s = [&](int i, int st) {
-        const uint32_t qa = sbase + i * C::kQBytes, ka = sbase + C::kOffK + st * C::kKVBytes;
+    // ---------------------------------------------------------------- MMA issuer
+    constexpr uint32_t id_qk = idesc_bf16(kBM, kBN, false);
+    constexpr uint32_t id_pv = idesc_bf16(kBM, D, true);
+    auto issue_s = [&](int i, int st) {
+      const uint32_t qa = sbase + i * C::kQBytes, ka = sbase + C::kOffK + st * C::kKVBytes;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::kBlk + (kk & 3) * 32;
-          mma_ss(tmem + i * kBN, smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(ka + off, 16, 1024), id_qk,
-                 kk > 0);
-        }
-        mma_commit(B.s_full + 8 * i);
-      };
-      auto issue_pv = [&](int i, int st, bool acc) {
-        const uint32_t va = sbase + C::kOffV + st * C::kKVBytes;
-#pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk)
-          mma_ts(tmem + C::kOCol + i * D, tmem + i * kBN + kk * 8, smem_desc_sw128(va + kk * 16 * 128, C::kBlk, 1024),
-                 id_pv, (acc || kk > 0) ? 1u : 0u);
-      };
-      bool ok = wait_bar(B.q_full, 0, abort, a.status);
-      if (ok && n > 0) {
-        ok = wait_bar(B.k_full, 0, abort, a.status);
-        fence_after_sync();
-        if (ok) {
-          issue_s(0, 0);
-          issue_s(1, 0);
-        }
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * C::kBlk + (kk & 3) * 32;
+        mma_ss(tmem + i * kBN, smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(ka + off, 16, 1024), id_qk,
+               kk > 0);
       }
-      for (int j = 0; ok && j < n; ++j) {
-        const int st = j % C::kNS, ph = (j / C::kNS) & 1;
-        const int st1 = (j + 1) % C::kNS, ph1 = ((j + 1) / C::kNS) & 1;
-        if (!wait_bar(B.v_full + 8 * st, ph, abort, a.status)) break;
-        if (!wait_bar(B.p_full, j & 1, abort, a.status)) break;
-        fence_after_sync();
-        issue_pv(0, st, j > 0);
-        if (j == n - 1) mma_commit(B.o_full);
-        if (j + 1 < n) {
-          if (!wait_bar(B.k_full + 8 * st1, ph1, abort, a.status)) break;
+      mma_commit(B.s_full + 8 * i);
+    };
+    auto issue_pv = [&](int i, int st, bool acc) {
+      const uint32_t va = sbase + C::kOffV + st * C::kKVBytes;
+#pragma unroll
+      for (int kk = 0; kk < kBN / 16; ++kk)
+        mma_ts(tmem + C::kOCol + i * D, tmem + i * kBN + kk * 8, smem_desc_sw128(va + kk * 16 * 128, C::kBlk, 1024),
+               id_pv, (acc || kk > 0) ? 1u : 0u);
+    };
+    long long J = 0;
+    int k = 0;
+    bool ok = true;
+    for (long long u = u_begin; ok && u < u_end; ++k) {
+      const Segment sg = make_segment(a, cta, u, u_end, lane);
+      u = (long long)sg.w * a.P + sg.ub;
+      if (lane == 0) {
+        const int n = sg.n;
+        ok = wait_bar(B.q_full, k & 1, abort, a.status);
+        if (ok && n > 0) {
+          const int st0 = (int)(J % C::kNS);
+          ok = wait_bar(B.k_full + 8 * st0, (uint32_t)((J / C::kNS) & 1), abort, a.status);
           fence_after_sync();
-          issue_s(0, st1);
+          if (ok) {
+            issue_s(0, st0);
+            issue_s(1, st0);
+            if (n == 1) mma_commit(q_empty);
+          }
         }
-        if (!wait_bar(B.p_full + 8, j & 1, abort, a.status)) break;
-        fence_after_sync();
-        issue_pv(1, st, j > 0);
-        mma_commit(B.kv_empty + 8 * st);
-        if (j == n - 1) mma_commit(B.o_full + 8);
-        if (j + 1 < n) issue_s(1, st1);
+        for (int j = 0; ok && j < n; ++j) {
+          const long long JJ = J + j, JJ1 = JJ + 1;
+          const int st = (int)(JJ % C::kNS), st1 = (int)(JJ1 % C::kNS);
+          const uint32_t ph = (uint32_t)((JJ / C::kNS) & 1), ph1 = (uint32_t)((JJ1 / C::kNS) & 1);
+          const uint32_t pp = (uint32_t)(JJ & 1);
+          if (!wait_bar(B.v_full + 8 * st, ph, abort, a.status)) { ok = false; break; }
+          if (!wait_bar(B.p_full, pp, abort, a.status)) { ok = false; break; }
+          fence_after_sync();
+          issue_pv(0, st, j > 0);
+          if (j == n - 1) mma_commit(B.o_full);
+          if (j + 1 < n) {
+            if (!wait_bar(B.k_full + 8 * st1, ph1, abort, a.status)) { ok = false; break; }
+            fence_after_sync();
+            issue_s(0, st1);
+          }
+          if (!wait_bar(B.p_full + 8, pp, abort, a.status)) { ok = false; break; }
+          fence_after_sync();
+          issue_pv(1, st, j > 0);
+          mma_commit(B.kv_empty + 8 * st);
+          if (j == n - 1) mma_commit(B.o_full + 8);
+          if (j + 1 < n) {
+            issue_s(1, st1);
+            if (j + 2 == n) mma_commit(q_empty);
+          }
+        }
+        if (ok && n == 0) {
+          mma_commit(q_empty);
+          mma_commit(B.o_full);
+          mma_commit(B.o_full + 8);
+        }
       }
-      if (n == 0) {
-        mma_commit(B.o_full);
-        mma_commit(B.o_full + 8);
-      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      J += sg.n;
+    }
+    if (lane == 0) {
       // every MMA of this CTA has completed before TMEM is released
       mma_commit(B.drain);
       wait_bar(B.drain, 0, abort, a.status);
@@ -246,139 +369,178 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ---------------------------------------------------------------- softmax + epilogue
     const int i = warp >> 2, q = warp & 3, r = q * 32 + lane;
-    const int m = m0 + i * kBM + r;
-    const bool valid = m < a.M;
-    int t = -1, start = 0, nanc = 0;
-    int2 anc[TREE ? kMaxDepth : 1];
-    if (valid) {
-      t = m / a.G;
-      const TokInfo inf = a.info[t];
-      start = inf.seg_start;
-      if (TREE) {
-        nanc = a.node_nanc[inf.node];
-        if (nanc < 0) t = -1;
-#pragma unroll
-        for (int k = 0; k < (TREE ? kMaxDepth : 1); ++k)
-          anc[k] = k < nanc ? a.node_anc[(size_t)inf.node * kMaxDepth + k] : make_int2(0, 0);
-      }
-    }
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     const uint32_t s_addr = tmem + i * kBN + lane_off;
     const uint32_t o_addr = tmem + C::kOCol + i * D + lane_off;
     const float sl2 = a.scale_log2;
-    float m_run = -CUDART_INF_F, l_run = 0.f;
+    long long J = 0;
+    int k = 0;
     bool ok = true;
-    for (int j = 0; j < n; ++j) {
-      if (!wait_bar(B.s_full + 8 * i, j & 1, abort, a.status)) {
-        ok = false;
-        break;
-      }
-      fence_after_sync();
-      float x[kBN];
-      {
-        uint32_t u[32];
+    for (long long u = u_begin; ok && u < u_end; ++k) {
+      const Segment sg = make_segment(a, cta, u, u_end, lane);
+      u = (long long)sg.w * a.P + sg.ub;
+      const int m = sg.m0 + i * kBM + r;
+      const bool valid = m < a.M;
+      int t = -1, start = 0, nanc = 0;
+      int2 anc[TREE ? kMaxDepth : 1];
 #pragma unroll
-        for (int c = 0; c < kBN / 32; ++c) {
-          tmem_ld32(s_addr + c * 32, u);
+      for (int kk = 0; kk < (TREE ? kMaxDepth : 1); ++kk) anc[kk] = make_int2(0, 0);
+      if (valid) {
+        t = m / a.G;
+        const TokInfo inf = a.info[t];
+        start = inf.seg_start;
+        if (TREE) {
+          nanc = a.node_nanc[inf.node];
+          if (nanc < 0) t = -1;
 #pragma unroll
-          for (int k = 0; k < 32; ++k) x[c * 32 + k] = __uint_as_float(u[k]) * sl2;
+          for (int kk = 0; kk < (TREE ? kMaxDepth : 1); ++kk)
+            if (kk < nanc) anc[kk] = a.node_anc[(size_t)inf.node * kMaxDepth + kk];
         }
       }
-      const int kb = key_base(j);
-      if (j < n_pre) {
-        const int lim = p_hi - kb;
-        if (lim < kBN) {
-#pragma unroll
-          for (int c = 0; c < kBN; ++c)
-            if (c >= lim) x[c] = -CUDART_INF_F;
+      float m_run = -CUDART_INF_F, l_run = 0.f;
+      for (int j = 0; j < sg.n; ++j) {
+        const long long JJ = J + j;
+        if (!wait_bar(B.s_full + 8 * i, (uint32_t)(JJ & 1), abort, a.status)) {
+          ok = false;
+          break;
         }
-      } else {
-        // suffix window: same branch up to the row's own token (+ ancestor nodes)
-        const int c_lo = start - kb, c_hi = t - kb;
+        fence_after_sync();
+        // the S row lives in xs as raw bits (unscaled scores); P is packed in
+        // place into the first half of each 64-column block
+        uint32_t xs[kBN];
+        tmem_ld128(s_addr, xs);
+        constexpr uint32_t kNegInf = 0xff800000u;
+        if (j < sg.n_pre) {
+          const int lim = a.Lp - (sg.ua + j) * kBN;  // keys past the prefix are padding
+          if (lim < kBN) {
 #pragma unroll
-        for (int c = 0; c < kBN; ++c) {
-          bool vis = c >= c_lo && c <= c_hi;
-          if (TREE) {
-#pragma unroll
-            for (int k = 0; k < (TREE ? kMaxDepth : 1); ++k)
-              if (k < nanc) vis |= (c >= anc[k].x - kb && c < anc[k].y - kb);
-          }
-          if (!vis) x[c] = -CUDART_INF_F;
-        }
-      }
-      float mx = x[0];
-#pragma unroll
-      for (int c = 1; c < kBN; ++c) mx = fmaxf(mx, x[c]);
-      float m_new = m_run;
-      if (mx > m_run + kLazy || (m_run == -CUDART_INF_F && mx > -CUDART_INF_F)) m_new = mx;
-      const float base = m_new == -CUDART_INF_F ? 0.f : m_new;
-      const float alpha = ex2(m_run - base);
-      float rs = 0.f;
-#pragma unroll
-      for (int h = 0; h < kBN / 64; ++h) {
-        uint32_t pk[32];
-#pragma unroll
-        for (int k = 0; k < 32; ++k) {
-          const float p0 = ex2(x[h * 64 + 2 * k] - base), p1 = ex2(x[h * 64 + 2 * k + 1] - base);
-          rs += p0 + p1;
-          pk[k] = pack_bf16(p0, p1);
-        }
-        tmem_st32(s_addr + h * 32, pk);
-      }
-      l_run = l_run * alpha + rs;
-      if (j > 0 && __any_sync(0xffffffffu, m_new != m_run)) {
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t u[32];
-          tmem_ld32(o_addr + c * 32, u);
-#pragma unroll
-          for (int k = 0; k < 32; ++k) u[k] = __float_as_uint(__uint_as_float(u[k]) * alpha);
-          tmem_st32(o_addr + c * 32, u);
-        }
-      }
-      m_run = m_new;
-      tmem_wait_st();
-      fence_before_sync();
-      mbar_arrive(B.p_full + 8 * i);
-    }
-    if (ok) ok = wait_bar(B.o_full + 8 * i, 0, abort, a.status);
-    fence_after_sync();
-    const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-    const bool write = ok && valid && t >= 0;
-    const int tt = valid ? m / a.G : 0;
-    const int h = valid ? min(max(a.hinv[g * a.G + (m - tt * a.G)], 0), a.Hq - 1) : 0;
-#pragma unroll
-    for (int c = 0; c < D / 32; ++c) {
-      uint32_t u[32];
-      tmem_ld32(o_addr + c * 32, u);
-      if (write) {
-        if (a.S == 1) {
-          uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + ((size_t)tt * a.Hq + h) * D + c * 32);
-#pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            uint4 w;
-            w.x = pack_bf16(__uint_as_float(u[8 * v + 0]) * inv, __uint_as_float(u[8 * v + 1]) * inv);
-            w.y = pack_bf16(__uint_as_float(u[8 * v + 2]) * inv, __uint_as_float(u[8 * v + 3]) * inv);
-            w.z = pack_bf16(__uint_as_float(u[8 * v + 4]) * inv, __uint_as_float(u[8 * v + 5]) * inv);
-            w.w = pack_bf16(__uint_as_float(u[8 * v + 6]) * inv, __uint_as_float(u[8 * v + 7]) * inv);
-            dst[v] = w;
+            for (int c = 0; c < kBN; ++c)
+              if (c >= lim) xs[c] = kNegInf;
           }
         } else {
-          float4* dst = reinterpret_cast<float4*>(a.o_part + (((size_t)split * a.Hkv + g) * a.M + m) * D + c * 32);
+          // suffix window: same branch up to the row's own token (+ ancestor nodes)
+          const int kb = sg.lo + (j - sg.n_pre) * kBN;
+          const int c_lo = start - kb, c_hi = t - kb;
 #pragma unroll
-          for (int v = 0; v < 8; ++v)
-            dst[v] = make_float4(__uint_as_float(u[4 * v]) * inv, __uint_as_float(u[4 * v + 1]) * inv,
-                                 __uint_as_float(u[4 * v + 2]) * inv, __uint_as_float(u[4 * v + 3]) * inv);
+          for (int c = 0; c < kBN; ++c) {
+            bool vis = c >= c_lo && c <= c_hi;
+            if (TREE) {
+#pragma unroll
+              for (int kk = 0; kk < (TREE ? kMaxDepth : 1); ++kk)
+                if (kk < nanc) vis |= (c >= anc[kk].x - kb && c < anc[kk].y - kb);
+            }
+            if (!vis) xs[c] = kNegInf;
+          }
+        }
+        // row max of the raw scores: 8 independent chains, then a tree
+        float pm[8];
+#pragma unroll
+        for (int q8 = 0; q8 < 8; ++q8) pm[q8] = __uint_as_float(xs[q8]);
+#pragma unroll
+        for (int c = 8; c < kBN; ++c) pm[c & 7] = fmaxf(pm[c & 7], __uint_as_float(xs[c]));
+        const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                               fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7]))) * sl2;
+        float m_new = m_run;
+        if (mx > m_run + kLazy || (m_run == -CUDART_INF_F && mx > -CUDART_INF_F)) m_new = mx;
+        const float base = m_new == -CUDART_INF_F ? 0.f : m_new;
+        const float alpha = ex2(m_run - base);
+        // p = 2^(s * scale * log2e - max): one FFMA and one ex2 per score
+        float ps[8];
+#pragma unroll
+        for (int q8 = 0; q8 < 8; ++q8) ps[q8] = 0.f;
+#pragma unroll
+        for (int h = 0; h < kBN / 64; ++h) {
+#pragma unroll
+          for (int kk = 0; kk < 32; ++kk) {
+            const float p0 = ex2(fmaf(__uint_as_float(xs[h * 64 + 2 * kk]), sl2, -base));
+            const float p1 = ex2(fmaf(__uint_as_float(xs[h * 64 + 2 * kk + 1]), sl2, -base));
+            ps[kk & 7] += p0 + p1;
+            xs[h * 64 + kk] = pack_bf16(p0, p1);
+          }
+          tmem_st32(s_addr + h * 32, *reinterpret_cast<const uint32_t(*)[32]>(&xs[h * 64]));
+        }
+        const float rs = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+        l_run = l_run * alpha + rs;
+        if (j > 0 && __any_sync(0xffffffffu, m_new != m_run)) {
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t uu[32];
+            tmem_ld32(o_addr + c * 32, uu);
+#pragma unroll
+            for (int kk = 0; kk < 32; ++kk) uu[kk] = __float_as_uint(__uint_as_float(uu[kk]) * alpha);
+            tmem_st32(o_addr + c * 32, uu);
+          }
+        }
+        m_run = m_new;
+        tmem_wait_st();
+        fence_before_sync();
+        mbar_arrive(B.p_full + 8 * i);
+      }
+      if (ok) ok = wait_bar(B.o_full + 8 * i, (uint32_t)(k & 1), abort, a.status);
+      fence_after_sync();
+      const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+      const bool write = ok && valid && t >= 0;
+      const int tt = valid ? m / a.G : 0;
+      const int h = valid ? min(max(a.hinv[sg.g * a.G + (m - tt * a.G)], 0), a.Hq - 1) : 0;
+      const size_t prow = (size_t)sg.slot * 2 * kBM + i * kBM + r;  // partial row of this thread
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t uu[32];
+        tmem_ld32(o_addr + c * 32, uu);
+        if (write) {
+          if (sg.complete) {
+            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + ((size_t)tt * a.Hq + h) * D + c * 32);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              uint4 w4;
+              w4.x = pack_bf16(__uint_as_float(uu[8 * v + 0]) * inv, __uint_as_float(uu[8 * v + 1]) * inv);
+              w4.y = pack_bf16(__uint_as_float(uu[8 * v + 2]) * inv, __uint_as_float(uu[8 * v + 3]) * inv);
+              w4.z = pack_bf16(__uint_as_float(uu[8 * v + 4]) * inv, __uint_as_float(uu[8 * v + 5]) * inv);
+              w4.w = pack_bf16(__uint_as_float(uu[8 * v + 6]) * inv, __uint_as_float(uu[8 * v + 7]) * inv);
+              dst[v] = w4;
+            }
+          } else {
+            float4* dst = reinterpret_cast<float4*>(a.o_part + prow * D + c * 32);
+#pragma unroll
+            for (int v = 0; v < 8; ++v)
+              dst[v] = make_float4(__uint_as_float(uu[4 * v]) * inv, __uint_as_float(uu[4 * v + 1]) * inv,
+                                   __uint_as_float(uu[4 * v + 2]) * inv, __uint_as_float(uu[4 * v + 3]) * inv);
+          }
         }
       }
-    }
-    if (write) {
-      const float lse2 = l_run > 0.f ? m_run + __log2f(l_run) : -CUDART_INF_F;
-      if (a.S == 1) {
-        if (a.lse) a.lse[(size_t)tt * a.Hq + h] = lse2 * 0.69314718055994531f;
-      } else {
-        a.l_part[((size_t)split * a.Hkv + g) * a.M + m] = lse2;
+      if (write) {
+        const float lse2 = l_run > 0.f ? m_run + __log2f(l_run) : -CUDART_INF_F;
+        if (sg.complete) {
+          if (a.lse) a.lse[(size_t)tt * a.Hq + h] = lse2 * 0.69314718055994531f;
+        } else {
+          a.l_part[prow] = lse2;
+        }
+      } else if (!sg.complete && ok) {
+        a.l_part[prow] = -CUDART_INF_F;  // rows outside the problem merge to nothing
       }
+      if (!sg.complete) {
+        // The CTA that finishes a split tile's last segment merges all of its
+        // segments (held by consecutive CTAs) with the exact log-sum-exp rule.
+        // Every softmax thread takes these barriers (the condition is uniform
+        // across them); only the counter and the merge depend on `ok`.
+        __threadfence();
+        named_sync(1, 256);
+        if (threadIdx.x == 0) {
+          bool last = false;
+          if (ok && !*abort) {
+            const int nseg = tc_cta_of(a, (long long)(sg.w + 1) * a.P - 1) - tc_cta_of(a, (long long)sg.w * a.P) + 1;
+            last = atomicAdd(&a.tile_count[sg.w], 1) == nseg - 1;
+          }
+          sh->last = last;
+        }
+        named_sync(1, 256);
+        if (sh->last && ok) {
+          __threadfence();
+          if (valid && t >= 0) merge_row<D>(a, sg.w, r + i * kBM, m, sg.g, tt, h);
+        }
+        named_sync(1, 256);
+      }
+      J += sg.n;
     }
   }
   fence_before_sync();
@@ -450,8 +612,7 @@ cudaError_t launch_dt(const AttnArgs& a, cudaStream_t s) {
     return cudaErrorInvalidValue;
   if (!map_2d(&mks, a.k_rot, (uint64_t)a.Hkv * D, a.T, row) || !map_2d(&mvs, a.v_suf, (uint64_t)a.Hkv * D, a.T, row))
     return cudaErrorInvalidValue;
-  dim3 grid((a.M + 2 * kBM - 1) / (2 * kBM), a.Hkv, a.S);
-  attn_tc_kernel<D, TREE><<<grid, kThreads, Cfg<D>::kSmem, s>>>(mq, mkp, mvp, mks, mvs, a);
+  attn_tc_kernel<D, TREE><<<a.n_ctas, kThreads, Cfg<D>::kSmem, s>>>(mq, mkp, mvp, mks, mvs, a);
   return cudaGetLastError();
 }
 
@@ -473,7 +634,7 @@ bool attn_tc_supported(int d) {
 }
 
 cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t s) {
-  if (a.M == 0) return cudaSuccess;
+  if (a.M == 0 || a.n_ctas == 0) return cudaSuccess;
   const bool tree = a.node_nanc != nullptr;
   if (a.d == 128) return tree ? launch_dt<128, true>(a, s) : launch_dt<128, false>(a, s);
   return tree ? launch_dt<64, true>(a, s) : launch_dt<64, false>(a, s);

@@ -9,6 +9,7 @@
 namespace jev {
 
 constexpr int kStatusBytes = 256;  // status word lives in the first 256 bytes of a workspace
+constexpr int kMaxSplits = 16;    // prefix splits the merge kernel combines
 
 __device__ __forceinline__ float to_f32(float x) { return x; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }

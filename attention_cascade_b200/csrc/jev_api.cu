@@ -126,52 +126,57 @@ bool use_tc(const jev_attn_desc* d) {
   return !forced && d->dtype == JEV_BF16 && attn_tc_supported(d->d);
 }
 
-// Prefix split plan: split_len is a multiple of 128 keys; the number of
-// splits depends only on Lp, the stacked row count and the SM count.
+// Work plan.  Tensor-core kernel: work tiles of 256 stacked rows of one kv
+// group, each with P = ceil(Lp/128) + 1 units (prefix key tiles + the suffix
+// window), spread evenly over n_ctas persistent CTAs (num_splits: 0 -> one CTA
+// per SM, 1 -> one CTA per tile, s -> about s CTAs per tile).  CUDA-core
+// kernel: S prefix splits of split_len keys (a multiple of 128) and a merge.
 struct Plan {
   int S, split_len, M, G;
+  bool tc, split;
+  int n_pairs, n_tiles, n_pre, P, n_ctas;
+  long long U;
 };
 Plan plan_of(const jev_attn_desc* d, int T) {
-  Plan p;
+  Plan p{};
   p.G = d->Hq / d->Hkv;
   p.M = T * p.G;
   const int ktiles = (d->Lp + 127) / 128;
+  p.tc = use_tc(d);
+  if (p.tc) {
+    p.n_pairs = (p.M + 255) / 256;
+    p.n_tiles = p.n_pairs * d->Hkv;
+    p.n_pre = ktiles;
+    p.P = ktiles + 1;
+    p.U = (long long)p.n_tiles * p.P;
+    const int s = d->num_splits;
+    long long n = s == 1 ? p.n_tiles : s > 1 ? (long long)p.n_tiles * s : (long long)num_sms();
+    // a tile spread over many CTAs costs a long merge; keep it within 64 segments
+    n = std::min(n, (long long)p.n_tiles * 64);
+    p.n_ctas = (int)std::max(1LL, std::min(n, p.U));
+    p.split = false;
+    for (int c = 1; c < p.n_ctas && !p.split; ++c)
+      if (((long long)c * p.U / p.n_ctas) % p.P != 0) p.split = true;
+    p.S = 1;
+    p.split_len = std::max(1, ktiles) * 128;
+    return p;
+  }
   int S = d->num_splits;
-  if (S <= 0 && use_tc(d)) {
-    // Tensor-core kernel: one CTA per SM, 256 stacked rows per CTA.  Pick the
-    // split count with the least estimated time: waves of CTAs times key
-    // tiles per split (+1 for the suffix window), plus the merge's traffic of
-    // fp32 partials when split.
-    const long ctas = (long)((p.M + 255) / 256) * d->Hkv;
-    const double sms = num_sms();
-    const double unit_us = 4.0 * 256 * 128 * d->d / (1.4e15 / sms) * 1e6;
-    const double rows = (double)p.M * d->Hkv;
-    double best = 1e30;
-    S = 1;
-    for (int s = 1; s <= std::min(16, std::max(1, ktiles)); ++s) {
-      const double waves = std::ceil(ctas * s / sms);
-      double t = waves * ((ktiles + s - 1) / s + 1) * unit_us;
-      if (s > 1) t += rows * d->d * 4.0 * (2 * s + 1) / 6.5e12 * 1e6 + 3.0;
-      if (t < best * 0.97) {
-        best = t;
-        S = s;
-      }
-    }
-  } else if (S <= 0) {
+  if (S <= 0) {
     const long ctas = (long)((p.M + 15) / 16) * d->Hkv;
     const long target = 4L * num_sms();
     S = ctas > 0 ? (int)((target + ctas - 1) / ctas) : 1;
     // keep at least 4 key tiles per split so partial traffic stays small
     S = std::min(S, std::max(1, ktiles / 4));
   }
-  S = std::max(1, std::min(S, std::max(1, ktiles)));
+  S = std::max(1, std::min(std::min(S, kMaxSplits), std::max(1, ktiles)));
   p.split_len = ktiles > 0 ? ((ktiles + S - 1) / S) * 128 : 128;
   p.S = d->Lp > 0 ? (d->Lp + p.split_len - 1) / p.split_len : 1;
   return p;
 }
 
 struct Layout {
-  size_t hinv, info, qrot, krot, opart, lpart, anc, nanc, total;
+  size_t hinv, info, qrot, krot, opart, lpart, count, anc, nanc, total;
 };
 Layout layout_of(const jev_attn_desc* d, int T, const Plan& p, int n_nodes) {
   Layout L;
@@ -183,7 +188,13 @@ Layout layout_of(const jev_attn_desc* d, int T, const Plan& p, int n_nodes) {
   L.krot = off; off += up256((size_t)T * d->Hkv * d->d * s);
   L.opart = off;
   L.lpart = off;
-  if (p.S > 1) {
+  L.count = off;
+  if (p.tc && p.split) {
+    const size_t rows = (size_t)2 * p.n_ctas * 256;  // two partial segments per CTA at most
+    L.opart = off; off += up256(rows * d->d * 4);
+    L.lpart = off; off += up256(rows * 4);
+    L.count = off; off += up256((size_t)p.n_tiles * 4);
+  } else if (!p.tc && p.S > 1) {
     L.opart = off; off += up256((size_t)p.S * d->Hkv * p.M * d->d * 4);
     L.lpart = off; off += up256((size_t)p.S * d->Hkv * p.M * 4);
   }
@@ -230,6 +241,9 @@ jev_status attention_core(const jev_attn_desc* d, int T, const Plan& p, const La
   r.n_segs = n_segs; r.T = T; r.Hq = d->Hq; r.Hkv = d->Hkv; r.d = d->d;
   r.pos_offset = d->pos_offset >= 0 ? d->pos_offset : d->Lp;
   r.theta = (double)d->rope_theta;
+  r.zero_buf = reinterpret_cast<int32_t*>(ws + L.count);
+  r.zero_n = (p.tc && p.split) ? p.n_tiles : 0;
+  for (int i = 0; i < d->d / 2; ++i) r.inv_freq[i] = std::pow(r.theta, -2.0 * i / d->d);
   jev_status st = run("rope_pack", s, [&] { return launch_rope_pack(r, d->dtype, s); });
   if (st) return st;
 
@@ -246,8 +260,10 @@ jev_status attention_core(const jev_attn_desc* d, int T, const Plan& p, const La
   a.T = T; a.M = p.M; a.Lp = d->Lp; a.Hq = d->Hq; a.Hkv = d->Hkv; a.G = p.G; a.d = d->d;
   a.S = p.S; a.split_len = p.split_len;
   a.scale_log2 = scale_log2_of(d);
-  if (use_tc(d)) st = run("attn_tc", s, [&] { return launch_attn_tc(a, s); });
-  else st = run("attn_simt", s, [&] { return launch_attn_simt(a, d->dtype, s); });
+  a.n_pairs = p.n_pairs; a.n_tiles = p.n_tiles; a.n_pre = p.n_pre; a.P = p.P; a.n_ctas = p.n_ctas; a.U = p.U;
+  a.tile_count = reinterpret_cast<int32_t*>(ws + L.count);
+  if (p.tc) return run("attn_tc", s, [&] { return launch_attn_tc(a, s); });
+  st = run("attn_simt", s, [&] { return launch_attn_simt(a, d->dtype, s); });
   if (st) return st;
   if (p.S > 1) {
     MergeArgs m{};

@@ -23,6 +23,9 @@ struct RopePackArgs {
   const int32_t* head_map; // [Hq] or nullptr
   int n_segs, T, Hq, Hkv, d, pos_offset;
   double theta;
+  double inv_freq[128];    // theta^(-2i/d), i < d/2, formed on the host in double
+  int32_t* zero_buf;       // zeroed before the attention kernel runs (its per-tile counters)
+  int zero_n;
 };
 cudaError_t launch_rope_pack(const RopePackArgs& a, jev_dtype dt, cudaStream_t s);
 
@@ -55,7 +58,17 @@ struct AttnArgs {
   int32_t* status;
   int T, M, Lp, Hq, Hkv, G, d, S, split_len;  // split_len: prefix keys per split (multiple of 128)
   float scale_log2;         // softmax scale * log2(e)
+  // tensor-core schedule: work tile w = (kv group w / n_pairs, 256-row pair w % n_pairs)
+  // has P = n_pre + 1 units (one per 128-key prefix tile, one for the suffix
+  // window); CTA c owns units [c*U/n_ctas, (c+1)*U/n_ctas).
+  int n_pairs, n_tiles, n_pre, P, n_ctas;
+  long long U;
+  int32_t* tile_count;      // [n_tiles] finished segments per split tile (zeroed by rope_pack)
 };
+// units of the tensor-core schedule owned by CTAs before c
+__host__ __device__ inline long long tc_unit_begin(const AttnArgs& a, int c) { return (long long)c * a.U / a.n_ctas; }
+// CTA owning unit u: the largest c with tc_unit_begin(c) <= u
+__host__ __device__ inline int tc_cta_of(const AttnArgs& a, long long u) { return (int)(((u + 1) * a.n_ctas - 1) / a.U); }
 cudaError_t launch_attn_simt(const AttnArgs& a, jev_dtype dt, cudaStream_t s);
 cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t s);  // bf16, d in {64,128}
 bool attn_tc_supported(int d);

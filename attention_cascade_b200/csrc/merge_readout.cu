@@ -15,25 +15,37 @@ namespace {
 template <typename T, int D>
 __global__ void __launch_bounds__(256) merge_kernel(MergeArgs a) {
   constexpr int C = D / 32;
+  constexpr int kMaxS = 16;
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   const int rows = a.Hkv * a.M;
   if (warp >= rows) return;
   const int g = warp / a.M, m = warp - g * a.M;
+  const size_t split_stride = (size_t)a.Hkv * a.M;
+  const size_t r0 = (size_t)g * a.M + m;
+  // pass 1: every split's normaliser (independent loads, all in flight)
+  float lp[kMaxS];
   float mx = -CUDART_INF_F;
-  for (int s = 0; s < a.S; ++s) mx = fmaxf(mx, a.l_part[((size_t)s * a.Hkv + g) * a.M + m]);
+#pragma unroll
+  for (int s = 0; s < kMaxS; ++s) {
+    lp[s] = s < a.S ? a.l_part[s * split_stride + r0] : -CUDART_INF_F;
+    mx = fmaxf(mx, lp[s]);
+  }
   float acc[C];
 #pragma unroll
   for (int c = 0; c < C; ++c) acc[c] = 0.f;
   float wsum = 0.f;
   if (mx != -CUDART_INF_F) {
-    for (int s = 0; s < a.S; ++s) {
-      const size_t r = ((size_t)s * a.Hkv + g) * a.M + m;
-      const float w = exp2f(a.l_part[r] - mx);
-      wsum += w;
-      const float* o = a.o_part + r * D;
+    // pass 2: weighted sum of the partial outputs
 #pragma unroll
-      for (int c = 0; c < C; ++c) acc[c] += w * o[lane + 32 * c];
+    for (int s = 0; s < kMaxS; ++s) {
+      if (s < a.S) {
+        const float w = exp2f(lp[s] - mx);
+        wsum += w;
+        const float* o = a.o_part + (s * split_stride + r0) * D;
+#pragma unroll
+        for (int c = 0; c < C; ++c) acc[c] += w * o[lane + 32 * c];
+      }
     }
   }
   const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
@@ -46,34 +58,56 @@ __global__ void __launch_bounds__(256) merge_kernel(MergeArgs a) {
     a.lse[(size_t)t * a.Hq + h] = wsum > 0.f ? (mx + log2f(wsum)) * 0.69314718055994531f : -CUDART_INF_F;
 }
 
-// dot of two length-H rows with 16-byte loads, fp32 accumulation, warp-wide
+// Dot of two length-H rows with 16-byte loads and fp32 accumulation, warp
+// wide.  Each lane issues up to kU independent loads of both rows before
+// using any of them, so a row costs ceil(H / (kU*32*per16B)) memory latencies.
+constexpr int kU = 16;
+__device__ __forceinline__ float dot8(uint4 a, uint4 b) {
+  const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
+  const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&b);
+  float acc = 0.f;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const float2 fa = __bfloat1622float2(a2[k]), fb = __bfloat1622float2(b2[k]);
+    acc = fmaf(fa.x, fb.x, acc);
+    acc = fmaf(fa.y, fb.y, acc);
+  }
+  return acc;
+}
 __device__ __forceinline__ float row_dot(const __nv_bfloat16* x, const __nv_bfloat16* w, int H, int lane) {
   const uint4* x4 = reinterpret_cast<const uint4*>(x);
   const uint4* w4 = reinterpret_cast<const uint4*>(w);
+  const int n = H >> 3;
   float acc = 0.f;
-  for (int i = lane; i < (H >> 3); i += 32) {
-    uint4 a = __ldg(x4 + i), b = __ldg(w4 + i);
-    const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
-    const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&b);
+  for (int base = 0; base < n; base += 32 * kU) {
+    uint4 xa[kU], wa[kU];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      float2 fa = __bfloat1622float2(a2[k]), fb = __bfloat1622float2(b2[k]);
-      acc = fmaf(fa.x, fb.x, acc);
-      acc = fmaf(fa.y, fb.y, acc);
+    for (int u = 0; u < kU; ++u) {
+      const int i = base + u * 32 + lane;
+      xa[u] = i < n ? __ldg(x4 + i) : make_uint4(0, 0, 0, 0);
+      wa[u] = i < n ? __ldg(w4 + i) : make_uint4(0, 0, 0, 0);
     }
+#pragma unroll
+    for (int u = 0; u < kU; ++u) acc += dot8(xa[u], wa[u]);
   }
   return acc;
 }
 __device__ __forceinline__ float row_dot(const float* x, const float* w, int H, int lane) {
   const float4* x4 = reinterpret_cast<const float4*>(x);
   const float4* w4 = reinterpret_cast<const float4*>(w);
+  const int n = H >> 2;
   float acc = 0.f;
-  for (int i = lane; i < (H >> 2); i += 32) {
-    float4 a = __ldg(x4 + i), b = __ldg(w4 + i);
-    acc = fmaf(a.x, b.x, acc);
-    acc = fmaf(a.y, b.y, acc);
-    acc = fmaf(a.z, b.z, acc);
-    acc = fmaf(a.w, b.w, acc);
+  for (int base = 0; base < n; base += 32 * kU) {
+    float4 xa[kU], wa[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int i = base + u * 32 + lane;
+      xa[u] = i < n ? __ldg(x4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+      wa[u] = i < n ? __ldg(w4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < kU; ++u)
+      acc += xa[u].x * wa[u].x + xa[u].y * wa[u].y + xa[u].z * wa[u].z + xa[u].w * wa[u].w;
   }
   return acc;
 }
@@ -81,19 +115,24 @@ __device__ __forceinline__ float row_dot(const float* x, const float* w, int H, 
 // One block per option set.  Warps take the set's candidates in turn; a
 // candidate's score is the sum over its (row, token) pairs of
 // hidden[row] . lm_head[token], gathered with 16-byte loads (only option rows
-// of the LM head are ever read).  Scores are parked in `logprob`, then warp 0
-// forms the set's log-sum-exp and argmax (lowest index on ties) and rewrites
-// them as log-probabilities.
+// of the LM head are ever read).  Scores go to shared memory (or, for sets
+// larger than it holds, through `logprob`); warp 0 then forms the set's
+// log-sum-exp and argmax (lowest index on ties) and writes log-probabilities.
+constexpr int kReadWarps = 8;
+constexpr int kReadSmem = 1024;
+
 template <typename T>
-__global__ void __launch_bounds__(128) readout_kernel(ReadoutArgs a) {
+__global__ void __launch_bounds__(kReadWarps * 32) readout_kernel(ReadoutArgs a) {
+  __shared__ float s_z[kReadSmem];
   const int s = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ca = a.set_offsets[s], ce = a.set_offsets[s + 1];
   const T* hid = reinterpret_cast<const T*>(a.hidden);
   const T* W = reinterpret_cast<const T*>(a.lm_head);
   const bool set_ok = ca >= 0 && ce >= ca && ce <= a.n_cands;
+  const bool in_smem = set_ok && ce - ca <= kReadSmem;
   if (set_ok) {
-    for (int c = ca + warp; c < ce; c += 4) {
+    for (int c = ca + warp; c < ce; c += kReadWarps) {
       int pa = c, pe = c + 1;
       if (a.cand_offsets) {
         pa = a.cand_offsets[c];
@@ -115,7 +154,8 @@ __global__ void __launch_bounds__(128) readout_kernel(ReadoutArgs a) {
       z = warp_sum(z);
       if (lane == 0) {
         const float zz = bad ? CUDART_NAN_F : z;
-        a.logprob[c] = zz;
+        if (in_smem) s_z[c - ca] = zz;
+        else a.logprob[c] = zz;
         if (a.score) a.score[c] = zz;
       }
     }
@@ -126,11 +166,12 @@ __global__ void __launch_bounds__(128) readout_kernel(ReadoutArgs a) {
     if (lane == 0) a.choice[s] = -1;
     return;
   }
+  auto zc = [&](int c) { return in_smem ? s_z[c - ca] : a.logprob[c]; };
   float mx = -CUDART_INF_F;
   int best = -1;
   bool any_nan = false;
   for (int c = ca + lane; c < ce; c += 32) {
-    const float z = a.logprob[c];
+    const float z = zc(c);
     if (isnan(z)) any_nan = true;
     else if (best < 0 || z > mx) { mx = z; best = c; }
   }
@@ -143,11 +184,11 @@ __global__ void __launch_bounds__(128) readout_kernel(ReadoutArgs a) {
     if (ob >= 0 && (best < 0 || om > mx || (om == mx && ob < best))) { mx = om; best = ob; }
   }
   float sum = 0.f;
-  for (int c = ca + lane; c < ce; c += 32) sum += exp2f((a.logprob[c] - mx) * 1.4426950408889634f);
+  for (int c = ca + lane; c < ce; c += 32) sum += exp2f((zc(c) - mx) * 1.4426950408889634f);
   sum = warp_sum(sum);
   const float lse = mx + log2f(sum) * 0.69314718055994531f;
   __syncwarp();
-  for (int c = ca + lane; c < ce; c += 32) a.logprob[c] = any_nan ? CUDART_NAN_F : a.logprob[c] - lse;
+  for (int c = ca + lane; c < ce; c += 32) a.logprob[c] = any_nan ? CUDART_NAN_F : zc(c) - lse;
   if (lane == 0) a.choice[s] = any_nan ? -1 : best - ca;
 }
 
@@ -169,8 +210,8 @@ cudaError_t launch_merge(const MergeArgs& a, jev_dtype dt, cudaStream_t s) {
 
 cudaError_t launch_readout(const ReadoutArgs& a, jev_dtype dt, cudaStream_t s) {
   if (a.n_sets == 0) return cudaSuccess;
-  if (dt == JEV_BF16) readout_kernel<__nv_bfloat16><<<a.n_sets, 128, 0, s>>>(a);
-  else readout_kernel<float><<<a.n_sets, 128, 0, s>>>(a);
+  if (dt == JEV_BF16) readout_kernel<__nv_bfloat16><<<a.n_sets, kReadWarps * 32, 0, s>>>(a);
+  else readout_kernel<float><<<a.n_sets, kReadWarps * 32, 0, s>>>(a);
   return cudaGetLastError();
 }
 

@@ -11,85 +11,138 @@
 namespace jev {
 namespace {
 
+// 8 consecutive elements of T as fp32 (one 16-byte load for bf16, two for fp32).
+__device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&f)[8]) {
+  const uint4 v = *reinterpret_cast<const uint4*>(p);
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const float2 x = __bfloat1622float2(h[k]);
+    f[2 * k] = x.x;
+    f[2 * k + 1] = x.y;
+  }
+}
+__device__ __forceinline__ void load8(const float* p, float (&f)[8]) {
+  const float4 a = reinterpret_cast<const float4*>(p)[0], b = reinterpret_cast<const float4*>(p)[1];
+  f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w; f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+}
+__device__ __forceinline__ void store8(__nv_bfloat16* p, const float (&f)[8]) {
+  uint4 v;
+  uint32_t* w = reinterpret_cast<uint32_t*>(&v);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(f[2 * k], f[2 * k + 1]);
+    w[k] = *reinterpret_cast<uint32_t*>(&h);
+  }
+  *reinterpret_cast<uint4*>(p) = v;
+}
+__device__ __forceinline__ void store8(float* p, const float (&f)[8]) {
+  reinterpret_cast<float4*>(p)[0] = make_float4(f[0], f[1], f[2], f[3]);
+  reinterpret_cast<float4*>(p)[1] = make_float4(f[4], f[5], f[6], f[7]);
+}
+
+constexpr int kTokPerBlock = 8;  // one warp per token
+constexpr int kSmemOffs = 4096;  // segment offsets searched in shared memory up to this many
+
+// One warp per packed token: find its segment and position, form cos/sin of
+// its angles (double angle, rounded once to float), then rotate all its query
+// and key heads, 8 pair indices per lane per head with 16-byte accesses.
 template <typename T>
 __global__ void __launch_bounds__(256) rope_pack_kernel(RopePackArgs a) {
-  const int t = blockIdx.x;
   const int half = a.d >> 1;
   const int G = a.Hq / a.Hkv;
-  __shared__ float cs[128], sn[128];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __shared__ float cs[kTokPerBlock][128], sn[kTokPerBlock][128];
   __shared__ int s_slot[256], s_grp[256];
-  __shared__ int s_start, s_pos, s_seg;
-
-  if (threadIdx.x == 0) {
-    int seg = upper_segment(a.offs, a.n_segs, t);
-    int start = a.offs[seg];
-    if (start > t) start = t;
-    if (start < 0) start = 0;
-    int base = a.pos0 ? a.pos0[seg] : a.pos_offset;
-    s_seg = seg;
-    s_start = start;
-    s_pos = base + (t - start);
-  }
+  __shared__ int s_offs[kSmemOffs];
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < a.zero_n; i += gridDim.x * blockDim.x) a.zero_buf[i] = 0;
+  const bool offs_in_smem = a.n_segs + 1 <= kSmemOffs;
+  if (offs_in_smem)
+    for (int i = threadIdx.x; i <= a.n_segs; i += blockDim.x) s_offs[i] = a.offs[i];
   // group and slot of every query head
   for (int h = threadIdx.x; h < a.Hq; h += blockDim.x) {
     int g = a.head_map ? a.head_map[h] : h / G;
     if (g < 0 || g >= a.Hkv) {
-      if (t == 0) raise_flag(a.status, JEV_DEV_BAD_HEAD_MAP);
+      if (blockIdx.x == 0) raise_flag(a.status, JEV_DEV_BAD_HEAD_MAP);
       g = 0;
     }
     s_grp[h] = g;
   }
   // block 0 owns the inverse table: identity first, so every entry stays a
   // valid head index even when a malformed map leaves a slot unclaimed
-  if (t == 0)
+  if (blockIdx.x == 0)
     for (int h = threadIdx.x; h < a.Hq; h += blockDim.x) a.hinv[h] = h;
   __syncthreads();
   for (int h = threadIdx.x; h < a.Hq; h += blockDim.x) {
     int g = s_grp[h], slot = 0;
     for (int h2 = 0; h2 < h; ++h2) slot += (s_grp[h2] == g);
     if (slot >= G) {
-      if (t == 0) raise_flag(a.status, JEV_DEV_BAD_HEAD_MAP);
+      if (blockIdx.x == 0) raise_flag(a.status, JEV_DEV_BAD_HEAD_MAP);
       slot = G - 1;
     }
     s_slot[h] = slot;
-    if (t == 0) a.hinv[g * G + slot] = h;
+    if (blockIdx.x == 0) a.hinv[g * G + slot] = h;
   }
-  if (t == 0) {
+  if (blockIdx.x == 0) {
     // offsets must start at 0, never decrease and end at T
     for (int i = threadIdx.x; i < a.n_segs; i += blockDim.x)
       if (a.offs[i + 1] < a.offs[i]) raise_flag(a.status, JEV_DEV_BAD_SEQLENS);
     if (threadIdx.x == 0 && (a.offs[0] != 0 || a.offs[a.n_segs] != a.T)) raise_flag(a.status, JEV_DEV_BAD_SEQLENS);
   }
-  for (int i = threadIdx.x; i < half; i += blockDim.x) {
-    double inv_freq = pow(a.theta, -2.0 * (double)i / (double)a.d);
-    double ang = (double)s_pos * inv_freq;
-    double sv, cv;
-    sincos(ang, &sv, &cv);
-    cs[i] = (float)cv;
-    sn[i] = (float)sv;
-  }
   __syncthreads();
-  const T* q = reinterpret_cast<const T*>(a.q) + (size_t)t * a.Hq * a.d;
-  T* qr = reinterpret_cast<T*>(a.q_rot);
+  const int t = blockIdx.x * kTokPerBlock + warp;
+  if (t >= a.T) return;
+  int seg = 0, start = 0, pos = 0;
+  if (lane == 0) {
+    seg = upper_segment(offs_in_smem ? s_offs : a.offs, a.n_segs, t);
+    start = offs_in_smem ? s_offs[seg] : a.offs[seg];
+    if (start > t) start = t;
+    if (start < 0) start = 0;
+    pos = (a.pos0 ? a.pos0[seg] : a.pos_offset) + (t - start);
+    a.info[t] = TokInfo{start, pos, seg, 0};
+  }
+  pos = __shfl_sync(0xffffffffu, pos, 0);
+  for (int i = lane; i < half; i += 32) {
+    double sv, cv;
+    sincos((double)pos * a.inv_freq[i], &sv, &cv);
+    cs[warp][i] = (float)cv;
+    sn[warp][i] = (float)sv;
+  }
+  __syncwarp();
+  const int lanes_per_head = half / 8;          // 8 (d = 128) or 4 (d = 64)
+  const int heads_per_it = 32 / lanes_per_head;  // 4 or 8
+  const int i0 = (lane % lanes_per_head) * 8, hsub = lane / lanes_per_head;
+  float c8[8], s8[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    c8[k] = cs[warp][i0 + k];
+    s8[k] = sn[warp][i0 + k];
+  }
   const size_t M = (size_t)a.T * G;
-  for (int e = threadIdx.x; e < a.Hq * half; e += blockDim.x) {
-    int h = e / half, i = e - h * half;
-    float x0 = to_f32(q[h * a.d + i]), x1 = to_f32(q[h * a.d + i + half]);
-    float c = cs[i], s = sn[i];
-    T* dst = qr + ((size_t)s_grp[h] * M + (size_t)t * G + s_slot[h]) * a.d;
-    dst[i] = from_f32<T>(x0 * c - x1 * s);
-    dst[i + half] = from_f32<T>(x1 * c + x0 * s);
+  const int H = a.Hq + a.Hkv;
+#pragma unroll 2
+  for (int hh = hsub; hh < H; hh += heads_per_it) {
+    const T* src;
+    T* dst;
+    if (hh < a.Hq) {
+      src = reinterpret_cast<const T*>(a.q) + ((size_t)t * a.Hq + hh) * a.d;
+      dst = reinterpret_cast<T*>(a.q_rot) + ((size_t)s_grp[hh] * M + (size_t)t * G + s_slot[hh]) * a.d;
+    } else {
+      const int g = hh - a.Hq;
+      src = reinterpret_cast<const T*>(a.k) + ((size_t)t * a.Hkv + g) * a.d;
+      dst = reinterpret_cast<T*>(a.k_rot) + ((size_t)t * a.Hkv + g) * a.d;
+    }
+    float x0[8], x1[8], y0[8], y1[8];
+    load8(src + i0, x0);
+    load8(src + i0 + half, x1);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      y0[k] = x0[k] * c8[k] - x1[k] * s8[k];
+      y1[k] = x1[k] * c8[k] + x0[k] * s8[k];
+    }
+    store8(dst + i0, y0);
+    store8(dst + i0 + half, y1);
   }
-  const T* k = reinterpret_cast<const T*>(a.k) + (size_t)t * a.Hkv * a.d;
-  T* kr = reinterpret_cast<T*>(a.k_rot) + (size_t)t * a.Hkv * a.d;
-  for (int e = threadIdx.x; e < a.Hkv * half; e += blockDim.x) {
-    int g = e / half, i = e - g * half;
-    float x0 = to_f32(k[g * a.d + i]), x1 = to_f32(k[g * a.d + i + half]);
-    float c = cs[i], s = sn[i];
-    kr[g * a.d + i] = from_f32<T>(x0 * c - x1 * s);
-    kr[g * a.d + i + half] = from_f32<T>(x1 * c + x0 * s);
-  }
-  if (threadIdx.x == 0) a.info[t] = TokInfo{s_start, s_pos, s_seg, 0};
 }
 
 // One thread per node: walk up to the root (parents must precede children, at
@@ -151,8 +204,9 @@ __global__ void rope_inplace_kernel(T* x, int L, int H, int d, int pos0, double 
 
 cudaError_t launch_rope_pack(const RopePackArgs& a, jev_dtype dt, cudaStream_t s) {
   if (a.T == 0) return cudaSuccess;
-  if (dt == JEV_BF16) rope_pack_kernel<__nv_bfloat16><<<a.T, 256, 0, s>>>(a);
-  else rope_pack_kernel<float><<<a.T, 256, 0, s>>>(a);
+  const int blocks = (a.T + kTokPerBlock - 1) / kTokPerBlock;
+  if (dt == JEV_BF16) rope_pack_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(a);
+  else rope_pack_kernel<float><<<blocks, 256, 0, s>>>(a);
   return cudaGetLastError();
 }
 

@@ -308,59 +308,76 @@ def jev_arm(args, wl_name):
     lp = torch.empty(c.pair_tok.size, dtype=torch.float32, device=dev)
     choice = torch.empty(cfg.B, dtype=torch.int32, device=dev)
     stream = torch.cuda.Stream(device=dev)
+    side = torch.cuda.Stream(device=dev)
 
     def step(cp, s):
+        # the readout's inputs (final hidden rows, option ids) do not depend on
+        # this attention layer, so it runs on a second stream, forked and
+        # joined inside the step
+        side.wait_stream(s)
+        jev.jev_candidate_readout(cp["hidden"], W, so, cp["pair_tok"], logprob=lp, choice=choice, stream=side)
         jev.jev_prefix_suffix_attn(cp["q"], cp["k_pre"], cp["v_pre"], cp["k_suf"], cp["v_suf"], cu, out=out, lse=lse,
                                    workspace=ws, rope_theta=cfg.theta, stream=s)
-        jev.jev_candidate_readout(cp["hidden"], W, so, cp["pair_tok"], logprob=lp, choice=choice, stream=s)
+        s.wait_stream(side)
 
-    # ---- graphs: one per input copy (at most one per timed step).  Kernel
-    # timing is on while they are captured, so every kernel launch in them is
-    # bracketed by CUDA event nodes on the launching stream.
+    # ---- graphs: one per input copy (at most one per timed step)
     with torch.cuda.stream(stream):
         for i in range(3):
             step(copies[i % ncopies], stream)
     stream.synchronize()
     ngraph = max(1, min(ncopies, args.steps))
-    jev.jev_profile_read()
-    jev.jev_profile_enable(True)
-    n0 = jev.jev_launch_count()
-    graphs = []
-    for cp in copies[:ngraph]:
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            step(cp, torch.cuda.current_stream())
-        graphs.append(g)
-    launches_per_step = (jev.jev_launch_count() - n0) // ngraph
-    jev.jev_profile_enable(False)
+
+    def capture(profiled: bool):
+        jev.jev_profile_enable(profiled)
+        n0 = jev.jev_launch_count()
+        gs = []
+        for cp in copies[:ngraph]:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                step(cp, torch.cuda.current_stream())
+            gs.append(g)
+        jev.jev_profile_enable(False)
+        return gs, (jev.jev_launch_count() - n0) // ngraph
+
+    graphs, launches_per_step = capture(False)
+
+    def timed_loop(gs):
+        with torch.cuda.stream(stream):
+            for i in range(args.warmup):
+                gs[i % ngraph].replay()
+        stream.synchronize()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            a0.record(stream)
+            for i in range(args.steps):
+                gs[i % ngraph].replay()
+            a1.record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        return a0.elapsed_time(a1)
 
     clocks = ClockSampler(local)
     clocks.start()
-    with torch.cuda.stream(stream):
-        for i in range(args.warmup):
-            graphs[i % ngraph].replay()
-    stream.synchronize()
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        e0.record(stream)
-        for i in range(args.steps):
-            graphs[i % ngraph].replay()
-        e1.record(stream)
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    ms = e0.elapsed_time(e1)
+    ms = timed_loop(graphs)
     clk = clocks.stop()
     if world > 1:
         t = torch.tensor([ms], device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms = float(t.item())
     assert jev.jev_check_device_status(ws, stream) == 0, "device status flags set during the bench"
-    # per-kernel durations: each graph's event nodes hold its last replay in the timed region
+
+    # ---- per-kernel durations: the same K steps replayed from graphs whose
+    # kernels are bracketed by CUDA event nodes on the launching stream; each
+    # graph's events hold its last replay, one sample per input copy
+    jev.jev_profile_read()
+    pgraphs, _ = capture(True)
+    prof_ms = timed_loop(pgraphs)
     prof = jev.jev_profile_read()
+    del pgraphs
 
     # ---- end to end through the public API: pinned host inputs in, results out, every step
     hq = {k: base[k].cpu().pin_memory() for k in ("q", "k_suf", "v_suf", "hidden", "pair_tok")}
@@ -379,9 +396,11 @@ def jev_arm(args, wl_name):
             d_in[k].copy_(hq[k], non_blocking=True)
         d_cu.copy_(h_cu, non_blocking=True)
         d_so.copy_(h_so, non_blocking=True)
+        side.wait_stream(s)
+        jev.jev_candidate_readout(d_in["hidden"], W, d_so, d_in["pair_tok"], logprob=lp, choice=choice, stream=side)
         jev.jev_prefix_suffix_attn(d_in["q"], k_pre, v_pre, d_in["k_suf"], d_in["v_suf"], d_cu, out=out, lse=lse,
                                    workspace=ws, rope_theta=cfg.theta, stream=s)
-        jev.jev_candidate_readout(d_in["hidden"], W, d_so, d_in["pair_tok"], logprob=lp, choice=choice, stream=s)
+        s.wait_stream(side)
         h_lp.copy_(lp, non_blocking=True)
         h_ch.copy_(choice, non_blocking=True)
 
@@ -426,7 +445,8 @@ def jev_arm(args, wl_name):
                    "suffix_tokens_per_replica": T, "parallelism": f"replicas{world}" if world > 1 else "single",
                    "l2": f"inputs rotate over {ncopies} device copies ({ncopies * per_copy / 2**20:.0f} MiB > 2x L2)",
                    "timing": "CUDA graph replay per step, CUDA events on the launching stream; per-kernel times "
-                             "from event nodes around each kernel in the replayed graphs"},
+                             "from a second replay of the K steps with event nodes around each kernel",
+                   "streams": "readout on a second stream, forked and joined inside each step"},
         "branches_per_s": world * cfg.B * args.steps / (ms / 1e3),
         "clocks": clk,
         "e2e": {"value": world * T * args.steps / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
@@ -442,6 +462,7 @@ def jev_arm(args, wl_name):
         "step_roofline": {"ideal_us": ideal * 1e6, "measured_us": step_s * 1e6, "frac": ideal / step_s,
                           "definition": "max(F / bf16 burst peak, U / HBM peak) over the whole step"},
         "kernels": per_kernel,
+        "profiled_pass_ms_per_step": prof_ms / args.steps,
     }
     if rank == 0 and world == 1 and os.environ.get("JEV_SKIP_CPU_BASELINE") != "1":
         del graphs
