@@ -277,6 +277,18 @@ def jev_rope_inplace(x: torch.Tensor, pos0: int, theta: float = 1e4, stream=None
     return x
 
 
+_lib.jev_selftest_exp2.argtypes = [_vp, _vp, _i32, _vp]
+_lib.jev_selftest_exp2.restype = C.c_int
+
+
+def jev_selftest_exp2(x: torch.Tensor, stream=None) -> torch.Tensor:
+    """2^x through the attention kernel's FMA-pipe exponential (float32 CUDA tensor)."""
+    _dev(x, "x", torch.float32)
+    y = torch.empty_like(x)
+    _check(_lib.jev_selftest_exp2(_p(x), _p(y), x.numel(), _stream(stream)), "jev_selftest_exp2")
+    return y
+
+
 def jev_workspace_init(workspace: torch.Tensor, stream=None):
     _check(_lib.jev_workspace_init(_p(workspace), workspace.numel(), _stream(stream)), "jev_workspace_init")
 

@@ -4,25 +4,33 @@
 // "FastJEV ...", §3.2-§3.3), so all branches' queries of one kv group are
 // stacked into one M dimension (row m = token m / G, query slot m % G) and the
 // prefix K/V of that group streams through shared memory once per 256 stacked
-// rows instead of once per branch.  After its prefix split, the CTA holding the
-// last split also runs the suffix window: the packed suffix keys its rows may
-// see (same branch up to the row's own token; for tree tokens every ancestor
-// node's keys too), masked per row.  With one split the CTA normalises and
-// writes the final output; with several it writes a normalised partial and
-// its log2 normaliser for the merge kernel.
+// rows instead of once per branch.  After the prefix, a work tile also runs
+// its suffix window: the packed suffix keys its rows may see (same branch up
+// to the row's own token; for tree tokens every ancestor node's keys too),
+// masked per row.
 //
-// CTA = 10 warps:
-//   warps 0-3  softmax + epilogue of Q tile 0 (TMEM lanes 0-127)
-//   warps 4-7  softmax + epilogue of Q tile 1
-//   warp 8     TMA producer (Q once, then K/V tiles through a ring of stages)
-//   warp 9     TMEM allocator and tcgen05.mma issuer (one thread)
+// Schedule.  A work tile (256 stacked rows of one kv group) has P = n_pre + 1
+// units: its 128-key prefix tiles and the suffix window.  The units of all
+// tiles are spread evenly over n_ctas persistent CTAs; a CTA visits its units
+// as segments (runs inside one tile).  A segment that covers its whole tile
+// writes the final output; other segments write a normalised fp32 partial and
+// its log2 normaliser, and tc_fixup_kernel merges the segments of each split
+// tile.
+//
+// CTA = 18 warps:
+//   warps 0-7   Q tile 0: warps 0-3 columns 0-63, warps 4-7 columns 64-127 of
+//               the S/P rows (TMEM lanes 0-127), and the matching halves of O
+//   warps 8-15  Q tile 1, same split
+//   warp 16     TMA producer (Q once per segment, then K/V through a ring of stages)
+//   warp 17     TMEM allocator and tcgen05.mma issuer (one thread)
 // TMEM (512 columns): S0/P0 [0,128), S1/P1 [128,256), O0 at 256, O1 at 256+D.
 // Per key tile j the MMA thread issues S_i = Q_i K_j^T (SS form), and after
-// softmax i has written P_i (bf16, aliasing S_i) it issues O_i += P_i V_j with
-// P_i read straight from TMEM (TS form); tile 0's softmax overlaps tile 1's
-// MMAs and the other way round.  The online softmax runs in the log2 domain
-// with a lazy running max: the max is only raised when a row's new maximum
-// exceeds it by more than 8, so O is rescaled rarely and P stays <= 2^8.
+// both halves of tile i have written P_i (bf16, aliasing S_i) it issues
+// O_i += P_i V_j with P_i read from TMEM (TS form); tile 0's softmax overlaps
+// tile 1's MMAs and the other way round.  The two halves of a row exchange
+// their maxima through shared memory each key tile; the softmax runs in the
+// log2 domain with a lazy running max (raised only when a row's maximum
+// exceeds it by more than 8, so O is rescaled rarely and P stays <= 2^8).
 // Every mbarrier wait is bounded; a wait that runs out raises
 // JEV_DEV_WAIT_TIMEOUT in the status word and the CTA winds down.
 #include <cuda.h>
@@ -38,11 +46,19 @@ using namespace tc;
 
 constexpr int kBM = 128;  // rows per Q tile (TMEM lanes)
 constexpr int kBN = 128;  // keys per K/V tile
-constexpr int kThreads = 320;
-constexpr int kProducerWarp = 8;
-constexpr int kMmaWarp = 9;
+constexpr int kSoftWarps = 16;
+constexpr int kThreads = (kSoftWarps + 2) * 32;
+constexpr int kProducerWarp = kSoftWarps;
+constexpr int kMmaWarp = kSoftWarps + 1;
 constexpr long long kWaitCycles = 1LL << 31;
 constexpr float kLazy = 8.0f;  // log2 headroom before the running max moves
+// Share of softmax exponentials computed on the FMA pipe (every kPolyEvery-th
+// score pair; 0 = none).  Measured on B200 at the wide workload: 0 is fastest
+// (the softmax is issue-bound, not MUFU-bound), so it is off by default.
+#ifndef JEV_POLY_EVERY
+#define JEV_POLY_EVERY 0
+#endif
+constexpr int kPolyEvery = JEV_POLY_EVERY;
 
 template <int D>
 struct Cfg {
@@ -53,21 +69,21 @@ struct Cfg {
   static constexpr int kOffK = 2 * kQBytes;
   static constexpr int kOffV = kOffK + kNS * kKVBytes;
   static constexpr int kOffBar = kOffV + kNS * kKVBytes;
-  static constexpr int kSmem = kOffBar + 256 + 1024;  // barriers + 1024-byte alignment slack
-  static constexpr int kOCol = 256;                   // first TMEM column of O0
+  static constexpr int kOffX = kOffBar + 256;                     // row-max exchange [tile][parity][half][row]
+  static constexpr int kOffL = kOffX + 2 * 2 * 2 * kBM * 4;       // row-sum exchange [tile][half][row]
+  static constexpr int kSmem = kOffL + 2 * 2 * kBM * 4 + 1024;    // + 1024-byte alignment slack
+  static constexpr int kOCol = 256;                               // first TMEM column of O0
 };
 
 struct Bars {
-  uint32_t q_full, k_full, v_full, kv_empty, s_full, p_full, o_full, drain;  // smem addresses (arrays: +8*i)
+  uint32_t q_full, q_empty, k_full, v_full, kv_empty, s_full, p_full, o_full, drain;  // arrays: +8*i
 };
 
 struct Shared {
   uint32_t tmem_base;
   int abort;
-  int last;
 };
 
-// barrier over the first `count` threads of the CTA (ids 1..15; 0 is __syncthreads)
 __device__ __forceinline__ void named_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
@@ -115,14 +131,14 @@ __device__ __forceinline__ void tile_window(const AttnArgs& a, int m0, int lane,
 struct Segment {
   int w, ua, ub;
   int g, m0;
-  int n_pre, n;  // prefix key tiles of the segment, key tiles in total
-  int lo;        // first suffix key of the window (valid when the segment holds the suffix unit)
-  bool complete; // the segment is the whole tile: write the final output
-  int slot;      // partial slot when not complete
+  int n_pre, n;   // prefix key tiles of the segment, key tiles in total
+  int lo;         // first suffix key of the window (when the segment holds the suffix unit)
+  bool complete;  // the segment is the whole tile: write the final output
+  int slot;       // partial slot when not complete
 };
 
-// Segments are visited by every role in the same order; each role derives
-// the same description (the window needs one warp-wide reduction).
+// Every role visits the same segments in the same order and derives the same
+// description (the window takes one warp-wide reduction).
 __device__ __forceinline__ Segment make_segment(const AttnArgs& a, int c, long long u, long long u_end, int lane) {
   Segment sg;
   sg.w = (int)(u / a.P);
@@ -146,55 +162,6 @@ __device__ __forceinline__ Segment make_segment(const AttnArgs& a, int c, long l
   return sg;
 }
 
-// Row r of split tile w: combine the normalised partials of every CTA that
-// holds a segment of the tile.  Segment of CTA c: its first segment (slot 2c)
-// when the CTA's range starts inside the tile, else its last (slot 2c + 1).
-template <int D>
-__device__ __forceinline__ void merge_row(const AttnArgs& a, int w, int r, int m, int g, int t, int h) {
-  const long long t0 = (long long)w * a.P;
-  const int c_lo = tc_cta_of(a, t0), c_hi = tc_cta_of(a, t0 + a.P - 1);
-  float mx = -CUDART_INF_F;
-  for (int c = c_lo; c <= c_hi; ++c) {
-    const int slot = tc_unit_begin(a, c) >= t0 ? 2 * c : 2 * c + 1;
-    mx = fmaxf(mx, a.l_part[(size_t)slot * 2 * kBM + r]);
-  }
-  float wsum = 0.f;
-  if (mx != -CUDART_INF_F)
-    for (int c = c_lo; c <= c_hi; ++c) {
-      const int slot = tc_unit_begin(a, c) >= t0 ? 2 * c : 2 * c + 1;
-      wsum += exp2f(a.l_part[(size_t)slot * 2 * kBM + r] - mx);
-    }
-  const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
-  __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(a.out) + ((size_t)t * a.Hq + h) * D;
-#pragma unroll 1
-  for (int c0 = 0; c0 < D; c0 += 32) {
-    float acc[32];
-#pragma unroll
-    for (int k = 0; k < 32; ++k) acc[k] = 0.f;
-    if (mx != -CUDART_INF_F)
-      for (int c = c_lo; c <= c_hi; ++c) {
-        const int slot = tc_unit_begin(a, c) >= t0 ? 2 * c : 2 * c + 1;
-        const size_t row = (size_t)slot * 2 * kBM + r;
-        const float wgt = exp2f(a.l_part[row] - mx) * inv;
-        const float4* src = reinterpret_cast<const float4*>(a.o_part + row * D + c0);
-#pragma unroll
-        for (int v = 0; v < 8; ++v) {
-          const float4 x = src[v];
-          acc[4 * v] += wgt * x.x;
-          acc[4 * v + 1] += wgt * x.y;
-          acc[4 * v + 2] += wgt * x.z;
-          acc[4 * v + 3] += wgt * x.w;
-        }
-      }
-    uint4* dst = reinterpret_cast<uint4*>(o + c0);
-#pragma unroll
-    for (int v = 0; v < 4; ++v)
-      dst[v] = make_uint4(pack_bf16(acc[8 * v], acc[8 * v + 1]), pack_bf16(acc[8 * v + 2], acc[8 * v + 3]),
-                          pack_bf16(acc[8 * v + 4], acc[8 * v + 5]), pack_bf16(acc[8 * v + 6], acc[8 * v + 7]));
-  }
-  if (a.lse) a.lse[(size_t)t * a.Hq + h] = wsum > 0.f ? (mx + log2f(wsum)) * 0.69314718055994531f : -CUDART_INF_F;
-}
-
 template <int D, bool TREE>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kp,
@@ -205,17 +172,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   const uint32_t sbase = smem_u32(smem);
   Shared* sh = reinterpret_cast<Shared*>(smem + C::kOffBar + 224);
+  float* xmax = reinterpret_cast<float*>(smem + C::kOffX);
+  float* xsum = reinterpret_cast<float*>(smem + C::kOffL);
   const uint32_t bar0 = sbase + C::kOffBar;
   Bars B;
   B.q_full = bar0;
-  B.k_full = bar0 + 8;
+  B.q_empty = bar0 + 8;
+  B.k_full = bar0 + 16;
   B.v_full = B.k_full + 8 * C::kNS;
   B.kv_empty = B.v_full + 8 * C::kNS;
   B.s_full = B.kv_empty + 8 * C::kNS;
   B.p_full = B.s_full + 16;
   B.o_full = B.p_full + 16;
   B.drain = B.o_full + 16;
-  const uint32_t q_empty = B.drain + 8;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int cta = blockIdx.x;
@@ -223,7 +192,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(B.q_full, 1);
-    mbar_init(q_empty, 1);
+    mbar_init(B.q_empty, 1);
     for (int s = 0; s < C::kNS; ++s) {
       mbar_init(B.k_full + 8 * s, 1);
       mbar_init(B.v_full + 8 * s, 1);
@@ -231,7 +200,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(B.s_full + 8 * i, 1);
-      mbar_init(B.p_full + 8 * i, 128);
+      mbar_init(B.p_full + 8 * i, 256);
       mbar_init(B.o_full + 8 * i, 1);
     }
     mbar_init(B.drain, 1);
@@ -258,7 +227,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Segment sg = make_segment(a, cta, u, u_end, lane);
       u = (long long)sg.w * a.P + sg.ub;
       if (lane == 0) {
-        if (k > 0 && !wait_bar(q_empty, (k - 1) & 1, abort, a.status)) ok = false;
+        if (k > 0 && !wait_bar(B.q_empty, (k - 1) & 1, abort, a.status)) ok = false;
         if (ok) {
           mbar_expect_tx(B.q_full, 2 * C::kQBytes);
           for (int i = 0; i < 2; ++i)
@@ -324,7 +293,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (ok) {
             issue_s(0, st0);
             issue_s(1, st0);
-            if (n == 1) mma_commit(q_empty);
+            if (n == 1) mma_commit(B.q_empty);
           }
         }
         for (int j = 0; ok && j < n; ++j) {
@@ -349,11 +318,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (j == n - 1) mma_commit(B.o_full + 8);
           if (j + 1 < n) {
             issue_s(1, st1);
-            if (j + 2 == n) mma_commit(q_empty);
+            if (j + 2 == n) mma_commit(B.q_empty);
           }
         }
         if (ok && n == 0) {
-          mma_commit(q_empty);
+          mma_commit(B.q_empty);
           mma_commit(B.o_full);
           mma_commit(B.o_full + 8);
         }
@@ -368,10 +337,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ---------------------------------------------------------------- softmax + epilogue
-    const int i = warp >> 2, q = warp & 3, r = q * 32 + lane;
+    constexpr int kHalfCols = kBN / 2;  // score columns per thread
+    constexpr int kHalfD = D / 2;       // output columns per thread
+    const int i = warp >> 3, hf = (warp >> 2) & 1, q = warp & 3, r = q * 32 + lane;
+    const int bar_id = 1 + i;  // named barrier of the 256 threads of tile i
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-    const uint32_t s_addr = tmem + i * kBN + lane_off;
-    const uint32_t o_addr = tmem + C::kOCol + i * D + lane_off;
+    const uint32_t s_addr = tmem + i * kBN + hf * kHalfCols + lane_off;       // this half's score columns
+    const uint32_t p_addr = tmem + i * kBN + hf * (kHalfCols / 2) + lane_off;  // its packed P columns
+    const uint32_t o_addr = tmem + C::kOCol + i * D + hf * kHalfD + lane_off;
+    const int c_base = hf * kHalfCols;  // key column of this thread's first score
     const float sl2 = a.scale_log2;
     long long J = 0;
     int k = 0;
@@ -405,24 +379,23 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         fence_after_sync();
-        // the S row lives in xs as raw bits (unscaled scores); P is packed in
-        // place into the first half of each 64-column block
-        uint32_t xs[kBN];
-        tmem_ld128(s_addr, xs);
+        // this half's 64 raw scores; P is later packed in place into xs[0..31]
+        uint32_t xs[kHalfCols];
+        tmem_ld64(s_addr, xs);
         constexpr uint32_t kNegInf = 0xff800000u;
         if (j < sg.n_pre) {
-          const int lim = a.Lp - (sg.ua + j) * kBN;  // keys past the prefix are padding
-          if (lim < kBN) {
+          const int lim = a.Lp - (sg.ua + j) * kBN - c_base;  // keys past the prefix are padding
+          if (lim < kHalfCols) {
 #pragma unroll
-            for (int c = 0; c < kBN; ++c)
+            for (int c = 0; c < kHalfCols; ++c)
               if (c >= lim) xs[c] = kNegInf;
           }
         } else {
           // suffix window: same branch up to the row's own token (+ ancestor nodes)
-          const int kb = sg.lo + (j - sg.n_pre) * kBN;
+          const int kb = sg.lo + (j - sg.n_pre) * kBN + c_base;
           const int c_lo = start - kb, c_hi = t - kb;
 #pragma unroll
-          for (int c = 0; c < kBN; ++c) {
+          for (int c = 0; c < kHalfCols; ++c) {
             bool vis = c >= c_lo && c <= c_hi;
             if (TREE) {
 #pragma unroll
@@ -432,38 +405,42 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!vis) xs[c] = kNegInf;
           }
         }
-        // row max of the raw scores: 8 independent chains, then a tree
         float pm[8];
 #pragma unroll
         for (int q8 = 0; q8 < 8; ++q8) pm[q8] = __uint_as_float(xs[q8]);
 #pragma unroll
-        for (int c = 8; c < kBN; ++c) pm[c & 7] = fmaxf(pm[c & 7], __uint_as_float(xs[c]));
-        const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
-                               fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7]))) * sl2;
+        for (int c = 8; c < kHalfCols; ++c) pm[c & 7] = fmaxf(pm[c & 7], __uint_as_float(xs[c]));
+        const float half_max = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                                     fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+        // both halves of the row agree on the maximum (double-buffered by tile parity)
+        float* xm = xmax + ((i * 2 + (int)(JJ & 1)) * 2) * kBM;
+        xm[hf * kBM + r] = half_max;
+        named_sync(bar_id, 256);
+        const float mx = fmaxf(half_max, xm[(1 - hf) * kBM + r]) * sl2;
         float m_new = m_run;
         if (mx > m_run + kLazy || (m_run == -CUDART_INF_F && mx > -CUDART_INF_F)) m_new = mx;
         const float base = m_new == -CUDART_INF_F ? 0.f : m_new;
         const float alpha = ex2(m_run - base);
-        // p = 2^(s * scale * log2e - max): one FFMA and one ex2 per score
+        // p = 2^(s * scale * log2e - max): one FFMA and one exponential per score
         float ps[8];
 #pragma unroll
         for (int q8 = 0; q8 < 8; ++q8) ps[q8] = 0.f;
 #pragma unroll
-        for (int h = 0; h < kBN / 64; ++h) {
-#pragma unroll
-          for (int kk = 0; kk < 32; ++kk) {
-            const float p0 = ex2(fmaf(__uint_as_float(xs[h * 64 + 2 * kk]), sl2, -base));
-            const float p1 = ex2(fmaf(__uint_as_float(xs[h * 64 + 2 * kk + 1]), sl2, -base));
-            ps[kk & 7] += p0 + p1;
-            xs[h * 64 + kk] = pack_bf16(p0, p1);
-          }
-          tmem_st32(s_addr + h * 32, *reinterpret_cast<const uint32_t(*)[32]>(&xs[h * 64]));
+        for (int kk = 0; kk < kHalfCols / 2; ++kk) {
+          const float x0 = fmaf(__uint_as_float(xs[2 * kk]), sl2, -base);
+          const float x1 = fmaf(__uint_as_float(xs[2 * kk + 1]), sl2, -base);
+          const bool fma_pipe = kPolyEvery > 0 && (kk % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1;
+          const float p0 = fma_pipe ? exp2_fma(x0) : ex2(x0);
+          const float p1 = fma_pipe ? exp2_fma(x1) : ex2(x1);
+          ps[kk & 7] += p0 + p1;
+          xs[kk] = pack_bf16(p0, p1);
         }
+        tmem_st32(p_addr, *reinterpret_cast<const uint32_t(*)[32]>(&xs[0]));
         const float rs = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
         l_run = l_run * alpha + rs;
         if (j > 0 && __any_sync(0xffffffffu, m_new != m_run)) {
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
+          for (int c = 0; c < kHalfD / 32; ++c) {
             uint32_t uu[32];
             tmem_ld32(o_addr + c * 32, uu);
 #pragma unroll
@@ -478,18 +455,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (ok) ok = wait_bar(B.o_full + 8 * i, (uint32_t)(k & 1), abort, a.status);
       fence_after_sync();
-      const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+      // the row's normaliser is the sum of both halves' partial sums
+      xsum[(i * 2 + hf) * kBM + r] = l_run;
+      named_sync(bar_id, 256);
+      const float l_row = l_run + xsum[(i * 2 + 1 - hf) * kBM + r];
+      named_sync(bar_id, 256);  // the exchange slots are free again
+      const float inv = l_row > 0.f ? 1.f / l_row : 0.f;
       const bool write = ok && valid && t >= 0;
       const int tt = valid ? m / a.G : 0;
       const int h = valid ? min(max(a.hinv[sg.g * a.G + (m - tt * a.G)], 0), a.Hq - 1) : 0;
       const size_t prow = (size_t)sg.slot * 2 * kBM + i * kBM + r;  // partial row of this thread
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < kHalfD / 32; ++c) {
         uint32_t uu[32];
         tmem_ld32(o_addr + c * 32, uu);
         if (write) {
+          const int col = hf * kHalfD + c * 32;
           if (sg.complete) {
-            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + ((size_t)tt * a.Hq + h) * D + c * 32);
+            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + ((size_t)tt * a.Hq + h) * D + col);
 #pragma unroll
             for (int v = 0; v < 4; ++v) {
               uint4 w4;
@@ -500,7 +483,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               dst[v] = w4;
             }
           } else {
-            float4* dst = reinterpret_cast<float4*>(a.o_part + prow * D + c * 32);
+            float4* dst = reinterpret_cast<float4*>(a.o_part + prow * D + col);
 #pragma unroll
             for (int v = 0; v < 8; ++v)
               dst[v] = make_float4(__uint_as_float(uu[4 * v]) * inv, __uint_as_float(uu[4 * v + 1]) * inv,
@@ -508,37 +491,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      if (write) {
-        const float lse2 = l_run > 0.f ? m_run + __log2f(l_run) : -CUDART_INF_F;
-        if (sg.complete) {
-          if (a.lse) a.lse[(size_t)tt * a.Hq + h] = lse2 * 0.69314718055994531f;
-        } else {
-          a.l_part[prow] = lse2;
-        }
-      } else if (!sg.complete && ok) {
-        a.l_part[prow] = -CUDART_INF_F;  // rows outside the problem merge to nothing
-      }
-      if (!sg.complete) {
-        // The CTA that finishes a split tile's last segment merges all of its
-        // segments (held by consecutive CTAs) with the exact log-sum-exp rule.
-        // Every softmax thread takes these barriers (the condition is uniform
-        // across them); only the counter and the merge depend on `ok`.
-        __threadfence();
-        named_sync(1, 256);
-        if (threadIdx.x == 0) {
-          bool last = false;
-          if (ok && !*abort) {
-            const int nseg = tc_cta_of(a, (long long)(sg.w + 1) * a.P - 1) - tc_cta_of(a, (long long)sg.w * a.P) + 1;
-            last = atomicAdd(&a.tile_count[sg.w], 1) == nseg - 1;
+      if (hf == 0) {
+        const float lse2 = l_row > 0.f ? m_run + __log2f(l_row) : -CUDART_INF_F;
+        if (write) {
+          if (sg.complete) {
+            if (a.lse) a.lse[(size_t)tt * a.Hq + h] = lse2 * 0.69314718055994531f;
+          } else {
+            a.l_part[prow] = lse2;
           }
-          sh->last = last;
+        } else if (!sg.complete && ok) {
+          a.l_part[prow] = -CUDART_INF_F;  // rows outside the problem merge to nothing
         }
-        named_sync(1, 256);
-        if (sh->last && ok) {
-          __threadfence();
-          if (valid && t >= 0) merge_row<D>(a, sg.w, r + i * kBM, m, sg.g, tt, h);
-        }
-        named_sync(1, 256);
       }
       J += sg.n;
     }
@@ -549,6 +512,106 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_after_sync();
     tmem_dealloc(tmem, 512);
   }
+}
+
+// Merge the partial segments of every work tile the schedule split.  Block
+// (b, y) looks at the boundary of CTA c = b + 1; if that boundary is the first
+// one strictly inside a tile, the block merges rows [32y, 32y + 32) of that
+// tile — each warp four rows, lanes over columns — from the segments held by
+// consecutive CTAs, with the exact log-sum-exp rule of the split merge.
+constexpr int kMaxSeg = 64;
+constexpr int kFixRows = 32;
+
+template <int D>
+__global__ void __launch_bounds__(256) tc_fixup_kernel(const AttnArgs a) {
+  constexpr int kE = D / 32;  // columns per lane
+  __shared__ int s_slot[kMaxSeg];
+  __shared__ int s_nseg, s_w;
+  const int c = blockIdx.x + 1;
+  if (threadIdx.x == 0) {
+    s_nseg = 0;
+    const long long u = tc_unit_begin(a, c);
+    const int w = (int)(u / a.P);
+    const long long t0 = (long long)w * a.P, t1 = t0 + a.P;
+    if (u % a.P != 0 && !(c >= 2 && tc_unit_begin(a, c - 1) > t0)) {
+      int n = 0;
+      for (int cc = c - 1; cc < a.n_ctas && n < kMaxSeg; ++cc) {
+        const long long ub = tc_unit_begin(a, cc);
+        if (ub >= t1) break;
+        s_slot[n++] = ub >= t0 ? 2 * cc : 2 * cc + 1;
+      }
+      s_nseg = n;
+      s_w = w;
+    }
+  }
+  __syncthreads();
+  const int nseg = s_nseg;
+  if (nseg == 0) return;
+  const int w = s_w;
+  const int g = w / a.n_pairs, m0 = (w - g * a.n_pairs) * 2 * kBM;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int kR = kFixRows / 8;  // rows per warp, merged side by side
+  const int r0 = blockIdx.y * kFixRows + warp * kR;
+  float mx[kR], wsum[kR], acc[kR][kE];
+  // normalisers: lanes read the segments side by side, for every row at once
+#pragma unroll
+  for (int q = 0; q < kR; ++q) {
+    mx[q] = -CUDART_INF_F;
+    for (int s = lane; s < nseg; s += 32) mx[q] = fmaxf(mx[q], a.l_part[(size_t)s_slot[s] * 2 * kBM + r0 + q]);
+  }
+#pragma unroll
+  for (int q = 0; q < kR; ++q) {
+    mx[q] = warp_max(mx[q]);
+    wsum[q] = 0.f;
+#pragma unroll
+    for (int e = 0; e < kE; ++e) acc[q][e] = 0.f;
+  }
+  // weighted sum of the segments' partial rows; loads of all rows are independent
+  for (int s = 0; s < nseg; ++s) {
+    const size_t base = (size_t)s_slot[s] * 2 * kBM + r0;
+    float lv[kR];
+    float4 ov[kR][kE / 4 > 0 ? kE / 4 : 1];
+    float2 ov2[kR];
+#pragma unroll
+    for (int q = 0; q < kR; ++q) {
+      lv[q] = a.l_part[base + q];
+      if (kE == 4) ov[q][0] = *reinterpret_cast<const float4*>(a.o_part + (base + q) * D + lane * kE);
+      else ov2[q] = *reinterpret_cast<const float2*>(a.o_part + (base + q) * D + lane * kE);
+    }
+#pragma unroll
+    for (int q = 0; q < kR; ++q) {
+      if (mx[q] == -CUDART_INF_F) continue;
+      const float wgt = exp2f(lv[q] - mx[q]);
+      wsum[q] += wgt;
+      if (kE == 4) {
+        acc[q][0] += wgt * ov[q][0].x;
+        acc[q][1 % kE] += wgt * ov[q][0].y;
+        acc[q][2 % kE] += wgt * ov[q][0].z;
+        acc[q][3 % kE] += wgt * ov[q][0].w;
+      } else {
+        acc[q][0] += wgt * ov2[q].x;
+        acc[q][1 % kE] += wgt * ov2[q].y;
+      }
+    }
+  }
+#pragma unroll
+  for (int q = 0; q < kR; ++q) {
+    const int m = m0 + r0 + q;
+    if (m >= a.M) break;
+    const float inv = wsum[q] > 0.f ? 1.f / wsum[q] : 0.f;
+    const int t = m / a.G;
+    const int h = min(max(a.hinv[g * a.G + (m - t * a.G)], 0), a.Hq - 1);
+    __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(a.out) + ((size_t)t * a.Hq + h) * D + lane * kE;
+#pragma unroll
+    for (int e = 0; e < kE; e += 2) *reinterpret_cast<uint32_t*>(o + e) = pack_bf16(acc[q][e] * inv, acc[q][e + 1] * inv);
+    if (a.lse && lane == 0)
+      a.lse[(size_t)t * a.Hq + h] = wsum[q] > 0.f ? (mx[q] + log2f(wsum[q])) * 0.69314718055994531f : -CUDART_INF_F;
+  }
+}
+
+__global__ void exp2_selftest_kernel(const float* x, float* y, int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) y[i] = exp2_fma(x[i]);
 }
 
 // ---------------------------------------------------------------- host side
@@ -618,6 +681,12 @@ cudaError_t launch_dt(const AttnArgs& a, cudaStream_t s) {
 
 }  // namespace
 
+cudaError_t launch_exp2_selftest(const float* x, float* y, int n, cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  exp2_selftest_kernel<<<(n + 255) / 256, 256, 0, s>>>(x, y, n);
+  return cudaGetLastError();
+}
+
 bool attn_tc_supported(int d) {
   if (d != 64 && d != 128) return false;
   static int cc = -1;
@@ -631,6 +700,14 @@ bool attn_tc_supported(int d) {
     cc = major;
   }
   return cc == 10 && encode_fn() != nullptr;
+}
+
+cudaError_t launch_tc_fixup(const AttnArgs& a, cudaStream_t s) {
+  if (a.n_ctas < 2) return cudaSuccess;
+  const dim3 grid(a.n_ctas - 1, 2 * kBM / kFixRows);
+  if (a.d == 128) tc_fixup_kernel<128><<<grid, 256, 0, s>>>(a);
+  else tc_fixup_kernel<64><<<grid, 256, 0, s>>>(a);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t s) {

@@ -150,7 +150,38 @@ Plan plan_of(const jev_attn_desc* d, int T) {
     p.P = ktiles + 1;
     p.U = (long long)p.n_tiles * p.P;
     const int s = d->num_splits;
-    long long n = s == 1 ? p.n_tiles : s > 1 ? (long long)p.n_tiles * s : (long long)num_sms();
+    long long n;
+    if (s == 1) {
+      n = p.n_tiles;
+    } else if (s > 1) {
+      n = (long long)p.n_tiles * s;
+    } else {
+      // Estimated time of each CTA count up to one per SM: the busiest CTA's
+      // units and segments, plus a merge launch when some tile is split
+      // (a fixed cost and a little per segment).  Times in microseconds.
+      const double unit_us = 4.0 * 256 * 128 * d->d / 6.8e12 * 1e6, seg_us = 3.0, merge_us = 0.5;
+      double best = 1e30;
+      n = 1;
+      const long long n_max = std::min<long long>(num_sms(), p.U);
+      for (long long cand = 1; cand <= n_max; ++cand) {
+        double worst = 0.0;
+        long long max_tile_segs = 1;
+        bool split = false;
+        for (long long c = 0; c < cand; ++c) {
+          const long long u0 = c * p.U / cand, u1 = (c + 1) * p.U / cand;
+          if (u1 <= u0) continue;
+          const long long segs = (u1 - 1) / p.P - u0 / p.P + 1;
+          worst = std::max(worst, (u1 - u0) * unit_us + segs * seg_us);
+          if (u0 % p.P) split = true;
+        }
+        if (split) max_tile_segs = (p.P * cand + p.U - 1) / p.U + 1;
+        const double t = worst + (split ? 6.0 + merge_us * max_tile_segs : 0.0);
+        if (t < best * 0.98) {
+          best = t;
+          n = cand;
+        }
+      }
+    }
     // a tile spread over many CTAs costs a long merge; keep it within 64 segments
     n = std::min(n, (long long)p.n_tiles * 64);
     p.n_ctas = (int)std::max(1LL, std::min(n, p.U));
@@ -176,7 +207,7 @@ Plan plan_of(const jev_attn_desc* d, int T) {
 }
 
 struct Layout {
-  size_t hinv, info, qrot, krot, opart, lpart, count, anc, nanc, total;
+  size_t hinv, info, qrot, krot, opart, lpart, anc, nanc, total;
 };
 Layout layout_of(const jev_attn_desc* d, int T, const Plan& p, int n_nodes) {
   Layout L;
@@ -188,12 +219,10 @@ Layout layout_of(const jev_attn_desc* d, int T, const Plan& p, int n_nodes) {
   L.krot = off; off += up256((size_t)T * d->Hkv * d->d * s);
   L.opart = off;
   L.lpart = off;
-  L.count = off;
   if (p.tc && p.split) {
     const size_t rows = (size_t)2 * p.n_ctas * 256;  // two partial segments per CTA at most
     L.opart = off; off += up256(rows * d->d * 4);
     L.lpart = off; off += up256(rows * 4);
-    L.count = off; off += up256((size_t)p.n_tiles * 4);
   } else if (!p.tc && p.S > 1) {
     L.opart = off; off += up256((size_t)p.S * d->Hkv * p.M * d->d * 4);
     L.lpart = off; off += up256((size_t)p.S * d->Hkv * p.M * 4);
@@ -241,8 +270,6 @@ jev_status attention_core(const jev_attn_desc* d, int T, const Plan& p, const La
   r.n_segs = n_segs; r.T = T; r.Hq = d->Hq; r.Hkv = d->Hkv; r.d = d->d;
   r.pos_offset = d->pos_offset >= 0 ? d->pos_offset : d->Lp;
   r.theta = (double)d->rope_theta;
-  r.zero_buf = reinterpret_cast<int32_t*>(ws + L.count);
-  r.zero_n = (p.tc && p.split) ? p.n_tiles : 0;
   for (int i = 0; i < d->d / 2; ++i) r.inv_freq[i] = std::pow(r.theta, -2.0 * i / d->d);
   jev_status st = run("rope_pack", s, [&] { return launch_rope_pack(r, d->dtype, s); });
   if (st) return st;
@@ -261,8 +288,11 @@ jev_status attention_core(const jev_attn_desc* d, int T, const Plan& p, const La
   a.S = p.S; a.split_len = p.split_len;
   a.scale_log2 = scale_log2_of(d);
   a.n_pairs = p.n_pairs; a.n_tiles = p.n_tiles; a.n_pre = p.n_pre; a.P = p.P; a.n_ctas = p.n_ctas; a.U = p.U;
-  a.tile_count = reinterpret_cast<int32_t*>(ws + L.count);
-  if (p.tc) return run("attn_tc", s, [&] { return launch_attn_tc(a, s); });
+  if (p.tc) {
+    st = run("attn_tc", s, [&] { return launch_attn_tc(a, s); });
+    if (st == JEV_OK && p.split) st = run("tc_fixup", s, [&] { return launch_tc_fixup(a, s); });
+    return st;
+  }
   st = run("attn_simt", s, [&] { return launch_attn_simt(a, d->dtype, s); });
   if (st) return st;
   if (p.S > 1) {
@@ -352,6 +382,11 @@ size_t jev_prefix_suffix_attn_workspace(const jev_attn_desc* d) {
   if (check_desc(d) != JEV_OK) return 0;
   Plan p = plan_of(d, d->T_total);
   return layout_of(d, d->T_total, p, 0).total;
+}
+
+jev_status jev_selftest_exp2(const float* x, float* y, int32_t n, jev_stream_t stream) {
+  if (n < 0 || (n > 0 && (!x || !y))) return fail(JEV_ERR_INVALID_ARG, "bad arguments");
+  return run("selftest_exp2", (cudaStream_t)stream, [&] { return launch_exp2_selftest(x, y, n, (cudaStream_t)stream); });
 }
 
 jev_status jev_workspace_init(void* ws, size_t ws_bytes, jev_stream_t stream) {

@@ -24,8 +24,6 @@ struct RopePackArgs {
   int n_segs, T, Hq, Hkv, d, pos_offset;
   double theta;
   double inv_freq[128];    // theta^(-2i/d), i < d/2, formed on the host in double
-  int32_t* zero_buf;       // zeroed before the attention kernel runs (its per-tile counters)
-  int zero_n;
 };
 cudaError_t launch_rope_pack(const RopePackArgs& a, jev_dtype dt, cudaStream_t s);
 
@@ -63,7 +61,6 @@ struct AttnArgs {
   // window); CTA c owns units [c*U/n_ctas, (c+1)*U/n_ctas).
   int n_pairs, n_tiles, n_pre, P, n_ctas;
   long long U;
-  int32_t* tile_count;      // [n_tiles] finished segments per split tile (zeroed by rope_pack)
 };
 // units of the tensor-core schedule owned by CTAs before c
 __host__ __device__ inline long long tc_unit_begin(const AttnArgs& a, int c) { return (long long)c * a.U / a.n_ctas; }
@@ -71,7 +68,10 @@ __host__ __device__ inline long long tc_unit_begin(const AttnArgs& a, int c) { r
 __host__ __device__ inline int tc_cta_of(const AttnArgs& a, long long u) { return (int)(((u + 1) * a.n_ctas - 1) / a.U); }
 cudaError_t launch_attn_simt(const AttnArgs& a, jev_dtype dt, cudaStream_t s);
 cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t s);  // bf16, d in {64,128}
+// merge the partial segments of work tiles that the schedule split across CTAs
+cudaError_t launch_tc_fixup(const AttnArgs& a, cudaStream_t s);
 bool attn_tc_supported(int d);
+cudaError_t launch_exp2_selftest(const float* x, float* y, int n, cudaStream_t s);
 
 struct MergeArgs {
   const float* o_part;  // [S, Hkv, M, d]

@@ -55,7 +55,6 @@ __global__ void __launch_bounds__(256) rope_pack_kernel(RopePackArgs a) {
   __shared__ float cs[kTokPerBlock][128], sn[kTokPerBlock][128];
   __shared__ int s_slot[256], s_grp[256];
   __shared__ int s_offs[kSmemOffs];
-  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < a.zero_n; i += gridDim.x * blockDim.x) a.zero_buf[i] = 0;
   const bool offs_in_smem = a.n_segs + 1 <= kSmemOffs;
   if (offs_in_smem)
     for (int i = threadIdx.x; i <= a.n_segs; i += blockDim.x) s_offs[i] = a.offs[i];
@@ -103,10 +102,20 @@ __global__ void __launch_bounds__(256) rope_pack_kernel(RopePackArgs a) {
   }
   pos = __shfl_sync(0xffffffffu, pos, 0);
   for (int i = lane; i < half; i += 32) {
+#ifdef JEV_ROPE_REDUCED_F32
+    // angle in double, reduced to [-pi, pi] in double, then a float sincos
+    const double ang = (double)pos * a.inv_freq[i];
+    const double r = ang - rint(ang * 0.15915494309189535) * 6.283185307179586;
+    float sf, cf;
+    sincosf((float)r, &sf, &cf);
+    cs[warp][i] = cf;
+    sn[warp][i] = sf;
+#else
     double sv, cv;
     sincos((double)pos * a.inv_freq[i], &sv, &cv);
     cs[warp][i] = (float)cv;
     sn[warp][i] = (float)sv;
+#endif
   }
   __syncwarp();
   const int lanes_per_head = half / 8;          // 8 (d = 128) or 4 (d = 64)

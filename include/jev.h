@@ -279,6 +279,12 @@ jev_status jev_tree_attn(const jev_attn_desc* desc, int32_t n_nodes, const int32
 jev_status jev_rope_inplace(void* x, int32_t L, int32_t H, int32_t d, int32_t pos0, float theta,
                             jev_dtype dtype, jev_stream_t stream);
 
+/* Self-test of the FMA-pipe 2^x the attention kernel uses for a share of its
+ * softmax exponentials (cubic on the reduced argument; relative error below
+ * 2e-4 for -125 <= x <= 2^22, about 2^-125 below -125): y[i] = 2^x[i] for
+ * n device floats. */
+jev_status jev_selftest_exp2(const float* x, float* y, int32_t n, jev_stream_t stream);
+
 /* Zero the status word at the start of a workspace (enqueued on stream). */
 jev_status jev_workspace_init(void* workspace, size_t ws_bytes, jev_stream_t stream);
 

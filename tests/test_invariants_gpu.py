@@ -130,3 +130,15 @@ def test_tree_status_flags_deep_chain(jev):
                                 synth.f32_to_bf16_bits(host_f64(vr).astype(np.float32)))
     ok_rows = 8  # nodes 1..8 have depth <= 8
     assert np.abs(host_f64(out)[:ok_rows] - ref_o[:ok_rows]).max() <= TOL[synth.BF16]["max_abs"]
+
+
+def test_fma_pipe_exp2_against_cuda_exp2(jev):
+    """The software 2^x used for a share of the softmax exponentials stays
+    within its stated bound of CUDA's exp2 over the range softmax feeds it."""
+    x = torch.linspace(-125.0, 8.5, 1_000_003, device="cuda", dtype=torch.float32)
+    y = jev.jev_selftest_exp2(x)
+    ref = torch.exp2(x.double())
+    rel = (y.double() / ref - 1.0).abs().max().item()
+    assert rel < 2e-4, rel
+    z = jev.jev_selftest_exp2(torch.tensor([-float("inf"), -1000.0, -200.0], device="cuda"))
+    assert (z >= 0).all() and (z < 1e-37).all()
