@@ -216,6 +216,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   fence_after_sync();
   const uint32_t tmem = sh->tmem_base;
   volatile int* abort = &sh->abort;
+  // everything above is independent of the previous kernel (the RoPE pack);
+  // its outputs are read only after this wait.  The merge kernel may launch now.
+  pdl_wait();
+  if (threadIdx.x == 0) pdl_trigger();
 
   if (warp == kProducerWarp) {
     // ---------------------------------------------------------------- TMA producer
@@ -547,6 +551,7 @@ __global__ void __launch_bounds__(256) tc_fixup_kernel(const AttnArgs a) {
   __syncthreads();
   const int nseg = s_nseg;
   if (nseg == 0) return;
+  pdl_wait();  // the partials are written by the attention kernel
   const int w = s_w;
   const int g = w / a.n_pairs, m0 = (w - g * a.n_pairs) * 2 * kBM;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -675,8 +680,17 @@ cudaError_t launch_dt(const AttnArgs& a, cudaStream_t s) {
     return cudaErrorInvalidValue;
   if (!map_2d(&mks, a.k_rot, (uint64_t)a.Hkv * D, a.T, row) || !map_2d(&mvs, a.v_suf, (uint64_t)a.Hkv * D, a.T, row))
     return cudaErrorInvalidValue;
-  attn_tc_kernel<D, TREE><<<a.n_ctas, kThreads, Cfg<D>::kSmem, s>>>(mq, mkp, mvp, mks, mvs, a);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = dim3(a.n_ctas);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = Cfg<D>::kSmem;
+  cfg.stream = s;
+  cfg.attrs = pdl;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, attn_tc_kernel<D, TREE>, mq, mkp, mvp, mks, mvs, a);
 }
 
 }  // namespace
@@ -704,10 +718,18 @@ bool attn_tc_supported(int d) {
 
 cudaError_t launch_tc_fixup(const AttnArgs& a, cudaStream_t s) {
   if (a.n_ctas < 2) return cudaSuccess;
-  const dim3 grid(a.n_ctas - 1, 2 * kBM / kFixRows);
-  if (a.d == 128) tc_fixup_kernel<128><<<grid, 256, 0, s>>>(a);
-  else tc_fixup_kernel<64><<<grid, 256, 0, s>>>(a);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = dim3(a.n_ctas - 1, 2 * kBM / kFixRows);
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (a.d == 128) return cudaLaunchKernelEx(&cfg, tc_fixup_kernel<128>, a);
+  return cudaLaunchKernelEx(&cfg, tc_fixup_kernel<64>, a);
 }
 
 cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t s) {

@@ -28,6 +28,14 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialization may start while the previous kernel of the stream finishes;
+// pdl_wait() blocks until that kernel has completed and its writes are
+// visible (a no-op for an ordinary launch), pdl_trigger() lets the next
+// kernel start launching once every CTA of this grid has issued it.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ void raise_flag(int32_t* status, int32_t bit) {
   if (status) atomicOr(status, bit);
 }

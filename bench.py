@@ -256,11 +256,148 @@ KERNEL_SRC = {
 }
 
 
+class FlatWorkload:
+    """Shared-prefix attention (one layer, all heads, all branches) + readout."""
+
+    def __init__(self, cfg, dev, jev, torch):
+        self.cfg, self.jev, self.torch = cfg, jev, torch
+        c = synth.flat_case(cfg, with_lm_head=False)
+        self.c = c
+        self.work = flat_work(c)
+        self.T, self.B = self.work["T"], cfg.B
+        self.tdt = torch.bfloat16 if cfg.dtype == synth.BF16 else torch.float32
+        self.W = load_lm_head(cfg, dev, torch, self.tdt)
+        self.base = dict(q=to_dev(c.q, dev, torch), k_pre=to_dev(c.k_pre, dev, torch), v_pre=to_dev(c.v_pre, dev, torch),
+                         k_suf=to_dev(c.k_suf, dev, torch), v_suf=to_dev(c.v_suf, dev, torch),
+                         hidden=to_dev(c.hidden, dev, torch), pair_tok=to_dev(c.pair_tok, dev, torch))
+        self.cu = to_dev(c.cu_seqlens, dev, torch)
+        self.so = to_dev(c.set_offsets, dev, torch)
+        desc = jev.make_attn_desc(cfg.B, cfg.Lp, cfg.Hq, cfg.Hkv, cfg.d, self.T,
+                                  jev.JEV_BF16 if self.tdt == torch.bfloat16 else jev.JEV_F32, cfg.theta)
+        self.ws = jev.new_workspace(jev.jev_prefix_suffix_attn_workspace(desc), dev)
+        self.out = torch.empty_like(self.base["q"])
+        self.lse = torch.empty((self.T, cfg.Hq), dtype=torch.float32, device=dev)
+        self.lp = torch.empty(c.pair_tok.size, dtype=torch.float32, device=dev)
+        self.choice = torch.empty(cfg.B, dtype=torch.int32, device=dev)
+        self.e2e_inputs = ("q", "k_suf", "v_suf", "hidden", "pair_tok")
+
+    def attn(self, cp, s):
+        self.jev.jev_prefix_suffix_attn(cp["q"], cp["k_pre"], cp["v_pre"], cp["k_suf"], cp["v_suf"], cp.get("cu", self.cu),
+                                        out=self.out, lse=self.lse, workspace=self.ws, rope_theta=self.cfg.theta, stream=s)
+
+    def readout(self, cp, s):
+        self.jev.jev_candidate_readout(cp["hidden"], self.W, cp.get("so", self.so), cp["pair_tok"], logprob=self.lp,
+                                       choice=self.choice, stream=s)
+
+    def e2e_host(self):
+        """Host-side inputs of one request (pinned) and the per-step host work."""
+        t = self.torch
+        h = {k: self.base[k].cpu().pin_memory() for k in self.e2e_inputs}
+        h["cu"] = self.cu.cpu().pin_memory()
+        h["so"] = self.so.cpu().pin_memory()
+        return h
+
+    def host_prep(self, h):
+        return h
+
+    def describe_e2e(self):
+        return ("per step: pinned H2D of suffix q/k/v, cu_seqlens, hidden rows and option sets; both C-ABI "
+                "calls; D2H of log-probs and choices (prefix cache and LM head stay resident)")
+
+
+class TreeWorkload(FlatWorkload):
+    """Candidate-prefix tree: trie-packed tokens attend to the root cache, their
+    ancestors and their own node; readout of each leaf over its siblings."""
+
+    def __init__(self, cfg, dev, jev, torch):
+        self.cfg, self.jev, self.torch = cfg, jev, torch
+        tc = synth.tree_case(cfg, with_lm_head=False)
+        self.tc = tc
+        trie = jev.jev_tree_build(tc.seq_off, tc.toks, cfg.Lp)
+        plan = jev.jev_tree_readout_plan(tc.seq_off, tc.toks, tc.score_from, trie["path_row"])
+        self.trie, self.plan = trie, plan
+        N = int(trie["tok_off"][-1])
+        # exact key count of every tree token: root cache + ancestors + own node up to itself
+        pos = np.concatenate([trie["pos0"][n] + np.arange(trie["tok_off"][n + 1] - trie["tok_off"][n])
+                              for n in range(1, trie["n_nodes"])])
+        keys = pos.astype(np.int64) + 1
+        s = 2
+        n_pairs = plan["pair_tok"].size
+        self.work = dict(T=N, B=int(tc.seq_off.size - 1),
+                         flops_attn=int(4 * cfg.Hq * cfg.d * keys.sum()),
+                         flops_readout=2 * cfg.H * n_pairs,
+                         bytes_attn=s * (2 * N * cfg.Hq * cfg.d + 2 * cfg.Lp * cfg.Hkv * cfg.d + 2 * N * cfg.Hkv * cfg.d) + 4 * N * cfg.Hq,
+                         bytes_readout=s * (N * cfg.H + n_pairs * cfg.H) + 8 * n_pairs)
+        self.T, self.B = N, self.work["B"]
+        self.tdt = torch.bfloat16
+        self.W = load_lm_head(cfg, dev, torch, self.tdt)
+        self.base = dict(q=to_dev(tc.q, dev, torch), k_pre=to_dev(tc.k_root, dev, torch), v_pre=to_dev(tc.v_root, dev, torch),
+                         k_suf=to_dev(tc.k, dev, torch), v_suf=to_dev(tc.v, dev, torch),
+                         hidden=to_dev(tc.hidden, dev, torch), pair_tok=to_dev(plan["pair_tok"], dev, torch))
+        self.parent = to_dev(trie["parent"], dev, torch)
+        self.tok_off = to_dev(trie["tok_off"], dev, torch)
+        self.pos0 = to_dev(trie["pos0"], dev, torch)
+        self.co = to_dev(plan["cand_offsets"], dev, torch)
+        self.prow = to_dev(plan["pair_row"], dev, torch)
+        self.so = to_dev(tc.set_offsets, dev, torch)
+        desc = jev.make_attn_desc(trie["n_nodes"] - 1, cfg.Lp, cfg.Hq, cfg.Hkv, cfg.d, N, jev.JEV_BF16, cfg.theta)
+        self.ws = jev.new_workspace(jev.jev_tree_attn_workspace(desc, trie["n_nodes"]), dev)
+        self.out = torch.empty_like(self.base["q"])
+        self.lse = torch.empty((N, cfg.Hq), dtype=torch.float32, device=dev)
+        self.lp = torch.empty(self.co.numel() - 1, dtype=torch.float32, device=dev)
+        self.choice = torch.empty(self.so.numel() - 1, dtype=torch.int32, device=dev)
+        self.e2e_inputs = ("q", "k_suf", "v_suf", "hidden")
+
+    def attn(self, cp, s):
+        self.jev.jev_tree_attn(cp.get("parent", self.parent), cp.get("tok_off", self.tok_off), cp.get("pos0", self.pos0),
+                               cp["q"], cp["k_pre"], cp["v_pre"], cp["k_suf"], cp["v_suf"], out=self.out, lse=self.lse,
+                               workspace=self.ws, rope_theta=self.cfg.theta, stream=s)
+
+    def readout(self, cp, s):
+        self.jev.jev_candidate_readout(cp["hidden"], self.W, cp.get("so", self.so), cp.get("pair_tok", self.base["pair_tok"]),
+                                       cand_offsets=cp.get("co", self.co), pair_row=cp.get("prow", self.prow),
+                                       logprob=self.lp, choice=self.choice, stream=s)
+
+    def e2e_host(self):
+        h = {k: self.base[k].cpu().pin_memory() for k in self.e2e_inputs}
+        return h
+
+    def host_prep(self, h):
+        """The trie build and readout plan of the request run on the host every step."""
+        tc, jev, t = self.tc, self.jev, self.torch
+        trie = jev.jev_tree_build(tc.seq_off, tc.toks, self.cfg.Lp)
+        plan = jev.jev_tree_readout_plan(tc.seq_off, tc.toks, tc.score_from, trie["path_row"])
+        h = dict(h)
+        for k, v in (("parent", trie["parent"]), ("tok_off", trie["tok_off"]), ("pos0", trie["pos0"]),
+                     ("co", plan["cand_offsets"]), ("prow", plan["pair_row"]), ("pair_tok", plan["pair_tok"]),
+                     ("so", tc.set_offsets)):
+            h[k] = t.from_numpy(np.ascontiguousarray(v, dtype=np.int32)).pin_memory()
+        return h
+
+    def describe_e2e(self):
+        return ("per step: host trie build and readout plan, pinned H2D of the tree arrays, tree-token q/k/v, "
+                "hidden rows and readout pairs; both C-ABI calls; D2H of log-probs and choices (root cache and "
+                "LM head stay resident)")
+
+
+def to_dev(a, dev, torch):
+    if a.dtype == np.uint16:
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev).view(torch.bfloat16)
+    return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+
+
+def load_lm_head(cfg, dev, torch, tdt):
+    W = torch.empty((cfg.V, cfg.H), dtype=tdt, device=dev)
+    for ch in range((cfg.V + synth.W_CHUNK_ROWS - 1) // synth.W_CHUNK_ROWS):
+        blk = synth.lm_head_block(cfg.seed, cfg.V, cfg.H, ch, cfg.dtype, cfg.w_std)
+        W[ch * synth.W_CHUNK_ROWS: ch * synth.W_CHUNK_ROWS + blk.shape[0]] = to_dev(blk, dev, torch)
+    return W
+
+
 def jev_arm(args, wl_name):
     import torch
     import torch.distributed as dist
     import attention_cascade_b200 as jev
-    from attention_cascade_b200 import _build  # noqa: F401  (the library is loaded at import)
 
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -270,43 +407,18 @@ def jev_arm(args, wl_name):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     dev = torch.device("cuda", local)
     cfg = synth.CONFIGS[wl_name]
-    if isinstance(cfg, synth.TreeConfig):
-        raise SystemExit("bench.py: the tree workload is measured by the parity tests; use a flat workload")
+    wl = (TreeWorkload if isinstance(cfg, synth.TreeConfig) else FlatWorkload)(cfg, dev, jev, torch)
+    work, T = wl.work, wl.T
 
-    # ---- inputs (host generation, one copy; device clones to exceed L2)
-    c = synth.flat_case(cfg, with_lm_head=False)
-    work = flat_work(c)
-    tdt = torch.bfloat16 if cfg.dtype == synth.BF16 else torch.float32
-
-    def to_dev(a):
-        if a.dtype == np.uint16:
-            return torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
-        return torch.from_numpy(a).to(dev)
-
-    W = torch.empty((cfg.V, cfg.H), dtype=tdt, device=dev)
-    for ch in range((cfg.V + synth.W_CHUNK_ROWS - 1) // synth.W_CHUNK_ROWS):
-        blk = synth.lm_head_block(cfg.seed, cfg.V, cfg.H, ch, cfg.dtype, cfg.w_std)
-        W[ch * synth.W_CHUNK_ROWS: ch * synth.W_CHUNK_ROWS + blk.shape[0]] = to_dev(blk)
-    base = dict(q=to_dev(c.q), k_pre=to_dev(c.k_pre), v_pre=to_dev(c.v_pre), k_suf=to_dev(c.k_suf),
-                v_suf=to_dev(c.v_suf), hidden=to_dev(c.hidden), pair_tok=to_dev(c.pair_tok))
-    per_copy = sum(t.numel() * t.element_size() for t in base.values())
+    # ---- device copies of the per-step inputs, enough to exceed twice the L2
+    per_copy = sum(t.numel() * t.element_size() for t in wl.base.values())
     ncopies = max(2, math.ceil(2 * L2_BYTES / per_copy))
     copies = []
     for i in range(ncopies):
-        cp = {k: v.clone() for k, v in base.items()}
+        cp = {k: v.clone() for k, v in wl.base.items()}
         # each copy reads different option rows of the LM head
-        cp["pair_tok"] = ((base["pair_tok"].long() + 7919 * i) % cfg.V).to(torch.int32)
+        cp["pair_tok"] = ((wl.base["pair_tok"].long() + 7919 * i) % cfg.V).to(torch.int32)
         copies.append(cp)
-    cu = to_dev(c.cu_seqlens)
-    so = to_dev(c.set_offsets)
-    T = work["T"]
-    desc = jev.make_attn_desc(cfg.B, cfg.Lp, cfg.Hq, cfg.Hkv, cfg.d, T, jev.JEV_BF16 if tdt == torch.bfloat16 else jev.JEV_F32,
-                              cfg.theta)
-    ws = jev.new_workspace(jev.jev_prefix_suffix_attn_workspace(desc), dev)
-    out = torch.empty_like(base["q"])
-    lse = torch.empty((T, cfg.Hq), dtype=torch.float32, device=dev)
-    lp = torch.empty(c.pair_tok.size, dtype=torch.float32, device=dev)
-    choice = torch.empty(cfg.B, dtype=torch.int32, device=dev)
     stream = torch.cuda.Stream(device=dev)
     side = torch.cuda.Stream(device=dev)
 
@@ -315,9 +427,8 @@ def jev_arm(args, wl_name):
         # this attention layer, so it runs on a second stream, forked and
         # joined inside the step
         side.wait_stream(s)
-        jev.jev_candidate_readout(cp["hidden"], W, so, cp["pair_tok"], logprob=lp, choice=choice, stream=side)
-        jev.jev_prefix_suffix_attn(cp["q"], cp["k_pre"], cp["v_pre"], cp["k_suf"], cp["v_suf"], cu, out=out, lse=lse,
-                                   workspace=ws, rope_theta=cfg.theta, stream=s)
+        wl.readout(cp, side)
+        wl.attn(cp, s)
         s.wait_stream(side)
 
     # ---- graphs: one per input copy (at most one per timed step)
@@ -368,7 +479,7 @@ def jev_arm(args, wl_name):
         t = torch.tensor([ms], device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms = float(t.item())
-    assert jev.jev_check_device_status(ws, stream) == 0, "device status flags set during the bench"
+    assert jev.jev_check_device_status(wl.ws, stream) == 0, "device status flags set during the bench"
 
     # ---- per-kernel durations: the same K steps replayed from graphs whose
     # kernels are bracketed by CUDA event nodes on the launching stream; each
@@ -380,29 +491,27 @@ def jev_arm(args, wl_name):
     del pgraphs
 
     # ---- end to end through the public API: pinned host inputs in, results out, every step
-    hq = {k: base[k].cpu().pin_memory() for k in ("q", "k_suf", "v_suf", "hidden", "pair_tok")}
-    h_cu = cu.cpu().pin_memory()
-    h_so = so.cpu().pin_memory()
-    d_in = {k: torch.empty_like(base[k]) for k in hq}
-    d_cu, d_so = torch.empty_like(cu), torch.empty_like(so)
-    h_lp = torch.empty(lp.shape, dtype=lp.dtype).pin_memory()
-    h_ch = torch.empty(choice.shape, dtype=choice.dtype).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in hq.values()) + h_cu.numel() * 4 + h_so.numel() * 4
-    d2h = h_lp.numel() * 4 + h_ch.numel() * 4
-    k_pre, v_pre = base["k_pre"], base["v_pre"]
+    hq = wl.e2e_host()
+    d_in = {}
+    h_lp = torch.empty(wl.lp.shape, dtype=wl.lp.dtype).pin_memory()
+    h_ch = torch.empty(wl.choice.shape, dtype=wl.choice.dtype).pin_memory()
+    cp_static = {k: v for k, v in wl.base.items() if k in ("k_pre", "v_pre")}
+    h2d_holder = {}
 
     def e2e_step(s):
-        for k in hq:
-            d_in[k].copy_(hq[k], non_blocking=True)
-        d_cu.copy_(h_cu, non_blocking=True)
-        d_so.copy_(h_so, non_blocking=True)
-        side.wait_stream(s)
-        jev.jev_candidate_readout(d_in["hidden"], W, d_so, d_in["pair_tok"], logprob=lp, choice=choice, stream=side)
-        jev.jev_prefix_suffix_attn(d_in["q"], k_pre, v_pre, d_in["k_suf"], d_in["v_suf"], d_cu, out=out, lse=lse,
-                                   workspace=ws, rope_theta=cfg.theta, stream=s)
-        s.wait_stream(side)
-        h_lp.copy_(lp, non_blocking=True)
-        h_ch.copy_(choice, non_blocking=True)
+        h = wl.host_prep(hq)
+        cp = dict(cp_static)
+        nbytes = 0
+        for k, v in h.items():
+            if k not in d_in or d_in[k].shape != v.shape:
+                d_in[k] = torch.empty(v.shape, dtype=v.dtype, device=dev)
+            d_in[k].copy_(v, non_blocking=True)
+            cp[k] = d_in[k]
+            nbytes += v.numel() * v.element_size()
+        h2d_holder["bytes"] = nbytes
+        step(cp, s)
+        h_lp.copy_(wl.lp, non_blocking=True)
+        h_ch.copy_(wl.choice, non_blocking=True)
 
     with torch.cuda.stream(stream):
         for _ in range(max(3, args.warmup)):
@@ -422,6 +531,8 @@ def jev_arm(args, wl_name):
         t = torch.tensor([e2e_ms], device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         e2e_ms = float(t.item())
+    h2d = h2d_holder.get("bytes", 0)
+    d2h = h_lp.numel() * 4 + h_ch.numel() * 4
 
     # ---- roofline of the dominant kernel
     pk, src = peaks()
@@ -431,7 +542,8 @@ def jev_arm(args, wl_name):
     avg_s = t_ms / 1e3 / max(n_l, 1)
     achieved = work["flops_attn"] / avg_s / 1e12
     peak = float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"]))
-    per_kernel = {k: {"launches": v[0], "avg_us": 1e3 * v[1] / max(v[0], 1), "share": v[1] / sum(x[1] for x in prof.values())}
+    tot_prof = sum(x[1] for x in prof.values()) or 1.0
+    per_kernel = {k: {"launches": v[0], "avg_us": 1e3 * v[1] / max(v[0], 1), "share": v[1] / tot_prof}
                   for k, v in prof.items()}
     step_s = ms / 1e3 / args.steps
     ideal = max((work["flops_attn"] + work["flops_readout"]) / (float(pk["bf16_tflops"]) * 1e12),
@@ -441,18 +553,16 @@ def jev_arm(args, wl_name):
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16" if cfg.dtype == synth.BF16 else "f32", "data": "synthetic",
-        "config": {"workload": synth.WORKLOAD_TEXT[wl_name], "global_batch": cfg.B * world, "seq_len": cfg.Lp,
+        "config": {"workload": synth.WORKLOAD_TEXT[wl_name], "global_batch": wl.B * world, "seq_len": cfg.Lp,
                    "suffix_tokens_per_replica": T, "parallelism": f"replicas{world}" if world > 1 else "single",
-                   "l2": f"inputs rotate over {ncopies} device copies ({ncopies * per_copy / 2**20:.0f} MiB > 2x L2)",
+                   "l2": f"inputs rotate over {ngraph} device copies ({ngraph * per_copy / 2**20:.0f} MiB > 2x L2)",
                    "timing": "CUDA graph replay per step, CUDA events on the launching stream; per-kernel times "
                              "from a second replay of the K steps with event nodes around each kernel",
                    "streams": "readout on a second stream, forked and joined inside each step"},
-        "branches_per_s": world * cfg.B * args.steps / (ms / 1e3),
+        "branches_per_s": world * wl.B * args.steps / (ms / 1e3),
         "clocks": clk,
         "e2e": {"value": world * T * args.steps / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h,
-                "note": "per step: pinned H2D of suffix q/k/v, cu_seqlens, hidden rows, option sets; both C-ABI "
-                        "calls; D2H of log-probs and choices (prefix cache and LM head stay resident)"},
+                "d2h_bytes_per_step": d2h, "note": wl.describe_e2e()},
         "gpu_launches": launches_per_step * args.steps,
         "roofline": {"bound": "tensor", "kernel": attn_name, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": traffic_of(attn_name, wl_name, KERNEL_SRC[attn_name]),
@@ -464,7 +574,8 @@ def jev_arm(args, wl_name):
         "kernels": per_kernel,
         "profiled_pass_ms_per_step": prof_ms / args.steps,
     }
-    if rank == 0 and world == 1 and os.environ.get("JEV_SKIP_CPU_BASELINE") != "1":
+    if rank == 0 and world == 1 and os.environ.get("JEV_SKIP_CPU_BASELINE") != "1" and isinstance(wl, FlatWorkload) \
+            and not isinstance(wl, TreeWorkload):
         del graphs
         budget = float(os.environ.get("JEV_CPU_BASELINE_S", "12"))
         smp = OracleSampler(cfg)
