@@ -359,20 +359,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       u = (long long)sg.w * a.P + sg.ub;
       const int m = sg.m0 + i * kBM + r;
       const bool valid = m < a.M;
-      int t = -1, start = 0, nanc = 0;
-      int2 anc[TREE ? kMaxDepth : 1];
-#pragma unroll
-      for (int kk = 0; kk < (TREE ? kMaxDepth : 1); ++kk) anc[kk] = make_int2(0, 0);
+      int t = -1, start = 0, nanc = 0, node = 0;
       if (valid) {
         t = m / a.G;
         const TokInfo inf = a.info[t];
         start = inf.seg_start;
+        node = inf.node;
         if (TREE) {
-          nanc = a.node_nanc[inf.node];
+          nanc = a.node_nanc[node];
           if (nanc < 0) t = -1;
-#pragma unroll
-          for (int kk = 0; kk < (TREE ? kMaxDepth : 1); ++kk)
-            if (kk < nanc) anc[kk] = a.node_anc[(size_t)inf.node * kMaxDepth + kk];
         }
       }
       float m_run = -CUDART_INF_F, l_run = 0.f;
@@ -398,15 +393,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           // suffix window: same branch up to the row's own token (+ ancestor nodes)
           const int kb = sg.lo + (j - sg.n_pre) * kBN + c_base;
           const int c_lo = start - kb, c_hi = t - kb;
+          if (!TREE || nanc <= 0) {
 #pragma unroll
-          for (int c = 0; c < kHalfCols; ++c) {
-            bool vis = c >= c_lo && c <= c_hi;
-            if (TREE) {
-#pragma unroll
-              for (int kk = 0; kk < (TREE ? kMaxDepth : 1); ++kk)
-                if (kk < nanc) vis |= (c >= anc[kk].x - kb && c < anc[kk].y - kb);
+            for (int c = 0; c < kHalfCols; ++c)
+              if (!(c >= c_lo && c <= c_hi)) xs[c] = kNegInf;
+          } else {
+            // a tree row also sees its ancestors' key ranges (read here, where needed)
+            uint64_t vis = 0;
+            for (int kk = 0; kk < nanc; ++kk) {
+              const int2 rg = a.node_anc[(size_t)node * kMaxDepth + kk];
+              const int lo_c = max(rg.x - kb, 0), hi_c = min(rg.y - kb, kHalfCols);
+              if (hi_c > lo_c) vis |= ((hi_c - lo_c == 64) ? ~0ull : ((1ull << (hi_c - lo_c)) - 1)) << lo_c;
             }
-            if (!vis) xs[c] = kNegInf;
+#pragma unroll
+            for (int c = 0; c < kHalfCols; ++c)
+              if (!((c >= c_lo && c <= c_hi) || ((vis >> c) & 1))) xs[c] = kNegInf;
           }
         }
         float pm[8];

@@ -112,66 +112,66 @@ __device__ __forceinline__ float row_dot(const float* x, const float* w, int H, 
   return acc;
 }
 
-// One block per option set.  Warps take the set's candidates in turn; a
-// candidate's score is the sum over its (row, token) pairs of
-// hidden[row] . lm_head[token], gathered with 16-byte loads (only option rows
-// of the LM head are ever read).  Scores go to shared memory (or, for sets
-// larger than it holds, through `logprob`); warp 0 then forms the set's
-// log-sum-exp and argmax (lowest index on ties) and writes log-probabilities.
-constexpr int kReadWarps = 8;
-constexpr int kReadSmem = 1024;
+// Candidate scores, one warp per candidate over the whole grid: the sum over
+// the candidate's (row, token) pairs of hidden[row] . lm_head[token], gathered
+// with 16-byte loads (only option rows of the LM head are ever read), in pair
+// order.  The score is parked in logprob[c] (NaN for an invalid pair).
+constexpr int kCandWarps = 4;
 
 template <typename T>
-__global__ void __launch_bounds__(kReadWarps * 32) readout_kernel(ReadoutArgs a) {
-  __shared__ float s_z[kReadSmem];
-  const int s = blockIdx.x;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int ca = a.set_offsets[s], ce = a.set_offsets[s + 1];
+__global__ void __launch_bounds__(kCandWarps * 32) readout_cand_kernel(ReadoutArgs a) {
+  const int c = blockIdx.x * kCandWarps + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (c >= a.n_cands) return;
   const T* hid = reinterpret_cast<const T*>(a.hidden);
   const T* W = reinterpret_cast<const T*>(a.lm_head);
-  const bool set_ok = ca >= 0 && ce >= ca && ce <= a.n_cands;
-  const bool in_smem = set_ok && ce - ca <= kReadSmem;
-  if (set_ok) {
-    for (int c = ca + warp; c < ce; c += kReadWarps) {
-      int pa = c, pe = c + 1;
-      if (a.cand_offsets) {
-        pa = a.cand_offsets[c];
-        pe = a.cand_offsets[c + 1];
+  int pa = c, pe = c + 1;
+  if (a.cand_offsets) {
+    pa = a.cand_offsets[c];
+    pe = a.cand_offsets[c + 1];
+  }
+  int set_of_c = 0;
+  if (!a.pair_row) set_of_c = upper_segment(a.set_offsets, a.n_sets, c);  // row = set index
+  float z = 0.f;
+  bool bad = pa < 0 || pe < pa || pe > a.n_pairs;
+  if (!bad) {
+    for (int k = pa; k < pe; ++k) {
+      const int row = a.pair_row ? a.pair_row[k] : set_of_c;
+      const int tok = a.pair_tok[k];
+      if (row < 0 || row >= a.R || tok < 0 || tok >= a.V) {
+        bad = true;
+        continue;
       }
-      float z = 0.f;
-      bool bad = pa < 0 || pe < pa || pe > a.n_pairs;
-      if (!bad) {
-        for (int k = pa; k < pe; ++k) {
-          const int row = a.pair_row ? a.pair_row[k] : s;
-          const int tok = a.pair_tok[k];
-          if (row < 0 || row >= a.R || tok < 0 || tok >= a.V) {
-            bad = true;
-            continue;
-          }
-          z += row_dot(hid + (size_t)row * a.H, W + (size_t)tok * a.H, a.H, lane);
-        }
-      }
-      z = warp_sum(z);
-      if (lane == 0) {
-        const float zz = bad ? CUDART_NAN_F : z;
-        if (in_smem) s_z[c - ca] = zz;
-        else a.logprob[c] = zz;
-        if (a.score) a.score[c] = zz;
-      }
+      z += row_dot(hid + (size_t)row * a.H, W + (size_t)tok * a.H, a.H, lane);
     }
   }
-  __syncthreads();
-  if (warp != 0) return;
-  if (!set_ok || ce == ca) {
+  z = warp_sum(z);
+  if (lane == 0) {
+    const float zz = bad ? CUDART_NAN_F : z;
+    a.logprob[c] = zz;
+    if (a.score) a.score[c] = zz;
+  }
+}
+
+// One warp per option set: log-sum-exp and argmax (lowest index on ties) of
+// the set's scores, written back as log-probabilities.
+constexpr int kSetWarps = 4;
+
+__global__ void __launch_bounds__(kSetWarps * 32) readout_set_kernel(ReadoutArgs a) {
+  pdl_wait();  // the candidate scores come from the previous kernel
+  const int s = blockIdx.x * kSetWarps + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (s >= a.n_sets) return;
+  const int ca = a.set_offsets[s], ce = a.set_offsets[s + 1];
+  if (!(ca >= 0 && ce >= ca && ce <= a.n_cands) || ce == ca) {
     if (lane == 0) a.choice[s] = -1;
     return;
   }
-  auto zc = [&](int c) { return in_smem ? s_z[c - ca] : a.logprob[c]; };
   float mx = -CUDART_INF_F;
   int best = -1;
   bool any_nan = false;
   for (int c = ca + lane; c < ce; c += 32) {
-    const float z = zc(c);
+    const float z = a.logprob[c];
     if (isnan(z)) any_nan = true;
     else if (best < 0 || z > mx) { mx = z; best = c; }
   }
@@ -184,11 +184,11 @@ __global__ void __launch_bounds__(kReadWarps * 32) readout_kernel(ReadoutArgs a)
     if (ob >= 0 && (best < 0 || om > mx || (om == mx && ob < best))) { mx = om; best = ob; }
   }
   float sum = 0.f;
-  for (int c = ca + lane; c < ce; c += 32) sum += exp2f((zc(c) - mx) * 1.4426950408889634f);
+  for (int c = ca + lane; c < ce; c += 32) sum += exp2f((a.logprob[c] - mx) * 1.4426950408889634f);
   sum = warp_sum(sum);
   const float lse = mx + log2f(sum) * 0.69314718055994531f;
   __syncwarp();
-  for (int c = ca + lane; c < ce; c += 32) a.logprob[c] = any_nan ? CUDART_NAN_F : zc(c) - lse;
+  for (int c = ca + lane; c < ce; c += 32) a.logprob[c] = any_nan ? CUDART_NAN_F : a.logprob[c] - lse;
   if (lane == 0) a.choice[s] = any_nan ? -1 : best - ca;
 }
 
@@ -210,9 +210,23 @@ cudaError_t launch_merge(const MergeArgs& a, jev_dtype dt, cudaStream_t s) {
 
 cudaError_t launch_readout(const ReadoutArgs& a, jev_dtype dt, cudaStream_t s) {
   if (a.n_sets == 0) return cudaSuccess;
-  if (dt == JEV_BF16) readout_kernel<__nv_bfloat16><<<a.n_sets, kReadWarps * 32, 0, s>>>(a);
-  else readout_kernel<float><<<a.n_sets, kReadWarps * 32, 0, s>>>(a);
-  return cudaGetLastError();
+  if (a.n_cands > 0) {
+    const int blocks = (a.n_cands + kCandWarps - 1) / kCandWarps;
+    if (dt == JEV_BF16) readout_cand_kernel<__nv_bfloat16><<<blocks, kCandWarps * 32, 0, s>>>(a);
+    else readout_cand_kernel<float><<<blocks, kCandWarps * 32, 0, s>>>(a);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = dim3((a.n_sets + kSetWarps - 1) / kSetWarps);
+  cfg.blockDim = dim3(kSetWarps * 32);
+  cfg.stream = s;
+  cfg.attrs = pdl;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, readout_set_kernel, a);
 }
 
 }  // namespace jev

@@ -41,6 +41,24 @@ __device__ __forceinline__ void store8(float* p, const float (&f)[8]) {
   reinterpret_cast<float4*>(p)[1] = make_float4(f[4], f[5], f[6], f[7]);
 }
 
+// 8 consecutive elements as one raw vector (16 bytes for bf16, 32 for fp32)
+struct F8 { float4 a, b; };
+template <typename T> struct RawVec;
+template <> struct RawVec<__nv_bfloat16> { using type = uint4; };
+template <> struct RawVec<float> { using type = F8; };
+__device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const float2 x = __bfloat1622float2(h[k]);
+    f[2 * k] = x.x;
+    f[2 * k + 1] = x.y;
+  }
+}
+__device__ __forceinline__ void unpack8(const F8& v, float (&f)[8]) {
+  f[0] = v.a.x; f[1] = v.a.y; f[2] = v.a.z; f[3] = v.a.w; f[4] = v.b.x; f[5] = v.b.y; f[6] = v.b.z; f[7] = v.b.w;
+}
+
 constexpr int kTokPerBlock = 8;  // one warp per token
 constexpr int kSmemOffs = 4096;  // segment offsets searched in shared memory up to this many
 
@@ -127,25 +145,52 @@ __global__ void __launch_bounds__(256) rope_pack_kernel(RopePackArgs a) {
   }
   const size_t M = (size_t)a.T * G;
   const int H = a.Hq + a.Hkv;
-#pragma unroll 2
-  for (int hh = hsub; hh < H; hh += heads_per_it) {
-    const T* src;
-    T* dst;
-    if (hh < a.Hq) {
-      src = reinterpret_cast<const T*>(a.q) + ((size_t)t * a.Hq + hh) * a.d;
-      dst = reinterpret_cast<T*>(a.q_rot) + ((size_t)s_grp[hh] * M + (size_t)t * G + s_slot[hh]) * a.d;
-    } else {
-      const int g = hh - a.Hq;
-      src = reinterpret_cast<const T*>(a.k) + ((size_t)t * a.Hkv + g) * a.d;
-      dst = reinterpret_cast<T*>(a.k_rot) + ((size_t)t * a.Hkv + g) * a.d;
+  // every head this lane rotates is loaded before any is used (one memory
+  // round trip per token instead of one per head group); raw 16-byte vectors
+  constexpr int kMaxIt = 8;  // covers Hq + Hkv <= 32 at d = 128 and <= 64 at d = 64
+  using Raw = typename RawVec<T>::type;
+  Raw r0[kMaxIt], r1[kMaxIt];
+#pragma unroll
+  for (int it = 0; it < kMaxIt; ++it) {
+    const int hh = hsub + it * heads_per_it;
+    if (hh < H) {
+      const T* src = hh < a.Hq ? reinterpret_cast<const T*>(a.q) + ((size_t)t * a.Hq + hh) * a.d
+                               : reinterpret_cast<const T*>(a.k) + ((size_t)t * a.Hkv + (hh - a.Hq)) * a.d;
+      r0[it] = *reinterpret_cast<const Raw*>(src + i0);
+      r1[it] = *reinterpret_cast<const Raw*>(src + i0 + half);
     }
-    float x0[8], x1[8], y0[8], y1[8];
-    load8(src + i0, x0);
-    load8(src + i0 + half, x1);
+  }
+#pragma unroll
+  for (int it = 0; it < kMaxIt; ++it) {
+    const int hh = hsub + it * heads_per_it;
+    if (hh < H) {
+      T* dst = hh < a.Hq ? reinterpret_cast<T*>(a.q_rot) + ((size_t)s_grp[hh] * M + (size_t)t * G + s_slot[hh]) * a.d
+                         : reinterpret_cast<T*>(a.k_rot) + ((size_t)t * a.Hkv + (hh - a.Hq)) * a.d;
+      float x0[8], x1[8], y0[8], y1[8];
+      unpack8(r0[it], x0);
+      unpack8(r1[it], x1);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        y0[k] = x0[k] * c8[k] - x1[k] * s8[k];
+        y1[k] = x1[k] * c8[k] + x0[k] * s8[k];
+      }
+      store8(dst + i0, y0);
+      store8(dst + i0 + half, y1);
+    }
+  }
+  // heads beyond kMaxIt iterations (very wide models) take a plain loop
+  for (int hh = hsub + kMaxIt * heads_per_it; hh < H; hh += heads_per_it) {
+    const T* src = hh < a.Hq ? reinterpret_cast<const T*>(a.q) + ((size_t)t * a.Hq + hh) * a.d
+                             : reinterpret_cast<const T*>(a.k) + ((size_t)t * a.Hkv + (hh - a.Hq)) * a.d;
+    T* dst = hh < a.Hq ? reinterpret_cast<T*>(a.q_rot) + ((size_t)s_grp[hh] * M + (size_t)t * G + s_slot[hh]) * a.d
+                       : reinterpret_cast<T*>(a.k_rot) + ((size_t)t * a.Hkv + (hh - a.Hq)) * a.d;
+    float u0[8], u1[8], y0[8], y1[8];
+    load8(src + i0, u0);
+    load8(src + i0 + half, u1);
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
-      y0[k] = x0[k] * c8[k] - x1[k] * s8[k];
-      y1[k] = x1[k] * c8[k] + x0[k] * s8[k];
+      y0[k] = u0[k] * c8[k] - u1[k] * s8[k];
+      y1[k] = u1[k] * c8[k] + u0[k] * s8[k];
     }
     store8(dst + i0, y0);
     store8(dst + i0 + half, y1);
