@@ -18,7 +18,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libjev.so")
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m attention_cascade_b200._build` "
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python attention_cascade_b200/_build.py` "
                       "(nvcc, sm_100a) — there is no non-CUDA fallback")
 
 _lib = C.CDLL(LIB_PATH)
@@ -42,6 +42,12 @@ class jev_attn_desc(C.Structure):
                 ("softmax_scale", C.c_float), ("pos_offset", C.c_int32), ("num_splits", C.c_int32)]
 
 
+class jev_attn_plan(C.Structure):
+    _fields_ = [("kernel", C.c_int32), ("n_tiles", C.c_int32), ("units_per_tile", C.c_int32), ("n_ctas", C.c_int32),
+                ("full_waves", C.c_int32), ("tail0", C.c_int32), ("tail_ctas", C.c_int32), ("split", C.c_int32),
+                ("tail_units", C.c_int64), ("simt_splits", C.c_int32), ("split_len", C.c_int32)]
+
+
 class jev_readout_desc(C.Structure):
     _fields_ = [("n_sets", C.c_int32), ("n_cands", C.c_int32), ("n_pairs", C.c_int32), ("R", C.c_int32),
                 ("H", C.c_int32), ("V", C.c_int32), ("dtype", C.c_int32)]
@@ -51,6 +57,7 @@ _vp, _i32, _sz = C.c_void_p, C.c_int32, C.c_size_t
 _lib.jev_last_error.restype = C.c_char_p
 _lib.jev_prefix_suffix_attn_workspace.argtypes = [C.POINTER(jev_attn_desc)]
 _lib.jev_prefix_suffix_attn_workspace.restype = _sz
+_lib.jev_prefix_suffix_attn_plan.argtypes = [C.POINTER(jev_attn_desc), _i32, _i32, C.POINTER(jev_attn_plan)]
 _lib.jev_prefix_suffix_attn.argtypes = [C.POINTER(jev_attn_desc)] + [_vp] * 10 + [_sz, _vp]
 _lib.jev_candidate_readout.argtypes = [C.POINTER(jev_readout_desc)] + [_vp] * 10
 _lib.jev_tree_build.argtypes = [_i32, _vp, _vp, _i32, _i32, _i32] + [_vp] * 7
@@ -65,8 +72,8 @@ _lib.jev_profile_enable.argtypes = [_i32]
 _lib.jev_profile_read.argtypes = [_i32, C.c_char_p, _vp, _vp, _i32]
 _lib.jev_profile_read.restype = _i32
 _lib.jev_launch_count.restype = C.c_int64
-for _f in ("jev_prefix_suffix_attn", "jev_candidate_readout", "jev_tree_build", "jev_tree_readout_plan",
-           "jev_tree_attn", "jev_rope_inplace", "jev_workspace_init", "jev_check_device_status",
+for _f in ("jev_prefix_suffix_attn", "jev_prefix_suffix_attn_plan", "jev_candidate_readout", "jev_tree_build",
+           "jev_tree_readout_plan", "jev_tree_attn", "jev_rope_inplace", "jev_workspace_init", "jev_check_device_status",
            "jev_profile_enable"):
     getattr(_lib, _f).restype = C.c_int
 
@@ -113,6 +120,14 @@ def make_attn_desc(B, Lp, Hq, Hkv, d, T_total, dtype_code, rope_theta=1e4, softm
 
 def jev_prefix_suffix_attn_workspace(desc: jev_attn_desc) -> int:
     return int(_lib.jev_prefix_suffix_attn_workspace(C.byref(desc)))
+
+
+def jev_prefix_suffix_attn_plan(desc: jev_attn_desc, kernel: int = -1, num_sms: int = 0) -> dict:
+    """The work plan for `desc` as a dict (host only; see include/jev.h)."""
+    p = jev_attn_plan()
+    _check(_lib.jev_prefix_suffix_attn_plan(C.byref(desc), int(kernel), int(num_sms), C.byref(p)),
+           "jev_prefix_suffix_attn_plan")
+    return {f: int(getattr(p, f)) for f, _ in jev_attn_plan._fields_}
 
 
 def new_workspace(nbytes: int, device, stream=None) -> torch.Tensor:

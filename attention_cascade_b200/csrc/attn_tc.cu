@@ -137,14 +137,39 @@ struct Segment {
   int slot;       // partial slot when not complete
 };
 
-// Every role visits the same segments in the same order and derives the same
-// description (the window takes one warp-wide reduction).
-__device__ __forceinline__ Segment make_segment(const AttnArgs& a, int c, long long u, long long u_end, int lane) {
+// A CTA's segments: first its whole tiles (k < full_waves: tile c + k*n_ctas),
+// then its tail units.  Every role visits them in the same order and derives
+// the same description (the window takes one warp-wide reduction).
+struct SegIter {
+  int k;                 // segment index
+  long long u, u_end;    // tail units still to visit
+};
+
+__device__ __forceinline__ bool seg_next(const AttnArgs& a, int c, SegIter& it, int& w, int& ua, int& ub, bool& tail) {
+  if (it.k < a.full_waves) {
+    w = c + it.k * a.n_ctas;
+    ua = 0;
+    ub = a.P;
+    tail = false;
+    return true;
+  }
+  if (it.u >= it.u_end) return false;
+  const int wt = (int)(it.u / a.P);
+  const long long t0 = (long long)wt * a.P;
+  w = a.tail0 + wt;
+  ua = (int)(it.u - t0);
+  ub = (int)(min(it.u_end, t0 + a.P) - t0);
+  tail = true;
+  it.u = t0 + ub;
+  return true;
+}
+
+__device__ __forceinline__ Segment make_segment(const AttnArgs& a, int c, int w, int ua, int ub, bool tail, int lane) {
   Segment sg;
-  sg.w = (int)(u / a.P);
-  const long long t0 = (long long)sg.w * a.P;
-  sg.ua = (int)(u - t0);
-  sg.ub = (int)(min(u_end, t0 + a.P) - t0);
+  sg.w = w;
+  sg.ua = ua;
+  sg.ub = ub;
+  const long long t0 = (long long)(w - a.tail0) * a.P;  // tail unit of the tile's first unit
   sg.g = sg.w / a.n_pairs;
   sg.m0 = (sg.w - sg.g * a.n_pairs) * 2 * kBM;
   sg.n_pre = max(0, min(sg.ub, a.n_pre) - sg.ua);
@@ -158,7 +183,7 @@ __device__ __forceinline__ Segment make_segment(const AttnArgs& a, int c, long l
   }
   sg.n = sg.n_pre + n_suf;
   sg.complete = sg.ua == 0 && sg.ub == a.P;
-  sg.slot = tc_unit_begin(a, c) >= t0 ? 2 * c : 2 * c + 1;
+  sg.slot = (tail && tc_unit_begin(a, c) >= t0) ? 2 * c : 2 * c + 1;
   return sg;
 }
 
@@ -188,7 +213,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int cta = blockIdx.x;
-  const long long u_begin = tc_unit_begin(a, cta), u_end = tc_unit_begin(a, cta + 1);
+  const bool has_tail = a.U > 0 && cta < a.tail_ctas;
+  const long long u_begin = has_tail ? tc_unit_begin(a, cta) : 0, u_end = has_tail ? tc_unit_begin(a, cta + 1) : 0;
 
   if (threadIdx.x == 0) {
     mbar_init(B.q_full, 1);
@@ -227,9 +253,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     int k = 0;
     bool ok = true;
     tma_prefetch_desc(&tm_q);
-    for (long long u = u_begin; ok && u < u_end; ++k) {
-      const Segment sg = make_segment(a, cta, u, u_end, lane);
-      u = (long long)sg.w * a.P + sg.ub;
+    SegIter it{0, u_begin, u_end};
+    int sw, sua, sub;
+    bool stail;
+    for (; ok && seg_next(a, cta, it, sw, sua, sub, stail); ++k, ++it.k) {
+      const Segment sg = make_segment(a, cta, sw, sua, sub, stail, lane);
       if (lane == 0) {
         if (k > 0 && !wait_bar(B.q_empty, (k - 1) & 1, abort, a.status)) ok = false;
         if (ok) {
@@ -284,9 +312,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     long long J = 0;
     int k = 0;
     bool ok = true;
-    for (long long u = u_begin; ok && u < u_end; ++k) {
-      const Segment sg = make_segment(a, cta, u, u_end, lane);
-      u = (long long)sg.w * a.P + sg.ub;
+    SegIter it{0, u_begin, u_end};
+    int sw, sua, sub;
+    bool stail;
+    for (; ok && seg_next(a, cta, it, sw, sua, sub, stail); ++k, ++it.k) {
+      const Segment sg = make_segment(a, cta, sw, sua, sub, stail, lane);
       if (lane == 0) {
         const int n = sg.n;
         ok = wait_bar(B.q_full, k & 1, abort, a.status);
@@ -354,9 +384,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     long long J = 0;
     int k = 0;
     bool ok = true;
-    for (long long u = u_begin; ok && u < u_end; ++k) {
-      const Segment sg = make_segment(a, cta, u, u_end, lane);
-      u = (long long)sg.w * a.P + sg.ub;
+    SegIter it{0, u_begin, u_end};
+    int sw, sua, sub;
+    bool stail;
+    for (; ok && seg_next(a, cta, it, sw, sua, sub, stail); ++k, ++it.k) {
+      const Segment sg = make_segment(a, cta, sw, sua, sub, stail, lane);
       const int m = sg.m0 + i * kBM + r;
       const bool valid = m < a.M;
       int t = -1, start = 0, nanc = 0, node = 0;
@@ -520,99 +552,84 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // Merge the partial segments of every work tile the schedule split.  Block
-// (b, y) looks at the boundary of CTA c = b + 1; if that boundary is the first
-// one strictly inside a tile, the block merges rows [32y, 32y + 32) of that
-// tile — each warp four rows, lanes over columns — from the segments held by
-// consecutive CTAs, with the exact log-sum-exp rule of the split merge.
-constexpr int kMaxSeg = 64;
-constexpr int kFixRows = 32;
+// (w, y) covers rows [8y, 8y + 8) of tail tile w, one row per warp; a tile
+// that one CTA finished is skipped.  The partials were just written and sit
+// in L2, so the merge is latency-bound: lanes read the segments' normalisers
+// side by side (32 at a time), then the partial rows of up to eight segments
+// are in flight together before the exact log-sum-exp rule of the split
+// merge combines them.
+constexpr int kFixRows = 8;
+constexpr int kFixBatch = 8;
 
 template <int D>
 __global__ void __launch_bounds__(256) tc_fixup_kernel(const AttnArgs a) {
-  constexpr int kE = D / 32;  // columns per lane
-  __shared__ int s_slot[kMaxSeg];
-  __shared__ int s_nseg, s_w;
-  const int c = blockIdx.x + 1;
-  if (threadIdx.x == 0) {
-    s_nseg = 0;
-    const long long u = tc_unit_begin(a, c);
-    const int w = (int)(u / a.P);
-    const long long t0 = (long long)w * a.P, t1 = t0 + a.P;
-    if (u % a.P != 0 && !(c >= 2 && tc_unit_begin(a, c - 1) > t0)) {
-      int n = 0;
-      for (int cc = c - 1; cc < a.n_ctas && n < kMaxSeg; ++cc) {
-        const long long ub = tc_unit_begin(a, cc);
-        if (ub >= t1) break;
-        s_slot[n++] = ub >= t0 ? 2 * cc : 2 * cc + 1;
-      }
-      s_nseg = n;
-      s_w = w;
-    }
-  }
-  __syncthreads();
-  const int nseg = s_nseg;
-  if (nseg == 0) return;
-  pdl_wait();  // the partials are written by the attention kernel
-  const int w = s_w;
-  const int g = w / a.n_pairs, m0 = (w - g * a.n_pairs) * 2 * kBM;
+  constexpr int kE = D / 32;  // columns per lane (4 or 2)
+  const int w = a.tail0 + blockIdx.x;  // only tail tiles can be split
+  const long long t0 = (long long)blockIdx.x * a.P;
+  const int c_lo = tc_cta_of(a, t0), c_hi = tc_cta_of(a, t0 + a.P - 1);
+  if (c_lo == c_hi) return;  // one CTA finished this tile and wrote it
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  constexpr int kR = kFixRows / 8;  // rows per warp, merged side by side
-  const int r0 = blockIdx.y * kFixRows + warp * kR;
-  float mx[kR], wsum[kR], acc[kR][kE];
-  // normalisers: lanes read the segments side by side, for every row at once
+  const int r = blockIdx.y * kFixRows + warp;
+  const int g = w / a.n_pairs, m = (w - g * a.n_pairs) * 2 * kBM + r;
+  if (m >= a.M) return;
+  const int nseg = c_hi - c_lo + 1;
+  // CTA c_lo holds this tile as its first segment only if its range starts here
+  const int slot_lo = tc_unit_begin(a, c_lo) >= t0 ? 2 * c_lo : 2 * c_lo + 1;
+  auto row_of = [&](int s) { return (size_t)(s == 0 ? slot_lo : 2 * (c_lo + s)) * 2 * kBM + r; };
+  pdl_wait();  // the partials are written by the attention kernel
+  // the largest normaliser (log2 domain) over all segments
+  float l0 = lane < nseg ? a.l_part[row_of(lane)] : -CUDART_INF_F;
+  float mx = l0;
+  for (int s = lane + 32; s < nseg; s += 32) mx = fmaxf(mx, a.l_part[row_of(s)]);
+  mx = warp_max(mx);
+  float wsum = 0.f, acc[kE];
 #pragma unroll
-  for (int q = 0; q < kR; ++q) {
-    mx[q] = -CUDART_INF_F;
-    for (int s = lane; s < nseg; s += 32) mx[q] = fmaxf(mx[q], a.l_part[(size_t)s_slot[s] * 2 * kBM + r0 + q]);
-  }
+  for (int e = 0; e < kE; ++e) acc[e] = 0.f;
+  if (mx != -CUDART_INF_F) {
+    for (int c0 = 0; c0 < nseg; c0 += 32) {
+      const float lc = c0 == 0 ? l0 : (c0 + lane < nseg ? a.l_part[row_of(c0 + lane)] : -CUDART_INF_F);
+      const float wl = exp2f(lc - mx);  // 0 for absent segments
+      wsum += wl;
+      const int cn = min(32, nseg - c0);
+      for (int b0 = 0; b0 < cn; b0 += kFixBatch) {
+        float ov[kFixBatch][kE];
 #pragma unroll
-  for (int q = 0; q < kR; ++q) {
-    mx[q] = warp_max(mx[q]);
-    wsum[q] = 0.f;
+        for (int i = 0; i < kFixBatch; ++i) {
+          if (b0 + i < cn) {
+            const float* src = a.o_part + row_of(c0 + b0 + i) * D + lane * kE;
+            if constexpr (kE == 4) {
+              const float4 v = *reinterpret_cast<const float4*>(src);
+              ov[i][0] = v.x; ov[i][1] = v.y; ov[i][2] = v.z; ov[i][3] = v.w;
+            } else {
+              const float2 v = *reinterpret_cast<const float2*>(src);
+              ov[i][0] = v.x; ov[i][1] = v.y;
+            }
+          } else {
 #pragma unroll
-    for (int e = 0; e < kE; ++e) acc[q][e] = 0.f;
-  }
-  // weighted sum of the segments' partial rows; loads of all rows are independent
-  for (int s = 0; s < nseg; ++s) {
-    const size_t base = (size_t)s_slot[s] * 2 * kBM + r0;
-    float lv[kR];
-    float4 ov[kR][kE / 4 > 0 ? kE / 4 : 1];
-    float2 ov2[kR];
+            for (int e = 0; e < kE; ++e) ov[i][e] = 0.f;
+          }
+        }
 #pragma unroll
-    for (int q = 0; q < kR; ++q) {
-      lv[q] = a.l_part[base + q];
-      if (kE == 4) ov[q][0] = *reinterpret_cast<const float4*>(a.o_part + (base + q) * D + lane * kE);
-      else ov2[q] = *reinterpret_cast<const float2*>(a.o_part + (base + q) * D + lane * kE);
-    }
+        for (int i = 0; i < kFixBatch; ++i) {
+          const float wi = __shfl_sync(0xffffffffu, wl, (b0 + i) & 31);
 #pragma unroll
-    for (int q = 0; q < kR; ++q) {
-      if (mx[q] == -CUDART_INF_F) continue;
-      const float wgt = exp2f(lv[q] - mx[q]);
-      wsum[q] += wgt;
-      if (kE == 4) {
-        acc[q][0] += wgt * ov[q][0].x;
-        acc[q][1 % kE] += wgt * ov[q][0].y;
-        acc[q][2 % kE] += wgt * ov[q][0].z;
-        acc[q][3 % kE] += wgt * ov[q][0].w;
-      } else {
-        acc[q][0] += wgt * ov2[q].x;
-        acc[q][1 % kE] += wgt * ov2[q].y;
+          for (int e = 0; e < kE; ++e) acc[e] = fmaf(wi, ov[i][e], acc[e]);
+        }
       }
     }
+    wsum = warp_sum(wsum);
   }
-#pragma unroll
-  for (int q = 0; q < kR; ++q) {
-    const int m = m0 + r0 + q;
-    if (m >= a.M) break;
-    const float inv = wsum[q] > 0.f ? 1.f / wsum[q] : 0.f;
-    const int t = m / a.G;
-    const int h = min(max(a.hinv[g * a.G + (m - t * a.G)], 0), a.Hq - 1);
-    __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(a.out) + ((size_t)t * a.Hq + h) * D + lane * kE;
-#pragma unroll
-    for (int e = 0; e < kE; e += 2) *reinterpret_cast<uint32_t*>(o + e) = pack_bf16(acc[q][e] * inv, acc[q][e + 1] * inv);
-    if (a.lse && lane == 0)
-      a.lse[(size_t)t * a.Hq + h] = wsum[q] > 0.f ? (mx[q] + log2f(wsum[q])) * 0.69314718055994531f : -CUDART_INF_F;
+  const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+  const int t = m / a.G;
+  const int h = min(max(a.hinv[g * a.G + (m - t * a.G)], 0), a.Hq - 1);
+  __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(a.out) + ((size_t)t * a.Hq + h) * D + lane * kE;
+  if constexpr (kE == 4) {
+    *reinterpret_cast<uint2*>(o) = make_uint2(pack_bf16(acc[0] * inv, acc[1] * inv), pack_bf16(acc[2] * inv, acc[3] * inv));
+  } else {
+    *reinterpret_cast<uint32_t*>(o) = pack_bf16(acc[0] * inv, acc[1] * inv);
   }
+  if (a.lse && lane == 0)
+    a.lse[(size_t)t * a.Hq + h] = wsum > 0.f ? (mx + log2f(wsum)) * 0.69314718055994531f : -CUDART_INF_F;
 }
 
 __global__ void exp2_selftest_kernel(const float* x, float* y, int n) {
@@ -718,12 +735,12 @@ bool attn_tc_supported(int d) {
 }
 
 cudaError_t launch_tc_fixup(const AttnArgs& a, cudaStream_t s) {
-  if (a.n_ctas < 2) return cudaSuccess;
+  if (a.tail_ctas < 2 || a.n_tiles <= a.tail0) return cudaSuccess;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.gridDim = dim3(a.n_ctas - 1, 2 * kBM / kFixRows);
+  cfg.gridDim = dim3(a.n_tiles - a.tail0, 2 * kBM / kFixRows);
   cfg.blockDim = dim3(256);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = s;

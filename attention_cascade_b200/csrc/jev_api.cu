@@ -3,6 +3,7 @@
 // host-side candidate-prefix trie.
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdarg>
@@ -128,66 +129,109 @@ bool use_tc(const jev_attn_desc* d) {
 
 // Work plan.  Tensor-core kernel: work tiles of 256 stacked rows of one kv
 // group, each with P = ceil(Lp/128) + 1 units (prefix key tiles + the suffix
-// window), spread evenly over n_ctas persistent CTAs (num_splits: 0 -> one CTA
-// per SM, 1 -> one CTA per tile, s -> about s CTAs per tile).  CUDA-core
-// kernel: S prefix splits of split_len keys (a multiple of 128) and a merge.
+// window).  n_ctas persistent CTAs first take full_waves rounds of whole
+// tiles; the remaining tail tiles' units are spread evenly over tail_ctas of
+// them, so a tail tile may be split across CTAs and merged afterwards.
+// num_splits: 1 -> no tile split (one CTA per tile up to one per SM),
+// s > 1 -> every tile spread over about s CTAs, 0 -> the cheapest schedule
+// under a cost model.  CUDA-core kernel: S prefix splits of split_len keys
+// (a multiple of 128) and a merge.
 struct Plan {
   int S, split_len, M, G;
   bool tc, split;
-  int n_pairs, n_tiles, n_pre, P, n_ctas;
+  int n_pairs, n_tiles, n_pre, P, n_ctas, full_waves, tail0, tail_ctas;
   long long U;
 };
-Plan plan_of(const jev_attn_desc* d, int T) {
+
+// Estimated time (microseconds) of the tensor-core schedule: the busiest
+// CTA's units and segments plus the merge of split tiles.  Calibrated on
+// B200 at d = 128: a unit (256 rows x 128 keys) costs about 2.5 us, the
+// first segment of a CTA about 8 us of pipeline fill and drain, each later
+// one about 3 us, a segment left partial about 2 us more (fp32 output), and
+// the merge about 5 us plus 0.7 us per eight segments of one tile.
+double tc_schedule_us(int P, int d, int full_waves, long long U, int tail_ctas) {
+  const double unit_us = 4.0 * 256 * 128 * d / 6.8e12 * 1e6;
+  const double first_us = 8.0, seg_us = 3.0, part_us = 2.0;
+  double worst = 0.0;
+  bool split = false;
+  long long max_tile_segs = 1;
+  for (int c = 0; c < std::max(1, tail_ctas); ++c) {
+    long long units = (long long)full_waves * P, segs = full_waves;
+    bool part = false;
+    if (U > 0 && c < tail_ctas) {
+      const long long u0 = c * U / tail_ctas, u1 = (c + 1) * U / tail_ctas;
+      if (u1 > u0) {
+        units += u1 - u0;
+        segs += (u1 - 1) / P - u0 / P + 1;
+        if (u0 % P || u1 % P) part = split = true;
+      }
+    }
+    if (segs == 0) continue;
+    worst = std::max(worst, first_us + (segs - 1) * seg_us + units * unit_us + (part ? part_us : 0.0));
+  }
+  if (split) {
+    max_tile_segs = (P * (long long)tail_ctas + U - 1) / U + 1;
+    worst += 5.0 + 0.7 * (double)((max_tile_segs + 7) / 8);
+  }
+  return worst;
+}
+
+// kernel: -1 as the device chooses, 0 CUDA-core, 1 tensor-core; sms <= 0: the device's count
+Plan plan_of(const jev_attn_desc* d, int T, int kernel = -1, int sms_hint = 0) {
   Plan p{};
   p.G = d->Hq / d->Hkv;
   p.M = T * p.G;
   const int ktiles = (d->Lp + 127) / 128;
-  p.tc = use_tc(d);
+  p.tc = kernel < 0 ? use_tc(d) : kernel == 1;
   if (p.tc) {
     p.n_pairs = (p.M + 255) / 256;
     p.n_tiles = p.n_pairs * d->Hkv;
     p.n_pre = ktiles;
     p.P = ktiles + 1;
-    p.U = (long long)p.n_tiles * p.P;
     const int s = d->num_splits;
-    long long n;
-    if (s == 1) {
-      n = p.n_tiles;
+    const int sms = std::max(1, sms_hint > 0 ? sms_hint : num_sms());
+    // whole tiles only: full_waves rounds over min(n_tiles, sms) CTAs, the
+    // rest one tile to each of the first tail_ctas CTAs
+    auto no_split = [&] {
+      p.n_ctas = std::max(1, std::min(p.n_tiles, sms));
+      p.full_waves = p.n_tiles / p.n_ctas;
+      p.tail0 = p.full_waves * p.n_ctas;
+      p.tail_ctas = std::max(1, p.n_tiles - p.tail0);
+      p.U = (long long)(p.n_tiles - p.tail0) * p.P;
+    };
+    if (s == 1 || p.n_tiles == 0) {
+      no_split();
     } else if (s > 1) {
-      n = (long long)p.n_tiles * s;
+      const long long U = (long long)p.n_tiles * p.P;
+      p.full_waves = 0;
+      p.tail0 = 0;
+      p.U = U;
+      p.n_ctas = p.tail_ctas = (int)std::max(1LL, std::min((long long)p.n_tiles * s, U));
     } else {
-      // Estimated time of each CTA count up to one per SM: the busiest CTA's
-      // units and segments, plus a merge launch when some tile is split
-      // (a fixed cost and a little per segment).  Times in microseconds.
-      const double unit_us = 4.0 * 256 * 128 * d->d / 6.8e12 * 1e6, seg_us = 3.0, merge_us = 0.5;
-      double best = 1e30;
-      n = 1;
-      const long long n_max = std::min<long long>(num_sms(), p.U);
-      for (long long cand = 1; cand <= n_max; ++cand) {
-        double worst = 0.0;
-        long long max_tile_segs = 1;
-        bool split = false;
-        for (long long c = 0; c < cand; ++c) {
-          const long long u0 = c * p.U / cand, u1 = (c + 1) * p.U / cand;
-          if (u1 <= u0) continue;
-          const long long segs = (u1 - 1) / p.P - u0 / p.P + 1;
-          worst = std::max(worst, (u1 - u0) * unit_us + segs * seg_us);
-          if (u0 % p.P) split = true;
-        }
-        if (split) max_tile_segs = (p.P * cand + p.U - 1) / p.U + 1;
-        const double t = worst + (split ? 6.0 + merge_us * max_tile_segs : 0.0);
-        if (t < best * 0.98) {
-          best = t;
-          n = cand;
+      no_split();
+      double best = tc_schedule_us(p.P, d->d, p.full_waves, p.U, p.tail_ctas);
+      // Spread the tail (every tile when there are fewer tiles than SMs)
+      // over more CTAs, up to one per SM; keep the cheapest estimate.
+      const int fw = p.n_tiles >= sms ? p.n_tiles / sms : 0;
+      const int r = p.n_tiles - fw * sms;
+      const long long U = (long long)r * p.P;
+      // a tile spread over many CTAs costs a long merge; keep it within 64 segments
+      const long long t_max = std::min<long long>({(long long)sms, U, (long long)std::max(1, r) * 64});
+      for (long long t = std::max(1, r); r > 0 && t <= t_max; ++t) {
+        const double e = tc_schedule_us(p.P, d->d, fw, U, (int)t);
+        if (e < best * 0.98) {
+          best = e;
+          p.full_waves = fw;
+          p.tail0 = fw * sms;
+          p.U = U;
+          p.tail_ctas = (int)t;
+          p.n_ctas = fw > 0 ? sms : (int)t;
         }
       }
     }
-    // a tile spread over many CTAs costs a long merge; keep it within 64 segments
-    n = std::min(n, (long long)p.n_tiles * 64);
-    p.n_ctas = (int)std::max(1LL, std::min(n, p.U));
     p.split = false;
-    for (int c = 1; c < p.n_ctas && !p.split; ++c)
-      if (((long long)c * p.U / p.n_ctas) % p.P != 0) p.split = true;
+    for (int c = 1; c < p.tail_ctas && p.U > 0 && !p.split; ++c)
+      if (((long long)c * p.U / p.tail_ctas) % p.P != 0) p.split = true;
     p.S = 1;
     p.split_len = std::max(1, ktiles) * 128;
     return p;
@@ -288,6 +332,7 @@ jev_status attention_core(const jev_attn_desc* d, int T, const Plan& p, const La
   a.S = p.S; a.split_len = p.split_len;
   a.scale_log2 = scale_log2_of(d);
   a.n_pairs = p.n_pairs; a.n_tiles = p.n_tiles; a.n_pre = p.n_pre; a.P = p.P; a.n_ctas = p.n_ctas; a.U = p.U;
+  a.full_waves = p.full_waves; a.tail0 = p.tail0; a.tail_ctas = p.tail_ctas;
   if (p.tc) {
     st = run("attn_tc", s, [&] { return launch_attn_tc(a, s); });
     if (st == JEV_OK && p.split) st = run("tc_fixup", s, [&] { return launch_tc_fixup(a, s); });
@@ -382,6 +427,21 @@ size_t jev_prefix_suffix_attn_workspace(const jev_attn_desc* d) {
   if (check_desc(d) != JEV_OK) return 0;
   Plan p = plan_of(d, d->T_total);
   return layout_of(d, d->T_total, p, 0).total;
+}
+
+jev_status jev_prefix_suffix_attn_plan(const jev_attn_desc* d, int32_t kernel, int32_t sms, jev_attn_plan* out) {
+  if (!out) return fail(JEV_ERR_INVALID_ARG, "plan is NULL");
+  if (kernel < -1 || kernel > 1) return fail(JEV_ERR_INVALID_ARG, "kernel must be -1, 0 or 1");
+  jev_status st = check_desc(d);
+  if (st) return st;
+  const Plan p = plan_of(d, d->T_total, kernel, sms);
+  jev_attn_plan r{};
+  r.kernel = p.tc ? 1 : 0;
+  r.n_tiles = p.n_tiles; r.units_per_tile = p.P; r.n_ctas = p.n_ctas; r.full_waves = p.full_waves;
+  r.tail0 = p.tail0; r.tail_ctas = p.tail_ctas; r.split = p.split ? 1 : 0; r.tail_units = p.U;
+  r.simt_splits = p.S; r.split_len = p.split_len;
+  *out = r;
+  return JEV_OK;
 }
 
 jev_status jev_selftest_exp2(const float* x, float* y, int32_t n, jev_stream_t stream) {

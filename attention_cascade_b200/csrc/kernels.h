@@ -56,16 +56,20 @@ struct AttnArgs {
   int32_t* status;
   int T, M, Lp, Hq, Hkv, G, d, S, split_len;  // split_len: prefix keys per split (multiple of 128)
   float scale_log2;         // softmax scale * log2(e)
-  // tensor-core schedule: work tile w = (kv group w / n_pairs, 256-row pair w % n_pairs)
-  // has P = n_pre + 1 units (one per 128-key prefix tile, one for the suffix
-  // window); CTA c owns units [c*U/n_ctas, (c+1)*U/n_ctas).
-  int n_pairs, n_tiles, n_pre, P, n_ctas;
+  // Tensor-core schedule.  Work tile w = (kv group w / n_pairs, 256-row pair
+  // w % n_pairs) has P = n_pre + 1 units (one per 128-key prefix tile, one for
+  // the suffix window).  The first full_waves * n_ctas tiles go whole, tile
+  // c + k * n_ctas to CTA c; the U units of the remaining (tail) tiles,
+  // counted from tile tail0 = full_waves * n_ctas, are spread evenly over the
+  // first tail_ctas CTAs: CTA c < tail_ctas owns tail units
+  // [c*U/tail_ctas, (c+1)*U/tail_ctas) after its whole tiles.
+  int n_pairs, n_tiles, n_pre, P, n_ctas, full_waves, tail0, tail_ctas;
   long long U;
 };
-// units of the tensor-core schedule owned by CTAs before c
-__host__ __device__ inline long long tc_unit_begin(const AttnArgs& a, int c) { return (long long)c * a.U / a.n_ctas; }
-// CTA owning unit u: the largest c with tc_unit_begin(c) <= u
-__host__ __device__ inline int tc_cta_of(const AttnArgs& a, long long u) { return (int)(((u + 1) * a.n_ctas - 1) / a.U); }
+// tail units owned by CTAs before c (c <= tail_ctas)
+__host__ __device__ inline long long tc_unit_begin(const AttnArgs& a, int c) { return (long long)c * a.U / a.tail_ctas; }
+// CTA owning tail unit u: the largest c with tc_unit_begin(c) <= u
+__host__ __device__ inline int tc_cta_of(const AttnArgs& a, long long u) { return (int)(((u + 1) * a.tail_ctas - 1) / a.U); }
 cudaError_t launch_attn_simt(const AttnArgs& a, jev_dtype dt, cudaStream_t s);
 cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t s);  // bf16, d in {64,128}
 // merge the partial segments of work tiles that the schedule split across CTAs

@@ -394,6 +394,129 @@ def load_lm_head(cfg, dev, torch, tdt):
     return W
 
 
+class Measured:
+    """One workload on this GPU: graphs over rotating input copies, the
+    device-timed loop, and a second pass with per-kernel event nodes."""
+
+    def __init__(self, wl_name, steps, warmup, world, dev, jev, torch, dist, clocks=None):
+        self.cfg = cfg = synth.CONFIGS[wl_name]
+        self.name, self.steps, self.warmup, self.world = wl_name, steps, warmup, world
+        self.jev, self.torch, self.dist, self.dev = jev, torch, dist, dev
+        self.wl = wl = (TreeWorkload if isinstance(cfg, synth.TreeConfig) else FlatWorkload)(cfg, dev, jev, torch)
+        # ---- device copies of the per-step inputs, enough to exceed twice the L2
+        self.per_copy = sum(t.numel() * t.element_size() for t in wl.base.values())
+        self.ncopies = max(2, math.ceil(2 * L2_BYTES / self.per_copy))
+        self.copies = []
+        for i in range(self.ncopies):
+            cp = {k: v.clone() for k, v in wl.base.items()}
+            # each copy reads different option rows of the LM head
+            cp["pair_tok"] = ((wl.base["pair_tok"].long() + 7919 * i) % cfg.V).to(torch.int32)
+            self.copies.append(cp)
+        self.stream = torch.cuda.Stream(device=dev)
+        self.side = torch.cuda.Stream(device=dev)
+        with torch.cuda.stream(self.stream):
+            for i in range(3):
+                self.step(self.copies[i % self.ncopies], self.stream)
+        self.stream.synchronize()
+        self.ngraph = max(1, min(self.ncopies, steps))
+        graphs, self.launches_per_step = self.capture(False)
+        if clocks:
+            clocks.start()
+        self.ms = self.timed_loop(graphs)
+        self.clk = clocks.stop() if clocks else None
+        self.ms = self.max_over_ranks(self.ms)
+        assert jev.jev_check_device_status(wl.ws, self.stream) == 0, "device status flags set during the bench"
+        del graphs
+        # ---- per-kernel durations: the same K steps replayed from graphs whose
+        # kernels are bracketed by CUDA event nodes on the launching stream; each
+        # graph's events hold its last replay, one sample per input copy
+        jev.jev_profile_read()
+        pgraphs, _ = self.capture(True)
+        self.prof_ms = self.timed_loop(pgraphs)
+        self.prof = jev.jev_profile_read()
+        del pgraphs
+
+    def step(self, cp, s):
+        # the readout's inputs (final hidden rows, option ids) do not depend on
+        # this attention layer, so it runs on a second stream, forked and
+        # joined inside the step
+        self.side.wait_stream(s)
+        self.wl.readout(cp, self.side)
+        self.wl.attn(cp, s)
+        s.wait_stream(self.side)
+
+    def capture(self, profiled: bool):
+        torch, jev = self.torch, self.jev
+        jev.jev_profile_enable(profiled)
+        n0 = jev.jev_launch_count()
+        gs = []
+        for cp in self.copies[:self.ngraph]:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=self.stream):
+                self.step(cp, torch.cuda.current_stream())
+            gs.append(g)
+        jev.jev_profile_enable(False)
+        return gs, (jev.jev_launch_count() - n0) // self.ngraph
+
+    def timed_loop(self, gs):
+        torch = self.torch
+        with torch.cuda.stream(self.stream):
+            for i in range(self.warmup):
+                gs[i % self.ngraph].replay()
+        self.stream.synchronize()
+        if self.world > 1:
+            self.dist.barrier()
+        torch.cuda.synchronize()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(self.stream):
+            a0.record(self.stream)
+            for i in range(self.steps):
+                gs[i % self.ngraph].replay()
+            a1.record(self.stream)
+        torch.cuda.synchronize()
+        if self.world > 1:
+            self.dist.barrier()
+        return a0.elapsed_time(a1)
+
+    def max_over_ranks(self, ms):
+        if self.world > 1:
+            t = self.torch.tensor([ms], device=self.dev)
+            self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+            ms = float(t.item())
+        return ms
+
+    def value(self):
+        return self.world * self.wl.T * self.steps / (self.ms / 1e3)
+
+    def summary(self):
+        """Per-kernel times and the roofline of the attention kernel."""
+        pk, src = peaks()
+        prof, work = self.prof, self.wl.work
+        attn_name = "attn_tc" if "attn_tc" in prof else "attn_simt"
+        dom = max(prof.items(), key=lambda kv: kv[1][1])[0] if prof else attn_name
+        n_l, t_ms = prof.get(attn_name, (1, float("nan")))
+        achieved = work["flops_attn"] / (t_ms / 1e3 / max(n_l, 1)) / 1e12
+        peak = float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"]))
+        tot_prof = sum(x[1] for x in prof.values()) or 1.0
+        per_kernel = {k: {"launches": v[0], "avg_us": 1e3 * v[1] / max(v[0], 1), "share": v[1] / tot_prof}
+                      for k, v in prof.items()}
+        step_s = self.ms / 1e3 / self.steps
+        ideal = max((work["flops_attn"] + work["flops_readout"]) / (float(pk["bf16_tflops"]) * 1e12),
+                    (work["bytes_attn"] + work["bytes_readout"]) / (float(pk["hbm_gbs"]) * 1e9))
+        roof = {"bound": "tensor", "kernel": attn_name, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": traffic_of(attn_name, self.name, KERNEL_SRC[attn_name]),
+                "peak_source": f"bf16_tflops_sustained, {src}",
+                "frac_of_burst_peak": achieved / float(pk["bf16_tflops"]),
+                "algorithmic_flops_per_launch": work["flops_attn"], "dominant_kernel_by_time": dom}
+        step_roof = {"ideal_us": ideal * 1e6, "measured_us": step_s * 1e6, "frac": ideal / step_s,
+                     "definition": "max(F / bf16 burst peak, U / HBM peak) over the whole step"}
+        return roof, step_roof, per_kernel
+
+    def free(self):
+        del self.copies, self.wl
+        self.torch.cuda.empty_cache()
+
+
 def jev_arm(args, wl_name):
     import torch
     import torch.distributed as dist
@@ -406,89 +529,8 @@ def jev_arm(args, wl_name):
     if world > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     dev = torch.device("cuda", local)
-    cfg = synth.CONFIGS[wl_name]
-    wl = (TreeWorkload if isinstance(cfg, synth.TreeConfig) else FlatWorkload)(cfg, dev, jev, torch)
-    work, T = wl.work, wl.T
-
-    # ---- device copies of the per-step inputs, enough to exceed twice the L2
-    per_copy = sum(t.numel() * t.element_size() for t in wl.base.values())
-    ncopies = max(2, math.ceil(2 * L2_BYTES / per_copy))
-    copies = []
-    for i in range(ncopies):
-        cp = {k: v.clone() for k, v in wl.base.items()}
-        # each copy reads different option rows of the LM head
-        cp["pair_tok"] = ((wl.base["pair_tok"].long() + 7919 * i) % cfg.V).to(torch.int32)
-        copies.append(cp)
-    stream = torch.cuda.Stream(device=dev)
-    side = torch.cuda.Stream(device=dev)
-
-    def step(cp, s):
-        # the readout's inputs (final hidden rows, option ids) do not depend on
-        # this attention layer, so it runs on a second stream, forked and
-        # joined inside the step
-        side.wait_stream(s)
-        wl.readout(cp, side)
-        wl.attn(cp, s)
-        s.wait_stream(side)
-
-    # ---- graphs: one per input copy (at most one per timed step)
-    with torch.cuda.stream(stream):
-        for i in range(3):
-            step(copies[i % ncopies], stream)
-    stream.synchronize()
-    ngraph = max(1, min(ncopies, args.steps))
-
-    def capture(profiled: bool):
-        jev.jev_profile_enable(profiled)
-        n0 = jev.jev_launch_count()
-        gs = []
-        for cp in copies[:ngraph]:
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=stream):
-                step(cp, torch.cuda.current_stream())
-            gs.append(g)
-        jev.jev_profile_enable(False)
-        return gs, (jev.jev_launch_count() - n0) // ngraph
-
-    graphs, launches_per_step = capture(False)
-
-    def timed_loop(gs):
-        with torch.cuda.stream(stream):
-            for i in range(args.warmup):
-                gs[i % ngraph].replay()
-        stream.synchronize()
-        if world > 1:
-            dist.barrier()
-        torch.cuda.synchronize()
-        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(stream):
-            a0.record(stream)
-            for i in range(args.steps):
-                gs[i % ngraph].replay()
-            a1.record(stream)
-        torch.cuda.synchronize()
-        if world > 1:
-            dist.barrier()
-        return a0.elapsed_time(a1)
-
-    clocks = ClockSampler(local)
-    clocks.start()
-    ms = timed_loop(graphs)
-    clk = clocks.stop()
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    assert jev.jev_check_device_status(wl.ws, stream) == 0, "device status flags set during the bench"
-
-    # ---- per-kernel durations: the same K steps replayed from graphs whose
-    # kernels are bracketed by CUDA event nodes on the launching stream; each
-    # graph's events hold its last replay, one sample per input copy
-    jev.jev_profile_read()
-    pgraphs, _ = capture(True)
-    prof_ms = timed_loop(pgraphs)
-    prof = jev.jev_profile_read()
-    del pgraphs
+    m = Measured(wl_name, args.steps, args.warmup, world, dev, jev, torch, dist, ClockSampler(local))
+    wl, cfg, ms, T = m.wl, m.cfg, m.ms, m.wl.T
 
     # ---- end to end through the public API: pinned host inputs in, results out, every step
     hq = wl.e2e_host()
@@ -509,10 +551,11 @@ def jev_arm(args, wl_name):
             cp[k] = d_in[k]
             nbytes += v.numel() * v.element_size()
         h2d_holder["bytes"] = nbytes
-        step(cp, s)
+        m.step(cp, s)
         h_lp.copy_(wl.lp, non_blocking=True)
         h_ch.copy_(wl.choice, non_blocking=True)
 
+    stream = m.stream
     with torch.cuda.stream(stream):
         for _ in range(max(3, args.warmup)):
             e2e_step(stream)
@@ -526,57 +569,58 @@ def jev_arm(args, wl_name):
             e2e_step(stream)
         f1.record(stream)
     stream.synchronize()
-    e2e_ms = f0.elapsed_time(f1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = m.max_over_ranks(f0.elapsed_time(f1))
     h2d = h2d_holder.get("bytes", 0)
     d2h = h_lp.numel() * 4 + h_ch.numel() * 4
 
-    # ---- roofline of the dominant kernel
-    pk, src = peaks()
-    attn_name = "attn_tc" if "attn_tc" in prof else "attn_simt"
-    dom = max(prof.items(), key=lambda kv: kv[1][1])[0] if prof else attn_name
-    n_l, t_ms = prof.get(attn_name, (1, float("nan")))
-    avg_s = t_ms / 1e3 / max(n_l, 1)
-    achieved = work["flops_attn"] / avg_s / 1e12
-    peak = float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"]))
-    tot_prof = sum(x[1] for x in prof.values()) or 1.0
-    per_kernel = {k: {"launches": v[0], "avg_us": 1e3 * v[1] / max(v[0], 1), "share": v[1] / tot_prof}
-                  for k, v in prof.items()}
-    step_s = ms / 1e3 / args.steps
-    ideal = max((work["flops_attn"] + work["flops_readout"]) / (float(pk["bf16_tflops"]) * 1e12),
-                (work["bytes_attn"] + work["bytes_readout"]) / (float(pk["hbm_gbs"]) * 1e9))
-    value = world * T * args.steps / (ms / 1e3)
+    roof, step_roof, per_kernel = m.summary()
     line = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "metric": METRIC, "value": m.value(), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16" if cfg.dtype == synth.BF16 else "f32", "data": "synthetic",
         "config": {"workload": synth.WORKLOAD_TEXT[wl_name], "global_batch": wl.B * world, "seq_len": cfg.Lp,
                    "suffix_tokens_per_replica": T, "parallelism": f"replicas{world}" if world > 1 else "single",
-                   "l2": f"inputs rotate over {ngraph} device copies ({ngraph * per_copy / 2**20:.0f} MiB > 2x L2)",
+                   "l2": f"inputs rotate over {m.ngraph} device copies ({m.ngraph * m.per_copy / 2**20:.0f} MiB "
+                         "> 2x L2)",
                    "timing": "CUDA graph replay per step, CUDA events on the launching stream; per-kernel times "
                              "from a second replay of the K steps with event nodes around each kernel",
                    "streams": "readout on a second stream, forked and joined inside each step"},
         "branches_per_s": world * wl.B * args.steps / (ms / 1e3),
-        "clocks": clk,
+        "clocks": m.clk,
         "e2e": {"value": world * T * args.steps / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "note": wl.describe_e2e()},
-        "gpu_launches": launches_per_step * args.steps,
-        "roofline": {"bound": "tensor", "kernel": attn_name, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "traffic": traffic_of(attn_name, wl_name, KERNEL_SRC[attn_name]),
-                     "peak_source": f"bf16_tflops_sustained, {src}",
-                     "frac_of_burst_peak": achieved / float(pk["bf16_tflops"]),
-                     "algorithmic_flops_per_launch": work["flops_attn"], "dominant_kernel_by_time": dom},
-        "step_roofline": {"ideal_us": ideal * 1e6, "measured_us": step_s * 1e6, "frac": ideal / step_s,
-                          "definition": "max(F / bf16 burst peak, U / HBM peak) over the whole step"},
+        "gpu_launches": m.launches_per_step * args.steps,
+        "roofline": roof,
+        "step_roofline": step_roof,
         "kernels": per_kernel,
-        "profiled_pass_ms_per_step": prof_ms / args.steps,
+        "profiled_pass_ms_per_step": m.prof_ms / args.steps,
     }
+    m.free()
+    del m
+
+    # ---- the other synthetic configs, same method, fewer steps (one GPU only)
+    if world == 1 and args.per_config:
+        per = {}
+        for name in sorted(synth.CONFIGS):
+            if name == wl_name:
+                continue
+            steps = max(50, min(args.steps, args.per_config_steps))
+            mc = Measured(name, steps, args.warmup, 1, dev, jev, torch, dist)
+            r, sr, pk_ = mc.summary()
+            per[name] = {"workload": synth.WORKLOAD_TEXT[name], "value": mc.value(), "unit": "tokens/s",
+                         "ms_per_step": mc.ms / steps, "steps": steps,
+                         "branches_per_s": mc.wl.B * steps / (mc.ms / 1e3),
+                         "dtype": "bf16" if mc.cfg.dtype == synth.BF16 else "f32",
+                         "roofline": {k: r[k] for k in ("bound", "kernel", "achieved", "peak", "unit", "frac",
+                                                        "traffic", "peak_source")},
+                         "step_roofline_frac": sr["frac"],
+                         "kernels": {k: round(v["avg_us"], 2) for k, v in pk_.items()}}
+            mc.free()
+            del mc
+        line["per_config"] = per
+
     if rank == 0 and world == 1 and os.environ.get("JEV_SKIP_CPU_BASELINE") != "1" and isinstance(wl, FlatWorkload) \
             and not isinstance(wl, TreeWorkload):
-        del graphs
         budget = float(os.environ.get("JEV_CPU_BASELINE_S", "12"))
         smp = OracleSampler(cfg)
         t0 = time.perf_counter()
@@ -597,6 +641,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=200)
     ap.add_argument("--workload", default="c1", choices=sorted(synth.CONFIGS))
     ap.add_argument("--impl", default="jev", choices=["jev", "reference"])
+    ap.add_argument("--no-per-config", dest="per_config", action="store_false",
+                    help="skip the other synthetic configs (reported under per_config on one GPU)")
+    ap.add_argument("--per-config-steps", type=int, default=2000)
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("bench.py: at least 3 warm-up steps")

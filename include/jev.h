@@ -86,6 +86,33 @@ typedef struct {
 size_t jev_prefix_suffix_attn_workspace(const jev_attn_desc* desc);
 
 /*
+ * The work plan jev_prefix_suffix_attn follows for `desc` (host only, no
+ * device work).  kernel: -1 -> the kernel the current device runs, 0 -> the
+ * CUDA-core plan, 1 -> the tensor-core plan (a what-if on any host; only
+ * bf16 with d 64 or 128 on sm_100a runs it).  num_sms <= 0 -> the current
+ * device's SM count (148 when no device is present); num_sms > 0 plans for
+ * that many SMs, as a what-if.  Tensor-core kernel (kernel == 1): stacked query rows of one
+ * kv head form work tiles of 256 rows, n_tiles in all, each of
+ * units_per_tile units (one per 128-key prefix tile plus one for the suffix
+ * window).  n_ctas persistent CTAs first take full_waves rounds of whole
+ * tiles (tile c + k*n_ctas to CTA c); the tail_units units of tiles
+ * tail0 .. n_tiles-1 are spread evenly over CTAs 0 .. tail_ctas-1, CTA c
+ * owning [c*tail_units/tail_ctas, (c+1)*tail_units/tail_ctas); split != 0
+ * when some tile is shared by several CTAs and a merge kernel combines it.
+ * CUDA-core kernel (kernel == 0): simt_splits prefix splits of split_len
+ * keys.  Returns the descriptor's error (as jev_prefix_suffix_attn would) or
+ * JEV_ERR_INVALID_ARG for a NULL `plan` or a kernel outside -1 .. 1.
+ */
+typedef struct {
+  int32_t kernel;          /* 1 tensor-core (bf16, d 64/128, sm_100a), 0 CUDA-core */
+  int32_t n_tiles, units_per_tile, n_ctas, full_waves, tail0, tail_ctas, split;
+  int64_t tail_units;
+  int32_t simt_splits, split_len;
+} jev_attn_plan;
+jev_status jev_prefix_suffix_attn_plan(const jev_attn_desc* desc, int32_t kernel, int32_t num_sms,
+                                      jev_attn_plan* plan);
+
+/*
  * jev_prefix_suffix_attn — one attention layer for B branches over a shared
  * prefix.  For branch b with suffix tokens t = cu_seqlens[b] .. cu_seqlens[b+1]-1
  * (local index j = t - cu_seqlens[b]) and query head h (kv head g = head_map[h]):

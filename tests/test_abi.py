@@ -16,9 +16,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 @pytest.fixture(scope="module")
 def jev():
-    from attention_cascade_b200 import _build
-    _build.build()
-    import attention_cascade_b200 as m
+    import attention_cascade_b200 as m  # built by conftest
     return m
 
 

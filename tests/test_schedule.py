@@ -1,0 +1,119 @@
+"""Host logic of the tensor-core work schedule, checked without a GPU.
+
+The plan comes from the C-ABI plan query; the enumeration below restates how
+each CTA walks its segments (whole tiles first, then its share of the tail
+units) and which partial slot it writes, and how the merge kernel finds the
+segments of a split tile.  Every (tile, unit) must be computed exactly once,
+every split tile merged from exactly the slots its CTAs wrote, and no slot
+may fall outside the workspace's two partial rows per CTA."""
+import itertools
+
+import pytest
+
+import attention_cascade_b200 as jev
+
+
+def _walk(p):
+    n, fw, tail0, tc, U, P = (p[k] for k in ("n_ctas", "full_waves", "tail0", "tail_ctas", "tail_units",
+                                             "units_per_tile"))
+    begin = lambda c: c * U // tc
+    cover, writes = {}, {}
+    for c in range(n):
+        has_tail = U > 0 and c < tc
+        u, u_end = (begin(c), begin(c + 1)) if has_tail else (0, 0)
+        k, slots = 0, []
+        while True:
+            if k < fw:
+                w, ua, ub, tail = c + k * n, 0, P, False
+            elif u < u_end:
+                wt = u // P
+                w, ua, ub, tail = tail0 + wt, u - wt * P, min(u_end, wt * P + P) - wt * P, True
+                u = wt * P + ub
+            else:
+                break
+            assert 0 <= w < p["n_tiles"]
+            for x in range(ua, ub):
+                assert (w, x) not in cover, "unit computed twice"
+                cover[(w, x)] = c
+            if not (ua == 0 and ub == P):
+                slot = 2 * c if begin(c) >= (w - tail0) * P else 2 * c + 1
+                slots.append(slot)
+                writes.setdefault(w, []).append(slot)
+            k += 1
+        assert len(slots) == len(set(slots)) <= 2
+    return cover, writes
+
+
+def _merged(p):
+    tc, U, P, tail0 = p["tail_ctas"], p["tail_units"], p["units_per_tile"], p["tail0"]
+    out = {}
+    if tc < 2 or p["n_tiles"] <= tail0:
+        return out
+    begin = lambda c: c * U // tc
+    cta_of = lambda u: ((u + 1) * tc - 1) // U
+    for bx in range(p["n_tiles"] - tail0):
+        t0 = bx * P
+        lo, hi = cta_of(t0), cta_of(t0 + P - 1)
+        if lo == hi:
+            continue
+        slot_lo = 2 * lo if begin(lo) >= t0 else 2 * lo + 1
+        out[tail0 + bx] = [slot_lo] + [2 * (lo + s) for s in range(1, hi - lo + 1)]
+    return out
+
+
+def _check(p):
+    cover, writes = _walk(p)
+    assert len(cover) == p["n_tiles"] * p["units_per_tile"]
+    merged = _merged(p)
+    assert set(merged) == set(writes)
+    for w, slots in merged.items():
+        assert sorted(slots) == sorted(writes[w])
+        assert max(slots) < 2 * p["n_ctas"]
+    assert bool(p["split"]) == bool(writes)
+
+
+SHAPES = [  # (B, T, Lp, Hq, Hkv)
+    (1, 1, 0, 4, 4), (3, 18, 128, 14, 2), (8, 138, 1024, 12, 2), (32, 700, 2048, 28, 4),
+    (128, 3072, 4096, 28, 4), (5, 333, 300, 8, 1), (64, 1500, 6000, 32, 8), (2, 40000, 128, 8, 8),
+]
+
+
+@pytest.mark.parametrize("shape", SHAPES)
+@pytest.mark.parametrize("num_splits", [0, 1, 2, 3, 7])
+@pytest.mark.parametrize("sms", [148, 132, 7, 1])
+def test_schedule_covers_every_unit_once(shape, num_splits, sms):
+    B, T, Lp, Hq, Hkv = shape
+    desc = jev.make_attn_desc(B, Lp, Hq, Hkv, 128, T, jev.JEV_BF16, num_splits=num_splits)
+    p = jev.jev_prefix_suffix_attn_plan(desc, kernel=1, num_sms=sms)
+    assert p["kernel"] == 1
+    assert p["n_tiles"] == -(-T * (Hq // Hkv) // 256) * Hkv
+    assert p["units_per_tile"] == -(-Lp // 128) + 1
+    if num_splits == 1:
+        assert p["split"] == 0 and p["n_ctas"] <= sms
+    if num_splits in (0, 1):
+        assert p["n_ctas"] <= sms  # persistent: at most one CTA per SM
+    _check(p)
+
+
+def test_auto_schedule_choices():
+    # fewer tiles than SMs and a long prefix: every tile is spread over several CTAs
+    p = jev.jev_prefix_suffix_attn_plan(jev.make_attn_desc(8, 1024, 12, 2, 128, 138, jev.JEV_BF16), 1, 148)
+    assert p["full_waves"] == 0 and p["split"] == 1 and p["n_ctas"] > p["n_tiles"]
+    # 352 tiles on 148 SMs: two whole waves, only the 56 tail tiles are shared
+    p = jev.jev_prefix_suffix_attn_plan(jev.make_attn_desc(128, 4096, 28, 4, 128, 3072, jev.JEV_BF16), 1, 148)
+    assert p["n_tiles"] == 336 or p["n_tiles"] == 352
+    assert p["full_waves"] == 2 and p["tail0"] == 296 and p["n_ctas"] == 148
+    # as many tiles as SMs: one whole tile each, nothing to merge
+    p = jev.jev_prefix_suffix_attn_plan(jev.make_attn_desc(1, 512, 4, 4, 128, 9472, jev.JEV_BF16), 1, 148)
+    assert p["n_tiles"] == 148 and p["split"] == 0 and p["full_waves"] == 1
+
+
+def test_plan_query_rejects_bad_arguments():
+    desc = jev.make_attn_desc(2, 128, 8, 2, 128, 10, jev.JEV_BF16)
+    with pytest.raises(jev.JevError):
+        jev.jev_prefix_suffix_attn_plan(desc, kernel=2)
+    with pytest.raises(jev.JevError):
+        jev.jev_prefix_suffix_attn_plan(jev.make_attn_desc(2, 128, 8, 3, 128, 10, jev.JEV_BF16))
+    # the CUDA-core plan: prefix splits of whole 128-key tiles covering Lp
+    p = jev.jev_prefix_suffix_attn_plan(jev.make_attn_desc(2, 1000, 8, 2, 128, 10, jev.JEV_F32, num_splits=3), 0)
+    assert p["kernel"] == 0 and p["split_len"] % 128 == 0 and p["simt_splits"] * p["split_len"] >= 1000
