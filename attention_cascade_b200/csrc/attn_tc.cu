@@ -71,7 +71,10 @@ struct Cfg {
   static constexpr int kOffBar = kOffV + kNS * kKVBytes;
   static constexpr int kOffX = kOffBar + 256;                     // row-max exchange [tile][parity][half][row]
   static constexpr int kOffL = kOffX + 2 * 2 * 2 * kBM * 4;       // row-sum exchange [tile][half][row]
-  static constexpr int kSmem = kOffL + 2 * 2 * kBM * 4 + 1024;    // + 1024-byte alignment slack
+  static constexpr int kOffStg = kOffL + 2 * 2 * kBM * 4;        // per-warp output staging
+  static constexpr int kStgBytes = 8 * 64;                         // 8 rows x 32 bf16 columns
+  static constexpr int kOffSeg = kOffStg + kSoftWarps * kStgBytes;  // two published segment descriptions
+  static constexpr int kSmem = kOffSeg + 128 + 1024;                   // + 1024-byte alignment slack
   static constexpr int kOCol = 256;                               // first TMEM column of O0
 };
 
@@ -136,6 +139,7 @@ struct Segment {
   bool complete;  // the segment is the whole tile: write the final output
   int slot;       // partial slot when not complete
 };
+static_assert(2 * sizeof(Segment) <= 128, "segment ring");
 
 // A CTA's segments: first its whole tiles (k < full_waves: tile c + k*n_ctas),
 // then its tail units.  Every role visits them in the same order and derives
@@ -199,6 +203,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   Shared* sh = reinterpret_cast<Shared*>(smem + C::kOffBar + 224);
   float* xmax = reinterpret_cast<float*>(smem + C::kOffX);
   float* xsum = reinterpret_cast<float*>(smem + C::kOffL);
+  // The producer derives each segment's description (its key window takes a
+  // warp-wide read of token info) and publishes it here before its arrive on
+  // q_full; the other roles read it after their wait on q_full.  Two slots:
+  // slot k & 1 is rewritten for segment k + 2 only after q_empty of segment
+  // k + 1, by which time every role has read it.
+  Segment* seg_sm = reinterpret_cast<Segment*>(smem + C::kOffSeg);
   const uint32_t bar0 = sbase + C::kOffBar;
   Bars B;
   B.q_full = bar0;
@@ -242,10 +252,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   fence_after_sync();
   const uint32_t tmem = sh->tmem_base;
   volatile int* abort = &sh->abort;
-  // everything above is independent of the previous kernel (the RoPE pack);
-  // its outputs are read only after this wait.  The merge kernel may launch now.
-  pdl_wait();
-  if (threadIdx.x == 0) pdl_trigger();
+  // Everything above is independent of the previous kernel (the RoPE pack);
+  // each role waits for it (pdl_wait) before it reads the pack's outputs:
+  // rotated queries and suffix keys, token info and the head map.
 
   if (warp == kProducerWarp) {
     // ---------------------------------------------------------------- TMA producer
@@ -253,6 +262,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     int k = 0;
     bool ok = true;
     tma_prefetch_desc(&tm_q);
+    // the first segment's leading prefix key tiles need nothing from the pack:
+    // their loads start before the wait
+    int pre0 = 0;
+    {
+      SegIter it0{0, u_begin, u_end};
+      int w0, ua0, ub0;
+      bool tl0;
+      if (seg_next(a, cta, it0, w0, ua0, ub0, tl0)) {
+        pre0 = min(max(0, min(ub0, a.n_pre) - ua0), C::kNS);
+        const int g0 = w0 / a.n_pairs;
+        if (lane == 0)
+          for (int j = 0; j < pre0; ++j) {
+            const uint32_t ks = sbase + C::kOffK + j * C::kKVBytes, vs = sbase + C::kOffV + j * C::kKVBytes;
+            mbar_expect_tx(B.k_full + 8 * j, C::kKVBytes);
+            for (int b = 0; b < D / 64; ++b)
+              tma_load_2d(ks + b * C::kBlk, &tm_kp, g0 * D + b * 64, (ua0 + j) * kBN, B.k_full + 8 * j);
+            mbar_expect_tx(B.v_full + 8 * j, C::kKVBytes);
+            for (int b = 0; b < D / 64; ++b)
+              tma_load_2d(vs + b * C::kBlk, &tm_vp, g0 * D + b * 64, (ua0 + j) * kBN, B.v_full + 8 * j);
+          }
+      }
+    }
+    pdl_wait();
     SegIter it{0, u_begin, u_end};
     int sw, sua, sub;
     bool stail;
@@ -261,12 +293,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) {
         if (k > 0 && !wait_bar(B.q_empty, (k - 1) & 1, abort, a.status)) ok = false;
         if (ok) {
+          seg_sm[k & 1] = sg;
           mbar_expect_tx(B.q_full, 2 * C::kQBytes);
           for (int i = 0; i < 2; ++i)
             for (int b = 0; b < D / 64; ++b)
               tma_load_3d(sbase + i * C::kQBytes + b * C::kBlk, &tm_q, b * 64, sg.m0 + i * kBM, sg.g, B.q_full);
         }
-        for (int j = 0; ok && j < sg.n; ++j) {
+        for (int j = k == 0 ? pre0 : 0; ok && j < sg.n; ++j) {
           const long long JJ = J + j;
           const int st = (int)(JJ % C::kNS);
           const long long use = JJ / C::kNS;
@@ -312,14 +345,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     long long J = 0;
     int k = 0;
     bool ok = true;
+    pdl_wait();
     SegIter it{0, u_begin, u_end};
     int sw, sua, sub;
     bool stail;
     for (; ok && seg_next(a, cta, it, sw, sua, sub, stail); ++k, ++it.k) {
-      const Segment sg = make_segment(a, cta, sw, sua, sub, stail, lane);
+      ok = wait_bar(B.q_full, k & 1, abort, a.status);
+      const Segment sg = seg_sm[k & 1];
       if (lane == 0) {
         const int n = sg.n;
-        ok = wait_bar(B.q_full, k & 1, abort, a.status);
         if (ok && n > 0) {
           const int st0 = (int)(J % C::kNS);
           ok = wait_bar(B.k_full + 8 * st0, (uint32_t)((J / C::kNS) & 1), abort, a.status);
@@ -384,11 +418,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     long long J = 0;
     int k = 0;
     bool ok = true;
+    pdl_wait();
+    // every CTA has passed its wait: the merge kernel may launch now
+    if (threadIdx.x == 0) pdl_trigger();
     SegIter it{0, u_begin, u_end};
     int sw, sua, sub;
     bool stail;
     for (; ok && seg_next(a, cta, it, sw, sua, sub, stail); ++k, ++it.k) {
-      const Segment sg = make_segment(a, cta, sw, sua, sub, stail, lane);
+      if (!wait_bar(B.q_full, k & 1, abort, a.status)) ok = false;
+      const Segment sg = seg_sm[k & 1];
       const int m = sg.m0 + i * kBM + r;
       const bool valid = m < a.M;
       int t = -1, start = 0, nanc = 0, node = 0;
@@ -501,33 +539,59 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool write = ok && valid && t >= 0;
       const int tt = valid ? m / a.G : 0;
       const int h = valid ? min(max(a.hinv[sg.g * a.G + (m - tt * a.G)], 0), a.Hq - 1) : 0;
-      const size_t prow = (size_t)sg.slot * 2 * kBM + i * kBM + r;  // partial row of this thread
+      if (sg.complete) {
+        // bf16 output rows (t, h) lie D*2 bytes apart or more; per 32 columns
+        // a warp stages eight of its half-rows at a time in shared memory so
+        // that each global store writes 64 contiguous bytes of each of 8 rows
+        const unsigned long long dst_row =
+            write ? reinterpret_cast<unsigned long long>(reinterpret_cast<__nv_bfloat16*>(a.out) +
+                                                         ((size_t)tt * a.Hq + h) * D + hf * kHalfD)
+                  : 0ull;
+        uint8_t* stg = smem + C::kOffStg + warp * C::kStgBytes;
+        const int rd_row = lane >> 2, rd_c = lane & 3;  // the 16-byte chunk this lane stores
 #pragma unroll
-      for (int c = 0; c < kHalfD / 32; ++c) {
-        uint32_t uu[32];
-        tmem_ld32(o_addr + c * 32, uu);
-        if (write) {
-          const int col = hf * kHalfD + c * 32;
-          if (sg.complete) {
-            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + ((size_t)tt * a.Hq + h) * D + col);
+        for (int c = 0; c < kHalfD / 32; ++c) {
+          uint32_t uu[32];
+          tmem_ld32(o_addr + c * 32, uu);
+          uint32_t* pk = uu;  // packed in place: entry kk reads entries 2kk, 2kk+1 >= kk
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              uint4 w4;
-              w4.x = pack_bf16(__uint_as_float(uu[8 * v + 0]) * inv, __uint_as_float(uu[8 * v + 1]) * inv);
-              w4.y = pack_bf16(__uint_as_float(uu[8 * v + 2]) * inv, __uint_as_float(uu[8 * v + 3]) * inv);
-              w4.z = pack_bf16(__uint_as_float(uu[8 * v + 4]) * inv, __uint_as_float(uu[8 * v + 5]) * inv);
-              w4.w = pack_bf16(__uint_as_float(uu[8 * v + 6]) * inv, __uint_as_float(uu[8 * v + 7]) * inv);
-              dst[v] = w4;
+          for (int kk = 0; kk < 16; ++kk)
+            pk[kk] = pack_bf16(__uint_as_float(uu[2 * kk]) * inv, __uint_as_float(uu[2 * kk + 1]) * inv);
+#pragma unroll
+          for (int rq = 0; rq < 4; ++rq) {
+            if ((lane >> 3) == rq) {
+              const int rr = lane & 7;
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                *reinterpret_cast<uint4*>(stg + rr * 64 + ((e ^ (rr & 3)) * 16)) =
+                    make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
             }
-          } else {
-            float4* dst = reinterpret_cast<float4*>(a.o_part + prow * D + col);
+            __syncwarp();
+            const uint4 v = *reinterpret_cast<const uint4*>(stg + rd_row * 64 + ((rd_c ^ (rd_row & 3)) * 16));
+            const unsigned long long d = __shfl_sync(0xffffffffu, dst_row, rq * 8 + rd_row);
+            if (d) reinterpret_cast<uint4*>(d)[c * 4 + rd_c] = v;
+            __syncwarp();
+          }
+        }
+      } else {
+        // fp32 partial rows, stored [slot][row / 32][column / 4][row % 32] as
+        // float4 so that a warp's 32 rows fill 512 contiguous bytes per store
+        float4* dst = reinterpret_cast<float4*>(a.o_part) +
+                      ((size_t)(sg.slot * (2 * kBM / 32) + i * (kBM / 32) + q) * (D / 4)) * 32 + lane;
+#pragma unroll
+        for (int c = 0; c < kHalfD / 32; ++c) {
+          uint32_t uu[32];
+          tmem_ld32(o_addr + c * 32, uu);
+          if (write) {
 #pragma unroll
             for (int v = 0; v < 8; ++v)
-              dst[v] = make_float4(__uint_as_float(uu[4 * v]) * inv, __uint_as_float(uu[4 * v + 1]) * inv,
-                                   __uint_as_float(uu[4 * v + 2]) * inv, __uint_as_float(uu[4 * v + 3]) * inv);
+              dst[(size_t)((hf * kHalfD + c * 32) / 4 + v) * 32] =
+                  make_float4(__uint_as_float(uu[4 * v]) * inv, __uint_as_float(uu[4 * v + 1]) * inv,
+                              __uint_as_float(uu[4 * v + 2]) * inv, __uint_as_float(uu[4 * v + 3]) * inv);
           }
         }
       }
+      const size_t prow = (size_t)sg.slot * 2 * kBM + i * kBM + r;  // partial row of this thread
       if (hf == 0) {
         const float lse2 = l_row > 0.f ? m_run + __log2f(l_row) : -CUDART_INF_F;
         if (write) {
@@ -552,83 +616,93 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // Merge the partial segments of every work tile the schedule split.  Block
-// (w, y) covers rows [8y, 8y + 8) of tail tile w, one row per warp; a tile
-// that one CTA finished is skipped.  The partials were just written and sit
-// in L2, so the merge is latency-bound: lanes read the segments' normalisers
-// side by side (32 at a time), then the partial rows of up to eight segments
-// are in flight together before the exact log-sum-exp rule of the split
-// merge combines them.
-constexpr int kFixRows = 8;
-constexpr int kFixBatch = 8;
+// (w, y, z) covers rows [32y, 32y + 32) of tail tile w, one row per lane, and
+// the z-th group of 8 * kCols float4 columns; warp c of the block takes
+// columns c, c + 8, ... of the group, so every load of a partial (stored
+// row-minor in float4 columns) or of a normaliser is one contiguous 512- or
+// 128-byte access.  The partials were just written and sit in L2, so the
+// merge is latency-bound: the normalisers and partial rows of kBatch segments
+// are in flight together, and an online log-sum-exp rescaling folds each
+// batch into the running result (the split merge rule applied
+// incrementally).  Tiles split into few segments take (kCols, kBatch) =
+// (all columns / 8, 4), tiles split into many take half the columns and 8.
+// A tile that one CTA finished is skipped.
+constexpr int kFixRows = 32;
 
-template <int D>
+template <int D, int kCols, int kFixBatch>
 __global__ void __launch_bounds__(256) tc_fixup_kernel(const AttnArgs a) {
-  constexpr int kE = D / 32;  // columns per lane (4 or 2)
   const int w = a.tail0 + blockIdx.x;  // only tail tiles can be split
   const long long t0 = (long long)blockIdx.x * a.P;
   const int c_lo = tc_cta_of(a, t0), c_hi = tc_cta_of(a, t0 + a.P - 1);
   if (c_lo == c_hi) return;  // one CTA finished this tile and wrote it
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int r = blockIdx.y * kFixRows + warp;
+  const int r = blockIdx.y * kFixRows + lane;  // row within the 256-row tile
   const int g = w / a.n_pairs, m = (w - g * a.n_pairs) * 2 * kBM + r;
   if (m >= a.M) return;
   const int nseg = c_hi - c_lo + 1;
   // CTA c_lo holds this tile as its first segment only if its range starts here
   const int slot_lo = tc_unit_begin(a, c_lo) >= t0 ? 2 * c_lo : 2 * c_lo + 1;
-  auto row_of = [&](int s) { return (size_t)(s == 0 ? slot_lo : 2 * (c_lo + s)) * 2 * kBM + r; };
+  auto slot_of = [&](int s) { return s == 0 ? slot_lo : 2 * (c_lo + s); };
+  const int t = m / a.G;
+  const int h = min(max(a.hinv[g * a.G + (m - t * a.G)], 0), a.Hq - 1);  // written before the attention kernel
+  const int c4 = blockIdx.z * 8 * kCols + warp;  // this thread's first float4 column
+  const float4* op = reinterpret_cast<const float4*>(a.o_part) + (size_t)(r >> 5) * (D / 4) * 32 + c4 * 32 + (r & 31);
   pdl_wait();  // the partials are written by the attention kernel
-  // the largest normaliser (log2 domain) over all segments
-  float l0 = lane < nseg ? a.l_part[row_of(lane)] : -CUDART_INF_F;
-  float mx = l0;
-  for (int s = lane + 32; s < nseg; s += 32) mx = fmaxf(mx, a.l_part[row_of(s)]);
-  mx = warp_max(mx);
-  float wsum = 0.f, acc[kE];
+  float mx = -CUDART_INF_F, wsum = 0.f;
+  float4 acc[kCols];
 #pragma unroll
-  for (int e = 0; e < kE; ++e) acc[e] = 0.f;
-  if (mx != -CUDART_INF_F) {
-    for (int c0 = 0; c0 < nseg; c0 += 32) {
-      const float lc = c0 == 0 ? l0 : (c0 + lane < nseg ? a.l_part[row_of(c0 + lane)] : -CUDART_INF_F);
-      const float wl = exp2f(lc - mx);  // 0 for absent segments
-      wsum += wl;
-      const int cn = min(32, nseg - c0);
-      for (int b0 = 0; b0 < cn; b0 += kFixBatch) {
-        float ov[kFixBatch][kE];
+  for (int c = 0; c < kCols; ++c) acc[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s0 = 0; s0 < nseg; s0 += kFixBatch) {
+    float lv[kFixBatch];
+    float4 ov[kFixBatch][kCols];
 #pragma unroll
-        for (int i = 0; i < kFixBatch; ++i) {
-          if (b0 + i < cn) {
-            const float* src = a.o_part + row_of(c0 + b0 + i) * D + lane * kE;
-            if constexpr (kE == 4) {
-              const float4 v = *reinterpret_cast<const float4*>(src);
-              ov[i][0] = v.x; ov[i][1] = v.y; ov[i][2] = v.z; ov[i][3] = v.w;
-            } else {
-              const float2 v = *reinterpret_cast<const float2*>(src);
-              ov[i][0] = v.x; ov[i][1] = v.y;
-            }
-          } else {
+    for (int e = 0; e < kFixBatch; ++e) {
+      lv[e] = -CUDART_INF_F;
+      if (s0 + e < nseg) {
+        const int slot = slot_of(s0 + e);
+        lv[e] = a.l_part[(size_t)slot * 2 * kBM + r];
+        const float4* src = op + (size_t)slot * (2 * kBM / 32) * (D / 4) * 32;
 #pragma unroll
-            for (int e = 0; e < kE; ++e) ov[i][e] = 0.f;
-          }
-        }
+        for (int c = 0; c < kCols; ++c) ov[e][c] = src[c * 8 * 32];
+      } else {
 #pragma unroll
-        for (int i = 0; i < kFixBatch; ++i) {
-          const float wi = __shfl_sync(0xffffffffu, wl, (b0 + i) & 31);
+        for (int c = 0; c < kCols; ++c) ov[e][c] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+    float bm = lv[0];
 #pragma unroll
-          for (int e = 0; e < kE; ++e) acc[e] = fmaf(wi, ov[i][e], acc[e]);
+    for (int e = 1; e < kFixBatch; ++e) bm = fmaxf(bm, lv[e]);
+    const float m_new = fmaxf(mx, bm);
+    if (m_new == -CUDART_INF_F) continue;
+    const float sc = exp2f(mx - m_new);  // 0 while nothing has been folded in
+    wsum *= sc;
+#pragma unroll
+    for (int c = 0; c < kCols; ++c) {
+      acc[c].x *= sc; acc[c].y *= sc; acc[c].z *= sc; acc[c].w *= sc;
+    }
+#pragma unroll
+    for (int e = 0; e < kFixBatch; ++e) {
+      const float we = exp2f(lv[e] - m_new);  // 0 for absent segments; their rows are never read
+      if (we > 0.f) {
+        wsum += we;
+#pragma unroll
+        for (int c = 0; c < kCols; ++c) {
+          acc[c].x = fmaf(we, ov[e][c].x, acc[c].x);
+          acc[c].y = fmaf(we, ov[e][c].y, acc[c].y);
+          acc[c].z = fmaf(we, ov[e][c].z, acc[c].z);
+          acc[c].w = fmaf(we, ov[e][c].w, acc[c].w);
         }
       }
     }
-    wsum = warp_sum(wsum);
+    mx = m_new;
   }
   const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
-  const int t = m / a.G;
-  const int h = min(max(a.hinv[g * a.G + (m - t * a.G)], 0), a.Hq - 1);
-  __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(a.out) + ((size_t)t * a.Hq + h) * D + lane * kE;
-  if constexpr (kE == 4) {
-    *reinterpret_cast<uint2*>(o) = make_uint2(pack_bf16(acc[0] * inv, acc[1] * inv), pack_bf16(acc[2] * inv, acc[3] * inv));
-  } else {
-    *reinterpret_cast<uint32_t*>(o) = pack_bf16(acc[0] * inv, acc[1] * inv);
-  }
-  if (a.lse && lane == 0)
+  __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(a.out) + ((size_t)t * a.Hq + h) * D + c4 * 4;
+#pragma unroll
+  for (int c = 0; c < kCols; ++c)
+    *reinterpret_cast<uint2*>(o + c * 32) =
+        make_uint2(pack_bf16(acc[c].x * inv, acc[c].y * inv), pack_bf16(acc[c].z * inv, acc[c].w * inv));
+  if (a.lse && c4 == 0)
     a.lse[(size_t)t * a.Hq + h] = wsum > 0.f ? (mx + log2f(wsum)) * 0.69314718055994531f : -CUDART_INF_F;
 }
 
@@ -740,14 +814,19 @@ cudaError_t launch_tc_fixup(const AttnArgs& a, cudaStream_t s) {
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.gridDim = dim3(a.n_tiles - a.tail0, 2 * kBM / kFixRows);
+  // the most segments any tail tile is split into
+  const long long max_segs = ((long long)a.P * a.tail_ctas + a.U - 1) / a.U + 1;
+  const bool many = max_segs > 4;
+  const int z = many ? 2 : 1;
+  cfg.gridDim = dim3(a.n_tiles - a.tail0, 2 * kBM / kFixRows, z);
   cfg.blockDim = dim3(256);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (a.d == 128) return cudaLaunchKernelEx(&cfg, tc_fixup_kernel<128>, a);
-  return cudaLaunchKernelEx(&cfg, tc_fixup_kernel<64>, a);
+  if (a.d == 128)
+    return many ? cudaLaunchKernelEx(&cfg, tc_fixup_kernel<128, 2, 8>, a) : cudaLaunchKernelEx(&cfg, tc_fixup_kernel<128, 4, 4>, a);
+  return many ? cudaLaunchKernelEx(&cfg, tc_fixup_kernel<64, 1, 8>, a) : cudaLaunchKernelEx(&cfg, tc_fixup_kernel<64, 2, 4>, a);
 }
 
 cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t s) {

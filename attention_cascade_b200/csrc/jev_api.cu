@@ -302,7 +302,8 @@ float scale_log2_of(const jev_attn_desc* d) {
 jev_status attention_core(const jev_attn_desc* d, int T, const Plan& p, const Layout& L, char* ws,
                           const void* q, const void* k_pre, const void* v_pre, const void* k_suf,
                           const void* v_suf, const int32_t* offs, int n_segs, const int32_t* pos0,
-                          const int32_t* head_map, bool tree, void* out, float* lse, cudaStream_t s) {
+                          const int32_t* head_map, bool tree, const int32_t* tree_parent, void* out, float* lse,
+                          cudaStream_t s) {
   int32_t* status = reinterpret_cast<int32_t*>(ws);
   RopePackArgs r{};
   r.q = q; r.k = k_suf;
@@ -311,6 +312,9 @@ jev_status attention_core(const jev_attn_desc* d, int T, const Plan& p, const La
   r.hinv = reinterpret_cast<int32_t*>(ws + L.hinv);
   r.status = status;
   r.offs = offs; r.pos0 = pos0; r.head_map = head_map;
+  r.parent = tree_parent;
+  r.node_anc = tree ? reinterpret_cast<int2*>(ws + L.anc) : nullptr;
+  r.node_nanc = tree ? reinterpret_cast<int32_t*>(ws + L.nanc) : nullptr;
   r.n_segs = n_segs; r.T = T; r.Hq = d->Hq; r.Hkv = d->Hkv; r.d = d->d;
   r.pos_offset = d->pos_offset >= 0 ? d->pos_offset : d->Lp;
   r.theta = (double)d->rope_theta;
@@ -490,7 +494,7 @@ jev_status jev_prefix_suffix_attn(const jev_attn_desc* d, const void* q, const v
   if (!workspace || ((uintptr_t)workspace & 255)) return fail(JEV_ERR_WORKSPACE, "workspace NULL or not 256-byte aligned");
   if (ws_bytes < L.total) return fail(JEV_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", ws_bytes, L.total);
   return attention_core(d, T, p, L, (char*)workspace, q, k_pre, v_pre, k_suf, v_suf, cu_seqlens, d->B, nullptr,
-                        head_map, false, out, lse, (cudaStream_t)stream);
+                        head_map, false, nullptr, out, lse, (cudaStream_t)stream);
 }
 
 }  // extern "C"
@@ -558,7 +562,7 @@ jev_status jev_prefix_suffix_attn_noalloc(const jev_attn_desc* d, const void* q,
   cudaError_t e = cudaMemsetAsync(scratch, 0, kStatusBytes, s);
   if (e != cudaSuccess) return fail(JEV_ERR_CUDA, "clearing the status word: %s", cudaGetErrorString(e));
   st = attention_core(&dd, T, p, L, (char*)scratch, q, k_pre, v_pre, k_suf, v_suf, cu_seqlens, dd.B, nullptr,
-                      head_map, false, out, lse, s);
+                      head_map, false, nullptr, out, lse, s);
   if (st) return st;
   if (status_flags) {
     e = cudaMemcpyAsync(status_flags, scratch, sizeof(int32_t), cudaMemcpyDeviceToDevice, s);
@@ -586,7 +590,9 @@ jev_status jev_candidate_readout(const jev_readout_desc* d, const void* hidden, 
   if (!pair_row && d->R < d->n_sets) return fail(JEV_ERR_INVALID_ARG, "R < n_sets with pair_row NULL");
   ReadoutArgs a{hidden, lm_head, set_offsets, cand_offsets, pair_row, pair_tok, logprob, choice, score,
                 d->n_sets, d->n_cands, d->n_pairs, d->R, d->H, d->V};
-  return run("readout", (cudaStream_t)stream, [&] { return launch_readout(a, d->dtype, (cudaStream_t)stream); });
+  const jev_status st = run("readout", (cudaStream_t)stream, [&] { return launch_readout(a, d->dtype, (cudaStream_t)stream); });
+  if (st == JEV_OK && d->n_cands > 0) g_launches++;  // candidate scores and set softmax: two kernels
+  return st;
 }
 
 jev_status jev_rope_inplace(void* x, int32_t L, int32_t H, int32_t d, int32_t pos0, float theta, jev_dtype dt,
@@ -701,12 +707,8 @@ jev_status jev_tree_attn(const jev_attn_desc* d, int32_t n_nodes, const int32_t*
   if (!workspace || ((uintptr_t)workspace & 255)) return fail(JEV_ERR_WORKSPACE, "workspace NULL or not 256-byte aligned");
   if (ws_bytes < L.total) return fail(JEV_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", ws_bytes, L.total);
   char* ws = (char*)workspace;
-  TreePlanArgs tp{parent, tok_off, reinterpret_cast<int2*>(ws + L.anc), reinterpret_cast<int32_t*>(ws + L.nanc),
-                  reinterpret_cast<int32_t*>(ws), n_nodes, T};
-  st = run("tree_plan", (cudaStream_t)stream, [&] { return launch_tree_plan(tp, (cudaStream_t)stream); });
-  if (st) return st;
-  return attention_core(d, T, p, L, ws, q, k_root, v_root, k, v, tok_off, n_nodes, pos0, head_map, true, out, lse,
-                        (cudaStream_t)stream);
+  return attention_core(d, T, p, L, ws, q, k_root, v_root, k, v, tok_off, n_nodes, pos0, head_map, true, parent, out,
+                        lse, (cudaStream_t)stream);
 }
 
 }  // extern "C"

@@ -21,22 +21,14 @@ struct RopePackArgs {
   const int32_t* offs;     // flat: cu_seqlens [n_segs+1]; tree: tok_off [n_segs+1]
   const int32_t* pos0;     // tree: [n_segs] first-token positions; flat: nullptr
   const int32_t* head_map; // [Hq] or nullptr
+  const int32_t* parent;   // tree: [n_segs] parent node of each node; flat: nullptr
+  int2* node_anc;          // tree: [n_segs, kMaxDepth] ancestor key ranges (written)
+  int32_t* node_nanc;      // tree: [n_segs] ancestor count, -1 for a malformed chain (written)
   int n_segs, T, Hq, Hkv, d, pos_offset;
   double theta;
   double inv_freq[128];    // theta^(-2i/d), i < d/2, formed on the host in double
 };
 cudaError_t launch_rope_pack(const RopePackArgs& a, jev_dtype dt, cudaStream_t s);
-
-// Per tree node, the packed key ranges of its non-root ancestors (root first).
-struct TreePlanArgs {
-  const int32_t* parent;   // [n_nodes]
-  const int32_t* tok_off;  // [n_nodes+1]
-  int2* node_anc;          // [n_nodes, kMaxDepth]
-  int32_t* node_nanc;      // [n_nodes]
-  int32_t* status;
-  int n_nodes, N;
-};
-cudaError_t launch_tree_plan(const TreePlanArgs& a, cudaStream_t s);
 
 // Attention over [prefix split s ; own suffix window] for the stacked rows of a kv group.
 struct AttnArgs {

@@ -112,10 +112,17 @@ __device__ __forceinline__ float row_dot(const float* x, const float* w, int H, 
   return acc;
 }
 
-// Candidate scores, one warp per candidate over the whole grid: the sum over
-// the candidate's (row, token) pairs of hidden[row] . lm_head[token], gathered
-// with 16-byte loads (only option rows of the LM head are ever read), in pair
-// order.  The score is parked in logprob[c] (NaN for an invalid pair).
+// Candidate scores: the sum over the candidate's (row, token) pairs of
+// hidden[row] . lm_head[token], gathered with 16-byte loads (only option rows
+// of the LM head are ever read).  The score is parked in logprob[c] (NaN for
+// an invalid pair).  Blocks are four warps of few registers, so one fits on
+// an SM beside a CTA of the tensor-core attention kernel (576 threads x 96
+// registers) that may run on another stream; the readout's blocks are kept
+// short so they do not hold back that kernel's CTAs.
+//   one pair per candidate (no candidate offsets): a warp per candidate;
+//   several pairs: a block per candidate, warp w taking pairs w, w + 4, ...,
+//   so the candidate's rows are in flight together; the warps' partial sums
+//   are added in warp order.
 constexpr int kCandWarps = 4;
 
 template <typename T>
@@ -148,6 +155,50 @@ __global__ void __launch_bounds__(kCandWarps * 32) readout_cand_kernel(ReadoutAr
   z = warp_sum(z);
   if (lane == 0) {
     const float zz = bad ? CUDART_NAN_F : z;
+    a.logprob[c] = zz;
+    if (a.score) a.score[c] = zz;
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kCandWarps * 32) readout_cand_block_kernel(ReadoutArgs a) {
+  __shared__ float part[kCandWarps];
+  __shared__ int part_bad[kCandWarps];
+  const int c = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const T* hid = reinterpret_cast<const T*>(a.hidden);
+  const T* W = reinterpret_cast<const T*>(a.lm_head);
+  const int pa = a.cand_offsets[c], pe = a.cand_offsets[c + 1];
+  int set_of_c = 0;
+  if (!a.pair_row) set_of_c = upper_segment(a.set_offsets, a.n_sets, c);  // row = set index
+  float z = 0.f;
+  bool bad = pa < 0 || pe < pa || pe > a.n_pairs;
+  if (!bad) {
+    for (int k = pa + warp; k < pe; k += kCandWarps) {
+      const int row = a.pair_row ? a.pair_row[k] : set_of_c;
+      const int tok = a.pair_tok[k];
+      if (row < 0 || row >= a.R || tok < 0 || tok >= a.V) {
+        bad = true;
+        continue;
+      }
+      z += row_dot(hid + (size_t)row * a.H, W + (size_t)tok * a.H, a.H, lane);
+    }
+  }
+  z = warp_sum(z);
+  if (lane == 0) {
+    part[warp] = z;
+    part_bad[warp] = bad;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float zz = 0.f;
+    bool b = false;
+#pragma unroll
+    for (int q = 0; q < kCandWarps; ++q) {
+      zz += part[q];
+      b |= part_bad[q] != 0;
+    }
+    zz = b ? CUDART_NAN_F : zz;
     a.logprob[c] = zz;
     if (a.score) a.score[c] = zz;
   }
@@ -211,9 +262,14 @@ cudaError_t launch_merge(const MergeArgs& a, jev_dtype dt, cudaStream_t s) {
 cudaError_t launch_readout(const ReadoutArgs& a, jev_dtype dt, cudaStream_t s) {
   if (a.n_sets == 0) return cudaSuccess;
   if (a.n_cands > 0) {
-    const int blocks = (a.n_cands + kCandWarps - 1) / kCandWarps;
-    if (dt == JEV_BF16) readout_cand_kernel<__nv_bfloat16><<<blocks, kCandWarps * 32, 0, s>>>(a);
-    else readout_cand_kernel<float><<<blocks, kCandWarps * 32, 0, s>>>(a);
+    if (a.cand_offsets) {
+      if (dt == JEV_BF16) readout_cand_block_kernel<__nv_bfloat16><<<a.n_cands, kCandWarps * 32, 0, s>>>(a);
+      else readout_cand_block_kernel<float><<<a.n_cands, kCandWarps * 32, 0, s>>>(a);
+    } else {
+      const int blocks = (a.n_cands + kCandWarps - 1) / kCandWarps;
+      if (dt == JEV_BF16) readout_cand_kernel<__nv_bfloat16><<<blocks, kCandWarps * 32, 0, s>>>(a);
+      else readout_cand_kernel<float><<<blocks, kCandWarps * 32, 0, s>>>(a);
+    }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }

@@ -1,5 +1,5 @@
 // rope.cu — RoPE of the suffix (or tree) tokens, group-major query packing,
-// per-token window info, and the tree ancestor plan.
+// per-token window info, and (tree) the ancestor plan of every node.
 //
 // Positions continue from the prefix: branch token j sits at pos_offset + j
 // ("FastJEV: Understanding Redundancy for Compact JEV Inference", TL;DR and
@@ -62,6 +62,40 @@ __device__ __forceinline__ void unpack8(const F8& v, float (&f)[8]) {
 constexpr int kTokPerBlock = 8;  // one warp per token
 constexpr int kSmemOffs = 4096;  // segment offsets searched in shared memory up to this many
 
+// Tree ancestor plan of node n: walk up to the root (parents must precede
+// children, at most kMaxDepth levels) and record the packed key ranges of the
+// node's non-root ancestors, root side first; a malformed chain flags
+// JEV_DEV_BAD_TREE and marks the node's rows to be skipped.
+__device__ void plan_node(const RopePackArgs& a, int n) {
+  const int32_t* tok_off = a.offs;
+  if (n == 0) {
+    if (a.parent[0] != -1 || tok_off[0] != 0 || tok_off[1] != 0 || tok_off[a.n_segs] != a.T)
+      raise_flag(a.status, JEV_DEV_BAD_TREE);
+    a.node_nanc[0] = 0;
+    return;
+  }
+  int chain[kMaxDepth];
+  int depth = 0, cur = n, ok = 1;
+  while (cur > 0) {
+    if (depth >= kMaxDepth) { ok = 0; break; }
+    chain[depth++] = cur;
+    int p = a.parent[cur];
+    if (p < 0 || p >= cur) { ok = 0; break; }
+    if (tok_off[cur + 1] < tok_off[cur] || tok_off[cur] < 0 || tok_off[cur + 1] > a.T) { ok = 0; break; }
+    cur = p;
+  }
+  int2* anc = a.node_anc + (size_t)n * kMaxDepth;
+  if (!ok) {
+    raise_flag(a.status, JEV_DEV_BAD_TREE);
+    a.node_nanc[n] = -1;  // rows of this node are skipped
+    return;
+  }
+  // chain[0] = n itself; ancestors are chain[depth-1] (root side) .. chain[1]
+  int w = 0;
+  for (int k = depth - 1; k >= 1; --k) anc[w++] = make_int2(tok_off[chain[k]], tok_off[chain[k] + 1]);
+  a.node_nanc[n] = w;
+}
+
 // One warp per packed token: find its segment and position, form cos/sin of
 // its angles (double angle, rounded once to float), then rotate all its query
 // and key heads, 8 pair indices per lane per head with 16-byte accesses.
@@ -104,6 +138,9 @@ __global__ void __launch_bounds__(256) rope_pack_kernel(RopePackArgs a) {
     s_slot[h] = slot;
     if (blockIdx.x == 0) a.hinv[g * G + slot] = h;
   }
+  // tree: the ancestor plan of every node (grid-stride over nodes)
+  if (a.parent)
+    for (int n = blockIdx.x * blockDim.x + threadIdx.x; n < a.n_segs; n += gridDim.x * blockDim.x) plan_node(a, n);
   if (blockIdx.x == 0) {
     // offsets must start at 0, never decrease and end at T
     for (int i = threadIdx.x; i < a.n_segs; i += blockDim.x)
@@ -197,39 +234,6 @@ __global__ void __launch_bounds__(256) rope_pack_kernel(RopePackArgs a) {
   }
 }
 
-// One thread per node: walk up to the root (parents must precede children, at
-// most kMaxDepth non-root levels) and record the ancestors' packed key ranges.
-__global__ void tree_plan_kernel(TreePlanArgs a) {
-  int n = blockIdx.x * blockDim.x + threadIdx.x;
-  if (n >= a.n_nodes) return;
-  if (n == 0) {
-    if (a.parent[0] != -1 || a.tok_off[0] != 0 || a.tok_off[1] != 0 || a.tok_off[a.n_nodes] != a.N)
-      raise_flag(a.status, JEV_DEV_BAD_TREE);
-    a.node_nanc[0] = 0;
-    return;
-  }
-  int chain[kMaxDepth];
-  int depth = 0, cur = n, ok = 1;
-  while (cur > 0) {
-    if (depth >= kMaxDepth) { ok = 0; break; }
-    chain[depth++] = cur;
-    int p = a.parent[cur];
-    if (p < 0 || p >= cur) { ok = 0; break; }
-    if (a.tok_off[cur + 1] < a.tok_off[cur] || a.tok_off[cur] < 0 || a.tok_off[cur + 1] > a.N) { ok = 0; break; }
-    cur = p;
-  }
-  int2* anc = a.node_anc + (size_t)n * kMaxDepth;
-  if (!ok) {
-    raise_flag(a.status, JEV_DEV_BAD_TREE);
-    a.node_nanc[n] = -1;  // rows of this node are skipped
-    return;
-  }
-  // chain[0] = n itself; ancestors are chain[depth-1] (root side) .. chain[1]
-  int w = 0;
-  for (int k = depth - 1; k >= 1; --k) anc[w++] = make_int2(a.tok_off[chain[k]], a.tok_off[chain[k] + 1]);
-  a.node_nanc[n] = w;
-}
-
 template <typename T>
 __global__ void rope_inplace_kernel(T* x, int L, int H, int d, int pos0, double theta) {
   int t = blockIdx.x;
@@ -269,11 +273,6 @@ cudaError_t launch_rope_pack(const RopePackArgs& a, jev_dtype dt, cudaStream_t s
   cfg.numAttrs = 1;
   if (dt == JEV_BF16) return cudaLaunchKernelEx(&cfg, rope_pack_kernel<__nv_bfloat16>, a);
   return cudaLaunchKernelEx(&cfg, rope_pack_kernel<float>, a);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_tree_plan(const TreePlanArgs& a, cudaStream_t s) {
-  tree_plan_kernel<<<(a.n_nodes + 127) / 128, 128, 0, s>>>(a);
   return cudaGetLastError();
 }
 
