@@ -90,6 +90,20 @@ struct Shared {
 __device__ __forceinline__ void named_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
+// named barrier that also ANDs a flag over its threads, so that they all
+// leave with the same answer
+__device__ __forceinline__ bool named_sync_and(int id, int count, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred pi, po;\n\t"
+      "setp.ne.u32 pi, %1, 0;\n\t"
+      "bar.red.and.pred po, %2, %3, pi;\n\t"
+      "selp.u32 %0, 1, 0, po;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v), "r"(id), "r"(count)
+      : "memory");
+  return r != 0;
+}
 
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort, int32_t* status) {
   if (mbar_try_wait(bar, parity)) return true;
@@ -441,12 +455,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       float m_run = -CUDART_INF_F, l_run = 0.f;
+      // A wait that fails (a timeout somewhere in the CTA) does not leave the
+      // loop: the thread runs the remaining tiles on whatever TMEM holds, so
+      // that every thread of the tile group meets the same named barriers, and
+      // the group agrees on the outcome at the epilogue's reducing barrier.
       for (int j = 0; j < sg.n; ++j) {
         const long long JJ = J + j;
-        if (!wait_bar(B.s_full + 8 * i, (uint32_t)(JJ & 1), abort, a.status)) {
-          ok = false;
-          break;
-        }
+        if (!wait_bar(B.s_full + 8 * i, (uint32_t)(JJ & 1), abort, a.status)) ok = false;
         fence_after_sync();
         // this half's 64 raw scores; P is later packed in place into xs[0..31]
         uint32_t xs[kHalfCols];
@@ -532,7 +547,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_after_sync();
       // the row's normaliser is the sum of both halves' partial sums
       xsum[(i * 2 + hf) * kBM + r] = l_run;
-      named_sync(bar_id, 256);
+      ok = named_sync_and(bar_id, 256, ok);
       const float l_row = l_run + xsum[(i * 2 + 1 - hf) * kBM + r];
       named_sync(bar_id, 256);  // the exchange slots are free again
       const float inv = l_row > 0.f ? 1.f / l_row : 0.f;

@@ -99,6 +99,8 @@ EDGE = [
     (synth.BF16, 2048, [40] * 12, 28, 4, 128, 5, -1, None),
     (synth.BF16, 384, [1] * 37, 12, 2, 64, 0, -1, None),
     (synth.F32, 200, [70, 1, 15], 4, 2, 128, 2, -1, None),
+    # more branches than the kernel's shared-memory offset table: offsets searched in global memory
+    (synth.BF16, 512, [1, 2] * 550, 8, 2, 64, 0, 700, None),
 ]
 
 
@@ -165,6 +167,19 @@ def test_tree_small_every_element(jev, seed, d):
     lp, ch = run_readout(jev, tc.hidden, dev(tc.W), tc.set_offsets, plan["pair_tok"],
                          cand_offsets=plan["cand_offsets"], pair_row=plan["pair_row"])
     check_readout(lp, ch, ref, cfg.dtype, "tree readout")
+
+
+def test_tree_more_nodes_than_the_shared_table(jev):
+    # ~1200 nodes: the kernel searches node offsets and first positions in global memory
+    cfg = synth.TreeConfig("tn", synth.BF16, 96, 170, 3, 5, 8, 1, 2, 4, 2, 64, 64, 500, seed=11)
+    tc = synth.tree_case(cfg, with_lm_head=False)
+    t, td = _tree_inputs(tc, jev)
+    assert t["n_nodes"] > 1024
+    out, lse = jev.jev_tree_attn(td["parent"], td["tok_off"], td["pos0"], dev(tc.q), dev(tc.k_root), dev(tc.v_root),
+                                 dev(tc.k), dev(tc.v))
+    ref_o, ref_l = oracle.tree_attn(oracle.trie_build(tc.seq_off, tc.toks, cfg.Lp), tc.q, tc.k, tc.v,
+                                    tc.k_root, tc.v_root)
+    check_attn(host_f64(out), host_f64(lse), ref_o, ref_l, cfg.dtype, "tree, many nodes")
 
 
 def test_tree_config_c4(jev):
