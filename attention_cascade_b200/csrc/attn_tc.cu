@@ -277,7 +277,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     tma_prefetch_desc(&tm_q);
     // the first segment's leading prefix key tiles need nothing from the pack:
-    // their loads start before the wait
+    // their loads start before the wait (the pack lets this kernel launch only
+    // once every kernel before it in the stream has completed)
     int pre0 = 0;
     {
       SegIter it0{0, u_begin, u_end};

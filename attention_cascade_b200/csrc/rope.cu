@@ -107,10 +107,13 @@ __global__ void __launch_bounds__(256) rope_pack_kernel(RopePackArgs a) {
   __shared__ float cs[kTokPerBlock][128], sn[kTokPerBlock][128];
   __shared__ int s_slot[256], s_grp[256];
   __shared__ int s_offs[kSmemOffs];
-  // the attention kernel may begin launching now; the previous kernels of the
-  // stream (which read this workspace) must be done before anything is written
-  if (threadIdx.x == 0) pdl_trigger();
+  // The previous kernels of the stream (which may write q, k or the prefix
+  // cache, or read this workspace) must be done before anything is read or
+  // written.  Only then may the attention kernel begin launching: it starts
+  // its prefix K/V loads before its own wait, so everything before this
+  // kernel has to be complete when it launches.
   pdl_wait();
+  if (threadIdx.x == 0) pdl_trigger();
   const bool offs_in_smem = a.n_segs + 1 <= kSmemOffs;
   if (offs_in_smem)
     for (int i = threadIdx.x; i <= a.n_segs; i += blockDim.x) s_offs[i] = a.offs[i];
