@@ -241,7 +241,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const long long u_begin = has_tail ? tc_unit_begin(a, cta) : 0, u_end = has_tail ? tc_unit_begin(a, cta + 1) : 0;
 
   if (threadIdx.x == 0) {
-    mbar_init(B.q_full, 1);
+    mbar_init(B.q_full, 2);  // the producer's expect-tx arrival, then its arrival after publishing the segment
     mbar_init(B.q_empty, 1);
     for (int s = 0; s < C::kNS; ++s) {
       mbar_init(B.k_full + 8 * s, 1);
@@ -304,15 +304,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     int sw, sua, sub;
     bool stail;
     for (; ok && seg_next(a, cta, it, sw, sua, sub, stail); ++k, ++it.k) {
-      const Segment sg = make_segment(a, cta, sw, sua, sub, stail, lane);
+      // The Q tile goes first: it needs only the tile's group and rows.
+      const int qg = sw / a.n_pairs, qm0 = (sw - qg * a.n_pairs) * 2 * kBM;
       if (lane == 0) {
         if (k > 0 && !wait_bar(B.q_empty, (k - 1) & 1, abort, a.status)) ok = false;
         if (ok) {
-          seg_sm[k & 1] = sg;
           mbar_expect_tx(B.q_full, 2 * C::kQBytes);
           for (int i = 0; i < 2; ++i)
             for (int b = 0; b < D / 64; ++b)
-              tma_load_3d(sbase + i * C::kQBytes + b * C::kBlk, &tm_q, b * 64, sg.m0 + i * kBM, sg.g, B.q_full);
+              tma_load_3d(sbase + i * C::kQBytes + b * C::kBlk, &tm_q, b * 64, qm0 + i * kBM, qg, B.q_full);
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      // The description (for the suffix unit, its key window: a warp-wide read
+      // of token info) is published with q_full's second arrival.
+      const Segment sg = make_segment(a, cta, sw, sua, sub, stail, lane);
+      if (lane == 0) {
+        if (ok) {
+          seg_sm[k & 1] = sg;
+          mbar_arrive(B.q_full);
         }
         for (int j = k == 0 ? pre0 : 0; ok && j < sg.n; ++j) {
           const long long JJ = J + j;

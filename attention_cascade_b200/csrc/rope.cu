@@ -114,6 +114,29 @@ __global__ void __launch_bounds__(256) rope_pack_kernel(RopePackArgs a) {
   // kernel has to be complete when it launches.
   pdl_wait();
   if (threadIdx.x == 0) pdl_trigger();
+  // Every head this lane rotates is loaded first, before any table work, so
+  // the token's one memory round trip overlaps the segment search and the
+  // sines and cosines; raw 16-byte vectors.
+  const int t = blockIdx.x * kTokPerBlock + warp;
+  const int lanes_per_head = half / 8;          // 8 (d = 128) or 4 (d = 64)
+  const int heads_per_it = 32 / lanes_per_head;  // 4 or 8
+  const int i0 = (lane % lanes_per_head) * 8, hsub = lane / lanes_per_head;
+  const int H = a.Hq + a.Hkv;
+  constexpr int kMaxIt = 8;  // covers Hq + Hkv <= 32 at d = 128 and <= 64 at d = 64
+  using Raw = typename RawVec<T>::type;
+  Raw r0[kMaxIt], r1[kMaxIt];
+  if (t < a.T) {
+#pragma unroll
+    for (int it = 0; it < kMaxIt; ++it) {
+      const int hh = hsub + it * heads_per_it;
+      if (hh < H) {
+        const T* src = hh < a.Hq ? reinterpret_cast<const T*>(a.q) + ((size_t)t * a.Hq + hh) * a.d
+                                 : reinterpret_cast<const T*>(a.k) + ((size_t)t * a.Hkv + (hh - a.Hq)) * a.d;
+        r0[it] = *reinterpret_cast<const Raw*>(src + i0);
+        r1[it] = *reinterpret_cast<const Raw*>(src + i0 + half);
+      }
+    }
+  }
   const bool offs_in_smem = a.n_segs + 1 <= kSmemOffs;
   if (offs_in_smem)
     for (int i = threadIdx.x; i <= a.n_segs; i += blockDim.x) s_offs[i] = a.offs[i];
@@ -151,7 +174,6 @@ __global__ void __launch_bounds__(256) rope_pack_kernel(RopePackArgs a) {
     if (threadIdx.x == 0 && (a.offs[0] != 0 || a.offs[a.n_segs] != a.T)) raise_flag(a.status, JEV_DEV_BAD_SEQLENS);
   }
   __syncthreads();
-  const int t = blockIdx.x * kTokPerBlock + warp;
   if (t >= a.T) return;
   int seg = 0, start = 0, pos = 0;
   if (lane == 0) {
@@ -174,9 +196,6 @@ __global__ void __launch_bounds__(256) rope_pack_kernel(RopePackArgs a) {
     sn[warp][i] = sf;
   }
   __syncwarp();
-  const int lanes_per_head = half / 8;          // 8 (d = 128) or 4 (d = 64)
-  const int heads_per_it = 32 / lanes_per_head;  // 4 or 8
-  const int i0 = (lane % lanes_per_head) * 8, hsub = lane / lanes_per_head;
   float c8[8], s8[8];
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
@@ -184,22 +203,6 @@ __global__ void __launch_bounds__(256) rope_pack_kernel(RopePackArgs a) {
     s8[k] = sn[warp][i0 + k];
   }
   const size_t M = (size_t)a.T * G;
-  const int H = a.Hq + a.Hkv;
-  // every head this lane rotates is loaded before any is used (one memory
-  // round trip per token instead of one per head group); raw 16-byte vectors
-  constexpr int kMaxIt = 8;  // covers Hq + Hkv <= 32 at d = 128 and <= 64 at d = 64
-  using Raw = typename RawVec<T>::type;
-  Raw r0[kMaxIt], r1[kMaxIt];
-#pragma unroll
-  for (int it = 0; it < kMaxIt; ++it) {
-    const int hh = hsub + it * heads_per_it;
-    if (hh < H) {
-      const T* src = hh < a.Hq ? reinterpret_cast<const T*>(a.q) + ((size_t)t * a.Hq + hh) * a.d
-                               : reinterpret_cast<const T*>(a.k) + ((size_t)t * a.Hkv + (hh - a.Hq)) * a.d;
-      r0[it] = *reinterpret_cast<const Raw*>(src + i0);
-      r1[it] = *reinterpret_cast<const Raw*>(src + i0 + half);
-    }
-  }
 #pragma unroll
   for (int it = 0; it < kMaxIt; ++it) {
     const int hh = hsub + it * heads_per_it;
