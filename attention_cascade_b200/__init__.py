@@ -118,6 +118,19 @@ def make_attn_desc(B, Lp, Hq, Hkv, d, T_total, dtype_code, rope_theta=1e4, softm
                          float(rope_theta), float(softmax_scale), int(pos_offset), int(num_splits))
 
 
+# descriptors of recent calls, reused as they are (the library only reads them)
+_desc_cache: dict = {}
+
+
+def _cached_desc(maker, key):
+    d = _desc_cache.get(key)
+    if d is None:
+        if len(_desc_cache) > 1024:
+            _desc_cache.clear()
+        d = _desc_cache[key] = maker(*key)
+    return d
+
+
 def jev_prefix_suffix_attn_workspace(desc: jev_attn_desc) -> int:
     return int(_lib.jev_prefix_suffix_attn_workspace(C.byref(desc)))
 
@@ -149,17 +162,16 @@ def jev_prefix_suffix_attn(q, k_pre, v_pre, k_suf, v_suf, cu_seqlens, *, head_ma
     _dev(cu_seqlens, "cu_seqlens", torch.int32)
     _dev(head_map, "head_map", torch.int32)
     B = cu_seqlens.numel() - 1
-    desc = make_attn_desc(B, Lp, Hq, Hkv, d, T if T_total is None else T_total, dt, rope_theta, softmax_scale,
-                          pos_offset, num_splits)
+    desc = _cached_desc(make_attn_desc, (B, Lp, Hq, Hkv, d, T if T_total is None else T_total, dt, rope_theta,
+                                         softmax_scale, pos_offset, num_splits))
     if out is None:
         out = torch.empty_like(q)
     if lse is None and want_lse:
         lse = torch.empty((T, Hq), dtype=torch.float32, device=q.device)
     _dev(out, "out", q.dtype)
     _dev(lse, "lse", torch.float32)
-    need = jev_prefix_suffix_attn_workspace(desc)
-    if workspace is None:
-        workspace = new_workspace(need, q.device)
+    if workspace is None:  # (a caller's workspace is size-checked by the library itself)
+        workspace = new_workspace(jev_prefix_suffix_attn_workspace(desc), q.device)
     _check(_lib.jev_prefix_suffix_attn(C.byref(desc), _p(q), _p(k_pre), _p(v_pre), _p(k_suf), _p(v_suf),
                                        _p(cu_seqlens), _p(head_map), _p(out), _p(lse), _p(workspace),
                                        workspace.numel(), _stream(stream)), "jev_prefix_suffix_attn")
@@ -206,7 +218,8 @@ def jev_candidate_readout(hidden, lm_head, set_offsets, pair_tok, *, cand_offset
         _dev(t, n, torch.int32)
     n_sets = set_offsets.numel() - 1
     n_cands = (cand_offsets.numel() - 1) if cand_offsets is not None else pair_tok.numel()
-    desc = jev_readout_desc(n_sets, n_cands, pair_tok.numel(), hidden.shape[0], hidden.shape[1], lm_head.shape[0], dt)
+    desc = _cached_desc(jev_readout_desc, (n_sets, n_cands, pair_tok.numel(), hidden.shape[0], hidden.shape[1],
+                                           lm_head.shape[0], dt))
     if logprob is None:
         logprob = torch.empty(n_cands, dtype=torch.float32, device=hidden.device)
     if choice is None:
@@ -270,14 +283,14 @@ def jev_tree_attn(parent, tok_off, pos0, q, k_root, v_root, k, v, *, head_map=No
     for t, n in ((parent, "parent"), (tok_off, "tok_off"), (pos0, "pos0"), (head_map, "head_map")):
         _dev(t, n, torch.int32)
     n_nodes = parent.numel()
-    desc = make_attn_desc(n_nodes - 1, Lp, Hq, Hkv, d, N, dt, rope_theta, softmax_scale, -1, num_splits)
+    desc = _cached_desc(make_attn_desc, (n_nodes - 1, Lp, Hq, Hkv, d, N, dt, rope_theta, softmax_scale, -1,
+                                         num_splits))
     if out is None:
         out = torch.empty_like(q)
     if lse is None and want_lse:
         lse = torch.empty((N, Hq), dtype=torch.float32, device=q.device)
-    need = jev_tree_attn_workspace(desc, n_nodes)
-    if workspace is None:
-        workspace = new_workspace(need, q.device)
+    if workspace is None:  # (a caller's workspace is size-checked by the library itself)
+        workspace = new_workspace(jev_tree_attn_workspace(desc, n_nodes), q.device)
     _check(_lib.jev_tree_attn(C.byref(desc), n_nodes, _p(parent), _p(tok_off), _p(pos0), _p(q), _p(k_root),
                               _p(v_root), _p(k), _p(v), _p(head_map), _p(out), _p(lse), _p(workspace),
                               workspace.numel(), _stream(stream)), "jev_tree_attn")

@@ -177,7 +177,7 @@ double tc_schedule_us(int P, int d, int full_waves, long long U, int tail_ctas) 
 }
 
 // kernel: -1 as the device chooses, 0 CUDA-core, 1 tensor-core; sms <= 0: the device's count
-Plan plan_of(const jev_attn_desc* d, int T, int kernel = -1, int sms_hint = 0) {
+Plan compute_plan(const jev_attn_desc* d, int T, int kernel, int sms_hint) {
   Plan p{};
   p.G = d->Hq / d->Hkv;
   p.M = T * p.G;
@@ -247,6 +247,42 @@ Plan plan_of(const jev_attn_desc* d, int T, int kernel = -1, int sms_hint = 0) {
   S = std::max(1, std::min(std::min(S, kMaxSplits), std::max(1, ktiles)));
   p.split_len = ktiles > 0 ? ((ktiles + S - 1) / S) * 128 : 128;
   p.S = d->Lp > 0 ? (d->Lp + p.split_len - 1) / p.split_len : 1;
+  return p;
+}
+
+// Plans are cached by the fields they depend on: the tensor-core schedule's
+// cost-model search takes tens to hundreds of microseconds of host time, and
+// every call (and every workspace query) needs the plan.
+Plan plan_of(const jev_attn_desc* d, int T, int kernel = -1, int sms_hint = 0) {
+  struct Key {
+    int T, Lp, Hq, Hkv, d, dtype, num_splits, kernel, sms;
+    bool operator==(const Key& o) const {
+      return T == o.T && Lp == o.Lp && Hq == o.Hq && Hkv == o.Hkv && d == o.d && dtype == o.dtype &&
+             num_splits == o.num_splits && kernel == o.kernel && sms == o.sms;
+    }
+  };
+  struct Hash {
+    size_t operator()(const Key& k) const {
+      size_t h = 1469598103934665603ull;
+      for (int v : {k.T, k.Lp, k.Hq, k.Hkv, k.d, k.dtype, k.num_splits, k.kernel, k.sms})
+        h = (h ^ (size_t)(uint32_t)v) * 1099511628211ull;
+      return h;
+    }
+  };
+  static std::mutex mu;
+  static std::unordered_map<Key, Plan, Hash> cache;
+  const int kern = kernel < 0 ? (use_tc(d) ? 1 : 0) : kernel;
+  const int sms = sms_hint > 0 ? sms_hint : num_sms();
+  const Key key{T, d->Lp, d->Hq, d->Hkv, d->d, (int)d->dtype, d->num_splits, kern, sms};
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    auto it = cache.find(key);
+    if (it != cache.end()) return it->second;
+  }
+  const Plan p = compute_plan(d, T, kern, sms);
+  std::lock_guard<std::mutex> lk(mu);
+  if (cache.size() > 4096) cache.clear();
+  cache.emplace(key, p);
   return p;
 }
 

@@ -99,8 +99,8 @@ EDGE = [
     (synth.BF16, 2048, [40] * 12, 28, 4, 128, 5, -1, None),
     (synth.BF16, 384, [1] * 37, 12, 2, 64, 0, -1, None),
     (synth.F32, 200, [70, 1, 15], 4, 2, 128, 2, -1, None),
-    # more branches than the kernel's shared-memory offset table: offsets searched in global memory
-    (synth.BF16, 512, [1, 2] * 550, 8, 2, 64, 0, 700, None),
+    # more branches than the RoPE pack's shared-memory offset table (4096): offsets searched in global memory
+    (synth.BF16, 512, [1, 2] * 2100, 8, 2, 64, 0, 700, None),
 ]
 
 
@@ -151,9 +151,9 @@ def _tree_inputs(tc, jev):
     return t, dict(parent=dev(t["parent"]), tok_off=dev(t["tok_off"]), pos0=dev(t["pos0"]))
 
 
-@pytest.mark.parametrize("seed,d", [(0, 64), (1, 128)])
-def test_tree_small_every_element(jev, seed, d):
-    cfg = synth.TreeConfig("t", synth.BF16, 300, 5, 9, 2, 6, 1, 5, 8, 2, d, 64, 500, seed=seed)
+@pytest.mark.parametrize("seed,d,dtype", [(0, 64, synth.BF16), (1, 128, synth.BF16), (2, 64, synth.F32)])
+def test_tree_small_every_element(jev, seed, d, dtype):
+    cfg = synth.TreeConfig("t", dtype, 300, 5, 9, 2, 6, 1, 5, 8, 2, d, 64, 500, seed=seed)
     tc = synth.tree_case(cfg, with_lm_head=True)
     t, td = _tree_inputs(tc, jev)
     out, lse = jev.jev_tree_attn(td["parent"], td["tok_off"], td["pos0"], dev(tc.q), dev(tc.k_root), dev(tc.v_root),
@@ -170,11 +170,11 @@ def test_tree_small_every_element(jev, seed, d):
 
 
 def test_tree_more_nodes_than_the_shared_table(jev):
-    # ~1200 nodes: the kernel searches node offsets and first positions in global memory
-    cfg = synth.TreeConfig("tn", synth.BF16, 96, 170, 3, 5, 8, 1, 2, 4, 2, 64, 64, 500, seed=11)
+    # more nodes than the RoPE pack's shared-memory offset table (4096): node offsets searched in global memory
+    cfg = synth.TreeConfig("tn", synth.BF16, 96, 560, 3, 5, 8, 1, 2, 4, 2, 64, 64, 5000, seed=11)
     tc = synth.tree_case(cfg, with_lm_head=False)
     t, td = _tree_inputs(tc, jev)
-    assert t["n_nodes"] > 1024
+    assert t["n_nodes"] > 4096
     out, lse = jev.jev_tree_attn(td["parent"], td["tok_off"], td["pos0"], dev(tc.q), dev(tc.k_root), dev(tc.v_root),
                                  dev(tc.k), dev(tc.v))
     ref_o, ref_l = oracle.tree_attn(oracle.trie_build(tc.seq_off, tc.toks, cfg.Lp), tc.q, tc.k, tc.v,
