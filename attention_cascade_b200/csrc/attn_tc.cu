@@ -434,6 +434,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr int kHalfD = D / 2;       // output columns per thread
     const int i = warp >> 3, hf = (warp >> 2) & 1, q = warp & 3, r = q * 32 + lane;
     const int bar_id = 1 + i;  // named barrier of the 256 threads of tile i
+    // named barrier of the two warps that hold the two halves of the same 32 rows
+    const int pair_bar = 3 + i * 4 + q;
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     const uint32_t s_addr = tmem + i * kBN + hf * kHalfCols + lane_off;       // this half's score columns
     const uint32_t p_addr = tmem + i * kBN + hf * (kHalfCols / 2) + lane_off;  // its packed P columns
@@ -506,38 +508,44 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (!((c >= c_lo && c <= c_hi) || ((vis >> c) & 1))) xs[c] = kNegInf;
           }
         }
+        // this half's maximum with three-input max instructions (8 independent chains)
         float pm[8];
 #pragma unroll
         for (int q8 = 0; q8 < 8; ++q8) pm[q8] = __uint_as_float(xs[q8]);
 #pragma unroll
-        for (int c = 8; c < kHalfCols; ++c) pm[c & 7] = fmaxf(pm[c & 7], __uint_as_float(xs[c]));
-        const float half_max = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
-                                     fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+        for (int c = 8; c < kHalfCols; c += 2)
+          pm[(c >> 1) & 7] = fmax3(pm[(c >> 1) & 7], __uint_as_float(xs[c]), __uint_as_float(xs[c + 1]));
+        const float half_max = fmax3(fmax3(pm[0], pm[1], pm[2]), fmax3(pm[3], pm[4], pm[5]), fmaxf(pm[6], pm[7]));
         // both halves of the row agree on the maximum (double-buffered by tile parity)
         float* xm = xmax + ((i * 2 + (int)(JJ & 1)) * 2) * kBM;
         xm[hf * kBM + r] = half_max;
-        named_sync(bar_id, 256);
+        named_sync(pair_bar, 64);
         const float mx = fmaxf(half_max, xm[(1 - hf) * kBM + r]) * sl2;
         float m_new = m_run;
         if (mx > m_run + kLazy || (m_run == -CUDART_INF_F && mx > -CUDART_INF_F)) m_new = mx;
         const float base = m_new == -CUDART_INF_F ? 0.f : m_new;
         const float alpha = ex2(m_run - base);
-        // p = 2^(s * scale * log2e - max): one FFMA and one exponential per score
-        float ps[8];
+        // p = 2^(s * scale * log2e - max): one exponential per score; the
+        // scale-and-subtract and the row sum run as packed f32x2 operations
+        // (one instruction per pair of scores)
+        const uint64_t sc2 = f2_pack(sl2, sl2), nb2 = f2_pack(-base, -base);
+        uint64_t ps2[4];
 #pragma unroll
-        for (int q8 = 0; q8 < 8; ++q8) ps[q8] = 0.f;
+        for (int q4 = 0; q4 < 4; ++q4) ps2[q4] = 0;
 #pragma unroll
         for (int kk = 0; kk < kHalfCols / 2; ++kk) {
-          const float x0 = fmaf(__uint_as_float(xs[2 * kk]), sl2, -base);
-          const float x1 = fmaf(__uint_as_float(xs[2 * kk + 1]), sl2, -base);
+          const uint64_t x2 = f2_fma(((uint64_t)xs[2 * kk + 1] << 32) | xs[2 * kk], sc2, nb2);
+          const float x0 = f2_lo(x2), x1 = f2_hi(x2);
           const bool fma_pipe = kPolyEvery > 0 && (kk % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1;
           const float p0 = fma_pipe ? exp2_fma(x0) : ex2(x0);
           const float p1 = fma_pipe ? exp2_fma(x1) : ex2(x1);
-          ps[kk & 7] += p0 + p1;
+          ps2[kk & 3] = f2_add(ps2[kk & 3], f2_pack(p0, p1));
           xs[kk] = pack_bf16(p0, p1);
         }
         tmem_st32(p_addr, *reinterpret_cast<const uint32_t(*)[32]>(&xs[0]));
-        const float rs = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+        const uint64_t s01 = f2_add(ps2[0], ps2[1]), s23 = f2_add(ps2[2], ps2[3]);
+        const uint64_t s03 = f2_add(s01, s23);
+        const float rs = f2_lo(s03) + f2_hi(s03);
         l_run = l_run * alpha + rs;
         if (j > 0 && __any_sync(0xffffffffu, m_new != m_run)) {
 #pragma unroll
