@@ -395,6 +395,21 @@ def load_lm_head(cfg, dev, torch, tdt):
     return W
 
 
+def max_over_ranks(ms: float, dist, device, world: int) -> float:
+    """This rank's device-timed milliseconds -> the slowest rank's, on every rank."""
+    if world > 1:
+        import torch
+        t = torch.tensor([ms], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    return ms
+
+
+def job_rate(world: int, units_per_rank_step: float, steps: int, ms: float) -> float:
+    """Whole-job throughput: the units every rank processed over the slowest rank's time."""
+    return world * units_per_rank_step * steps / (ms / 1e3)
+
+
 class Measured:
     """One workload on this GPU: graphs over rotating input copies, the
     device-timed loop, and a second pass with per-kernel event nodes."""
@@ -480,14 +495,10 @@ class Measured:
         return a0.elapsed_time(a1)
 
     def max_over_ranks(self, ms):
-        if self.world > 1:
-            t = self.torch.tensor([ms], device=self.dev)
-            self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
-            ms = float(t.item())
-        return ms
+        return max_over_ranks(ms, self.dist, self.dev, self.world)
 
     def value(self):
-        return self.world * self.wl.T * self.steps / (self.ms / 1e3)
+        return job_rate(self.world, self.wl.T, self.steps, self.ms)
 
     def summary(self):
         """Per-kernel times and the roofline of the attention kernel."""
@@ -605,9 +616,9 @@ def jev_arm(args, wl_name):
                    "timing": "CUDA graph replay per step, CUDA events on the launching stream; per-kernel times "
                              "from a second replay of the K steps with event nodes around each kernel",
                    "streams": "readout on a second stream, forked and joined inside each step"},
-        "branches_per_s": world * wl.B * args.steps / (ms / 1e3),
+        "branches_per_s": job_rate(world, wl.B, args.steps, ms),
         "clocks": m.clk,
-        "e2e": {"value": world * T * args.steps / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+        "e2e": {"value": job_rate(world, T, args.steps, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "note": wl.describe_e2e()},
         "gpu_launches": m.launches_per_step * args.steps,
         "roofline": roof,
