@@ -395,6 +395,102 @@ def load_lm_head(cfg, dev, torch, tdt):
     return W
 
 
+def graph_us(torch, fn, stream, steps: int, warmup: int) -> float:
+    """Average device time of fn() replayed from one CUDA graph, after warm-up."""
+    with torch.cuda.stream(stream):
+        fn()
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        fn()
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            g.replay()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(steps):
+            g.replay()
+        a1.record(stream)
+    torch.cuda.synchronize()
+    return 1e3 * a0.elapsed_time(a1) / steps
+
+
+def diagnostics(dev, jev, torch) -> dict:
+    """Streaming efficiency of the HBM-bound kernels at sizes where it can be
+    measured (the configs move kilobytes to a few megabytes per launch, below
+    launch latency): the readout over 4096 option sets of 9 one-token options
+    at the 7B shape (H = 3584, V = 152064), and the RoPE pack at the wide
+    shape with 1024 branches.  Inputs are synthetic and seeded."""
+    import dataclasses
+    pk, src = peaks()
+    hbm = float(pk["hbm_gbs"])
+    out = {"peak_hbm_GBps": hbm, "peak_source": src}
+    stream = torch.cuda.Stream(device=dev)
+    # ---- readout
+    cfg = synth.CONFIGS["c3"]
+    W = load_lm_head(cfg, dev, torch, torch.bfloat16)
+    n_sets, opts = 4096, 9
+    rng = np.random.default_rng(7)
+    hidden = to_dev(synth.f32_to_bf16_bits(rng.standard_normal((n_sets, cfg.H)).astype(np.float32)), dev, torch)
+    base = rng.integers(0, cfg.V, n_sets)
+    toks = ((base[:, None] + 16411 * np.arange(opts)[None, :]) % cfg.V).astype(np.int32).reshape(-1)
+    so = torch.arange(0, n_sets * opts + 1, opts, dtype=torch.int32, device=dev)
+    pt = torch.from_numpy(toks).to(dev)
+    lp = torch.empty(toks.size, dtype=torch.float32, device=dev)
+    ch = torch.empty(n_sets, dtype=torch.int32, device=dev)
+    us = graph_us(torch, lambda: jev.jev_candidate_readout(hidden, W, so, pt, logprob=lp, choice=ch,
+                                                           stream=torch.cuda.current_stream()), stream, 200, 10)
+    nbytes = (toks.size + n_sets) * cfg.H * 2 + toks.size * 8 + n_sets * 4
+    out["readout"] = {"sets": n_sets, "options": opts, "H": cfg.H, "bytes_per_call": nbytes, "us": us,
+                      "GBps": nbytes / us / 1e3, "frac_of_hbm": nbytes / us / 1e3 / hbm,
+                      "note": "option rows of the LM head gathered from HBM; two kernels (scores, set softmax)"}
+    del W, hidden
+    torch.cuda.empty_cache()
+    # ---- RoPE pack (and the attention call around it) at the wide shape with 1024 branches
+    cw = dataclasses.replace(synth.CONFIGS["c3"], B=1024)
+    c = synth.flat_case(cw, with_lm_head=False)
+    args_ = [to_dev(x, dev, torch) for x in (c.q, c.k_pre, c.v_pre, c.k_suf, c.v_suf)]
+    cu = torch.from_numpy(c.cu_seqlens).to(dev)
+    desc = jev.make_attn_desc(cw.B, cw.Lp, cw.Hq, cw.Hkv, cw.d, c.T, jev.JEV_BF16, cw.theta)
+    ws = jev.new_workspace(jev.jev_prefix_suffix_attn_workspace(desc), dev)
+    o = torch.empty_like(args_[0])
+    lse = torch.empty((c.T, cw.Hq), dtype=torch.float32, device=dev)
+
+    def attn():
+        jev.jev_prefix_suffix_attn(*args_, cu, out=o, lse=lse, workspace=ws, rope_theta=cw.theta,
+                                   stream=torch.cuda.current_stream())
+    graph_us(torch, attn, stream, 3, 2)  # warm-up, no profiling
+    # per-kernel times: one graph with event nodes around each kernel, replayed
+    jev.jev_profile_read()
+    jev.jev_profile_enable(True)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        attn()
+    jev.jev_profile_enable(False)
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            g.replay()
+    torch.cuda.synchronize()
+    prof = jev.jev_profile_read()
+    del g
+    # the pack reads q and k and writes their rotated copies (bf16), plus 16 bytes of token info
+    rbytes = 2 * 2 * c.T * (cw.Hq + cw.Hkv) * cw.d + 16 * c.T
+    n_l, t_ms = prof.get("rope_pack", (1, float("nan")))
+    rus = 1e3 * t_ms / max(n_l, 1)
+    out["rope_pack"] = {"workload": f"wide shape, B=1024 ({c.T} suffix tokens)", "bytes_per_call": rbytes,
+                        "us": rus, "GBps": rbytes / rus / 1e3, "frac_of_hbm": rbytes / rus / 1e3 / hbm,
+                        "note": "per-kernel event time (includes launch latency)"}
+    out["attn_call_us"] = {k: 1e3 * v[1] / max(v[0], 1) for k, v in prof.items()}
+    # the tensor-core kernel at this size: many waves of whole tiles
+    if "attn_tc" in prof:
+        flops = flat_work(c)["flops_attn"]
+        aus = out["attn_call_us"]["attn_tc"]
+        peak = float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"]))
+        out["attn_tc"] = {"workload": out["rope_pack"]["workload"], "flops_per_call": flops, "us": aus,
+                          "TFLOPs": flops / aus / 1e6, "frac_of_sustained_bf16": flops / aus / 1e6 / peak}
+    return out
+
+
 def max_over_ranks(ms: float, dist, device, world: int) -> float:
     """This rank's device-timed milliseconds -> the slowest rank's, on every rank."""
     if world > 1:
@@ -442,6 +538,18 @@ class Measured:
         self.clk = clocks.stop() if clocks else None
         self.ms = self.max_over_ranks(self.ms)
         assert jev.jev_check_device_status(wl.ws, self.stream) == 0, "device status flags set during the bench"
+        # per-step spread: up to 500 more steps, each between its own pair of events
+        n = min(steps, 500)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+        with torch.cuda.stream(self.stream):
+            for i, (e0, e1) in enumerate(evs):
+                e0.record(self.stream)
+                graphs[i % self.ngraph].replay()
+                e1.record(self.stream)
+        torch.cuda.synchronize()
+        per = sorted(1e3 * e0.elapsed_time(e1) for e0, e1 in evs)
+        self.pct = {"p10": per[n // 10], "p50": per[n // 2], "p90": per[(9 * n) // 10], "steps": n,
+                    "note": "each step between its own pair of events, which adds a few microseconds"}
         del graphs
         # ---- per-kernel durations: the same K steps replayed from graphs whose
         # kernels are bracketed by CUDA event nodes on the launching stream; each
@@ -608,6 +716,7 @@ def jev_arm(args, wl_name):
     line = {
         "metric": METRIC, "value": m.value(), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "step_us_spread": m.pct,
         "vs_baseline": None, "dtype": "bf16" if cfg.dtype == synth.BF16 else "f32", "data": "synthetic",
         "config": {"workload": synth.WORKLOAD_TEXT[wl_name], "global_batch": wl.B * world, "seq_len": cfg.Lp,
                    "suffix_tokens_per_replica": T, "parallelism": f"replicas{world}" if world > 1 else "single",
@@ -649,6 +758,8 @@ def jev_arm(args, wl_name):
             mc.free()
             del mc
         line["per_config"] = per
+        if args.diagnostics:
+            line["diagnostics"] = diagnostics(dev, jev, torch)
 
     if rank == 0 and world == 1 and os.environ.get("JEV_SKIP_CPU_BASELINE") != "1" and isinstance(wl, FlatWorkload) \
             and not isinstance(wl, TreeWorkload):
@@ -675,6 +786,8 @@ def main():
     ap.add_argument("--no-per-config", dest="per_config", action="store_false",
                     help="skip the other synthetic configs (reported under per_config on one GPU)")
     ap.add_argument("--per-config-steps", type=int, default=2000)
+    ap.add_argument("--no-diagnostics", dest="diagnostics", action="store_false",
+                    help="skip the streaming diagnostics at larger sizes (one GPU, with per_config)")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("bench.py: at least 3 warm-up steps")
