@@ -1,6 +1,8 @@
 // merge_readout.cu — log-sum-exp merge of split partials, and candidate readout.
 #include <math_constants.h>
 
+#include <algorithm>
+
 #include "kernels.h"
 
 namespace jev {
@@ -124,6 +126,7 @@ __device__ __forceinline__ float row_dot(const float* x, const float* w, int H, 
 //   so the candidate's rows are in flight together; the warps' partial sums
 //   are added in warp order.
 constexpr int kCandWarps = 4;
+constexpr int kWideCands = 16384;  // from this many one-pair candidates on, the wide kernel
 
 template <typename T>
 __global__ void __launch_bounds__(kCandWarps * 32) readout_cand_kernel(ReadoutArgs a) {
@@ -150,6 +153,51 @@ __global__ void __launch_bounds__(kCandWarps * 32) readout_cand_kernel(ReadoutAr
         continue;
       }
       z += row_dot(hid + (size_t)row * a.H, W + (size_t)tok * a.H, a.H, lane);
+    }
+  }
+  z = warp_sum(z);
+  if (lane == 0) {
+    const float zz = bad ? CUDART_NAN_F : z;
+    a.logprob[c] = zz;
+    if (a.score) a.score[c] = zz;
+  }
+}
+
+// Large one-pair readouts (many candidates, nothing else competing for the
+// SMs): a warp per candidate as above, but every 16-byte load of the two rows
+// is issued before any is used (ordered asm loads), W row first.
+__device__ __forceinline__ uint4 ld_row16(const uint4* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+  return v;
+}
+
+__global__ void __launch_bounds__(kCandWarps * 32) readout_cand_wide_kernel(ReadoutArgs a) {
+  const int c = blockIdx.x * kCandWarps + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (c >= a.n_cands) return;
+  const int row = upper_segment(a.set_offsets, a.n_sets, c);  // one pair per candidate: row = set index
+  const int tok = a.pair_tok[c];
+  const bool bad = row < 0 || row >= a.R || tok < 0 || tok >= a.V;
+  float z = 0.f;
+  if (!bad) {
+    const uint4* x4 = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(a.hidden) + (size_t)row * a.H);
+    const uint4* w4 = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(a.lm_head) + (size_t)tok * a.H);
+    const int n = a.H >> 3;
+    for (int base = 0; base < n; base += 32 * kU) {
+      uint4 xa[kU], wa[kU];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int i = base + u * 32 + lane;
+        wa[u] = i < n ? ld_row16(w4 + i) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int i = base + u * 32 + lane;
+        xa[u] = i < n ? ld_row16(x4 + i) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int u = 0; u < kU; ++u) z += dot8(xa[u], wa[u]);
     }
   }
   z = warp_sum(z);
@@ -267,7 +315,9 @@ cudaError_t launch_readout(const ReadoutArgs& a, jev_dtype dt, cudaStream_t s) {
       else readout_cand_block_kernel<float><<<a.n_cands, kCandWarps * 32, 0, s>>>(a);
     } else {
       const int blocks = (a.n_cands + kCandWarps - 1) / kCandWarps;
-      if (dt == JEV_BF16) readout_cand_kernel<__nv_bfloat16><<<blocks, kCandWarps * 32, 0, s>>>(a);
+      if (dt == JEV_BF16 && !a.pair_row && a.n_cands >= kWideCands) {
+        readout_cand_wide_kernel<<<blocks, kCandWarps * 32, 0, s>>>(a);
+      } else if (dt == JEV_BF16) readout_cand_kernel<__nv_bfloat16><<<blocks, kCandWarps * 32, 0, s>>>(a);
       else readout_cand_kernel<float><<<blocks, kCandWarps * 32, 0, s>>>(a);
     }
     cudaError_t e = cudaGetLastError();

@@ -137,6 +137,24 @@ def test_readout_multi_token_invalid_and_empty(jev, dtype):
     assert ch[1] == -1 and ch[2] == -1 and np.all(np.isnan(lp[3:5]))
 
 
+def test_readout_many_one_pair_candidates(jev):
+    # 2000 sets of 9 one-token options (18000 candidates): the wide one-pair readout kernel,
+    # with an invalid token in set 7 and an empty set 11
+    rng = np.random.default_rng(5)
+    n_sets, opts, H, V = 2000, 9, 256, 4096
+    hidden = synth.f32_to_bf16_bits(rng.standard_normal((n_sets, H)).astype(np.float32))
+    W = synth.f32_to_bf16_bits((0.05 * rng.standard_normal((V, H))).astype(np.float32))
+    sizes = np.full(n_sets, opts)
+    sizes[11] = 0
+    so = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
+    toks = rng.integers(0, V, int(so[-1])).astype(np.int32)
+    toks[so[7] + 2] = -3
+    ref = oracle.candidate_readout(hidden, W, so, toks)
+    lp, ch = run_readout(jev, hidden, dev(W), so, toks)
+    check_readout(lp, ch, ref, synth.BF16, "wide readout")
+    assert ch[7] == -1 and ch[11] == -1 and np.all(np.isnan(lp[so[7]:so[8]]))
+
+
 def test_readout_tie_goes_to_first(jev):
     hidden = np.ones((2, 8), np.float32)
     W = np.zeros((4, 8), np.float32)
