@@ -297,6 +297,31 @@ def jev_tree_attn(parent, tok_off, pos0, q, k_root, v_root, k, v, *, head_map=No
     return out, lse
 
 
+_lib.jev_sink_block_plan.argtypes = [_i32, _vp, _i32, _vp, _vp, _vp]
+_lib.jev_sink_block_plan.restype = C.c_int
+
+
+def jev_sink_block_plan(cu_seqlens: np.ndarray, sink_len: int) -> dict:
+    """Host tree arrays of sink-block parallel encoding (see include/jev.h); numpy int32."""
+    cu = np.ascontiguousarray(cu_seqlens, dtype=np.int32)
+    nb = cu.size - 1
+    parent = np.zeros(nb + 1, np.int32); tok_off = np.zeros(nb + 2, np.int32); pos0 = np.zeros(nb + 1, np.int32)
+    _check(_lib.jev_sink_block_plan(nb, cu.ctypes.data, int(sink_len), parent.ctypes.data, tok_off.ctypes.data,
+                                    pos0.ctypes.data), "jev_sink_block_plan")
+    return dict(parent=parent, tok_off=tok_off, pos0=pos0)
+
+
+def jev_sink_block_attn(q, k_sink, v_sink, k, v, cu_seqlens: np.ndarray, **kw):
+    """Sink-block parallel encoding: each block's tokens attend to the whole
+    sink cache and to their own block up to themselves, at the positions of
+    the unsplit sequence.  cu_seqlens is on the host; the plan's arrays are
+    copied to q's device and jev_tree_attn runs; returns (out, lse)."""
+    plan = jev_sink_block_plan(cu_seqlens, k_sink.shape[0])
+    dev = q.device
+    arrs = [torch.from_numpy(plan[n]).to(dev, non_blocking=False) for n in ("parent", "tok_off", "pos0")]
+    return jev_tree_attn(*arrs, q, k_sink, v_sink, k, v, **kw)
+
+
 def jev_rope_inplace(x: torch.Tensor, pos0: int, theta: float = 1e4, stream=None) -> torch.Tensor:
     _dev(x, "x")
     L, H, d = x.shape

@@ -641,6 +641,26 @@ jev_status jev_rope_inplace(void* x, int32_t L, int32_t H, int32_t d, int32_t po
              [&] { return launch_rope_inplace(x, L, H, d, pos0, (double)theta, dt, (cudaStream_t)stream); });
 }
 
+jev_status jev_sink_block_plan(int32_t n_blocks, const int32_t* cu, int32_t sink_len, int32_t* parent,
+                               int32_t* tok_off, int32_t* pos0) {
+  if (n_blocks < 0 || sink_len < 0 || !cu || !parent || !tok_off || !pos0) return fail(JEV_ERR_INVALID_ARG, "bad arguments");
+  if (cu[0] != 0) return fail(JEV_ERR_INVALID_ARG, "cu_seqlens[0] != 0");
+  for (int b = 0; b < n_blocks; ++b)
+    if (cu[b + 1] < cu[b]) return fail(JEV_ERR_INVALID_ARG, "cu_seqlens decreases at %d", b);
+  if ((long long)sink_len + cu[n_blocks] > INT32_MAX) return fail(JEV_ERR_INVALID_ARG, "positions overflow");
+  // node 0: the sink (the root cache, no packed tokens); node b + 1: block b
+  parent[0] = -1;
+  tok_off[0] = 0;
+  pos0[0] = 0;
+  for (int b = 0; b < n_blocks; ++b) {
+    parent[b + 1] = 0;
+    tok_off[b + 1] = cu[b];
+    pos0[b + 1] = sink_len + cu[b];
+  }
+  tok_off[n_blocks + 1] = cu[n_blocks];
+  return JEV_OK;
+}
+
 jev_status jev_tree_build(int32_t n_cands, const int32_t* seq_off, const int32_t* toks, int32_t root_len,
                           int32_t cap_nodes, int32_t cap_toks, int32_t* parent, int32_t* tok_off, int32_t* pos0,
                           int32_t* leaf_of, int32_t* node_toks, int32_t* path_row, int32_t* n_nodes_out) {

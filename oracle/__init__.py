@@ -222,6 +222,28 @@ def tree_readout_pairs(seq_off, score_from, path_row, set_offsets):
     return np.asarray(co, np.int32), np.asarray(rows, np.int32), np.asarray(tix, np.int64)
 
 
+def sink_block_attn(q, k, v, k_sink, v_sink, cu_seqlens, *, theta=1e4, scale=0.0, head_map=None):
+    """Sink-block parallel encoding ("PEVLM: Parallel Encoding for Vision-
+    Language Models", abstract: context blocks share a sink block, position
+    embeddings stay sequential), read plainly: block b is one branch over the
+    sink cache whose first token sits at position len(sink) + cu_seqlens[b],
+    the position it has in the unsplit sequence.  Each block is evaluated as
+    its own single-branch problem; returns (out, lse) as float64."""
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    S = k_sink.shape[0]
+    T, Hq, d = q.shape
+    out = np.zeros((T, Hq, d), np.float64)
+    lse = np.zeros((T, Hq), np.float64)
+    for b in range(cu.size - 1):
+        a, e = int(cu[b]), int(cu[b + 1])
+        if e == a:
+            continue
+        ob, lb = prefix_suffix_attn(q[a:e], k_sink, v_sink, k[a:e], v[a:e], np.array([0, e - a], np.int32),
+                                    theta=theta, scale=scale, pos_offset=S + a, head_map=head_map)
+        out[a:e], lse[a:e] = ob, lb
+    return out, lse
+
+
 def tree_attn(trie, q, k, v, k_root, v_root, *, theta=1e4, scale=0.0, head_map=None, n_threads=0):
     """Tree attention by flattening every root->node path; (out, lse) float64."""
     q, k, v, k_root, v_root = (_c(a) for a in (q, k, v, k_root, v_root))

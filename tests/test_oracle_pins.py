@@ -93,6 +93,52 @@ def test_hand_two_token_case():
     assert abs(lse[0, 0] - (s1 + math.log1p(math.exp(s0 - s1)))) < 1e-12
 
 
+def test_sink_block_matches_sdpa_per_block():
+    """Sink-block parallel encoding ("PEVLM", abstract): block b's rows equal
+    the last rows of causal fp64 SDPA over [sink; block b] with the block's
+    tokens at their positions in the unsplit sequence, S + cu[b] + j."""
+    theta, S, Hq, Hkv, d = 1e4, 7, 4, 2, 16
+    rng = np.random.default_rng(17)
+    lens = np.array([3, 1, 6, 4], np.int32)
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    T = int(cu[-1])
+    k_sink_raw = rng.standard_normal((S, Hkv, d))
+    k_sink = _rope_complex(k_sink_raw.transpose(1, 0, 2), np.arange(S), theta).transpose(1, 0, 2).astype(np.float32)
+    v_sink, q, k, v = (rng.standard_normal(s).astype(np.float32)
+                       for s in ((S, Hkv, d), (T, Hq, d), (T, Hkv, d), (T, Hkv, d)))
+    out, lse = oracle.sink_block_attn(q, k, v, k_sink, v_sink, cu, theta=theta)
+    scale = 1.0 / math.sqrt(d)
+    hm = torch.from_numpy(np.arange(Hq) // (Hq // Hkv)).long()
+    for b in range(lens.size):
+        a, e = cu[b], cu[b + 1]
+        pos = S + a + np.arange(e - a)
+        q_b = _rope_complex(_f64(q)[a:e].transpose(1, 0, 2), pos, theta).transpose(1, 0, 2)
+        k_b = _rope_complex(_f64(k)[a:e].transpose(1, 0, 2), pos, theta).transpose(1, 0, 2)
+        o_ref, l_ref = _sdpa_branch(np.concatenate([np.zeros((S, Hq, d)), q_b]),
+                                    np.concatenate([_f64(k_sink), k_b]),
+                                    np.concatenate([_f64(v_sink), _f64(v)[a:e]]), None, Hkv, hm, theta, scale)
+        np.testing.assert_allclose(out[a:e], o_ref[S:], atol=1e-12)
+        np.testing.assert_allclose(lse[a:e], l_ref[S:], atol=1e-12)
+
+
+def test_sink_block_first_block_is_full_attention():
+    """The first block sees exactly what full causal attention over the unsplit
+    sequence gives it (the pages' alignment with Full-Attention is exact there);
+    later blocks, which no longer see earlier blocks, differ."""
+    rng = np.random.default_rng(23)
+    S, Hq, Hkv, d = 5, 2, 1, 8
+    lens = np.array([4, 3], np.int32)
+    cu = np.array([0, 4, 7], np.int32)
+    f32 = lambda *sh: rng.standard_normal(sh).astype(np.float32)
+    k_sink, v_sink = f32(S, Hkv, d), f32(S, Hkv, d)
+    q, k, v = f32(7, Hq, d), f32(7, Hkv, d), f32(7, Hkv, d)
+    out, lse = oracle.sink_block_attn(q, k, v, k_sink, v_sink, cu)
+    full_o, full_l = oracle.prefix_suffix_attn(q, k_sink, v_sink, k, v, np.array([0, 7], np.int32), pos_offset=S)
+    np.testing.assert_allclose(out[:4], full_o[:4], atol=1e-13)
+    np.testing.assert_allclose(lse[:4], full_l[:4], atol=1e-13)
+    assert np.abs(out[4:] - full_o[4:]).max() > 1e-3
+
+
 def _small_case(B=3, Lp=9, lens=(1, 4, 6), Hq=4, Hkv=2, d=8, seed=5, dtype=synth.F32):
     cfg = synth.FlatConfig("t", dtype, Lp, B, 1, 1, Hq, Hkv, d, 16, 32, 2, 3, seed=seed)
     return synth.flat_case(cfg, with_lm_head=False, lengths=np.array(lens, np.int32))
