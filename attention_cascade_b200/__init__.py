@@ -39,7 +39,8 @@ class JevError(RuntimeError):
 class jev_attn_desc(C.Structure):
     _fields_ = [("B", C.c_int32), ("Lp", C.c_int32), ("Hq", C.c_int32), ("Hkv", C.c_int32), ("d", C.c_int32),
                 ("T_total", C.c_int32), ("dtype", C.c_int32), ("rope_theta", C.c_float),
-                ("softmax_scale", C.c_float), ("pos_offset", C.c_int32), ("num_splits", C.c_int32)]
+                ("softmax_scale", C.c_float), ("pos_offset", C.c_int32), ("num_splits", C.c_int32),
+                ("pos_mode", C.c_int32)]
 
 
 class jev_attn_plan(C.Structure):
@@ -113,9 +114,9 @@ def _stream(stream) -> int:
 
 
 def make_attn_desc(B, Lp, Hq, Hkv, d, T_total, dtype_code, rope_theta=1e4, softmax_scale=0.0, pos_offset=-1,
-                   num_splits=0) -> jev_attn_desc:
+                   num_splits=0, pos_mode=0) -> jev_attn_desc:
     return jev_attn_desc(int(B), int(Lp), int(Hq), int(Hkv), int(d), int(T_total), int(dtype_code),
-                         float(rope_theta), float(softmax_scale), int(pos_offset), int(num_splits))
+                         float(rope_theta), float(softmax_scale), int(pos_offset), int(num_splits), int(pos_mode))
 
 
 # descriptors of recent calls, reused as they are (the library only reads them)
@@ -152,7 +153,7 @@ def new_workspace(nbytes: int, device, stream=None) -> torch.Tensor:
 
 def jev_prefix_suffix_attn(q, k_pre, v_pre, k_suf, v_suf, cu_seqlens, *, head_map=None, out=None, lse=None,
                            workspace=None, rope_theta=1e4, softmax_scale=0.0, pos_offset=-1, num_splits=0,
-                           T_total: Optional[int] = None, want_lse=True, stream=None):
+                           T_total: Optional[int] = None, want_lse=True, stream=None, pos_mode=0):
     """Shared-prefix attention for B ragged suffix branches; returns (out, lse)."""
     dt = _dtype_code(q)
     T, Hq, d = q.shape
@@ -163,7 +164,7 @@ def jev_prefix_suffix_attn(q, k_pre, v_pre, k_suf, v_suf, cu_seqlens, *, head_ma
     _dev(head_map, "head_map", torch.int32)
     B = cu_seqlens.numel() - 1
     desc = _cached_desc(make_attn_desc, (B, Lp, Hq, Hkv, d, T if T_total is None else T_total, dt, rope_theta,
-                                         softmax_scale, pos_offset, num_splits))
+                                         softmax_scale, pos_offset, num_splits, pos_mode))
     if out is None:
         out = torch.empty_like(q)
     if lse is None and want_lse:
@@ -297,29 +298,12 @@ def jev_tree_attn(parent, tok_off, pos0, q, k_root, v_root, k, v, *, head_map=No
     return out, lse
 
 
-_lib.jev_sink_block_plan.argtypes = [_i32, _vp, _i32, _vp, _vp, _vp]
-_lib.jev_sink_block_plan.restype = C.c_int
-
-
-def jev_sink_block_plan(cu_seqlens: np.ndarray, sink_len: int) -> dict:
-    """Host tree arrays of sink-block parallel encoding (see include/jev.h); numpy int32."""
-    cu = np.ascontiguousarray(cu_seqlens, dtype=np.int32)
-    nb = cu.size - 1
-    parent = np.zeros(nb + 1, np.int32); tok_off = np.zeros(nb + 2, np.int32); pos0 = np.zeros(nb + 1, np.int32)
-    _check(_lib.jev_sink_block_plan(nb, cu.ctypes.data, int(sink_len), parent.ctypes.data, tok_off.ctypes.data,
-                                    pos0.ctypes.data), "jev_sink_block_plan")
-    return dict(parent=parent, tok_off=tok_off, pos0=pos0)
-
-
-def jev_sink_block_attn(q, k_sink, v_sink, k, v, cu_seqlens: np.ndarray, **kw):
-    """Sink-block parallel encoding: each block's tokens attend to the whole
-    sink cache and to their own block up to themselves, at the positions of
-    the unsplit sequence.  cu_seqlens is on the host; the plan's arrays are
-    copied to q's device and jev_tree_attn runs; returns (out, lse)."""
-    plan = jev_sink_block_plan(cu_seqlens, k_sink.shape[0])
-    dev = q.device
-    arrs = [torch.from_numpy(plan[n]).to(dev, non_blocking=False) for n in ("parent", "tok_off", "pos0")]
-    return jev_tree_attn(*arrs, q, k_sink, v_sink, k, v, **kw)
+def jev_sink_block_attn(q, k_sink, v_sink, k, v, cu_seqlens, **kw):
+    """Sink-block parallel encoding: each block of the packed input attends to
+    the whole sink cache and to its own block up to itself; packed token t
+    sits at position len(sink) + t, its position in the unsplit sequence
+    (jev_prefix_suffix_attn with pos_mode 1); returns (out, lse)."""
+    return jev_prefix_suffix_attn(q, k_sink, v_sink, k, v, cu_seqlens, pos_mode=1, **kw)
 
 
 def jev_rope_inplace(x: torch.Tensor, pos0: int, theta: float = 1e4, stream=None) -> torch.Tensor:

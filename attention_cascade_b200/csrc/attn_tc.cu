@@ -491,10 +491,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           // suffix window: same branch up to the row's own token (+ ancestor nodes)
           const int kb = sg.lo + (j - sg.n_pre) * kBN + c_base;
           const int c_lo = start - kb, c_hi = t - kb;
-          if (!TREE || nanc <= 0) {
+          const bool flat_row = !TREE || nanc <= 0;
+          // the mask is skipped when every row of the warp sees all 64 of its keys in this tile
+          const bool whole = __all_sync(0xffffffffu, flat_row && c_lo <= 0 && c_hi >= kHalfCols - 1);
+          if (flat_row) {
+            if (!whole) {
 #pragma unroll
-            for (int c = 0; c < kHalfCols; ++c)
-              if (!(c >= c_lo && c <= c_hi)) xs[c] = kNegInf;
+              for (int c = 0; c < kHalfCols; ++c)
+                if (!(c >= c_lo && c <= c_hi)) xs[c] = kNegInf;
+            }
           } else {
             // a tree row also sees its ancestors' key ranges (read here, where needed)
             uint64_t vis = 0;

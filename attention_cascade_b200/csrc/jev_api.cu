@@ -325,6 +325,7 @@ jev_status check_desc(const jev_attn_desc* d) {
   if (d->dtype != JEV_BF16 && d->dtype != JEV_F32) return fail(JEV_ERR_UNSUPPORTED, "dtype");
   if (!(d->rope_theta > 0.f)) return fail(JEV_ERR_INVALID_ARG, "rope_theta must be > 0");
   if (d->softmax_scale < 0.f) return fail(JEV_ERR_INVALID_ARG, "softmax_scale must be >= 0");
+  if (d->pos_mode != 0 && d->pos_mode != 1) return fail(JEV_ERR_INVALID_ARG, "pos_mode must be 0 or 1");
   if ((long long)d->T_total * (d->Hq / d->Hkv) > (1LL << 30)) return fail(JEV_ERR_UNSUPPORTED, "too many rows");
   return JEV_OK;
 }
@@ -353,6 +354,7 @@ jev_status attention_core(const jev_attn_desc* d, int T, const Plan& p, const La
   r.node_nanc = tree ? reinterpret_cast<int32_t*>(ws + L.nanc) : nullptr;
   r.n_segs = n_segs; r.T = T; r.Hq = d->Hq; r.Hkv = d->Hkv; r.d = d->d;
   r.pos_offset = d->pos_offset >= 0 ? d->pos_offset : d->Lp;
+  r.pos_seq = d->pos_mode == 1 ? 1 : 0;
   r.theta = (double)d->rope_theta;
   for (int i = 0; i < d->d / 2; ++i) r.inv_freq[i] = std::pow(r.theta, -2.0 * i / d->d);
   jev_status st = run("rope_pack", s, [&] { return launch_rope_pack(r, d->dtype, s); });
@@ -641,26 +643,6 @@ jev_status jev_rope_inplace(void* x, int32_t L, int32_t H, int32_t d, int32_t po
              [&] { return launch_rope_inplace(x, L, H, d, pos0, (double)theta, dt, (cudaStream_t)stream); });
 }
 
-jev_status jev_sink_block_plan(int32_t n_blocks, const int32_t* cu, int32_t sink_len, int32_t* parent,
-                               int32_t* tok_off, int32_t* pos0) {
-  if (n_blocks < 0 || sink_len < 0 || !cu || !parent || !tok_off || !pos0) return fail(JEV_ERR_INVALID_ARG, "bad arguments");
-  if (cu[0] != 0) return fail(JEV_ERR_INVALID_ARG, "cu_seqlens[0] != 0");
-  for (int b = 0; b < n_blocks; ++b)
-    if (cu[b + 1] < cu[b]) return fail(JEV_ERR_INVALID_ARG, "cu_seqlens decreases at %d", b);
-  if ((long long)sink_len + cu[n_blocks] > INT32_MAX) return fail(JEV_ERR_INVALID_ARG, "positions overflow");
-  // node 0: the sink (the root cache, no packed tokens); node b + 1: block b
-  parent[0] = -1;
-  tok_off[0] = 0;
-  pos0[0] = 0;
-  for (int b = 0; b < n_blocks; ++b) {
-    parent[b + 1] = 0;
-    tok_off[b + 1] = cu[b];
-    pos0[b + 1] = sink_len + cu[b];
-  }
-  tok_off[n_blocks + 1] = cu[n_blocks];
-  return JEV_OK;
-}
-
 jev_status jev_tree_build(int32_t n_cands, const int32_t* seq_off, const int32_t* toks, int32_t root_len,
                           int32_t cap_nodes, int32_t cap_toks, int32_t* parent, int32_t* tok_off, int32_t* pos0,
                           int32_t* leaf_of, int32_t* node_toks, int32_t* path_row, int32_t* n_nodes_out) {
@@ -751,6 +733,7 @@ jev_status jev_tree_attn(const jev_attn_desc* d, int32_t n_nodes, const int32_t*
   jev_status st = check_desc(d);
   if (st) return st;
   if (n_nodes < 1) return fail(JEV_ERR_INVALID_ARG, "n_nodes < 1");
+  if (d->pos_mode != 0) return fail(JEV_ERR_INVALID_ARG, "tree positions come from pos0 (pos_mode must be 0)");
   if (d->T_total == 0) return JEV_OK;
   if (!parent || !tok_off || !pos0 || !q || !k || !v || !out) return fail(JEV_ERR_INVALID_ARG, "required pointer is NULL");
   if (d->Lp > 0 && (!k_root || !v_root)) return fail(JEV_ERR_INVALID_ARG, "root pointers are NULL with Lp > 0");

@@ -25,6 +25,7 @@ struct RopePackArgs {
   int2* node_anc;          // tree: [n_segs, kMaxDepth] ancestor key ranges (written)
   int32_t* node_nanc;      // tree: [n_segs] ancestor count, -1 for a malformed chain (written)
   int n_segs, T, Hq, Hkv, d, pos_offset;
+  int pos_seq;             // 1: token t at pos_offset + t (sequential across segments)
   double theta;
   double inv_freq[128];    // theta^(-2i/d), i < d/2, formed on the host in double
 };

@@ -181,7 +181,7 @@ __global__ void __launch_bounds__(256) rope_pack_kernel(RopePackArgs a) {
     start = offs_in_smem ? s_offs[seg] : a.offs[seg];
     if (start > t) start = t;
     if (start < 0) start = 0;
-    pos = (a.pos0 ? a.pos0[seg] : a.pos_offset) + (t - start);
+    pos = a.pos_seq ? a.pos_offset + t : (a.pos0 ? a.pos0[seg] : a.pos_offset) + (t - start);
     a.info[t] = TokInfo{start, pos, seg, 0};
   }
   pos = __shfl_sync(0xffffffffu, pos, 0);

@@ -481,7 +481,46 @@ def diagnostics(dev, jev, torch) -> dict:
                         "us": rus, "GBps": rbytes / rus / 1e3, "frac_of_hbm": rbytes / rus / 1e3 / hbm,
                         "note": "per-kernel event time (includes launch latency)"}
     out["attn_call_us"] = {k: 1e3 * v[1] / max(v[0], 1) for k, v in prof.items()}
-    # the tensor-core kernel at this size: many waves of whole tiles
+    del args_, o, lse, ws
+    torch.cuda.empty_cache()
+    # ---- sink-block parallel encoding (flat kernels, sequential positions): 32 blocks of 1024 tokens over a
+    # 64-token sink
+    S, nb, bl, Hq, Hkv, d = 64, 32, 1024, 28, 4, 128
+    cu_sb = np.arange(0, nb * bl + 1, bl, dtype=np.int32)
+    Tsb = nb * bl
+    mk = lambda *sh: to_dev(synth.f32_to_bf16_bits(rng.standard_normal(sh).astype(np.float32)), dev, torch)
+    sq, sk, sv, ssk, ssv = mk(Tsb, Hq, d), mk(Tsb, Hkv, d), mk(Tsb, Hkv, d), mk(S, Hkv, d), mk(S, Hkv, d)
+    cu_d = torch.from_numpy(cu_sb).to(dev)
+    sdesc = jev.make_attn_desc(nb, S, Hq, Hkv, d, Tsb, jev.JEV_BF16, pos_mode=1)
+    sws = jev.new_workspace(jev.jev_prefix_suffix_attn_workspace(sdesc), dev)
+    so_, sl_ = torch.empty_like(sq), torch.empty((Tsb, Hq), dtype=torch.float32, device=dev)
+
+    def sink_block():
+        jev.jev_sink_block_attn(sq, ssk, ssv, sk, sv, cu_d, out=so_, lse=sl_, workspace=sws,
+                                stream=torch.cuda.current_stream())
+    graph_us(torch, sink_block, stream, 3, 2)
+    jev.jev_profile_read()
+    jev.jev_profile_enable(True)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        sink_block()
+    jev.jev_profile_enable(False)
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            g.replay()
+    torch.cuda.synchronize()
+    sprof = jev.jev_profile_read()
+    del g
+    sflops = 4 * Hq * d * nb * (bl * S + bl * (bl + 1) // 2)
+    speak = float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"]))
+    s_us = {k: 1e3 * v[1] / max(v[0], 1) for k, v in sprof.items()}
+    if "attn_tc" in s_us:
+        out["sink_block"] = {"workload": f"{nb} blocks of {bl} tokens over a {S}-token sink, Hq={Hq}, Hkv={Hkv}, "
+                                         f"d={d}", "flops_per_call": sflops, "kernels_us": s_us,
+                             "TFLOPs": sflops / s_us["attn_tc"] / 1e6,
+                             "frac_of_sustained_bf16": sflops / s_us["attn_tc"] / 1e6 / speak,
+                             "tokens_per_s": Tsb / (sum(s_us.values()) / 1e6)}
+    # the tensor-core kernel at the wide size: many waves of whole tiles
     if "attn_tc" in prof:
         flops = flat_work(c)["flops_attn"]
         aus = out["attn_call_us"]["attn_tc"]

@@ -80,6 +80,12 @@ typedef struct {
   float softmax_scale;   /* 0 -> 1/sqrt(d)                                          */
   int32_t pos_offset;    /* position of every branch's first suffix token; <0 -> Lp */
   int32_t num_splits;    /* prefix key splits; 0 -> chosen from Lp and the SM count */
+  int32_t pos_mode;      /* 0: token j of every branch at pos_offset + j;
+                            1: sequential positions (sink-block parallel encoding,
+                            "PEVLM: Parallel Encoding for Vision-Language Models",
+                            abstract: blocks share a sink and keep the positions of
+                            the unsplit sequence): packed token t at pos_offset + t.
+                            jev_prefix_suffix_attn only.                              */
 } jev_attn_desc;
 
 /* Bytes of workspace jev_prefix_suffix_attn needs for `desc`. */
@@ -271,25 +277,6 @@ jev_status jev_tree_readout_plan(int32_t n_cands, const int32_t* seq_off, const 
                                  const int32_t* score_from, const int32_t* path_row, int32_t cap_pairs,
                                  int32_t* cand_offsets, int32_t* pair_row, int32_t* pair_tok,
                                  int32_t* n_pairs);
-
-/*
- * jev_sink_block_plan (HOST) — the tree arrays of sink-block parallel
- * encoding ("PEVLM: Parallel Encoding for Vision-Language Models", abstract:
- * the input is cut into context blocks that share one sink block, and the
- * position embeddings stay sequential).  Block b (tokens cu_seqlens[b] ..
- * cu_seqlens[b+1]-1 of the packed input) becomes node b+1, a child of the
- * root (the sink, sink_len cached keys at positions 0..sink_len-1), and its
- * j-th token sits at position sink_len + cu_seqlens[b] + j — the position
- * it would have in the unsplit sequence.  jev_tree_attn on these arrays
- * gives each block token attention over the whole sink plus its own block
- * up to itself; other blocks are not visible.
- *   cu_seqlens [n_blocks+1] (host, cu[0] = 0, non-decreasing)
- *   outputs (host): parent [n_blocks+1], tok_off [n_blocks+2], pos0 [n_blocks+1]
- *   JEV_ERR_INVALID_ARG for NULL pointers, n_blocks < 0, sink_len < 0 or
- *   malformed cu_seqlens.
- */
-jev_status jev_sink_block_plan(int32_t n_blocks, const int32_t* cu_seqlens, int32_t sink_len, int32_t* parent,
-                               int32_t* tok_off, int32_t* pos0);
 
 /* Bytes of workspace jev_tree_attn needs. */
 size_t jev_tree_attn_workspace(const jev_attn_desc* desc, int32_t n_nodes);

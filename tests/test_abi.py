@@ -113,15 +113,3 @@ def test_tree_build_capacity_and_errors(jev):
     with pytest.raises(jev.JevError):
         jev.jev_tree_readout_plan(so, toks, np.array([0, 1], np.int32), np.zeros(5, np.int32))
 
-
-def test_sink_block_plan(jev):
-    """Host arrays of sink-block encoding: block b is node b + 1 under the
-    root, its tokens cu[b] .. cu[b+1] at positions sink_len + cu[b] + j."""
-    p = jev.jev_sink_block_plan(np.array([0, 3, 3, 10], np.int32), 64)
-    assert p["parent"].tolist() == [-1, 0, 0, 0]
-    assert p["tok_off"].tolist() == [0, 0, 3, 3, 10]
-    assert p["pos0"].tolist() == [0, 64, 67, 67]
-    with pytest.raises(jev.JevError):
-        jev.jev_sink_block_plan(np.array([0, 5, 2], np.int32), 8)
-    with pytest.raises(jev.JevError):
-        jev.jev_sink_block_plan(np.array([1, 5], np.int32), 8)
