@@ -113,3 +113,18 @@ def test_tree_build_capacity_and_errors(jev):
     with pytest.raises(jev.JevError):
         jev.jev_tree_readout_plan(so, toks, np.array([0, 1], np.int32), np.zeros(5, np.int32))
 
+
+
+def test_position_mode_is_checked_on_the_host(jev):
+    """pos_mode is 0 (per-branch positions) or 1 (sequential, sink-block
+    encoding); anything else, and sequential positions on the tree entry point,
+    are rejected before anything is enqueued."""
+    bad = jev.make_attn_desc(2, 128, 8, 2, 128, 10, jev.JEV_BF16, pos_mode=2)
+    assert jev.jev_prefix_suffix_attn_workspace(bad) == 0
+    with pytest.raises(jev.JevError):
+        jev.jev_prefix_suffix_attn_plan(bad)
+    n0 = jev.jev_launch_count()
+    seq = jev.make_attn_desc(2, 128, 8, 2, 128, 10, jev.JEV_BF16, pos_mode=1)
+    assert jev.jev_prefix_suffix_attn_workspace(seq) > 0
+    st = jev._lib.jev_tree_attn(C.byref(seq), 3, *([C.c_void_p(16)] * 12), C.c_size_t(1 << 20), None)
+    assert st == 1 and jev.jev_launch_count() == n0

@@ -219,17 +219,20 @@ def test_tree_config_c4(jev):
     check_readout(lp, ch, ref, cfg.dtype, "c4 readout")
 
 
-@pytest.mark.parametrize("lens,S,d", [([50, 1, 130, 77, 200], 128, 128), ([256] * 16, 256, 128), ([33, 0, 70], 64, 64)])
-def test_sink_block_parallel_encoding(jev, lens, S, d):
+@pytest.mark.parametrize("lens,S,d,dtype", [([50, 1, 130, 77, 200], 128, 128, synth.BF16),
+                                             ([256] * 16, 256, 128, synth.BF16), ([33, 0, 70], 64, 64, synth.BF16),
+                                             ([20, 7, 41], 48, 64, synth.F32)])
+def test_sink_block_parallel_encoding(jev, lens, S, d, dtype):
     """Blocks over a shared sink at their unsplit positions (PEVLM; the flat
     kernels with sequential positions), every element against the per-block oracle."""
     rng = np.random.default_rng(sum(lens) + S)
     Hq, Hkv = 8, 2
     cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
     T = int(cu[-1])
-    mk = lambda *sh: synth.f32_to_bf16_bits(rng.standard_normal(sh).astype(np.float32))
+    mk = lambda *sh: (synth.f32_to_bf16_bits(rng.standard_normal(sh).astype(np.float32)) if dtype == synth.BF16
+                      else rng.standard_normal(sh).astype(np.float32))
     q, k, v, k_sink, v_sink = mk(T, Hq, d), mk(T, Hkv, d), mk(T, Hkv, d), mk(S, Hkv, d), mk(S, Hkv, d)
     out, lse = jev.jev_sink_block_attn(dev(q), dev(k_sink), dev(v_sink), dev(k), dev(v), dev(cu))
     torch.cuda.synchronize()
     ref_o, ref_l = oracle.sink_block_attn(q, k, v, k_sink, v_sink, cu)
-    check_attn(host_f64(out), host_f64(lse), ref_o, ref_l, synth.BF16, f"sink-block {lens[:3]}")
+    check_attn(host_f64(out), host_f64(lse), ref_o, ref_l, dtype, f"sink-block {lens[:3]}")
