@@ -10,12 +10,13 @@
 // masked per row.
 //
 // Schedule.  A work tile (256 stacked rows of one kv group) has P = n_pre + 1
-// units: its 128-key prefix tiles and the suffix window.  The units of all
-// tiles are spread evenly over n_ctas persistent CTAs; a CTA visits its units
-// as segments (runs inside one tile).  A segment that covers its whole tile
-// writes the final output; other segments write a normalised fp32 partial and
-// its log2 normaliser, and tc_fixup_kernel merges the segments of each split
-// tile.
+// units: its 128-key prefix tiles and the suffix window.  n_ctas persistent
+// CTAs first take whole tiles for full_waves rounds; the units of the
+// remaining tail tiles are spread evenly over tail_ctas of them.  A CTA visits
+// its work as segments (runs inside one tile).  A segment that covers its
+// whole tile writes the final output; other segments write a normalised fp32
+// partial and its log2 normaliser, and tc_fixup_kernel merges the segments of
+// each split tail tile.
 //
 // CTA = 18 warps:
 //   warps 0-7   Q tile 0: warps 0-3 columns 0-63, warps 4-7 columns 64-127 of
@@ -28,9 +29,11 @@
 // both halves of tile i have written P_i (bf16, aliasing S_i) it issues
 // O_i += P_i V_j with P_i read from TMEM (TS form); tile 0's softmax overlaps
 // tile 1's MMAs and the other way round.  The two halves of a row exchange
-// their maxima through shared memory each key tile; the softmax runs in the
-// log2 domain with a lazy running max (raised only when a row's maximum
-// exceeds it by more than 8, so O is rescaled rarely and P stays <= 2^8).
+// their maxima through shared memory each key tile (a 64-thread barrier per
+// pair of warps); the softmax runs in the log2 domain with a lazy running max
+// (raised only when a row's maximum exceeds it by more than 8, so O is
+// rescaled rarely and P stays <= 2^8), its scale-and-subtract and row sums as
+// packed f32x2 operations.
 // Every mbarrier wait is bounded; a wait that runs out raises
 // JEV_DEV_WAIT_TIMEOUT in the status word and the CTA winds down.
 #include <cuda.h>
