@@ -61,6 +61,7 @@ _lib.jev_prefix_suffix_attn_workspace.restype = _sz
 _lib.jev_prefix_suffix_attn_plan.argtypes = [C.POINTER(jev_attn_desc), _i32, _i32, C.POINTER(jev_attn_plan)]
 _lib.jev_prefix_suffix_attn.argtypes = [C.POINTER(jev_attn_desc)] + [_vp] * 10 + [_sz, _vp]
 _lib.jev_candidate_readout.argtypes = [C.POINTER(jev_readout_desc)] + [_vp] * 10
+_lib.jev_candidate_readout_normalized.argtypes = [C.POINTER(jev_readout_desc)] + [_vp] * 11
 _lib.jev_tree_build.argtypes = [_i32, _vp, _vp, _i32, _i32, _i32] + [_vp] * 7
 _lib.jev_tree_readout_plan.argtypes = [_i32, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp]
 _lib.jev_tree_attn_workspace.argtypes = [C.POINTER(jev_attn_desc), _i32]
@@ -73,9 +74,12 @@ _lib.jev_profile_enable.argtypes = [_i32]
 _lib.jev_profile_read.argtypes = [_i32, C.c_char_p, _vp, _vp, _i32]
 _lib.jev_profile_read.restype = _i32
 _lib.jev_launch_count.restype = C.c_int64
+_lib.jev_vocab_lse_workspace.argtypes = [_i32, _i32]
+_lib.jev_vocab_lse_workspace.restype = _sz
+_lib.jev_vocab_lse.argtypes = [_vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _sz, _vp]
 for _f in ("jev_prefix_suffix_attn", "jev_prefix_suffix_attn_plan", "jev_candidate_readout", "jev_tree_build",
            "jev_tree_readout_plan", "jev_tree_attn", "jev_rope_inplace", "jev_workspace_init", "jev_check_device_status",
-           "jev_profile_enable"):
+           "jev_profile_enable", "jev_vocab_lse", "jev_candidate_readout_normalized"):
     getattr(_lib, _f).restype = C.c_int
 
 
@@ -209,8 +213,10 @@ def jev_prefix_suffix_attn_noalloc(q, k_pre, v_pre, k_suf, v_suf, cu_seqlens, ou
 
 
 def jev_candidate_readout(hidden, lm_head, set_offsets, pair_tok, *, cand_offsets=None, pair_row=None,
-                          logprob=None, choice=None, score=None, stream=None):
-    """Per-option log-probs and argmax over each option set; returns (logprob, choice)."""
+                          logprob=None, choice=None, score=None, row_lse=None, stream=None):
+    """Per-option log-probs and argmax over each option set; returns (logprob, choice).
+    With row_lse (fp32 [R], from jev_vocab_lse) every pair's logit is
+    normalised over the vocabulary first (jev_candidate_readout_normalized)."""
     dt = _dtype_code(hidden)
     _dev(hidden, "hidden", hidden.dtype)
     _dev(lm_head, "lm_head", hidden.dtype)
@@ -228,10 +234,52 @@ def jev_candidate_readout(hidden, lm_head, set_offsets, pair_tok, *, cand_offset
     _dev(logprob, "logprob", torch.float32)
     _dev(choice, "choice", torch.int32)
     _dev(score, "score", torch.float32)
-    _check(_lib.jev_candidate_readout(C.byref(desc), _p(hidden), _p(lm_head), _p(set_offsets), _p(cand_offsets),
-                                      _p(pair_row), _p(pair_tok), _p(logprob), _p(choice), _p(score),
-                                      _stream(stream)), "jev_candidate_readout")
+    if row_lse is None:
+        _check(_lib.jev_candidate_readout(C.byref(desc), _p(hidden), _p(lm_head), _p(set_offsets), _p(cand_offsets),
+                                          _p(pair_row), _p(pair_tok), _p(logprob), _p(choice), _p(score),
+                                          _stream(stream)), "jev_candidate_readout")
+    else:
+        _dev(row_lse, "row_lse", torch.float32)
+        _check(_lib.jev_candidate_readout_normalized(C.byref(desc), _p(hidden), _p(lm_head), _p(set_offsets),
+                                                     _p(cand_offsets), _p(pair_row), _p(pair_tok), _p(row_lse),
+                                                     _p(logprob), _p(choice), _p(score), _stream(stream)),
+               "jev_candidate_readout_normalized")
     return logprob, choice
+
+
+def jev_sequence_logprob(hidden, lm_head, cand_offsets, pair_row, pair_tok, *, lse=None, workspace=None,
+                         stream=None):
+    """Sequence log-probability of every multi-token candidate over the whole
+    vocabulary: jev_vocab_lse of the hidden rows, then the normalised readout
+    with all candidates in one set.  Returns fp32 [n_cands]."""
+    lse = jev_vocab_lse(hidden, lm_head, lse=lse, workspace=workspace, stream=stream)
+    n_cands = cand_offsets.numel() - 1
+    so = torch.tensor([0, n_cands], dtype=torch.int32, device=hidden.device)
+    score = torch.empty(n_cands, dtype=torch.float32, device=hidden.device)
+    jev_candidate_readout(hidden, lm_head, so, pair_tok, cand_offsets=cand_offsets, pair_row=pair_row, score=score,
+                          row_lse=lse, stream=stream)
+    return score
+
+
+def jev_vocab_lse_workspace(R: int, V: int) -> int:
+    return int(_lib.jev_vocab_lse_workspace(R, V))
+
+
+def jev_vocab_lse(hidden, lm_head, *, lse=None, workspace=None, stream=None):
+    """Full-vocabulary log-sum-exp of every hidden row, lse [R] fp32."""
+    dt = _dtype_code(hidden)
+    _dev(hidden, "hidden", hidden.dtype)
+    _dev(lm_head, "lm_head", hidden.dtype)
+    R, H = hidden.shape
+    V = lm_head.shape[0]
+    if lse is None:
+        lse = torch.empty(R, dtype=torch.float32, device=hidden.device)
+    _dev(lse, "lse", torch.float32)
+    if workspace is None:
+        workspace = new_workspace(jev_vocab_lse_workspace(R, V), hidden.device)
+    _check(_lib.jev_vocab_lse(_p(hidden), _p(lm_head), R, H, V, dt, _p(lse), _p(workspace), workspace.numel(),
+                              _stream(stream)), "jev_vocab_lse")
+    return lse
 
 
 def jev_tree_build(seq_off: np.ndarray, toks: np.ndarray, root_len: int) -> dict:

@@ -613,6 +613,14 @@ jev_status jev_candidate_readout(const jev_readout_desc* d, const void* hidden, 
                                  const int32_t* set_offsets, const int32_t* cand_offsets, const int32_t* pair_row,
                                  const int32_t* pair_tok, float* logprob, int32_t* choice, float* score,
                                  jev_stream_t stream) {
+  return jev_candidate_readout_normalized(d, hidden, lm_head, set_offsets, cand_offsets, pair_row, pair_tok, nullptr,
+                                          logprob, choice, score, stream);
+}
+
+jev_status jev_candidate_readout_normalized(const jev_readout_desc* d, const void* hidden, const void* lm_head,
+                                            const int32_t* set_offsets, const int32_t* cand_offsets,
+                                            const int32_t* pair_row, const int32_t* pair_tok, const float* row_lse,
+                                            float* logprob, int32_t* choice, float* score, jev_stream_t stream) {
   if (!d) return fail(JEV_ERR_INVALID_ARG, "desc is NULL");
   if (d->n_sets < 0 || d->n_cands < 0 || d->n_pairs < 0 || d->R < 0 || d->V <= 0 || d->H <= 0)
     return fail(JEV_ERR_INVALID_ARG, "negative or zero sizes");
@@ -626,10 +634,38 @@ jev_status jev_candidate_readout(const jev_readout_desc* d, const void* hidden, 
   if ((hidden && !aligned16(hidden)) || (lm_head && !aligned16(lm_head)))
     return fail(JEV_ERR_INVALID_ARG, "hidden / lm_head not 16-byte aligned");
   if (!pair_row && d->R < d->n_sets) return fail(JEV_ERR_INVALID_ARG, "R < n_sets with pair_row NULL");
+  if (row_lse && ((uintptr_t)row_lse & 3)) return fail(JEV_ERR_INVALID_ARG, "row_lse misaligned");
   ReadoutArgs a{hidden, lm_head, set_offsets, cand_offsets, pair_row, pair_tok, logprob, choice, score,
-                d->n_sets, d->n_cands, d->n_pairs, d->R, d->H, d->V};
+                d->n_sets, d->n_cands, d->n_pairs, d->R, d->H, d->V, row_lse};
   const jev_status st = run("readout", (cudaStream_t)stream, [&] { return launch_readout(a, d->dtype, (cudaStream_t)stream); });
   if (st == JEV_OK && d->n_cands > 0) g_launches++;  // candidate scores and set softmax: two kernels
+  return st;
+}
+
+size_t jev_vocab_lse_workspace(int32_t R, int32_t V) {
+  if (R < 0 || V <= 0) return 0;
+  return kStatusBytes + up256(vocab_lse_partial_bytes(R, vocab_lse_ctas(V, num_sms())));
+}
+
+jev_status jev_vocab_lse(const void* hidden, const void* lm_head, int32_t R, int32_t H, int32_t V, jev_dtype dt,
+                         float* lse, void* workspace, size_t ws_bytes, jev_stream_t stream) {
+  if (R < 0 || V <= 0 || H <= 0) return fail(JEV_ERR_INVALID_ARG, "negative or zero sizes");
+  if (dt != JEV_BF16) return fail(JEV_ERR_UNSUPPORTED, "vocab_lse takes bf16 only");
+  if (H % 64) return fail(JEV_ERR_UNSUPPORTED, "hidden size must be a multiple of 64");
+  if (!attn_tc_supported(128)) return fail(JEV_ERR_UNSUPPORTED, "vocab_lse needs an sm_100a device");
+  if (R == 0) return JEV_OK;
+  if (!hidden || !lm_head || !lse) return fail(JEV_ERR_INVALID_ARG, "required pointer is NULL");
+  if (!aligned16(hidden) || !aligned16(lm_head)) return fail(JEV_ERR_INVALID_ARG, "hidden / lm_head not 16-byte aligned");
+  if (((uintptr_t)lse & 3)) return fail(JEV_ERR_INVALID_ARG, "lse misaligned");
+  const size_t need = jev_vocab_lse_workspace(R, V);
+  if (!workspace || ((uintptr_t)workspace & 255)) return fail(JEV_ERR_WORKSPACE, "workspace NULL or not 256-byte aligned");
+  if (ws_bytes < need) return fail(JEV_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", ws_bytes, need);
+  const int n_ctas = vocab_lse_ctas(V, num_sms());
+  char* ws = (char*)workspace;
+  VocabLseArgs a{hidden, lm_head, R, H, V, (V + 255) / 256, (float2*)(ws + kStatusBytes), lse, (int32_t*)ws};
+  const jev_status st =
+      run("vocab_lse", (cudaStream_t)stream, [&] { return launch_vocab_lse(a, n_ctas, (cudaStream_t)stream); });
+  if (st == JEV_OK) g_launches++;  // GEMM + online LSE, then the partial merge: two kernels
   return st;
 }
 

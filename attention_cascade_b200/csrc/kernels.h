@@ -85,8 +85,21 @@ struct ReadoutArgs {
   const int32_t* set_offsets; const int32_t* cand_offsets; const int32_t* pair_row; const int32_t* pair_tok;
   float* logprob; int32_t* choice; float* score;
   int n_sets, n_cands, n_pairs, R, H, V;
+  const float* row_lse;  // [R] or null: each pair's term becomes logit - row_lse[row]
 };
 cudaError_t launch_readout(const ReadoutArgs& a, jev_dtype dt, cudaStream_t s);
+
+// Full-vocabulary log-sum-exp of bf16 hidden rows (vocab_lse.cu).
+struct VocabLseArgs {
+  const void* hidden; const void* lm_head;
+  int R, H, V, n_vtiles;
+  float2* part;  // [ceil(R/256)][n_ctas][2][256] (max, sum) partials, log2 domain
+  float* lse;    // [R] natural log
+  int32_t* status;
+};
+int vocab_lse_ctas(int V, int sms);
+size_t vocab_lse_partial_bytes(int R, int n_ctas);
+cudaError_t launch_vocab_lse(const VocabLseArgs& a, int n_ctas, cudaStream_t s);
 
 cudaError_t launch_rope_inplace(void* x, int L, int H, int d, int pos0, double theta, jev_dtype dt,
                                 cudaStream_t s);

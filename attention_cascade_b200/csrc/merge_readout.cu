@@ -153,6 +153,7 @@ __global__ void __launch_bounds__(kCandWarps * 32) readout_cand_kernel(ReadoutAr
         continue;
       }
       z += row_dot(hid + (size_t)row * a.H, W + (size_t)tok * a.H, a.H, lane);
+      if (a.row_lse && lane == 0) z -= a.row_lse[row];
     }
   }
   z = warp_sum(z);
@@ -202,7 +203,7 @@ __global__ void __launch_bounds__(kCandWarps * 32) readout_cand_wide_kernel(Read
   }
   z = warp_sum(z);
   if (lane == 0) {
-    const float zz = bad ? CUDART_NAN_F : z;
+    const float zz = bad ? CUDART_NAN_F : (a.row_lse ? z - a.row_lse[row] : z);
     a.logprob[c] = zz;
     if (a.score) a.score[c] = zz;
   }
@@ -230,6 +231,7 @@ __global__ void __launch_bounds__(kCandWarps * 32) readout_cand_block_kernel(Rea
         continue;
       }
       z += row_dot(hid + (size_t)row * a.H, W + (size_t)tok * a.H, a.H, lane);
+      if (a.row_lse && lane == 0) z -= a.row_lse[row];
     }
   }
   z = warp_sum(z);

@@ -444,7 +444,21 @@ def diagnostics(dev, jev, torch) -> dict:
     out["readout"] = {"sets": n_sets, "options": opts, "H": cfg.H, "bytes_per_call": nbytes, "us": us,
                       "GBps": nbytes / us / 1e3, "frac_of_hbm": nbytes / us / 1e3 / hbm,
                       "note": "option rows of the LM head gathered from HBM; two kernels (scores, set softmax)"}
-    del W, hidden
+    # ---- full-vocabulary LSE (normalised multi-token scoring): 256 hidden rows against the whole head
+    R_l = 256
+    hl = to_dev(synth.f32_to_bf16_bits(rng.standard_normal((R_l, cfg.H)).astype(np.float32)), dev, torch)
+    lse_l = torch.empty(R_l, dtype=torch.float32, device=dev)
+    ws_l = jev.new_workspace(jev.jev_vocab_lse_workspace(R_l, cfg.V), dev)
+    us_l = graph_us(torch, lambda: jev.jev_vocab_lse(hl, W, lse=lse_l, workspace=ws_l,
+                                                     stream=torch.cuda.current_stream()), stream, 20, 3)
+    lflops = 2 * R_l * cfg.V * cfg.H
+    lpeak = float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"]))
+    out["vocab_lse"] = {"workload": f"{R_l} rows x LM head {cfg.V} x {cfg.H}", "flops_per_call": lflops,
+                        "head_bytes": cfg.V * cfg.H * 2, "us": us_l, "TFLOPs": lflops / us_l / 1e6,
+                        "frac_of_sustained_bf16": lflops / us_l / 1e6 / lpeak,
+                        "head_GBps": cfg.V * cfg.H * 2 / us_l / 1e3,
+                        "note": "GEMM with an on-chip online LSE and the partial merge; no logits in HBM"}
+    del W, hidden, hl, ws_l
     torch.cuda.empty_cache()
     # ---- RoPE pack (and the attention call around it) at the wide shape with 1024 branches
     cw = dataclasses.replace(synth.CONFIGS["c3"], B=1024)
@@ -797,8 +811,8 @@ def jev_arm(args, wl_name):
             mc.free()
             del mc
         line["per_config"] = per
-        if args.diagnostics:
-            line["diagnostics"] = diagnostics(dev, jev, torch)
+    if world == 1 and args.diagnostics:
+        line["diagnostics"] = diagnostics(dev, jev, torch)
 
     if rank == 0 and world == 1 and os.environ.get("JEV_SKIP_CPU_BASELINE") != "1" and isinstance(wl, FlatWorkload) \
             and not isinstance(wl, TreeWorkload):

@@ -237,6 +237,52 @@ jev_status jev_candidate_readout(const jev_readout_desc* desc, const void* hidde
                                  const int32_t* pair_row, const int32_t* pair_tok, float* logprob,
                                  int32_t* choice, float* score, jev_stream_t stream);
 
+/*
+ * Full-vocabulary log-sum-exp (normalised multi-token candidate scoring):
+ *
+ *   lse[r] = log sum_{v < V} exp(hidden[r] . lm_head[v]),   r < R
+ *
+ * the normaliser that turns an unmasked option logit into a log-probability
+ * over the whole vocabulary, log p(tok | r) = hidden[r] . lm_head[tok] -
+ * lse[r] ("How to Deploy Visual Jev ...", Step 3 reads its logits from the
+ * full LM-head projection; FastJEV §3.3 names the vocabulary projection as a
+ * cost of the tree readout).  A candidate of several tokens scored as a
+ * sequence log-probability sums those terms over its teacher-forced pairs.
+ * The product is formed tile by tile on the tensor cores and reduced on
+ * chip: no logit is written to memory.
+ *
+ *   hidden   [R, H] bf16, row-major, 16-byte aligned
+ *   lm_head  [V, H] bf16, row-major, 16-byte aligned
+ *   H        multiple of 64;  R >= 0;  V >= 1
+ *   lse      [R] fp32 DEVICE output
+ *   workspace >= jev_vocab_lse_workspace(R, V) bytes, 256-byte aligned; its
+ *            first 256 bytes hold the device status word (jev_workspace_init
+ *            once, jev_check_device_status to read it).  A pipeline wait
+ *            that gives up sets JEV_DEV_WAIT_TIMEOUT and makes lse NaN.
+ *
+ * bf16 on sm_100a only (JEV_ERR_UNSUPPORTED otherwise); R == 0 enqueues nothing.
+ */
+size_t jev_vocab_lse_workspace(int32_t R, int32_t V);
+jev_status jev_vocab_lse(const void* hidden, const void* lm_head, int32_t R, int32_t H, int32_t V,
+                         jev_dtype dtype, float* lse, void* workspace, size_t ws_bytes, jev_stream_t stream);
+
+/*
+ * jev_candidate_readout_normalized — jev_candidate_readout with every pair's
+ * term normalised over the whole vocabulary: a candidate's score becomes its
+ * sequence log-probability
+ *
+ *   score[c]   = sum over c's pairs (r, tok) of  hidden[r] . lm_head[tok] - row_lse[r]
+ *
+ * and logprob / choice are the log-softmax and argmax of those scores over
+ * each set.  row_lse [R] fp32 DEVICE, normally jev_vocab_lse of the same
+ * hidden rows and head; NULL gives jev_candidate_readout exactly.  Other
+ * arguments and errors as jev_candidate_readout.
+ */
+jev_status jev_candidate_readout_normalized(const jev_readout_desc* desc, const void* hidden, const void* lm_head,
+                                            const int32_t* set_offsets, const int32_t* cand_offsets,
+                                            const int32_t* pair_row, const int32_t* pair_tok, const float* row_lse,
+                                            float* logprob, int32_t* choice, float* score, jev_stream_t stream);
+
 /* ------------------------------------------------------------------------ */
 /* Candidate-prefix tree                                                     */
 /* ------------------------------------------------------------------------ */

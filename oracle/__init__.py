@@ -183,6 +183,35 @@ def candidate_readout(hidden, lm_head, set_offsets, pair_tok, *, cand_offsets=No
     return dict(score=score, logprob=lp, choice=choice, gap=gap, row_lse=row_lse, n_invalid=bad)
 
 
+def vocab_lse(hidden, lm_head, n_threads=0):
+    """Full-vocabulary log-sum-exp of every hidden row, lse[r] = log sum_v
+    exp(hidden[r] . lm_head[v]), in fp64: the normaliser of a log-probability
+    over the whole vocabulary ("How to Deploy Visual Jev ...", Step 3 takes
+    its logits from the full LM-head projection).  Every row is made a used
+    row of a one-candidate readout so the full-vocab pass computes its LSE."""
+    hidden = _c(hidden)
+    R = hidden.shape[0]
+    so = np.arange(R + 1, dtype=np.int32)
+    toks = np.zeros(R, np.int32)
+    return candidate_readout(hidden, lm_head, so, toks, n_threads=n_threads)["row_lse"]
+
+
+def sequence_logprob(hidden, lm_head, cand_offsets, pair_row, pair_tok, n_threads=0):
+    """Normalised score of multi-token candidates: the sum over a candidate's
+    teacher-forced (row, token) pairs of the full-vocabulary log-probability
+    hidden[row] . lm_head[tok] - lse[row].  Returns float64 [n_cands]."""
+    co = _c(cand_offsets, np.int32); prw = _c(pair_row, np.int32); pt = _c(pair_tok, np.int32)
+    n_cands = co.size - 1
+    so = np.array([0, n_cands], np.int32)  # one set: the scores do not depend on the grouping
+    r = candidate_readout(hidden, lm_head, so, pt, cand_offsets=co, pair_row=prw, n_threads=n_threads)
+    lse = r["row_lse"]
+    out = r["score"].copy()
+    for c in range(n_cands):
+        for k in range(int(co[c]), int(co[c + 1])):
+            out[c] -= lse[prw[k]]
+    return out
+
+
 def trie_build(seq_off, toks, root_len: int):
     """Canonical compressed trie; returns a dict of int32 arrays."""
     so = _c(seq_off, np.int32); tk = _c(toks, np.int32)

@@ -128,3 +128,19 @@ def test_position_mode_is_checked_on_the_host(jev):
     assert jev.jev_prefix_suffix_attn_workspace(seq) > 0
     st = jev._lib.jev_tree_attn(C.byref(seq), 3, *([C.c_void_p(16)] * 12), C.c_size_t(1 << 20), None)
     assert st == 1 and jev.jev_launch_count() == n0
+
+
+def test_vocab_lse_host_checks(jev):
+    lib = jev._lib
+    # bf16 only, H a multiple of 64, sizes positive: rejected before any device query or launch
+    assert lib.jev_vocab_lse(None, None, 4, 128, 100, jev.JEV_F32, None, None, 0, None) == 2
+    assert lib.jev_vocab_lse(None, None, 4, 96, 100, jev.JEV_BF16, None, None, 0, None) == 2
+    assert lib.jev_vocab_lse(None, None, -1, 128, 100, jev.JEV_BF16, None, None, 0, None) == 1
+    assert lib.jev_vocab_lse(None, None, 4, 128, 0, jev.JEV_BF16, None, None, 0, None) == 1
+    # workspace grows with the row count; the status word comes first
+    w1, w2 = jev.jev_vocab_lse_workspace(1, 152064), jev.jev_vocab_lse_workspace(600, 152064)
+    assert 256 < w1 < w2
+    assert jev.jev_vocab_lse_workspace(-1, 10) == 0
+    # the normalised readout runs the readout's own checks
+    r = jev.jev_readout_desc(3, 5, 5, 3, 100, 1000, jev.JEV_BF16)
+    assert lib.jev_candidate_readout_normalized(C.byref(r), *([None] * 11)) == 2

@@ -556,3 +556,61 @@ def test_tree_readout_pairs_teacher_forcing():
         # first scored token is predicted from the last question token's row
         assert prow[k] == t["path_row"][a + tc.score_from[c] - 1]
         assert tix[k] == a + tc.score_from[c]
+
+
+# ---------------------------------------------------------------- full-vocabulary LSE (normalised scoring)
+
+def test_vocab_lse_closed_forms():
+    rng = np.random.default_rng(11)
+    R, H, V = 4, 16, 37
+    h = rng.standard_normal((R, H)).astype(np.float32)
+    # all logits zero: log V
+    np.testing.assert_allclose(oracle.vocab_lse(h, np.zeros((V, H), np.float32)), math.log(V), rtol=0, atol=1e-12)
+    # every vocabulary row the same vector w: log V + h . w
+    w = rng.standard_normal(H).astype(np.float32)
+    got = oracle.vocab_lse(h, np.tile(w, (V, 1)))
+    np.testing.assert_allclose(got, math.log(V) + _f64(h) @ _f64(w), rtol=0, atol=1e-10)
+    # one-hot rows: hidden e_j against W = c * I gives one logit c and V - 1 zeros
+    c = 3.5
+    W = (c * np.eye(H)).astype(np.float32)
+    e = np.eye(H, dtype=np.float32)[[0, 5, 15]]
+    np.testing.assert_allclose(oracle.vocab_lse(e, W), math.log(math.exp(c) + H - 1), rtol=0, atol=1e-12)
+
+
+def test_vocab_lse_shift_and_bf16():
+    rng = np.random.default_rng(12)
+    R, H, V = 3, 24, 41
+    h = rng.standard_normal((R, H)).astype(np.float32)
+    W = (0.5 * rng.standard_normal((V, H))).astype(np.float32)
+    a = rng.standard_normal(H).astype(np.float32)
+    # adding one vector to every vocabulary row shifts every logit of row r by h_r . a
+    base = oracle.vocab_lse(h, W)
+    shifted = oracle.vocab_lse(h, (W.astype(np.float64) + a).astype(np.float32))
+    ref_shift = _f64(h) @ _f64(a)
+    # (the float32 rounding of W + a is the only difference)
+    np.testing.assert_allclose(shifted - base, ref_shift, rtol=0, atol=1e-4)
+    # bf16 inputs are widened exactly: same answer as the float32 copy of the bf16 values
+    hb, Wb = synth.f32_to_bf16_bits(h), synth.f32_to_bf16_bits(W)
+    np.testing.assert_allclose(oracle.vocab_lse(hb, Wb), oracle.vocab_lse(_f64(hb).astype(np.float32),
+                                                                           _f64(Wb).astype(np.float32)),
+                               rtol=0, atol=1e-12)
+
+
+def test_sequence_logprob_is_a_distribution_and_adds():
+    rng = np.random.default_rng(13)
+    R, H, V = 2, 8, 19
+    h = rng.standard_normal((R, H)).astype(np.float32)
+    W = rng.standard_normal((V, H)).astype(np.float32)
+    # every one-token continuation of row 0: the probabilities over the vocabulary sum to 1
+    co = np.arange(V + 1, dtype=np.int32)
+    lp = oracle.sequence_logprob(h, W, co, np.zeros(V, np.int32), np.arange(V, dtype=np.int32))
+    assert abs(np.exp(lp).sum() - 1.0) < 1e-12
+    assert np.all(lp < 0)
+    # a two-token candidate scores the sum of its two one-token terms
+    lp2 = oracle.sequence_logprob(h, W, np.array([0, 2, 3, 4], np.int32), np.array([0, 1, 0, 1], np.int32),
+                                  np.array([4, 7, 4, 7], np.int32))
+    assert abs(lp2[0] - (lp2[1] + lp2[2])) < 1e-12
+    # and the all-pairs table of row 1 also normalises
+    lp1 = oracle.sequence_logprob(h, W, co, np.ones(V, np.int32), np.arange(V, dtype=np.int32))
+    assert abs(np.exp(lp1).sum() - 1.0) < 1e-12
+    assert abs(lp2[2] - lp1[7]) < 1e-12 and abs(lp2[1] - lp[4]) < 1e-12
