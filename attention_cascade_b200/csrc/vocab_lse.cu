@@ -62,7 +62,7 @@ __device__ __forceinline__ bool lwait(uint32_t bar, uint32_t parity, volatile in
 
 __global__ void __launch_bounds__(kLThreads, 1)
     vocab_lse_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
-                     const VocabLseArgs a) {
+                     const __grid_constant__ CUtensorMap tm_w16, const VocabLseArgs a) {
   extern __shared__ uint8_t lsm_raw[];
   uint8_t* smem = lsm_raw + ((1024 - (smem_u32(lsm_raw) & 1023)) & 1023);
   const uint32_t sbase = smem_u32(smem);
@@ -72,8 +72,11 @@ __global__ void __launch_bounds__(kLThreads, 1)
                  b_sempty = b_sfull + 8, b_drain = b_sfull + 16;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int cta = blockIdx.x;
-  // this CTA's vocabulary tiles
-  const int nt0 = (int)((long long)cta * a.n_vtiles / gridDim.x), nt1 = (int)((long long)(cta + 1) * a.n_vtiles / gridDim.x);
+  // this CTA's vocabulary rows [v_lo, v_hi): an even share of 16-row slabs, walked in 256-row tiles
+  // whose last one may be narrower (an MMA of N = its rows rounded up to 16)
+  const int n16 = (a.V + 15) / 16;
+  const int v_lo = (int)((long long)cta * n16 / gridDim.x) * 16;
+  const int v_hi = min(a.V, (int)((long long)(cta + 1) * n16 / gridDim.x) * 16);
   const int n_mb = (a.R + 2 * kLM - 1) / (2 * kLM);  // 256-row blocks of hidden rows
   const int nk = a.H / kLK;
 
@@ -95,6 +98,7 @@ __global__ void __launch_bounds__(kLThreads, 1)
   if (warp == kLProducer && lane == 0) {
     tma_prefetch_desc(&tm_x);
     tma_prefetch_desc(&tm_w);
+    tma_prefetch_desc(&tm_w16);
   }
   fence_before_sync();
   __syncthreads();
@@ -109,7 +113,8 @@ __global__ void __launch_bounds__(kLThreads, 1)
       long long it = 0;
       bool ok = true;
       for (int mb = 0; ok && mb < n_mb; ++mb)
-        for (int nt = nt0; ok && nt < nt1; ++nt)
+        for (int v0 = v_lo; ok && v0 < v_hi; v0 += kLN) {
+          const int n_t = (min(kLN, v_hi - v0) + 15) & ~15;  // rows of this tile's W chunk
           for (int kc = 0; ok && kc < nk; ++kc, ++it) {
             const int st = (int)(it % kLStages);
             const long long use = it / kLStages;
@@ -119,22 +124,25 @@ __global__ void __launch_bounds__(kLThreads, 1)
             }
             const uint32_t base = sbase + st * kStageBytes;
             const bool two = mb * 2 * kLM + kLM < a.R;  // the block's second half holds rows
-            mbar_expect_tx(b_full + 8 * st, two ? kStageBytes : kStageBytes - kXBytes);
+            mbar_expect_tx(b_full + 8 * st, (two ? 2 * kXBytes : kXBytes) + n_t * kLK * 2);
             tma_load_2d(base, &tm_x, kc * kLK, mb * 2 * kLM, b_full + 8 * st);
             if (two) tma_load_2d(base + kXBytes, &tm_x, kc * kLK, mb * 2 * kLM + kLM, b_full + 8 * st);
-            tma_load_2d(base + 2 * kXBytes, &tm_w, kc * kLK, nt * kLN, b_full + 8 * st);
-            tma_load_2d(base + 2 * kXBytes + kXBytes, &tm_w, kc * kLK, nt * kLN + kLM, b_full + 8 * st);
+            // 128-row boxes, then 16-row boxes for a narrow tail (row `o` lands at o * 128 bytes)
+            int o = 0;
+            for (; o + kLM <= n_t; o += kLM) tma_load_2d(base + 2 * kXBytes + o * 128, &tm_w, kc * kLK, v0 + o, b_full + 8 * st);
+            for (; o < n_t; o += 16) tma_load_2d(base + 2 * kXBytes + o * 128, &tm_w16, kc * kLK, v0 + o, b_full + 8 * st);
           }
+        }
     }
   } else if (warp == kLMma) {
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16(kLM, kLN, false);
       long long it = 0, tile = 0;
       bool ok = true;
       for (int mb = 0; ok && mb < n_mb; ++mb) {
         const int halves = mb * 2 * kLM + kLM < a.R ? 2 : 1;
-        for (int nt = nt0; ok && nt < nt1; ++nt, ++tile) {
+        for (int v0 = v_lo; ok && v0 < v_hi; v0 += kLN, ++tile) {
+          const uint32_t idesc = idesc_bf16(kLM, (min(kLN, v_hi - v0) + 15) & ~15, false);
           // the statistics threads have read the previous tile out of TMEM
           if (tile > 0 && !lwait(b_sempty, (uint32_t)((tile - 1) & 1), abort, a.status)) {
             ok = false;
@@ -173,18 +181,18 @@ __global__ void __launch_bounds__(kLThreads, 1)
     for (int mb = 0; mb < n_mb; ++mb) {
       const bool live = mb * 2 * kLM + i * kLM < a.R;  // warp-uniform: this half holds rows
       float m_run = -CUDART_INF_F, l_run = 0.f;  // log2 domain
-      for (int nt = nt0; nt < nt1; ++nt, ++tile) {
+      for (int t0 = v_lo; t0 < v_hi; t0 += kLN, ++tile) {
         // warp-uniform (the TMEM loads below are warp-wide instructions); a
         // failed wait runs the remaining tiles on stale TMEM so the loop shape stays uniform
         ok = __all_sync(0xffffffffu, ok && lwait(b_sfull, (uint32_t)(tile & 1), abort, a.status));
         fence_after_sync();
-        const int v0 = nt * kLN + hf * (kLN / 2);  // vocabulary row of this thread's first column
+        const int v0 = t0 + hf * (kLN / 2);  // vocabulary row of this thread's first column
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
-          if (!live) break;
+          const int lim = v_hi - (v0 + c * 64);  // columns past this CTA's rows are padding
+          if (!live || lim <= 0) break;
           uint32_t xs[64];
           tmem_ld64(s_addr + c * 64, xs);
-          const int lim = a.V - (v0 + c * 64);  // columns past the vocabulary are padding
           // four independent max / sum chains
           float mx[4] = {-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F};
 #pragma unroll
@@ -264,11 +272,11 @@ EncodeTiledFnL encode_fn_l() {
 }
 
 // bf16 rows of H elements (H*2 bytes apart), `rows` rows; 64 x 128 boxes, 128-byte swizzle
-bool map_rows(CUtensorMap* m, const void* base, uint64_t H, uint64_t rows) {
+bool map_rows(CUtensorMap* m, const void* base, uint64_t H, uint64_t rows, uint32_t box_rows = 128) {
   if (!encode_fn_l()) return false;
   cuuint64_t dims[2] = {H, rows};
   cuuint64_t strides[1] = {H * 2};
-  cuuint32_t box[2] = {64, 128};
+  cuuint32_t box[2] = {64, box_rows};
   cuuint32_t es[2] = {1, 1};
   return encode_fn_l()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -278,8 +286,8 @@ bool map_rows(CUtensorMap* m, const void* base, uint64_t H, uint64_t rows) {
 }  // namespace
 
 int vocab_lse_ctas(int V, int sms) {
-  const int nt = (V + kLN - 1) / kLN;
-  return std::max(1, std::min(nt, sms));
+  const int n16 = (V + 15) / 16;
+  return std::max(1, std::min(n16, sms));
 }
 
 size_t vocab_lse_partial_bytes(int R, int n_ctas) {
@@ -295,8 +303,9 @@ cudaError_t launch_vocab_lse(const VocabLseArgs& a, int n_ctas, cudaStream_t s) 
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  CUtensorMap mx, mw;
-  if (!map_rows(&mx, a.hidden, (uint64_t)a.H, (uint64_t)a.R) || !map_rows(&mw, a.lm_head, (uint64_t)a.H, (uint64_t)a.V))
+  CUtensorMap mx, mw, mw16;
+  if (!map_rows(&mx, a.hidden, (uint64_t)a.H, (uint64_t)a.R) || !map_rows(&mw, a.lm_head, (uint64_t)a.H, (uint64_t)a.V) ||
+      !map_rows(&mw16, a.lm_head, (uint64_t)a.H, (uint64_t)a.V, 16))
     return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute pdl[1];
@@ -308,7 +317,7 @@ cudaError_t launch_vocab_lse(const VocabLseArgs& a, int n_ctas, cudaStream_t s) 
   cfg.stream = s;
   cfg.attrs = pdl;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, vocab_lse_kernel, mx, mw, a);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, vocab_lse_kernel, mx, mw, mw16, a);
   if (e != cudaSuccess) return e;
   cfg.gridDim = dim3((a.R + 255) / 256);
   cfg.blockDim = dim3(256);

@@ -397,6 +397,7 @@ def load_lm_head(cfg, dev, torch, tdt):
 
 def graph_us(torch, fn, stream, steps: int, warmup: int) -> float:
     """Average device time of fn() replayed from one CUDA graph, after warm-up."""
+    stream.wait_stream(torch.cuda.current_stream())  # inputs were made on the current stream
     with torch.cuda.stream(stream):
         fn()
     stream.synchronize()
@@ -413,6 +414,30 @@ def graph_us(torch, fn, stream, steps: int, warmup: int) -> float:
         a1.record(stream)
     torch.cuda.synchronize()
     return 1e3 * a0.elapsed_time(a1) / steps
+
+
+def diag_vocab_lse(dev, jev, torch, stream, W=None) -> dict:
+    """Full-vocabulary LSE (normalised multi-token scoring): 256 hidden rows
+    against the whole 7B-shaped LM head (152064 x 3584, N(0, 0.02)), graph-replayed."""
+    cfg = synth.CONFIGS["c3"]
+    pk, _ = peaks()
+    if W is None:
+        W = load_lm_head(cfg, dev, torch, torch.bfloat16)
+    rng = np.random.default_rng(8)
+    R_l = 256
+    hl = to_dev(synth.f32_to_bf16_bits(rng.standard_normal((R_l, cfg.H)).astype(np.float32)), dev, torch)
+    lse_l = torch.empty(R_l, dtype=torch.float32, device=dev)
+    ws_l = jev.new_workspace(jev.jev_vocab_lse_workspace(R_l, cfg.V), dev)
+    us_l = graph_us(torch, lambda: jev.jev_vocab_lse(hl, W, lse=lse_l, workspace=ws_l,
+                                                     stream=torch.cuda.current_stream()), stream, 20, 3)
+    flags = jev.jev_check_device_status(ws_l)
+    lflops = 2 * R_l * cfg.V * cfg.H
+    lpeak = float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"]))
+    return {"workload": f"{R_l} rows x LM head {cfg.V} x {cfg.H}", "flops_per_call": lflops,
+            "head_bytes": cfg.V * cfg.H * 2, "us": us_l, "TFLOPs": lflops / us_l / 1e6,
+            "frac_of_sustained_bf16": lflops / us_l / 1e6 / lpeak, "head_GBps": cfg.V * cfg.H * 2 / us_l / 1e3,
+            "device_flags": flags,
+            "note": "GEMM with an on-chip online LSE and the partial merge; no logits in HBM"}
 
 
 def diagnostics(dev, jev, torch) -> dict:
@@ -444,21 +469,8 @@ def diagnostics(dev, jev, torch) -> dict:
     out["readout"] = {"sets": n_sets, "options": opts, "H": cfg.H, "bytes_per_call": nbytes, "us": us,
                       "GBps": nbytes / us / 1e3, "frac_of_hbm": nbytes / us / 1e3 / hbm,
                       "note": "option rows of the LM head gathered from HBM; two kernels (scores, set softmax)"}
-    # ---- full-vocabulary LSE (normalised multi-token scoring): 256 hidden rows against the whole head
-    R_l = 256
-    hl = to_dev(synth.f32_to_bf16_bits(rng.standard_normal((R_l, cfg.H)).astype(np.float32)), dev, torch)
-    lse_l = torch.empty(R_l, dtype=torch.float32, device=dev)
-    ws_l = jev.new_workspace(jev.jev_vocab_lse_workspace(R_l, cfg.V), dev)
-    us_l = graph_us(torch, lambda: jev.jev_vocab_lse(hl, W, lse=lse_l, workspace=ws_l,
-                                                     stream=torch.cuda.current_stream()), stream, 20, 3)
-    lflops = 2 * R_l * cfg.V * cfg.H
-    lpeak = float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"]))
-    out["vocab_lse"] = {"workload": f"{R_l} rows x LM head {cfg.V} x {cfg.H}", "flops_per_call": lflops,
-                        "head_bytes": cfg.V * cfg.H * 2, "us": us_l, "TFLOPs": lflops / us_l / 1e6,
-                        "frac_of_sustained_bf16": lflops / us_l / 1e6 / lpeak,
-                        "head_GBps": cfg.V * cfg.H * 2 / us_l / 1e3,
-                        "note": "GEMM with an on-chip online LSE and the partial merge; no logits in HBM"}
-    del W, hidden, hl, ws_l
+    out["vocab_lse"] = diag_vocab_lse(dev, jev, torch, stream, W)
+    del W, hidden
     torch.cuda.empty_cache()
     # ---- RoPE pack (and the attention call around it) at the wide shape with 1024 branches
     cw = dataclasses.replace(synth.CONFIGS["c3"], B=1024)
@@ -840,11 +852,19 @@ def main():
                     help="skip the other synthetic configs (reported under per_config on one GPU)")
     ap.add_argument("--per-config-steps", type=int, default=2000)
     ap.add_argument("--no-diagnostics", dest="diagnostics", action="store_false",
-                    help="skip the streaming diagnostics at larger sizes (one GPU, with per_config)")
+                    help="skip the streaming diagnostics at larger sizes (one GPU)")
+    ap.add_argument("--diag", choices=["vocab_lse"], default=None,
+                    help="run only this diagnostic on cuda:0 and print its JSON (a small case for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("bench.py: at least 3 warm-up steps")
-    if args.impl == "reference":
+    if args.diag:
+        import torch
+        import attention_cascade_b200 as jev
+        torch.cuda.set_device(0)
+        print(json.dumps({"diagnostic": args.diag,
+                          **diag_vocab_lse("cuda:0", jev, torch, torch.cuda.Stream(device="cuda:0"))}))
+    elif args.impl == "reference":
         reference_arm(args, args.workload)
     else:
         jev_arm(args, args.workload)

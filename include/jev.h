@@ -245,8 +245,9 @@ jev_status jev_candidate_readout(const jev_readout_desc* desc, const void* hidde
  * the normaliser that turns an unmasked option logit into a log-probability
  * over the whole vocabulary, log p(tok | r) = hidden[r] . lm_head[tok] -
  * lse[r] ("How to Deploy Visual Jev ...", Step 3 reads its logits from the
- * full LM-head projection; FastJEV §3.3 names the vocabulary projection as a
- * cost of the tree readout).  A candidate of several tokens scored as a
+ * full LM-head projection; FastJEV, Appendix A (Additional Experimental
+ * Results), counts vocabulary-projection scheduling among the tree path's
+ * costs).  A candidate of several tokens scored as a
  * sequence log-probability sums those terms over its teacher-forced pairs.
  * The product is formed tile by tile on the tensor cores and reduced on
  * chip: no logit is written to memory.

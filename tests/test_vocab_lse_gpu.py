@@ -47,9 +47,11 @@ def _run(jev, h, W):
 
 # (R, H, V, w_scale): rows in one half and in both halves of a 256-row block, a
 # second block holding one row, vocabulary tails of 1 and 255 rows, H of one and
-# of several 64-column chunks, logits of a few units and of ~+-60
+# of several 64-column chunks, logits of a few units and of ~+-60; V = 59200 gives
+# each of 148 CTAs 400 rows: a whole 256-row tile, then a 144-row tile loaded as a
+# 128-row box and a 16-row box
 CASES = [(5, 128, 1000, 0.2, 0), (129, 64, 257, 0.5, 1), (300, 256, 5000, 0.3, 2), (257, 192, 511, 0.1, 3),
-         (64, 512, 2048, 2.5, 4), (1, 64, 1, 1.0, 5)]
+         (64, 512, 2048, 2.5, 4), (1, 64, 1, 1.0, 5), (200, 128, 59200, 0.3, 8)]
 
 
 @pytest.mark.parametrize("R,H,V,w_scale,seed", CASES, ids=[f"v{i}" for i in range(len(CASES))])
