@@ -203,6 +203,14 @@ __device__ __forceinline__ Segment make_segment(const AttnArgs& a, int c, int w,
     n_suf = lo <= hi ? (hi - lo + kBN) / kBN : 0;
   }
   sg.n = sg.n_pre + n_suf;
+  // A segment always has a key tile: the q_empty / p_full handshake that
+  // keeps the roles within one q_full phase of each other runs per key tile.
+  // n would be 0 only for a suffix unit whose rows are all outside the tree
+  // (nanc < 0); its one tile is then fully masked and nothing is written.
+  if (sg.n == 0) {
+    sg.lo = 0;
+    sg.n = 1;
+  }
   sg.complete = sg.ua == 0 && sg.ub == a.P;
   sg.slot = (tail && tc_unit_begin(a, c) >= t0) ? 2 * c : 2 * c + 1;
   return sg;
@@ -381,15 +389,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = wait_bar(B.q_full, k & 1, abort, a.status);
       const Segment sg = seg_sm[k & 1];
       if (lane == 0) {
-        const int n = sg.n;
-        if (ok && n > 0) {
+        const int n = sg.n;  // >= 1
+        if (ok) {
           const int st0 = (int)(J % C::kNS);
           ok = wait_bar(B.k_full + 8 * st0, (uint32_t)((J / C::kNS) & 1), abort, a.status);
           fence_after_sync();
           if (ok) {
             issue_s(0, st0);
             issue_s(1, st0);
-            if (n == 1) mma_commit(B.q_empty);
           }
         }
         for (int j = 0; ok && j < n; ++j) {
@@ -412,15 +419,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           issue_pv(1, st, j > 0);
           mma_commit(B.kv_empty + 8 * st);
           if (j == n - 1) mma_commit(B.o_full + 8);
+          // q_empty releases the Q buffer and lets the producer publish the next
+          // segment.  It is committed only after both p_full waits of a tile of
+          // this segment, i.e. after all 512 softmax threads have passed their
+          // q_full wait for it: were q_full to complete two phases ahead of a
+          // softmax thread still in the previous epilogue, that thread's parity
+          // wait would alias the later phase and never return.
           if (j + 1 < n) {
             issue_s(1, st1);
             if (j + 2 == n) mma_commit(B.q_empty);
+          } else if (n == 1) {
+            mma_commit(B.q_empty);
           }
-        }
-        if (ok && n == 0) {
-          mma_commit(B.q_empty);
-          mma_commit(B.o_full);
-          mma_commit(B.o_full + 8);
         }
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);

@@ -440,6 +440,65 @@ def diag_vocab_lse(dev, jev, torch, stream, W=None) -> dict:
             "note": "GEMM with an on-chip online LSE and the partial merge; no logits in HBM"}
 
 
+def _tree_timer(dev, jev, torch, stream, tc) -> dict:
+    """Graph-replayed time of one jev_tree_attn call over a synthetic trie, with its exact work."""
+    cfg = tc.cfg
+    trie = jev.jev_tree_build(tc.seq_off, tc.toks, cfg.Lp)
+    parent, tok_off, pos0 = (to_dev(trie[k], dev, torch) for k in ("parent", "tok_off", "pos0"))
+    q, kr, vr, k, v = (to_dev(x, dev, torch) for x in (tc.q, tc.k_root, tc.v_root, tc.k, tc.v))
+    N = int(trie["tok_off"][-1])
+    out = torch.empty_like(q)
+    lse = torch.empty((N, cfg.Hq), dtype=torch.float32, device=dev)
+    desc = jev.make_attn_desc(trie["n_nodes"] - 1, cfg.Lp, cfg.Hq, cfg.Hkv, cfg.d, N, jev.JEV_BF16, cfg.theta)
+    ws = jev.new_workspace(jev.jev_tree_attn_workspace(desc, trie["n_nodes"]), dev)
+    us = graph_us(torch, lambda: jev.jev_tree_attn(parent, tok_off, pos0, q, kr, vr, k, v, out=out, lse=lse,
+                                                   workspace=ws, rope_theta=cfg.theta,
+                                                   stream=torch.cuda.current_stream()), stream, 50, 5)
+    pos = np.concatenate([trie["pos0"][n] + np.arange(trie["tok_off"][n + 1] - trie["tok_off"][n])
+                          for n in range(1, trie["n_nodes"])])
+    flops = int(4 * cfg.Hq * cfg.d * (pos.astype(np.int64) + 1).sum())
+    logical = int(tc.seq_off[-1])
+    return {"us": us, "unique_tokens": N, "logical_tokens": logical, "merged_frac": 1 - N / logical,
+            "nodes": int(trie["n_nodes"]), "flops": flops, "TFLOPs": flops / us / 1e6,
+            "device_flags": jev.jev_check_device_status(ws)}
+
+
+def diag_tree_schedule(dev, jev, torch, stream) -> dict:
+    """Tree schedule study at the 7B shape (root / prefix 2048 tokens, Hq 28, Hkv 4, d 128), after
+    FastJEV §4.5 and §A.3: 64 candidates whose content is 75% shared, run as 64 flat branches
+    (no merging) and as a two-level trie (16 questions of 24 tokens, 4 options of 8 tokens each);
+    then a flat trie (64 disjoint 14-token candidates) with the same 896 unique tokens as the
+    two-level trie.  Plus the multi-image variant (Ochevid, "One question, multiple images"):
+    8 images of 400 tokens plus a 16-token question each, 3 one-token options, an empty root."""
+    import dataclasses
+    B, BF = synth.BF16, synth.CONFIGS["c2"]
+    res = {}
+    # 64 flat branches of 32 tokens: 2048 suffix tokens, nothing merged
+    fc = synth.flat_case(dataclasses.replace(BF, B=64), with_lm_head=False, lengths=np.full(64, 32, np.int32))
+    a = [to_dev(x, dev, torch) for x in (fc.q, fc.k_pre, fc.v_pre, fc.k_suf, fc.v_suf)]
+    cu = torch.from_numpy(fc.cu_seqlens).to(dev)
+    desc = jev.make_attn_desc(64, BF.Lp, BF.Hq, BF.Hkv, BF.d, fc.T, jev.JEV_BF16, BF.theta)
+    ws = jev.new_workspace(jev.jev_prefix_suffix_attn_workspace(desc), dev)
+    o = torch.empty_like(a[0])
+    lse = torch.empty((fc.T, BF.Hq), dtype=torch.float32, device=dev)
+    us = graph_us(torch, lambda: jev.jev_prefix_suffix_attn(*a, cu, out=o, lse=lse, workspace=ws, rope_theta=BF.theta,
+                                                            stream=torch.cuda.current_stream()), stream, 50, 5)
+    fl = flat_work(fc)["flops_attn"]
+    res["branches_64x32"] = {"us": us, "unique_tokens": fc.T, "logical_tokens": fc.T, "merged_frac": 0.0,
+                             "flops": fl, "TFLOPs": fl / us / 1e6}
+    two = synth.TreeConfig("two_level", B, BF.Lp, 16, 24, 4, 4, 8, 8, BF.Hq, BF.Hkv, BF.d, BF.H, BF.V, seed=31)
+    res["trie_two_level_16x24_4x8"] = _tree_timer(dev, jev, torch, stream, synth.tree_case(two, with_lm_head=False))
+    flat = synth.TreeConfig("flat_trie", B, BF.Lp, 64, 13, 1, 1, 1, 1, BF.Hq, BF.Hkv, BF.d, BF.H, BF.V, seed=32)
+    res["trie_flat_64x14"] = _tree_timer(dev, jev, torch, stream, synth.tree_case(flat, with_lm_head=False))
+    res["speedup_trie_vs_branches"] = res["branches_64x32"]["us"] / res["trie_two_level_16x24_4x8"]["us"]
+    res["two_level_over_flat_trie_time"] = res["trie_two_level_16x24_4x8"]["us"] / res["trie_flat_64x14"]["us"]
+    mi = synth.TreeConfig("multi_image", B, 0, 8, 416, 3, 3, 1, 1, BF.Hq, BF.Hkv, BF.d, BF.H, BF.V, seed=33)
+    r = _tree_timer(dev, jev, torch, stream, synth.tree_case(mi, with_lm_head=False))
+    r["images_per_s"] = 8 / (r["us"] / 1e6)
+    res["multi_image_8x416"] = r
+    return res
+
+
 def diagnostics(dev, jev, torch) -> dict:
     """Streaming efficiency of the HBM-bound kernels at sizes where it can be
     measured (the configs move kilobytes to a few megabytes per launch, below
@@ -471,6 +530,8 @@ def diagnostics(dev, jev, torch) -> dict:
                       "note": "option rows of the LM head gathered from HBM; two kernels (scores, set softmax)"}
     out["vocab_lse"] = diag_vocab_lse(dev, jev, torch, stream, W)
     del W, hidden
+    torch.cuda.empty_cache()
+    out["tree_schedule"] = diag_tree_schedule(dev, jev, torch, stream)
     torch.cuda.empty_cache()
     # ---- RoPE pack (and the attention call around it) at the wide shape with 1024 branches
     cw = dataclasses.replace(synth.CONFIGS["c3"], B=1024)
@@ -853,7 +914,7 @@ def main():
     ap.add_argument("--per-config-steps", type=int, default=2000)
     ap.add_argument("--no-diagnostics", dest="diagnostics", action="store_false",
                     help="skip the streaming diagnostics at larger sizes (one GPU)")
-    ap.add_argument("--diag", choices=["vocab_lse"], default=None,
+    ap.add_argument("--diag", choices=["vocab_lse", "tree_schedule"], default=None,
                     help="run only this diagnostic on cuda:0 and print its JSON (a small case for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -862,8 +923,8 @@ def main():
         import torch
         import attention_cascade_b200 as jev
         torch.cuda.set_device(0)
-        print(json.dumps({"diagnostic": args.diag,
-                          **diag_vocab_lse("cuda:0", jev, torch, torch.cuda.Stream(device="cuda:0"))}))
+        fn = {"vocab_lse": diag_vocab_lse, "tree_schedule": diag_tree_schedule}[args.diag]
+        print(json.dumps({"diagnostic": args.diag, **fn("cuda:0", jev, torch, torch.cuda.Stream(device="cuda:0"))}))
     elif args.impl == "reference":
         reference_arm(args, args.workload)
     else:

@@ -510,8 +510,11 @@ def _small_tree(seed=0, nq=3, qlen=4, Lp=6, Hq=4, Hkv=2, d=16, V=40, dtype=synth
     return synth.tree_case(cfg, with_lm_head=False)
 
 
-def test_tree_matches_sdpa_on_every_path():
-    tc = _small_tree()
+@pytest.mark.parametrize("Lp", [6, 0])
+def test_tree_matches_sdpa_on_every_path(Lp):
+    # Lp = 0: an empty root, so every first-level node is its own prefix (one question over
+    # several images, each an independent row: Ochevid, "One question, multiple images")
+    tc = _small_tree(Lp=Lp)
     t = oracle.trie_build(tc.seq_off, tc.toks, tc.cfg.Lp)
     assert t["tok_off"][-1] == tc.n_unique
     out, lse = oracle.tree_attn(t, tc.q, tc.k, tc.v, tc.k_root, tc.v_root)

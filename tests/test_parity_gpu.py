@@ -200,6 +200,69 @@ def test_tree_more_nodes_than_the_shared_table(jev):
     check_attn(host_f64(out), host_f64(lse), ref_o, ref_l, cfg.dtype, "tree, many nodes")
 
 
+def test_multi_image_tree(jev):
+    # one question over four images (Ochevid, "One question, multiple images"): an empty root, one
+    # first-level node per image + question (300 tokens, positions 0..299), three one- or two-token
+    # options under each.  Every image row is its own causal problem: against the oracle on every
+    # element, and the first image run alone matches the same oracle rows.
+    cfg = synth.TreeConfig("mi", synth.BF16, 0, 4, 300, 3, 3, 1, 2, 8, 2, 128, 64, 500, seed=21)
+    tc = synth.tree_case(cfg, with_lm_head=False)
+    t, td = _tree_inputs(tc, jev)
+    assert t["n_nodes"] == 1 + 4 + 12 and np.all(t["pos0"][t["parent"] == 0][1:] == 0)
+    out, lse = jev.jev_tree_attn(td["parent"], td["tok_off"], td["pos0"], dev(tc.q), dev(tc.k_root), dev(tc.v_root),
+                                 dev(tc.k), dev(tc.v))
+    ref_o, ref_l = oracle.tree_attn(oracle.trie_build(tc.seq_off, tc.toks, 0), tc.q, tc.k, tc.v, tc.k_root, tc.v_root)
+    check_attn(host_f64(out), host_f64(lse), ref_o, ref_l, cfg.dtype, "multi-image tree")
+    # the first image alone: its candidates are the first set
+    c1 = int(tc.set_offsets[1])
+    so1 = tc.seq_off[:c1 + 1]
+    t1 = jev.jev_tree_build(so1, tc.toks[:so1[-1]], 0)
+    n1 = int(t1["tok_off"][-1])
+    o1, l1 = jev.jev_tree_attn(dev(t1["parent"]), dev(t1["tok_off"]), dev(t1["pos0"]), dev(tc.q[:n1]),
+                               dev(tc.k_root), dev(tc.v_root), dev(tc.k[:n1]), dev(tc.v[:n1]))
+    check_attn(host_f64(o1), host_f64(l1), ref_o[:n1], ref_l[:n1], cfg.dtype, "first image alone")
+
+
+def test_single_key_tile_segments_keep_the_pipeline_in_step(jev):
+    # Schedules whose CTAs run a segment of one key tile followed by more segments: 64 branches
+    # of 32 tokens over a 2048-token prefix at the 7B heads (a one-unit tail segment), and a
+    # multi-image tree (empty root, 8 nodes of 416 tokens: many one-tile windows).  The MMA warp
+    # may release the Q buffer for the next segment only after every softmax thread has passed
+    # this segment's q_full wait; otherwise a softmax thread still in the previous epilogue waits
+    # on an aliased phase.  Five back-to-back calls on one workspace must leave the status word
+    # clear, and sampled rows match the oracle.
+    import dataclasses
+    cfg = dataclasses.replace(synth.CONFIGS["c2"], B=64)
+    c = synth.flat_case(cfg, with_lm_head=False, lengths=np.full(64, 32, np.int32))
+    desc = jev.make_attn_desc(64, cfg.Lp, cfg.Hq, cfg.Hkv, cfg.d, c.T, jev.JEV_BF16, cfg.theta)
+    plan = jev.jev_prefix_suffix_attn_plan(desc, 1, 148)
+    assert plan["full_waves"] >= 1 and plan["tail_ctas"] < plan["n_ctas"]
+    ws = jev.new_workspace(jev.jev_prefix_suffix_attn_workspace(desc), "cuda")
+    q, kp, vp, ks, vs = (dev(x) for x in (c.q, c.k_pre, c.v_pre, c.k_suf, c.v_suf))
+    cu = dev(c.cu_seqlens)
+    for _ in range(5):
+        out, lse = jev.jev_prefix_suffix_attn(q, kp, vp, ks, vs, cu, workspace=ws, rope_theta=cfg.theta)
+    assert jev.jev_check_device_status(ws) == 0
+    rows = _sample_rows(c, 256, 17)
+    ref_o, ref_l = oracle.prefix_suffix_attn(c.q, c.k_pre, c.v_pre, c.k_suf, c.v_suf, c.cu_seqlens, rows=rows)
+    o, l = host_f64(out), host_f64(lse)
+    check_attn(o[rows[:, 0], rows[:, 1]], l[rows[:, 0], rows[:, 1]], ref_o, ref_l, cfg.dtype, "64 x 32 branches")
+
+    BF = synth.CONFIGS["c2"]
+    mi = synth.TreeConfig("mi8", synth.BF16, 0, 8, 416, 3, 3, 1, 1, BF.Hq, BF.Hkv, BF.d, 64, 500, seed=33)
+    tc = synth.tree_case(mi, with_lm_head=False)
+    t, td = _tree_inputs(tc, jev)
+    N = int(t["tok_off"][-1])
+    tdesc = jev.make_attn_desc(t["n_nodes"] - 1, 0, BF.Hq, BF.Hkv, BF.d, N, jev.JEV_BF16, 1e4)
+    tws = jev.new_workspace(jev.jev_tree_attn_workspace(tdesc, t["n_nodes"]), "cuda")
+    tq, tkr, tvr, tk, tv = (dev(x) for x in (tc.q, tc.k_root, tc.v_root, tc.k, tc.v))
+    for _ in range(5):
+        out, lse = jev.jev_tree_attn(td["parent"], td["tok_off"], td["pos0"], tq, tkr, tvr, tk, tv, workspace=tws)
+    assert jev.jev_check_device_status(tws) == 0
+    ref_o, ref_l = oracle.tree_attn(oracle.trie_build(tc.seq_off, tc.toks, 0), tc.q, tc.k, tc.v, tc.k_root, tc.v_root)
+    check_attn(host_f64(out), host_f64(lse), ref_o, ref_l, mi.dtype, "8-image tree")
+
+
 def test_tree_config_c4(jev):
     cfg = synth.CONFIGS["c4"]
     tc = synth.tree_case(cfg, with_lm_head=False)
