@@ -118,6 +118,9 @@ int num_sms() {
   return sms;
 }
 
+// The tcgen05 / TMA kernels run on an sm_100a device with the tensor-map encoder available.
+bool tcgen05_device() { return attn_tc_supported(128); }
+
 bool use_tc(const jev_attn_desc* d) {
   static int forced = -1;
   if (forced < 0) {
@@ -652,7 +655,7 @@ jev_status jev_vocab_lse(const void* hidden, const void* lm_head, int32_t R, int
   if (R < 0 || V <= 0 || H <= 0) return fail(JEV_ERR_INVALID_ARG, "negative or zero sizes");
   if (dt != JEV_BF16) return fail(JEV_ERR_UNSUPPORTED, "vocab_lse takes bf16 only");
   if (H % 64) return fail(JEV_ERR_UNSUPPORTED, "hidden size must be a multiple of 64");
-  if (!attn_tc_supported(128)) return fail(JEV_ERR_UNSUPPORTED, "vocab_lse needs an sm_100a device");
+  if (!tcgen05_device()) return fail(JEV_ERR_UNSUPPORTED, "vocab_lse needs an sm_100a device");
   if (R == 0) return JEV_OK;
   if (!hidden || !lm_head || !lse) return fail(JEV_ERR_INVALID_ARG, "required pointer is NULL");
   if (!aligned16(hidden) || !aligned16(lm_head)) return fail(JEV_ERR_INVALID_ARG, "hidden / lm_head not 16-byte aligned");
