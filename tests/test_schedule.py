@@ -8,6 +8,8 @@ every split tile merged from exactly the slots its CTAs wrote, and no slot
 may fall outside the workspace's two partial rows per CTA."""
 import itertools
 
+import numpy as np
+
 import pytest
 
 import attention_cascade_b200 as jev
@@ -117,3 +119,30 @@ def test_plan_query_rejects_bad_arguments():
     # the CUDA-core plan: prefix splits of whole 128-key tiles covering Lp
     p = jev.jev_prefix_suffix_attn_plan(jev.make_attn_desc(2, 1000, 8, 2, 128, 10, jev.JEV_F32, num_splits=3), 0)
     assert p["kernel"] == 0 and p["split_len"] % 128 == 0 and p["simt_splits"] * p["split_len"] >= 1000
+
+
+def test_tree_schedule_study_inputs():
+    """The tree schedule study's synthetic candidate sets (bench.py diag_tree_schedule) have the
+    properties the study is about: 75% of each two-level candidate's tokens lie in its question,
+    the two-level and flat tries pack the same number of unique tokens, and the multi-image
+    tree has one first-level node per image with an empty root."""
+    import synth
+    import oracle
+    BF = synth.CONFIGS["c2"]
+    two = synth.tree_case(synth.TreeConfig("two_level", synth.BF16, BF.Lp, 16, 24, 4, 4, 8, 8, BF.Hq, BF.Hkv,
+                                           BF.d, BF.H, BF.V, seed=31), with_lm_head=False)
+    flat = synth.tree_case(synth.TreeConfig("flat_trie", synth.BF16, BF.Lp, 64, 13, 1, 1, 1, 1, BF.Hq, BF.Hkv,
+                                            BF.d, BF.H, BF.V, seed=32), with_lm_head=False)
+    mi = synth.tree_case(synth.TreeConfig("multi_image", synth.BF16, 0, 8, 416, 3, 3, 1, 1, BF.Hq, BF.Hkv,
+                                          BF.d, BF.H, BF.V, seed=33), with_lm_head=False)
+    t2 = oracle.trie_build(two.seq_off, two.toks, BF.Lp)
+    tf = oracle.trie_build(flat.seq_off, flat.toks, BF.Lp)
+    tm = oracle.trie_build(mi.seq_off, mi.toks, 0)
+    lens = np.diff(two.seq_off)
+    assert two.seq_off.size - 1 == 64 and np.all(lens == 32) and np.all(two.score_from == 24)  # 24 of 32 shared
+    assert int(t2["tok_off"][-1]) == int(tf["tok_off"][-1]) == 896
+    assert int(two.seq_off[-1]) == 2048 and int(flat.seq_off[-1]) == 896
+    assert t2["n_nodes"] == 1 + 16 + 64 and np.all(tf["parent"][1:] == 0) and tf["n_nodes"] == 65
+    first = np.nonzero(tm["parent"] == 0)[0]
+    assert first.size == 8 and np.all(tm["pos0"][first] == 0)
+    assert np.all(np.diff(tm["tok_off"])[first] == 416) and int(tm["tok_off"][-1]) == 3352
