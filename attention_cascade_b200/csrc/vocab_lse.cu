@@ -251,7 +251,7 @@ __global__ void __launch_bounds__(256) vocab_lse_merge_kernel(const VocabLseArgs
   a.lse[row] = nan ? CUDART_NAN_F : (m + log2f(l)) * 0.69314718055994531f;
 }
 
-// The driver's tensor-map encoder, looked up once through the runtime (the
+// cuTensorMapEncodeTiled from the CUDA driver API, looked up once through the runtime (the
 // attention kernels' translation unit keeps its own copy of this lookup).
 typedef CUresult (*EncodeTiledFnL)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
