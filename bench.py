@@ -8,7 +8,7 @@ tokens/s.  Steps are replayed from CUDA graphs over rotating copies of the
 inputs whose total size exceeds twice the L2, so every step reads its prefix
 cache and suffix tensors from HBM.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c1] [--impl jev|reference]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload qwen2vl_2b] [--impl jev|reference]
 
 With N > 1 (torchrun) every rank runs an independent replica of the workload
 on its own GPU (no collective on the data path; weak scaling); the step time
@@ -419,7 +419,7 @@ def graph_us(torch, fn, stream, steps: int, warmup: int) -> float:
 def diag_vocab_lse(dev, jev, torch, stream, W=None) -> dict:
     """Full-vocabulary LSE (normalised multi-token scoring): 256 hidden rows
     against the whole 7B-shaped LM head (152064 x 3584, N(0, 0.02)), graph-replayed."""
-    cfg = synth.CONFIGS["c3"]
+    cfg = synth.CONFIGS["wide_7b"]
     pk, _ = peaks()
     if W is None:
         W = load_lm_head(cfg, dev, torch, torch.bfloat16)
@@ -471,7 +471,7 @@ def diag_tree_schedule(dev, jev, torch, stream) -> dict:
     two-level trie.  Plus the multi-image variant (Ochevid, "One question, multiple images"):
     8 images of 400 tokens plus a 16-token question each, 3 one-token options, an empty root."""
     import dataclasses
-    B, BF = synth.BF16, synth.CONFIGS["c2"]
+    B, BF = synth.BF16, synth.CONFIGS["qwen25vl_7b"]
     res = {}
     # 64 flat branches of 32 tokens: 2048 suffix tokens, nothing merged
     fc = synth.flat_case(dataclasses.replace(BF, B=64), with_lm_head=False, lengths=np.full(64, 32, np.int32))
@@ -511,7 +511,7 @@ def diagnostics(dev, jev, torch) -> dict:
     out = {"peak_hbm_GBps": hbm, "peak_source": src}
     stream = torch.cuda.Stream(device=dev)
     # ---- readout
-    cfg = synth.CONFIGS["c3"]
+    cfg = synth.CONFIGS["wide_7b"]
     W = load_lm_head(cfg, dev, torch, torch.bfloat16)
     n_sets, opts = 4096, 9
     rng = np.random.default_rng(7)
@@ -534,7 +534,7 @@ def diagnostics(dev, jev, torch) -> dict:
     out["tree_schedule"] = diag_tree_schedule(dev, jev, torch, stream)
     torch.cuda.empty_cache()
     # ---- RoPE pack (and the attention call around it) at the wide shape with 1024 branches
-    cw = dataclasses.replace(synth.CONFIGS["c3"], B=1024)
+    cw = dataclasses.replace(synth.CONFIGS["wide_7b"], B=1024)
     c = synth.flat_case(cw, with_lm_head=False)
     args_ = [to_dev(x, dev, torch) for x in (c.q, c.k_pre, c.v_pre, c.k_suf, c.v_suf)]
     cu = torch.from_numpy(c.cu_seqlens).to(dev)
@@ -907,7 +907,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20000)
     ap.add_argument("--warmup", type=int, default=200)
-    ap.add_argument("--workload", default="c1", choices=sorted(synth.CONFIGS))
+    ap.add_argument("--workload", default="qwen2vl_2b", choices=sorted(synth.CONFIGS))
     ap.add_argument("--impl", default="jev", choices=["jev", "reference"])
     ap.add_argument("--no-per-config", dest="per_config", action="store_false",
                     help="skip the other synthetic configs (reported under per_config on one GPU)")

@@ -9,11 +9,11 @@ LM-head weight, can be regenerated on its own.
 
 Workload shapes follow the five synthetic configurations of the hot path:
 
-* c0  tiny fp32   Lp=256,  B=4,   Ls=16,        Hq=2,  Hkv=1, d=64,  H=256,  V=1024,   3 options
-* c1  2B-shaped   Lp=1024, B=8,   Ls~U[8,24],   Hq=12, Hkv=2, d=128, H=1536, V=151936, U[3,9] options
-* c2  7B-shaped   Lp=2048, B=32,  Ls~U[12,32],  Hq=28, Hkv=4, d=128, H=3584, V=152064, U[2,3] options
-* c3  wide        Lp=4096, B=128, Ls~U[8,40],   Hq=28, Hkv=4, d=128, H=3584, V=152064, 3 options
-* c4  tree        root Lp=2048; 16 question nodes of 24 tokens, each with U[3,9]
+* tiny_f32     tiny fp32   Lp=256,  B=4,   Ls=16,        Hq=2,  Hkv=1, d=64,  H=256,  V=1024,   3 options
+* qwen2vl_2b   2B-shaped   Lp=1024, B=8,   Ls~U[8,24],   Hq=12, Hkv=2, d=128, H=1536, V=151936, U[3,9] options
+* qwen25vl_7b  7B-shaped   Lp=2048, B=32,  Ls~U[12,32],  Hq=28, Hkv=4, d=128, H=3584, V=152064, U[2,3] options
+* wide_7b      wide        Lp=4096, B=128, Ls~U[8,40],   Hq=28, Hkv=4, d=128, H=3584, V=152064, 3 options
+* tree_7b      tree        root Lp=2048; 16 question nodes of 24 tokens, each with U[3,9]
                   option leaves of U[1,4] tokens (distinct first tokens among
                   siblings); Hq=28, Hkv=4, d=128; readout H=3584, V=152064.
 
@@ -104,19 +104,19 @@ class TreeConfig:
 
 
 CONFIGS = {
-    "c0": FlatConfig("c0", F32, 256, 4, 16, 16, 2, 1, 64, 256, 1024, 3, 3, seed=0),
-    "c1": FlatConfig("c1", BF16, 1024, 8, 8, 24, 12, 2, 128, 1536, 151936, 3, 9, seed=1),
-    "c2": FlatConfig("c2", BF16, 2048, 32, 12, 32, 28, 4, 128, 3584, 152064, 2, 3, seed=2),
-    "c3": FlatConfig("c3", BF16, 4096, 128, 8, 40, 28, 4, 128, 3584, 152064, 3, 3, seed=3),
-    "c4": TreeConfig("c4", BF16, 2048, 16, 24, 3, 9, 1, 4, 28, 4, 128, 3584, 152064, seed=4),
+    "tiny_f32": FlatConfig("tiny_f32", F32, 256, 4, 16, 16, 2, 1, 64, 256, 1024, 3, 3, seed=0),
+    "qwen2vl_2b": FlatConfig("qwen2vl_2b", BF16, 1024, 8, 8, 24, 12, 2, 128, 1536, 151936, 3, 9, seed=1),
+    "qwen25vl_7b": FlatConfig("qwen25vl_7b", BF16, 2048, 32, 12, 32, 28, 4, 128, 3584, 152064, 2, 3, seed=2),
+    "wide_7b": FlatConfig("wide_7b", BF16, 4096, 128, 8, 40, 28, 4, 128, 3584, 152064, 3, 3, seed=3),
+    "tree_7b": TreeConfig("tree_7b", BF16, 2048, 16, 24, 3, 9, 1, 4, 28, 4, 128, 3584, 152064, seed=4),
 }
 
 WORKLOAD_TEXT = {
-    "c0": "tiny fp32: Lp=256, B=4, Ls=16, Hq=2, Hkv=1, d=64; readout H=256, V=1024, 3 options/branch",
-    "c1": "2B-shaped bf16: Lp=1024, B=8, Ls~U[8,24], Hq=12, Hkv=2, d=128; readout H=1536, V=151936, 3-9 options/branch",
-    "c2": "7B-shaped bf16: Lp=2048, B=32, Ls~U[12,32], Hq=28, Hkv=4, d=128; readout H=3584, V=152064, 2-3 options/branch",
-    "c3": "wide bf16: Lp=4096, B=128, Ls~U[8,40], Hq=28, Hkv=4, d=128; readout H=3584, V=152064, 3 options/branch",
-    "c4": "tree bf16: root Lp=2048; 16 question nodes x 24 tokens, 3-9 option leaves of 1-4 tokens each; Hq=28, Hkv=4, d=128; readout H=3584, V=152064 per leaf over its siblings",
+    "tiny_f32": "tiny fp32: Lp=256, B=4, Ls=16, Hq=2, Hkv=1, d=64; readout H=256, V=1024, 3 options/branch",
+    "qwen2vl_2b": "2B-shaped bf16: Lp=1024, B=8, Ls~U[8,24], Hq=12, Hkv=2, d=128; readout H=1536, V=151936, 3-9 options/branch",
+    "qwen25vl_7b": "7B-shaped bf16: Lp=2048, B=32, Ls~U[12,32], Hq=28, Hkv=4, d=128; readout H=3584, V=152064, 2-3 options/branch",
+    "wide_7b": "wide bf16: Lp=4096, B=128, Ls~U[8,40], Hq=28, Hkv=4, d=128; readout H=3584, V=152064, 3 options/branch",
+    "tree_7b": "tree bf16: root Lp=2048; 16 question nodes x 24 tokens, 3-9 option leaves of 1-4 tokens each; Hq=28, Hkv=4, d=128; readout H=3584, V=152064 per leaf over its siblings",
 }
 
 

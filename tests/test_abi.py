@@ -88,7 +88,7 @@ def test_tree_build_matches_oracle_bitwise(jev):
 
 def test_tree_build_on_tree_workload(jev):
     import synth
-    tc = synth.tree_case(synth.CONFIGS["c4"], with_lm_head=False)
+    tc = synth.tree_case(synth.CONFIGS["tree_7b"], with_lm_head=False)
     a = jev.jev_tree_build(tc.seq_off, tc.toks, tc.cfg.Lp)
     b = oracle.trie_build(tc.seq_off, tc.toks, tc.cfg.Lp)
     for k in ("parent", "tok_off", "pos0", "leaf_of", "node_toks", "path_row"):

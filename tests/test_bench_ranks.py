@@ -68,5 +68,5 @@ def test_reference_arm_prints_only_on_rank_0(monkeypatch):
     monkeypatch.setenv("RANK", "1")
     buf = io.StringIO()
     with redirect_stdout(buf):
-        bench.reference_arm(Args, "c1")
+        bench.reference_arm(Args, "qwen2vl_2b")
     assert buf.getvalue() == ""

@@ -1,9 +1,9 @@
 """GPU parity: the CUDA path through the C ABI against the fp64 oracle on the
 same seeded inputs, element by element.
 
-* c0 and c1 are compared on every output element (c1 readout against the
+* tiny_f32 and qwen2vl_2b are compared on every output element (the qwen2vl_2b readout against the
   oracle's full-vocabulary logits, the pages' plain definition).
-* c2 and c3 run at full size in the launch configuration bench.py times
+* qwen25vl_7b and wide_7b run at full size in the launch configuration bench.py times
   (automatic split count, default kernel) and are compared on sampled rows the
   oracle forms one by one: every branch's first and last token at every head
   plus random rows; the readout is compared on every set.
@@ -48,7 +48,7 @@ def run_readout(jev, hidden, W_dev, so, toks, **kw):
     return lp.cpu().numpy().astype(np.float64), ch.cpu().numpy()
 
 
-@pytest.mark.parametrize("name", ["c0", "c1"])
+@pytest.mark.parametrize("name", ["tiny_f32", "qwen2vl_2b"])
 def test_flat_config_every_element(jev, name):
     cfg = synth.CONFIGS[name]
     c = synth.flat_case(cfg)
@@ -73,7 +73,7 @@ def _sample_rows(c, n_random, seed):
     return np.array(rows, np.int32)
 
 
-@pytest.mark.parametrize("name", ["c2", "c3"])
+@pytest.mark.parametrize("name", ["qwen25vl_7b", "wide_7b"])
 def test_flat_config_full_size_sampled(jev, name):
     cfg = synth.CONFIGS[name]
     c = synth.flat_case(cfg, with_lm_head=False)
@@ -232,7 +232,7 @@ def test_single_key_tile_segments_keep_the_pipeline_in_step(jev):
     # on an aliased phase.  Five back-to-back calls on one workspace must leave the status word
     # clear, and sampled rows match the oracle.
     import dataclasses
-    cfg = dataclasses.replace(synth.CONFIGS["c2"], B=64)
+    cfg = dataclasses.replace(synth.CONFIGS["qwen25vl_7b"], B=64)
     c = synth.flat_case(cfg, with_lm_head=False, lengths=np.full(64, 32, np.int32))
     desc = jev.make_attn_desc(64, cfg.Lp, cfg.Hq, cfg.Hkv, cfg.d, c.T, jev.JEV_BF16, cfg.theta)
     plan = jev.jev_prefix_suffix_attn_plan(desc, 1, 148)
@@ -248,7 +248,7 @@ def test_single_key_tile_segments_keep_the_pipeline_in_step(jev):
     o, l = host_f64(out), host_f64(lse)
     check_attn(o[rows[:, 0], rows[:, 1]], l[rows[:, 0], rows[:, 1]], ref_o, ref_l, cfg.dtype, "64 x 32 branches")
 
-    BF = synth.CONFIGS["c2"]
+    BF = synth.CONFIGS["qwen25vl_7b"]
     mi = synth.TreeConfig("mi8", synth.BF16, 0, 8, 416, 3, 3, 1, 1, BF.Hq, BF.Hkv, BF.d, 64, 500, seed=33)
     tc = synth.tree_case(mi, with_lm_head=False)
     t, td = _tree_inputs(tc, jev)
@@ -263,8 +263,8 @@ def test_single_key_tile_segments_keep_the_pipeline_in_step(jev):
     check_attn(host_f64(out), host_f64(lse), ref_o, ref_l, mi.dtype, "8-image tree")
 
 
-def test_tree_config_c4(jev):
-    cfg = synth.CONFIGS["c4"]
+def test_tree_config_tree_7b(jev):
+    cfg = synth.CONFIGS["tree_7b"]
     tc = synth.tree_case(cfg, with_lm_head=False)
     t, td = _tree_inputs(tc, jev)
     out, lse = jev.jev_tree_attn(td["parent"], td["tok_off"], td["pos0"], dev(tc.q), dev(tc.k_root), dev(tc.v_root),
@@ -272,14 +272,14 @@ def test_tree_config_c4(jev):
     torch.cuda.synchronize()
     ref_o, ref_l = oracle.tree_attn(oracle.trie_build(tc.seq_off, tc.toks, cfg.Lp), tc.q, tc.k, tc.v,
                                     tc.k_root, tc.v_root)
-    check_attn(host_f64(out), host_f64(lse), ref_o, ref_l, cfg.dtype, "c4 tree")
+    check_attn(host_f64(out), host_f64(lse), ref_o, ref_l, cfg.dtype, "tree_7b")
     plan = jev.jev_tree_readout_plan(tc.seq_off, tc.toks, tc.score_from, t["path_row"])
     Wd, Wrows, inv = compact_lm_head(cfg, plan["pair_tok"])
     ref = oracle.candidate_readout(tc.hidden, Wrows, tc.set_offsets, inv, cand_offsets=plan["cand_offsets"],
                                    pair_row=plan["pair_row"], full_vocab=False)
     lp, ch = run_readout(jev, tc.hidden, Wd, tc.set_offsets, plan["pair_tok"], cand_offsets=plan["cand_offsets"],
                          pair_row=plan["pair_row"])
-    check_readout(lp, ch, ref, cfg.dtype, "c4 readout")
+    check_readout(lp, ch, ref, cfg.dtype, "tree_7b readout")
 
 
 @pytest.mark.parametrize("lens,S,d,dtype", [([50, 1, 130, 77, 200], 128, 128, synth.BF16),

@@ -128,7 +128,7 @@ def test_tree_schedule_study_inputs():
     tree has one first-level node per image with an empty root."""
     import synth
     import oracle
-    BF = synth.CONFIGS["c2"]
+    BF = synth.CONFIGS["qwen25vl_7b"]
     two = synth.tree_case(synth.TreeConfig("two_level", synth.BF16, BF.Lp, 16, 24, 4, 4, 8, 8, BF.Hq, BF.Hkv,
                                            BF.d, BF.H, BF.V, seed=31), with_lm_head=False)
     flat = synth.tree_case(synth.TreeConfig("flat_trie", synth.BF16, BF.Lp, 64, 13, 1, 1, 1, 1, BF.Hq, BF.Hkv,

@@ -7,7 +7,7 @@ import synth
 
 
 def test_flat_case_is_deterministic_and_shaped():
-    cfg = synth.scaled(synth.CONFIGS["c1"], V=4096, H=64)
+    cfg = synth.scaled(synth.CONFIGS["qwen2vl_2b"], V=4096, H=64)
     a = synth.flat_case(cfg)
     b = synth.flat_case(cfg)
     for x, y in ((a.q, b.q), (a.k_pre, b.k_pre), (a.W, b.W), (a.pair_tok, b.pair_tok), (a.cu_seqlens, b.cu_seqlens)):
@@ -23,7 +23,7 @@ def test_flat_case_is_deterministic_and_shaped():
 
 
 def test_full_config_lengths():
-    for name, lo, hi, B in (("c2", 12, 32, 32), ("c3", 8, 40, 128)):
+    for name, lo, hi, B in (("qwen25vl_7b", 12, 32, 32), ("wide_7b", 8, 40, 128)):
         Ls = synth.suffix_lengths(synth.CONFIGS[name])
         assert Ls.size == B and Ls.min() >= lo and Ls.max() <= hi
 
@@ -43,7 +43,7 @@ def test_bf16_rounding_matches_torch():
 
 
 def test_tree_case_structure():
-    tc = synth.tree_case(synth.CONFIGS["c4"], with_lm_head=False)
+    tc = synth.tree_case(synth.CONFIGS["tree_7b"], with_lm_head=False)
     assert tc.set_offsets.size == 17
     nleaf = np.diff(tc.set_offsets)
     assert nleaf.min() >= 3 and nleaf.max() <= 9
