@@ -146,3 +146,33 @@ def test_tree_schedule_study_inputs():
     first = np.nonzero(tm["parent"] == 0)[0]
     assert first.size == 8 and np.all(tm["pos0"][first] == 0)
     assert np.all(np.diff(tm["tok_off"])[first] == 416) and int(tm["tok_off"][-1]) == 3352
+
+
+@pytest.mark.parametrize("V", [1, 15, 16, 17, 255, 257, 5000, 59200, 151936, 152064])
+@pytest.mark.parametrize("R", [1, 128, 129, 256, 300, 1024])
+def test_vocab_lse_partition_and_workspace(R, V):
+    """The full-vocabulary LSE kernel's work split, as its CTAs derive it: CTA c of n owns
+    vocabulary rows [c*n16/n*16, min(V, (c+1)*n16/n*16)) (n16 = 16-row granules), walked in
+    256-row tiles whose MMA width is the tile's rows rounded up to 16.  Every row is owned once,
+    every MMA width is a legal N (16..256, step 16), and every (max, sum) partial the CTAs write,
+    [row block][CTA][column half][256 rows], fits the workspace the library asks for after its
+    256-byte status word."""
+    # the SM count the library plans for (the device's, or 148 without one): a problem with
+    # many whole-tile waves gets one persistent CTA per SM
+    big = jev.make_attn_desc(1024, 4096, 28, 4, 128, 24000, jev.JEV_BF16)
+    sms = jev.jev_prefix_suffix_attn_plan(big, 1, 0)["n_ctas"]
+    n16 = -(-V // 16)
+    n = max(1, min(n16, sms))
+    owned = np.zeros(V, np.int32)
+    for c in range(n):
+        lo = c * n16 // n * 16
+        hi = min(V, (c + 1) * n16 // n * 16)
+        assert hi > lo
+        owned[lo:hi] += 1
+        for v0 in range(lo, hi, 256):
+            width = -(-min(256, hi - v0) // 16) * 16
+            assert 16 <= width <= 256 and width % 16 == 0
+    assert np.all(owned == 1)
+    n_mb = -(-R // 256)
+    last = (((n_mb - 1) * n + (n - 1)) * 2 + 1) * 256 + 255  # largest partial index
+    assert 256 + (last + 1) * 8 <= jev.jev_vocab_lse_workspace(R, V)
