@@ -34,14 +34,19 @@ class Bar:
         self.count, self.pending, self.phase = count, 0, 0
 
 
-def producer(segs):
+def producer(segs, pre0=0):
+    # pre0: the first segment's leading prefix tiles, loaded into stages 0 .. pre0-1 before
+    # anything else (before the kernel's wait on the previous launch and before the first Q)
+    for j in range(pre0):
+        yield ("arrive", f"k_full{j}")
+        yield ("arrive", f"v_full{j}")
     J = 0
     for k, n in enumerate(segs):
         if k > 0:
             yield ("wait", "q_empty", k - 1)
         yield ("arrive", "q_full")
         yield ("arrive", "q_full")
-        for j in range(n):
+        for j in range(pre0 if k == 0 else 0, n):
             JJ = J + j
             st = JJ % NS
             if JJ >= NS:
@@ -102,14 +107,14 @@ def softmax(segs, i):
 SOFT = 2  # softmax threads per tile group in the model
 
 
-def run(segs, early_release, seed):
+def run(segs, early_release, seed, pre0=0):
     """Returns None when every role finishes cleanly, else a description."""
     bars = {"q_full": Bar(2), "q_empty": Bar(1), "s_full0": Bar(1), "s_full1": Bar(1),
             "p_full0": Bar(SOFT), "p_full1": Bar(SOFT), "o_full0": Bar(1), "o_full1": Bar(1)}
     for s in range(NS):
         for b in ("k_full", "v_full", "kv_empty"):
             bars[f"{b}{s}"] = Bar(1)
-    threads = {"producer": producer(segs), "mma": mma(segs, early_release)}
+    threads = {"producer": producer(segs, pre0), "mma": mma(segs, early_release)}
     for i in range(2):
         for t in range(SOFT):
             threads[f"soft{i}.{t}"] = softmax(segs, i)
@@ -177,10 +182,12 @@ def run(segs, early_release, seed):
 PATTERNS = [[17, 9], [17, 8, 1], [3, 1, 2], [1, 1, 1, 1], [2, 1, 1, 3], [4, 1, 4, 1], [1, 2], [5]]
 
 
+@pytest.mark.parametrize("prefetch", [False, True])
 @pytest.mark.parametrize("segs", PATTERNS, ids=["-".join(map(str, p)) for p in PATTERNS])
-def test_protocol_has_no_stall_or_aliased_wait(segs):
+def test_protocol_has_no_stall_or_aliased_wait(segs, prefetch):
+    pre0 = min(segs[0], NS) if prefetch else 0  # a first segment of prefix tiles
     for seed in range(150):
-        msg = run(segs, early_release=False, seed=seed)
+        msg = run(segs, early_release=False, seed=seed, pre0=pre0)
         assert msg is None, f"seed {seed}: {msg}"
 
 
