@@ -144,3 +144,26 @@ def test_vocab_lse_host_checks(jev):
     # the normalised readout runs the readout's own checks
     r = jev.jev_readout_desc(3, 5, 5, 3, 100, 1000, jev.JEV_BF16)
     assert lib.jev_candidate_readout_normalized(C.byref(r), *([None] * 11)) == 2
+
+
+def test_header_is_plain_c_and_links(jev, tmp_path):
+    """include/jev.h compiles as C99 with every warning on, and a C program links against the
+    library and calls a host-only entry point through it."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    names = sorted(_declared())
+    src = tmp_path / "abi.c"
+    src.write_text("#include <stdio.h>\n#include \"jev.h\"\nint main(void) {\n"
+                   "  void (*fns[])(void) = {" + ", ".join(f"(void (*)(void)){n}" for n in names) + "};\n"
+                   "  printf(\"%d %zu\\n\", (int)(sizeof fns / sizeof fns[0]), jev_vocab_lse_workspace(256, 152064));\n"
+                   "  return 0;\n}\n")
+    exe = tmp_path / "abi"
+    lib = jev.LIB_PATH
+    r = subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", os.path.join(ROOT, "include"),
+                        str(src), lib, "-Wl,-rpath," + os.path.dirname(lib), "-o", str(exe)],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()
+    assert int(out[0]) == len(names) and int(out[1]) == jev.jev_vocab_lse_workspace(256, 152064)
