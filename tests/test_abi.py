@@ -102,6 +102,23 @@ def test_tree_build_on_tree_workload(jev):
     assert np.array_equal(plan["pair_tok"], tc.toks[tix])
 
 
+
+def test_tree_readout_plan_matches_hand_golden(jev):
+    """The library's trie and readout plan reproduce the hand-derived pairs of
+    a question with 1-, 2- and 3-token options (tests/golden/tree_readout.json)."""
+    import json
+    import os
+    with open(os.path.join(os.path.dirname(__file__), "golden", "tree_readout.json")) as f:
+        g = json.load(f)
+    so, toks = _csr(g["cands"])
+    a = jev.jev_tree_build(so, toks, g["root_len"])
+    pr = a["path_row"]
+    assert [pr[so[c]:so[c + 1]].tolist() for c in range(len(g["cands"]))] == g["path_row"]
+    plan = jev.jev_tree_readout_plan(so, toks, np.asarray(g["score_from"], np.int32), pr)
+    assert plan["cand_offsets"].tolist() == g["cand_offsets"]
+    assert plan["pair_row"].tolist() == g["pair_row"]
+    assert plan["pair_tok"].tolist() == g["pair_tok"]
+
 def test_tree_build_capacity_and_errors(jev):
     so, toks = _csr([[1, 2, 3], [1, 4]])
     lib = jev._lib

@@ -561,6 +561,55 @@ def test_tree_readout_pairs_teacher_forcing():
         assert tix[k] == a + tc.score_from[c]
 
 
+def test_tree_readout_hand_golden():
+    """Multi-token options against a hand-derived case: every (row, token) pair
+    of a 1-, 2- and 3-token option, the summed scores, the set log-softmax and
+    the choice.  Scoring a token from the question's last row, or from its own
+    row, changes the expected scores."""
+    g = _gold("tree_readout.json")
+    so, toks = _trie_csr(g["cands"])
+    t = oracle.trie_build(so, toks, g["root_len"])
+    pr = t["path_row"]
+    assert [pr[so[c]:so[c + 1]].tolist() for c in range(len(g["cands"]))] == g["path_row"]
+    co, prow, tix = oracle.tree_readout_pairs(so, np.asarray(g["score_from"], np.int32), pr,
+                                              np.asarray(g["set_offsets"], np.int32))
+    assert co.tolist() == g["cand_offsets"]
+    assert prow.tolist() == g["pair_row"]
+    assert toks[tix].tolist() == g["pair_tok"]
+    h = np.asarray(g["hidden"], np.float32)
+    W = np.asarray(g["lm_head"], np.float32)
+    r = oracle.candidate_readout(h, W, np.asarray(g["set_offsets"], np.int32), toks[tix], cand_offsets=co,
+                                 pair_row=prow)
+    tol = g["tolerance"]
+    np.testing.assert_allclose(r["score"], g["expected_score"], rtol=0, atol=tol)
+    np.testing.assert_allclose(r["logprob"], g["expected_logprob"], rtol=0, atol=tol)
+    assert r["choice"].tolist() == [g["expected_choice"]]
+    # the rows of each option's last token are never read
+    h2 = h.copy()
+    h2[[2, 4, 7]] = 100.0
+    r2 = oracle.candidate_readout(h2, W, np.asarray(g["set_offsets"], np.int32), toks[tix], cand_offsets=co,
+                                  pair_row=prow)
+    assert np.array_equal(r2["score"], r["score"])
+
+
+def test_tree_readout_of_one_token_leaves_is_the_flat_readout():
+    """A tree whose options are all one token reads out exactly as the flat
+    problem whose branch hidden state is each question's last-token row."""
+    cfg = synth.TreeConfig("t1", synth.F32, 5, 4, 3, 2, 5, 1, 1, 4, 2, 16, 24, 60, seed=9)
+    tc = synth.tree_case(cfg, with_lm_head=True)
+    t = oracle.trie_build(tc.seq_off, tc.toks, cfg.Lp)
+    co, prow, tix = oracle.tree_readout_pairs(tc.seq_off, tc.score_from, t["path_row"], tc.set_offsets)
+    assert np.array_equal(co, np.arange(co.size, dtype=np.int32))  # one pair per candidate
+    tree = oracle.candidate_readout(tc.hidden, tc.W, tc.set_offsets, tc.toks[tix], cand_offsets=co, pair_row=prow)
+    # flat: branch b's hidden state is the row of its question's last token
+    n_sets = tc.set_offsets.size - 1
+    last_q = [int(t["path_row"][tc.seq_off[tc.set_offsets[b]] + cfg.q_len - 1]) for b in range(n_sets)]
+    opt_tok = np.array([tc.toks[tc.seq_off[c] + cfg.q_len] for c in range(tc.seq_off.size - 1)], np.int32)
+    flat = oracle.candidate_readout(tc.hidden[last_q], tc.W, tc.set_offsets, opt_tok)
+    for k in ("score", "logprob", "choice", "gap"):
+        assert np.array_equal(tree[k], flat[k]), k
+
+
 # ---------------------------------------------------------------- full-vocabulary LSE (normalised scoring)
 
 def test_vocab_lse_closed_forms():
