@@ -588,8 +588,10 @@ jev_status jev_prefix_suffix_attn_noalloc(const jev_attn_desc* d, const void* q,
   jev_attn_desc dd = *d;
   Plan p = plan_of(&dd, T);
   Layout L = layout_of(&dd, T, p, 0);
-  if (L.total > JEV_NOALLOC_SCRATCH_BYTES && p.S > 1) {
-    dd.num_splits = 1;  // a single split needs no partials
+  // the tensor-core plan holds split partials when it splits a tile, the
+  // CUDA-core plan when it has more than one prefix split
+  if (L.total > JEV_NOALLOC_SCRATCH_BYTES && (p.tc ? p.split : p.S > 1)) {
+    dd.num_splits = 1;  // no split: no partials
     p = plan_of(&dd, T);
     L = layout_of(&dd, T, p, 0);
   }

@@ -172,8 +172,9 @@ jev_status jev_prefix_suffix_attn(const jev_attn_desc* desc, const void* q, cons
  * Scratch comes from one file-scope device array of JEV_NOALLOC_SCRATCH_BYTES
  * bytes that every GPU loading the library holds until the process exits.
  * The call allocates nothing (no cudaMalloc, no cudaFree, no allocating
- * library routine).  If the automatic split plan does not fit in the array
- * the call falls back to a single prefix split; if that does not fit either
+ * library routine).  If the automatic plan, with its split partials, does
+ * not fit in the array the call falls back to the plan that splits no work
+ * (num_splits = 1, no partials); if that does not fit either
  * it returns JEV_ERR_UNSUPPORTED, naming the bytes needed, before enqueuing
  * anything.
  *

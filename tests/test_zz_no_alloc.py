@@ -53,6 +53,34 @@ def test_noalloc_matches_workspace_entry_point_twice(jev):
         assert (lse - ref_l).abs().max().item() <= tol["lse"]
 
 
+def test_noalloc_falls_back_to_an_unsplit_plan_at_the_wide_shape(jev):
+    """At the wide shape (128 branches over a 4096-token prefix) the automatic
+    plan's split partials do not fit in the static scratch, but the unsplit
+    plan does: the call must take it and still match the workspace entry
+    point, twice in a row."""
+    cfg = synth.CONFIGS["wide_7b"]
+    c = synth.flat_case(cfg, with_lm_head=False)
+    q, kp, vp, ks, vs, cu = [dev(x) for x in (c.q, c.k_pre, c.v_pre, c.k_suf, c.v_suf, c.cu_seqlens)]
+    T, Hq, d = q.shape
+    desc = jev.make_attn_desc(cfg.B, cfg.Lp, Hq, cfg.Hkv, d, T, jev.JEV_BF16)
+    one = jev.make_attn_desc(cfg.B, cfg.Lp, Hq, cfg.Hkv, d, T, jev.JEV_BF16, num_splits=1)
+    assert jev.jev_prefix_suffix_attn_workspace(desc) > jev.JEV_NOALLOC_SCRATCH_BYTES
+    assert jev.jev_prefix_suffix_attn_workspace(one) <= jev.JEV_NOALLOC_SCRATCH_BYTES
+    ref_o, ref_l = jev.jev_prefix_suffix_attn(q, kp, vp, ks, vs, cu)
+    tol = TOL[synth.BF16]
+    flags = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+    for _ in range(2):
+        out = torch.full_like(q, float("nan"))
+        lse = torch.full(ref_l.shape, float("nan"), dtype=torch.float32, device="cuda")
+        jev.jev_prefix_suffix_attn_noalloc(q, kp, vp, ks, vs, cu, out, lse, status_flags=flags)
+        torch.cuda.synchronize()
+        assert flags.item() == 0
+        assert torch.isfinite(out.float()).all()
+        err = (out.float() - ref_o.float()).abs()
+        assert err.max().item() <= tol["max_abs"] and err.mean().item() <= tol["mean_abs"]
+        assert (lse - ref_l).abs().max().item() <= tol["lse"]
+
+
 def test_noalloc_rejects_problems_beyond_the_static_scratch(jev):
     # 20000 tokens x 28 heads x 128 of bf16 rotated queries alone exceed 32 MiB
     T, Hq, Hkv, d = 20000, 28, 4, 128
