@@ -8,7 +8,7 @@ tokens/s.  Steps are replayed from CUDA graphs over rotating copies of the
 inputs whose total size exceeds twice the L2, so every step reads its prefix
 cache and suffix tensors from HBM.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload qwen2vl_2b] [--impl jev|reference]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload wide_7b] [--impl jev|reference]
 
 With N > 1 (torchrun) every rank runs an independent replica of the workload
 on its own GPU (no collective on the data path; weak scaling); the step time
@@ -151,6 +151,10 @@ class OracleSampler:
         self.t_sets = self.n_sets = 0
         self.cost_row = self._attn(16)[0] / 16
         self.cost_set = self._readout(1)[0]
+        self.reset()
+
+    def reset(self):
+        """Forget the sampled times so far (after warm-up)."""
         self.t_rows = self.n_rows = self.t_sets = self.n_sets = 0
 
     def _attn(self, n):
@@ -198,35 +202,151 @@ class OracleSampler:
                 f"of oracle time, scaled to the whole workload")
 
 
+class TreeOracleSampler:
+    """Times the fp64 oracle on bounded samples of the tree workload and
+    scales them to the whole workload.  Attention is sampled by question: one
+    question's subtree (its tokens and all its option leaves over the root
+    cache) is an independent tree problem, so its oracle time over its unique
+    tokens gives a time per tree token.  The readout is sampled by option set
+    (one question's leaves, full-vocabulary logits of every used row).
+    Workload time = N * (time per sampled token) + sets * (time per sampled
+    set); tokens/s = N / workload time."""
+
+    def __init__(self, cfg):
+        import oracle
+        self.oracle = oracle
+        self.cfg = cfg
+        self.tc = tc = synth.tree_case(cfg, with_lm_head=False)
+        self.W = synth.lm_head(cfg.seed, cfg.V, cfg.H, cfg.dtype, cfg.w_std)
+        self.trie = oracle.trie_build(tc.seq_off, tc.toks, cfg.Lp)
+        self.T = int(self.trie["tok_off"][-1])
+        self.n_sets = tc.set_offsets.size - 1
+        self.co, self.prow, self.tix = oracle.tree_readout_pairs(tc.seq_off, tc.score_from, self.trie["path_row"],
+                                                                 tc.set_offsets)
+        self.rng = np.random.default_rng(1234)
+        self.t_tok = self.n_tok = self.t_sets = self.n_sets_done = 0
+        self.cost_tok = self._attn()[0] / max(1, self.n_tok)
+        self.cost_set = self._readout()[0]
+        self.reset()
+
+    def reset(self):
+        """Forget the sampled times so far (after warm-up)."""
+        self.t_tok = self.n_tok = self.t_sets = self.n_sets_done = 0
+
+    def _attn(self):
+        tc, cfg = self.tc, self.cfg
+        qi = int(self.rng.integers(0, self.n_sets))
+        c0, c1 = int(tc.set_offsets[qi]), int(tc.set_offsets[qi + 1])
+        so = (tc.seq_off[c0:c1 + 1] - tc.seq_off[c0]).astype(np.int32)
+        toks = tc.toks[tc.seq_off[c0]:tc.seq_off[c1]]
+        sub = self.oracle.trie_build(so, toks, cfg.Lp)
+        n = int(sub["tok_off"][-1])
+        gather = np.zeros(n, np.int64)
+        gather[sub["path_row"]] = self.trie["path_row"][tc.seq_off[c0]:tc.seq_off[c1]]
+        q, k, v = tc.q[gather], tc.k[gather], tc.v[gather]
+        t0 = time.perf_counter()
+        self.oracle.tree_attn(sub, q, k, v, tc.k_root, tc.v_root, theta=cfg.theta)
+        dt = time.perf_counter() - t0
+        self.t_tok += dt
+        self.n_tok += n
+        return dt, n
+
+    def _readout(self):
+        tc = self.tc
+        qi = int(self.rng.integers(0, self.n_sets))
+        c0, c1 = int(tc.set_offsets[qi]), int(tc.set_offsets[qi + 1])
+        p0, p1 = int(self.co[c0]), int(self.co[c1])
+        co = (self.co[c0:c1 + 1] - p0).astype(np.int32)
+        t0 = time.perf_counter()
+        self.oracle.candidate_readout(tc.hidden, self.W, np.array([0, c1 - c0], np.int32),
+                                      tc.toks[self.tix[p0:p1]], cand_offsets=co, pair_row=self.prow[p0:p1],
+                                      full_vocab=True)
+        dt = time.perf_counter() - t0
+        self.t_sets += dt
+        self.n_sets_done += 1
+        return dt, 1
+
+    def step(self, budget_s):
+        full_attn = self.cost_tok * self.T
+        full_read = self.cost_set * self.n_sets
+        f_attn = full_attn / (full_attn + full_read)
+        spent = 0.0
+        while spent < f_attn * budget_s or self.n_tok == 0:
+            spent += self._attn()[0]
+        spent = 0.0
+        while spent < (1 - f_attn) * budget_s or self.n_sets_done == 0:
+            spent += self._readout()[0]
+
+    def tokens_per_s(self):
+        t = (self.t_tok / self.n_tok) * self.T + (self.t_sets / self.n_sets_done) * self.n_sets
+        return self.T / t
+
+    def describe(self):
+        return (f"{self.n_tok} tree tokens of question subtrees (all heads, root {self.cfg.Lp} keys) and "
+                f"{self.n_sets_done} option sets (full-vocabulary logits) of the workload ({self.T} tree tokens, "
+                f"{self.n_sets} sets), {self.t_tok + self.t_sets:.1f} s of oracle time, scaled to the whole workload")
+
+
+def make_sampler(cfg):
+    return TreeOracleSampler(cfg) if isinstance(cfg, synth.TreeConfig) else OracleSampler(cfg)
+
+
+def workload_tokens(cfg) -> tuple:
+    """(suffix or tree tokens, branches or candidates) of a workload, from the generator alone."""
+    if isinstance(cfg, synth.TreeConfig):
+        tc = synth.tree_case(cfg, with_lm_head=False)
+        return int(tc.n_unique), int(tc.seq_off.size - 1)
+    return int(synth.suffix_lengths(cfg).sum()), cfg.B
+
+
+L2_NOTE = "per-step inputs rotate over device copies totalling more than twice the 126 MB L2"
+
+
+def bench_config(wl_name: str, world: int, T: int, B: int) -> dict:
+    """The workload description both arms print (identical keys and values)."""
+    cfg = synth.CONFIGS[wl_name]
+    return {"workload": synth.WORKLOAD_TEXT[wl_name], "global_batch": B * world, "seq_len": cfg.Lp,
+            "suffix_tokens_per_replica": T, "parallelism": f"replicas{world}" if world > 1 else "single",
+            "l2": L2_NOTE}
+
+
 def reference_arm(args, wl_name):
     rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
     if rank != 0:
         return
     cfg = synth.CONFIGS[wl_name]
-    if isinstance(cfg, synth.TreeConfig):
-        print(json.dumps({"impl": "reference", "unavailable": "the oracle's tree arm is timed only by the parity tests"}))
-        return
     total_budget = float(os.environ.get("JEV_REF_TOTAL_S", "120"))
     per_step = max(0.002, total_budget / (args.steps + args.warmup))
-    smp = OracleSampler(cfg)
+    smp = make_sampler(cfg)
     for _ in range(args.warmup):
         smp.step(per_step)
-    smp.t_rows = smp.n_rows = smp.t_sets = smp.n_sets = 0
+    smp.reset()
     t0 = time.perf_counter()
     for _ in range(args.steps):
         smp.step(per_step)
     wall = time.perf_counter() - t0
     value = smp.tokens_per_s()
     cores = host_cores()
+    T, B = workload_tokens(cfg)
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * wall / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": synth.WORKLOAD_TEXT[wl_name], "global_batch": cfg.B,
-                                            "seq_len": cfg.Lp, "parallelism": "cpu"},
+            "data": "synthetic", "config": bench_config(wl_name, world, T, B),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                              "sample": "all timed steps together: " + smp.describe()},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line))
+
+
+def cpu_baseline(cfg, budget_s: float) -> dict:
+    """The oracle timed on bounded samples of the workload for about budget_s seconds."""
+    smp = make_sampler(cfg)
+    t0 = time.perf_counter()
+    while time.perf_counter() - t0 < budget_s:
+        smp.step(min(2.0, budget_s / 4))
+    return {"value": smp.tokens_per_s(), "unit": "tokens/s", "cores": host_cores(), "kind": "oracle",
+            "sample": smp.describe()}
 
 
 # ----------------------------------------------------------------------------- jev arm
@@ -432,10 +552,12 @@ def diag_vocab_lse(dev, jev, torch, stream, W=None) -> dict:
                                                      stream=torch.cuda.current_stream()), stream, 20, 3)
     flags = jev.jev_check_device_status(ws_l)
     lflops = 2 * R_l * cfg.V * cfg.H
-    lpeak = float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"]))
+    lpeak = float(pk["bf16_tflops"])
+    lsus = float(pk.get("bf16_tflops_sustained", lpeak))
     return {"workload": f"{R_l} rows x LM head {cfg.V} x {cfg.H}", "flops_per_call": lflops,
             "head_bytes": cfg.V * cfg.H * 2, "us": us_l, "TFLOPs": lflops / us_l / 1e6,
-            "frac_of_sustained_bf16": lflops / us_l / 1e6 / lpeak, "head_GBps": cfg.V * cfg.H * 2 / us_l / 1e3,
+            "frac_of_burst_bf16": lflops / us_l / 1e6 / lpeak, "frac_of_sustained_bf16": lflops / us_l / 1e6 / lsus,
+            "head_GBps": cfg.V * cfg.H * 2 / us_l / 1e3,
             "device_flags": flags,
             "note": "GEMM with an on-chip online LSE and the partial merge; no logits in HBM"}
 
@@ -497,6 +619,44 @@ def diag_tree_schedule(dev, jev, torch, stream) -> dict:
     r["images_per_s"] = 8 / (r["us"] / 1e6)
     res["multi_image_8x416"] = r
     return res
+
+
+def diag_attn(dev, jev, torch, stream, wl_name: str) -> dict:
+    """The workload's attention call alone (no LM head on the device, one set
+    of inputs): a small case for ncu captures of the attention kernels.
+    Runs 3 warm-up calls, then 3 calls between CUDA events."""
+    cfg = synth.CONFIGS[wl_name]
+    if isinstance(cfg, synth.TreeConfig):
+        tc = synth.tree_case(cfg, with_lm_head=False)
+        trie = jev.jev_tree_build(tc.seq_off, tc.toks, cfg.Lp)
+        parent, tok_off, pos0 = (to_dev(trie[k], dev, torch) for k in ("parent", "tok_off", "pos0"))
+        q, kr, vr, k, v = (to_dev(x, dev, torch) for x in (tc.q, tc.k_root, tc.v_root, tc.k, tc.v))
+        out = torch.empty_like(q)
+
+        def call():
+            jev.jev_tree_attn(parent, tok_off, pos0, q, kr, vr, k, v, out=out, rope_theta=cfg.theta, stream=stream)
+    else:
+        c = synth.flat_case(cfg, with_lm_head=False)
+        a = [to_dev(x, dev, torch) for x in (c.q, c.k_pre, c.v_pre, c.k_suf, c.v_suf)]
+        cu = torch.from_numpy(c.cu_seqlens).to(dev)
+        out = torch.empty_like(a[0])
+        desc = jev.make_attn_desc(cfg.B, cfg.Lp, cfg.Hq, cfg.Hkv, cfg.d, c.T,
+                                  jev.JEV_BF16 if cfg.dtype == synth.BF16 else jev.JEV_F32, cfg.theta)
+        ws = jev.new_workspace(jev.jev_prefix_suffix_attn_workspace(desc), dev)
+
+        def call():
+            jev.jev_prefix_suffix_attn(*a, cu, out=out, workspace=ws, rope_theta=cfg.theta, stream=stream)
+    torch.cuda.synchronize()
+    for _ in range(3):
+        call()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(3):
+        call()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return {"workload": wl_name, "us_per_call": 1e3 * e0.elapsed_time(e1) / 3,
+            "note": "direct launches, not graph-replayed; for profiling captures, not a bench number"}
 
 
 def diagnostics(dev, jev, torch) -> dict:
@@ -599,21 +759,21 @@ def diagnostics(dev, jev, torch) -> dict:
     sprof = jev.jev_profile_read()
     del g
     sflops = 4 * Hq * d * nb * (bl * S + bl * (bl + 1) // 2)
-    speak = float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"]))
+    speak = float(pk["bf16_tflops"])
     s_us = {k: 1e3 * v[1] / max(v[0], 1) for k, v in sprof.items()}
     if "attn_tc" in s_us:
         out["sink_block"] = {"workload": f"{nb} blocks of {bl} tokens over a {S}-token sink, Hq={Hq}, Hkv={Hkv}, "
                                          f"d={d}", "flops_per_call": sflops, "kernels_us": s_us,
                              "TFLOPs": sflops / s_us["attn_tc"] / 1e6,
-                             "frac_of_sustained_bf16": sflops / s_us["attn_tc"] / 1e6 / speak,
+                             "frac_of_burst_bf16": sflops / s_us["attn_tc"] / 1e6 / speak,
                              "tokens_per_s": Tsb / (sum(s_us.values()) / 1e6)}
     # the tensor-core kernel at the wide size: many waves of whole tiles
     if "attn_tc" in prof:
         flops = flat_work(c)["flops_attn"]
         aus = out["attn_call_us"]["attn_tc"]
-        peak = float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"]))
+        peak = float(pk["bf16_tflops"])
         out["attn_tc"] = {"workload": out["rope_pack"]["workload"], "flops_per_call": flops, "us": aus,
-                          "TFLOPs": flops / aus / 1e6, "frac_of_sustained_bf16": flops / aus / 1e6 / peak}
+                          "TFLOPs": flops / aus / 1e6, "frac_of_burst_bf16": flops / aus / 1e6 / peak}
     return out
 
 
@@ -742,7 +902,10 @@ class Measured:
         dom = max(prof.items(), key=lambda kv: kv[1][1])[0] if prof else attn_name
         n_l, t_ms = prof.get(attn_name, (1, float("nan")))
         achieved = work["flops_attn"] / (t_ms / 1e3 / max(n_l, 1)) / 1e12
-        peak = float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"]))
+        # the kernel is event-timed over launches of tens to hundreds of
+        # microseconds at full clock: the burst GEMM figure is its peak
+        peak = float(pk["bf16_tflops"])
+        sustained = float(pk.get("bf16_tflops_sustained", peak))
         tot_prof = sum(x[1] for x in prof.values()) or 1.0
         per_kernel = {k: {"launches": v[0], "avg_us": 1e3 * v[1] / max(v[0], 1), "share": v[1] / tot_prof}
                       for k, v in prof.items()}
@@ -751,8 +914,8 @@ class Measured:
                     (work["bytes_attn"] + work["bytes_readout"]) / (float(pk["hbm_gbs"]) * 1e9))
         roof = {"bound": "tensor", "kernel": attn_name, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak, "traffic": traffic_of(attn_name, self.name, KERNEL_SRC[attn_name]),
-                "peak_source": f"bf16_tflops_sustained, {src}",
-                "frac_of_burst_peak": achieved / float(pk["bf16_tflops"]),
+                "peak_source": f"bf16_tflops (burst), {src}",
+                "frac_of_sustained_peak": achieved / sustained,
                 "algorithmic_flops_per_launch": work["flops_attn"], "dominant_kernel_by_time": dom}
         step_roof = {"ideal_us": ideal * 1e6, "measured_us": step_s * 1e6, "frac": ideal / step_s,
                      "definition": "max(F / bf16 burst peak, U / HBM peak) over the whole step"}
@@ -844,9 +1007,8 @@ def jev_arm(args, wl_name):
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
         "step_us_spread": m.pct,
         "vs_baseline": None, "dtype": "bf16" if cfg.dtype == synth.BF16 else "f32", "data": "synthetic",
-        "config": {"workload": synth.WORKLOAD_TEXT[wl_name], "global_batch": wl.B * world, "seq_len": cfg.Lp,
-                   "suffix_tokens_per_replica": T, "parallelism": f"replicas{world}" if world > 1 else "single",
-                   "l2": f"inputs rotate over {m.ngraph} device copies ({m.ngraph * m.per_copy / 2**20:.0f} MiB "
+        "config": bench_config(wl_name, world, T, wl.B),
+        "method": {"l2": f"inputs rotate over {m.ngraph} device copies ({m.ngraph * m.per_copy / 2**20:.0f} MiB "
                          "> 2x L2)",
                    "timing": "CUDA graph replay per step, CUDA events on the launching stream; per-kernel times "
                              "from a second replay of the K steps with event nodes around each kernel",
@@ -878,24 +1040,20 @@ def jev_arm(args, wl_name):
                          "branches_per_s": mc.wl.B * steps / (mc.ms / 1e3),
                          "dtype": "bf16" if mc.cfg.dtype == synth.BF16 else "f32",
                          "roofline": {k: r[k] for k in ("bound", "kernel", "achieved", "peak", "unit", "frac",
-                                                        "traffic", "peak_source")},
+                                                        "traffic", "peak_source", "frac_of_sustained_peak")},
                          "step_roofline_frac": sr["frac"],
                          "kernels": {k: round(v["avg_us"], 2) for k, v in pk_.items()}}
             mc.free()
             del mc
+            if os.environ.get("JEV_SKIP_CPU_BASELINE") != "1":
+                per[name]["cpu_baseline"] = cpu_baseline(synth.CONFIGS[name],
+                                                         float(os.environ.get("JEV_CPU_BASELINE_CONFIG_S", "5")))
         line["per_config"] = per
     if world == 1 and args.diagnostics:
         line["diagnostics"] = diagnostics(dev, jev, torch)
 
-    if rank == 0 and world == 1 and os.environ.get("JEV_SKIP_CPU_BASELINE") != "1" and isinstance(wl, FlatWorkload) \
-            and not isinstance(wl, TreeWorkload):
-        budget = float(os.environ.get("JEV_CPU_BASELINE_S", "12"))
-        smp = OracleSampler(cfg)
-        t0 = time.perf_counter()
-        while time.perf_counter() - t0 < budget:
-            smp.step(min(2.0, budget / 4))
-        line["cpu_baseline"] = {"value": smp.tokens_per_s(), "unit": "tokens/s", "cores": host_cores(),
-                                "kind": "oracle", "sample": smp.describe()}
+    if rank == 0 and world == 1 and os.environ.get("JEV_SKIP_CPU_BASELINE") != "1":
+        line["cpu_baseline"] = cpu_baseline(cfg, float(os.environ.get("JEV_CPU_BASELINE_S", "12")))
     if rank == 0:
         print(json.dumps(line))
     if world > 1:
@@ -907,14 +1065,15 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20000)
     ap.add_argument("--warmup", type=int, default=200)
-    ap.add_argument("--workload", default="qwen2vl_2b", choices=sorted(synth.CONFIGS))
+    # the default is the largest single-GPU workload
+    ap.add_argument("--workload", default="wide_7b", choices=sorted(synth.CONFIGS))
     ap.add_argument("--impl", default="jev", choices=["jev", "reference"])
     ap.add_argument("--no-per-config", dest="per_config", action="store_false",
                     help="skip the other synthetic configs (reported under per_config on one GPU)")
     ap.add_argument("--per-config-steps", type=int, default=2000)
     ap.add_argument("--no-diagnostics", dest="diagnostics", action="store_false",
                     help="skip the streaming diagnostics at larger sizes (one GPU)")
-    ap.add_argument("--diag", choices=["vocab_lse", "tree_schedule"], default=None,
+    ap.add_argument("--diag", choices=["vocab_lse", "tree_schedule", "attn"], default=None,
                     help="run only this diagnostic on cuda:0 and print its JSON (a small case for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -923,8 +1082,13 @@ def main():
         import torch
         import attention_cascade_b200 as jev
         torch.cuda.set_device(0)
-        fn = {"vocab_lse": diag_vocab_lse, "tree_schedule": diag_tree_schedule}[args.diag]
-        print(json.dumps({"diagnostic": args.diag, **fn("cuda:0", jev, torch, torch.cuda.Stream(device="cuda:0"))}))
+        stream = torch.cuda.Stream(device="cuda:0")
+        if args.diag == "attn":
+            res = diag_attn("cuda:0", jev, torch, stream, args.workload)
+        else:
+            fn = {"vocab_lse": diag_vocab_lse, "tree_schedule": diag_tree_schedule}[args.diag]
+            res = fn("cuda:0", jev, torch, stream)
+        print(json.dumps({"diagnostic": args.diag, **res}))
     elif args.impl == "reference":
         reference_arm(args, args.workload)
     else:
