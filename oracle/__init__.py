@@ -53,6 +53,15 @@ class _AttnProblem(C.Structure):
                 ("n_rows", C.c_int), ("rows", C.c_void_p), ("n_threads", C.c_int)]
 
 
+class _CacheProblem(C.Structure):
+    _fields_ = [("B", C.c_int), ("Lp", C.c_int), ("Hq", C.c_int), ("Hkv", C.c_int), ("d", C.c_int),
+                ("dtype", C.c_int), ("theta", C.c_double), ("scale", C.c_double), ("pos_offset", C.c_int),
+                ("q", C.c_void_p), ("k_new", C.c_void_p), ("v_new", C.c_void_p), ("k_pre", C.c_void_p),
+                ("v_pre", C.c_void_p), ("k_cache", C.c_void_p), ("v_cache", C.c_void_p),
+                ("cache_off", C.c_void_p), ("cache_len", C.c_void_p), ("cu_new", C.c_void_p),
+                ("head_map", C.c_void_p), ("n_threads", C.c_int)]
+
+
 class _ReadoutProblem(C.Structure):
     _fields_ = [("n_sets", C.c_int), ("n_cands", C.c_int), ("n_pairs", C.c_int), ("R", C.c_int),
                 ("H", C.c_int), ("V", C.c_int), ("dtype", C.c_int), ("hidden", C.c_void_p),
@@ -81,6 +90,8 @@ def lib():
                                        C.c_double, C.c_void_p, C.c_void_p]
         _lib.oracle_prefix_suffix_attn.argtypes = [C.POINTER(_AttnProblem), C.c_void_p, C.c_void_p]
         _lib.oracle_prefix_suffix_attn.restype = C.c_int
+        _lib.oracle_cache_attn.argtypes = [C.POINTER(_CacheProblem), C.c_void_p, C.c_void_p, C.c_void_p]
+        _lib.oracle_cache_attn.restype = C.c_int
         _lib.oracle_candidate_readout.argtypes = [C.POINTER(_ReadoutProblem)] + [C.c_void_p] * 5
         _lib.oracle_candidate_readout.restype = C.c_int
         _lib.oracle_trie_build.argtypes = [C.c_int, C.c_void_p, C.c_void_p, C.c_int, C.c_int, C.c_int] + [C.c_void_p] * 6
@@ -156,6 +167,30 @@ def prefix_suffix_attn(q, k_pre, v_pre, k_suf, v_suf, cu_seqlens, *, theta=1e4, 
     if rc != 0:
         raise ValueError("oracle_prefix_suffix_attn: bad arguments")
     return out, lse
+
+
+def cache_attn(q, k_new, v_new, k_pre, v_pre, k_cache, v_cache, cache_off, cache_len, cu_new, *, theta=1e4,
+               scale=0.0, pos_offset=-1, head_map=None, n_threads=0):
+    """A generation step over per-branch suffix caches, unshared; returns
+    (out [T, Hq, d], lse [T, Hq], k_new_rot [T, Hkv, d]) as float64, the last
+    being the rotated new keys the step appends to the cache."""
+    q, k_new, v_new, k_pre, v_pre, k_cache, v_cache = (_c(a) for a in (q, k_new, v_new, k_pre, v_pre, k_cache,
+                                                                       v_cache))
+    dt = _dtype_of(q)
+    for a in (k_new, v_new, k_pre, v_pre, k_cache, v_cache):
+        assert _dtype_of(a) == dt
+    co, cl, cu, hm = (_c(a, np.int32) for a in (cache_off, cache_len, cu_new, head_map))
+    T, Hq, d = q.shape
+    Lp, Hkv, _ = k_pre.shape
+    out = np.zeros((T, Hq, d), np.float64)
+    lse = np.full((T, Hq), -np.inf, np.float64)
+    krot = np.zeros((T, Hkv, d), np.float64)
+    pr = _CacheProblem(cu.size - 1, Lp, Hq, Hkv, d, dt, float(theta), float(scale), int(pos_offset),
+                       _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_pre), _ptr(v_pre), _ptr(k_cache), _ptr(v_cache),
+                       _ptr(co), _ptr(cl), _ptr(cu), _ptr(hm), int(n_threads))
+    if lib().oracle_cache_attn(C.byref(pr), _ptr(out), _ptr(lse), _ptr(krot)) != 0:
+        raise ValueError("oracle_cache_attn: bad arguments")
+    return out, lse, krot
 
 
 def candidate_readout(hidden, lm_head, set_offsets, pair_tok, *, cand_offsets=None, pair_row=None,

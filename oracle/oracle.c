@@ -175,6 +175,83 @@ int oracle_prefix_suffix_attn(const oracle_attn_problem* p, double* out, double*
 }
 
 /* ------------------------------------------------------------------------ */
+/* Generation over per-branch suffix caches: branch b's key list is the prefix,
+ * then its cached (already rotated) suffix keys, then its new keys rotated at
+ * the positions that follow the cached ones; new token j sees the prefix, the
+ * whole cache and new tokens 0..j.                                           */
+
+int oracle_cache_attn(const oracle_cache_problem* p, double* out, double* lse, double* k_new_rot) {
+  if (!p || p->B < 0 || p->Lp < 0 || p->Hq <= 0 || p->Hkv <= 0 || p->d <= 0 || (p->d & 1)) return -1;
+  if (!p->head_map && (p->Hq % p->Hkv)) return -1;
+  const int B = p->B, Lp = p->Lp, Hq = p->Hq, Hkv = p->Hkv, d = p->d, G = Hq / Hkv;
+  const int32_t *cu = p->cu_new, *co = p->cache_off, *cl = p->cache_len;
+  if (B > 0 && (!cu || !co || !cl || cu[0] != 0)) return -1;
+  for (int b = 0; b < B; ++b) {
+    if (cu[b + 1] < cu[b] || co[b + 1] < co[b] || co[b] < 0 || cl[b] < 0) return -1;
+    if ((long)cl[b] + (cu[b + 1] - cu[b]) > (long)(co[b + 1] - co[b])) return -1;
+  }
+  if (p->head_map)
+    for (int h = 0; h < Hq; ++h)
+      if (p->head_map[h] < 0 || p->head_map[h] >= Hkv) return -1;
+  const int T = B > 0 ? cu[B] : 0;
+  const double scale = p->scale > 0 ? p->scale : 1.0 / sqrt((double)d);
+  const int pos_off = p->pos_offset >= 0 ? p->pos_offset : Lp;
+
+  /* the appended keys: new token j of branch b rotated at pos_off + cache_len[b] + j */
+  double* x = (double*)malloc(sizeof(double) * (size_t)d);
+  for (int b = 0; b < B; ++b)
+    for (int t = cu[b]; t < cu[b + 1]; ++t)
+      for (int g = 0; g < Hkv; ++g) {
+        for (int i = 0; i < d; ++i) x[i] = widen(p->k_new, p->dtype, ((size_t)t * Hkv + g) * d + i);
+        oracle_rope(x, k_new_rot + ((size_t)t * Hkv + g) * d, d, (double)(pos_off + cl[b] + (t - cu[b])), p->theta);
+      }
+  free(x);
+
+  set_threads(p->n_threads);
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int task = 0; task < B * Hq; ++task) {
+    const int b = task / Hq, h = task % Hq;
+    const int g = p->head_map ? p->head_map[h] : h / G;
+    const int Lc = cl[b], Ln = cu[b + 1] - cu[b];
+    if (Ln == 0) continue;
+    const int n = Lp + Lc + Ln;
+    double* Kb = (double*)malloc(sizeof(double) * (size_t)n * d);
+    double* Vb = (double*)malloc(sizeof(double) * (size_t)n * d);
+    double* xq = (double*)malloc(sizeof(double) * (size_t)d);
+    double* qr = (double*)malloc(sizeof(double) * (size_t)d);
+    for (int t = 0; t < Lp; ++t)
+      for (int i = 0; i < d; ++i) {
+        size_t src = ((size_t)t * Hkv + g) * d + i;
+        Kb[(size_t)t * d + i] = widen(p->k_pre, p->dtype, src);
+        Vb[(size_t)t * d + i] = widen(p->v_pre, p->dtype, src);
+      }
+    for (int c = 0; c < Lc; ++c)
+      for (int i = 0; i < d; ++i) {
+        size_t src = ((size_t)(co[b] + c) * Hkv + g) * d + i;
+        Kb[(size_t)(Lp + c) * d + i] = widen(p->k_cache, p->dtype, src);
+        Vb[(size_t)(Lp + c) * d + i] = widen(p->v_cache, p->dtype, src);
+      }
+    for (int j = 0; j < Ln; ++j)
+      for (int i = 0; i < d; ++i) {
+        size_t src = ((size_t)(cu[b] + j) * Hkv + g) * d + i;
+        Kb[(size_t)(Lp + Lc + j) * d + i] = k_new_rot[src];
+        Vb[(size_t)(Lp + Lc + j) * d + i] = widen(p->v_new, p->dtype, src);
+      }
+    for (int j = 0; j < Ln; ++j) {
+      const size_t row = (size_t)(cu[b] + j);
+      for (int i = 0; i < d; ++i) xq[i] = widen(p->q, p->dtype, (row * Hq + h) * d + i);
+      oracle_rope(xq, qr, d, (double)(pos_off + Lc + j), p->theta);
+      double l;
+      oracle_attend(qr, Kb, Vb, Lp + Lc + j + 1, d, d, scale, out + (row * Hq + h) * d, &l);
+      if (lse) lse[row * Hq + h] = l;
+    }
+    free(Kb); free(Vb); free(xq); free(qr);
+  }
+  (void)T;
+  return 0;
+}
+
+/* ------------------------------------------------------------------------ */
 /* Candidate readout: logits of the used hidden rows against the LM head, the
  * candidate score as the sum of its (row, token) logits, and a log-softmax
  * over each option set.  Ties pick the lowest candidate index.              */

@@ -74,6 +74,34 @@ typedef struct {
 int oracle_prefix_suffix_attn(const oracle_attn_problem* p, double* out, double* lse);
 
 typedef struct {
+  int B, Lp, Hq, Hkv, d, dtype;
+  double theta;        /* RoPE base */
+  double scale;        /* 0 -> 1/sqrt(d) */
+  int pos_offset;      /* < 0 -> Lp */
+  const void* q;       /* [T, Hq, d] new tokens, pre-RoPE */
+  const void* k_new;   /* [T, Hkv, d] new tokens' keys, pre-RoPE */
+  const void* v_new;   /* [T, Hkv, d] */
+  const void* k_pre;   /* [Lp, Hkv, d] post-RoPE prefix cache */
+  const void* v_pre;   /* [Lp, Hkv, d] */
+  const void* k_cache; /* [C, Hkv, d] cached suffix keys, post-RoPE */
+  const void* v_cache; /* [C, Hkv, d] */
+  const int32_t* cache_off; /* [B+1] branch b's cache rows start at cache_off[b] */
+  const int32_t* cache_len; /* [B] tokens cached per branch */
+  const int32_t* cu_new;    /* [B+1] new-token offsets */
+  const int32_t* head_map;  /* [Hq] or NULL */
+  int n_threads;
+} oracle_cache_problem;
+
+/* A generation step over per-branch suffix caches, computed unshared: for
+ * branch b the key list is [K_pre ; its cache_len[b] cached keys ; RoPE(its
+ * new keys)], new token j sits at position pos_offset + cache_len[b] + j and
+ * sees keys 0 .. Lp + cache_len[b] + j.  out [T, Hq, d], lse [T, Hq];
+ * k_new_rot [T, Hkv, d] receives the rotated new keys (what the step appends
+ * to the cache).  Returns 0, or -1 on bad arguments (including a branch whose
+ * cache rows cannot hold its tokens). */
+int oracle_cache_attn(const oracle_cache_problem* p, double* out, double* lse, double* k_new_rot);
+
+typedef struct {
   int n_sets, n_cands, n_pairs, R, H, V, dtype;
   const void* hidden;          /* [R, H] */
   const void* lm_head;         /* [V, H] */

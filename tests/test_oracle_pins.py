@@ -666,3 +666,116 @@ def test_sequence_logprob_is_a_distribution_and_adds():
     lp1 = oracle.sequence_logprob(h, W, co, np.ones(V, np.int32), np.arange(V, dtype=np.int32))
     assert abs(np.exp(lp1).sum() - 1.0) < 1e-12
     assert abs(lp2[2] - lp1[7]) < 1e-12 and abs(lp2[1] - lp[4]) < 1e-12
+
+
+# ---------------------------------------------------------------- generation over per-branch suffix caches
+
+
+def _cache_case(rng, Lp=7, Hq=4, Hkv=2, d=16, cached=(0, 3, 5, 2), new=(2, 1, 0, 3), spare=(1, 0, 2, 1),
+                dtype=np.float32, theta=1e4, pos_offset=-1):
+    """Random new tokens and caches whose keys are the independent complex
+    rotation of raw keys at the positions the cached tokens held."""
+    B = len(cached)
+    po = Lp if pos_offset < 0 else pos_offset
+    cap = [c + n + s for c, n, s in zip(cached, new, spare)]
+    co = np.concatenate([[0], np.cumsum(cap)]).astype(np.int32)
+    cu = np.concatenate([[0], np.cumsum(new)]).astype(np.int32)
+    C, T = int(co[-1]), int(cu[-1])
+    k_pre = rng.standard_normal((Lp, Hkv, d)).astype(np.float32)
+    v_pre = rng.standard_normal((Lp, Hkv, d)).astype(np.float32)
+    k_cache = np.zeros((C, Hkv, d), np.float32)
+    v_cache = rng.standard_normal((C, Hkv, d)).astype(np.float32)
+    k_cached_raw = []
+    for b in range(B):
+        raw = rng.standard_normal((cached[b], Hkv, d))
+        k_cached_raw.append(raw)
+        rot = _rope_complex(raw.transpose(1, 0, 2), po + np.arange(cached[b]), theta).transpose(1, 0, 2)
+        k_cache[co[b]:co[b] + cached[b]] = rot
+    q = rng.standard_normal((T, Hq, d)).astype(np.float32)
+    k_new = rng.standard_normal((T, Hkv, d)).astype(np.float32)
+    v_new = rng.standard_normal((T, Hkv, d)).astype(np.float32)
+    return dict(q=q, k_new=k_new, v_new=v_new, k_pre=k_pre, v_pre=v_pre, k_cache=k_cache, v_cache=v_cache,
+                cache_off=co, cache_len=np.array(cached, np.int32), cu_new=cu, k_cached_raw=k_cached_raw, po=po)
+
+
+def test_cache_attn_matches_sdpa_over_prefix_cache_and_new_tokens():
+    """Each new token's row equals causal fp64 SDPA over [prefix; the branch's
+    cached keys; its rotated new keys] at the row of that token, and the
+    appended keys are the complex rotation of the new keys."""
+    rng = np.random.default_rng(21)
+    theta, Hq, Hkv, d = 1e4, 4, 2, 16
+    for pos_offset, head_map in ((-1, None), (40, np.array([1, 0, 1, 0], np.int32))):
+        c = _cache_case(rng, theta=theta, pos_offset=pos_offset)
+        out, lse, krot = oracle.cache_attn(c["q"], c["k_new"], c["v_new"], c["k_pre"], c["v_pre"], c["k_cache"],
+                                           c["v_cache"], c["cache_off"], c["cache_len"], c["cu_new"], theta=theta,
+                                           pos_offset=pos_offset, head_map=head_map)
+        hm = torch.from_numpy(head_map).long() if head_map is not None else torch.arange(Hq) // (Hq // Hkv)
+        cu, co, cl, po = c["cu_new"], c["cache_off"], c["cache_len"], c["po"]
+        Lp = c["k_pre"].shape[0]
+        for b in range(cu.size - 1):
+            n = int(cu[b + 1] - cu[b])
+            if n == 0:
+                continue
+            pos_new = po + cl[b] + np.arange(n)
+            kn = _rope_complex(c["k_new"][cu[b]:cu[b + 1]].astype(np.float64).transpose(1, 0, 2), pos_new,
+                               theta).transpose(1, 0, 2)
+            np.testing.assert_allclose(krot[cu[b]:cu[b + 1]], kn, atol=1e-12)
+            qn = _rope_complex(c["q"][cu[b]:cu[b + 1]].astype(np.float64).transpose(1, 0, 2), pos_new,
+                               theta).transpose(1, 0, 2)
+            L0 = Lp + int(cl[b])
+            kf = np.concatenate([c["k_pre"].astype(np.float64), c["k_cache"][co[b]:co[b] + cl[b]].astype(np.float64), kn])
+            vf = np.concatenate([c["v_pre"], c["v_cache"][co[b]:co[b] + cl[b]], c["v_new"][cu[b]:cu[b + 1]]]).astype(np.float64)
+            qf = np.concatenate([np.zeros((L0, Hq, d)), qn])
+            o_ref, l_ref = _sdpa_branch(qf, kf, vf, None, Hkv, hm, theta, 1 / math.sqrt(d))
+            np.testing.assert_allclose(out[cu[b]:cu[b + 1]], o_ref[L0:], atol=1e-12)
+            np.testing.assert_allclose(lse[cu[b]:cu[b + 1]], l_ref[L0:], atol=1e-12)
+
+
+def test_cache_attn_with_empty_caches_is_the_prefill():
+    """With nothing cached, the step is jev's flat problem on the new tokens."""
+    c = _small_case(B=4, lens=(3, 1, 5, 2))
+    cu = c.cu_seqlens
+    co = cu.copy()  # caches exactly as large as the new tokens
+    out, lse, krot = oracle.cache_attn(c.q, c.k_suf, c.v_suf, c.k_pre, c.v_pre, np.zeros_like(c.k_suf),
+                                       np.zeros_like(c.v_suf), co, np.zeros(4, np.int32), cu)
+    o_ref, l_ref = oracle.prefix_suffix_attn(c.q, c.k_pre, c.v_pre, c.k_suf, c.v_suf, cu)
+    np.testing.assert_allclose(out, o_ref, atol=1e-13)
+    np.testing.assert_allclose(lse, l_ref, atol=1e-13)
+
+
+def test_cache_attn_step_is_the_next_row_of_the_whole_suffix():
+    """Decoding the last m tokens over a cache of the first ones (rotated
+    keys stored in float32) gives the rows of the whole suffix's attention."""
+    rng = np.random.default_rng(22)
+    lens, m = np.array([4, 1, 6], np.int32), np.array([1, 2, 1], np.int32)
+    c = _small_case(B=3, lens=tuple(lens + m), Hq=6, Hkv=2, d=16)
+    cu_full = c.cu_seqlens
+    full_o, full_l = oracle.prefix_suffix_attn(c.q, c.k_pre, c.v_pre, c.k_suf, c.v_suf, cu_full)
+    Lp = c.k_pre.shape[0]
+    co = np.concatenate([[0], np.cumsum(lens + m + 2)]).astype(np.int32)
+    k_cache = np.zeros((co[-1], 2, 16), np.float32)
+    v_cache = rng.standard_normal((co[-1], 2, 16)).astype(np.float32)
+    new_rows = []
+    for b in range(3):
+        a = cu_full[b]
+        raw = c.k_suf[a:a + lens[b]].astype(np.float64)
+        k_cache[co[b]:co[b] + lens[b]] = _rope_complex(raw.transpose(1, 0, 2), Lp + np.arange(lens[b]),
+                                                        1e4).transpose(1, 0, 2)
+        v_cache[co[b]:co[b] + lens[b]] = c.v_suf[a:a + lens[b]]
+        new_rows.append(np.arange(a + lens[b], a + lens[b] + m[b]))
+    idx = np.concatenate(new_rows)
+    cu_new = np.concatenate([[0], np.cumsum(m)]).astype(np.int32)
+    out, lse, _ = oracle.cache_attn(c.q[idx], c.k_suf[idx], c.v_suf[idx], c.k_pre, c.v_pre, k_cache, v_cache, co,
+                                    lens, cu_new)
+    np.testing.assert_allclose(out, full_o[idx], atol=1e-5)
+    np.testing.assert_allclose(lse, full_l[idx], atol=1e-5)
+
+
+def test_cache_attn_rejects_a_branch_beyond_its_cache_rows():
+    rng = np.random.default_rng(23)
+    c = _cache_case(rng, cached=(2, 1), new=(1, 2), spare=(0, 0))
+    cl = c["cache_len"].copy()
+    cl[1] += 1  # one more cached token than the branch's rows leave room for
+    with pytest.raises(ValueError):
+        oracle.cache_attn(c["q"], c["k_new"], c["v_new"], c["k_pre"], c["v_pre"], c["k_cache"], c["v_cache"],
+                          c["cache_off"], cl, c["cu_new"])
