@@ -3,16 +3,17 @@
 A model of the roles in attn_tc.cu, each a sequence of barrier operations per
 segment of n key tiles:
   * producer: wait q_empty of the previous segment, two arrivals on q_full
-    (expect-tx and the published descriptor), then per key tile wait kv_empty
-    of the stage's previous use and arrive on k_full / v_full;
-  * MMA warp: wait q_full, k_full, commit s_full of both tiles; per key tile
-    wait v_full and p_full of each tile, commit o_full after the last PV,
-    commit kv_empty, and commit q_empty after the segment's last S MMA (the
-    rule under test);
-  * softmax threads (two per tile group here, standing for the 256 that
-    p_full counts): wait q_full, per key tile wait s_full and arrive on
-    p_full, with a pair barrier per tile; wait o_full and two group barriers
-    in the epilogue.
+    (expect-tx and the published descriptor), then the K of tile 0 and per
+    key tile j the K of tile j + 1 ahead of the V of tile j, each after a wait
+    on its ring stage's empty barrier (K and V rings of NK and NV stages);
+  * MMA warp: wait q_full, k_full, commit s_full of both tiles and k_empty;
+    per key tile wait v_full and p_full of each tile, commit o_full after the
+    last PV, v_empty after the tile's last PV, k_empty after the next tile's
+    last S MMA, and q_empty after the segment's last S MMA (the rule under
+    test);
+  * softmax threads (two per tile here, standing for the 128 rows that
+    p_full counts, one thread per row): wait q_full, per key tile wait
+    s_full and arrive on p_full; wait o_full before the epilogue.
 MMA commits and TMA completions are modelled as immediate (one possible
 timing).  A wait follows the hardware rule for parity waits (it passes when
 the barrier's completed-phase count has the other parity), and the checker
@@ -26,7 +27,7 @@ import random
 
 import pytest
 
-NS = 2  # K/V stages at d = 128
+NK, NV = 3, 2  # K and V ring stages at d = 128
 
 
 class Bar:
@@ -34,25 +35,51 @@ class Bar:
         self.count, self.pending, self.phase = count, 0, 0
 
 
-def producer(segs, pre0=0):
-    # pre0: the first segment's leading prefix tiles, loaded into stages 0 .. pre0-1 before
-    # anything else (before the kernel's wait on the previous launch and before the first Q)
-    for j in range(pre0):
-        yield ("arrive", f"k_full{j}")
-        yield ("arrive", f"v_full{j}")
+def _producer_order(n, first):
+    """(kind, j) loads of one segment of n key tiles: K of tile 0, then for
+    each tile j the K of tile j + 1 ahead of the V of tile j.  `first` drops
+    the tiles already loaded before the segment (counts of K and of V)."""
+    dk, dv = first
+    out = [] if dk > 0 else [("k", 0)]
+    for j in range(n):
+        if j + 1 < n and j + 1 >= dk:
+            out.append(("k", j + 1))
+        if j >= dv:
+            out.append(("v", j))
+    return out
+
+
+def _preload(segs, prefetch):
+    """Loads issued before anything else: the first segment's leading K and V
+    tiles, into stages not used before, in the same order as the main loop."""
+    if not prefetch:
+        return 0, 0, []
+    pk, pv = min(segs[0], NK), min(segs[0], NV)
+    out = [("k", 0)] if pk > 0 else []
+    for j in range(max(pk, pv)):
+        if j + 1 < pk:
+            out.append(("k", j + 1))
+        if j < pv:
+            out.append(("v", j))
+    return pk, pv, out
+
+
+def producer(segs, prefetch=False):
+    pk, pv, pre = _preload(segs, prefetch)
+    for kind, j in pre:
+        yield ("arrive", f"{kind}_full{j % (NK if kind == 'k' else NV)}")
     J = 0
     for k, n in enumerate(segs):
         if k > 0:
             yield ("wait", "q_empty", k - 1)
         yield ("arrive", "q_full")
         yield ("arrive", "q_full")
-        for j in range(pre0 if k == 0 else 0, n):
+        for kind, j in _producer_order(n, (pk, pv) if k == 0 else (0, 0)):
             JJ = J + j
-            st = JJ % NS
-            if JJ >= NS:
-                yield ("wait", f"kv_empty{st}", JJ // NS - 1)
-            yield ("arrive", f"k_full{st}")
-            yield ("arrive", f"v_full{st}")
+            ns = NK if kind == "k" else NV
+            if JJ >= ns:
+                yield ("wait", f"{kind}_empty{JJ % ns}", JJ // ns - 1)
+            yield ("arrive", f"{kind}_full{JJ % ns}")
         J += n
 
 
@@ -60,28 +87,28 @@ def mma(segs, early_release):
     J = 0
     for k, n in enumerate(segs):
         yield ("wait", "q_full", k)
-        st0 = J % NS
-        yield ("wait", f"k_full{st0}", J // NS)
+        yield ("wait", f"k_full{J % NK}", J // NK)
         yield ("arrive", "s_full0")
         yield ("arrive", "s_full1")
+        yield ("arrive", f"k_empty{J % NK}")
         if early_release and n == 1:
             yield ("arrive", "q_empty")  # the earlier rule: released before any softmax acknowledgement
         for j in range(n):
             JJ = J + j
-            st, st1 = JJ % NS, (JJ + 1) % NS
-            yield ("wait", f"v_full{st}", JJ // NS)
+            yield ("wait", f"v_full{JJ % NV}", JJ // NV)
             yield ("wait", "p_full0", JJ)
             if j == n - 1:
                 yield ("arrive", "o_full0")
             if j + 1 < n:
-                yield ("wait", f"k_full{st1}", (JJ + 1) // NS)
+                yield ("wait", f"k_full{(JJ + 1) % NK}", (JJ + 1) // NK)
                 yield ("arrive", "s_full0")
             yield ("wait", "p_full1", JJ)
-            yield ("arrive", f"kv_empty{st}")
+            yield ("arrive", f"v_empty{JJ % NV}")
             if j == n - 1:
                 yield ("arrive", "o_full1")
             if j + 1 < n:
                 yield ("arrive", "s_full1")
+                yield ("arrive", f"k_empty{(JJ + 1) % NK}")
                 if j + 2 == n:
                     yield ("arrive", "q_empty")
             elif n == 1 and not early_release:
@@ -90,31 +117,30 @@ def mma(segs, early_release):
 
 
 def softmax(segs, i):
+    # one thread per row: no barrier among the softmax threads
     J = 0
     for k, n in enumerate(segs):
         yield ("wait", "q_full", k)
         for j in range(n):
             JJ = J + j
             yield ("wait", f"s_full{i}", JJ)
-            yield ("sync", f"pair{i}")
             yield ("arrive", f"p_full{i}")
         yield ("wait", f"o_full{i}", k)
-        yield ("sync", f"grp{i}")
-        yield ("sync", f"grp{i}")
         J += n
 
 
 SOFT = 2  # softmax threads per tile group in the model
 
 
-def run(segs, early_release, seed, pre0=0):
+def run(segs, early_release, seed, prefetch=False):
     """Returns None when every role finishes cleanly, else a description."""
     bars = {"q_full": Bar(2), "q_empty": Bar(1), "s_full0": Bar(1), "s_full1": Bar(1),
             "p_full0": Bar(SOFT), "p_full1": Bar(SOFT), "o_full0": Bar(1), "o_full1": Bar(1)}
-    for s in range(NS):
-        for b in ("k_full", "v_full", "kv_empty"):
-            bars[f"{b}{s}"] = Bar(1)
-    threads = {"producer": producer(segs, pre0), "mma": mma(segs, early_release)}
+    for s in range(NK):
+        bars[f"k_full{s}"], bars[f"k_empty{s}"] = Bar(1), Bar(1)
+    for s in range(NV):
+        bars[f"v_full{s}"], bars[f"v_empty{s}"] = Bar(1), Bar(1)
+    threads = {"producer": producer(segs, prefetch), "mma": mma(segs, early_release)}
     for i in range(2):
         for t in range(SOFT):
             threads[f"soft{i}.{t}"] = softmax(segs, i)
@@ -185,9 +211,8 @@ PATTERNS = [[17, 9], [17, 8, 1], [3, 1, 2], [1, 1, 1, 1], [2, 1, 1, 3], [4, 1, 4
 @pytest.mark.parametrize("prefetch", [False, True])
 @pytest.mark.parametrize("segs", PATTERNS, ids=["-".join(map(str, p)) for p in PATTERNS])
 def test_protocol_has_no_stall_or_aliased_wait(segs, prefetch):
-    pre0 = min(segs[0], NS) if prefetch else 0  # a first segment of prefix tiles
     for seed in range(150):
-        msg = run(segs, early_release=False, seed=seed, pre0=pre0)
+        msg = run(segs, early_release=False, seed=seed, prefetch=prefetch)
         assert msg is None, f"seed {seed}: {msg}"
 
 
@@ -270,3 +295,340 @@ def run_lse(tiles, nk, n_stats, seed):
 def test_lse_protocol_has_no_stall_or_aliased_wait(tiles, nk):
     for seed in range(100):
         assert run_lse(tiles, nk, 3, seed) is None
+
+
+# ---------------------------------------------------------------- the timeout path: nothing in flight at exit
+#
+# A second model with the asynchronous parts made explicit.  TMA loads are
+# in-flight items that arrive on their barrier when they land (in any order);
+# tcgen05 MMAs and commits are a queue that the tensor core executes in order,
+# a commit arriving on its barrier once every MMA before it has completed.  At
+# some random moment a thread blocked on a wait times out: the CTA's abort
+# flag is set, and from then on every wait that checks the flag and is not
+# already satisfied returns false at once.  Each role then winds down the way
+# the kernel does, meets the others at the final CTA barrier, and the MMA warp
+# frees TMEM.  The check: when TMEM is freed and the CTA exits, no TMA load
+# and no MMA or commit may still be pending (a load landing in the shared
+# memory of an exited CTA, or an MMA writing freed TMEM, is what the drain
+# exists to prevent).  Under the earlier rule (the producer leaves without
+# waiting for its loads, the MMA warp's final drain wait gives up as soon as
+# the flag is set) the check fails; under the drain rule it holds.
+
+
+def a_producer(segs, drain, prefetch=True):
+    pk, pv, pre = _preload(segs, prefetch)
+    armed = {"k": 0, "v": 0}
+    for kind, j in pre:
+        yield ("tma", f"{kind}_full{j % (NK if kind == 'k' else NV)}")
+        armed[kind] = j + 1
+    J, q_armed, ok = 0, 0, True
+    for k, n in enumerate(segs):
+        if not ok:
+            break
+        if k > 0:
+            ok = yield ("wait", "q_empty", k - 1, True)
+            if not ok:
+                break
+        yield ("tma", "q_full")
+        q_armed += 1
+        yield ("arrive", "q_full")  # the published segment description
+        for kind, j in _producer_order(n, (pk, pv) if k == 0 else (0, 0)):
+            JJ = J + j
+            ns = NK if kind == "k" else NV
+            if JJ >= ns:
+                ok = yield ("wait", f"{kind}_empty{JJ % ns}", JJ // ns - 1, True)
+                if not ok:
+                    break
+            yield ("tma", f"{kind}_full{JJ % ns}")
+            armed[kind] = JJ + 1
+        J += n
+    if drain:
+        # the last phase of every stage it armed, and of the Q buffer, ignoring the flag
+        for kind, ns in (("k", NK), ("v", NV)):
+            for s in range(ns):
+                uses = (armed[kind] - s + ns - 1) // ns if armed[kind] > s else 0
+                if uses:
+                    yield ("wait", f"{kind}_full{s}", uses - 1, False)
+        if q_armed:
+            yield ("wait", "q_full", q_armed - 1, False)
+    yield ("final",)
+
+
+def a_mma(segs, drain):
+    J, ok = 0, True
+    for k, n in enumerate(segs):
+        if not ok:
+            break
+        ok = yield ("wait", "q_full", k, True)
+        if ok:
+            ok = yield ("wait", f"k_full{J % NK}", J // NK, True)
+            if ok:
+                for i in range(2):
+                    yield ("mma",)
+                    yield ("commit", f"s_full{i}")
+                yield ("commit", f"k_empty{J % NK}")
+        for j in range(n):
+            if not ok:
+                break
+            JJ = J + j
+            ok = yield ("wait", f"v_full{JJ % NV}", JJ // NV, True)
+            if ok:
+                ok = yield ("wait", "p_full0", JJ, True)
+            if not ok:
+                break
+            yield ("mma",)
+            if j == n - 1:
+                yield ("commit", "o_full0")
+            if j + 1 < n:
+                ok = yield ("wait", f"k_full{(JJ + 1) % NK}", (JJ + 1) // NK, True)
+                if not ok:
+                    break
+                yield ("mma",)
+                yield ("commit", "s_full0")
+            ok = yield ("wait", "p_full1", JJ, True)
+            if not ok:
+                break
+            yield ("mma",)
+            yield ("commit", f"v_empty{JJ % NV}")
+            if j == n - 1:
+                yield ("commit", "o_full1")
+            if j + 1 < n:
+                yield ("mma",)
+                yield ("commit", "s_full1")
+                yield ("commit", f"k_empty{(JJ + 1) % NK}")
+                if j + 2 == n:
+                    yield ("commit", "q_empty")
+            elif n == 1:
+                yield ("commit", "q_empty")
+        J += n
+    yield ("commit", "drain")
+    yield ("wait", "drain", 0, not drain)  # the drain rule ignores the flag
+    yield ("final",)
+    yield ("dealloc",)
+
+
+def a_softmax(segs, i):
+    # a failed wait ends the thread's work (its warp leaves together)
+    J, ok = 0, True
+    for k, n in enumerate(segs):
+        ok = yield ("wait", "q_full", k, True)
+        if not ok:
+            break
+        for j in range(n):
+            ok = yield ("wait", f"s_full{i}", J + j, True)
+            if not ok:
+                break
+            yield ("arrive", f"p_full{i}")
+        if not ok:
+            break
+        ok = yield ("wait", f"o_full{i}", k, True)
+        if not ok:
+            break
+        J += n
+    yield ("final",)
+
+
+def _async_run(threads, bars, group_of, seed, p_timeout):
+    """Random interleaving of roles, in-flight TMA loads and the tensor-core
+    queue, with at most one timeout; None when the CTA exits with nothing in
+    flight, else a description."""
+    cur = {name: next(g) for name, g in threads.items()}
+    tma, tc_queue = [], []  # loads in flight (barrier names); MMA / commit queue
+    rng = random.Random(seed)
+    state = {"abort": False}
+
+    def arrive(name):
+        b = bars[name]
+        b.pending += 1
+        if b.pending == b.count:
+            b.pending, b.phase = 0, b.phase + 1
+
+    def ready(op):
+        return (bars[op[1]].phase & 1) != (op[2] & 1)
+
+    def advance(n, value=None):
+        try:
+            cur[n] = threads[n].send(value)
+        except StopIteration:
+            cur[n] = None
+
+    for _ in range(400000):
+        live = [n for n, op in cur.items() if op is not None]
+        if not live:
+            return None
+        moves = []
+        for n in live:
+            op = cur[n]
+            if op[0] in ("arrive", "tma", "mma", "commit", "dealloc"):
+                moves.append(("run", n))
+            elif op[0] == "wait":
+                if ready(op) or (op[3] and state["abort"]):
+                    moves.append(("run", n))
+                elif op[3] and not state["abort"] and rng.random() < p_timeout:
+                    moves.append(("timeout", n))
+            elif all(cur[m] is not None and cur[m][:2] == op[:2] for m in group_of(op)):
+                moves.append(("run", n))
+        if tma:
+            moves.append(("tma_done", None))
+        if tc_queue:
+            moves.append(("tc_step", None))
+        if not moves:
+            return "deadlock: " + ", ".join(f"{n}@{cur[n]}" for n in live)
+        kind, n = rng.choice(moves)
+        if kind == "tma_done":
+            arrive(tma.pop(rng.randrange(len(tma))))
+            continue
+        if kind == "tc_step":
+            item = tc_queue.pop(0)
+            if item[0] == "commit":
+                arrive(item[1])
+            continue
+        op = cur[n]
+        if kind == "timeout":
+            state["abort"] = True
+            advance(n, False)
+            continue
+        if op[0] == "arrive":
+            arrive(op[1])
+            advance(n)
+        elif op[0] == "tma":
+            tma.append(op[1])
+            advance(n)
+        elif op[0] in ("mma", "commit"):
+            tc_queue.append(op)
+            advance(n)
+        elif op[0] == "dealloc":
+            if tma or tc_queue:
+                return f"TMEM freed and CTA exiting with {len(tma)} loads and {len(tc_queue)} tensor-core ops pending"
+            advance(n)
+        elif op[0] == "wait":
+            advance(n, ready(op))
+        else:  # sync / syncand / final: release the whole group together
+            members = group_of(op)
+            val = all(cur[m][2] for m in members) if op[0] == "syncand" else None
+            for m in members:
+                advance(m, val)
+    return "step limit"
+
+
+def run_abort(segs, drain, seed, p_timeout=0.02):
+    bars = {"q_full": Bar(2), "q_empty": Bar(1), "s_full0": Bar(1), "s_full1": Bar(1), "drain": Bar(1),
+            "p_full0": Bar(SOFT), "p_full1": Bar(SOFT), "o_full0": Bar(1), "o_full1": Bar(1)}
+    for s in range(NK):
+        bars[f"k_full{s}"], bars[f"k_empty{s}"] = Bar(1), Bar(1)
+    for s in range(NV):
+        bars[f"v_full{s}"], bars[f"v_empty{s}"] = Bar(1), Bar(1)
+    threads = {"producer": a_producer(segs, drain), "mma": a_mma(segs, drain)}
+    for i in range(2):
+        for t in range(SOFT):
+            threads[f"soft{i}.{t}"] = a_softmax(segs, i)
+
+    def group_of(op):
+        if op[0] == "final":
+            return list(threads)
+        return [m for m in threads if m.startswith("soft" + op[1][-1] + ".")]
+    return _async_run(threads, bars, group_of, seed, p_timeout)
+
+
+ABORT_PATTERNS = [[5], [3, 2], [17, 9], [1, 1, 1], [4, 1, 4, 1], [2, 3]]
+
+
+@pytest.mark.parametrize("segs", ABORT_PATTERNS, ids=["-".join(map(str, p)) for p in ABORT_PATTERNS])
+def test_timeout_path_drains_before_exit(segs):
+    for seed in range(300):
+        msg = run_abort(segs, drain=True, seed=seed)
+        assert msg is None, f"seed {seed}: {msg}"
+
+
+def test_timeout_path_without_drain_can_exit_with_work_in_flight():
+    bad = [run_abort(s, drain=False, seed=seed) for s in ABORT_PATTERNS for seed in range(200)]
+    bad = [m for m in bad if m is not None]
+    assert bad and all("pending" in m for m in bad), bad[:3]
+
+
+def test_normal_path_of_the_async_model_is_clean():
+    # no timeout at all: both rules exit cleanly
+    for segs in ABORT_PATTERNS:
+        for seed in range(50):
+            assert run_abort(segs, drain=True, seed=seed, p_timeout=0.0) is None
+            assert run_abort(segs, drain=False, seed=seed, p_timeout=0.0) is None
+
+
+# the full-vocabulary LSE kernel's roles with the same asynchronous parts and timeout
+
+
+def a_lse_producer(tiles, nk, drain):
+    it, ok = 0, True
+    for _ in range(tiles):
+        for _ in range(nk):
+            st = it % LS
+            if it >= LS:
+                ok = yield ("wait", f"empty{st}", it // LS - 1, True)
+                if not ok:
+                    break
+            yield ("tma", f"full{st}")
+            it += 1
+        if not ok:
+            break
+    if drain:
+        for s in range(LS):
+            uses = (it - s + LS - 1) // LS if it > s else 0
+            if uses:
+                yield ("wait", f"full{s}", uses - 1, False)
+    yield ("final",)
+
+
+def a_lse_mma(tiles, nk, drain):
+    it, ok = 0, True
+    for tile in range(tiles):
+        if tile > 0:
+            ok = yield ("wait", "sempty", tile - 1, True)
+            if not ok:
+                break
+        for _ in range(nk):
+            st = it % LS
+            ok = yield ("wait", f"full{st}", it // LS, True)
+            if not ok:
+                break
+            yield ("mma",)
+            yield ("commit", f"empty{st}")
+            it += 1
+        if not ok:
+            break
+        yield ("commit", "sfull")
+    yield ("commit", "drain")
+    yield ("wait", "drain", 0, not drain)
+    yield ("final",)
+    yield ("dealloc",)
+
+
+def a_lse_stats(tiles):
+    for tile in range(tiles):
+        yield ("wait", "sfull", tile, True)
+        yield ("arrive", "sempty")
+    yield ("final",)
+
+
+def run_lse_abort(tiles, nk, n_stats, drain, seed, p_timeout=0.02):
+    bars = {"sfull": Bar(1), "sempty": Bar(n_stats), "drain": Bar(1)}
+    for s in range(LS):
+        bars[f"full{s}"], bars[f"empty{s}"] = Bar(1), Bar(1)
+    threads = {"producer": a_lse_producer(tiles, nk, drain), "mma": a_lse_mma(tiles, nk, drain)}
+    for t in range(n_stats):
+        threads[f"stats{t}"] = a_lse_stats(tiles)
+    return _async_run(threads, bars, lambda op: list(threads), seed, p_timeout)
+
+
+@pytest.mark.parametrize("tiles,nk", [(1, 1), (5, 2), (4, 7), (9, 3)])
+def test_lse_timeout_path_drains_before_exit(tiles, nk):
+    for seed in range(300):
+        msg = run_lse_abort(tiles, nk, 3, drain=True, seed=seed)
+        assert msg is None, f"seed {seed}: {msg}"
+
+
+def test_lse_timeout_path_without_drain_can_exit_with_work_in_flight():
+    bad = [run_lse_abort(t, k, 3, drain=False, seed=seed) for t, k in [(5, 2), (4, 7)] for seed in range(300)]
+    bad = [m for m in bad if m is not None]
+    assert bad and all("pending" in m for m in bad), bad[:3]
+    for seed in range(50):  # no timeout: both rules exit cleanly
+        assert run_lse_abort(4, 7, 3, drain=False, seed=seed, p_timeout=0.0) is None
