@@ -25,6 +25,7 @@ _lib = C.CDLL(LIB_PATH)
 
 JEV_F32, JEV_BF16 = 0, 1
 JEV_DEV_BAD_SEQLENS, JEV_DEV_BAD_HEAD_MAP, JEV_DEV_BAD_TREE, JEV_DEV_WAIT_TIMEOUT, JEV_DEV_BAD_WINDOW = 1, 2, 4, 8, 16
+JEV_DEV_BAD_CACHE = 32
 STATUS_NAMES = {0: "JEV_OK", 1: "JEV_ERR_INVALID_ARG", 2: "JEV_ERR_UNSUPPORTED", 3: "JEV_ERR_WORKSPACE",
                 4: "JEV_ERR_CUDA", 5: "JEV_ERR_DEVICE", 6: "JEV_ERR_CAPACITY"}
 
@@ -180,6 +181,48 @@ def jev_prefix_suffix_attn(q, k_pre, v_pre, k_suf, v_suf, cu_seqlens, *, head_ma
     _check(_lib.jev_prefix_suffix_attn(C.byref(desc), _p(q), _p(k_pre), _p(v_pre), _p(k_suf), _p(v_suf),
                                        _p(cu_seqlens), _p(head_map), _p(out), _p(lse), _p(workspace),
                                        workspace.numel(), _stream(stream)), "jev_prefix_suffix_attn")
+    return out, lse
+
+
+_lib.jev_suffix_cache_attn_workspace.argtypes = [C.POINTER(jev_attn_desc)]
+_lib.jev_suffix_cache_attn_workspace.restype = _sz
+_lib.jev_suffix_cache_attn.argtypes = [C.POINTER(jev_attn_desc)] + [_vp] * 7 + [_i32] + [_vp] * 7 + [_sz, _vp]
+_lib.jev_suffix_cache_attn.restype = C.c_int
+
+
+def jev_suffix_cache_attn_workspace(desc: jev_attn_desc) -> int:
+    return int(_lib.jev_suffix_cache_attn_workspace(C.byref(desc)))
+
+
+def jev_suffix_cache_attn(q, k_new, v_new, k_pre, v_pre, k_cache, v_cache, cache_off, cache_len, cu_new, *,
+                          head_map=None, out=None, lse=None, workspace=None, rope_theta=1e4, softmax_scale=0.0,
+                          pos_offset=-1, num_splits=0, want_lse=True, stream=None):
+    """New tokens of B branches over the shared prefix and each branch's cached
+    suffix; appends their rotated keys and values to the caches (cache_len is
+    not changed).  Returns (out, lse)."""
+    dt = _dtype_code(q)
+    T, Hq, d = q.shape
+    Lp, Hkv = k_pre.shape[0], k_pre.shape[1]
+    for t, n in ((q, "q"), (k_new, "k_new"), (v_new, "v_new"), (k_pre, "k_pre"), (v_pre, "v_pre"),
+                 (k_cache, "k_cache"), (v_cache, "v_cache")):
+        _dev(t, n, q.dtype)
+    for t, n in ((cache_off, "cache_off"), (cache_len, "cache_len"), (cu_new, "cu_new"), (head_map, "head_map")):
+        _dev(t, n, torch.int32)
+    B = cu_new.numel() - 1
+    desc = _cached_desc(make_attn_desc, (B, Lp, Hq, Hkv, d, T, dt, rope_theta, softmax_scale, pos_offset,
+                                         num_splits, 0))
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((T, Hq), dtype=torch.float32, device=q.device)
+    _dev(out, "out", q.dtype)
+    _dev(lse, "lse", torch.float32)
+    if workspace is None:
+        workspace = new_workspace(jev_suffix_cache_attn_workspace(desc), q.device)
+    _check(_lib.jev_suffix_cache_attn(C.byref(desc), _p(q), _p(k_new), _p(v_new), _p(k_pre), _p(v_pre),
+                                      _p(k_cache), _p(v_cache), int(k_cache.shape[0]), _p(cache_off),
+                                      _p(cache_len), _p(cu_new), _p(head_map), _p(out), _p(lse), _p(workspace),
+                                      workspace.numel(), _stream(stream)), "jev_suffix_cache_attn")
     return out, lse
 
 
@@ -408,3 +451,12 @@ def jev_profile_read(keep: bool = False) -> dict:
 
 def jev_launch_count() -> int:
     return int(_lib.jev_launch_count())
+
+
+_lib.jev_debug_set_wait_limit.argtypes = [C.c_int64]
+_lib.jev_debug_set_wait_limit.restype = C.c_int
+
+
+def jev_debug_set_wait_limit(cycles: int):
+    """Bound of the tensor-core kernels' mbarrier waits for later launches (0: the default)."""
+    _check(_lib.jev_debug_set_wait_limit(int(cycles)), "jev_debug_set_wait_limit")

@@ -8,8 +8,8 @@
 // scores and d/32 output columns for P.V.  The online softmax runs in the
 // log2 domain.  The block that holds the last prefix split also walks the
 // suffix keys its rows may see: for a flat branch, the keys of the same branch
-// up to the row's own token; for a tree token, every non-root ancestor's keys
-// plus its own node's keys up to itself.
+// up to the row's own token (or its slot in the branch's cache); for a tree
+// token, every non-root ancestor's keys plus its own node's keys up to itself.
 #include <math_constants.h>
 
 #include "kernels.h"
@@ -27,9 +27,9 @@ __global__ void __launch_bounds__(kThreads) attn_simt_kernel(AttnArgs a) {
   __shared__ float Qs[kRows][D];
   __shared__ float Ks[kKeys][D + 1];
   __shared__ float Vs[kKeys][D];
-  __shared__ int r_t[kRows], r_start[kRows], r_nanc[kRows];
-  __shared__ int2 r_anc[kRows][kMaxDepth];
+  __shared__ int r_t[kRows], r_start[kRows], r_last[kRows];
   __shared__ int s_lo, s_hi;
+  const bool tree = a.key_end != nullptr;
 
   const int g = blockIdx.y, split = blockIdx.z;
   const int m0 = blockIdx.x * kRows;
@@ -43,22 +43,17 @@ __global__ void __launch_bounds__(kThreads) attn_simt_kernel(AttnArgs a) {
   }
   if (tid < kRows) {
     int m = m0 + tid;
+    r_t[tid] = -1;
+    r_start[tid] = 0;
+    r_last[tid] = -1;
     if (m < a.M) {
-      int t = m / a.G;
-      TokInfo inf = a.info[t];
-      int nanc = 0;
-      if (a.node_nanc) {
-        nanc = a.node_nanc[inf.node];
-        if (nanc < 0) t = -1;  // malformed tree: row sees no suffix keys and is not written
-        for (int k = 0; k < nanc; ++k) r_anc[tid][k] = a.node_anc[(size_t)inf.node * kMaxDepth + k];
+      const int t = m / a.G;
+      const TokInfo inf = a.info[t];
+      if (inf.node >= 0) {  // a skipped row sees no suffix keys and is not written
+        r_t[tid] = t;
+        r_start[tid] = inf.seg_start;
+        r_last[tid] = tree ? t : inf.last;
       }
-      r_t[tid] = t;
-      r_start[tid] = inf.seg_start;
-      r_nanc[tid] = nanc > 0 ? nanc : 0;
-    } else {
-      r_t[tid] = -1;
-      r_start[tid] = 0;
-      r_nanc[tid] = 0;
     }
   }
   __syncthreads();
@@ -66,9 +61,8 @@ __global__ void __launch_bounds__(kThreads) attn_simt_kernel(AttnArgs a) {
     int lo = INT_MAX, hi = -1;
     for (int r = 0; r < kRows; ++r) {
       if (r_t[r] < 0) continue;
-      int start = r_nanc[r] > 0 ? min(r_anc[r][0].x, r_start[r]) : r_start[r];
-      lo = min(lo, start);
-      hi = max(hi, r_t[r]);
+      lo = min(lo, r_start[r]);
+      hi = max(hi, r_last[r]);
     }
     s_lo = lo;
     s_hi = hi;
@@ -95,6 +89,9 @@ __global__ void __launch_bounds__(kThreads) attn_simt_kernel(AttnArgs a) {
     }
     __syncthreads();
     float p[4];
+    const int key = kb + lane;
+    // tree key: the end of the packed tokens of its node's subtree
+    const int kend = suffix && tree && lane < n ? a.key_end[key] : -1;
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
       const int rr = warp * 4 + r;
@@ -102,13 +99,9 @@ __global__ void __launch_bounds__(kThreads) attn_simt_kernel(AttnArgs a) {
 #pragma unroll 8
       for (int i = 0; i < D; ++i) s += Qs[rr][i] * Ks[lane][i];
       s *= a.scale_log2;
-      const int key = kb + lane;
       bool ok = lane < n && r_t[rr] >= 0;
-      if (ok && suffix) {
-        bool vis = key >= r_start[rr] && key <= r_t[rr];
-        for (int k = 0; k < r_nanc[rr]; ++k) vis |= (key >= r_anc[rr][k].x && key < r_anc[rr][k].y);
-        ok = vis;
-      }
+      if (ok && suffix)
+        ok = tree ? (key <= r_t[rr] && r_t[rr] < kend) : (key >= r_start[rr] && key <= r_last[rr]);
       s = ok ? s : -CUDART_INF_F;
       const float mx = warp_max(s);
       const float m_new = fmaxf(m_r[r], mx);

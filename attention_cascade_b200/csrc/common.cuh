@@ -50,15 +50,22 @@ __device__ __forceinline__ int upper_segment(const int32_t* offs, int n, int t) 
   return lo;
 }
 
-// Per packed token: where its own segment starts and its RoPE position.
-// Tree tokens additionally carry up to kMaxAnc ancestor key ranges.
-constexpr int kMaxDepth = 8;  // non-root ancestors + own node
-
+// Per query token, written by the RoPE pack.  Suffix keys are rows of the
+// suffix key tensor (the packed suffix, the tree tokens, or a per-branch
+// cache); a row sees the keys [seg_start, last] that pass its mask.
+//   flat row:  keys seg_start .. last of its own branch (its own token, or its
+//              slot in the branch's cache), all visible;
+//   tree token: as a row, the keys from seg_start (the first token of its
+//              top-level ancestor) up to itself that lie on its root path;
+//              as a key, `last` is the end of the packed-token range of its
+//              node's subtree, so key k is visible to tree row t exactly when
+//              k <= t < last(k) (nodes and tokens in depth-first preorder).
+// node < 0 marks a row that is not computed (malformed input, already flagged).
 struct TokInfo {
-  int32_t seg_start;  // first packed key of the token's own segment (branch or node)
+  int32_t seg_start;  // first suffix key of the row's window
   int32_t pos;        // RoPE position of the token
-  int32_t node;       // tree node (flat: branch index)
-  int32_t n_anc;      // number of ancestor ranges (flat: 0)
+  int32_t node;       // tree node / branch index; -1: row skipped
+  int32_t last;       // flat: last visible key; tree: subtree token end (key side)
 };
 
 }  // namespace jev

@@ -41,6 +41,10 @@ std::vector<Rec> g_recs;
 std::vector<cudaEvent_t> g_pool;
 std::vector<std::string> g_names;
 std::atomic<long long> g_launches{0};
+// bound of the tensor-core kernels' mbarrier waits, in clock cycles (about a
+// second at the B200's clock); jev_debug_set_wait_limit changes it
+constexpr long long kDefaultWaitCycles = 1LL << 31;
+std::atomic<long long> g_wait_cycles{kDefaultWaitCycles};
 
 int name_id(const char* n) {
   for (size_t i = 0; i < g_names.size(); ++i)
@@ -290,16 +294,19 @@ Plan plan_of(const jev_attn_desc* d, int T, int kernel = -1, int sms_hint = 0) {
 }
 
 struct Layout {
-  size_t hinv, info, qrot, krot, opart, lpart, anc, nanc, total;
+  size_t hinv, info, qrot, krot, opart, lpart, kend, total;
 };
-Layout layout_of(const jev_attn_desc* d, int T, const Plan& p, int n_nodes) {
+// cache: a generation step writes its rotated keys into the caller's cache,
+// so the workspace holds no rotated-key buffer
+Layout layout_of(const jev_attn_desc* d, int T, const Plan& p, int n_nodes, bool cache = false) {
   Layout L;
   const size_t s = esize(d->dtype);
   size_t off = kStatusBytes;
   L.hinv = off; off += up256((size_t)d->Hq * 4);
   L.info = off; off += up256((size_t)T * sizeof(TokInfo));
   L.qrot = off; off += up256((size_t)p.M * d->Hkv * d->d * s);
-  L.krot = off; off += up256((size_t)T * d->Hkv * d->d * s);
+  L.krot = off;
+  if (!cache) off += up256((size_t)T * d->Hkv * d->d * s);
   L.opart = off;
   L.lpart = off;
   if (p.tc && p.split) {
@@ -310,10 +317,9 @@ Layout layout_of(const jev_attn_desc* d, int T, const Plan& p, int n_nodes) {
     L.opart = off; off += up256((size_t)p.S * d->Hkv * p.M * d->d * 4);
     L.lpart = off; off += up256((size_t)p.S * d->Hkv * p.M * 4);
   }
-  L.anc = off; L.nanc = off;
+  L.kend = off;
   if (n_nodes > 0) {
-    L.anc = off; off += up256((size_t)n_nodes * kMaxDepth * sizeof(int2));
-    L.nanc = off; off += up256((size_t)n_nodes * 4);
+    L.kend = off; off += up256((size_t)T * 4);
   }
   L.total = off;
   return L;
@@ -338,36 +344,54 @@ float scale_log2_of(const jev_attn_desc* d) {
   return (float)(sc * 1.4426950408889634);
 }
 
-// Shared tail of the flat and tree entry points.
+// Per-branch suffix caches of a generation step (jev_suffix_cache_attn).
+struct CacheArgs {
+  void* k_cache;
+  void* v_cache;
+  int rows;
+  const int32_t* off;
+  const int32_t* len;
+};
+
+// Shared tail of the flat, tree and cache entry points.
 jev_status attention_core(const jev_attn_desc* d, int T, const Plan& p, const Layout& L, char* ws,
                           const void* q, const void* k_pre, const void* v_pre, const void* k_suf,
                           const void* v_suf, const int32_t* offs, int n_segs, const int32_t* pos0,
                           const int32_t* head_map, bool tree, const int32_t* tree_parent, void* out, float* lse,
-                          cudaStream_t s) {
+                          cudaStream_t s, const CacheArgs* cache = nullptr) {
   int32_t* status = reinterpret_cast<int32_t*>(ws);
+  jev_status st = JEV_OK;
   RopePackArgs r{};
   r.q = q; r.k = k_suf;
-  r.q_rot = ws + L.qrot; r.k_rot = ws + L.krot;
+  r.q_rot = ws + L.qrot;
+  r.k_rot = cache ? cache->k_cache : ws + L.krot;
   r.info = reinterpret_cast<TokInfo*>(ws + L.info);
   r.hinv = reinterpret_cast<int32_t*>(ws + L.hinv);
   r.status = status;
   r.offs = offs; r.pos0 = pos0; r.head_map = head_map;
-  r.parent = tree_parent;
-  r.node_anc = tree ? reinterpret_cast<int2*>(ws + L.anc) : nullptr;
-  r.node_nanc = tree ? reinterpret_cast<int32_t*>(ws + L.nanc) : nullptr;
+  r.parent = tree ? tree_parent : nullptr;
+  r.key_end = tree ? reinterpret_cast<int32_t*>(ws + L.kend) : nullptr;
+  if (cache) {
+    r.cache_off = cache->off;
+    r.cache_len = cache->len;
+    r.v = v_suf;
+    r.v_cache = cache->v_cache;
+  }
+  r.key_rows = cache ? cache->rows : T;
   r.n_segs = n_segs; r.T = T; r.Hq = d->Hq; r.Hkv = d->Hkv; r.d = d->d;
   r.pos_offset = d->pos_offset >= 0 ? d->pos_offset : d->Lp;
   r.pos_seq = d->pos_mode == 1 ? 1 : 0;
   r.theta = (double)d->rope_theta;
   for (int i = 0; i < d->d / 2; ++i) r.inv_freq[i] = std::pow(r.theta, -2.0 * i / d->d);
-  jev_status st = run("rope_pack", s, [&] { return launch_rope_pack(r, d->dtype, s); });
+  st = run("rope_pack", s, [&] { return launch_rope_pack(r, d->dtype, s); });
   if (st) return st;
 
   AttnArgs a{};
-  a.q_rot = r.q_rot; a.k_pre = k_pre; a.v_pre = v_pre; a.k_rot = r.k_rot; a.v_suf = v_suf;
+  a.q_rot = r.q_rot; a.k_pre = k_pre; a.v_pre = v_pre; a.k_rot = r.k_rot;
+  a.v_suf = cache ? cache->v_cache : v_suf;
   a.info = r.info;
-  a.node_anc = tree ? reinterpret_cast<const int2*>(ws + L.anc) : nullptr;
-  a.node_nanc = tree ? reinterpret_cast<const int32_t*>(ws + L.nanc) : nullptr;
+  a.key_end = r.key_end;
+  a.key_rows = r.key_rows;
   a.hinv = r.hinv;
   a.out = out; a.lse = lse;
   a.o_part = reinterpret_cast<float*>(ws + L.opart);
@@ -378,6 +402,7 @@ jev_status attention_core(const jev_attn_desc* d, int T, const Plan& p, const La
   a.scale_log2 = scale_log2_of(d);
   a.n_pairs = p.n_pairs; a.n_tiles = p.n_tiles; a.n_pre = p.n_pre; a.P = p.P; a.n_ctas = p.n_ctas; a.U = p.U;
   a.full_waves = p.full_waves; a.tail0 = p.tail0; a.tail_ctas = p.tail_ctas;
+  a.wait_cycles = g_wait_cycles.load();
   if (p.tc) {
     st = run("attn_tc", s, [&] { return launch_attn_tc(a, s); });
     if (st == JEV_OK && p.split) st = run("tc_fixup", s, [&] { return launch_tc_fixup(a, s); });
@@ -387,7 +412,7 @@ jev_status attention_core(const jev_attn_desc* d, int T, const Plan& p, const La
   if (st) return st;
   if (p.S > 1) {
     MergeArgs m{};
-    m.o_part = a.o_part; m.l_part = a.l_part; m.hinv = a.hinv; m.out = out; m.lse = lse;
+    m.o_part = a.o_part; m.l_part = a.l_part; m.info = a.info; m.hinv = a.hinv; m.out = out; m.lse = lse;
     m.M = p.M; m.Hq = d->Hq; m.Hkv = d->Hkv; m.G = p.G; m.d = d->d; m.S = p.S;
     st = run("merge_splits", s, [&] { return launch_merge(m, d->dtype, s); });
   }
@@ -428,6 +453,12 @@ extern "C" {
 const char* jev_last_error(void) { return g_err; }
 
 int64_t jev_launch_count(void) { return (int64_t)g_launches.load(); }
+
+jev_status jev_debug_set_wait_limit(int64_t cycles) {
+  if (cycles < 0) return fail(JEV_ERR_INVALID_ARG, "wait limit must be >= 0");
+  g_wait_cycles.store(cycles == 0 ? kDefaultWaitCycles : (long long)cycles);
+  return JEV_OK;
+}
 
 jev_status jev_profile_enable(int32_t on) {
   g_prof.store(on != 0);
@@ -536,6 +567,40 @@ jev_status jev_prefix_suffix_attn(const jev_attn_desc* d, const void* q, const v
   if (ws_bytes < L.total) return fail(JEV_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", ws_bytes, L.total);
   return attention_core(d, T, p, L, (char*)workspace, q, k_pre, v_pre, k_suf, v_suf, cu_seqlens, d->B, nullptr,
                         head_map, false, nullptr, out, lse, (cudaStream_t)stream);
+}
+
+size_t jev_suffix_cache_attn_workspace(const jev_attn_desc* d) {
+  if (check_desc(d) != JEV_OK) return 0;
+  Plan p = plan_of(d, d->T_total);
+  return layout_of(d, d->T_total, p, 0, true).total;
+}
+
+jev_status jev_suffix_cache_attn(const jev_attn_desc* d, const void* q, const void* k_new, const void* v_new,
+                                 const void* k_pre, const void* v_pre, void* k_cache, void* v_cache,
+                                 int32_t cache_rows, const int32_t* cache_off, const int32_t* cache_len,
+                                 const int32_t* cu_new, const int32_t* head_map, void* out, float* lse,
+                                 void* workspace, size_t ws_bytes, jev_stream_t stream) {
+  jev_status st = check_desc(d);
+  if (st) return st;
+  if (d->pos_mode != 0) return fail(JEV_ERR_INVALID_ARG, "positions follow each branch's cache (pos_mode must be 0)");
+  if (d->B == 0 || d->T_total == 0) return JEV_OK;
+  if (!q || !k_new || !v_new || !k_cache || !v_cache || !cache_off || !cache_len || !cu_new || !out)
+    return fail(JEV_ERR_INVALID_ARG, "required pointer is NULL");
+  if (d->Lp > 0 && (!k_pre || !v_pre)) return fail(JEV_ERR_INVALID_ARG, "prefix pointers are NULL with Lp > 0");
+  if (cache_rows < 1) return fail(JEV_ERR_INVALID_ARG, "cache_rows must be >= 1");
+  const void* ptrs[] = {q, k_new, v_new, k_pre, v_pre, k_cache, v_cache, out, lse};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return fail(JEV_ERR_INVALID_ARG, "tensor pointer not 16-byte aligned");
+  if (((uintptr_t)cache_off | (uintptr_t)cache_len | (uintptr_t)cu_new) & 3)
+    return fail(JEV_ERR_INVALID_ARG, "index array misaligned");
+  const int T = d->T_total;
+  Plan p = plan_of(d, T);
+  Layout L = layout_of(d, T, p, 0, true);
+  if (!workspace || ((uintptr_t)workspace & 255)) return fail(JEV_ERR_WORKSPACE, "workspace NULL or not 256-byte aligned");
+  if (ws_bytes < L.total) return fail(JEV_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", ws_bytes, L.total);
+  const CacheArgs ca{k_cache, v_cache, cache_rows, cache_off, cache_len};
+  return attention_core(d, T, p, L, (char*)workspace, q, k_pre, v_pre, k_new, v_new, cu_new, d->B, nullptr,
+                        head_map, false, nullptr, out, lse, (cudaStream_t)stream, &ca);
 }
 
 }  // extern "C"
@@ -667,7 +732,8 @@ jev_status jev_vocab_lse(const void* hidden, const void* lm_head, int32_t R, int
   if (ws_bytes < need) return fail(JEV_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", ws_bytes, need);
   const int n_ctas = vocab_lse_ctas(V, num_sms());
   char* ws = (char*)workspace;
-  VocabLseArgs a{hidden, lm_head, R, H, V, (V + 255) / 256, (float2*)(ws + kStatusBytes), lse, (int32_t*)ws};
+  VocabLseArgs a{hidden, lm_head, R, H, V, (V + 255) / 256, (float2*)(ws + kStatusBytes), lse, (int32_t*)ws,
+                 g_wait_cycles.load()};
   const jev_status st =
       run("vocab_lse", (cudaStream_t)stream, [&] { return launch_vocab_lse(a, n_ctas, (cudaStream_t)stream); });
   if (st == JEV_OK) g_launches++;  // GEMM + online LSE, then the partial merge: two kernels

@@ -14,16 +14,25 @@ struct RopePackArgs {
   const void* q;           // [T, Hq, d]
   const void* k;           // [T, Hkv, d]
   void* q_rot;             // [Hkv, T*G, d]
-  void* k_rot;             // [T, Hkv, d]
+  void* k_rot;             // [T, Hkv, d]; cache mode: the key cache [key_rows, Hkv, d]
   TokInfo* info;           // [T]
   int32_t* hinv;           // [Hq]: q-head of group-major slot g*G + s
   int32_t* status;
   const int32_t* offs;     // flat: cu_seqlens [n_segs+1]; tree: tok_off [n_segs+1]
   const int32_t* pos0;     // tree: [n_segs] first-token positions; flat: nullptr
   const int32_t* head_map; // [Hq] or nullptr
-  const int32_t* parent;   // tree: [n_segs] parent node of each node; flat: nullptr
-  int2* node_anc;          // tree: [n_segs, kMaxDepth] ancestor key ranges (written)
-  int32_t* node_nanc;      // tree: [n_segs] ancestor count, -1 for a malformed chain (written)
+  // tree: the parent of every node, and per token (written) the end of the
+  // packed tokens of its node's subtree, for the key side of the mask
+  const int32_t* parent;
+  int32_t* key_end;
+  // cache mode (a generation step over per-branch suffix caches): branch b
+  // owns cache rows [cache_off[b], cache_off[b+1]) of which cache_len[b] are
+  // filled; its new tokens go to the rows after them
+  const int32_t* cache_off;  // [n_segs+1] or nullptr
+  const int32_t* cache_len;  // [n_segs]
+  const void* v;             // cache mode: new values [T, Hkv, d]
+  void* v_cache;             // cache mode: value cache [key_rows, Hkv, d]
+  int key_rows;              // rows of the key tensor the attention reads
   int n_segs, T, Hq, Hkv, d, pos_offset;
   int pos_seq;             // 1: token t at pos_offset + t (sequential across segments)
   double theta;
@@ -31,16 +40,17 @@ struct RopePackArgs {
 };
 cudaError_t launch_rope_pack(const RopePackArgs& a, jev_dtype dt, cudaStream_t s);
 
+
+
 // Attention over [prefix split s ; own suffix window] for the stacked rows of a kv group.
 struct AttnArgs {
   const void* q_rot;        // [Hkv, M, d]
   const void* k_pre;        // [Lp, Hkv, d]
   const void* v_pre;        // [Lp, Hkv, d]
-  const void* k_rot;        // [T, Hkv, d]
-  const void* v_suf;        // [T, Hkv, d]
+  const void* k_rot;        // [key_rows, Hkv, d] rotated suffix keys (or the key cache)
+  const void* v_suf;        // [key_rows, Hkv, d]
   const TokInfo* info;      // [T]
-  const int2* node_anc;     // tree: [n_nodes, kMaxDepth]; flat: nullptr
-  const int32_t* node_nanc; // tree: [n_nodes]; flat: nullptr
+  const int32_t* key_end;   // tree: [T] subtree token end of each key's node; flat: nullptr
   const int32_t* hinv;      // [Hq]
   void* out;                // [T, Hq, d] (num_splits == 1)
   float* lse;               // [T, Hq] or nullptr
@@ -48,6 +58,7 @@ struct AttnArgs {
   float* l_part;            // [S, Hkv, M] log2-domain
   int32_t* status;
   int T, M, Lp, Hq, Hkv, G, d, S, split_len;  // split_len: prefix keys per split (multiple of 128)
+  int key_rows;             // rows of k_rot / v_suf
   float scale_log2;         // softmax scale * log2(e)
   // Tensor-core schedule.  Work tile w = (kv group w / n_pairs, 256-row pair
   // w % n_pairs) has P = n_pre + 1 units (one per 128-key prefix tile, one for
@@ -58,6 +69,7 @@ struct AttnArgs {
   // [c*U/tail_ctas, (c+1)*U/tail_ctas) after its whole tiles.
   int n_pairs, n_tiles, n_pre, P, n_ctas, full_waves, tail0, tail_ctas;
   long long U;
+  long long wait_cycles;  // bound of every mbarrier wait (clock cycles)
 };
 // tail units owned by CTAs before c (c <= tail_ctas)
 __host__ __device__ inline long long tc_unit_begin(const AttnArgs& a, int c) { return (long long)c * a.U / a.tail_ctas; }
@@ -73,6 +85,7 @@ cudaError_t launch_exp2_selftest(const float* x, float* y, int n, cudaStream_t s
 struct MergeArgs {
   const float* o_part;  // [S, Hkv, M, d]
   const float* l_part;  // [S, Hkv, M]
+  const TokInfo* info;  // [T]: rows of skipped tokens (node < 0) are not written
   const int32_t* hinv;
   void* out;            // [T, Hq, d]
   float* lse;
@@ -96,6 +109,7 @@ struct VocabLseArgs {
   float2* part;  // [ceil(R/256)][n_ctas][2][256] (max, sum) partials, log2 domain
   float* lse;    // [R] natural log
   int32_t* status;
+  long long wait_cycles;  // bound of every mbarrier wait (clock cycles)
 };
 int vocab_lse_ctas(int V, int sms);
 size_t vocab_lse_partial_bytes(int R, int n_ctas);

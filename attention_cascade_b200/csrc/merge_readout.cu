@@ -52,6 +52,7 @@ __global__ void __launch_bounds__(256) merge_kernel(MergeArgs a) {
   }
   const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
   const int t = m / a.G;
+  if (a.info[t].node < 0) return;  // a skipped row is left as it was
   const int h = min(max(a.hinv[g * a.G + (m - t * a.G)], 0), a.Hq - 1);
   T* out = reinterpret_cast<T*>(a.out) + ((size_t)t * a.Hq + h) * D;
 #pragma unroll

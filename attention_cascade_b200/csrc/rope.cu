@@ -1,5 +1,6 @@
 // rope.cu — RoPE of the suffix (or tree) tokens, group-major query packing,
-// per-token window info, and (tree) the ancestor plan of every node.
+// per-token window info, (tree) the plan of each token's node, and (cache mode) the
+// append of the new tokens' rotated keys and values to per-branch caches.
 //
 // Positions continue from the prefix: branch token j sits at pos_offset + j
 // ("FastJEV: Understanding Redundancy for Compact JEV Inference", TL;DR and
@@ -62,38 +63,63 @@ __device__ __forceinline__ void unpack8(const F8& v, float (&f)[8]) {
 constexpr int kTokPerBlock = 8;  // one warp per token
 constexpr int kSmemOffs = 4096;  // segment offsets searched in shared memory up to this many
 
-// Tree ancestor plan of node n: walk up to the root (parents must precede
-// children, at most kMaxDepth levels) and record the packed key ranges of the
-// node's non-root ancestors, root side first; a malformed chain flags
-// JEV_DEV_BAD_TREE and marks the node's rows to be skipped.
-__device__ void plan_node(const RopePackArgs& a, int n) {
+// Tree plan of node m, computed by the warp of each of m's tokens (nodes in
+// depth-first preorder, packed tokens in node order).  The keys a token of m
+// may see beyond the root are the tokens of m's ancestors and its own, all of
+// which lie in [first token of m's top-level ancestor, the token itself]; a
+// key of node a is visible to a token t exactly when a's subtree, whose tokens
+// are the contiguous range [tok_off[a], tok_off[e(a)]), contains t and the key
+// is not after t.  Checks: the parent precedes the node and every node
+// between the two descends from the parent (preorder), token offsets are in
+// order; a node that fails is flagged and its rows are skipped.  The scans
+// read 32 nodes per step; their length is the node's distance to its parent,
+// to the end of its subtree and to its top-level ancestor, in node order.
+struct NodePlan {
+  int start;  // first key of the node's rows' windows; -1: malformed
+  int end;    // end of the packed tokens of the node's subtree
+};
+__device__ NodePlan plan_node(const RopePackArgs& a, int m, int lane) {
+  const int32_t* parent = a.parent;
   const int32_t* tok_off = a.offs;
-  if (n == 0) {
-    if (a.parent[0] != -1 || tok_off[0] != 0 || tok_off[1] != 0 || tok_off[a.n_segs] != a.T)
-      raise_flag(a.status, JEV_DEV_BAD_TREE);
-    a.node_nanc[0] = 0;
-    return;
+  const int n = a.n_segs;
+  NodePlan r{-1, -1};
+  if (m <= 0 || m >= n) return r;
+  const int p = parent[m];
+  bool ok = p >= 0 && p < m && tok_off[m] >= 0 && tok_off[m] <= tok_off[m + 1] && tok_off[m + 1] <= a.T;
+  if (ok) {
+    bool bad = false;
+    for (int j0 = p + 1; j0 < m; j0 += 32) {
+      const int j = j0 + lane;
+      bad |= j < m && parent[j] < p;
+    }
+    ok = !__any_sync(0xffffffffu, bad);
   }
-  int chain[kMaxDepth];
-  int depth = 0, cur = n, ok = 1;
-  while (cur > 0) {
-    if (depth >= kMaxDepth) { ok = 0; break; }
-    chain[depth++] = cur;
-    int p = a.parent[cur];
-    if (p < 0 || p >= cur) { ok = 0; break; }
-    if (tok_off[cur + 1] < tok_off[cur] || tok_off[cur] < 0 || tok_off[cur + 1] > a.T) { ok = 0; break; }
-    cur = p;
+  // the subtree is nodes m .. e-1: e is the first later node whose parent precedes m
+  int e = n;
+  for (int j0 = m + 1; j0 < n; j0 += 32) {
+    const int j = j0 + lane;
+    const unsigned hit = __ballot_sync(0xffffffffu, j < n && parent[j] < m);
+    if (hit) {
+      e = j0 + __ffs(hit) - 1;
+      break;
+    }
   }
-  int2* anc = a.node_anc + (size_t)n * kMaxDepth;
-  if (!ok) {
-    raise_flag(a.status, JEV_DEV_BAD_TREE);
-    a.node_nanc[n] = -1;  // rows of this node are skipped
-    return;
+  // the top-level ancestor: the last node at or before m whose parent is the root
+  int top = 0;
+  for (int j0 = m; j0 > 0; j0 -= 32) {
+    const int j = j0 - lane;
+    const unsigned hit = __ballot_sync(0xffffffffu, j > 0 && parent[j] == 0);
+    if (hit) {
+      top = j0 - (__ffs(hit) - 1);
+      break;
+    }
   }
-  // chain[0] = n itself; ancestors are chain[depth-1] (root side) .. chain[1]
-  int w = 0;
-  for (int k = depth - 1; k >= 1; --k) anc[w++] = make_int2(tok_off[chain[k]], tok_off[chain[k] + 1]);
-  a.node_nanc[n] = w;
+  ok = ok && top > 0;
+  if (ok) {
+    r.start = min(max(tok_off[top], 0), a.T);
+    r.end = min(max(tok_off[e], 0), a.T);
+  }
+  return r;
 }
 
 // One warp per packed token: find its segment and position, form cos/sin of
@@ -164,9 +190,9 @@ __global__ void __launch_bounds__(256) rope_pack_kernel(RopePackArgs a) {
     s_slot[h] = slot;
     if (blockIdx.x == 0) a.hinv[g * G + slot] = h;
   }
-  // tree: the ancestor plan of every node (grid-stride over nodes)
-  if (a.parent)
-    for (int n = blockIdx.x * blockDim.x + threadIdx.x; n < a.n_segs; n += gridDim.x * blockDim.x) plan_node(a, n);
+  if (a.parent && blockIdx.x == 0 && threadIdx.x == 0 &&
+      (a.parent[0] != -1 || a.offs[0] != 0 || (a.n_segs > 0 && a.offs[1] != 0)))
+    raise_flag(a.status, JEV_DEV_BAD_TREE);  // node 0 is the root: no parent, no packed tokens
   if (blockIdx.x == 0) {
     // offsets must start at 0, never decrease and end at T
     for (int i = threadIdx.x; i < a.n_segs; i += blockDim.x)
@@ -175,16 +201,41 @@ __global__ void __launch_bounds__(256) rope_pack_kernel(RopePackArgs a) {
   }
   __syncthreads();
   if (t >= a.T) return;
-  int seg = 0, start = 0, pos = 0;
+  int seg = 0, start = 0, pos = 0, krow = t, kvalid = 1;
   if (lane == 0) {
     seg = upper_segment(offs_in_smem ? s_offs : a.offs, a.n_segs, t);
     start = offs_in_smem ? s_offs[seg] : a.offs[seg];
     if (start > t) start = t;
     if (start < 0) start = 0;
-    pos = a.pos_seq ? a.pos_offset + t : (a.pos0 ? a.pos0[seg] : a.pos_offset) + (t - start);
-    a.info[t] = TokInfo{start, pos, seg, 0};
+  }
+  if (a.parent) {
+    // tree token: window from its top-level ancestor; as a key, its node's subtree end
+    seg = __shfl_sync(0xffffffffu, seg, 0);
+    const NodePlan np = plan_node(a, seg, lane);
+    if (lane == 0) {
+      if (np.start < 0) raise_flag(a.status, JEV_DEV_BAD_TREE);
+      pos = a.pos0[seg] + (t - start);
+      a.info[t] = TokInfo{max(np.start, 0), pos, np.start < 0 ? -1 : seg, np.end};
+      a.key_end[t] = np.start < 0 ? -1 : np.end;
+    }
+  } else if (lane == 0) {
+    if (a.cache_off) {
+      // new token j of branch seg: after the branch's cached tokens, in its cache rows
+      const int j = t - start, n_new = (offs_in_smem ? s_offs[seg + 1] : a.offs[seg + 1]) - start;
+      const int len = a.cache_len[seg], c0 = a.cache_off[seg], c1 = a.cache_off[seg + 1];
+      kvalid = len >= 0 && c0 >= 0 && c1 <= a.key_rows && (long long)c0 + len + n_new <= (long long)c1;
+      if (!kvalid) raise_flag(a.status, JEV_DEV_BAD_CACHE);
+      krow = kvalid ? c0 + len + j : 0;
+      pos = a.pos_offset + (kvalid ? len : 0) + j;
+      a.info[t] = TokInfo{max(c0, 0), pos, kvalid ? seg : -1, krow};
+    } else {
+      pos = a.pos_seq ? a.pos_offset + t : (a.pos0 ? a.pos0[seg] : a.pos_offset) + (t - start);
+      a.info[t] = TokInfo{start, pos, seg, t};
+    }
   }
   pos = __shfl_sync(0xffffffffu, pos, 0);
+  krow = __shfl_sync(0xffffffffu, krow, 0);
+  kvalid = __shfl_sync(0xffffffffu, kvalid, 0);
   for (int i = lane; i < half; i += 32) {
     // angle formed in double and reduced to [-pi, pi] in double (the error of
     // the reduction is ~1e-12 rad for positions up to 1e6), then one float sincos
@@ -207,8 +258,9 @@ __global__ void __launch_bounds__(256) rope_pack_kernel(RopePackArgs a) {
   for (int it = 0; it < kMaxIt; ++it) {
     const int hh = hsub + it * heads_per_it;
     if (hh < H) {
+      if (hh >= a.Hq && !kvalid) continue;  // a cache row outside the branch's rows is not written
       T* dst = hh < a.Hq ? reinterpret_cast<T*>(a.q_rot) + ((size_t)s_grp[hh] * M + (size_t)t * G + s_slot[hh]) * a.d
-                         : reinterpret_cast<T*>(a.k_rot) + ((size_t)t * a.Hkv + (hh - a.Hq)) * a.d;
+                         : reinterpret_cast<T*>(a.k_rot) + ((size_t)krow * a.Hkv + (hh - a.Hq)) * a.d;
       float x0[8], x1[8], y0[8], y1[8];
       unpack8(r0[it], x0);
       unpack8(r1[it], x1);
@@ -223,10 +275,11 @@ __global__ void __launch_bounds__(256) rope_pack_kernel(RopePackArgs a) {
   }
   // heads beyond kMaxIt iterations (very wide models) take a plain loop
   for (int hh = hsub + kMaxIt * heads_per_it; hh < H; hh += heads_per_it) {
+    if (hh >= a.Hq && !kvalid) continue;
     const T* src = hh < a.Hq ? reinterpret_cast<const T*>(a.q) + ((size_t)t * a.Hq + hh) * a.d
                              : reinterpret_cast<const T*>(a.k) + ((size_t)t * a.Hkv + (hh - a.Hq)) * a.d;
     T* dst = hh < a.Hq ? reinterpret_cast<T*>(a.q_rot) + ((size_t)s_grp[hh] * M + (size_t)t * G + s_slot[hh]) * a.d
-                       : reinterpret_cast<T*>(a.k_rot) + ((size_t)t * a.Hkv + (hh - a.Hq)) * a.d;
+                       : reinterpret_cast<T*>(a.k_rot) + ((size_t)krow * a.Hkv + (hh - a.Hq)) * a.d;
     float u0[8], u1[8], y0[8], y1[8];
     load8(src + i0, u0);
     load8(src + i0 + half, u1);
@@ -237,6 +290,13 @@ __global__ void __launch_bounds__(256) rope_pack_kernel(RopePackArgs a) {
     }
     store8(dst + i0, y0);
     store8(dst + i0 + half, y1);
+  }
+  // cache mode: the new token's values go to the same cache row as its key
+  if (a.v_cache && kvalid) {
+    constexpr int kVec = 16 / sizeof(T);
+    const uint4* src = reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(a.v) + (size_t)t * a.Hkv * a.d);
+    uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<T*>(a.v_cache) + (size_t)krow * a.Hkv * a.d);
+    for (int e = lane; e < a.Hkv * a.d / kVec; e += 32) dst[e] = src[e];
   }
 }
 

@@ -15,7 +15,8 @@
 //
 // CTA = 18 warps: 16 statistics warps, 1 TMA producer, 1 MMA issuer (which
 // also owns TMEM).  Every mbarrier wait is bounded; a wait that runs out
-// raises JEV_DEV_WAIT_TIMEOUT in the status word and the CTA winds down.
+// raises JEV_DEV_WAIT_TIMEOUT in the status word and the CTA winds down, the
+// producer and the MMA warp first waiting for the loads and MMAs they issued.
 #include <cuda.h>
 #include <math_constants.h>
 
@@ -34,7 +35,6 @@ constexpr int kLStages = 3;
 constexpr int kLStatWarps = 16;
 constexpr int kLThreads = (kLStatWarps + 2) * 32;
 constexpr int kLProducer = kLStatWarps, kLMma = kLStatWarps + 1;
-constexpr long long kLWaitCycles = 1LL << 31;
 constexpr int kXBytes = kLM * kLK * 2;               // 16 KB: one half's chunk
 constexpr int kWBytes = kLN * kLK * 2;               // 32 KB: the tile's chunk
 constexpr int kStageBytes = 2 * kXBytes + kWBytes;   // 64 KB
@@ -46,16 +46,30 @@ struct LShared {
   int abort;
 };
 
-__device__ __forceinline__ bool lwait(uint32_t bar, uint32_t parity, volatile int* abort, int32_t* status) {
+__device__ __forceinline__ bool lwait(uint32_t bar, uint32_t parity, volatile int* abort, int32_t* status,
+                                      long long limit) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   for (;;) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
-    if (clock64() - t0 > kLWaitCycles) {
+    if (clock64() - t0 > limit) {
       *abort = 1;
       raise_flag(status, JEV_DEV_WAIT_TIMEOUT);
       return false;
+    }
+  }
+}
+
+// Exit-path wait: bounded but blind to the abort flag (in-flight loads and
+// MMAs complete within microseconds; running out of the bound only raises the flag).
+constexpr long long kLDrainCycles = 1LL << 28;
+__device__ __forceinline__ void ldrain(uint32_t bar, uint32_t parity, int32_t* status) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (clock64() - t0 > kLDrainCycles) {
+      raise_flag(status, JEV_DEV_WAIT_TIMEOUT);
+      return;
     }
   }
 }
@@ -118,7 +132,7 @@ __global__ void __launch_bounds__(kLThreads, 1)
           for (int kc = 0; ok && kc < nk; ++kc, ++it) {
             const int st = (int)(it % kLStages);
             const long long use = it / kLStages;
-            if (it >= kLStages && !lwait(b_empty + 8 * st, (uint32_t)((use - 1) & 1), abort, a.status)) {
+            if (it >= kLStages && !lwait(b_empty + 8 * st, (uint32_t)((use - 1) & 1), abort, a.status, a.wait_cycles)) {
               ok = false;
               break;
             }
@@ -133,6 +147,12 @@ __global__ void __launch_bounds__(kLThreads, 1)
             for (; o < n_t; o += 16) tma_load_2d(base + 2 * kXBytes + o * 128, &tm_w16, kc * kLK, v0 + o, b_full + 8 * st);
           }
         }
+      // drain: the last phase of every stage armed (it loads so far) has
+      // completed, so no load lands after the CTA exits
+      for (int st = 0; st < kLStages; ++st) {
+        const long long uses = it > st ? (it - st + kLStages - 1) / kLStages : 0;
+        if (uses > 0) ldrain(b_full + 8 * st, (uint32_t)((uses - 1) & 1), a.status);
+      }
     }
   } else if (warp == kLMma) {
     // ---------------------------------------------------------------- MMA issuer
@@ -144,14 +164,14 @@ __global__ void __launch_bounds__(kLThreads, 1)
         for (int v0 = v_lo; ok && v0 < v_hi; v0 += kLN, ++tile) {
           const uint32_t idesc = idesc_bf16(kLM, (min(kLN, v_hi - v0) + 15) & ~15, false);
           // the statistics threads have read the previous tile out of TMEM
-          if (tile > 0 && !lwait(b_sempty, (uint32_t)((tile - 1) & 1), abort, a.status)) {
+          if (tile > 0 && !lwait(b_sempty, (uint32_t)((tile - 1) & 1), abort, a.status, a.wait_cycles)) {
             ok = false;
             break;
           }
           fence_after_sync();
           for (int kc = 0; kc < nk; ++kc, ++it) {
             const int st = (int)(it % kLStages);
-            if (!lwait(b_full + 8 * st, (uint32_t)((it / kLStages) & 1), abort, a.status)) {
+            if (!lwait(b_full + 8 * st, (uint32_t)((it / kLStages) & 1), abort, a.status, a.wait_cycles)) {
               ok = false;
               break;
             }
@@ -167,9 +187,10 @@ __global__ void __launch_bounds__(kLThreads, 1)
           if (ok) mma_commit(b_sfull);
         }
       }
-      // every MMA of this CTA has completed before TMEM is released
+      // every MMA of this CTA has completed before TMEM is released, on the
+      // timeout path too (the wait ignores the abort flag)
       mma_commit(b_drain);
-      lwait(b_drain, 0, abort, a.status);
+      ldrain(b_drain, 0, a.status);
     }
   } else {
     // ---------------------------------------------------------------- statistics
@@ -184,7 +205,7 @@ __global__ void __launch_bounds__(kLThreads, 1)
       for (int t0 = v_lo; t0 < v_hi; t0 += kLN, ++tile) {
         // warp-uniform (the TMEM loads below are warp-wide instructions); a
         // failed wait runs the remaining tiles on stale TMEM so the loop shape stays uniform
-        ok = __all_sync(0xffffffffu, ok && lwait(b_sfull, (uint32_t)(tile & 1), abort, a.status));
+        ok = __all_sync(0xffffffffu, ok && lwait(b_sfull, (uint32_t)(tile & 1), abort, a.status, a.wait_cycles));
         fence_after_sync();
         const int v0 = t0 + hf * (kLN / 2);  // vocabulary row of this thread's first column
 #pragma unroll

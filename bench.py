@@ -621,6 +621,55 @@ def diag_tree_schedule(dev, jev, torch, stream) -> dict:
     return res
 
 
+def diag_decode(dev, jev, torch, stream, names=("qwen25vl_7b", "wide_7b")) -> dict:
+    """One generation step after the decision (jev_suffix_cache_attn): every
+    branch of the workload appends one token over the shared prefix and its
+    cached suffix (U[lo, hi] tokens, as drawn for the workload; cache rows
+    packed with 8 spare rows per branch).  Graph-replayed; per-kernel times
+    from a second replay with event nodes.  Attention FLOPs count the keys
+    each new token sees: 4 * Hq * d * sum_b (Lp + cached_b + 1)."""
+    pk, src = peaks()
+    res = {}
+    for name in names:
+        cfg = synth.CONFIGS[name]
+        Ls = synth.suffix_lengths(cfg)
+        B = cfg.B
+        rng = np.random.default_rng(9)
+        mk = lambda *sh: to_dev(synth.f32_to_bf16_bits(rng.standard_normal(sh).astype(np.float32)), dev, torch)
+        co = np.concatenate([[0], np.cumsum(Ls + 8)]).astype(np.int32)
+        kc, vc = mk(int(co[-1]), cfg.Hkv, cfg.d), mk(int(co[-1]), cfg.Hkv, cfg.d)
+        kp, vp = mk(cfg.Lp, cfg.Hkv, cfg.d), mk(cfg.Lp, cfg.Hkv, cfg.d)
+        q, kn, vn = mk(B, cfg.Hq, cfg.d), mk(B, cfg.Hkv, cfg.d), mk(B, cfg.Hkv, cfg.d)
+        cod, cld = torch.from_numpy(co).to(dev), torch.from_numpy(Ls).to(dev)
+        cu = torch.arange(B + 1, dtype=torch.int32, device=dev)
+        desc = jev.make_attn_desc(B, cfg.Lp, cfg.Hq, cfg.Hkv, cfg.d, B, jev.JEV_BF16, cfg.theta)
+        ws = jev.new_workspace(jev.jev_suffix_cache_attn_workspace(desc), dev)
+        out = torch.empty_like(q)
+        lse = torch.empty((B, cfg.Hq), dtype=torch.float32, device=dev)
+
+        def step():
+            jev.jev_suffix_cache_attn(q, kn, vn, kp, vp, kc, vc, cod, cld, cu, out=out, lse=lse, workspace=ws,
+                                      rope_theta=cfg.theta, stream=torch.cuda.current_stream())
+        us = graph_us(torch, step, stream, 200, 10)
+        jev.jev_profile_read()
+        jev.jev_profile_enable(True)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            step()
+        jev.jev_profile_enable(False)
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                g.replay()
+        torch.cuda.synchronize()
+        prof = {k: 1e3 * v[1] / max(v[0], 1) for k, v in jev.jev_profile_read().items()}
+        del g
+        flops = 4 * cfg.Hq * cfg.d * int((cfg.Lp + Ls.astype(np.int64) + 1).sum())
+        res[name] = {"branches": B, "cached_tokens": int(Ls.sum()), "us_per_step": us,
+                     "new_tokens_per_s": B / (us / 1e6), "kernels_us": prof, "flops_per_step": flops,
+                     "TFLOPs": flops / us / 1e6, "device_flags": jev.jev_check_device_status(ws)}
+    return res
+
+
 def diag_attn(dev, jev, torch, stream, wl_name: str) -> dict:
     """The workload's attention call alone (no LM head on the device, one set
     of inputs): a small case for ncu captures of the attention kernels.
@@ -692,6 +741,8 @@ def diagnostics(dev, jev, torch) -> dict:
     del W, hidden
     torch.cuda.empty_cache()
     out["tree_schedule"] = diag_tree_schedule(dev, jev, torch, stream)
+    torch.cuda.empty_cache()
+    out["decode_step"] = diag_decode(dev, jev, torch, stream)
     torch.cuda.empty_cache()
     # ---- RoPE pack (and the attention call around it) at the wide shape with 1024 branches
     cw = dataclasses.replace(synth.CONFIGS["wide_7b"], B=1024)
@@ -1073,7 +1124,7 @@ def main():
     ap.add_argument("--per-config-steps", type=int, default=2000)
     ap.add_argument("--no-diagnostics", dest="diagnostics", action="store_false",
                     help="skip the streaming diagnostics at larger sizes (one GPU)")
-    ap.add_argument("--diag", choices=["vocab_lse", "tree_schedule", "attn"], default=None,
+    ap.add_argument("--diag", choices=["vocab_lse", "tree_schedule", "attn", "decode"], default=None,
                     help="run only this diagnostic on cuda:0 and print its JSON (a small case for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -1086,7 +1137,7 @@ def main():
         if args.diag == "attn":
             res = diag_attn("cuda:0", jev, torch, stream, args.workload)
         else:
-            fn = {"vocab_lse": diag_vocab_lse, "tree_schedule": diag_tree_schedule}[args.diag]
+            fn = {"vocab_lse": diag_vocab_lse, "tree_schedule": diag_tree_schedule, "decode": diag_decode}[args.diag]
             res = fn("cuda:0", jev, torch, stream)
         print(json.dumps({"diagnostic": args.diag, **res}))
     elif args.impl == "reference":

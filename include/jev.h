@@ -59,9 +59,10 @@ typedef enum { JEV_F32 = 0, JEV_BF16 = 1 } jev_dtype;
 enum {
   JEV_DEV_BAD_SEQLENS = 1,   /* cu_seqlens / tok_off not monotone or != T   */
   JEV_DEV_BAD_HEAD_MAP = 2,  /* head map entry out of range or groups uneven */
-  JEV_DEV_BAD_TREE = 4,      /* parent not earlier than child, or too deep  */
+  JEV_DEV_BAD_TREE = 4,      /* nodes not in depth-first preorder, or bad offsets */
   JEV_DEV_WAIT_TIMEOUT = 8,  /* a bounded pipeline wait gave up             */
-  JEV_DEV_BAD_WINDOW = 16    /* a row's key window exceeded the kernel limit */
+  JEV_DEV_BAD_WINDOW = 16,   /* a row's key window exceeded the kernel limit */
+  JEV_DEV_BAD_CACHE = 32     /* a branch's cache rows cannot hold its tokens */
 };
 
 /* ------------------------------------------------------------------------ */
@@ -151,6 +152,64 @@ jev_status jev_prefix_suffix_attn(const jev_attn_desc* desc, const void* q, cons
                                   const void* v_pre, const void* k_suf, const void* v_suf,
                                   const int32_t* cu_seqlens, const int32_t* head_map, void* out,
                                   float* lse, void* workspace, size_t ws_bytes, jev_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Generation over per-branch suffix caches                                  */
+/* ------------------------------------------------------------------------ */
+
+/* Bytes of workspace jev_suffix_cache_attn needs for `desc`. */
+size_t jev_suffix_cache_attn_workspace(const jev_attn_desc* desc);
+
+/*
+ * jev_suffix_cache_attn — one attention layer for the new tokens of B
+ * branches that continue over the shared prefix and their own cached suffix
+ * tokens: a generation step after the decision, each branch decoding its own
+ * continuation ("How to Deploy Visual Jev ...", Step 3 batches the branches
+ * over the one cached prefix; "FastJEV ...", Abstract and §5: what is shared
+ * and how the work is scheduled are designed together).  Branch b has
+ * cache_len[b] suffix tokens already cached: rotated keys and values in rows
+ * cache_off[b] .. cache_off[b] + cache_len[b] - 1 of k_cache / v_cache.  Its
+ * new tokens are rows cu_new[b] .. cu_new[b+1]-1 of q / k_new / v_new; new
+ * token j sits at position pos_offset + cache_len[b] + j and
+ *
+ *     keys     = [ k_pre[0..Lp) ; cached keys of b ; RoPE(new keys of b, 0..j) ]
+ *     out[t,h] = softmax(scale * RoPE(q[t,h]) . keys^T) . values,  lse as in
+ *                jev_prefix_suffix_attn
+ *
+ * which is the row jev_prefix_suffix_attn gives token cache_len[b] + j of the
+ * branch's whole suffix.  The call also appends: new token j's rotated key and
+ * its value are written to cache row cache_off[b] + cache_len[b] + j.  It does
+ * not change cache_len; the caller advances it by the new token counts.  A
+ * first call with cache_len = 0 is the prefill and fills the caches.
+ *
+ *   desc       B, Lp, Hq, Hkv, d, dtype, rope_theta, softmax_scale, pos_offset
+ *              (<0 -> Lp), num_splits as for jev_prefix_suffix_attn; T_total
+ *              = new tokens (cu_new[B]); pos_mode must be 0
+ *   q          [T_total, Hq, d]  new tokens' queries before RoPE
+ *   k_new      [T_total, Hkv, d] new tokens' keys before RoPE
+ *   v_new      [T_total, Hkv, d]
+ *   k_pre/v_pre [Lp, Hkv, d]     the shared prefix cache (k rotated)
+ *   k_cache/v_cache [cache_rows, Hkv, d] in/out, same dtype; branch b owns
+ *              rows cache_off[b] .. cache_off[b+1]-1
+ *   cache_off  device [B+1] int32, non-decreasing, cache_off[B] <= cache_rows
+ *   cache_len  device [B] int32, cached tokens per branch
+ *   cu_new     device [B+1] int32, new-token offsets, cu_new[0] = 0
+ *   head_map, out [T_total, Hq, d], lse [T_total, Hq] fp32 or NULL, workspace
+ *              (>= jev_suffix_cache_attn_workspace(desc) bytes) as for
+ *              jev_prefix_suffix_attn
+ *
+ * A branch whose rows cannot hold its new tokens (cache_len[b] + new tokens >
+ * cache_off[b+1] - cache_off[b]) sets JEV_DEV_BAD_CACHE; its rows and its cache
+ * are left untouched and the other branches are computed.  Rows of the window
+ * a work tile reads lie between its branches' first cache rows and last new
+ * slots, so caches packed tightly (little unused capacity between branches)
+ * cost the fewest masked key tiles.
+ */
+jev_status jev_suffix_cache_attn(const jev_attn_desc* desc, const void* q, const void* k_new, const void* v_new,
+                                 const void* k_pre, const void* v_pre, void* k_cache, void* v_cache,
+                                 int32_t cache_rows, const int32_t* cache_off, const int32_t* cache_len,
+                                 const int32_t* cu_new, const int32_t* head_map, void* out, float* lse,
+                                 void* workspace, size_t ws_bytes, jev_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
 /* Fixed-scratch variant (no allocation)                                     */
@@ -343,8 +402,14 @@ size_t jev_tree_attn_workspace(const jev_attn_desc* desc, int32_t n_nodes);
  *   q [N, Hq, d], k/v [N, Hkv, d] before RoPE, in packed node order;
  *   k_root/v_root [Lp, Hkv, d] the root cache (k already rotated);
  *   out [N, Hq, d]; lse [N, Hq] fp32 or NULL.
- *   Depth (non-root ancestors + self) is limited to 8; deeper trees set
- *   JEV_DEV_BAD_TREE and leave their rows unwritten.
+ *   Nodes must be numbered in depth-first preorder with their tokens packed
+ *   in node order (as jev_tree_build returns them); any depth is allowed.  A
+ *   node whose parent is not earlier than itself, or not on the path of the
+ *   node before it, or whose token offsets are out of order, sets
+ *   JEV_DEV_BAD_TREE and its rows are left unwritten.  The RoPE pack plans
+ *   each token's node with warp-wide scans whose length grows with the node's
+ *   distance to its parent, to the end of its subtree and to its top-level
+ *   ancestor, in node order.
  */
 jev_status jev_tree_attn(const jev_attn_desc* desc, int32_t n_nodes, const int32_t* parent,
                          const int32_t* tok_off, const int32_t* pos0, const void* q, const void* k_root,
@@ -388,6 +453,20 @@ int32_t jev_profile_read(int32_t cap, char* names, int32_t* launches, double* ms
 
 /* Kernels launched by this process since load (all entry points). */
 int64_t jev_launch_count(void);
+
+/*
+ * jev_debug_set_wait_limit — bound, in SM clock cycles, of every mbarrier
+ * wait in the tensor-core kernels (attention and full-vocabulary LSE) launched
+ * after the call; 0 restores the default of 2^31 cycles (about a second).  A
+ * wait that runs out sets JEV_DEV_WAIT_TIMEOUT in the status word and the CTA
+ * winds down: the remaining waits give up, the TMA producer waits for every
+ * load it issued and the MMA warp for every MMA it issued, and the kernel
+ * returns with its outputs undefined.  Failure handling is tested with a
+ * short limit on an ordinary problem, so that waits run out without any GPU
+ * fault; the setting is process-wide.  JEV_ERR_INVALID_ARG for cycles < 0.
+ * No page has a counterpart: this is the library's failure detection.
+ */
+jev_status jev_debug_set_wait_limit(int64_t cycles);
 
 #ifdef __cplusplus
 }

@@ -106,30 +106,46 @@ def test_status_word_flags_bad_inputs_without_faulting(jev):
     assert torch.isfinite(torch.ones(4, device="cuda").sum())
 
 
-def test_tree_status_flags_deep_chain(jev):
-    # a chain of 10 single-token nodes (each candidate ends one token deeper) exceeds the depth limit of 8
-    cands = [list(range(1, k + 1)) for k in range(1, 11)]
+def _tree_case(jev, cands, root=64, Hq=4, Hkv=2, d=64, seed=0):
     so = np.concatenate([[0], np.cumsum([len(x) for x in cands])]).astype(np.int32)
     toks = np.array([t for x in cands for t in x], np.int32)
-    t = jev.jev_tree_build(so, toks, 64)
-    assert t["n_nodes"] == 11
+    t = jev.jev_tree_build(so, toks, root)
     N = int(t["tok_off"][-1])
-    rng = np.random.default_rng(0)
+    rng = np.random.default_rng(seed)
+    mk = lambda *s: synth.f32_to_bf16_bits(rng.standard_normal(s).astype(np.float32))
+    return so, toks, t, (mk(N, Hq, d), mk(N, Hkv, d), mk(N, Hkv, d), mk(root, Hkv, d), mk(root, Hkv, d))
+
+
+def test_tree_status_flags_malformed_trees_without_faulting(jev):
+    """A node whose parent is not earlier than itself, and a tree numbered
+    breadth-first instead of in depth-first preorder, set JEV_DEV_BAD_TREE;
+    rows of the well-formed nodes of the first tree are still exact."""
+    cands = [[1, 2], [1, 3], [4, 5, 6], [4, 7]]
+    so, toks, t, (q, k, v, kr, vr) = _tree_case(jev, cands)
+    parent = t["parent"].copy()
+    last = t["n_nodes"] - 1
+    parent[last] = last  # a node that is its own parent
+    desc = jev.make_attn_desc(t["n_nodes"] - 1, 64, 4, 2, 64, int(t["tok_off"][-1]), jev.JEV_BF16)
+    ws = jev.new_workspace(jev.jev_tree_attn_workspace(desc, t["n_nodes"]), "cuda")
+    out, lse = jev.jev_tree_attn(dev(parent), dev(t["tok_off"]), dev(t["pos0"]), dev(q), dev(kr), dev(vr), dev(k),
+                                 dev(v), workspace=ws)
+    assert jev.jev_check_device_status(ws) & jev.JEV_DEV_BAD_TREE
+    ref_o, _ = oracle.tree_attn(oracle.trie_build(so, toks, 64), q, k, v, kr, vr)
+    good = np.arange(int(t["tok_off"][last]))  # every token before the corrupted node
+    assert np.abs(host_f64(out)[good] - ref_o[good]).max() <= TOL[synth.BF16]["max_abs"]
+    # breadth-first numbering: root children A = 1, B = 2, then A's child C = 3
+    bfs_parent = np.array([-1, 0, 0, 1], np.int32)
+    tok_off = np.array([0, 0, 2, 4, 6], np.int32)
+    pos0 = np.array([0, 64, 64, 66], np.int32)
+    rng = np.random.default_rng(1)
     mk = lambda *s: dev(synth.f32_to_bf16_bits(rng.standard_normal(s).astype(np.float32)))
-    q, k, v, kr, vr = mk(N, 4, 64), mk(N, 2, 64), mk(N, 2, 64), mk(64, 2, 64), mk(64, 2, 64)
-    desc = jev.make_attn_desc(10, 64, 4, 2, 64, N, jev.JEV_BF16)
-    ws = jev.new_workspace(jev.jev_tree_attn_workspace(desc, 11), "cuda")
-    out, lse = jev.jev_tree_attn(dev(t["parent"]), dev(t["tok_off"]), dev(t["pos0"]), q, kr, vr, k, v, workspace=ws)
-    flags = jev.jev_check_device_status(ws)
-    assert flags & jev.JEV_DEV_BAD_TREE
-    # rows of nodes within the depth limit are still correct
-    ref_o, _ = oracle.tree_attn(oracle.trie_build(so, toks, 64), synth.f32_to_bf16_bits(host_f64(q).astype(np.float32)),
-                                synth.f32_to_bf16_bits(host_f64(k).astype(np.float32)),
-                                synth.f32_to_bf16_bits(host_f64(v).astype(np.float32)),
-                                synth.f32_to_bf16_bits(host_f64(kr).astype(np.float32)),
-                                synth.f32_to_bf16_bits(host_f64(vr).astype(np.float32)))
-    ok_rows = 8  # nodes 1..8 have depth <= 8
-    assert np.abs(host_f64(out)[:ok_rows] - ref_o[:ok_rows]).max() <= TOL[synth.BF16]["max_abs"]
+    desc = jev.make_attn_desc(3, 64, 4, 2, 64, 6, jev.JEV_BF16)
+    ws = jev.new_workspace(jev.jev_tree_attn_workspace(desc, 4), "cuda")
+    jev.jev_tree_attn(dev(bfs_parent), dev(tok_off), dev(pos0), mk(6, 4, 64), mk(64, 2, 64), mk(64, 2, 64),
+                      mk(6, 2, 64), mk(6, 2, 64), workspace=ws)
+    assert jev.jev_check_device_status(ws) & jev.JEV_DEV_BAD_TREE
+    torch.cuda.synchronize()
+    assert torch.isfinite(torch.ones(4, device="cuda").sum())
 
 
 def test_fma_pipe_exp2_against_cuda_exp2(jev):
@@ -142,3 +158,38 @@ def test_fma_pipe_exp2_against_cuda_exp2(jev):
     assert rel < 2e-4, rel
     z = jev.jev_selftest_exp2(torch.tensor([-float("inf"), -1000.0, -200.0], device="cuda"))
     assert (z >= 0).all() and (z < 1e-37).all()
+
+
+def test_short_wait_limit_flags_a_timeout_and_leaves_the_context_usable(jev):
+    """Failure detection without a GPU fault: with the tensor-core kernels'
+    wait bound cut to 256 cycles on an ordinary problem, waits run out.  Each
+    call must set JEV_DEV_WAIT_TIMEOUT and return (its CTAs drain the loads
+    and MMAs they issued before exiting), and the next call with the default
+    bound must reproduce the earlier result exactly."""
+    c = _case([17, 3, 40, 9, 25], seed=8, Lp=1024, Hq=28, Hkv=4)
+    args = [dev(x) for x in (c.q, c.k_pre, c.v_pre, c.k_suf, c.v_suf)] + [dev(c.cu_seqlens)]
+    desc = jev.make_attn_desc(5, 1024, 28, 4, 128, int(c.cu_seqlens[-1]), jev.JEV_BF16)
+    ws = jev.new_workspace(jev.jev_prefix_suffix_attn_workspace(desc), "cuda")
+    o, l = jev.jev_prefix_suffix_attn(*args, workspace=ws)
+    assert jev.jev_check_device_status(ws) == 0
+    ref_o, ref_l = o.clone(), l.clone()
+    rng = np.random.default_rng(4)
+    h = dev(synth.f32_to_bf16_bits(rng.standard_normal((300, 512)).astype(np.float32)))
+    W = dev(synth.f32_to_bf16_bits((0.05 * rng.standard_normal((20000, 512))).astype(np.float32)))
+    lws = jev.new_workspace(jev.jev_vocab_lse_workspace(300, 20000), "cuda")
+    ref_lse = jev.jev_vocab_lse(h, W, workspace=lws).clone()
+    assert jev.jev_check_device_status(lws) == 0
+    jev.jev_debug_set_wait_limit(256)
+    try:
+        for _ in range(2):
+            jev.jev_prefix_suffix_attn(*args, workspace=ws)
+            assert jev.jev_check_device_status(ws) & jev.JEV_DEV_WAIT_TIMEOUT
+            jev.jev_vocab_lse(h, W, workspace=lws)
+            assert jev.jev_check_device_status(lws) & jev.JEV_DEV_WAIT_TIMEOUT
+    finally:
+        jev.jev_debug_set_wait_limit(0)
+    o, l = jev.jev_prefix_suffix_attn(*args, workspace=ws)
+    assert jev.jev_check_device_status(ws) == 0
+    assert torch.equal(o, ref_o) and torch.equal(l, ref_l)
+    assert torch.equal(jev.jev_vocab_lse(h, W, workspace=lws), ref_lse)
+    assert jev.jev_check_device_status(lws) == 0

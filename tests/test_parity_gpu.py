@@ -187,6 +187,36 @@ def test_tree_small_every_element(jev, seed, d, dtype):
     check_readout(lp, ch, ref, cfg.dtype, "tree readout")
 
 
+@pytest.mark.parametrize("shape", ["chain", "zigzag"])
+def test_deep_token_tries_every_element(jev, shape):
+    """Tries 12 levels deep and more: a chain of one-token nodes each ending a
+    candidate, and a zigzag whose path always continues through the second
+    child, so a token's ancestors' keys are not one contiguous range."""
+    if shape == "chain":
+        cands = [list(range(1, k + 1)) for k in range(1, 15)]
+    else:
+        cands = [[100 + i for i in range(k)] + [200 + k] for k in range(13)] + [[100 + i for i in range(13)]]
+    so = np.concatenate([[0], np.cumsum([len(x) for x in cands])]).astype(np.int32)
+    toks = np.array([t for x in cands for t in x], np.int32)
+    Lp, Hq, Hkv, d = 130, 8, 2, 64
+    t = jev.jev_tree_build(so, toks, Lp)
+    depth = np.zeros(t["n_nodes"], np.int32)
+    for n in range(1, t["n_nodes"]):
+        depth[n] = depth[t["parent"][n]] + 1
+    assert depth.max() >= 12
+    N = int(t["tok_off"][-1])
+    rng = np.random.default_rng(4)
+    mk = lambda *s: synth.f32_to_bf16_bits(rng.standard_normal(s).astype(np.float32))
+    q, k, v, kr, vr = mk(N, Hq, d), mk(N, Hkv, d), mk(N, Hkv, d), mk(Lp, Hkv, d), mk(Lp, Hkv, d)
+    desc = jev.make_attn_desc(t["n_nodes"] - 1, Lp, Hq, Hkv, d, N, jev.JEV_BF16)
+    ws = jev.new_workspace(jev.jev_tree_attn_workspace(desc, t["n_nodes"]), "cuda")
+    out, lse = jev.jev_tree_attn(dev(t["parent"]), dev(t["tok_off"]), dev(t["pos0"]), dev(q), dev(kr), dev(vr),
+                                 dev(k), dev(v), workspace=ws)
+    assert jev.jev_check_device_status(ws) == 0
+    ref_o, ref_l = oracle.tree_attn(oracle.trie_build(so, toks, Lp), q, k, v, kr, vr)
+    check_attn(host_f64(out), host_f64(lse), ref_o, ref_l, synth.BF16, f"deep tree ({shape})")
+
+
 def test_tree_more_nodes_than_the_shared_table(jev):
     # more nodes than the RoPE pack's shared-memory offset table (4096): node offsets searched in global memory
     cfg = synth.TreeConfig("tn", synth.BF16, 96, 560, 3, 5, 8, 1, 2, 4, 2, 64, 64, 5000, seed=11)
