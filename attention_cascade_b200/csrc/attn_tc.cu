@@ -428,22 +428,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------------------------------------------------------- MMA issuer
     constexpr uint32_t id_qk = idesc_bf16(kBM, kBN, false);
     constexpr uint32_t id_pv = idesc_bf16(kBM, D, true);
+    // Shared-memory descriptors are formed once; an operand's descriptor is a
+    // base plus its byte offset >> 4 in the address field (every operand lies
+    // below 256 KB of shared memory, so the 14-bit field never carries), so
+    // the one issuing thread spends a couple of instructions per MMA.
+    const uint64_t dq0 = smem_desc_sw128(sbase, 16, 1024);
+    const uint64_t dk0 = smem_desc_sw128(sbase + C::kOffK, 16, 1024);
+    const uint64_t dv0 = smem_desc_sw128(sbase + C::kOffV, C::kBlk, 1024);
     auto issue_s = [&](int i, int st) {
-      const uint32_t qa = sbase + i * C::kQBytes, ka = sbase + C::kOffK + st * C::kKVBytes;
+      const uint64_t qa = dq0 + (uint32_t)((i * C::kQBytes) >> 4), ka = dk0 + (uint32_t)((st * C::kKVBytes) >> 4);
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t off = (kk >> 2) * C::kBlk + (kk & 3) * 32;
-        mma_ss(tmem + i * kBN, smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(ka + off, 16, 1024), id_qk,
-               kk > 0);
+        constexpr int kBlk4 = C::kBlk >> 4;
+        const uint32_t off = (uint32_t)((kk >> 2) * kBlk4 + (kk & 3) * 2);
+        mma_ss(tmem + i * kBN, qa + off, ka + off, id_qk, kk > 0);
       }
       mma_commit(B.s_full + 8 * i);
     };
     auto issue_pv = [&](int i, int st, bool acc) {
-      const uint32_t va = sbase + C::kOffV + st * C::kKVBytes;
+      const uint64_t va = dv0 + (uint32_t)((st * C::kKVBytes) >> 4);
 #pragma unroll
       for (int kk = 0; kk < kBN / 16; ++kk)
-        mma_ts(tmem + C::kOCol + i * D, tmem + i * kBN + kk * 8, smem_desc_sw128(va + kk * 16 * 128, C::kBlk, 1024),
-               id_pv, (acc || kk > 0) ? 1u : 0u);
+        mma_ts(tmem + C::kOCol + i * D, tmem + i * kBN + kk * 8, va + (uint32_t)(kk * 16 * 128 / 16), id_pv,
+               (acc || kk > 0) ? 1u : 0u);
     };
     long long J = 0;
     int k = 0;
@@ -554,71 +561,101 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_after_sync();
         // the row's 128 raw scores; P is later packed in place into xs[0..63]
         uint32_t xs[kBN];
-        tmem_ld128(s_addr, xs);
         constexpr uint32_t kNegInf = 0xff800000u;
-        if (j < sg.n_pre) {
-          const int lim = a.Lp - pre_unit(sg.ua, sg.rot, sg.n_pre, j) * kBN;  // keys past the prefix are padding
-          if (lim < kBN) {
-#pragma unroll
-            for (int c = 0; c < kBN; ++c)
-              if (c >= lim) xs[c] = kNegInf;
-          }
-        } else {
-          // suffix window
-          const int kb = sg.lo + (j - sg.n_pre) * kBN;
-          if (!TREE) {
-            // flat row: the keys start .. last of its own branch
-            const int c_lo = start - kb, c_hi = last - kb;
-            // the mask is skipped when every row of the warp sees every key of this tile
-            const bool whole = __all_sync(0xffffffffu, c_lo <= 0 && c_hi >= kBN - 1);
-            if (!whole) {
+        auto load_masked = [&]() {
+          tmem_ld128(s_addr, xs);
+          if (j < sg.n_pre) {
+            const int lim = a.Lp - pre_unit(sg.ua, sg.rot, sg.n_pre, j) * kBN;  // keys past the prefix are padding
+            if (lim < kBN) {
 #pragma unroll
               for (int c = 0; c < kBN; ++c)
-                if (!(c >= c_lo && c <= c_hi)) xs[c] = kNegInf;
+                if (c >= lim) xs[c] = kNegInf;
             }
           } else {
-            // tree row t: key k is on its root path when k <= t and t lies in the
-            // packed tokens of k's node's subtree (read here, where needed)
+            // suffix window
+            const int kb = sg.lo + (j - sg.n_pre) * kBN;
+            if (!TREE) {
+              // flat row: the keys start .. last of its own branch
+              const int c_lo = start - kb, c_hi = last - kb;
+              // the mask is skipped when every row of the warp sees every key of this tile
+              const bool whole = __all_sync(0xffffffffu, c_lo <= 0 && c_hi >= kBN - 1);
+              if (!whole) {
 #pragma unroll
-            for (int c = 0; c < kBN; ++c) {
-              const int kk = kb + c;
-              const int e = kk < a.key_rows ? __ldg(a.key_end + kk) : -1;
-              if (!(kk <= t && t < e)) xs[c] = kNegInf;
+                for (int c = 0; c < kBN; ++c)
+                  if (!(c >= c_lo && c <= c_hi)) xs[c] = kNegInf;
+              }
+            } else {
+              // tree row t: key k is on its root path when k <= t and t lies in the
+              // packed tokens of k's node's subtree (read here, where needed)
+#pragma unroll
+              for (int c = 0; c < kBN; ++c) {
+                const int kk = kb + c;
+                const int e = kk < a.key_rows ? __ldg(a.key_end + kk) : -1;
+                if (!(kk <= t && t < e)) xs[c] = kNegInf;
+              }
             }
           }
+        };
+        // p = 2^(s * scale * log2e - base) for the row's 128 scores, packed in
+        // place as bf16 pairs into xs[0..63]; returns the row sum.  The
+        // scale-and-subtract and the sum run as packed f32x2 operations, every
+        // kPolyEvery-th pair of exponentials on the FMA pipe, the rest on
+        // MUFU.  With `mxp`, the maximum of the raw scores is taken alongside.
+        auto exp_pack = [&](float base, float* mxp) -> float {
+          const uint64_t sc2 = f2_pack(sl2, sl2), nb2 = f2_pack(-base, -base);
+          uint64_t ps2[4];
+          float pm[4];
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            ps2[q4] = 0;
+            pm[q4] = -CUDART_INF_F;
+          }
+#pragma unroll
+          for (int kk = 0; kk < kBN / 2; ++kk) {
+            if (mxp) pm[kk & 3] = fmax3(pm[kk & 3], __uint_as_float(xs[2 * kk]), __uint_as_float(xs[2 * kk + 1]));
+            const uint64_t x2 = f2_fma(((uint64_t)xs[2 * kk + 1] << 32) | xs[2 * kk], sc2, nb2);
+            const bool fma_pipe = kPolyEvery > 0 && (kk % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1;
+            const uint64_t p2 = fma_pipe ? exp2_fma2(x2) : f2_pack(ex2(f2_lo(x2)), ex2(f2_hi(x2)));
+            ps2[kk & 3] = f2_add(ps2[kk & 3], p2);
+            xs[kk] = pack_bf16(f2_lo(p2), f2_hi(p2));
+          }
+          if (mxp) *mxp = fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3]));
+          const uint64_t s03 = f2_add(f2_add(ps2[0], ps2[1]), f2_add(ps2[2], ps2[3]));
+          return f2_lo(s03) + f2_hi(s03);
+        };
+        load_masked();
+        float m_new, rs;
+        if (__all_sync(0xffffffffu, m_run != -CUDART_INF_F)) {
+          // every row of the warp has a running maximum: the exponentials start
+          // from it at once and the tile's maximum is found alongside; only a
+          // row whose maximum rises by more than kLazy (rare) makes the warp
+          // reload S and start again from the new maxima
+          float mxs;
+          rs = exp_pack(m_run, &mxs);
+          const float mx = mxs * sl2;
+          const bool raise = mx > m_run + kLazy;
+          m_new = raise ? mx : m_run;
+          if (__any_sync(0xffffffffu, raise)) {
+            load_masked();
+            rs = exp_pack(m_new, nullptr);
+          }
+        } else {
+          // the row's maximum first (the first tile, or rows still without one)
+          float pm[8];
+#pragma unroll
+          for (int q8 = 0; q8 < 8; ++q8) pm[q8] = __uint_as_float(xs[q8]);
+#pragma unroll
+          for (int c = 8; c < kBN; c += 2)
+            pm[(c >> 1) & 7] = fmax3(pm[(c >> 1) & 7], __uint_as_float(xs[c]), __uint_as_float(xs[c + 1]));
+          const float mx = fmax3(fmax3(pm[0], pm[1], pm[2]), fmax3(pm[3], pm[4], pm[5]), fmaxf(pm[6], pm[7])) * sl2;
+          m_new = m_run;
+          if (mx > m_run + kLazy || (m_run == -CUDART_INF_F && mx > -CUDART_INF_F)) m_new = mx;
+          rs = exp_pack(m_new == -CUDART_INF_F ? 0.f : m_new, nullptr);
         }
-        // the row's maximum with three-input max instructions (8 independent chains)
-        float pm[8];
-#pragma unroll
-        for (int q8 = 0; q8 < 8; ++q8) pm[q8] = __uint_as_float(xs[q8]);
-#pragma unroll
-        for (int c = 8; c < kBN; c += 2)
-          pm[(c >> 1) & 7] = fmax3(pm[(c >> 1) & 7], __uint_as_float(xs[c]), __uint_as_float(xs[c + 1]));
-        const float mx = fmax3(fmax3(pm[0], pm[1], pm[2]), fmax3(pm[3], pm[4], pm[5]), fmaxf(pm[6], pm[7])) * sl2;
-        float m_new = m_run;
-        if (mx > m_run + kLazy || (m_run == -CUDART_INF_F && mx > -CUDART_INF_F)) m_new = mx;
-        const float base = m_new == -CUDART_INF_F ? 0.f : m_new;
-        const float alpha = ex2(m_run - base);
-        // p = 2^(s * scale * log2e - max): the scale-and-subtract and the row
-        // sum as packed f32x2 operations; every kPolyEvery-th pair of
-        // exponentials on the FMA pipe, the rest on MUFU
-        const uint64_t sc2 = f2_pack(sl2, sl2), nb2 = f2_pack(-base, -base);
-        uint64_t ps2[4];
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) ps2[q4] = 0;
-#pragma unroll
-        for (int kk = 0; kk < kBN / 2; ++kk) {
-          const uint64_t x2 = f2_fma(((uint64_t)xs[2 * kk + 1] << 32) | xs[2 * kk], sc2, nb2);
-          const bool fma_pipe = kPolyEvery > 0 && (kk % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1;
-          const uint64_t p2 = fma_pipe ? exp2_fma2(x2) : f2_pack(ex2(f2_lo(x2)), ex2(f2_hi(x2)));
-          ps2[kk & 3] = f2_add(ps2[kk & 3], p2);
-          xs[kk] = pack_bf16(f2_lo(p2), f2_hi(p2));
-        }
+        const float alpha = ex2(m_run - (m_new == -CUDART_INF_F ? 0.f : m_new));
         tmem_st32(s_addr, *reinterpret_cast<const uint32_t(*)[32]>(&xs[0]));
         tmem_st32(s_addr + 32, *reinterpret_cast<const uint32_t(*)[32]>(&xs[32]));
-        const uint64_t s01 = f2_add(ps2[0], ps2[1]), s23 = f2_add(ps2[2], ps2[3]);
-        const uint64_t s03 = f2_add(s01, s23);
-        l_run = l_run * alpha + (f2_lo(s03) + f2_hi(s03));
+        l_run = l_run * alpha + rs;
         // O holds the tiles before j (their PV completed before this tile's S
         // did); rescale it when some row of the warp raised its maximum
         if (j > 0 && __any_sync(0xffffffffu, m_new != m_run)) {

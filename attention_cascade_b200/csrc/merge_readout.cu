@@ -118,16 +118,14 @@ __device__ __forceinline__ float row_dot(const float* x, const float* w, int H, 
 // Candidate scores: the sum over the candidate's (row, token) pairs of
 // hidden[row] . lm_head[token], gathered with 16-byte loads (only option rows
 // of the LM head are ever read).  The score is parked in logprob[c] (NaN for
-// an invalid pair).  Blocks are four warps of few registers, so one fits on
-// an SM beside a CTA of the tensor-core attention kernel (576 threads x 96
-// registers) that may run on another stream; the readout's blocks are kept
-// short so they do not hold back that kernel's CTAs.
+// an invalid pair) for the set kernel below.
 //   one pair per candidate (no candidate offsets): a warp per candidate;
 //   several pairs: a block per candidate, warp w taking pairs w, w + 4, ...,
 //   so the candidate's rows are in flight together; the warps' partial sums
 //   are added in warp order.
+// One-pair bf16 candidates with H <= 4096 take the fused kernel further down
+// instead.
 constexpr int kCandWarps = 4;
-constexpr int kWideCands = 16384;  // from this many one-pair candidates on, the wide kernel
 
 template <typename T>
 __global__ void __launch_bounds__(kCandWarps * 32) readout_cand_kernel(ReadoutArgs a) {
@@ -165,49 +163,105 @@ __global__ void __launch_bounds__(kCandWarps * 32) readout_cand_kernel(ReadoutAr
   }
 }
 
-// Large one-pair readouts (many candidates, nothing else competing for the
-// SMs): a warp per candidate as above, but every 16-byte load of the two rows
-// is issued before any is used (ordered asm loads), W row first.
+// One 16-byte load of an LM-head or hidden row, through the read-only path.
 __device__ __forceinline__ uint4 ld_row16(const uint4* p) {
   uint4 v;
   asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
   return v;
 }
 
-__global__ void __launch_bounds__(kCandWarps * 32) readout_cand_wide_kernel(ReadoutArgs a) {
-  const int c = blockIdx.x * kCandWarps + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (c >= a.n_cands) return;
-  const int row = upper_segment(a.set_offsets, a.n_sets, c);  // one pair per candidate: row = set index
-  const int tok = a.pair_tok[c];
-  const bool bad = row < 0 || row >= a.R || tok < 0 || tok >= a.V;
+// One-pair candidates of bf16 rows with H <= 32 * 8 * NU: a warp per option
+// set.  The set's hidden row is loaded once into registers; the candidates'
+// LM-head rows stream through two register buffers, the next row's 16-byte
+// loads all issued before the current row's dot product, so two rows per warp
+// are always in flight.  The scores go to logprob and the same warp then takes
+// the set's log-softmax and argmax: no second kernel.  NU (16-byte vectors
+// per lane and row) is the smallest of a few sizes that covers H.
+template <int NU>
+__device__ __forceinline__ void ld_row_chunk(const uint4* p, int n, int lane, uint4 (&v)[NU]) {
+#pragma unroll
+  for (int u = 0; u < NU; ++u) {
+    const int i = u * 32 + lane;
+    v[u] = i < n ? ld_row16(p + i) : make_uint4(0, 0, 0, 0);
+  }
+}
+template <int NU>
+__device__ __forceinline__ float dot_chunk(const uint4 (&x)[NU], const uint4 (&w)[NU]) {
   float z = 0.f;
-  if (!bad) {
-    const uint4* x4 = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(a.hidden) + (size_t)row * a.H);
-    const uint4* w4 = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(a.lm_head) + (size_t)tok * a.H);
-    const int n = a.H >> 3;
-    for (int base = 0; base < n; base += 32 * kU) {
-      uint4 xa[kU], wa[kU];
 #pragma unroll
-      for (int u = 0; u < kU; ++u) {
-        const int i = base + u * 32 + lane;
-        wa[u] = i < n ? ld_row16(w4 + i) : make_uint4(0, 0, 0, 0);
-      }
+  for (int u = 0; u < NU; ++u) z += dot8(x[u], w[u]);
+  return z;
+}
+// log-softmax over a set's scores (in logprob[ca .. ce)) and the argmax, lowest
+// index on ties; a NaN score (an invalid pair) makes the set's log-probs NaN
+// and its choice -1
+__device__ __forceinline__ void set_softmax(const ReadoutArgs& a, int s, int ca, int ce, int lane) {
+  float mx = -CUDART_INF_F;
+  int best = -1;
+  bool any_nan = false;
+  for (int c = ca + lane; c < ce; c += 32) {
+    const float z = a.logprob[c];
+    if (isnan(z)) any_nan = true;
+    else if (best < 0 || z > mx) { mx = z; best = c; }
+  }
+  any_nan = __any_sync(0xffffffffu, any_nan);
 #pragma unroll
-      for (int u = 0; u < kU; ++u) {
-        const int i = base + u * 32 + lane;
-        xa[u] = i < n ? ld_row16(x4 + i) : make_uint4(0, 0, 0, 0);
-      }
-#pragma unroll
-      for (int u = 0; u < kU; ++u) z += dot8(xa[u], wa[u]);
+  for (int o = 16; o > 0; o >>= 1) {
+    const float om = __shfl_xor_sync(0xffffffffu, mx, o);
+    const int ob = __shfl_xor_sync(0xffffffffu, best, o);
+    if (ob >= 0 && (best < 0 || om > mx || (om == mx && ob < best))) { mx = om; best = ob; }
+  }
+  float sum = 0.f;
+  for (int c = ca + lane; c < ce; c += 32) sum += exp2f((a.logprob[c] - mx) * 1.4426950408889634f);
+  sum = warp_sum(sum);
+  const float lse = mx + log2f(sum) * 0.69314718055994531f;
+  __syncwarp();
+  for (int c = ca + lane; c < ce; c += 32) a.logprob[c] = any_nan ? CUDART_NAN_F : a.logprob[c] - lse;
+  if (lane == 0) a.choice[s] = any_nan ? -1 : best - ca;
+}
+
+template <int NU>
+__global__ void __launch_bounds__(kCandWarps * 32) readout_set_fused_kernel(ReadoutArgs a) {
+  const int s = blockIdx.x * kCandWarps + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (s >= a.n_sets) return;
+  const int ca = a.set_offsets[s], ce = a.set_offsets[s + 1];
+  if (!(ca >= 0 && ce >= ca && ce <= a.n_cands) || ce == ca) {
+    if (lane == 0) a.choice[s] = -1;
+    return;
+  }
+  const int n = a.H >> 3;  // 16-byte vectors per row
+  const bool row_ok = s < a.R;
+  const __nv_bfloat16* W = reinterpret_cast<const __nv_bfloat16*>(a.lm_head);
+  uint4 x[NU], w0[NU], w1[NU];
+  ld_row_chunk(reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(a.hidden) + (size_t)(row_ok ? s : 0) * a.H),
+               n, lane, x);
+  auto tok_of = [&](int c) { const int tk = a.pair_tok[c]; return (tk >= 0 && tk < a.V) ? tk : -1; };
+  int tk = tok_of(ca);
+  if (tk >= 0) ld_row_chunk(reinterpret_cast<const uint4*>(W + (size_t)tk * a.H), n, lane, w0);
+  for (int c = ca; c < ce; c += 2) {
+    // candidate c is in w0; load c + 1 into w1 before using w0, then c + 2 into w0
+    const int tk1 = c + 1 < ce ? tok_of(c + 1) : -1;
+    if (tk1 >= 0) ld_row_chunk(reinterpret_cast<const uint4*>(W + (size_t)tk1 * a.H), n, lane, w1);
+    float z = warp_sum(dot_chunk(x, w0));
+    if (lane == 0) {
+      const float zz = (tk < 0 || !row_ok) ? CUDART_NAN_F : (a.row_lse ? z - a.row_lse[s] : z);
+      a.logprob[c] = zz;
+      if (a.score) a.score[c] = zz;
     }
+    if (c + 1 >= ce) break;
+    const int tk2 = c + 2 < ce ? tok_of(c + 2) : -1;
+    if (tk2 >= 0) ld_row_chunk(reinterpret_cast<const uint4*>(W + (size_t)tk2 * a.H), n, lane, w0);
+    z = warp_sum(dot_chunk(x, w1));
+    if (lane == 0) {
+      const float zz = (tk1 < 0 || !row_ok) ? CUDART_NAN_F : (a.row_lse ? z - a.row_lse[s] : z);
+      a.logprob[c + 1] = zz;
+      if (a.score) a.score[c + 1] = zz;
+    }
+    tk = tk2;
   }
-  z = warp_sum(z);
-  if (lane == 0) {
-    const float zz = bad ? CUDART_NAN_F : (a.row_lse ? z - a.row_lse[row] : z);
-    a.logprob[c] = zz;
-    if (a.score) a.score[c] = zz;
-  }
+  __syncwarp();
+  set_softmax(a, s, ca, ce, lane);
 }
 
 template <typename T>
@@ -269,29 +323,7 @@ __global__ void __launch_bounds__(kSetWarps * 32) readout_set_kernel(ReadoutArgs
     if (lane == 0) a.choice[s] = -1;
     return;
   }
-  float mx = -CUDART_INF_F;
-  int best = -1;
-  bool any_nan = false;
-  for (int c = ca + lane; c < ce; c += 32) {
-    const float z = a.logprob[c];
-    if (isnan(z)) any_nan = true;
-    else if (best < 0 || z > mx) { mx = z; best = c; }
-  }
-  any_nan = __any_sync(0xffffffffu, any_nan);
-  // warp argmax: larger value wins, lower index breaks ties
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const float om = __shfl_xor_sync(0xffffffffu, mx, o);
-    const int ob = __shfl_xor_sync(0xffffffffu, best, o);
-    if (ob >= 0 && (best < 0 || om > mx || (om == mx && ob < best))) { mx = om; best = ob; }
-  }
-  float sum = 0.f;
-  for (int c = ca + lane; c < ce; c += 32) sum += exp2f((a.logprob[c] - mx) * 1.4426950408889634f);
-  sum = warp_sum(sum);
-  const float lse = mx + log2f(sum) * 0.69314718055994531f;
-  __syncwarp();
-  for (int c = ca + lane; c < ce; c += 32) a.logprob[c] = any_nan ? CUDART_NAN_F : a.logprob[c] - lse;
-  if (lane == 0) a.choice[s] = any_nan ? -1 : best - ca;
+  set_softmax(a, s, ca, ce, lane);
 }
 
 }  // namespace
@@ -318,9 +350,19 @@ cudaError_t launch_readout(const ReadoutArgs& a, jev_dtype dt, cudaStream_t s) {
       else readout_cand_block_kernel<float><<<a.n_cands, kCandWarps * 32, 0, s>>>(a);
     } else {
       const int blocks = (a.n_cands + kCandWarps - 1) / kCandWarps;
-      if (dt == JEV_BF16 && !a.pair_row && a.n_cands >= kWideCands) {
-        readout_cand_wide_kernel<<<blocks, kCandWarps * 32, 0, s>>>(a);
-      } else if (dt == JEV_BF16) readout_cand_kernel<__nv_bfloat16><<<blocks, kCandWarps * 32, 0, s>>>(a);
+      const int nu = (a.H / 8 + 31) / 32;  // 16-byte vectors per lane and row
+      if (dt == JEV_BF16 && !a.pair_row && nu <= 16) {
+        // a warp per set: scores and the set's softmax in one kernel
+        const dim3 g((a.n_sets + kCandWarps - 1) / kCandWarps), b(kCandWarps * 32);
+        if (nu <= 4) readout_set_fused_kernel<4><<<g, b, 0, s>>>(a);
+        else if (nu <= 6) readout_set_fused_kernel<6><<<g, b, 0, s>>>(a);
+        else if (nu <= 8) readout_set_fused_kernel<8><<<g, b, 0, s>>>(a);
+        else if (nu <= 12) readout_set_fused_kernel<12><<<g, b, 0, s>>>(a);
+        else if (nu <= 14) readout_set_fused_kernel<14><<<g, b, 0, s>>>(a);
+        else readout_set_fused_kernel<16><<<g, b, 0, s>>>(a);
+        return cudaGetLastError();
+      }
+      if (dt == JEV_BF16) readout_cand_kernel<__nv_bfloat16><<<blocks, kCandWarps * 32, 0, s>>>(a);
       else readout_cand_kernel<float><<<blocks, kCandWarps * 32, 0, s>>>(a);
     }
     cudaError_t e = cudaGetLastError();

@@ -708,6 +708,32 @@ def diag_attn(dev, jev, torch, stream, wl_name: str) -> dict:
             "note": "direct launches, not graph-replayed; for profiling captures, not a bench number"}
 
 
+def diag_readout(dev, jev, torch, stream, W=None) -> dict:
+    """The readout over 4096 option sets of 9 one-token options at the 7B
+    shape (H = 3584, V = 152064): the option rows of the LM head gathered from
+    HBM, one warp per set, scores and set softmax fused."""
+    pk, _ = peaks()
+    hbm = float(pk["hbm_gbs"])
+    cfg = synth.CONFIGS["wide_7b"]
+    if W is None:
+        W = load_lm_head(cfg, dev, torch, torch.bfloat16)
+    n_sets, opts = 4096, 9
+    rng = np.random.default_rng(7)
+    hidden = to_dev(synth.f32_to_bf16_bits(rng.standard_normal((n_sets, cfg.H)).astype(np.float32)), dev, torch)
+    base = rng.integers(0, cfg.V, n_sets)
+    toks = ((base[:, None] + 16411 * np.arange(opts)[None, :]) % cfg.V).astype(np.int32).reshape(-1)
+    so = torch.arange(0, n_sets * opts + 1, opts, dtype=torch.int32, device=dev)
+    pt = torch.from_numpy(toks).to(dev)
+    lp = torch.empty(toks.size, dtype=torch.float32, device=dev)
+    ch = torch.empty(n_sets, dtype=torch.int32, device=dev)
+    us = graph_us(torch, lambda: jev.jev_candidate_readout(hidden, W, so, pt, logprob=lp, choice=ch,
+                                                           stream=torch.cuda.current_stream()), stream, 200, 10)
+    nbytes = (toks.size + n_sets) * cfg.H * 2 + toks.size * 8 + n_sets * 4
+    return {"sets": n_sets, "options": opts, "H": cfg.H, "bytes_per_call": nbytes, "us": us,
+            "GBps": nbytes / us / 1e3, "frac_of_hbm": nbytes / us / 1e3 / hbm,
+            "note": "option rows of the LM head gathered from HBM; one kernel (scores and set softmax fused)"}
+
+
 def diagnostics(dev, jev, torch) -> dict:
     """Streaming efficiency of the HBM-bound kernels at sizes where it can be
     measured (the configs move kilobytes to a few megabytes per launch, below
@@ -722,23 +748,10 @@ def diagnostics(dev, jev, torch) -> dict:
     # ---- readout
     cfg = synth.CONFIGS["wide_7b"]
     W = load_lm_head(cfg, dev, torch, torch.bfloat16)
-    n_sets, opts = 4096, 9
     rng = np.random.default_rng(7)
-    hidden = to_dev(synth.f32_to_bf16_bits(rng.standard_normal((n_sets, cfg.H)).astype(np.float32)), dev, torch)
-    base = rng.integers(0, cfg.V, n_sets)
-    toks = ((base[:, None] + 16411 * np.arange(opts)[None, :]) % cfg.V).astype(np.int32).reshape(-1)
-    so = torch.arange(0, n_sets * opts + 1, opts, dtype=torch.int32, device=dev)
-    pt = torch.from_numpy(toks).to(dev)
-    lp = torch.empty(toks.size, dtype=torch.float32, device=dev)
-    ch = torch.empty(n_sets, dtype=torch.int32, device=dev)
-    us = graph_us(torch, lambda: jev.jev_candidate_readout(hidden, W, so, pt, logprob=lp, choice=ch,
-                                                           stream=torch.cuda.current_stream()), stream, 200, 10)
-    nbytes = (toks.size + n_sets) * cfg.H * 2 + toks.size * 8 + n_sets * 4
-    out["readout"] = {"sets": n_sets, "options": opts, "H": cfg.H, "bytes_per_call": nbytes, "us": us,
-                      "GBps": nbytes / us / 1e3, "frac_of_hbm": nbytes / us / 1e3 / hbm,
-                      "note": "option rows of the LM head gathered from HBM; two kernels (scores, set softmax)"}
+    out["readout"] = diag_readout(dev, jev, torch, stream, W)
     out["vocab_lse"] = diag_vocab_lse(dev, jev, torch, stream, W)
-    del W, hidden
+    del W
     torch.cuda.empty_cache()
     out["tree_schedule"] = diag_tree_schedule(dev, jev, torch, stream)
     torch.cuda.empty_cache()
@@ -1124,7 +1137,7 @@ def main():
     ap.add_argument("--per-config-steps", type=int, default=2000)
     ap.add_argument("--no-diagnostics", dest="diagnostics", action="store_false",
                     help="skip the streaming diagnostics at larger sizes (one GPU)")
-    ap.add_argument("--diag", choices=["vocab_lse", "tree_schedule", "attn", "decode"], default=None,
+    ap.add_argument("--diag", choices=["vocab_lse", "tree_schedule", "attn", "decode", "readout"], default=None,
                     help="run only this diagnostic on cuda:0 and print its JSON (a small case for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -1137,7 +1150,8 @@ def main():
         if args.diag == "attn":
             res = diag_attn("cuda:0", jev, torch, stream, args.workload)
         else:
-            fn = {"vocab_lse": diag_vocab_lse, "tree_schedule": diag_tree_schedule, "decode": diag_decode}[args.diag]
+            fn = {"vocab_lse": diag_vocab_lse, "tree_schedule": diag_tree_schedule, "decode": diag_decode,
+                  "readout": diag_readout}[args.diag]
             res = fn("cuda:0", jev, torch, stream)
         print(json.dumps({"diagnostic": args.diag, **res}))
     elif args.impl == "reference":

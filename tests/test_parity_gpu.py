@@ -137,22 +137,26 @@ def test_readout_multi_token_invalid_and_empty(jev, dtype):
     assert ch[1] == -1 and ch[2] == -1 and np.all(np.isnan(lp[3:5]))
 
 
-def test_readout_many_one_pair_candidates(jev):
-    # 2000 sets of 9 one-token options (18000 candidates): the wide one-pair readout kernel,
-    # with an invalid token in set 7 and an empty set 11
+@pytest.mark.parametrize("H", [256, 1544, 4096, 4104])
+def test_readout_many_one_pair_candidates(jev, H):
+    # 2000 sets of one-token options (mostly 9; set 3 has 1, set 5 has 40): at H <= 4096 one warp
+    # per set takes the scores and the set softmax (H = 1544 leaves a ragged last vector per lane
+    # group); at H = 4104 a warp per candidate, then the set kernel.  An invalid token in set 7,
+    # an empty set 11.
     rng = np.random.default_rng(5)
-    n_sets, opts, H, V = 2000, 9, 256, 4096
+    n_sets, opts, V = 2000, 9, 4096
     hidden = synth.f32_to_bf16_bits(rng.standard_normal((n_sets, H)).astype(np.float32))
     W = synth.f32_to_bf16_bits((0.05 * rng.standard_normal((V, H))).astype(np.float32))
     sizes = np.full(n_sets, opts)
-    sizes[11] = 0
+    sizes[3], sizes[5], sizes[11] = 1, 40, 0
     so = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
     toks = rng.integers(0, V, int(so[-1])).astype(np.int32)
     toks[so[7] + 2] = -3
     ref = oracle.candidate_readout(hidden, W, so, toks)
     lp, ch = run_readout(jev, hidden, dev(W), so, toks)
-    check_readout(lp, ch, ref, synth.BF16, "wide readout")
+    check_readout(lp, ch, ref, synth.BF16, f"one-pair readout H={H}")
     assert ch[7] == -1 and ch[11] == -1 and np.all(np.isnan(lp[so[7]:so[8]]))
+    assert ch[3] == 0 and lp[so[3]] == 0.0
 
 
 def test_readout_tie_goes_to_first(jev):
