@@ -18,24 +18,22 @@
 // partial and its log2 normaliser, and tc_fixup_kernel merges the segments of
 // each split tail tile.
 //
-// CTA = 12 warps (384 threads, 168 registers each):
-//   warps 0-3   Q tile 0: one thread per row (TMEM lane), all 128 score
-//               columns of the row, then the row's output (the epilogue)
-//   warps 4-7   Q tile 1, the same
-//   warp 8      TMA producer (Q once per segment, then K/V through a ring of stages)
-//   warp 9      TMEM allocator and tcgen05.mma issuer (one thread)
-//   warps 10-11 no role (they complete the third warpgroup)
+// CTA = 18 warps:
+//   warps 0-7   Q tile 0: warps 0-3 columns 0-63, warps 4-7 columns 64-127 of
+//               the S/P rows (TMEM lanes 0-127), and the matching halves of O
+//   warps 8-15  Q tile 1, same split
+//   warp 16     TMA producer (Q once per segment, then K/V through a ring of stages)
+//   warp 17     TMEM allocator and tcgen05.mma issuer (one thread)
 // TMEM (512 columns): S0/P0 [0,128), S1/P1 [128,256), O0 at 256, O1 at 256+D.
 // Per key tile j the MMA thread issues S_i = Q_i K_j^T (SS form), and after
-// the 128 threads of tile i have written P_i (bf16, aliasing S_i) it issues
+// both halves of tile i have written P_i (bf16, aliasing S_i) it issues
 // O_i += P_i V_j with P_i read from TMEM (TS form); tile 0's softmax overlaps
-// tile 1's MMAs and the other way round.  A thread owns a whole row, so the
-// row maximum needs no exchange; the softmax runs in the log2 domain with a
-// lazy running max (raised only when a row's maximum exceeds it by more than
-// 8, so O is rescaled rarely and P stays <= 2^8), its scale-and-subtract and
-// row sums as packed f32x2 operations, and a share of its exponentials on the
-// FMA pipe (a cubic with shifter range reduction): one exponential per score
-// on the MUFU unit alone would take as long as the tile's MMAs.
+// tile 1's MMAs and the other way round.  The two halves of a row exchange
+// their maxima through shared memory each key tile (a 64-thread barrier per
+// pair of warps); the softmax runs in the log2 domain with a lazy running max
+// (raised only when a row's maximum exceeds it by more than 8, so O is
+// rescaled rarely and P stays <= 2^8), its scale-and-subtract and row sums as
+// packed f32x2 operations.
 // Every mbarrier wait is bounded; a wait that runs out raises
 // JEV_DEV_WAIT_TIMEOUT in the status word and the CTA winds down: the other
 // waits give up, but before the CTA exits the producer waits for every load
@@ -53,11 +51,8 @@ using namespace tc;
 
 constexpr int kBM = 128;  // rows per Q tile (TMEM lanes)
 constexpr int kBN = 128;  // keys per K/V tile
-constexpr int kSoftWarps = 8;  // two warpgroups: one thread per row of each 128-row Q tile
-// + the TMA producer and the MMA issuer, and two warps that only complete the
-// last warpgroup: 384 threads leave 168 registers to a thread, room for a
-// row's 128 scores
-constexpr int kThreads = (kSoftWarps + 4) * 32;
+constexpr int kSoftWarps = 16;
+constexpr int kThreads = (kSoftWarps + 2) * 32;
 constexpr int kProducerWarp = kSoftWarps;
 constexpr int kMmaWarp = kSoftWarps + 1;
 constexpr float kLazy = 8.0f;  // log2 headroom before the running max moves
@@ -69,44 +64,50 @@ constexpr float kLazy = 8.0f;  // log2 headroom before the running max moves
 #endif
 constexpr int kPolyEvery = JEV_POLY_EVERY;
 
-// K and V tiles stream through separate rings: a K tile is released as soon
-// as its last S MMA has run, a V tile after its last PV MMA.
-#ifndef JEV_K_STAGES
-#define JEV_K_STAGES 3
-#endif
-#ifndef JEV_V_STAGES
-#define JEV_V_STAGES 2
-#endif
-// Each segment sweeps its prefix key tiles starting at a tile that depends on
-// its work tile, so the CTAs of one kv group are not all reading the same
-// tile at the same moment.
-#ifndef JEV_STAGGER
-#define JEV_STAGGER 1
-#endif
-
 template <int D>
 struct Cfg {
-  static constexpr int kNK = D == 128 ? JEV_K_STAGES : 4;  // K stages
-  static constexpr int kNV = D == 128 ? JEV_V_STAGES : 4;  // V stages
+  static constexpr int kNS = D == 128 ? 2 : 4;  // K/V stages
   static constexpr int kQBytes = kBM * D * 2;
   static constexpr int kKVBytes = kBN * D * 2;
   static constexpr int kBlk = 128 * 128;  // one 64-column, 128-row swizzled block
   static constexpr int kOffK = 2 * kQBytes;
-  static constexpr int kOffV = kOffK + kNK * kKVBytes;
-  static constexpr int kOffBar = kOffV + kNV * kKVBytes;
-  static constexpr int kOffSeg = kOffBar + 256;                  // two published segment descriptions
+  static constexpr int kOffV = kOffK + kNS * kKVBytes;
+  static constexpr int kOffBar = kOffV + kNS * kKVBytes;
+  static constexpr int kOffX = kOffBar + 256;                     // row-max exchange [tile][parity][half][row]
+  static constexpr int kOffL = kOffX + 2 * 2 * 2 * kBM * 4;       // row-sum exchange [tile][half][row]
+  static constexpr int kOffStg = kOffL + 2 * 2 * kBM * 4;        // per-warp output staging
+  static constexpr int kStgBytes = 8 * 64;                         // 8 rows x 32 bf16 columns
+  static constexpr int kOffSeg = kOffStg + kSoftWarps * kStgBytes;  // two published segment descriptions
   static constexpr int kSmem = kOffSeg + 128 + 1024;                   // + 1024-byte alignment slack
   static constexpr int kOCol = 256;                               // first TMEM column of O0
 };
 
 struct Bars {
-  uint32_t q_full, q_empty, k_full, k_empty, v_full, v_empty, s_full, p_full, o_full, drain;  // arrays: +8*i
+  uint32_t q_full, q_empty, k_full, v_full, kv_empty, s_full, p_full, o_full, drain;  // arrays: +8*i
 };
 
 struct Shared {
   uint32_t tmem_base;
   int abort;
 };
+
+__device__ __forceinline__ void named_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+// named barrier that also ANDs a flag over its threads, so that they all
+// leave with the same answer
+__device__ __forceinline__ bool named_sync_and(int id, int count, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred pi, po;\n\t"
+      "setp.ne.u32 pi, %1, 0;\n\t"
+      "bar.red.and.pred po, %2, %3, pi;\n\t"
+      "selp.u32 %0, 1, 0, po;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v), "r"(id), "r"(count)
+      : "memory");
+  return r != 0;
+}
 
 // Bounded wait (limit: AttnArgs::wait_cycles); once any wait of the CTA has
 // run out, the others give up at their first unsatisfied check.
@@ -177,18 +178,7 @@ struct Segment {
   int lo;         // first suffix key of the window (when the segment holds the suffix unit)
   bool complete;  // the segment is the whole tile: write the final output
   int slot;       // partial slot when not complete
-  int rot;        // the segment's prefix tiles are visited from tile ua + rot on, cyclically
 };
-
-// The prefix tiles of work tile w's segment of n_pre of them start at this offset.
-__device__ __forceinline__ int seg_rot(int w, int n_pre) {
-  return (JEV_STAGGER && n_pre > 1) ? (int)(((long long)w * 7) % n_pre) : 0;
-}
-// Unit (128-key prefix tile) of the segment's j-th prefix tile, j < n_pre.
-__device__ __forceinline__ int pre_unit(int ua, int rot, int n_pre, int j) {
-  const int x = j + rot;
-  return ua + (x >= n_pre ? x - n_pre : x);
-}
 static_assert(2 * sizeof(Segment) <= 128, "segment ring");
 
 // A CTA's segments: first its whole tiles (k < full_waves: tile c + k*n_ctas),
@@ -246,7 +236,6 @@ __device__ __forceinline__ Segment make_segment(const AttnArgs& a, int c, int w,
   }
   sg.complete = sg.ua == 0 && sg.ub == a.P;
   sg.slot = (tail && tc_unit_begin(a, c) >= t0) ? 2 * c : 2 * c + 1;
-  sg.rot = seg_rot(w, sg.n_pre);
   return sg;
 }
 
@@ -260,6 +249,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   const uint32_t sbase = smem_u32(smem);
   Shared* sh = reinterpret_cast<Shared*>(smem + C::kOffBar + 224);
+  float* xmax = reinterpret_cast<float*>(smem + C::kOffX);
+  float* xsum = reinterpret_cast<float*>(smem + C::kOffL);
   // The producer derives each segment's description (its key window takes a
   // warp-wide read of token info) and publishes it here before its arrive on
   // q_full; the other roles read it after their wait on q_full.  Two slots:
@@ -271,10 +262,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   B.q_full = bar0;
   B.q_empty = bar0 + 8;
   B.k_full = bar0 + 16;
-  B.k_empty = B.k_full + 8 * C::kNK;
-  B.v_full = B.k_empty + 8 * C::kNK;
-  B.v_empty = B.v_full + 8 * C::kNV;
-  B.s_full = B.v_empty + 8 * C::kNV;
+  B.v_full = B.k_full + 8 * C::kNS;
+  B.kv_empty = B.v_full + 8 * C::kNS;
+  B.s_full = B.kv_empty + 8 * C::kNS;
   B.p_full = B.s_full + 16;
   B.o_full = B.p_full + 16;
   B.drain = B.o_full + 16;
@@ -287,17 +277,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(B.q_full, 2);  // the producer's expect-tx arrival, then its arrival after publishing the segment
     mbar_init(B.q_empty, 1);
-    for (int s = 0; s < C::kNK; ++s) {
+    for (int s = 0; s < C::kNS; ++s) {
       mbar_init(B.k_full + 8 * s, 1);
-      mbar_init(B.k_empty + 8 * s, 1);
-    }
-    for (int s = 0; s < C::kNV; ++s) {
       mbar_init(B.v_full + 8 * s, 1);
-      mbar_init(B.v_empty + 8 * s, 1);
+      mbar_init(B.kv_empty + 8 * s, 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(B.s_full + 8 * i, 1);
-      mbar_init(B.p_full + 8 * i, kBM);  // one arrival per row of the tile
+      mbar_init(B.p_full + 8 * i, 256);
       mbar_init(B.o_full + 8 * i, 1);
     }
     mbar_init(B.drain, 1);
@@ -319,59 +306,34 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == kProducerWarp) {
     // ---------------------------------------------------------------- TMA producer
-    // Per segment: Q, then key tile 0's K, then for each tile j the K of tile
-    // j + 1 ahead of the V of tile j (a K tile is needed one MMA earlier than
-    // the V tile of the same index).  Key tile JJ (counted over the CTA's
-    // segments) goes to K stage JJ % kNK and V stage JJ % kNV.
     long long J = 0;
-    long long k_armed = 0, v_armed = 0;  // K / V tiles whose loads this warp has issued
-    int q_armed = 0;                     // Q tiles loaded
+    long long kv_armed = 0;  // key tiles whose K and V loads this warp has issued
+    int q_armed = 0;         // Q tiles loaded
     int k = 0;
     bool ok = true;
-    // lane 0: load the K (or V) tile of the segment's j-th key tile (global index JJ)
-    auto load_kv = [&](bool is_k, const Segment& sg, int j, long long JJ) -> bool {
-      const int ns = is_k ? C::kNK : C::kNV;
-      const int st = (int)(JJ % ns);
-      const long long use = JJ / ns;
-      if (JJ >= ns && !wait_bar((is_k ? B.k_empty : B.v_empty) + 8 * st, (uint32_t)((use - 1) & 1), abort, a.status,
-                                a.wait_cycles))
-        return false;
-      const bool pre = j < sg.n_pre;
-      const int kb = pre ? pre_unit(sg.ua, sg.rot, sg.n_pre, j) * kBN : sg.lo + (j - sg.n_pre) * kBN;
-      const CUtensorMap* m = is_k ? (pre ? &tm_kp : &tm_ks) : (pre ? &tm_vp : &tm_vs);
-      const uint32_t dst = sbase + (is_k ? C::kOffK : C::kOffV) + st * C::kKVBytes;
-      const uint32_t full = (is_k ? B.k_full : B.v_full) + 8 * st;
-      mbar_expect_tx(full, C::kKVBytes);
-      for (int b = 0; b < D / 64; ++b) tma_load_2d(dst + b * C::kBlk, m, sg.g * D + b * 64, kb, full);
-      if (is_k) k_armed = JJ + 1;
-      else v_armed = JJ + 1;
-      return true;
-    };
     tma_prefetch_desc(&tm_q);
     // the first segment's leading prefix key tiles need nothing from the pack:
     // their loads start before the wait (the pack lets this kernel launch only
-    // once every kernel before it in the stream has completed), in the same
-    // order as below and only into stages not used before
-    int pre_k = 0, pre_v = 0;
+    // once every kernel before it in the stream has completed)
+    int pre0 = 0;
     {
       SegIter it0{0, u_begin, u_end};
       int w0, ua0, ub0;
       bool tl0;
       if (seg_next(a, cta, it0, w0, ua0, ub0, tl0)) {
-        Segment s0{};
-        s0.ua = ua0;
-        s0.g = w0 / a.n_pairs;
-        s0.n_pre = max(0, min(ub0, a.n_pre) - ua0);
-        s0.rot = seg_rot(w0, s0.n_pre);
-        pre_k = min(s0.n_pre, C::kNK);
-        pre_v = min(s0.n_pre, C::kNV);
-        if (lane == 0) {
-          if (pre_k > 0) load_kv(true, s0, 0, 0);
-          for (int j = 0; j < max(pre_k, pre_v); ++j) {
-            if (j + 1 < pre_k) load_kv(true, s0, j + 1, j + 1);
-            if (j < pre_v) load_kv(false, s0, j, j);
+        pre0 = min(max(0, min(ub0, a.n_pre) - ua0), C::kNS);
+        const int g0 = w0 / a.n_pairs;
+        if (lane == 0)
+          for (int j = 0; j < pre0; ++j) {
+            const uint32_t ks = sbase + C::kOffK + j * C::kKVBytes, vs = sbase + C::kOffV + j * C::kKVBytes;
+            mbar_expect_tx(B.k_full + 8 * j, C::kKVBytes);
+            for (int b = 0; b < D / 64; ++b)
+              tma_load_2d(ks + b * C::kBlk, &tm_kp, g0 * D + b * 64, (ua0 + j) * kBN, B.k_full + 8 * j);
+            mbar_expect_tx(B.v_full + 8 * j, C::kKVBytes);
+            for (int b = 0; b < D / 64; ++b)
+              tma_load_2d(vs + b * C::kBlk, &tm_vp, g0 * D + b * 64, (ua0 + j) * kBN, B.v_full + 8 * j);
           }
-        }
+        kv_armed = pre0;
       }
     }
     pdl_wait();
@@ -400,11 +362,25 @@ __global__ void __launch_bounds__(kThreads, 1)
           seg_sm[k & 1] = sg;
           mbar_arrive(B.q_full);
         }
-        const int dk = k == 0 ? pre_k : 0, dv = k == 0 ? pre_v : 0;  // tiles already loaded
-        if (ok && dk == 0) ok = load_kv(true, sg, 0, J);
-        for (int j = 0; ok && j < sg.n; ++j) {
-          if (j + 1 < sg.n && j + 1 >= dk) ok = load_kv(true, sg, j + 1, J + j + 1);
-          if (ok && j >= dv) ok = load_kv(false, sg, j, J + j);
+        for (int j = k == 0 ? pre0 : 0; ok && j < sg.n; ++j) {
+          const long long JJ = J + j;
+          const int st = (int)(JJ % C::kNS);
+          const long long use = JJ / C::kNS;
+          if (JJ >= C::kNS &&
+              !wait_bar(B.kv_empty + 8 * st, (uint32_t)((use - 1) & 1), abort, a.status, a.wait_cycles)) {
+            ok = false;
+            break;
+          }
+          const bool pre = j < sg.n_pre;
+          const int kb = pre ? (sg.ua + j) * kBN : sg.lo + (j - sg.n_pre) * kBN;
+          const CUtensorMap* mk = pre ? &tm_kp : &tm_ks;
+          const CUtensorMap* mv = pre ? &tm_vp : &tm_vs;
+          const uint32_t ks = sbase + C::kOffK + st * C::kKVBytes, vs = sbase + C::kOffV + st * C::kKVBytes;
+          mbar_expect_tx(B.k_full + 8 * st, C::kKVBytes);
+          for (int b = 0; b < D / 64; ++b) tma_load_2d(ks + b * C::kBlk, mk, sg.g * D + b * 64, kb, B.k_full + 8 * st);
+          mbar_expect_tx(B.v_full + 8 * st, C::kKVBytes);
+          for (int b = 0; b < D / 64; ++b) tma_load_2d(vs + b * C::kBlk, mv, sg.g * D + b * 64, kb, B.v_full + 8 * st);
+          kv_armed = JJ + 1;
         }
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -414,13 +390,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       // Drain: the last phase of every stage this warp armed, and of the Q
       // buffer, has completed (its loads have landed) before the CTA may
       // exit.  On the normal path these phases completed long ago.
-      for (int st = 0; st < C::kNK; ++st) {
-        const long long uses = k_armed > st ? (k_armed - st + C::kNK - 1) / C::kNK : 0;
-        if (uses > 0) drain_bar(B.k_full + 8 * st, (uint32_t)((uses - 1) & 1), a.status);
-      }
-      for (int st = 0; st < C::kNV; ++st) {
-        const long long uses = v_armed > st ? (v_armed - st + C::kNV - 1) / C::kNV : 0;
-        if (uses > 0) drain_bar(B.v_full + 8 * st, (uint32_t)((uses - 1) & 1), a.status);
+      for (int st = 0; st < C::kNS; ++st) {
+        const long long uses = kv_armed > st ? (kv_armed - st + C::kNS - 1) / C::kNS : 0;
+        if (uses > 0) {
+          drain_bar(B.k_full + 8 * st, (uint32_t)((uses - 1) & 1), a.status);
+          drain_bar(B.v_full + 8 * st, (uint32_t)((uses - 1) & 1), a.status);
+        }
       }
       if (q_armed > 0) drain_bar(B.q_full, (uint32_t)((q_armed - 1) & 1), a.status);
     }
@@ -465,34 +440,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) {
         const int n = sg.n;  // >= 1
         if (ok) {
-          const int sk0 = (int)(J % C::kNK);
-          ok = wait_bar(B.k_full + 8 * sk0, (uint32_t)((J / C::kNK) & 1), abort, a.status, a.wait_cycles);
+          const int st0 = (int)(J % C::kNS);
+          ok = wait_bar(B.k_full + 8 * st0, (uint32_t)((J / C::kNS) & 1), abort, a.status, a.wait_cycles);
           fence_after_sync();
           if (ok) {
-            issue_s(0, sk0);
-            issue_s(1, sk0);
-            mma_commit(B.k_empty + 8 * sk0);  // the K tile's last MMA
+            issue_s(0, st0);
+            issue_s(1, st0);
           }
         }
         for (int j = 0; ok && j < n; ++j) {
           const long long JJ = J + j, JJ1 = JJ + 1;
-          const int sv = (int)(JJ % C::kNV), sk1 = (int)(JJ1 % C::kNK);
-          const uint32_t phv = (uint32_t)((JJ / C::kNV) & 1), phk1 = (uint32_t)((JJ1 / C::kNK) & 1);
+          const int st = (int)(JJ % C::kNS), st1 = (int)(JJ1 % C::kNS);
+          const uint32_t ph = (uint32_t)((JJ / C::kNS) & 1), ph1 = (uint32_t)((JJ1 / C::kNS) & 1);
           const uint32_t pp = (uint32_t)(JJ & 1);
-          if (!wait_bar(B.v_full + 8 * sv, phv, abort, a.status, a.wait_cycles)) { ok = false; break; }
+          if (!wait_bar(B.v_full + 8 * st, ph, abort, a.status, a.wait_cycles)) { ok = false; break; }
           if (!wait_bar(B.p_full, pp, abort, a.status, a.wait_cycles)) { ok = false; break; }
           fence_after_sync();
-          issue_pv(0, sv, j > 0);
+          issue_pv(0, st, j > 0);
           if (j == n - 1) mma_commit(B.o_full);
           if (j + 1 < n) {
-            if (!wait_bar(B.k_full + 8 * sk1, phk1, abort, a.status, a.wait_cycles)) { ok = false; break; }
+            if (!wait_bar(B.k_full + 8 * st1, ph1, abort, a.status, a.wait_cycles)) { ok = false; break; }
             fence_after_sync();
-            issue_s(0, sk1);
+            issue_s(0, st1);
           }
           if (!wait_bar(B.p_full + 8, pp, abort, a.status, a.wait_cycles)) { ok = false; break; }
           fence_after_sync();
-          issue_pv(1, sv, j > 0);
-          mma_commit(B.v_empty + 8 * sv);  // the V tile's last MMA
+          issue_pv(1, st, j > 0);
+          mma_commit(B.kv_empty + 8 * st);
           if (j == n - 1) mma_commit(B.o_full + 8);
           // q_empty releases the Q buffer and lets the producer publish the next
           // segment.  It is committed only after both p_full waits of a tile of
@@ -501,8 +475,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // softmax thread still in the previous epilogue, that thread's parity
           // wait would alias the later phase and never return.
           if (j + 1 < n) {
-            issue_s(1, sk1);
-            mma_commit(B.k_empty + 8 * sk1);
+            issue_s(1, st1);
             if (j + 2 == n) mma_commit(B.q_empty);
           } else if (n == 1) {
             mma_commit(B.q_empty);
@@ -518,14 +491,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_commit(B.drain);
       drain_bar(B.drain, 0, a.status);
     }
-  } else if (warp < kSoftWarps) {
+  } else {
     // ---------------------------------------------------------------- softmax + epilogue
-    // warp w: tile i = w / 4, TMEM lanes 32 (w % 4) .. +31; thread = one row of
-    // the tile's 128, holding all 128 of its scores (no exchange with another thread)
-    const int i = warp >> 2, q = warp & 3, r = q * 32 + lane;
+    constexpr int kHalfCols = kBN / 2;  // score columns per thread
+    constexpr int kHalfD = D / 2;       // output columns per thread
+    const int i = warp >> 3, hf = (warp >> 2) & 1, q = warp & 3, r = q * 32 + lane;
+    const int bar_id = 1 + i;  // named barrier of the 256 threads of tile i
+    // named barrier of the two warps that hold the two halves of the same 32 rows
+    const int pair_bar = 3 + i * 4 + q;
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-    const uint32_t s_addr = tmem + i * kBN + lane_off;  // the row's 128 score columns; P packed over the first 64
-    const uint32_t o_addr = tmem + C::kOCol + i * D + lane_off;
+    const uint32_t s_addr = tmem + i * kBN + hf * kHalfCols + lane_off;       // this half's score columns
+    const uint32_t p_addr = tmem + i * kBN + hf * (kHalfCols / 2) + lane_off;  // its packed P columns
+    const uint32_t o_addr = tmem + C::kOCol + i * D + hf * kHalfD + lane_off;
+    const int c_base = hf * kHalfCols;  // key column of this thread's first score
     const float sl2 = a.scale_log2;
     long long J = 0;
     int k = 0;
@@ -537,8 +515,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     int sw, sua, sub;
     bool stail;
     for (; ok && seg_next(a, cta, it, sw, sua, sub, stail); ++k, ++it.k) {
-      // waits are warp-uniform: the TMEM loads and stores below are warp-wide
-      ok = __all_sync(0xffffffffu, wait_bar(B.q_full, k & 1, abort, a.status, a.wait_cycles));
+      // The 256 threads of the tile group agree on the q_full wait before any
+      // reads the segment description: a thread whose wait gave up must not
+      // read a description the producer may not have published, and the
+      // group must run the same number of key tiles (the same named barriers).
+      ok = named_sync_and(bar_id, 256, wait_bar(B.q_full, k & 1, abort, a.status, a.wait_cycles));
       if (!ok) break;
       const Segment sg = seg_sm[k & 1];
       const int m = sg.m0 + i * kBM + r;
@@ -554,117 +535,95 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       float m_run = -CUDART_INF_F, l_run = 0.f;
+      // A wait that fails (a timeout somewhere in the CTA) does not leave the
+      // loop: the thread runs the remaining tiles on whatever TMEM holds, so
+      // that every thread of the tile group meets the same named barriers, and
+      // the group agrees on the outcome at the epilogue's reducing barrier.
       for (int j = 0; j < sg.n; ++j) {
         const long long JJ = J + j;
-        ok = __all_sync(0xffffffffu, wait_bar(B.s_full + 8 * i, (uint32_t)(JJ & 1), abort, a.status, a.wait_cycles));
-        if (!ok) break;
+        if (!wait_bar(B.s_full + 8 * i, (uint32_t)(JJ & 1), abort, a.status, a.wait_cycles)) ok = false;
         fence_after_sync();
-        // the row's 128 raw scores; P is later packed in place into xs[0..63]
-        uint32_t xs[kBN];
+        // this half's 64 raw scores; P is later packed in place into xs[0..31]
+        uint32_t xs[kHalfCols];
+        tmem_ld64(s_addr, xs);
         constexpr uint32_t kNegInf = 0xff800000u;
-        auto load_masked = [&]() {
-          tmem_ld128(s_addr, xs);
-          if (j < sg.n_pre) {
-            const int lim = a.Lp - pre_unit(sg.ua, sg.rot, sg.n_pre, j) * kBN;  // keys past the prefix are padding
-            if (lim < kBN) {
+        if (j < sg.n_pre) {
+          const int lim = a.Lp - (sg.ua + j) * kBN - c_base;  // keys past the prefix are padding
+          if (lim < kHalfCols) {
 #pragma unroll
-              for (int c = 0; c < kBN; ++c)
-                if (c >= lim) xs[c] = kNegInf;
-            }
-          } else {
-            // suffix window
-            const int kb = sg.lo + (j - sg.n_pre) * kBN;
-            if (!TREE) {
-              // flat row: the keys start .. last of its own branch
-              const int c_lo = start - kb, c_hi = last - kb;
-              // the mask is skipped when every row of the warp sees every key of this tile
-              const bool whole = __all_sync(0xffffffffu, c_lo <= 0 && c_hi >= kBN - 1);
-              if (!whole) {
-#pragma unroll
-                for (int c = 0; c < kBN; ++c)
-                  if (!(c >= c_lo && c <= c_hi)) xs[c] = kNegInf;
-              }
-            } else {
-              // tree row t: key k is on its root path when k <= t and t lies in the
-              // packed tokens of k's node's subtree (read here, where needed)
-#pragma unroll
-              for (int c = 0; c < kBN; ++c) {
-                const int kk = kb + c;
-                const int e = kk < a.key_rows ? __ldg(a.key_end + kk) : -1;
-                if (!(kk <= t && t < e)) xs[c] = kNegInf;
-              }
-            }
-          }
-        };
-        // p = 2^(s * scale * log2e - base) for the row's 128 scores, packed in
-        // place as bf16 pairs into xs[0..63]; returns the row sum.  The
-        // scale-and-subtract and the sum run as packed f32x2 operations, every
-        // kPolyEvery-th pair of exponentials on the FMA pipe, the rest on
-        // MUFU.  With `mxp`, the maximum of the raw scores is taken alongside.
-        auto exp_pack = [&](float base, float* mxp) -> float {
-          const uint64_t sc2 = f2_pack(sl2, sl2), nb2 = f2_pack(-base, -base);
-          uint64_t ps2[4];
-          float pm[4];
-#pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            ps2[q4] = 0;
-            pm[q4] = -CUDART_INF_F;
-          }
-#pragma unroll
-          for (int kk = 0; kk < kBN / 2; ++kk) {
-            if (mxp) pm[kk & 3] = fmax3(pm[kk & 3], __uint_as_float(xs[2 * kk]), __uint_as_float(xs[2 * kk + 1]));
-            const uint64_t x2 = f2_fma(((uint64_t)xs[2 * kk + 1] << 32) | xs[2 * kk], sc2, nb2);
-            const bool fma_pipe = kPolyEvery > 0 && (kk % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1;
-            const uint64_t p2 = fma_pipe ? exp2_fma2(x2) : f2_pack(ex2(f2_lo(x2)), ex2(f2_hi(x2)));
-            ps2[kk & 3] = f2_add(ps2[kk & 3], p2);
-            xs[kk] = pack_bf16(f2_lo(p2), f2_hi(p2));
-          }
-          if (mxp) *mxp = fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3]));
-          const uint64_t s03 = f2_add(f2_add(ps2[0], ps2[1]), f2_add(ps2[2], ps2[3]));
-          return f2_lo(s03) + f2_hi(s03);
-        };
-        load_masked();
-        float m_new, rs;
-        if (__all_sync(0xffffffffu, m_run != -CUDART_INF_F)) {
-          // every row of the warp has a running maximum: the exponentials start
-          // from it at once and the tile's maximum is found alongside; only a
-          // row whose maximum rises by more than kLazy (rare) makes the warp
-          // reload S and start again from the new maxima
-          float mxs;
-          rs = exp_pack(m_run, &mxs);
-          const float mx = mxs * sl2;
-          const bool raise = mx > m_run + kLazy;
-          m_new = raise ? mx : m_run;
-          if (__any_sync(0xffffffffu, raise)) {
-            load_masked();
-            rs = exp_pack(m_new, nullptr);
+            for (int c = 0; c < kHalfCols; ++c)
+              if (c >= lim) xs[c] = kNegInf;
           }
         } else {
-          // the row's maximum first (the first tile, or rows still without one)
-          float pm[8];
+          // suffix window
+          const int kb = sg.lo + (j - sg.n_pre) * kBN + c_base;
+          if (!TREE) {
+            // flat row: the keys start .. last of its own branch
+            const int c_lo = start - kb, c_hi = last - kb;
+            // the mask is skipped when every row of the warp sees all 64 of its keys in this tile
+            const bool whole = __all_sync(0xffffffffu, c_lo <= 0 && c_hi >= kHalfCols - 1);
+            if (!whole) {
 #pragma unroll
-          for (int q8 = 0; q8 < 8; ++q8) pm[q8] = __uint_as_float(xs[q8]);
+              for (int c = 0; c < kHalfCols; ++c)
+                if (!(c >= c_lo && c <= c_hi)) xs[c] = kNegInf;
+            }
+          } else {
+            // tree row t: key k is on its root path when k <= t and t lies in the
+            // packed tokens of k's node's subtree (read here, where needed)
 #pragma unroll
-          for (int c = 8; c < kBN; c += 2)
-            pm[(c >> 1) & 7] = fmax3(pm[(c >> 1) & 7], __uint_as_float(xs[c]), __uint_as_float(xs[c + 1]));
-          const float mx = fmax3(fmax3(pm[0], pm[1], pm[2]), fmax3(pm[3], pm[4], pm[5]), fmaxf(pm[6], pm[7])) * sl2;
-          m_new = m_run;
-          if (mx > m_run + kLazy || (m_run == -CUDART_INF_F && mx > -CUDART_INF_F)) m_new = mx;
-          rs = exp_pack(m_new == -CUDART_INF_F ? 0.f : m_new, nullptr);
+            for (int c = 0; c < kHalfCols; ++c) {
+              const int kk = kb + c;
+              const int e = kk < a.key_rows ? __ldg(a.key_end + kk) : -1;
+              if (!(kk <= t && t < e)) xs[c] = kNegInf;
+            }
+          }
         }
-        const float alpha = ex2(m_run - (m_new == -CUDART_INF_F ? 0.f : m_new));
-        tmem_st32(s_addr, *reinterpret_cast<const uint32_t(*)[32]>(&xs[0]));
-        tmem_st32(s_addr + 32, *reinterpret_cast<const uint32_t(*)[32]>(&xs[32]));
+        // this half's maximum with three-input max instructions (8 independent chains)
+        float pm[8];
+#pragma unroll
+        for (int q8 = 0; q8 < 8; ++q8) pm[q8] = __uint_as_float(xs[q8]);
+#pragma unroll
+        for (int c = 8; c < kHalfCols; c += 2)
+          pm[(c >> 1) & 7] = fmax3(pm[(c >> 1) & 7], __uint_as_float(xs[c]), __uint_as_float(xs[c + 1]));
+        const float half_max = fmax3(fmax3(pm[0], pm[1], pm[2]), fmax3(pm[3], pm[4], pm[5]), fmaxf(pm[6], pm[7]));
+        // both halves of the row agree on the maximum (double-buffered by tile parity)
+        float* xm = xmax + ((i * 2 + (int)(JJ & 1)) * 2) * kBM;
+        xm[hf * kBM + r] = half_max;
+        named_sync(pair_bar, 64);
+        const float mx = fmaxf(half_max, xm[(1 - hf) * kBM + r]) * sl2;
+        float m_new = m_run;
+        if (mx > m_run + kLazy || (m_run == -CUDART_INF_F && mx > -CUDART_INF_F)) m_new = mx;
+        const float base = m_new == -CUDART_INF_F ? 0.f : m_new;
+        const float alpha = ex2(m_run - base);
+        // p = 2^(s * scale * log2e - max): one exponential per score; the
+        // scale-and-subtract and the row sum run as packed f32x2 operations
+        // (one instruction per pair of scores)
+        const uint64_t sc2 = f2_pack(sl2, sl2), nb2 = f2_pack(-base, -base);
+        uint64_t ps2[4];
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) ps2[q4] = 0;
+#pragma unroll
+        for (int kk = 0; kk < kHalfCols / 2; ++kk) {
+          const uint64_t x2 = f2_fma(((uint64_t)xs[2 * kk + 1] << 32) | xs[2 * kk], sc2, nb2);
+          const float x0 = f2_lo(x2), x1 = f2_hi(x2);
+          const bool fma_pipe = kPolyEvery > 0 && (kk % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1;
+          const float p0 = fma_pipe ? exp2_fma(x0) : ex2(x0);
+          const float p1 = fma_pipe ? exp2_fma(x1) : ex2(x1);
+          ps2[kk & 3] = f2_add(ps2[kk & 3], f2_pack(p0, p1));
+          xs[kk] = pack_bf16(p0, p1);
+        }
+        tmem_st32(p_addr, *reinterpret_cast<const uint32_t(*)[32]>(&xs[0]));
+        const uint64_t s01 = f2_add(ps2[0], ps2[1]), s23 = f2_add(ps2[2], ps2[3]);
+        const uint64_t s03 = f2_add(s01, s23);
+        const float rs = f2_lo(s03) + f2_hi(s03);
         l_run = l_run * alpha + rs;
-        // O holds the tiles before j (their PV completed before this tile's S
-        // did); rescale it when some row of the warp raised its maximum
         if (j > 0 && __any_sync(0xffffffffu, m_new != m_run)) {
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
+          for (int c = 0; c < kHalfD / 32; ++c) {
             uint32_t uu[32];
             tmem_ld32(o_addr + c * 32, uu);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) uu[e] = __float_as_uint(__uint_as_float(uu[e]) * alpha);
+            for (int kk = 0; kk < 32; ++kk) uu[kk] = __float_as_uint(__uint_as_float(uu[kk]) * alpha);
             tmem_st32(o_addr + c * 32, uu);
           }
         }
@@ -673,28 +632,49 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_before_sync();
         mbar_arrive(B.p_full + 8 * i);
       }
-      if (!ok) break;
-      ok = __all_sync(0xffffffffu, wait_bar(B.o_full + 8 * i, (uint32_t)(k & 1), abort, a.status, a.wait_cycles));
-      if (!ok) break;
+      if (ok) ok = wait_bar(B.o_full + 8 * i, (uint32_t)(k & 1), abort, a.status, a.wait_cycles);
       fence_after_sync();
-      const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-      const bool write = valid && t >= 0;
+      // the row's normaliser is the sum of both halves' partial sums
+      xsum[(i * 2 + hf) * kBM + r] = l_run;
+      ok = named_sync_and(bar_id, 256, ok);
+      const float l_row = l_run + xsum[(i * 2 + 1 - hf) * kBM + r];
+      named_sync(bar_id, 256);  // the exchange slots are free again
+      const float inv = l_row > 0.f ? 1.f / l_row : 0.f;
+      const bool write = ok && valid && t >= 0;
       const int tt = valid ? m / a.G : 0;
       const int h = valid ? min(max(a.hinv[sg.g * a.G + (m - tt * a.G)], 0), a.Hq - 1) : 0;
       if (sg.complete) {
-        // bf16 output row (t, h): D * 2 contiguous bytes, 64 per 32 columns
-        uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + ((size_t)tt * a.Hq + h) * D);
+        // bf16 output rows (t, h) lie D*2 bytes apart or more; per 32 columns
+        // a warp stages eight of its half-rows at a time in shared memory so
+        // that each global store writes 64 contiguous bytes of each of 8 rows
+        const unsigned long long dst_row =
+            write ? reinterpret_cast<unsigned long long>(reinterpret_cast<__nv_bfloat16*>(a.out) +
+                                                         ((size_t)tt * a.Hq + h) * D + hf * kHalfD)
+                  : 0ull;
+        uint8_t* stg = smem + C::kOffStg + warp * C::kStgBytes;
+        const int rd_row = lane >> 2, rd_c = lane & 3;  // the 16-byte chunk this lane stores
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = 0; c < kHalfD / 32; ++c) {
           uint32_t uu[32];
           tmem_ld32(o_addr + c * 32, uu);
-          if (write) {
+          uint32_t* pk = uu;  // packed in place: entry kk reads entries 2kk, 2kk+1 >= kk
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-              dst[c * 4 + e] = make_uint4(pack_bf16(__uint_as_float(uu[8 * e]) * inv, __uint_as_float(uu[8 * e + 1]) * inv),
-                                          pack_bf16(__uint_as_float(uu[8 * e + 2]) * inv, __uint_as_float(uu[8 * e + 3]) * inv),
-                                          pack_bf16(__uint_as_float(uu[8 * e + 4]) * inv, __uint_as_float(uu[8 * e + 5]) * inv),
-                                          pack_bf16(__uint_as_float(uu[8 * e + 6]) * inv, __uint_as_float(uu[8 * e + 7]) * inv));
+          for (int kk = 0; kk < 16; ++kk)
+            pk[kk] = pack_bf16(__uint_as_float(uu[2 * kk]) * inv, __uint_as_float(uu[2 * kk + 1]) * inv);
+#pragma unroll
+          for (int rq = 0; rq < 4; ++rq) {
+            if ((lane >> 3) == rq) {
+              const int rr = lane & 7;
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                *reinterpret_cast<uint4*>(stg + rr * 64 + ((e ^ (rr & 3)) * 16)) =
+                    make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+            }
+            __syncwarp();
+            const uint4 v = *reinterpret_cast<const uint4*>(stg + rd_row * 64 + ((rd_c ^ (rd_row & 3)) * 16));
+            const unsigned long long d = __shfl_sync(0xffffffffu, dst_row, rq * 8 + rd_row);
+            if (d) reinterpret_cast<uint4*>(d)[c * 4 + rd_c] = v;
+            __syncwarp();
           }
         }
       } else {
@@ -703,24 +683,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         float4* dst = reinterpret_cast<float4*>(a.o_part) +
                       ((size_t)(sg.slot * (2 * kBM / 32) + i * (kBM / 32) + q) * (D / 4)) * 32 + lane;
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = 0; c < kHalfD / 32; ++c) {
           uint32_t uu[32];
           tmem_ld32(o_addr + c * 32, uu);
           if (write) {
 #pragma unroll
             for (int v = 0; v < 8; ++v)
-              dst[(size_t)(c * 8 + v) * 32] =
+              dst[(size_t)((hf * kHalfD + c * 32) / 4 + v) * 32] =
                   make_float4(__uint_as_float(uu[4 * v]) * inv, __uint_as_float(uu[4 * v + 1]) * inv,
                               __uint_as_float(uu[4 * v + 2]) * inv, __uint_as_float(uu[4 * v + 3]) * inv);
           }
         }
       }
-      const float lse2 = l_run > 0.f ? m_run + __log2f(l_run) : -CUDART_INF_F;
-      if (sg.complete) {
-        if (write && a.lse) a.lse[(size_t)tt * a.Hq + h] = lse2 * 0.69314718055994531f;
-      } else {
-        // rows outside the problem merge to nothing
-        a.l_part[(size_t)sg.slot * 2 * kBM + i * kBM + r] = write ? lse2 : -CUDART_INF_F;
+      const size_t prow = (size_t)sg.slot * 2 * kBM + i * kBM + r;  // partial row of this thread
+      if (hf == 0) {
+        const float lse2 = l_row > 0.f ? m_run + __log2f(l_row) : -CUDART_INF_F;
+        if (write) {
+          if (sg.complete) {
+            if (a.lse) a.lse[(size_t)tt * a.Hq + h] = lse2 * 0.69314718055994531f;
+          } else {
+            a.l_part[prow] = lse2;
+          }
+        } else if (!sg.complete && ok) {
+          a.l_part[prow] = -CUDART_INF_F;  // rows outside the problem merge to nothing
+        }
       }
       J += sg.n;
     }

@@ -2,18 +2,20 @@
 
 A model of the roles in attn_tc.cu, each a sequence of barrier operations per
 segment of n key tiles:
-  * producer: wait q_empty of the previous segment, two arrivals on q_full
-    (expect-tx and the published descriptor), then the K of tile 0 and per
-    key tile j the K of tile j + 1 ahead of the V of tile j, each after a wait
-    on its ring stage's empty barrier (K and V rings of NK and NV stages);
-  * MMA warp: wait q_full, k_full, commit s_full of both tiles and k_empty;
-    per key tile wait v_full and p_full of each tile, commit o_full after the
-    last PV, v_empty after the tile's last PV, k_empty after the next tile's
-    last S MMA, and q_empty after the segment's last S MMA (the rule under
-    test);
-  * softmax threads (two per tile here, standing for the 128 rows that
-    p_full counts, one thread per row): wait q_full, per key tile wait
-    s_full and arrive on p_full; wait o_full before the epilogue.
+  * producer: the first segment's leading key tiles first (into stages not
+    used before), then per segment: wait q_empty of the previous segment, two
+    arrivals on q_full (expect-tx and the published descriptor), and per key
+    tile its K and V into ring stage JJ % NS after a wait on that stage's
+    kv_empty;
+  * MMA warp: wait q_full, k_full, commit s_full of both tiles; per key tile
+    wait v_full and p_full of each tile, commit o_full after the last PV,
+    kv_empty after the tile's last PV, and q_empty after the segment's last S
+    MMA (the rule under test);
+  * softmax threads (two per tile here, standing for the 256 threads of a
+    tile group: two per row, one per half of its score columns): wait q_full
+    and agree on it at the group barrier, per key tile wait s_full, meet the
+    other half of the row at the pair barrier and arrive on p_full; wait
+    o_full and meet at the group barrier before the epilogue.
 MMA commits and TMA completions are modelled as immediate (one possible
 timing).  A wait follows the hardware rule for parity waits (it passes when
 the barrier's completed-phase count has the other parity), and the checker
@@ -27,7 +29,7 @@ import random
 
 import pytest
 
-NK, NV = 3, 2  # K and V ring stages at d = 128
+NS = 2  # K/V ring stages at d = 128
 
 
 class Bar:
@@ -35,51 +37,29 @@ class Bar:
         self.count, self.pending, self.phase = count, 0, 0
 
 
-def _producer_order(n, first):
-    """(kind, j) loads of one segment of n key tiles: K of tile 0, then for
-    each tile j the K of tile j + 1 ahead of the V of tile j.  `first` drops
-    the tiles already loaded before the segment (counts of K and of V)."""
-    dk, dv = first
-    out = [] if dk > 0 else [("k", 0)]
-    for j in range(n):
-        if j + 1 < n and j + 1 >= dk:
-            out.append(("k", j + 1))
-        if j >= dv:
-            out.append(("v", j))
-    return out
-
-
 def _preload(segs, prefetch):
-    """Loads issued before anything else: the first segment's leading K and V
-    tiles, into stages not used before, in the same order as the main loop."""
-    if not prefetch:
-        return 0, 0, []
-    pk, pv = min(segs[0], NK), min(segs[0], NV)
-    out = [("k", 0)] if pk > 0 else []
-    for j in range(max(pk, pv)):
-        if j + 1 < pk:
-            out.append(("k", j + 1))
-        if j < pv:
-            out.append(("v", j))
-    return pk, pv, out
+    """Key tiles loaded before anything else: the first segment's leading
+    tiles, one per stage."""
+    return min(segs[0], NS) if prefetch else 0
 
 
 def producer(segs, prefetch=False):
-    pk, pv, pre = _preload(segs, prefetch)
-    for kind, j in pre:
-        yield ("arrive", f"{kind}_full{j % (NK if kind == 'k' else NV)}")
+    pre = _preload(segs, prefetch)
+    for j in range(pre):
+        yield ("arrive", f"k_full{j}")
+        yield ("arrive", f"v_full{j}")
     J = 0
     for k, n in enumerate(segs):
         if k > 0:
             yield ("wait", "q_empty", k - 1)
         yield ("arrive", "q_full")
         yield ("arrive", "q_full")
-        for kind, j in _producer_order(n, (pk, pv) if k == 0 else (0, 0)):
+        for j in range(pre if k == 0 else 0, n):
             JJ = J + j
-            ns = NK if kind == "k" else NV
-            if JJ >= ns:
-                yield ("wait", f"{kind}_empty{JJ % ns}", JJ // ns - 1)
-            yield ("arrive", f"{kind}_full{JJ % ns}")
+            if JJ >= NS:
+                yield ("wait", f"kv_empty{JJ % NS}", JJ // NS - 1)
+            yield ("arrive", f"k_full{JJ % NS}")
+            yield ("arrive", f"v_full{JJ % NS}")
         J += n
 
 
@@ -87,28 +67,26 @@ def mma(segs, early_release):
     J = 0
     for k, n in enumerate(segs):
         yield ("wait", "q_full", k)
-        yield ("wait", f"k_full{J % NK}", J // NK)
+        yield ("wait", f"k_full{J % NS}", J // NS)
         yield ("arrive", "s_full0")
         yield ("arrive", "s_full1")
-        yield ("arrive", f"k_empty{J % NK}")
         if early_release and n == 1:
             yield ("arrive", "q_empty")  # the earlier rule: released before any softmax acknowledgement
         for j in range(n):
             JJ = J + j
-            yield ("wait", f"v_full{JJ % NV}", JJ // NV)
+            yield ("wait", f"v_full{JJ % NS}", JJ // NS)
             yield ("wait", "p_full0", JJ)
             if j == n - 1:
                 yield ("arrive", "o_full0")
             if j + 1 < n:
-                yield ("wait", f"k_full{(JJ + 1) % NK}", (JJ + 1) // NK)
+                yield ("wait", f"k_full{(JJ + 1) % NS}", (JJ + 1) // NS)
                 yield ("arrive", "s_full0")
             yield ("wait", "p_full1", JJ)
-            yield ("arrive", f"v_empty{JJ % NV}")
+            yield ("arrive", f"kv_empty{JJ % NS}")
             if j == n - 1:
                 yield ("arrive", "o_full1")
             if j + 1 < n:
                 yield ("arrive", "s_full1")
-                yield ("arrive", f"k_empty{(JJ + 1) % NK}")
                 if j + 2 == n:
                     yield ("arrive", "q_empty")
             elif n == 1 and not early_release:
@@ -117,15 +95,18 @@ def mma(segs, early_release):
 
 
 def softmax(segs, i):
-    # one thread per row: no barrier among the softmax threads
     J = 0
     for k, n in enumerate(segs):
         yield ("wait", "q_full", k)
+        yield ("sync", f"qa{i}")  # the group agrees on the wait before reading the description
         for j in range(n):
             JJ = J + j
             yield ("wait", f"s_full{i}", JJ)
+            yield ("sync", f"pair{i}")  # the two halves of a row exchange their maxima
             yield ("arrive", f"p_full{i}")
         yield ("wait", f"o_full{i}", k)
+        yield ("sync", f"ep{i}")
+        yield ("sync", f"eq{i}")
         J += n
 
 
@@ -136,10 +117,8 @@ def run(segs, early_release, seed, prefetch=False):
     """Returns None when every role finishes cleanly, else a description."""
     bars = {"q_full": Bar(2), "q_empty": Bar(1), "s_full0": Bar(1), "s_full1": Bar(1),
             "p_full0": Bar(SOFT), "p_full1": Bar(SOFT), "o_full0": Bar(1), "o_full1": Bar(1)}
-    for s in range(NK):
-        bars[f"k_full{s}"], bars[f"k_empty{s}"] = Bar(1), Bar(1)
-    for s in range(NV):
-        bars[f"v_full{s}"], bars[f"v_empty{s}"] = Bar(1), Bar(1)
+    for s in range(NS):
+        bars[f"k_full{s}"], bars[f"v_full{s}"], bars[f"kv_empty{s}"] = Bar(1), Bar(1), Bar(1)
     threads = {"producer": producer(segs, prefetch), "mma": mma(segs, early_release)}
     for i in range(2):
         for t in range(SOFT):
@@ -316,11 +295,11 @@ def test_lse_protocol_has_no_stall_or_aliased_wait(tiles, nk):
 
 
 def a_producer(segs, drain, prefetch=True):
-    pk, pv, pre = _preload(segs, prefetch)
-    armed = {"k": 0, "v": 0}
-    for kind, j in pre:
-        yield ("tma", f"{kind}_full{j % (NK if kind == 'k' else NV)}")
-        armed[kind] = j + 1
+    pre = _preload(segs, prefetch)
+    for j in range(pre):
+        yield ("tma", f"k_full{j}")
+        yield ("tma", f"v_full{j}")
+    armed = pre  # key tiles whose K and V loads were issued
     J, q_armed, ok = 0, 0, True
     for k, n in enumerate(segs):
         if not ok:
@@ -332,23 +311,23 @@ def a_producer(segs, drain, prefetch=True):
         yield ("tma", "q_full")
         q_armed += 1
         yield ("arrive", "q_full")  # the published segment description
-        for kind, j in _producer_order(n, (pk, pv) if k == 0 else (0, 0)):
+        for j in range(pre if k == 0 else 0, n):
             JJ = J + j
-            ns = NK if kind == "k" else NV
-            if JJ >= ns:
-                ok = yield ("wait", f"{kind}_empty{JJ % ns}", JJ // ns - 1, True)
+            if JJ >= NS:
+                ok = yield ("wait", f"kv_empty{JJ % NS}", JJ // NS - 1, True)
                 if not ok:
                     break
-            yield ("tma", f"{kind}_full{JJ % ns}")
-            armed[kind] = JJ + 1
+            yield ("tma", f"k_full{JJ % NS}")
+            yield ("tma", f"v_full{JJ % NS}")
+            armed = JJ + 1
         J += n
     if drain:
         # the last phase of every stage it armed, and of the Q buffer, ignoring the flag
-        for kind, ns in (("k", NK), ("v", NV)):
-            for s in range(ns):
-                uses = (armed[kind] - s + ns - 1) // ns if armed[kind] > s else 0
-                if uses:
-                    yield ("wait", f"{kind}_full{s}", uses - 1, False)
+        for s in range(NS):
+            uses = (armed - s + NS - 1) // NS if armed > s else 0
+            if uses:
+                yield ("wait", f"k_full{s}", uses - 1, False)
+                yield ("wait", f"v_full{s}", uses - 1, False)
         if q_armed:
             yield ("wait", "q_full", q_armed - 1, False)
     yield ("final",)
@@ -361,17 +340,16 @@ def a_mma(segs, drain):
             break
         ok = yield ("wait", "q_full", k, True)
         if ok:
-            ok = yield ("wait", f"k_full{J % NK}", J // NK, True)
+            ok = yield ("wait", f"k_full{J % NS}", J // NS, True)
             if ok:
                 for i in range(2):
                     yield ("mma",)
                     yield ("commit", f"s_full{i}")
-                yield ("commit", f"k_empty{J % NK}")
         for j in range(n):
             if not ok:
                 break
             JJ = J + j
-            ok = yield ("wait", f"v_full{JJ % NV}", JJ // NV, True)
+            ok = yield ("wait", f"v_full{JJ % NS}", JJ // NS, True)
             if ok:
                 ok = yield ("wait", "p_full0", JJ, True)
             if not ok:
@@ -380,7 +358,7 @@ def a_mma(segs, drain):
             if j == n - 1:
                 yield ("commit", "o_full0")
             if j + 1 < n:
-                ok = yield ("wait", f"k_full{(JJ + 1) % NK}", (JJ + 1) // NK, True)
+                ok = yield ("wait", f"k_full{(JJ + 1) % NS}", (JJ + 1) // NS, True)
                 if not ok:
                     break
                 yield ("mma",)
@@ -389,13 +367,12 @@ def a_mma(segs, drain):
             if not ok:
                 break
             yield ("mma",)
-            yield ("commit", f"v_empty{JJ % NV}")
+            yield ("commit", f"kv_empty{JJ % NS}")
             if j == n - 1:
                 yield ("commit", "o_full1")
             if j + 1 < n:
                 yield ("mma",)
                 yield ("commit", "s_full1")
-                yield ("commit", f"k_empty{(JJ + 1) % NK}")
                 if j + 2 == n:
                     yield ("commit", "q_empty")
             elif n == 1:
@@ -408,20 +385,24 @@ def a_mma(segs, drain):
 
 
 def a_softmax(segs, i):
-    # a failed wait ends the thread's work (its warp leaves together)
+    # the tile group agrees on the q_full wait before reading the segment; a
+    # failed wait inside a segment does not leave it (the group must meet the
+    # same pair and group barriers), the group leaves after its epilogue barrier
     J, ok = 0, True
     for k, n in enumerate(segs):
-        ok = yield ("wait", "q_full", k, True)
+        w = yield ("wait", "q_full", k, True)
+        ok = yield ("syncand", f"qa{i}", w)
         if not ok:
             break
         for j in range(n):
-            ok = yield ("wait", f"s_full{i}", J + j, True)
-            if not ok:
-                break
+            w = yield ("wait", f"s_full{i}", J + j, True)
+            ok = ok and w
+            yield ("sync", f"pair{i}")
             yield ("arrive", f"p_full{i}")
-        if not ok:
-            break
-        ok = yield ("wait", f"o_full{i}", k, True)
+        if ok:
+            ok = yield ("wait", f"o_full{i}", k, True)
+        ok = yield ("syncand", f"ep{i}", ok)
+        yield ("sync", f"eq{i}")
         if not ok:
             break
         J += n
@@ -514,10 +495,8 @@ def _async_run(threads, bars, group_of, seed, p_timeout):
 def run_abort(segs, drain, seed, p_timeout=0.02):
     bars = {"q_full": Bar(2), "q_empty": Bar(1), "s_full0": Bar(1), "s_full1": Bar(1), "drain": Bar(1),
             "p_full0": Bar(SOFT), "p_full1": Bar(SOFT), "o_full0": Bar(1), "o_full1": Bar(1)}
-    for s in range(NK):
-        bars[f"k_full{s}"], bars[f"k_empty{s}"] = Bar(1), Bar(1)
-    for s in range(NV):
-        bars[f"v_full{s}"], bars[f"v_empty{s}"] = Bar(1), Bar(1)
+    for s in range(NS):
+        bars[f"k_full{s}"], bars[f"v_full{s}"], bars[f"kv_empty{s}"] = Bar(1), Bar(1), Bar(1)
     threads = {"producer": a_producer(segs, drain), "mma": a_mma(segs, drain)}
     for i in range(2):
         for t in range(SOFT):
