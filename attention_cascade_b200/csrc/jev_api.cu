@@ -707,8 +707,10 @@ jev_status jev_candidate_readout_normalized(const jev_readout_desc* d, const voi
   if (row_lse && ((uintptr_t)row_lse & 3)) return fail(JEV_ERR_INVALID_ARG, "row_lse misaligned");
   ReadoutArgs a{hidden, lm_head, set_offsets, cand_offsets, pair_row, pair_tok, logprob, choice, score,
                 d->n_sets, d->n_cands, d->n_pairs, d->R, d->H, d->V, row_lse};
-  const jev_status st = run("readout", (cudaStream_t)stream, [&] { return launch_readout(a, d->dtype, (cudaStream_t)stream); });
-  if (st == JEV_OK && d->n_cands > 0) g_launches++;  // candidate scores and set softmax: two kernels
+  int n_kernels = 0;
+  const jev_status st =
+      run("readout", (cudaStream_t)stream, [&] { return launch_readout(a, d->dtype, (cudaStream_t)stream, &n_kernels); });
+  if (st == JEV_OK && n_kernels > 1) g_launches += n_kernels - 1;  // run() counted one
   return st;
 }
 

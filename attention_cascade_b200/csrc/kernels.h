@@ -100,7 +100,8 @@ struct ReadoutArgs {
   int n_sets, n_cands, n_pairs, R, H, V;
   const float* row_lse;  // [R] or null: each pair's term becomes logit - row_lse[row]
 };
-cudaError_t launch_readout(const ReadoutArgs& a, jev_dtype dt, cudaStream_t s);
+// *n_kernels: how many kernels the call launched (1 or 2)
+cudaError_t launch_readout(const ReadoutArgs& a, jev_dtype dt, cudaStream_t s, int* n_kernels);
 
 // Full-vocabulary log-sum-exp of bf16 hidden rows (vocab_lse.cu).
 struct VocabLseArgs {

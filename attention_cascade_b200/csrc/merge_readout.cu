@@ -342,7 +342,8 @@ cudaError_t launch_merge(const MergeArgs& a, jev_dtype dt, cudaStream_t s) {
   return cudaGetLastError();
 }
 
-cudaError_t launch_readout(const ReadoutArgs& a, jev_dtype dt, cudaStream_t s) {
+cudaError_t launch_readout(const ReadoutArgs& a, jev_dtype dt, cudaStream_t s, int* n_kernels) {
+  *n_kernels = 0;
   if (a.n_sets == 0) return cudaSuccess;
   if (a.n_cands > 0) {
     if (a.cand_offsets) {
@@ -360,6 +361,7 @@ cudaError_t launch_readout(const ReadoutArgs& a, jev_dtype dt, cudaStream_t s) {
         else if (nu <= 12) readout_set_fused_kernel<12><<<g, b, 0, s>>>(a);
         else if (nu <= 14) readout_set_fused_kernel<14><<<g, b, 0, s>>>(a);
         else readout_set_fused_kernel<16><<<g, b, 0, s>>>(a);
+        *n_kernels = 1;
         return cudaGetLastError();
       }
       if (dt == JEV_BF16) readout_cand_kernel<__nv_bfloat16><<<blocks, kCandWarps * 32, 0, s>>>(a);
@@ -367,6 +369,7 @@ cudaError_t launch_readout(const ReadoutArgs& a, jev_dtype dt, cudaStream_t s) {
     }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
+    *n_kernels = 1;
   }
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute pdl[1];
@@ -377,6 +380,7 @@ cudaError_t launch_readout(const ReadoutArgs& a, jev_dtype dt, cudaStream_t s) {
   cfg.stream = s;
   cfg.attrs = pdl;
   cfg.numAttrs = 1;
+  ++*n_kernels;
   return cudaLaunchKernelEx(&cfg, readout_set_kernel, a);
 }
 

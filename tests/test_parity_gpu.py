@@ -153,7 +153,9 @@ def test_readout_many_one_pair_candidates(jev, H):
     toks = rng.integers(0, V, int(so[-1])).astype(np.int32)
     toks[so[7] + 2] = -3
     ref = oracle.candidate_readout(hidden, W, so, toks)
+    n0 = jev.jev_launch_count()
     lp, ch = run_readout(jev, hidden, dev(W), so, toks)
+    assert jev.jev_launch_count() - n0 == (1 if H <= 4096 else 2)  # fused, or scores then set softmax
     check_readout(lp, ch, ref, synth.BF16, f"one-pair readout H={H}")
     assert ch[7] == -1 and ch[11] == -1 and np.all(np.isnan(lp[so[7]:so[8]]))
     assert ch[3] == 0 and lp[so[3]] == 0.0
