@@ -913,10 +913,13 @@ class Measured:
     def step(self, cp, s):
         # the readout's inputs (final hidden rows, option ids) do not depend on
         # this attention layer, so it runs on a second stream, forked and
-        # joined inside the step
+        # joined inside the step.  It is enqueued after the attention kernels
+        # so that their persistent CTAs take the SMs first and the readout's
+        # blocks fill SMs as the attention's tail frees them (measured about
+        # 1% faster per step than launching the readout first).
         self.side.wait_stream(s)
-        self.wl.readout(cp, self.side)
         self.wl.attn(cp, s)
+        self.wl.readout(cp, self.side)
         s.wait_stream(self.side)
 
     def capture(self, profiled: bool):
@@ -1076,7 +1079,7 @@ def jev_arm(args, wl_name):
                          "> 2x L2)",
                    "timing": "CUDA graph replay per step, CUDA events on the launching stream; per-kernel times "
                              "from a second replay of the K steps with event nodes around each kernel",
-                   "streams": "readout on a second stream, forked and joined inside each step"},
+                   "streams": "readout on a second stream, forked before and enqueued after the attention kernels, joined inside each step"},
         "branches_per_s": job_rate(world, wl.B, args.steps, ms),
         "clocks": m.clk,
         "e2e": {"value": job_rate(world, T, args.steps, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
