@@ -534,6 +534,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           last = TREE ? t : inf.last;
         }
       }
+      // tree: the warp's first and last computed rows (tokens), for the
+      // whole-tile test of the suffix window
+      int w_lo = 0, w_hi = -1;
+      if (TREE) {
+        w_lo = warp_min_i(t >= 0 ? t : INT_MAX);
+        w_hi = warp_max_i(t);
+      }
       float m_run = -CUDART_INF_F, l_run = 0.f;
       // A wait that fails (a timeout somewhere in the CTA) does not leave the
       // loop: the thread runs the remaining tiles on whatever TMEM holds, so
@@ -569,12 +576,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           } else {
             // tree row t: key k is on its root path when k <= t and t lies in the
-            // packed tokens of k's node's subtree (read here, where needed)
+            // packed tokens of k's node's subtree.  The warp's rows share the
+            // tile's 64 keys: lane l reads the subtree ends of keys l and l + 32
+            // once, and the mask is skipped when every key is at or before the
+            // warp's first row and every subtree holds its last row.
+            const int e_a = kb + lane < a.key_rows ? __ldg(a.key_end + kb + lane) : -1;
+            const int e_b = kb + 32 + lane < a.key_rows ? __ldg(a.key_end + kb + 32 + lane) : -1;
+            const bool whole = kb + kHalfCols - 1 <= w_lo && warp_min_i(min(e_a, e_b)) > w_hi;
+            if (!whole) {
 #pragma unroll
-            for (int c = 0; c < kHalfCols; ++c) {
-              const int kk = kb + c;
-              const int e = kk < a.key_rows ? __ldg(a.key_end + kk) : -1;
-              if (!(kk <= t && t < e)) xs[c] = kNegInf;
+              for (int c = 0; c < kHalfCols; ++c) {
+                const int e = __shfl_sync(0xffffffffu, c < 32 ? e_a : e_b, c & 31);
+                if (!(kb + c <= t && t < e)) xs[c] = kNegInf;
+              }
             }
           }
         }
