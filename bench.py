@@ -1082,6 +1082,18 @@ def jev_arm(args, wl_name):
             e2e_step(stream)
         f1.record(stream)
     torch.cuda.synchronize()
+    # the pipelined steps computed what a step computes alone: the last step's
+    # results, read back, against one more step run by itself from a slot
+    # (every kernel on this path is deterministic)
+    last = h_out.clone()
+    with torch.cuda.stream(stream):
+        cp = dict(cp_static)
+        cp.update(d_ins[0])
+        m.step(cp, stream)
+        h_out.copy_(d_out, non_blocking=True)
+    torch.cuda.synchronize()
+    if not torch.equal(last, h_out):
+        raise SystemExit("bench.py: end-to-end results differ from a step run alone")
     e2e_ms = m.max_over_ranks(f0.elapsed_time(f1))
     h2d = h_packs[0].numel()
     d2h = h_out.numel()
