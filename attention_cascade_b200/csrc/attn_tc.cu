@@ -57,10 +57,13 @@ constexpr int kProducerWarp = kSoftWarps;
 constexpr int kMmaWarp = kSoftWarps + 1;
 constexpr float kLazy = 8.0f;  // log2 headroom before the running max moves
 // Share of softmax exponentials computed on the FMA pipe (every kPolyEvery-th
-// score pair; 0 = none).  Measured on B200 at the wide workload: 0 is fastest
-// (the softmax is issue-bound, not MUFU-bound), so it is off by default.
+// score pair, as one packed f32x2 polynomial; 0 = none).  Measured on B200,
+// attention call alone: every 8th pair (12.5%) is fastest, about 1.8% below
+// none at the wide workload; every 2nd, 4th, 6th or 12th pair is slower than
+// none (the softmax is mostly bound by issue and latency, and MUFU is about
+// half busy).
 #ifndef JEV_POLY_EVERY
-#define JEV_POLY_EVERY 0
+#define JEV_POLY_EVERY 8
 #endif
 constexpr int kPolyEvery = JEV_POLY_EVERY;
 
@@ -619,12 +622,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < kHalfCols / 2; ++kk) {
           const uint64_t x2 = f2_fma(((uint64_t)xs[2 * kk + 1] << 32) | xs[2 * kk], sc2, nb2);
-          const float x0 = f2_lo(x2), x1 = f2_hi(x2);
           const bool fma_pipe = kPolyEvery > 0 && (kk % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1;
-          const float p0 = fma_pipe ? exp2_fma(x0) : ex2(x0);
-          const float p1 = fma_pipe ? exp2_fma(x1) : ex2(x1);
-          ps2[kk & 3] = f2_add(ps2[kk & 3], f2_pack(p0, p1));
-          xs[kk] = pack_bf16(p0, p1);
+          const uint64_t p2 = fma_pipe ? exp2_fma2(x2) : f2_pack(ex2(f2_lo(x2)), ex2(f2_hi(x2)));
+          ps2[kk & 3] = f2_add(ps2[kk & 3], p2);
+          xs[kk] = pack_bf16(f2_lo(p2), f2_hi(p2));
         }
         tmem_st32(p_addr, *reinterpret_cast<const uint32_t(*)[32]>(&xs[0]));
         const uint64_t s01 = f2_add(ps2[0], ps2[1]), s23 = f2_add(ps2[2], ps2[3]);
@@ -825,9 +826,17 @@ __global__ void __launch_bounds__(256) tc_fixup_kernel(const AttnArgs a) {
     a.lse[(size_t)t * a.Hq + h] = wsum > 0.f ? (mx + log2f(wsum)) * 0.69314718055994531f : -CUDART_INF_F;
 }
 
+// The softmax's FMA-pipe 2^x as the kernel runs it: packed pairs (the last
+// element of an odd count through the scalar form, the same arithmetic).
 __global__ void exp2_selftest_kernel(const float* x, float* y, int n) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i < n) y[i] = exp2_fma(x[i]);
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i + 1 < n) {
+    const uint64_t p2 = exp2_fma2(f2_pack(x[i], x[i + 1]));
+    y[i] = f2_lo(p2);
+    y[i + 1] = f2_hi(p2);
+  } else if (i < n) {
+    y[i] = exp2_fma(x[i]);
+  }
 }
 
 // ---------------------------------------------------------------- host side
@@ -909,7 +918,7 @@ cudaError_t launch_dt(const AttnArgs& a, cudaStream_t s) {
 
 cudaError_t launch_exp2_selftest(const float* x, float* y, int n, cudaStream_t s) {
   if (n <= 0) return cudaSuccess;
-  exp2_selftest_kernel<<<(n + 255) / 256, 256, 0, s>>>(x, y, n);
+  exp2_selftest_kernel<<<((n + 1) / 2 + 255) / 256, 256, 0, s>>>(x, y, n);
   return cudaGetLastError();
 }
 

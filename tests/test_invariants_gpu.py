@@ -149,8 +149,10 @@ def test_tree_status_flags_malformed_trees_without_faulting(jev):
 
 
 def test_fma_pipe_exp2_against_cuda_exp2(jev):
-    """The software 2^x used for a share of the softmax exponentials stays
-    within its stated bound of CUDA's exp2 over the range softmax feeds it."""
+    """The software 2^x used for a share of the softmax exponentials (the
+    packed-pair form the attention kernel runs; an odd last element through
+    the scalar form) stays within its stated bound of CUDA's exp2 over the
+    range softmax feeds it."""
     x = torch.linspace(-125.0, 8.5, 1_000_003, device="cuda", dtype=torch.float32)
     y = jev.jev_selftest_exp2(x)
     ref = torch.exp2(x.double())
