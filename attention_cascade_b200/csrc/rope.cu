@@ -12,21 +12,7 @@
 namespace jev {
 namespace {
 
-// 8 consecutive elements of T as fp32 (one 16-byte load for bf16, two for fp32).
-__device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&f)[8]) {
-  const uint4 v = *reinterpret_cast<const uint4*>(p);
-  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const float2 x = __bfloat1622float2(h[k]);
-    f[2 * k] = x.x;
-    f[2 * k + 1] = x.y;
-  }
-}
-__device__ __forceinline__ void load8(const float* p, float (&f)[8]) {
-  const float4 a = reinterpret_cast<const float4*>(p)[0], b = reinterpret_cast<const float4*>(p)[1];
-  f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w; f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
-}
+// 8 fp32 values stored as 8 consecutive elements of T (one 16-byte store for bf16, two for fp32).
 __device__ __forceinline__ void store8(__nv_bfloat16* p, const float (&f)[8]) {
   uint4 v;
   uint32_t* w = reinterpret_cast<uint32_t*>(&v);
@@ -60,8 +46,8 @@ __device__ __forceinline__ void unpack8(const F8& v, float (&f)[8]) {
   f[0] = v.a.x; f[1] = v.a.y; f[2] = v.a.z; f[3] = v.a.w; f[4] = v.b.x; f[5] = v.b.y; f[6] = v.b.z; f[7] = v.b.w;
 }
 
-constexpr int kTokPerBlock = 8;  // one warp per token
-constexpr int kSmemOffs = 4096;  // segment offsets searched in shared memory up to this many
+constexpr int kPackWarps = 4;  // warps per block
+constexpr int kChunkIt = 2;    // head iterations per warp (8 heads at d = 128, 16 at d = 64)
 
 // Tree plan of node m, computed by the warp of each of m's tokens (nodes in
 // depth-first preorder, packed tokens in node order).  The keys a token of m
@@ -122,17 +108,58 @@ __device__ NodePlan plan_node(const RopePackArgs& a, int m, int lane) {
   return r;
 }
 
-// One warp per packed token: find its segment and position, form cos/sin of
-// its angles (double angle, rounded once to float), then rotate all its query
-// and key heads, 8 pair indices per lane per head with 16-byte accesses.
+// Segment of token t: the largest s < n with offs[s] <= t, by a 32-ary
+// search of the warp over offs in global memory (one load per lane and round;
+// two rounds up to 1024 segments).  Malformed offsets give some s < n.
+__device__ __forceinline__ int warp_upper_segment(const int32_t* offs, int n, int t, int lane) {
+  int lo = 0;
+  while (n > 32) {
+    const int step = (n + 31) / 32;
+    const int idx = lo + lane * step;
+    const unsigned b = __ballot_sync(0xffffffffu, lane * step < n && offs[idx] <= t);
+    const int k = b ? 31 - __clz((int)b) : 0;
+    lo += k * step;
+    n = min(step, n - k * step);
+  }
+  const unsigned b = __ballot_sync(0xffffffffu, lane < n && offs[lo + lane] <= t);
+  return lo + (b ? 31 - __clz((int)b) : 0);
+}
+
+// kv group and slot (the query head's place among its group's heads, in head
+// order) of query head h
+__device__ __forceinline__ void head_slot(const RopePackArgs& a, int G, int h, int& g, int& slot) {
+  if (!a.head_map) {
+    g = h / G;
+    slot = h - g * G;
+    return;
+  }
+  g = a.head_map[h];
+  if (g < 0 || g >= a.Hkv) g = 0;  // flagged by block 0
+  slot = 0;
+  for (int h2 = 0; h2 < h; ++h2) {
+    int g2 = a.head_map[h2];
+    if (g2 < 0 || g2 >= a.Hkv) g2 = 0;
+    slot += g2 == g;
+  }
+  slot = min(slot, G - 1);  // an uneven map is flagged by block 0
+}
+
+// Work item = (token t, chunk c of its Hq + Hkv heads): a warp loads its
+// chunk's heads first, then locates the token (segment, position; for a tree
+// its node plan, for a generation step its cache row), forms the cosines and
+// sines of the token's angles (double angle, rounded once to float) and
+// rotates its heads, 8 pair indices per lane and head with 16-byte accesses.
+// The chunks of a token are consecutive warps; the token's info (and its
+// node plan or cache bookkeeping) is written by the warp of chunk 0.  No
+// block-wide barrier outside block 0, which also checks the inputs and
+// writes the inverse head table.
 template <typename T>
-__global__ void __launch_bounds__(256) rope_pack_kernel(RopePackArgs a) {
+__global__ void __launch_bounds__(kPackWarps * 32) rope_pack_kernel(RopePackArgs a) {
   const int half = a.d >> 1;
   const int G = a.Hq / a.Hkv;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  __shared__ float cs[kTokPerBlock][128], sn[kTokPerBlock][128];
-  __shared__ int s_slot[256], s_grp[256];
-  __shared__ int s_offs[kSmemOffs];
+  __shared__ float cs[kPackWarps][64], sn[kPackWarps][64];
+  __shared__ int s_grp[256];
   // The previous kernels of the stream (which may write q, k or the prefix
   // cache, or read this workspace) must be done before anything is read or
   // written.  Only then may the attention kernel begin launching: it starts
@@ -140,21 +167,22 @@ __global__ void __launch_bounds__(256) rope_pack_kernel(RopePackArgs a) {
   // kernel has to be complete when it launches.
   pdl_wait();
   if (threadIdx.x == 0) pdl_trigger();
-  // Every head this lane rotates is loaded first, before any table work, so
-  // the token's one memory round trip overlaps the segment search and the
-  // sines and cosines; raw 16-byte vectors.
-  const int t = blockIdx.x * kTokPerBlock + warp;
-  const int lanes_per_head = half / 8;          // 8 (d = 128) or 4 (d = 64)
+  const int lanes_per_head = half / 8;           // 8 (d = 128) or 4 (d = 64)
   const int heads_per_it = 32 / lanes_per_head;  // 4 or 8
-  const int i0 = (lane % lanes_per_head) * 8, hsub = lane / lanes_per_head;
+  const int per_warp = kChunkIt * heads_per_it;
   const int H = a.Hq + a.Hkv;
-  constexpr int kMaxIt = 8;  // covers Hq + Hkv <= 32 at d = 128 and <= 64 at d = 64
+  const int n_chunks = (H + per_warp - 1) / per_warp;
+  const long long wid = (long long)blockIdx.x * kPackWarps + warp;
+  const int t = (int)min(wid / n_chunks, (long long)a.T);
+  const int chunk = (int)(wid - (long long)t * n_chunks);
+  const int h_base = chunk * per_warp;
+  const int i0 = (lane % lanes_per_head) * 8, hsub = lane / lanes_per_head;
   using Raw = typename RawVec<T>::type;
-  Raw r0[kMaxIt], r1[kMaxIt];
+  Raw r0[kChunkIt], r1[kChunkIt];
   if (t < a.T) {
 #pragma unroll
-    for (int it = 0; it < kMaxIt; ++it) {
-      const int hh = hsub + it * heads_per_it;
+    for (int it = 0; it < kChunkIt; ++it) {
+      const int hh = h_base + it * heads_per_it + hsub;
       if (hh < H) {
         const T* src = hh < a.Hq ? reinterpret_cast<const T*>(a.q) + ((size_t)t * a.Hq + hh) * a.d
                                  : reinterpret_cast<const T*>(a.k) + ((size_t)t * a.Hkv + (hh - a.Hq)) * a.d;
@@ -163,79 +191,69 @@ __global__ void __launch_bounds__(256) rope_pack_kernel(RopePackArgs a) {
       }
     }
   }
-  const bool offs_in_smem = a.n_segs + 1 <= kSmemOffs;
-  if (offs_in_smem)
-    for (int i = threadIdx.x; i <= a.n_segs; i += blockDim.x) s_offs[i] = a.offs[i];
-  // group and slot of every query head
-  for (int h = threadIdx.x; h < a.Hq; h += blockDim.x) {
-    int g = a.head_map ? a.head_map[h] : h / G;
-    if (g < 0 || g >= a.Hkv) {
-      if (blockIdx.x == 0) raise_flag(a.status, JEV_DEV_BAD_HEAD_MAP);
-      g = 0;
-    }
-    s_grp[h] = g;
-  }
-  // block 0 owns the inverse table: identity first, so every entry stays a
-  // valid head index even when a malformed map leaves a slot unclaimed
-  if (blockIdx.x == 0)
-    for (int h = threadIdx.x; h < a.Hq; h += blockDim.x) a.hinv[h] = h;
-  __syncthreads();
-  for (int h = threadIdx.x; h < a.Hq; h += blockDim.x) {
-    int g = s_grp[h], slot = 0;
-    for (int h2 = 0; h2 < h; ++h2) slot += (s_grp[h2] == g);
-    if (slot >= G) {
-      if (blockIdx.x == 0) raise_flag(a.status, JEV_DEV_BAD_HEAD_MAP);
-      slot = G - 1;
-    }
-    s_slot[h] = slot;
-    if (blockIdx.x == 0) a.hinv[g * G + slot] = h;
-  }
-  if (a.parent && blockIdx.x == 0 && threadIdx.x == 0 &&
-      (a.parent[0] != -1 || a.offs[0] != 0 || (a.n_segs > 0 && a.offs[1] != 0)))
-    raise_flag(a.status, JEV_DEV_BAD_TREE);  // node 0 is the root: no parent, no packed tokens
   if (blockIdx.x == 0) {
+    // input checks and the inverse head table: identity first, so that every
+    // entry stays a valid head index even when a malformed map leaves a slot
+    // unclaimed
+    for (int h = threadIdx.x; h < a.Hq; h += blockDim.x) {
+      int g = a.head_map ? a.head_map[h] : h / G;
+      if (g < 0 || g >= a.Hkv) {
+        raise_flag(a.status, JEV_DEV_BAD_HEAD_MAP);
+        g = 0;
+      }
+      s_grp[h] = g;
+      a.hinv[h] = h;
+    }
+    __syncthreads();
+    for (int h = threadIdx.x; h < a.Hq; h += blockDim.x) {
+      const int g = s_grp[h];
+      int slot = 0;
+      for (int h2 = 0; h2 < h; ++h2) slot += (s_grp[h2] == g);
+      if (slot >= G) {
+        raise_flag(a.status, JEV_DEV_BAD_HEAD_MAP);
+        slot = G - 1;
+      }
+      a.hinv[g * G + slot] = h;
+    }
+    if (a.parent && threadIdx.x == 0 && (a.parent[0] != -1 || a.offs[0] != 0 || (a.n_segs > 0 && a.offs[1] != 0)))
+      raise_flag(a.status, JEV_DEV_BAD_TREE);  // node 0 is the root: no parent, no packed tokens
     // offsets must start at 0, never decrease and end at T
     for (int i = threadIdx.x; i < a.n_segs; i += blockDim.x)
       if (a.offs[i + 1] < a.offs[i]) raise_flag(a.status, JEV_DEV_BAD_SEQLENS);
     if (threadIdx.x == 0 && (a.offs[0] != 0 || a.offs[a.n_segs] != a.T)) raise_flag(a.status, JEV_DEV_BAD_SEQLENS);
   }
-  __syncthreads();
   if (t >= a.T) return;
-  int seg = 0, start = 0, pos = 0, krow = t, kvalid = 1;
-  if (lane == 0) {
-    seg = upper_segment(offs_in_smem ? s_offs : a.offs, a.n_segs, t);
-    start = offs_in_smem ? s_offs[seg] : a.offs[seg];
-    if (start > t) start = t;
-    if (start < 0) start = 0;
-  }
+  const int seg = warp_upper_segment(a.offs, a.n_segs, t, lane);
+  int start = a.offs[seg];
+  if (start > t) start = t;
+  if (start < 0) start = 0;
+  int pos = 0, krow = t, kvalid = 1;
   if (a.parent) {
     // tree token: window from its top-level ancestor; as a key, its node's subtree end
-    seg = __shfl_sync(0xffffffffu, seg, 0);
-    const NodePlan np = plan_node(a, seg, lane);
-    if (lane == 0) {
-      if (np.start < 0) raise_flag(a.status, JEV_DEV_BAD_TREE);
-      pos = a.pos0[seg] + (t - start);
-      a.info[t] = TokInfo{max(np.start, 0), pos, np.start < 0 ? -1 : seg, np.end};
-      a.key_end[t] = np.start < 0 ? -1 : np.end;
+    pos = a.pos0[seg] + (t - start);
+    if (chunk == 0) {
+      const NodePlan np = plan_node(a, seg, lane);
+      if (lane == 0) {
+        if (np.start < 0) raise_flag(a.status, JEV_DEV_BAD_TREE);
+        a.info[t] = TokInfo{max(np.start, 0), pos, np.start < 0 ? -1 : seg, np.end};
+        a.key_end[t] = np.start < 0 ? -1 : np.end;
+      }
     }
-  } else if (lane == 0) {
-    if (a.cache_off) {
-      // new token j of branch seg: after the branch's cached tokens, in its cache rows
-      const int j = t - start, n_new = (offs_in_smem ? s_offs[seg + 1] : a.offs[seg + 1]) - start;
-      const int len = a.cache_len[seg], c0 = a.cache_off[seg], c1 = a.cache_off[seg + 1];
-      kvalid = len >= 0 && c0 >= 0 && c1 <= a.key_rows && (long long)c0 + len + n_new <= (long long)c1;
+  } else if (a.cache_off) {
+    // new token j of branch seg: after the branch's cached tokens, in its cache rows
+    const int j = t - start, n_new = a.offs[seg + 1] - start;
+    const int len = a.cache_len[seg], c0 = a.cache_off[seg], c1 = a.cache_off[seg + 1];
+    kvalid = len >= 0 && c0 >= 0 && c1 <= a.key_rows && (long long)c0 + len + n_new <= (long long)c1;
+    krow = kvalid ? c0 + len + j : 0;
+    pos = a.pos_offset + (kvalid ? len : 0) + j;
+    if (chunk == 0 && lane == 0) {
       if (!kvalid) raise_flag(a.status, JEV_DEV_BAD_CACHE);
-      krow = kvalid ? c0 + len + j : 0;
-      pos = a.pos_offset + (kvalid ? len : 0) + j;
       a.info[t] = TokInfo{max(c0, 0), pos, kvalid ? seg : -1, krow};
-    } else {
-      pos = a.pos_seq ? a.pos_offset + t : (a.pos0 ? a.pos0[seg] : a.pos_offset) + (t - start);
-      a.info[t] = TokInfo{start, pos, seg, t};
     }
+  } else {
+    pos = a.pos_seq ? a.pos_offset + t : (a.pos0 ? a.pos0[seg] : a.pos_offset) + (t - start);
+    if (chunk == 0 && lane == 0) a.info[t] = TokInfo{start, pos, seg, t};
   }
-  pos = __shfl_sync(0xffffffffu, pos, 0);
-  krow = __shfl_sync(0xffffffffu, krow, 0);
-  kvalid = __shfl_sync(0xffffffffu, kvalid, 0);
   for (int i = lane; i < half; i += 32) {
     // angle formed in double and reduced to [-pi, pi] in double (the error of
     // the reduction is ~1e-12 rad for positions up to 1e6), then one float sincos
@@ -255,12 +273,18 @@ __global__ void __launch_bounds__(256) rope_pack_kernel(RopePackArgs a) {
   }
   const size_t M = (size_t)a.T * G;
 #pragma unroll
-  for (int it = 0; it < kMaxIt; ++it) {
-    const int hh = hsub + it * heads_per_it;
+  for (int it = 0; it < kChunkIt; ++it) {
+    const int hh = h_base + it * heads_per_it + hsub;
     if (hh < H) {
       if (hh >= a.Hq && !kvalid) continue;  // a cache row outside the branch's rows is not written
-      T* dst = hh < a.Hq ? reinterpret_cast<T*>(a.q_rot) + ((size_t)s_grp[hh] * M + (size_t)t * G + s_slot[hh]) * a.d
-                         : reinterpret_cast<T*>(a.k_rot) + ((size_t)krow * a.Hkv + (hh - a.Hq)) * a.d;
+      T* dst;
+      if (hh < a.Hq) {
+        int g, slot;
+        head_slot(a, G, hh, g, slot);
+        dst = reinterpret_cast<T*>(a.q_rot) + ((size_t)g * M + (size_t)t * G + slot) * a.d;
+      } else {
+        dst = reinterpret_cast<T*>(a.k_rot) + ((size_t)krow * a.Hkv + (hh - a.Hq)) * a.d;
+      }
       float x0[8], x1[8], y0[8], y1[8];
       unpack8(r0[it], x0);
       unpack8(r1[it], x1);
@@ -273,26 +297,8 @@ __global__ void __launch_bounds__(256) rope_pack_kernel(RopePackArgs a) {
       store8(dst + i0 + half, y1);
     }
   }
-  // heads beyond kMaxIt iterations (very wide models) take a plain loop
-  for (int hh = hsub + kMaxIt * heads_per_it; hh < H; hh += heads_per_it) {
-    if (hh >= a.Hq && !kvalid) continue;
-    const T* src = hh < a.Hq ? reinterpret_cast<const T*>(a.q) + ((size_t)t * a.Hq + hh) * a.d
-                             : reinterpret_cast<const T*>(a.k) + ((size_t)t * a.Hkv + (hh - a.Hq)) * a.d;
-    T* dst = hh < a.Hq ? reinterpret_cast<T*>(a.q_rot) + ((size_t)s_grp[hh] * M + (size_t)t * G + s_slot[hh]) * a.d
-                       : reinterpret_cast<T*>(a.k_rot) + ((size_t)krow * a.Hkv + (hh - a.Hq)) * a.d;
-    float u0[8], u1[8], y0[8], y1[8];
-    load8(src + i0, u0);
-    load8(src + i0 + half, u1);
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      y0[k] = u0[k] * c8[k] - u1[k] * s8[k];
-      y1[k] = u1[k] * c8[k] + u0[k] * s8[k];
-    }
-    store8(dst + i0, y0);
-    store8(dst + i0 + half, y1);
-  }
   // cache mode: the new token's values go to the same cache row as its key
-  if (a.v_cache && kvalid) {
+  if (a.v_cache && kvalid && chunk == 0) {
     constexpr int kVec = 16 / sizeof(T);
     const uint4* src = reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(a.v) + (size_t)t * a.Hkv * a.d);
     uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<T*>(a.v_cache) + (size_t)krow * a.Hkv * a.d);
@@ -326,13 +332,16 @@ __global__ void rope_inplace_kernel(T* x, int L, int H, int d, int pos0, double 
 
 cudaError_t launch_rope_pack(const RopePackArgs& a, jev_dtype dt, cudaStream_t s) {
   if (a.T == 0) return cudaSuccess;
-  const int blocks = (a.T + kTokPerBlock - 1) / kTokPerBlock;
+  // warps: the token's heads in chunks of kChunkIt iterations (d / 16 lanes per head)
+  const int per_warp = kChunkIt * (32 / (a.d / 16));
+  const long long warps = (long long)a.T * ((a.Hq + a.Hkv + per_warp - 1) / per_warp);
+  const int blocks = (int)((warps + kPackWarps - 1) / kPackWarps);
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.gridDim = dim3(blocks);
-  cfg.blockDim = dim3(256);
+  cfg.blockDim = dim3(kPackWarps * 32);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = s;
   cfg.attrs = attr;
