@@ -744,12 +744,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 // are in flight together, and an online log-sum-exp rescaling folds each
 // batch into the running result (the split merge rule applied
 // incrementally).  Tiles split into few segments take (kCols, kBatch) =
-// (all columns / 8, 4), tiles split into many take half the columns and 8.
-// A tile that one CTA finished is skipped.
+// (2, 4), tiles split into many (1, 8); grid.z covers the rest of the
+// columns, and 64 registers a thread keep four blocks on an SM, so the grid
+// runs in about one wave.  A tile that one CTA finished is skipped.
 constexpr int kFixRows = 32;
 
 template <int D, int kCols, int kFixBatch>
-__global__ void __launch_bounds__(256) tc_fixup_kernel(const AttnArgs a) {
+__global__ void __launch_bounds__(256, 4) tc_fixup_kernel(const AttnArgs a) {
   const int w = a.tail0 + blockIdx.x;  // only tail tiles can be split
   const long long t0 = (long long)blockIdx.x * a.P;
   const int c_lo = tc_cta_of(a, t0), c_hi = tc_cta_of(a, t0 + a.P - 1);
@@ -937,6 +938,15 @@ bool attn_tc_supported(int d) {
   return cc == 10 && encode_fn() != nullptr;
 }
 
+// One launch of the merge kernel: grid.z covers the D / 4 float4 columns in
+// groups of 8 warps x kCols.
+template <int D, int kCols, int kFixBatch>
+cudaError_t launch_fix(cudaLaunchConfig_t cfg, const AttnArgs& a) {
+  static_assert((D / 4) % (8 * kCols) == 0, "column groups");
+  cfg.gridDim.z = (D / 4) / (8 * kCols);
+  return cudaLaunchKernelEx(&cfg, tc_fixup_kernel<D, kCols, kFixBatch>, a);
+}
+
 cudaError_t launch_tc_fixup(const AttnArgs& a, cudaStream_t s) {
   if (a.tail_ctas < 2 || a.n_tiles <= a.tail0) return cudaSuccess;
   cudaLaunchConfig_t cfg = {};
@@ -946,16 +956,14 @@ cudaError_t launch_tc_fixup(const AttnArgs& a, cudaStream_t s) {
   // the most segments any tail tile is split into
   const long long max_segs = ((long long)a.P * a.tail_ctas + a.U - 1) / a.U + 1;
   const bool many = max_segs > 4;
-  const int z = many ? 2 : 1;
-  cfg.gridDim = dim3(a.n_tiles - a.tail0, 2 * kBM / kFixRows, z);
+  cfg.gridDim = dim3(a.n_tiles - a.tail0, 2 * kBM / kFixRows, 1);
   cfg.blockDim = dim3(256);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (a.d == 128)
-    return many ? cudaLaunchKernelEx(&cfg, tc_fixup_kernel<128, 2, 8>, a) : cudaLaunchKernelEx(&cfg, tc_fixup_kernel<128, 4, 4>, a);
-  return many ? cudaLaunchKernelEx(&cfg, tc_fixup_kernel<64, 1, 8>, a) : cudaLaunchKernelEx(&cfg, tc_fixup_kernel<64, 2, 4>, a);
+  if (a.d == 128) return many ? launch_fix<128, 1, 8>(cfg, a) : launch_fix<128, 2, 4>(cfg, a);
+  return many ? launch_fix<64, 1, 8>(cfg, a) : launch_fix<64, 2, 4>(cfg, a);
 }
 
 cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t s) {
