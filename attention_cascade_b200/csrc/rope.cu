@@ -47,7 +47,6 @@ __device__ __forceinline__ void unpack8(const F8& v, float (&f)[8]) {
 }
 
 constexpr int kPackWarps = 4;  // warps per block
-constexpr int kChunkIt = 2;    // head iterations per warp (8 heads at d = 128, 16 at d = 64)
 
 // Tree plan of node m, computed by the warp of each of m's tokens (nodes in
 // depth-first preorder, packed tokens in node order).  The keys a token of m
@@ -153,7 +152,11 @@ __device__ __forceinline__ void head_slot(const RopePackArgs& a, int G, int h, i
 // node plan or cache bookkeeping) is written by the warp of chunk 0.  No
 // block-wide barrier outside block 0, which also checks the inputs and
 // writes the inverse head table.
-template <typename T>
+// kChunkIt: head iterations per warp (4 or 8 heads per iteration at d = 128
+// or 64).  Two iterations give the most parallel, shortest chains for a
+// few thousand tokens; four keep more bytes in flight per warp when the grid
+// is several waves deep.
+template <typename T, int kChunkIt>
 __global__ void __launch_bounds__(kPackWarps * 32) rope_pack_kernel(RopePackArgs a) {
   const int half = a.d >> 1;
   const int G = a.Hq / a.Hkv;
@@ -332,10 +335,15 @@ __global__ void rope_inplace_kernel(T* x, int L, int H, int d, int pos0, double 
 
 cudaError_t launch_rope_pack(const RopePackArgs& a, jev_dtype dt, cudaStream_t s) {
   if (a.T == 0) return cudaSuccess;
-  // warps: the token's heads in chunks of kChunkIt iterations (d / 16 lanes per head)
-  const int per_warp = kChunkIt * (32 / (a.d / 16));
-  const long long warps = (long long)a.T * ((a.Hq + a.Hkv + per_warp - 1) / per_warp);
-  const int blocks = (int)((warps + kPackWarps - 1) / kPackWarps);
+  // warps: the token's heads in chunks of `it` iterations of 32 / (d / 16)
+  // heads each; four iterations once two would need more than 8192 warps
+  // (about two waves of resident warps on 148 SMs)
+  auto n_warps = [&](int it) {
+    const int per_warp = it * (32 / (a.d / 16));
+    return (long long)a.T * ((a.Hq + a.Hkv + per_warp - 1) / per_warp);
+  };
+  const int it = n_warps(2) > 8192 ? 4 : 2;
+  const int blocks = (int)((n_warps(it) + kPackWarps - 1) / kPackWarps);
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -346,8 +354,10 @@ cudaError_t launch_rope_pack(const RopePackArgs& a, jev_dtype dt, cudaStream_t s
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (dt == JEV_BF16) return cudaLaunchKernelEx(&cfg, rope_pack_kernel<__nv_bfloat16>, a);
-  return cudaLaunchKernelEx(&cfg, rope_pack_kernel<float>, a);
+  if (dt == JEV_BF16)
+    return it == 4 ? cudaLaunchKernelEx(&cfg, rope_pack_kernel<__nv_bfloat16, 4>, a)
+                   : cudaLaunchKernelEx(&cfg, rope_pack_kernel<__nv_bfloat16, 2>, a);
+  return it == 4 ? cudaLaunchKernelEx(&cfg, rope_pack_kernel<float, 4>, a) : cudaLaunchKernelEx(&cfg, rope_pack_kernel<float, 2>, a);
   return cudaGetLastError();
 }
 
