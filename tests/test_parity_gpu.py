@@ -88,6 +88,21 @@ def test_flat_config_full_size_sampled(jev, name):
     check_readout(lp, ch, ref, cfg.dtype, name)
 
 
+@pytest.mark.parametrize("dtype", [synth.BF16, synth.F32])
+def test_many_tokens_at_d64_sampled(jev, dtype):
+    """About 9000 suffix tokens at d = 64: the RoPE pack's grid is deep enough
+    for its sixteen-heads-a-warp form (more than 8192 warps at eight), which
+    the other shapes reach only in bf16 at d = 128.  Sampled rows (first and
+    last token of every branch plus random ones) against the oracle."""
+    cfg = synth.FlatConfig("many_d64", dtype, 64, 600, 8, 22, 8, 2, 64, 64, 256, 2, 2, seed=31)
+    c = synth.flat_case(cfg, with_lm_head=False)
+    assert c.T > 8192
+    out, lse = run_flat(jev, c)
+    rows = _sample_rows(c, 300, seed=8)
+    ref_o, ref_l = oracle.prefix_suffix_attn(c.q, c.k_pre, c.v_pre, c.k_suf, c.v_suf, c.cu_seqlens, rows=rows)
+    check_attn(out[rows[:, 0], rows[:, 1]], lse[rows[:, 0], rows[:, 1]], ref_o, ref_l, dtype, "many tokens d64")
+
+
 EDGE = [
     # dtype, Lp, lens, Hq, Hkv, d, splits, pos_offset, head_map
     (synth.BF16, 300, [1, 7, 0, 33, 130], 8, 2, 128, 0, -1, None),
