@@ -4,8 +4,9 @@
 //
 // Each block holds 16 stacked rows (row m of group g is token m / G, query
 // slot m % G) and streams 32-key tiles of the prefix split through shared
-// memory; one warp owns four rows, a lane owns one key of the tile for the
-// scores and d/32 output columns for P.V.  The online softmax runs in the
+// memory, the next tile's K and V loaded into registers while the current one
+// is computed; one warp owns four rows, a lane owns one key of the tile for
+// the scores and d/32 output columns for P.V.  The online softmax runs in the
 // log2 domain.  The block that holds the last prefix split also walks the
 // suffix keys its rows may see: for a flat branch, the keys of the same branch
 // up to the row's own token (or its slot in the branch's cache); for a tree
@@ -77,17 +78,59 @@ __global__ void __launch_bounds__(kThreads) attn_simt_kernel(AttnArgs a) {
     for (int c = 0; c < C; ++c) acc[r][c] = 0.f;
   }
 
-  // one 32-key tile: keys [kb, kb + n) of K/V with row stride Hkv*D
-  auto tile = [&](const T* Kg, const T* Vg, int kb, int n, bool suffix) {
-    __syncthreads();
-    for (int e = tid; e < kKeys * D; e += kThreads) {
-      int j = e / D, i = e - j * D;
-      bool ok = j < n;
-      size_t off = ((size_t)(kb + j) * a.Hkv) * D + i;
-      Ks[j][i] = ok ? to_f32(Kg[off]) : 0.f;
-      Vs[j][i] = ok ? to_f32(Vg[off]) : 0.f;
+  // The key tiles of this block, in order: the prefix split, then (for the
+  // last split) the suffix window.  Each thread stages kPer elements of a
+  // tile's K and of its V; the next tile's are loaded into registers before
+  // the current tile is computed.
+  constexpr int kPer = kKeys * D / kThreads;
+  const T* kp = reinterpret_cast<const T*>(a.k_pre) + (size_t)g * D;
+  const T* vp = reinterpret_cast<const T*>(a.v_pre) + (size_t)g * D;
+  const T* ks = reinterpret_cast<const T*>(a.k_rot) + (size_t)g * D;
+  const T* vs = reinterpret_cast<const T*>(a.v_suf) + (size_t)g * D;
+  const int p_lo = split * a.split_len;
+  const int p_hi = min(a.Lp, p_lo + a.split_len);
+  const int n_pre = p_hi > p_lo ? (p_hi - p_lo + kKeys - 1) / kKeys : 0;
+  __syncthreads();  // the window (s_lo, s_hi) is published
+  const int lo = s_lo, hi = s_hi;
+  const int n_suf = split == a.S - 1 && lo <= hi ? (hi - lo + kKeys) / kKeys : 0;
+  // tile i: keys [kb, kb + n) of (Kg, Vg); suffix tiles after the prefix ones
+  auto tile_src = [&](int i, const T*& Kg, const T*& Vg, int& kb, int& n) {
+    if (i < n_pre) {
+      Kg = kp; Vg = vp; kb = p_lo + i * kKeys; n = min(kKeys, p_hi - kb);
+    } else {
+      Kg = ks; Vg = vs; kb = lo + (i - n_pre) * kKeys; n = min(kKeys, hi + 1 - kb);
+    }
+  };
+  float kr[kPer], vr[kPer];
+  auto fetch = [&](int i) {
+    const T* Kg; const T* Vg; int kb, n;
+    tile_src(i, Kg, Vg, kb, n);
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int e = tid + u * kThreads;
+      const int j = e / D, c = e - j * D;
+      const bool ok = j < n;
+      const size_t off = ((size_t)(kb + j) * a.Hkv) * D + c;
+      kr[u] = ok ? to_f32(Kg[off]) : 0.f;
+      vr[u] = ok ? to_f32(Vg[off]) : 0.f;
+    }
+  };
+  const int n_tiles = n_pre + n_suf;
+  if (n_tiles > 0) fetch(0);
+  for (int i = 0; i < n_tiles; ++i) {
+    const T* Kg_; const T* Vg_; int kb, n;
+    tile_src(i, Kg_, Vg_, kb, n);
+    const bool suffix = i >= n_pre;
+    __syncthreads();  // every warp is done with the previous tile
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int e = tid + u * kThreads;
+      const int j = e / D, c = e - j * D;
+      Ks[j][c] = kr[u];
+      Vs[j][c] = vr[u];
     }
     __syncthreads();
+    if (i + 1 < n_tiles) fetch(i + 1);  // in flight while this tile is computed
     float p[4];
     const int key = kb + lane;
     // tree key: the end of the packed tokens of its node's subtree
@@ -95,15 +138,15 @@ __global__ void __launch_bounds__(kThreads) attn_simt_kernel(AttnArgs a) {
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
       const int rr = warp * 4 + r;
-      float s = 0.f;
+      float sc = 0.f;
 #pragma unroll 8
-      for (int i = 0; i < D; ++i) s += Qs[rr][i] * Ks[lane][i];
-      s *= a.scale_log2;
+      for (int c = 0; c < D; ++c) sc += Qs[rr][c] * Ks[lane][c];
+      sc *= a.scale_log2;
       bool ok = lane < n && r_t[rr] >= 0;
       if (ok && suffix)
         ok = tree ? (key <= r_t[rr] && r_t[rr] < kend) : (key >= r_start[rr] && key <= r_last[rr]);
-      s = ok ? s : -CUDART_INF_F;
-      const float mx = warp_max(s);
+      sc = ok ? sc : -CUDART_INF_F;
+      const float mx = warp_max(sc);
       const float m_new = fmaxf(m_r[r], mx);
       float alpha, pv;
       if (m_new == -CUDART_INF_F) {
@@ -111,7 +154,7 @@ __global__ void __launch_bounds__(kThreads) attn_simt_kernel(AttnArgs a) {
         pv = 0.f;
       } else {
         alpha = exp2f(m_r[r] - m_new);
-        pv = exp2f(s - m_new);
+        pv = exp2f(sc - m_new);
       }
       l_r[r] = l_r[r] * alpha + warp_sum(pv);
       m_r[r] = m_new;
@@ -127,19 +170,6 @@ __global__ void __launch_bounds__(kThreads) attn_simt_kernel(AttnArgs a) {
         for (int c = 0; c < C; ++c) acc[r][c] += pj * Vs[j][lane + 32 * c];
       }
     }
-  };
-
-  const T* kp = reinterpret_cast<const T*>(a.k_pre) + (size_t)g * D;
-  const T* vp = reinterpret_cast<const T*>(a.v_pre) + (size_t)g * D;
-  const int p_lo = split * a.split_len;
-  const int p_hi = min(a.Lp, p_lo + a.split_len);
-  for (int kb = p_lo; kb < p_hi; kb += kKeys) tile(kp, vp, kb, min(kKeys, p_hi - kb), false);
-  if (split == a.S - 1) {
-    __syncthreads();
-    const int lo = s_lo, hi = s_hi;
-    const T* ks = reinterpret_cast<const T*>(a.k_rot) + (size_t)g * D;
-    const T* vs = reinterpret_cast<const T*>(a.v_suf) + (size_t)g * D;
-    for (int kb = lo; kb <= hi; kb += kKeys) tile(ks, vs, kb, min(kKeys, hi + 1 - kb), true);
   }
 
 #pragma unroll
