@@ -184,3 +184,37 @@ def test_header_is_plain_c_and_links(jev, tmp_path):
     assert r.returncode == 0, r.stderr
     out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()
     assert int(out[0]) == len(names) and int(out[1]) == jev.jev_vocab_lse_workspace(256, 152064)
+
+
+def test_host_calls_are_reentrant_across_threads(jev):
+    """The host-only entry points (trie build, readout plan, work plan) give the
+    same answers when eight threads call them at once (ctypes releases the
+    interpreter lock, so the calls overlap inside the library)."""
+    from concurrent.futures import ThreadPoolExecutor
+    rng = np.random.default_rng(12)
+    problems = []
+    for i in range(8):
+        n = int(rng.integers(5, 40))
+        lens = rng.integers(1, 9, n)
+        seq_off = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+        toks = rng.integers(0, 6, int(seq_off[-1])).astype(np.int32)
+        problems.append((seq_off, toks))
+    descs = [jev.make_attn_desc(8 + i, 256 * (i + 1), 28, 4, 128, 100 * (i + 1), jev.JEV_BF16) for i in range(8)]
+
+    def work(i):
+        seq_off, toks = problems[i]
+        out = []
+        for _ in range(30):
+            t = jev.jev_tree_build(seq_off, toks, 16)
+            score_from = np.ones(seq_off.size - 1, np.int32)
+            p = jev.jev_tree_readout_plan(seq_off, toks, score_from, t["path_row"])
+            plan = jev.jev_prefix_suffix_attn_plan(descs[i], 1, 148)
+            out.append((t["parent"].tobytes(), t["tok_off"].tobytes(), p["pair_row"].tobytes(),
+                        p["pair_tok"].tobytes(), tuple(sorted(plan.items()))))
+        return out
+
+    serial = [work(i)[0] for i in range(8)]
+    with ThreadPoolExecutor(8) as ex:
+        results = list(ex.map(work, range(8)))
+    for i in range(8):
+        assert all(r == serial[i] for r in results[i])
