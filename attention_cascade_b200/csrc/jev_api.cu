@@ -243,16 +243,18 @@ Plan compute_plan(const jev_attn_desc* d, int T, int kernel, int sms_hint) {
     p.split_len = std::max(1, ktiles) * 128;
     return p;
   }
+  // CUDA-core kernel: splits of whole 32-key tiles (the kernel's tile)
+  const int kt32 = (d->Lp + 31) / 32;
   int S = d->num_splits;
   if (S <= 0) {
     const long ctas = (long)((p.M + 15) / 16) * d->Hkv;
     const long target = 4L * num_sms();
     S = ctas > 0 ? (int)((target + ctas - 1) / ctas) : 1;
-    // keep at least 4 key tiles per split so partial traffic stays small
-    S = std::min(S, std::max(1, ktiles / 4));
+    // keep at least 2 key tiles per split so partial traffic stays small
+    S = std::min(S, std::max(1, kt32 / 2));
   }
-  S = std::max(1, std::min(std::min(S, kMaxSplits), std::max(1, ktiles)));
-  p.split_len = ktiles > 0 ? ((ktiles + S - 1) / S) * 128 : 128;
+  S = std::max(1, std::min(std::min(S, kMaxSplits), std::max(1, kt32)));
+  p.split_len = kt32 > 0 ? ((kt32 + S - 1) / S) * 32 : 32;
   p.S = d->Lp > 0 ? (d->Lp + p.split_len - 1) / p.split_len : 1;
   return p;
 }

@@ -57,7 +57,7 @@ struct AttnArgs {
   float* o_part;            // [S, Hkv, M, d] (num_splits > 1)
   float* l_part;            // [S, Hkv, M] log2-domain
   int32_t* status;
-  int T, M, Lp, Hq, Hkv, G, d, S, split_len;  // split_len: prefix keys per split (multiple of 128)
+  int T, M, Lp, Hq, Hkv, G, d, S, split_len;  // split_len: prefix keys per split (CUDA-core kernel: a multiple of 32)
   int key_rows;             // rows of k_rot / v_suf
   float scale_log2;         // softmax scale * log2(e)
   // Tensor-core schedule.  Work tile w = (kv group w / n_pairs, 256-row pair

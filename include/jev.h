@@ -107,7 +107,7 @@ size_t jev_prefix_suffix_attn_workspace(const jev_attn_desc* desc);
  * owning [c*tail_units/tail_ctas, (c+1)*tail_units/tail_ctas); split != 0
  * when some tile is shared by several CTAs and a merge kernel combines it.
  * CUDA-core kernel (kernel == 0): simt_splits prefix splits of split_len
- * keys.  Returns the descriptor's error (as jev_prefix_suffix_attn would) or
+ * keys (a multiple of 32).  Returns the descriptor's error (as jev_prefix_suffix_attn would) or
  * JEV_ERR_INVALID_ARG for a NULL `plan` or a kernel outside -1 .. 1.
  */
 typedef struct {

@@ -116,9 +116,15 @@ def test_plan_query_rejects_bad_arguments():
         jev.jev_prefix_suffix_attn_plan(desc, kernel=2)
     with pytest.raises(jev.JevError):
         jev.jev_prefix_suffix_attn_plan(jev.make_attn_desc(2, 128, 8, 3, 128, 10, jev.JEV_BF16))
-    # the CUDA-core plan: prefix splits of whole 128-key tiles covering Lp
-    p = jev.jev_prefix_suffix_attn_plan(jev.make_attn_desc(2, 1000, 8, 2, 128, 10, jev.JEV_F32, num_splits=3), 0)
-    assert p["kernel"] == 0 and p["split_len"] % 128 == 0 and p["simt_splits"] * p["split_len"] >= 1000
+    # the CUDA-core plan: prefix splits of whole 32-key tiles covering Lp exactly once
+    for Lp, ns in ((1000, 3), (1000, 0), (256, 0), (33, 0), (20, 5)):
+        p = jev.jev_prefix_suffix_attn_plan(jev.make_attn_desc(2, Lp, 8, 2, 128, 10, jev.JEV_F32, num_splits=ns), 0)
+        L, S = p["split_len"], p["simt_splits"]
+        assert p["kernel"] == 0 and L % 32 == 0 and S >= 1
+        assert S * L >= Lp and (S - 1) * L < Lp  # every split holds keys
+    # a small problem gets several splits (two 32-key tiles each at least)
+    p = jev.jev_prefix_suffix_attn_plan(jev.make_attn_desc(4, 256, 2, 1, 64, 64, jev.JEV_F32), 0)
+    assert p["simt_splits"] == 4 and p["split_len"] == 64
 
 
 def test_tree_schedule_study_inputs():
