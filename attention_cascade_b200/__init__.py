@@ -460,3 +460,12 @@ _lib.jev_debug_set_wait_limit.restype = C.c_int
 def jev_debug_set_wait_limit(cycles: int):
     """Bound of the tensor-core kernels' mbarrier waits for later launches (0: the default)."""
     _check(_lib.jev_debug_set_wait_limit(int(cycles)), "jev_debug_set_wait_limit")
+
+
+_lib.jev_debug_set_wait_probe.argtypes = [C.c_int32]
+_lib.jev_debug_set_wait_probe.restype = C.c_int
+
+
+def jev_debug_set_wait_probe(on: bool):
+    """Failure-detection probe for later launches: each CTA's MMA warp also waits on a barrier nothing completes."""
+    _check(_lib.jev_debug_set_wait_probe(1 if on else 0), "jev_debug_set_wait_probe")

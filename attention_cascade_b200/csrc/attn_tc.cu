@@ -86,7 +86,7 @@ struct Cfg {
 };
 
 struct Bars {
-  uint32_t q_full, q_empty, k_full, v_full, kv_empty, s_full, p_full, o_full, drain;  // arrays: +8*i
+  uint32_t q_full, q_empty, k_full, v_full, kv_empty, s_full, p_full, o_full, drain, probe;  // arrays: +8*i
 };
 
 struct Shared {
@@ -129,6 +129,22 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
   }
 }
 
+// The failure-detection probe: a bounded wait on a barrier that nothing
+// completes.  It runs out after the wait bound (checking the clock at least
+// every microsecond) and winds the CTA down like any other timeout.
+__device__ __forceinline__ bool probe_wait(uint32_t bar, volatile int* abort, int32_t* status, long long limit) {
+  const long long t0 = clock64();
+  for (;;) {
+    if (mbar_try_wait_hint(bar, 0, 1000)) return true;
+    if (*abort) return false;
+    if (clock64() - t0 > limit) {
+      *abort = 1;
+      raise_flag(status, JEV_DEV_WAIT_TIMEOUT);
+      return false;
+    }
+  }
+}
+
 // Wait on the exit path: bounded, but blind to the abort flag, so that a CTA
 // that is winding down still sees every load it armed land and every MMA it
 // issued complete before it frees TMEM and exits.  Such work completes within
@@ -142,6 +158,13 @@ __device__ __forceinline__ void drain_bar(uint32_t bar, uint32_t parity, int32_t
       return;
     }
   }
+}
+
+// Bounded wait taken by a whole warp: every lane polls, and all take lane 0's
+// answer, so that the warp stays converged for the elected issue that follows.
+__device__ __forceinline__ bool wait_bar_w(uint32_t bar, uint32_t parity, volatile int* abort, int32_t* status,
+                                           long long limit) {
+  return __shfl_sync(0xffffffffu, wait_bar(bar, parity, abort, status, limit), 0);
 }
 
 __device__ __forceinline__ int warp_min_i(int v) {
@@ -271,6 +294,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   B.p_full = B.s_full + 16;
   B.o_full = B.p_full + 16;
   B.drain = B.o_full + 16;
+  B.probe = B.drain + 8;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int cta = blockIdx.x;
@@ -291,6 +315,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(B.o_full + 8 * i, 1);
     }
     mbar_init(B.drain, 1);
+    mbar_init(B.probe, 1);  // nothing arrives on it
     sh->abort = 0;
     mbar_fence_init();
   }
@@ -309,12 +334,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == kProducerWarp) {
     // ---------------------------------------------------------------- TMA producer
+    // The whole warp runs the loop (its values stay warp-uniform); one
+    // elected lane issues each load.
     long long J = 0;
     long long kv_armed = 0;  // key tiles whose K and V loads this warp has issued
     int q_armed = 0;         // Q tiles loaded
     int k = 0;
     bool ok = true;
-    tma_prefetch_desc(&tm_q);
+    if (lane == 0) tma_prefetch_desc(&tm_q);
     // the first segment's leading prefix key tiles need nothing from the pack:
     // their loads start before the wait (the pack lets this kernel launch only
     // once every kernel before it in the stream has completed)
@@ -326,16 +353,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (seg_next(a, cta, it0, w0, ua0, ub0, tl0)) {
         pre0 = min(max(0, min(ub0, a.n_pre) - ua0), C::kNS);
         const int g0 = w0 / a.n_pairs;
-        if (lane == 0)
-          for (int j = 0; j < pre0; ++j) {
-            const uint32_t ks = sbase + C::kOffK + j * C::kKVBytes, vs = sbase + C::kOffV + j * C::kKVBytes;
-            mbar_expect_tx(B.k_full + 8 * j, C::kKVBytes);
-            for (int b = 0; b < D / 64; ++b)
-              tma_load_2d(ks + b * C::kBlk, &tm_kp, g0 * D + b * 64, (ua0 + j) * kBN, B.k_full + 8 * j);
-            mbar_expect_tx(B.v_full + 8 * j, C::kKVBytes);
-            for (int b = 0; b < D / 64; ++b)
-              tma_load_2d(vs + b * C::kBlk, &tm_vp, g0 * D + b * 64, (ua0 + j) * kBN, B.v_full + 8 * j);
-          }
+        for (int j = 0; j < pre0; ++j) {
+          const uint32_t ks = sbase + C::kOffK + j * C::kKVBytes, vs = sbase + C::kOffV + j * C::kKVBytes;
+          mbar_expect_tx_w(B.k_full + 8 * j, C::kKVBytes);
+          for (int b = 0; b < D / 64; ++b)
+            tma_load_2d_w(ks + b * C::kBlk, &tm_kp, g0 * D + b * 64, (ua0 + j) * kBN, B.k_full + 8 * j);
+          mbar_expect_tx_w(B.v_full + 8 * j, C::kKVBytes);
+          for (int b = 0; b < D / 64; ++b)
+            tma_load_2d_w(vs + b * C::kBlk, &tm_vp, g0 * D + b * 64, (ua0 + j) * kBN, B.v_full + 8 * j);
+        }
         kv_armed = pre0;
       }
     }
@@ -346,31 +372,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (; ok && seg_next(a, cta, it, sw, sua, sub, stail); ++k, ++it.k) {
       // The Q tile goes first: it needs only the tile's group and rows.
       const int qg = sw / a.n_pairs, qm0 = (sw - qg * a.n_pairs) * 2 * kBM;
-      if (lane == 0) {
-        if (k > 0 && !wait_bar(B.q_empty, (k - 1) & 1, abort, a.status, a.wait_cycles)) ok = false;
-        if (ok) {
-          mbar_expect_tx(B.q_full, 2 * C::kQBytes);
-          for (int i = 0; i < 2; ++i)
-            for (int b = 0; b < D / 64; ++b)
-              tma_load_3d(sbase + i * C::kQBytes + b * C::kBlk, &tm_q, b * 64, qm0 + i * kBM, qg, B.q_full);
-          ++q_armed;
-        }
+      if (k > 0 && !wait_bar_w(B.q_empty, (k - 1) & 1, abort, a.status, a.wait_cycles)) ok = false;
+      if (ok) {
+        mbar_expect_tx_w(B.q_full, 2 * C::kQBytes);
+        for (int i = 0; i < 2; ++i)
+          for (int b = 0; b < D / 64; ++b)
+            tma_load_3d_w(sbase + i * C::kQBytes + b * C::kBlk, &tm_q, b * 64, qm0 + i * kBM, qg, B.q_full);
+        ++q_armed;
       }
-      ok = __shfl_sync(0xffffffffu, ok, 0);
       // The description (for the suffix unit, its key window: a warp-wide read
       // of token info) is published with q_full's second arrival.
       const Segment sg = make_segment(a, cta, sw, sua, sub, stail, lane);
-      if (lane == 0) {
-        if (ok) {
+      if (ok) {
+        if (lane == 0) {
           seg_sm[k & 1] = sg;
           mbar_arrive(B.q_full);
         }
+        __syncwarp();
         for (int j = k == 0 ? pre0 : 0; ok && j < sg.n; ++j) {
           const long long JJ = J + j;
           const int st = (int)(JJ % C::kNS);
           const long long use = JJ / C::kNS;
           if (JJ >= C::kNS &&
-              !wait_bar(B.kv_empty + 8 * st, (uint32_t)((use - 1) & 1), abort, a.status, a.wait_cycles)) {
+              !wait_bar_w(B.kv_empty + 8 * st, (uint32_t)((use - 1) & 1), abort, a.status, a.wait_cycles)) {
             ok = false;
             break;
           }
@@ -379,14 +403,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           const CUtensorMap* mk = pre ? &tm_kp : &tm_ks;
           const CUtensorMap* mv = pre ? &tm_vp : &tm_vs;
           const uint32_t ks = sbase + C::kOffK + st * C::kKVBytes, vs = sbase + C::kOffV + st * C::kKVBytes;
-          mbar_expect_tx(B.k_full + 8 * st, C::kKVBytes);
-          for (int b = 0; b < D / 64; ++b) tma_load_2d(ks + b * C::kBlk, mk, sg.g * D + b * 64, kb, B.k_full + 8 * st);
-          mbar_expect_tx(B.v_full + 8 * st, C::kKVBytes);
-          for (int b = 0; b < D / 64; ++b) tma_load_2d(vs + b * C::kBlk, mv, sg.g * D + b * 64, kb, B.v_full + 8 * st);
+          mbar_expect_tx_w(B.k_full + 8 * st, C::kKVBytes);
+          for (int b = 0; b < D / 64; ++b)
+            tma_load_2d_w(ks + b * C::kBlk, mk, sg.g * D + b * 64, kb, B.k_full + 8 * st);
+          mbar_expect_tx_w(B.v_full + 8 * st, C::kKVBytes);
+          for (int b = 0; b < D / 64; ++b)
+            tma_load_2d_w(vs + b * C::kBlk, mv, sg.g * D + b * 64, kb, B.v_full + 8 * st);
           kv_armed = JJ + 1;
         }
       }
-      ok = __shfl_sync(0xffffffffu, ok, 0);
       J += sg.n;
     }
     if (lane == 0) {
@@ -404,6 +429,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == kMmaWarp) {
     // ---------------------------------------------------------------- MMA issuer
+    // The whole warp runs the loop, so descriptors and addresses stay
+    // warp-uniform; one elected lane issues each MMA and commit.
     constexpr uint32_t id_qk = idesc_bf16(kBM, kBN, false);
     constexpr uint32_t id_pv = idesc_bf16(kBM, D, true);
     // Shared-memory descriptors are formed once; an operand's descriptor is a
@@ -419,15 +446,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int kk = 0; kk < D / 16; ++kk) {
         constexpr int kBlk4 = C::kBlk >> 4;
         const uint32_t off = (uint32_t)((kk >> 2) * kBlk4 + (kk & 3) * 2);
-        mma_ss(tmem + i * kBN, qa + off, ka + off, id_qk, kk > 0);
+        mma_ss_w(tmem + i * kBN, qa + off, ka + off, id_qk, kk > 0);
       }
-      mma_commit(B.s_full + 8 * i);
+      mma_commit_w(B.s_full + 8 * i);
     };
     auto issue_pv = [&](int i, int st, bool acc) {
       const uint64_t va = dv0 + (uint32_t)((st * C::kKVBytes) >> 4);
 #pragma unroll
       for (int kk = 0; kk < kBN / 16; ++kk)
-        mma_ts(tmem + C::kOCol + i * D, tmem + i * kBN + kk * 8, va + (uint32_t)(kk * 16 * 128 / 16), id_pv,
+        mma_ts_w(tmem + C::kOCol + i * D, tmem + i * kBN + kk * 8, va + (uint32_t)(kk * 16 * 128 / 16), id_pv,
                (acc || kk > 0) ? 1u : 0u);
     };
     long long J = 0;
@@ -438,39 +465,43 @@ __global__ void __launch_bounds__(kThreads, 1)
     int sw, sua, sub;
     bool stail;
     for (; ok && seg_next(a, cta, it, sw, sua, sub, stail); ++k, ++it.k) {
-      ok = wait_bar(B.q_full, k & 1, abort, a.status, a.wait_cycles);
+      ok = wait_bar_w(B.q_full, k & 1, abort, a.status, a.wait_cycles);
       const Segment sg = seg_sm[k & 1];
-      if (lane == 0) {
+      {
         const int n = sg.n;  // >= 1
         if (ok) {
           const int st0 = (int)(J % C::kNS);
-          ok = wait_bar(B.k_full + 8 * st0, (uint32_t)((J / C::kNS) & 1), abort, a.status, a.wait_cycles);
+          ok = wait_bar_w(B.k_full + 8 * st0, (uint32_t)((J / C::kNS) & 1), abort, a.status, a.wait_cycles);
           fence_after_sync();
           if (ok) {
             issue_s(0, st0);
             issue_s(1, st0);
           }
+          // failure-detection probe (off unless a test sets it): a wait that
+          // nothing completes, with this segment's first MMAs in flight
+          if (ok && k == 0 && a.wait_probe)
+            ok = __shfl_sync(0xffffffffu, probe_wait(B.probe, abort, a.status, a.wait_cycles), 0);
         }
         for (int j = 0; ok && j < n; ++j) {
           const long long JJ = J + j, JJ1 = JJ + 1;
           const int st = (int)(JJ % C::kNS), st1 = (int)(JJ1 % C::kNS);
           const uint32_t ph = (uint32_t)((JJ / C::kNS) & 1), ph1 = (uint32_t)((JJ1 / C::kNS) & 1);
           const uint32_t pp = (uint32_t)(JJ & 1);
-          if (!wait_bar(B.v_full + 8 * st, ph, abort, a.status, a.wait_cycles)) { ok = false; break; }
-          if (!wait_bar(B.p_full, pp, abort, a.status, a.wait_cycles)) { ok = false; break; }
+          if (!wait_bar_w(B.v_full + 8 * st, ph, abort, a.status, a.wait_cycles)) { ok = false; break; }
+          if (!wait_bar_w(B.p_full, pp, abort, a.status, a.wait_cycles)) { ok = false; break; }
           fence_after_sync();
           issue_pv(0, st, j > 0);
-          if (j == n - 1) mma_commit(B.o_full);
+          if (j == n - 1) mma_commit_w(B.o_full);
           if (j + 1 < n) {
-            if (!wait_bar(B.k_full + 8 * st1, ph1, abort, a.status, a.wait_cycles)) { ok = false; break; }
+            if (!wait_bar_w(B.k_full + 8 * st1, ph1, abort, a.status, a.wait_cycles)) { ok = false; break; }
             fence_after_sync();
             issue_s(0, st1);
           }
-          if (!wait_bar(B.p_full + 8, pp, abort, a.status, a.wait_cycles)) { ok = false; break; }
+          if (!wait_bar_w(B.p_full + 8, pp, abort, a.status, a.wait_cycles)) { ok = false; break; }
           fence_after_sync();
           issue_pv(1, st, j > 0);
-          mma_commit(B.kv_empty + 8 * st);
-          if (j == n - 1) mma_commit(B.o_full + 8);
+          mma_commit_w(B.kv_empty + 8 * st);
+          if (j == n - 1) mma_commit_w(B.o_full + 8);
           // q_empty releases the Q buffer and lets the producer publish the next
           // segment.  It is committed only after both p_full waits of a tile of
           // this segment, i.e. after all 512 softmax threads have passed their
@@ -479,21 +510,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           // wait would alias the later phase and never return.
           if (j + 1 < n) {
             issue_s(1, st1);
-            if (j + 2 == n) mma_commit(B.q_empty);
+            if (j + 2 == n) mma_commit_w(B.q_empty);
           } else if (n == 1) {
-            mma_commit(B.q_empty);
+            mma_commit_w(B.q_empty);
           }
         }
       }
-      ok = __shfl_sync(0xffffffffu, ok, 0);
       J += sg.n;
     }
-    if (lane == 0) {
-      // every MMA of this CTA has completed before TMEM is released, on the
-      // timeout path too (the wait ignores the abort flag)
-      mma_commit(B.drain);
-      drain_bar(B.drain, 0, a.status);
-    }
+    // every MMA of this CTA has completed before TMEM is released, on the
+    // timeout path too (the wait ignores the abort flag); the commit comes
+    // from the lane that issued the MMAs
+    mma_commit_w(B.drain);
+    drain_bar(B.drain, 0, a.status);
   } else {
     // ---------------------------------------------------------------- softmax + epilogue
     constexpr int kHalfCols = kBN / 2;  // score columns per thread

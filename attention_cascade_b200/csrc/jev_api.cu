@@ -45,6 +45,7 @@ std::atomic<long long> g_launches{0};
 // second at the B200's clock); jev_debug_set_wait_limit changes it
 constexpr long long kDefaultWaitCycles = 1LL << 31;
 std::atomic<long long> g_wait_cycles{kDefaultWaitCycles};
+std::atomic<int> g_wait_probe{0};
 
 int name_id(const char* n) {
   for (size_t i = 0; i < g_names.size(); ++i)
@@ -405,6 +406,7 @@ jev_status attention_core(const jev_attn_desc* d, int T, const Plan& p, const La
   a.n_pairs = p.n_pairs; a.n_tiles = p.n_tiles; a.n_pre = p.n_pre; a.P = p.P; a.n_ctas = p.n_ctas; a.U = p.U;
   a.full_waves = p.full_waves; a.tail0 = p.tail0; a.tail_ctas = p.tail_ctas;
   a.wait_cycles = g_wait_cycles.load();
+  a.wait_probe = g_wait_probe.load();
   if (p.tc) {
     st = run("attn_tc", s, [&] { return launch_attn_tc(a, s); });
     if (st == JEV_OK && p.split) st = run("tc_fixup", s, [&] { return launch_tc_fixup(a, s); });
@@ -459,6 +461,11 @@ int64_t jev_launch_count(void) { return (int64_t)g_launches.load(); }
 jev_status jev_debug_set_wait_limit(int64_t cycles) {
   if (cycles < 0) return fail(JEV_ERR_INVALID_ARG, "wait limit must be >= 0");
   g_wait_cycles.store(cycles == 0 ? kDefaultWaitCycles : (long long)cycles);
+  return JEV_OK;
+}
+
+jev_status jev_debug_set_wait_probe(int32_t on) {
+  g_wait_probe.store(on != 0 ? 1 : 0);
   return JEV_OK;
 }
 
@@ -737,7 +744,7 @@ jev_status jev_vocab_lse(const void* hidden, const void* lm_head, int32_t R, int
   const int n_ctas = vocab_lse_ctas(V, num_sms());
   char* ws = (char*)workspace;
   VocabLseArgs a{hidden, lm_head, R, H, V, (V + 255) / 256, (float2*)(ws + kStatusBytes), lse, (int32_t*)ws,
-                 g_wait_cycles.load()};
+                 g_wait_cycles.load(), g_wait_probe.load()};
   const jev_status st =
       run("vocab_lse", (cudaStream_t)stream, [&] { return launch_vocab_lse(a, n_ctas, (cudaStream_t)stream); });
   if (st == JEV_OK) g_launches++;  // GEMM + online LSE, then the partial merge: two kernels

@@ -70,6 +70,7 @@ struct AttnArgs {
   int n_pairs, n_tiles, n_pre, P, n_ctas, full_waves, tail0, tail_ctas;
   long long U;
   long long wait_cycles;  // bound of every mbarrier wait (clock cycles)
+  int wait_probe;         // failure-detection probe: the MMA warp also waits on a barrier nothing completes
 };
 // tail units owned by CTAs before c (c <= tail_ctas)
 __host__ __device__ inline long long tc_unit_begin(const AttnArgs& a, int c) { return (long long)c * a.U / a.tail_ctas; }
@@ -111,6 +112,7 @@ struct VocabLseArgs {
   float* lse;    // [R] natural log
   int32_t* status;
   long long wait_cycles;  // bound of every mbarrier wait (clock cycles)
+  int wait_probe;         // failure-detection probe: the MMA warp also waits on a barrier nothing completes
 };
 int vocab_lse_ctas(int V, int sms);
 size_t vocab_lse_partial_bytes(int R, int n_ctas);

@@ -61,6 +61,22 @@ __device__ __forceinline__ bool lwait(uint32_t bar, uint32_t parity, volatile in
   }
 }
 
+// The failure-detection probe: a bounded wait on a barrier that nothing
+// completes; it runs out after the wait bound (checking the clock at least
+// every microsecond) and winds the CTA down like any other timeout.
+__device__ __forceinline__ bool lprobe(uint32_t bar, volatile int* abort, int32_t* status, long long limit) {
+  const long long t0 = clock64();
+  for (;;) {
+    if (mbar_try_wait_hint(bar, 0, 1000)) return true;
+    if (*abort) return false;
+    if (clock64() - t0 > limit) {
+      *abort = 1;
+      raise_flag(status, JEV_DEV_WAIT_TIMEOUT);
+      return false;
+    }
+  }
+}
+
 // Exit-path wait: bounded but blind to the abort flag (in-flight loads and
 // MMAs complete within microseconds; running out of the bound only raises the flag).
 constexpr long long kLDrainCycles = 1LL << 28;
@@ -83,7 +99,7 @@ __global__ void __launch_bounds__(kLThreads, 1)
   LShared* sh = reinterpret_cast<LShared*>(smem + kOffBar + 200);
   const uint32_t bar0 = sbase + kOffBar;
   const uint32_t b_full = bar0, b_empty = bar0 + 8 * kLStages, b_sfull = bar0 + 16 * kLStages,
-                 b_sempty = b_sfull + 8, b_drain = b_sfull + 16;
+                 b_sempty = b_sfull + 8, b_drain = b_sfull + 16, b_probe = b_sfull + 24;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int cta = blockIdx.x;
   // this CTA's vocabulary rows [v_lo, v_hi): an even share of 16-row slabs, walked in 256-row tiles
@@ -102,6 +118,7 @@ __global__ void __launch_bounds__(kLThreads, 1)
     mbar_init(b_sfull, 1);
     mbar_init(b_sempty, kLStatWarps * 32);
     mbar_init(b_drain, 1);
+    mbar_init(b_probe, 1);  // nothing arrives on it
     sh->abort = 0;
     mbar_fence_init();
   }
@@ -123,75 +140,92 @@ __global__ void __launch_bounds__(kLThreads, 1)
 
   if (warp == kLProducer) {
     // ---------------------------------------------------------------- TMA producer
-    if (lane == 0) {
-      long long it = 0;
-      bool ok = true;
-      for (int mb = 0; ok && mb < n_mb; ++mb)
-        for (int v0 = v_lo; ok && v0 < v_hi; v0 += kLN) {
-          const int n_t = (min(kLN, v_hi - v0) + 15) & ~15;  // rows of this tile's W chunk
-          for (int kc = 0; ok && kc < nk; ++kc, ++it) {
-            const int st = (int)(it % kLStages);
-            const long long use = it / kLStages;
-            if (it >= kLStages && !lwait(b_empty + 8 * st, (uint32_t)((use - 1) & 1), abort, a.status, a.wait_cycles)) {
-              ok = false;
-              break;
-            }
-            const uint32_t base = sbase + st * kStageBytes;
-            const bool two = mb * 2 * kLM + kLM < a.R;  // the block's second half holds rows
-            mbar_expect_tx(b_full + 8 * st, (two ? 2 * kXBytes : kXBytes) + n_t * kLK * 2);
-            tma_load_2d(base, &tm_x, kc * kLK, mb * 2 * kLM, b_full + 8 * st);
-            if (two) tma_load_2d(base + kXBytes, &tm_x, kc * kLK, mb * 2 * kLM + kLM, b_full + 8 * st);
-            // 128-row boxes, then 16-row boxes for a narrow tail (row `o` lands at o * 128 bytes)
-            int o = 0;
-            for (; o + kLM <= n_t; o += kLM) tma_load_2d(base + 2 * kXBytes + o * 128, &tm_w, kc * kLK, v0 + o, b_full + 8 * st);
-            for (; o < n_t; o += 16) tma_load_2d(base + 2 * kXBytes + o * 128, &tm_w16, kc * kLK, v0 + o, b_full + 8 * st);
+    // The whole warp runs the loop (its values stay warp-uniform, and lane
+    // 0's view of each wait is taken by all); one elected lane issues each
+    // load.
+    auto wait_w = [&](uint32_t bar, uint32_t parity) {
+      return __shfl_sync(0xffffffffu, lwait(bar, parity, abort, a.status, a.wait_cycles), 0);
+    };
+    long long it = 0;
+    bool ok = true;
+    for (int mb = 0; ok && mb < n_mb; ++mb)
+      for (int v0 = v_lo; ok && v0 < v_hi; v0 += kLN) {
+        const int n_t = (min(kLN, v_hi - v0) + 15) & ~15;  // rows of this tile's W chunk
+        for (int kc = 0; ok && kc < nk; ++kc, ++it) {
+          const int st = (int)(it % kLStages);
+          const long long use = it / kLStages;
+          if (it >= kLStages && !wait_w(b_empty + 8 * st, (uint32_t)((use - 1) & 1))) {
+            ok = false;
+            break;
           }
+          const uint32_t base = sbase + st * kStageBytes;
+          const bool two = mb * 2 * kLM + kLM < a.R;  // the block's second half holds rows
+          mbar_expect_tx_w(b_full + 8 * st, (two ? 2 * kXBytes : kXBytes) + n_t * kLK * 2);
+          tma_load_2d_w(base, &tm_x, kc * kLK, mb * 2 * kLM, b_full + 8 * st);
+          if (two) tma_load_2d_w(base + kXBytes, &tm_x, kc * kLK, mb * 2 * kLM + kLM, b_full + 8 * st);
+          // 128-row boxes, then 16-row boxes for a narrow tail (row `o` lands at o * 128 bytes)
+          int o = 0;
+          for (; o + kLM <= n_t; o += kLM)
+            tma_load_2d_w(base + 2 * kXBytes + o * 128, &tm_w, kc * kLK, v0 + o, b_full + 8 * st);
+          for (; o < n_t; o += 16)
+            tma_load_2d_w(base + 2 * kXBytes + o * 128, &tm_w16, kc * kLK, v0 + o, b_full + 8 * st);
         }
-      // drain: the last phase of every stage armed (it loads so far) has
-      // completed, so no load lands after the CTA exits
+      }
+    // drain: the last phase of every stage armed (it loads so far) has
+    // completed, so no load lands after the CTA exits
+    if (lane == 0)
       for (int st = 0; st < kLStages; ++st) {
         const long long uses = it > st ? (it - st + kLStages - 1) / kLStages : 0;
         if (uses > 0) ldrain(b_full + 8 * st, (uint32_t)((uses - 1) & 1), a.status);
       }
-    }
   } else if (warp == kLMma) {
     // ---------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      long long it = 0, tile = 0;
-      bool ok = true;
-      for (int mb = 0; ok && mb < n_mb; ++mb) {
-        const int halves = mb * 2 * kLM + kLM < a.R ? 2 : 1;
-        for (int v0 = v_lo; ok && v0 < v_hi; v0 += kLN, ++tile) {
-          const uint32_t idesc = idesc_bf16(kLM, (min(kLN, v_hi - v0) + 15) & ~15, false);
-          // the statistics threads have read the previous tile out of TMEM
-          if (tile > 0 && !lwait(b_sempty, (uint32_t)((tile - 1) & 1), abort, a.status, a.wait_cycles)) {
+    // The whole warp runs the loop; one elected lane issues each MMA and
+    // commit (the same lane every time, so the commits track its MMAs).
+    auto wait_w = [&](uint32_t bar, uint32_t parity) {
+      return __shfl_sync(0xffffffffu, lwait(bar, parity, abort, a.status, a.wait_cycles), 0);
+    };
+    long long it = 0, tile = 0;
+    bool ok = true;
+    for (int mb = 0; ok && mb < n_mb; ++mb) {
+      const int halves = mb * 2 * kLM + kLM < a.R ? 2 : 1;
+      for (int v0 = v_lo; ok && v0 < v_hi; v0 += kLN, ++tile) {
+        const uint32_t idesc = idesc_bf16(kLM, (min(kLN, v_hi - v0) + 15) & ~15, false);
+        // the statistics threads have read the previous tile out of TMEM
+        if (tile > 0 && !wait_w(b_sempty, (uint32_t)((tile - 1) & 1))) {
+          ok = false;
+          break;
+        }
+        fence_after_sync();
+        for (int kc = 0; kc < nk; ++kc, ++it) {
+          const int st = (int)(it % kLStages);
+          if (!wait_w(b_full + 8 * st, (uint32_t)((it / kLStages) & 1))) {
             ok = false;
             break;
           }
           fence_after_sync();
-          for (int kc = 0; kc < nk; ++kc, ++it) {
-            const int st = (int)(it % kLStages);
-            if (!lwait(b_full + 8 * st, (uint32_t)((it / kLStages) & 1), abort, a.status, a.wait_cycles)) {
-              ok = false;
-              break;
-            }
-            fence_after_sync();
-            const uint32_t base = sbase + st * kStageBytes;
-            for (int i = 0; i < halves; ++i)
+          const uint32_t base = sbase + st * kStageBytes;
+          for (int i = 0; i < halves; ++i)
 #pragma unroll
-              for (int kk = 0; kk < kLK / 16; ++kk)
-                mma_ss(tmem + i * kLN, smem_desc_sw128(base + i * kXBytes + kk * 32, 16, 1024),
+            for (int kk = 0; kk < kLK / 16; ++kk)
+              mma_ss_w(tmem + i * kLN, smem_desc_sw128(base + i * kXBytes + kk * 32, 16, 1024),
                        smem_desc_sw128(base + 2 * kXBytes + kk * 32, 16, 1024), idesc, (kc > 0 || kk > 0) ? 1u : 0u);
-            mma_commit(b_empty + 8 * st);
+          mma_commit_w(b_empty + 8 * st);
+          // failure-detection probe (off unless a test sets it): a wait that
+          // nothing completes, with this CTA's first MMAs in flight
+          if (it == 0 && a.wait_probe &&
+              !__shfl_sync(0xffffffffu, lprobe(b_probe, abort, a.status, a.wait_cycles), 0)) {
+            ok = false;
+            break;
           }
-          if (ok) mma_commit(b_sfull);
         }
+        if (ok) mma_commit_w(b_sfull);
       }
-      // every MMA of this CTA has completed before TMEM is released, on the
-      // timeout path too (the wait ignores the abort flag)
-      mma_commit(b_drain);
-      ldrain(b_drain, 0, a.status);
     }
+    // every MMA of this CTA has completed before TMEM is released, on the
+    // timeout path too (the wait ignores the abort flag)
+    mma_commit_w(b_drain);
+    ldrain(b_drain, 0, a.status);
   } else {
     // ---------------------------------------------------------------- statistics
     const int i = warp >> 3, hf = (warp >> 2) & 1, q = warp & 3, r = q * 32 + lane;

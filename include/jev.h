@@ -468,6 +468,20 @@ int64_t jev_launch_count(void);
  */
 jev_status jev_debug_set_wait_limit(int64_t cycles);
 
+/*
+ * jev_debug_set_wait_probe — failure-detection probe.  When on (nonzero),
+ * every CTA of the tensor-core kernels launched after the call (attention and
+ * full-vocabulary LSE), once its MMA warp has issued its first MMAs, also
+ * waits on an mbarrier that nothing completes, as a stalled pipeline would
+ * leave it.  That wait is bounded like every other: with the bound of
+ * jev_debug_set_wait_limit cut short it runs out, raises
+ * JEV_DEV_WAIT_TIMEOUT, and the CTA winds down with loads and MMAs in flight,
+ * draining them before it exits; outputs are undefined.  Under the default
+ * bound each CTA waits about a second.  Off (0) by default; process-wide.
+ * Always JEV_OK.  No page has a counterpart.
+ */
+jev_status jev_debug_set_wait_probe(int32_t on);
+
 #ifdef __cplusplus
 }
 #endif

@@ -164,10 +164,13 @@ def test_fma_pipe_exp2_against_cuda_exp2(jev):
 
 def test_short_wait_limit_flags_a_timeout_and_leaves_the_context_usable(jev):
     """Failure detection without a GPU fault: with the tensor-core kernels'
-    wait bound cut to 256 cycles on an ordinary problem, waits run out.  Each
-    call must set JEV_DEV_WAIT_TIMEOUT and return (its CTAs drain the loads
-    and MMAs they issued before exiting), and the next call with the default
-    bound must reproduce the earlier result exactly."""
+    wait bound cut to 256 cycles and the probe on (each CTA's MMA warp, with
+    its first MMAs issued, also waits on a barrier that nothing completes, as
+    a stalled pipeline would leave it), that wait runs out on an ordinary
+    problem.  Each call must set JEV_DEV_WAIT_TIMEOUT and return (its CTAs
+    drain the loads and MMAs they issued before exiting), and the next call
+    with the probe off and the default bound must reproduce the earlier result
+    exactly."""
     c = _case([17, 3, 40, 9, 25], seed=8, Lp=1024, Hq=28, Hkv=4)
     args = [dev(x) for x in (c.q, c.k_pre, c.v_pre, c.k_suf, c.v_suf)] + [dev(c.cu_seqlens)]
     desc = jev.make_attn_desc(5, 1024, 28, 4, 128, int(c.cu_seqlens[-1]), jev.JEV_BF16)
@@ -182,6 +185,7 @@ def test_short_wait_limit_flags_a_timeout_and_leaves_the_context_usable(jev):
     ref_lse = jev.jev_vocab_lse(h, W, workspace=lws).clone()
     assert jev.jev_check_device_status(lws) == 0
     jev.jev_debug_set_wait_limit(256)
+    jev.jev_debug_set_wait_probe(True)
     try:
         for _ in range(2):
             jev.jev_prefix_suffix_attn(*args, workspace=ws)
@@ -189,6 +193,7 @@ def test_short_wait_limit_flags_a_timeout_and_leaves_the_context_usable(jev):
             jev.jev_vocab_lse(h, W, workspace=lws)
             assert jev.jev_check_device_status(lws) & jev.JEV_DEV_WAIT_TIMEOUT
     finally:
+        jev.jev_debug_set_wait_probe(False)
         jev.jev_debug_set_wait_limit(0)
     o, l = jev.jev_prefix_suffix_attn(*args, workspace=ws)
     assert jev.jev_check_device_status(ws) == 0

@@ -103,6 +103,43 @@ def test_many_tokens_at_d64_sampled(jev, dtype):
     check_attn(out[rows[:, 0], rows[:, 1]], lse[rows[:, 0], rows[:, 1]], ref_o, ref_l, dtype, "many tokens d64")
 
 
+def _scale_rows(a, lo, hi, f, dtype):
+    """a[lo:hi] *= f, on the host arrays both sides read (bf16 as its bits)."""
+    a = a.copy()
+    if dtype == synth.BF16:
+        a[lo:hi] = synth.f32_to_bf16_bits(synth.bf16_bits_to_f32(a[lo:hi]) * np.float32(f))
+    else:
+        a[lo:hi] *= np.float32(f)
+    return a
+
+
+@pytest.mark.parametrize("dtype", [synth.BF16, synth.F32])
+@pytest.mark.parametrize("splits", [0, 1])
+def test_running_max_jumps_between_key_tiles(jev, dtype, splits):
+    """Scores that grow from key tile to key tile: prefix keys 128..383 scaled
+    by 3, keys from 384 on and every suffix key by 6, so that in about half of
+    the rows the maximum jumps past the softmax's lazy threshold (8 in log2
+    units) at a tile boundary, some rows twice.  The running max must move and
+    O be rescaled, and tiles whose scores fall back must not move it.  Every
+    element against the oracle, split and unsplit.  The bf16 path stores the
+    rotated queries and keys in bf16, and a score's rounding error grows with
+    the size of its key: with keys up to 6 times those of the N(0, 1) cases
+    the bf16 tolerances here are 4 times theirs (a rescale that went wrong
+    would be off by a factor of 2^8 or more)."""
+    cfg = synth.FlatConfig("jump", dtype, 520, 5, 1, 1, 8, 2, 128, 16, 32, 2, 3, seed=41)
+    c = synth.flat_case(cfg, with_lm_head=False, lengths=np.array([3, 40, 1, 150, 9], np.int32))
+    c.k_pre = _scale_rows(_scale_rows(c.k_pre, 128, 384, 3.0, dtype), 384, 520, 6.0, dtype)
+    c.k_suf = _scale_rows(c.k_suf, 0, c.T, 6.0, dtype)
+    out, lse = run_flat(jev, c, num_splits=splits)
+    ref_o, ref_l = oracle.prefix_suffix_attn(c.q, c.k_pre, c.v_pre, c.k_suf, c.v_suf, c.cu_seqlens)
+    assert ref_l.max() > 10.0  # the later tiles dominate: far above the first tile's scores
+    tol = TOL[dtype] if dtype == synth.F32 else {k: 4 * v for k, v in TOL[dtype].items()}
+    err = np.abs(out - ref_o)
+    assert np.all(np.isfinite(out))
+    assert err.max() <= tol["max_abs"] and err.mean() <= tol["mean_abs"], (err.max(), err.mean())
+    assert np.abs(lse - ref_l).max() <= tol["lse"], np.abs(lse - ref_l).max()
+
+
 EDGE = [
     # dtype, Lp, lens, Hq, Hkv, d, splits, pos_offset, head_map
     (synth.BF16, 300, [1, 7, 0, 33, 130], 8, 2, 128, 0, -1, None),

@@ -333,7 +333,7 @@ def a_producer(segs, drain, prefetch=True):
     yield ("final",)
 
 
-def a_mma(segs, drain):
+def a_mma(segs, drain, probe=False):
     J, ok = 0, True
     for k, n in enumerate(segs):
         if not ok:
@@ -345,6 +345,10 @@ def a_mma(segs, drain):
                 for i in range(2):
                     yield ("mma",)
                     yield ("commit", f"s_full{i}")
+        if ok and k == 0 and probe:
+            # the failure-detection probe: a barrier that nothing completes,
+            # waited on with the first MMAs in flight (only a timeout ends it)
+            ok = yield ("wait", "probe", 0, True)
         for j in range(n):
             if not ok:
                 break
@@ -453,6 +457,11 @@ def _async_run(threads, bars, group_of, seed, p_timeout):
             moves.append(("tma_done", None))
         if tc_queue:
             moves.append(("tc_step", None))
+        if not moves and p_timeout > 0:
+            # nothing can move until time passes: a bounded wait runs out
+            # (with timeouts off, a stall here is reported as a deadlock)
+            moves = [("timeout", n) for n in live
+                     if cur[n][0] == "wait" and cur[n][3] and not state["abort"]]
         if not moves:
             return "deadlock: " + ", ".join(f"{n}@{cur[n]}" for n in live)
         kind, n = rng.choice(moves)
@@ -492,12 +501,12 @@ def _async_run(threads, bars, group_of, seed, p_timeout):
     return "step limit"
 
 
-def run_abort(segs, drain, seed, p_timeout=0.02):
+def run_abort(segs, drain, seed, p_timeout=0.02, probe=False):
     bars = {"q_full": Bar(2), "q_empty": Bar(1), "s_full0": Bar(1), "s_full1": Bar(1), "drain": Bar(1),
-            "p_full0": Bar(SOFT), "p_full1": Bar(SOFT), "o_full0": Bar(1), "o_full1": Bar(1)}
+            "p_full0": Bar(SOFT), "p_full1": Bar(SOFT), "o_full0": Bar(1), "o_full1": Bar(1), "probe": Bar(1)}
     for s in range(NS):
         bars[f"k_full{s}"], bars[f"v_full{s}"], bars[f"kv_empty{s}"] = Bar(1), Bar(1), Bar(1)
-    threads = {"producer": a_producer(segs, drain), "mma": a_mma(segs, drain)}
+    threads = {"producer": a_producer(segs, drain), "mma": a_mma(segs, drain, probe)}
     for i in range(2):
         for t in range(SOFT):
             threads[f"soft{i}.{t}"] = a_softmax(segs, i)
@@ -516,6 +525,15 @@ ABORT_PATTERNS = [[5], [3, 2], [17, 9], [1, 1, 1], [4, 1, 4, 1], [2, 3]]
 def test_timeout_path_drains_before_exit(segs):
     for seed in range(300):
         msg = run_abort(segs, drain=True, seed=seed)
+        assert msg is None, f"seed {seed}: {msg}"
+
+
+@pytest.mark.parametrize("segs", ABORT_PATTERNS, ids=["-".join(map(str, p)) for p in ABORT_PATTERNS])
+def test_probe_timeout_drains_before_exit(segs):
+    # with the probe on, the run always ends in a timeout (nothing completes
+    # the probe's barrier); the CTA must still exit with nothing in flight
+    for seed in range(200):
+        msg = run_abort(segs, drain=True, seed=seed, p_timeout=0.05, probe=True)
         assert msg is None, f"seed {seed}: {msg}"
 
 
