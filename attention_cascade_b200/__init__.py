@@ -47,7 +47,8 @@ class jev_attn_desc(C.Structure):
 class jev_attn_plan(C.Structure):
     _fields_ = [("kernel", C.c_int32), ("n_tiles", C.c_int32), ("units_per_tile", C.c_int32), ("n_ctas", C.c_int32),
                 ("full_waves", C.c_int32), ("tail0", C.c_int32), ("tail_ctas", C.c_int32), ("split", C.c_int32),
-                ("tail_units", C.c_int64), ("simt_splits", C.c_int32), ("split_len", C.c_int32)]
+                ("tail_units", C.c_int64), ("simt_splits", C.c_int32), ("split_len", C.c_int32),
+                ("tile_rows", C.c_int32)]
 
 
 class jev_readout_desc(C.Structure):
@@ -460,6 +461,15 @@ _lib.jev_debug_set_wait_limit.restype = C.c_int
 def jev_debug_set_wait_limit(cycles: int):
     """Bound of the tensor-core kernels' mbarrier waits for later launches (0: the default)."""
     _check(_lib.jev_debug_set_wait_limit(int(cycles)), "jev_debug_set_wait_limit")
+
+
+_lib.jev_debug_set_tc_tile_rows.argtypes = [C.c_int32]
+_lib.jev_debug_set_tc_tile_rows.restype = C.c_int
+
+
+def jev_debug_set_tc_tile_rows(rows: int):
+    """Rows per tensor-core work tile for later plans: 128 or 256 forces a kernel, 0 lets the plan choose."""
+    _check(_lib.jev_debug_set_tc_tile_rows(int(rows)), "jev_debug_set_tc_tile_rows")
 
 
 _lib.jev_debug_set_wait_probe.argtypes = [C.c_int32]

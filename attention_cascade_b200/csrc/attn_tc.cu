@@ -41,13 +41,13 @@
 #include <cuda.h>
 #include <math_constants.h>
 
-#include "kernels.h"
-#include "tc_ptx.cuh"
+#include "attn_tc_common.cuh"
 
 namespace jev {
 namespace {
 
 using namespace tc;
+using namespace tca;
 
 constexpr int kBM = 128;  // rows per Q tile (TMEM lanes)
 constexpr int kBN = 128;  // keys per K/V tile
@@ -93,177 +93,6 @@ struct Shared {
   uint32_t tmem_base;
   int abort;
 };
-
-__device__ __forceinline__ void named_sync(int id, int count) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
-// named barrier that also ANDs a flag over its threads, so that they all
-// leave with the same answer
-__device__ __forceinline__ bool named_sync_and(int id, int count, bool v) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred pi, po;\n\t"
-      "setp.ne.u32 pi, %1, 0;\n\t"
-      "bar.red.and.pred po, %2, %3, pi;\n\t"
-      "selp.u32 %0, 1, 0, po;\n\t}"
-      : "=r"(r)
-      : "r"((uint32_t)v), "r"(id), "r"(count)
-      : "memory");
-  return r != 0;
-}
-
-// Bounded wait (limit: AttnArgs::wait_cycles); once any wait of the CTA has
-// run out, the others give up at their first unsatisfied check.
-__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort, int32_t* status,
-                                         long long limit) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const long long t0 = clock64();
-  for (;;) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if (*abort) return false;
-    if (clock64() - t0 > limit) {
-      *abort = 1;
-      raise_flag(status, JEV_DEV_WAIT_TIMEOUT);
-      return false;
-    }
-  }
-}
-
-// The failure-detection probe: a bounded wait on a barrier that nothing
-// completes.  It runs out after the wait bound (checking the clock at least
-// every microsecond) and winds the CTA down like any other timeout.
-__device__ __forceinline__ bool probe_wait(uint32_t bar, volatile int* abort, int32_t* status, long long limit) {
-  const long long t0 = clock64();
-  for (;;) {
-    if (mbar_try_wait_hint(bar, 0, 1000)) return true;
-    if (*abort) return false;
-    if (clock64() - t0 > limit) {
-      *abort = 1;
-      raise_flag(status, JEV_DEV_WAIT_TIMEOUT);
-      return false;
-    }
-  }
-}
-
-// Wait on the exit path: bounded, but blind to the abort flag, so that a CTA
-// that is winding down still sees every load it armed land and every MMA it
-// issued complete before it frees TMEM and exits.  Such work completes within
-// microseconds; running out of the bound only raises the flag.
-constexpr long long kDrainCycles = 1LL << 28;
-__device__ __forceinline__ void drain_bar(uint32_t bar, uint32_t parity, int32_t* status) {
-  const long long t0 = clock64();
-  while (!mbar_try_wait(bar, parity)) {
-    if (clock64() - t0 > kDrainCycles) {
-      raise_flag(status, JEV_DEV_WAIT_TIMEOUT);
-      return;
-    }
-  }
-}
-
-// Bounded wait taken by a whole warp: every lane polls, and all take lane 0's
-// answer, so that the warp stays converged for the elected issue that follows.
-__device__ __forceinline__ bool wait_bar_w(uint32_t bar, uint32_t parity, volatile int* abort, int32_t* status,
-                                           long long limit) {
-  return __shfl_sync(0xffffffffu, wait_bar(bar, parity, abort, status, limit), 0);
-}
-
-__device__ __forceinline__ int warp_min_i(int v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = min(v, __shfl_xor_sync(0xffffffffu, v, o));
-  return v;
-}
-
-__device__ __forceinline__ int warp_max_i(int v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(0xffffffffu, v, o));
-  return v;
-}
-
-// The suffix keys any row of the work tile may see: from the lowest window
-// start to the highest last key (a tree row's last key is its own token).
-__device__ __forceinline__ void tile_window(const AttnArgs& a, int m0, int lane, int& lo, int& hi) {
-  const int m_end = min(m0 + 2 * kBM, a.M);
-  const int t0 = m0 / a.G, t1 = (m_end - 1) / a.G;
-  const bool tree = a.key_end != nullptr;
-  int mn = INT_MAX, mx = -1;
-  for (int t = t0 + lane; t <= t1; t += 32) {
-    const TokInfo inf = a.info[t];
-    if (inf.node < 0) continue;
-    mn = min(mn, inf.seg_start);
-    mx = max(mx, tree ? t : inf.last);
-  }
-  lo = warp_min_i(mn);
-  hi = warp_max_i(mx);
-}
-
-// One segment of a CTA's unit range: units [ua, ub) of work tile w.
-struct Segment {
-  int w, ua, ub;
-  int g, m0;
-  int n_pre, n;   // prefix key tiles of the segment, key tiles in total
-  int lo;         // first suffix key of the window (when the segment holds the suffix unit)
-  bool complete;  // the segment is the whole tile: write the final output
-  int slot;       // partial slot when not complete
-};
-static_assert(2 * sizeof(Segment) <= 128, "segment ring");
-
-// A CTA's segments: first its whole tiles (k < full_waves: tile c + k*n_ctas),
-// then its tail units.  Every role visits them in the same order and derives
-// the same description (the window takes one warp-wide reduction).
-struct SegIter {
-  int k;                 // segment index
-  long long u, u_end;    // tail units still to visit
-};
-
-__device__ __forceinline__ bool seg_next(const AttnArgs& a, int c, SegIter& it, int& w, int& ua, int& ub, bool& tail) {
-  if (it.k < a.full_waves) {
-    w = c + it.k * a.n_ctas;
-    ua = 0;
-    ub = a.P;
-    tail = false;
-    return true;
-  }
-  if (it.u >= it.u_end) return false;
-  const int wt = (int)(it.u / a.P);
-  const long long t0 = (long long)wt * a.P;
-  w = a.tail0 + wt;
-  ua = (int)(it.u - t0);
-  ub = (int)(min(it.u_end, t0 + a.P) - t0);
-  tail = true;
-  it.u = t0 + ub;
-  return true;
-}
-
-__device__ __forceinline__ Segment make_segment(const AttnArgs& a, int c, int w, int ua, int ub, bool tail, int lane) {
-  Segment sg;
-  sg.w = w;
-  sg.ua = ua;
-  sg.ub = ub;
-  const long long t0 = (long long)(w - a.tail0) * a.P;  // tail unit of the tile's first unit
-  sg.g = sg.w / a.n_pairs;
-  sg.m0 = (sg.w - sg.g * a.n_pairs) * 2 * kBM;
-  sg.n_pre = max(0, min(sg.ub, a.n_pre) - sg.ua);
-  int n_suf = 0;
-  sg.lo = 0;
-  if (sg.ub == a.P) {
-    int lo, hi;
-    tile_window(a, sg.m0, lane, lo, hi);
-    sg.lo = lo;
-    n_suf = lo <= hi ? (hi - lo + kBN) / kBN : 0;
-  }
-  sg.n = sg.n_pre + n_suf;
-  // A segment always has a key tile: the q_empty / p_full handshake that
-  // keeps the roles within one q_full phase of each other runs per key tile.
-  // n would be 0 only for a suffix-only unit whose rows are all skipped
-  // (malformed input); its one tile is then fully masked and nothing is written.
-  if (sg.n == 0) {
-    sg.lo = 0;
-    sg.n = 1;
-  }
-  sg.complete = sg.ua == 0 && sg.ub == a.P;
-  sg.slot = (tail && tc_unit_begin(a, c) >= t0) ? 2 * c : 2 * c + 1;
-  return sg;
-}
 
 template <int D, bool TREE>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -352,7 +181,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool tl0;
       if (seg_next(a, cta, it0, w0, ua0, ub0, tl0)) {
         pre0 = min(max(0, min(ub0, a.n_pre) - ua0), C::kNS);
-        const int g0 = w0 / a.n_pairs;
+        const int g0 = w0 / a.n_mt;
         for (int j = 0; j < pre0; ++j) {
           const uint32_t ks = sbase + C::kOffK + j * C::kKVBytes, vs = sbase + C::kOffV + j * C::kKVBytes;
           mbar_expect_tx_w(B.k_full + 8 * j, C::kKVBytes);
@@ -371,7 +200,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool stail;
     for (; ok && seg_next(a, cta, it, sw, sua, sub, stail); ++k, ++it.k) {
       // The Q tile goes first: it needs only the tile's group and rows.
-      const int qg = sw / a.n_pairs, qm0 = (sw - qg * a.n_pairs) * 2 * kBM;
+      const int qg = sw / a.n_mt, qm0 = (sw - qg * a.n_mt) * 2 * kBM;
       if (k > 0 && !wait_bar_w(B.q_empty, (k - 1) & 1, abort, a.status, a.wait_cycles)) ok = false;
       if (ok) {
         mbar_expect_tx_w(B.q_full, 2 * C::kQBytes);
@@ -382,7 +211,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // The description (for the suffix unit, its key window: a warp-wide read
       // of token info) is published with q_full's second arrival.
-      const Segment sg = make_segment(a, cta, sw, sua, sub, stail, lane);
+      const Segment sg = make_segment<2 * kBM>(a, cta, sw, sua, sub, stail, lane);
       if (ok) {
         if (lane == 0) {
           seg_sm[k & 1] = sg;
@@ -785,8 +614,8 @@ __global__ void __launch_bounds__(256, 4) tc_fixup_kernel(const AttnArgs a) {
   const int c_lo = tc_cta_of(a, t0), c_hi = tc_cta_of(a, t0 + a.P - 1);
   if (c_lo == c_hi) return;  // one CTA finished this tile and wrote it
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int r = blockIdx.y * kFixRows + lane;  // row within the 256-row tile
-  const int g = w / a.n_pairs, m = (w - g * a.n_pairs) * 2 * kBM + r;
+  const int r = blockIdx.y * kFixRows + lane;  // row within the work tile
+  const int g = w / a.n_mt, m = (w - g * a.n_mt) * a.tile_rows + r;
   if (m >= a.M) return;
   const int nseg = c_hi - c_lo + 1;
   // CTA c_lo holds this tile as its first segment only if its range starts here
@@ -810,8 +639,8 @@ __global__ void __launch_bounds__(256, 4) tc_fixup_kernel(const AttnArgs a) {
       lv[e] = -CUDART_INF_F;
       if (s0 + e < nseg) {
         const int slot = slot_of(s0 + e);
-        lv[e] = a.l_part[(size_t)slot * 2 * kBM + r];
-        const float4* src = op + (size_t)slot * (2 * kBM / 32) * (D / 4) * 32;
+        lv[e] = a.l_part[(size_t)slot * a.tile_rows + r];
+        const float4* src = op + (size_t)slot * (a.tile_rows / 32) * (D / 4) * 32;
 #pragma unroll
         for (int c = 0; c < kCols; ++c) ov[e][c] = src[c * 8 * 32];
       } else {
@@ -870,47 +699,6 @@ __global__ void exp2_selftest_kernel(const float* x, float* y, int n) {
 }
 
 // ---------------------------------------------------------------- host side
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  static bool tried = false;
-  if (!tried) {
-    tried = true;
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult qr;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &qr) == cudaSuccess &&
-        qr == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-    else
-      cudaGetLastError();
-  }
-  return fn;
-}
-
-// bf16 rows of `inner` elements, `rows` rows `stride` bytes apart; 64 x 128 boxes, 128-byte swizzle
-bool map_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t stride) {
-  cuuint64_t dims[2] = {inner, rows};
-  cuuint64_t strides[1] = {stride};
-  cuuint32_t box[2] = {64, 128};
-  cuuint32_t es[2] = {1, 1};
-  return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-bool map_q(CUtensorMap* m, const void* base, int D, int M, int Hkv) {
-  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)M, (cuuint64_t)Hkv};
-  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)M * D * 2};
-  cuuint32_t box[3] = {64, 128, 1};
-  cuuint32_t es[3] = {1, 1, 1};
-  return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <int D, bool TREE>
 cudaError_t launch_dt(const AttnArgs& a, cudaStream_t s) {
   static bool attr = false;
@@ -921,16 +709,7 @@ cudaError_t launch_dt(const AttnArgs& a, cudaStream_t s) {
     attr = true;
   }
   CUtensorMap mq, mkp, mvp, mks, mvs;
-  memset(&mkp, 0, sizeof mkp);
-  memset(&mvp, 0, sizeof mvp);
-  const uint64_t row = (uint64_t)a.Hkv * D * 2;
-  if (!map_q(&mq, a.q_rot, D, a.M, a.Hkv)) return cudaErrorInvalidValue;
-  if (a.Lp > 0 && (!map_2d(&mkp, a.k_pre, (uint64_t)a.Hkv * D, a.Lp, row) ||
-                   !map_2d(&mvp, a.v_pre, (uint64_t)a.Hkv * D, a.Lp, row)))
-    return cudaErrorInvalidValue;
-  if (!map_2d(&mks, a.k_rot, (uint64_t)a.Hkv * D, a.key_rows, row) ||
-      !map_2d(&mvs, a.v_suf, (uint64_t)a.Hkv * D, a.key_rows, row))
-    return cudaErrorInvalidValue;
+  if (!attn_maps(a, D, &mq, &mkp, &mvp, &mks, &mvs)) return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute pdl[1];
   pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -985,7 +764,7 @@ cudaError_t launch_tc_fixup(const AttnArgs& a, cudaStream_t s) {
   // the most segments any tail tile is split into
   const long long max_segs = ((long long)a.P * a.tail_ctas + a.U - 1) / a.U + 1;
   const bool many = max_segs > 4;
-  cfg.gridDim = dim3(a.n_tiles - a.tail0, 2 * kBM / kFixRows, 1);
+  cfg.gridDim = dim3(a.n_tiles - a.tail0, a.tile_rows / kFixRows, 1);
   cfg.blockDim = dim3(256);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = s;
@@ -997,6 +776,7 @@ cudaError_t launch_tc_fixup(const AttnArgs& a, cudaStream_t s) {
 
 cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t s) {
   if (a.M == 0 || a.n_ctas == 0) return cudaSuccess;
+  if (a.tile_rows == 128) return launch_attn_tc1(a, s);
   const bool tree = a.key_end != nullptr;
   if (a.d == 128) return tree ? launch_dt<128, true>(a, s) : launch_dt<128, false>(a, s);
   return tree ? launch_dt<64, true>(a, s) : launch_dt<64, false>(a, s);

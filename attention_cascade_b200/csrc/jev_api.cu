@@ -46,6 +46,7 @@ std::atomic<long long> g_launches{0};
 constexpr long long kDefaultWaitCycles = 1LL << 31;
 std::atomic<long long> g_wait_cycles{kDefaultWaitCycles};
 std::atomic<int> g_wait_probe{0};
+std::atomic<int> g_tile_rows{0};  // 0: rows per tensor-core work tile as the plan chooses, else 128 or 256
 
 int name_id(const char* n) {
   for (size_t i = 0; i < g_names.size(); ++i)
@@ -135,9 +136,12 @@ bool use_tc(const jev_attn_desc* d) {
   return !forced && d->dtype == JEV_BF16 && attn_tc_supported(d->d);
 }
 
-// Work plan.  Tensor-core kernel: work tiles of 256 stacked rows of one kv
-// group, each with P = ceil(Lp/128) + 1 units (prefix key tiles + the suffix
-// window).  n_ctas persistent CTAs first take full_waves rounds of whole
+// Work plan.  Tensor-core kernel: work tiles of tile_rows stacked rows of one
+// kv group, each with P = ceil(Lp/128) + 1 units (prefix key tiles + the
+// suffix window).  256-row tiles run on the two-Q-tile kernel, which is the
+// faster per unit once there are several waves of tiles; 128-row tiles on the
+// one-Q-tile kernel, chosen when 256-row tiles would not fill one wave of
+// CTAs (twice the tiles, so fewer of them are split and merged).  n_ctas persistent CTAs first take full_waves rounds of whole
 // tiles; the remaining tail tiles' units are spread evenly over tail_ctas of
 // them, so a tail tile may be split across CTAs and merged afterwards.
 // num_splits: 1 -> no tile split (one CTA per tile up to one per SM),
@@ -147,18 +151,19 @@ bool use_tc(const jev_attn_desc* d) {
 struct Plan {
   int S, split_len, M, G;
   bool tc, split;
-  int n_pairs, n_tiles, n_pre, P, n_ctas, full_waves, tail0, tail_ctas;
+  int tile_rows, n_mt, n_tiles, n_pre, P, n_ctas, full_waves, tail0, tail_ctas;
   long long U;
 };
 
 // Estimated time (microseconds) of the tensor-core schedule: the busiest
 // CTA's units and segments plus the merge of split tiles.  Calibrated on
-// B200 at d = 128: a unit (256 rows x 128 keys) costs about 2.5 us, the
+// B200 at d = 128: a unit of 256 rows x 128 keys costs about 2.5 us (one of
+// 128 rows, on the one-Q-tile kernel, about 0.6 of that), the
 // first segment of a CTA about 8 us of pipeline fill and drain, each later
 // one about 3 us, a segment left partial about 2 us more (fp32 output), and
 // the merge about 5 us plus 0.7 us per eight segments of one tile.
-double tc_schedule_us(int P, int d, int full_waves, long long U, int tail_ctas) {
-  const double unit_us = 4.0 * 256 * 128 * d / 6.8e12 * 1e6;
+double tc_schedule_us(int P, int d, int full_waves, long long U, int tail_ctas, int tile_rows) {
+  const double unit_us = (tile_rows == 256 ? 1.0 : 0.6) * 4.0 * 256 * 128 * d / 6.8e12 * 1e6;
   const double first_us = 8.0, seg_us = 3.0, part_us = 2.0;
   double worst = 0.0;
   bool split = false;
@@ -192,8 +197,11 @@ Plan compute_plan(const jev_attn_desc* d, int T, int kernel, int sms_hint) {
   const int ktiles = (d->Lp + 127) / 128;
   p.tc = kernel < 0 ? use_tc(d) : kernel == 1;
   if (p.tc) {
-    p.n_pairs = (p.M + 255) / 256;
-    p.n_tiles = p.n_pairs * d->Hkv;
+    const int sms0 = std::max(1, sms_hint > 0 ? sms_hint : num_sms());
+    const int forced_rows = g_tile_rows.load();
+    p.tile_rows = forced_rows ? forced_rows : ((p.M + 255) / 256 * d->Hkv < sms0 ? 128 : 256);
+    p.n_mt = (p.M + p.tile_rows - 1) / p.tile_rows;
+    p.n_tiles = p.n_mt * d->Hkv;
     p.n_pre = ktiles;
     p.P = ktiles + 1;
     const int s = d->num_splits;
@@ -217,7 +225,7 @@ Plan compute_plan(const jev_attn_desc* d, int T, int kernel, int sms_hint) {
       p.n_ctas = p.tail_ctas = (int)std::max(1LL, std::min((long long)p.n_tiles * s, U));
     } else {
       no_split();
-      double best = tc_schedule_us(p.P, d->d, p.full_waves, p.U, p.tail_ctas);
+      double best = tc_schedule_us(p.P, d->d, p.full_waves, p.U, p.tail_ctas, p.tile_rows);
       // Spread the tail (every tile when there are fewer tiles than SMs)
       // over more CTAs, up to one per SM; keep the cheapest estimate.
       const int fw = p.n_tiles >= sms ? p.n_tiles / sms : 0;
@@ -226,7 +234,7 @@ Plan compute_plan(const jev_attn_desc* d, int T, int kernel, int sms_hint) {
       // a tile spread over many CTAs costs a long merge; keep it within 64 segments
       const long long t_max = std::min<long long>({(long long)sms, U, (long long)std::max(1, r) * 64});
       for (long long t = std::max(1, r); r > 0 && t <= t_max; ++t) {
-        const double e = tc_schedule_us(p.P, d->d, fw, U, (int)t);
+        const double e = tc_schedule_us(p.P, d->d, fw, U, (int)t, p.tile_rows);
         if (e < best * 0.98) {
           best = e;
           p.full_waves = fw;
@@ -265,16 +273,16 @@ Plan compute_plan(const jev_attn_desc* d, int T, int kernel, int sms_hint) {
 // every call (and every workspace query) needs the plan.
 Plan plan_of(const jev_attn_desc* d, int T, int kernel = -1, int sms_hint = 0) {
   struct Key {
-    int T, Lp, Hq, Hkv, d, dtype, num_splits, kernel, sms;
+    int T, Lp, Hq, Hkv, d, dtype, num_splits, kernel, sms, rows;
     bool operator==(const Key& o) const {
       return T == o.T && Lp == o.Lp && Hq == o.Hq && Hkv == o.Hkv && d == o.d && dtype == o.dtype &&
-             num_splits == o.num_splits && kernel == o.kernel && sms == o.sms;
+             num_splits == o.num_splits && kernel == o.kernel && sms == o.sms && rows == o.rows;
     }
   };
   struct Hash {
     size_t operator()(const Key& k) const {
       size_t h = 1469598103934665603ull;
-      for (int v : {k.T, k.Lp, k.Hq, k.Hkv, k.d, k.dtype, k.num_splits, k.kernel, k.sms})
+      for (int v : {k.T, k.Lp, k.Hq, k.Hkv, k.d, k.dtype, k.num_splits, k.kernel, k.sms, k.rows})
         h = (h ^ (size_t)(uint32_t)v) * 1099511628211ull;
       return h;
     }
@@ -283,7 +291,7 @@ Plan plan_of(const jev_attn_desc* d, int T, int kernel = -1, int sms_hint = 0) {
   static std::unordered_map<Key, Plan, Hash> cache;
   const int kern = kernel < 0 ? (use_tc(d) ? 1 : 0) : kernel;
   const int sms = sms_hint > 0 ? sms_hint : num_sms();
-  const Key key{T, d->Lp, d->Hq, d->Hkv, d->d, (int)d->dtype, d->num_splits, kern, sms};
+  const Key key{T, d->Lp, d->Hq, d->Hkv, d->d, (int)d->dtype, d->num_splits, kern, sms, g_tile_rows.load()};
   {
     std::lock_guard<std::mutex> lk(mu);
     auto it = cache.find(key);
@@ -313,7 +321,7 @@ Layout layout_of(const jev_attn_desc* d, int T, const Plan& p, int n_nodes, bool
   L.opart = off;
   L.lpart = off;
   if (p.tc && p.split) {
-    const size_t rows = (size_t)2 * p.n_ctas * 256;  // two partial segments per CTA at most
+    const size_t rows = (size_t)2 * p.n_ctas * p.tile_rows;  // two partial segments per CTA at most
     L.opart = off; off += up256(rows * d->d * 4);
     L.lpart = off; off += up256(rows * 4);
   } else if (!p.tc && p.S > 1) {
@@ -403,7 +411,7 @@ jev_status attention_core(const jev_attn_desc* d, int T, const Plan& p, const La
   a.T = T; a.M = p.M; a.Lp = d->Lp; a.Hq = d->Hq; a.Hkv = d->Hkv; a.G = p.G; a.d = d->d;
   a.S = p.S; a.split_len = p.split_len;
   a.scale_log2 = scale_log2_of(d);
-  a.n_pairs = p.n_pairs; a.n_tiles = p.n_tiles; a.n_pre = p.n_pre; a.P = p.P; a.n_ctas = p.n_ctas; a.U = p.U;
+  a.tile_rows = p.tile_rows; a.n_mt = p.n_mt; a.n_tiles = p.n_tiles; a.n_pre = p.n_pre; a.P = p.P; a.n_ctas = p.n_ctas; a.U = p.U;
   a.full_waves = p.full_waves; a.tail0 = p.tail0; a.tail_ctas = p.tail_ctas;
   a.wait_cycles = g_wait_cycles.load();
   a.wait_probe = g_wait_probe.load();
@@ -461,6 +469,12 @@ int64_t jev_launch_count(void) { return (int64_t)g_launches.load(); }
 jev_status jev_debug_set_wait_limit(int64_t cycles) {
   if (cycles < 0) return fail(JEV_ERR_INVALID_ARG, "wait limit must be >= 0");
   g_wait_cycles.store(cycles == 0 ? kDefaultWaitCycles : (long long)cycles);
+  return JEV_OK;
+}
+
+jev_status jev_debug_set_tc_tile_rows(int32_t rows) {
+  if (rows != 0 && rows != 128 && rows != 256) return fail(JEV_ERR_INVALID_ARG, "tile rows must be 0, 128 or 256");
+  g_tile_rows.store(rows);
   return JEV_OK;
 }
 
@@ -525,6 +539,7 @@ jev_status jev_prefix_suffix_attn_plan(const jev_attn_desc* d, int32_t kernel, i
   r.n_tiles = p.n_tiles; r.units_per_tile = p.P; r.n_ctas = p.n_ctas; r.full_waves = p.full_waves;
   r.tail0 = p.tail0; r.tail_ctas = p.tail_ctas; r.split = p.split ? 1 : 0; r.tail_units = p.U;
   r.simt_splits = p.S; r.split_len = p.split_len;
+  r.tile_rows = p.tc ? p.tile_rows : 0;
   *out = r;
   return JEV_OK;
 }

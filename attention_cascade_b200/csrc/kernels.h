@@ -60,14 +60,15 @@ struct AttnArgs {
   int T, M, Lp, Hq, Hkv, G, d, S, split_len;  // split_len: prefix keys per split (CUDA-core kernel: a multiple of 32)
   int key_rows;             // rows of k_rot / v_suf
   float scale_log2;         // softmax scale * log2(e)
-  // Tensor-core schedule.  Work tile w = (kv group w / n_pairs, 256-row pair
-  // w % n_pairs) has P = n_pre + 1 units (one per 128-key prefix tile, one for
+  // Tensor-core schedule.  Work tile w = (kv group w / n_mt, tile_rows-row
+  // tile w % n_mt of its stacked rows; 256 rows run on the two-Q-tile kernel,
+  // 128 on the one-Q-tile kernel) has P = n_pre + 1 units (one per 128-key prefix tile, one for
   // the suffix window).  The first full_waves * n_ctas tiles go whole, tile
   // c + k * n_ctas to CTA c; the U units of the remaining (tail) tiles,
   // counted from tile tail0 = full_waves * n_ctas, are spread evenly over the
   // first tail_ctas CTAs: CTA c < tail_ctas owns tail units
   // [c*U/tail_ctas, (c+1)*U/tail_ctas) after its whole tiles.
-  int n_pairs, n_tiles, n_pre, P, n_ctas, full_waves, tail0, tail_ctas;
+  int tile_rows, n_mt, n_tiles, n_pre, P, n_ctas, full_waves, tail0, tail_ctas;
   long long U;
   long long wait_cycles;  // bound of every mbarrier wait (clock cycles)
   int wait_probe;         // failure-detection probe: the MMA warp also waits on a barrier nothing completes
@@ -77,7 +78,8 @@ __host__ __device__ inline long long tc_unit_begin(const AttnArgs& a, int c) { r
 // CTA owning tail unit u: the largest c with tc_unit_begin(c) <= u
 __host__ __device__ inline int tc_cta_of(const AttnArgs& a, long long u) { return (int)(((u + 1) * a.tail_ctas - 1) / a.U); }
 cudaError_t launch_attn_simt(const AttnArgs& a, jev_dtype dt, cudaStream_t s);
-cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t s);  // bf16, d in {64,128}
+cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t s);   // bf16, d in {64,128}; by a.tile_rows:
+cudaError_t launch_attn_tc1(const AttnArgs& a, cudaStream_t s);  // the one-Q-tile kernel (tile_rows 128)
 // merge the partial segments of work tiles that the schedule split across CTAs
 cudaError_t launch_tc_fixup(const AttnArgs& a, cudaStream_t s);
 bool attn_tc_supported(int d);

@@ -99,13 +99,16 @@ size_t jev_prefix_suffix_attn_workspace(const jev_attn_desc* desc);
  * bf16 with d 64 or 128 on sm_100a runs it).  num_sms <= 0 -> the current
  * device's SM count (148 when no device is present); num_sms > 0 plans for
  * that many SMs, as a what-if.  Tensor-core kernel (kernel == 1): stacked query rows of one
- * kv head form work tiles of 256 rows, n_tiles in all, each of
+ * kv head form work tiles of tile_rows rows, n_tiles in all, each of
  * units_per_tile units (one per 128-key prefix tile plus one for the suffix
  * window).  n_ctas persistent CTAs first take full_waves rounds of whole
  * tiles (tile c + k*n_ctas to CTA c); the tail_units units of tiles
  * tail0 .. n_tiles-1 are spread evenly over CTAs 0 .. tail_ctas-1, CTA c
  * owning [c*tail_units/tail_ctas, (c+1)*tail_units/tail_ctas); split != 0
  * when some tile is shared by several CTAs and a merge kernel combines it.
+ * tile_rows is 256 (a kernel with two 128-row Q tiles a CTA) when 256-row
+ * tiles fill at least one wave of num_sms CTAs, else 128 (a kernel with one
+ * Q tile a CTA, for twice as many tiles); 0 for the CUDA-core plan.
  * CUDA-core kernel (kernel == 0): simt_splits prefix splits of split_len
  * keys (a multiple of 32).  Returns the descriptor's error (as jev_prefix_suffix_attn would) or
  * JEV_ERR_INVALID_ARG for a NULL `plan` or a kernel outside -1 .. 1.
@@ -115,6 +118,7 @@ typedef struct {
   int32_t n_tiles, units_per_tile, n_ctas, full_waves, tail0, tail_ctas, split;
   int64_t tail_units;
   int32_t simt_splits, split_len;
+  int32_t tile_rows;       /* tensor-core plan: stacked rows per work tile (128 or 256) */
 } jev_attn_plan;
 jev_status jev_prefix_suffix_attn_plan(const jev_attn_desc* desc, int32_t kernel, int32_t num_sms,
                                       jev_attn_plan* plan);
@@ -467,6 +471,14 @@ int64_t jev_launch_count(void);
  * No page has a counterpart: this is the library's failure detection.
  */
 jev_status jev_debug_set_wait_limit(int64_t cycles);
+
+/*
+ * jev_debug_set_tc_tile_rows — rows per tensor-core work tile for plans made
+ * after the call: 128 or 256 forces the one- or the two-Q-tile attention
+ * kernel, 0 (the default) lets the plan choose (see jev_attn_plan).  For
+ * tests and timing; process-wide.  JEV_ERR_INVALID_ARG for other values.
+ */
+jev_status jev_debug_set_tc_tile_rows(int32_t rows);
 
 /*
  * jev_debug_set_wait_probe — failure-detection probe.  When on (nonzero),

@@ -24,6 +24,16 @@ def pytest_configure(config):
     _builder().build()  # incremental: a no-op when libjev.so is current
 
 
+@pytest.fixture
+def force_tile_rows():
+    """Setter of the rows per tensor-core work tile for the test's calls (128:
+    the one-Q-tile attention kernel, 256: the two-Q-tile one, 0: the plan
+    chooses); the automatic choice is restored afterwards."""
+    import attention_cascade_b200 as jev
+    yield jev.jev_debug_set_tc_tile_rows
+    jev.jev_debug_set_tc_tile_rows(0)
+
+
 @pytest.fixture(scope="session", autouse=True)
 def _build_oracle():
     import oracle

@@ -162,7 +162,8 @@ def test_fma_pipe_exp2_against_cuda_exp2(jev):
     assert (z >= 0).all() and (z < 1e-37).all()
 
 
-def test_short_wait_limit_flags_a_timeout_and_leaves_the_context_usable(jev):
+@pytest.mark.parametrize("rows", [0, 256])
+def test_short_wait_limit_flags_a_timeout_and_leaves_the_context_usable(jev, rows, force_tile_rows):
     """Failure detection without a GPU fault: with the tensor-core kernels'
     wait bound cut to 256 cycles and the probe on (each CTA's MMA warp, with
     its first MMAs issued, also waits on a barrier that nothing completes, as
@@ -171,6 +172,7 @@ def test_short_wait_limit_flags_a_timeout_and_leaves_the_context_usable(jev):
     drain the loads and MMAs they issued before exiting), and the next call
     with the probe off and the default bound must reproduce the earlier result
     exactly."""
+    force_tile_rows(rows)  # 0: 128-row tiles (the one-Q-tile kernel) at this size
     c = _case([17, 3, 40, 9, 25], seed=8, Lp=1024, Hq=28, Hkv=4)
     args = [dev(x) for x in (c.q, c.k_pre, c.v_pre, c.k_suf, c.v_suf)] + [dev(c.cu_seqlens)]
     desc = jev.make_attn_desc(5, 1024, 28, 4, 128, int(c.cu_seqlens[-1]), jev.JEV_BF16)

@@ -113,9 +113,10 @@ def _scale_rows(a, lo, hi, f, dtype):
     return a
 
 
+@pytest.mark.parametrize("rows", [0, 256])
 @pytest.mark.parametrize("dtype", [synth.BF16, synth.F32])
 @pytest.mark.parametrize("splits", [0, 1])
-def test_running_max_jumps_between_key_tiles(jev, dtype, splits):
+def test_running_max_jumps_between_key_tiles(jev, dtype, splits, rows, force_tile_rows):
     """Scores that grow from key tile to key tile: prefix keys 128..383 scaled
     by 3, keys from 384 on and every suffix key by 6, so that in about half of
     the rows the maximum jumps past the softmax's lazy threshold (8 in log2
@@ -126,6 +127,7 @@ def test_running_max_jumps_between_key_tiles(jev, dtype, splits):
     the size of its key: with keys up to 6 times those of the N(0, 1) cases
     the bf16 tolerances here are 4 times theirs (a rescale that went wrong
     would be off by a factor of 2^8 or more)."""
+    force_tile_rows(rows)
     cfg = synth.FlatConfig("jump", dtype, 520, 5, 1, 1, 8, 2, 128, 16, 32, 2, 3, seed=41)
     c = synth.flat_case(cfg, with_lm_head=False, lengths=np.array([3, 40, 1, 150, 9], np.int32))
     c.k_pre = _scale_rows(_scale_rows(c.k_pre, 128, 384, 3.0, dtype), 384, 520, 6.0, dtype)
@@ -156,8 +158,12 @@ EDGE = [
 ]
 
 
+@pytest.mark.parametrize("rows", [0, 256])
 @pytest.mark.parametrize("case", EDGE, ids=[f"e{i}" for i in range(len(EDGE))])
-def test_flat_edge_shapes(jev, case):
+def test_flat_edge_shapes(jev, case, rows, force_tile_rows):
+    # rows 0: the plan's choice (128-row tiles, the one-Q-tile kernel, at these
+    # sizes); 256: the two-Q-tile kernel on the same shapes
+    force_tile_rows(rows)
     dtype, Lp, lens, Hq, Hkv, d, splits, pos_off, hm = case
     cfg = synth.FlatConfig("edge", dtype, Lp, len(lens), 1, 1, Hq, Hkv, d, 16, 32, 2, 3, seed=sum(lens) + Lp)
     c = synth.flat_case(cfg, with_lm_head=False, lengths=np.array(lens, np.int32))
@@ -227,8 +233,10 @@ def _tree_inputs(tc, jev):
     return t, dict(parent=dev(t["parent"]), tok_off=dev(t["tok_off"]), pos0=dev(t["pos0"]))
 
 
+@pytest.mark.parametrize("rows", [0, 256])
 @pytest.mark.parametrize("seed,d,dtype", [(0, 64, synth.BF16), (1, 128, synth.BF16), (2, 64, synth.F32)])
-def test_tree_small_every_element(jev, seed, d, dtype):
+def test_tree_small_every_element(jev, seed, d, dtype, rows, force_tile_rows):
+    force_tile_rows(rows)
     cfg = synth.TreeConfig("t", dtype, 300, 5, 9, 2, 6, 1, 5, 8, 2, d, 64, 500, seed=seed)
     tc = synth.tree_case(cfg, with_lm_head=True)
     t, td = _tree_inputs(tc, jev)
@@ -245,8 +253,10 @@ def test_tree_small_every_element(jev, seed, d, dtype):
     check_readout(lp, ch, ref, cfg.dtype, "tree readout")
 
 
+@pytest.mark.parametrize("rows", [0, 256])
 @pytest.mark.parametrize("shape", ["chain", "zigzag"])
-def test_deep_token_tries_every_element(jev, shape):
+def test_deep_token_tries_every_element(jev, shape, rows, force_tile_rows):
+    force_tile_rows(rows)
     """Tries 12 levels deep and more: a chain of one-token nodes each ending a
     candidate, and a zigzag whose path always continues through the second
     child, so a token's ancestors' keys are not one contiguous range."""
@@ -311,7 +321,8 @@ def test_multi_image_tree(jev):
     check_attn(host_f64(o1), host_f64(l1), ref_o[:n1], ref_l[:n1], cfg.dtype, "first image alone")
 
 
-def test_single_key_tile_segments_keep_the_pipeline_in_step(jev):
+@pytest.mark.parametrize("rows", [128, 256])
+def test_single_key_tile_segments_keep_the_pipeline_in_step(jev, rows, force_tile_rows):
     # Schedules whose CTAs run a segment of one key tile followed by more segments: 64 branches
     # of 32 tokens over a 2048-token prefix at the 7B heads (a one-unit tail segment), and a
     # multi-image tree (empty root, 8 nodes of 416 tokens: many one-tile windows).  The MMA warp
@@ -320,6 +331,7 @@ def test_single_key_tile_segments_keep_the_pipeline_in_step(jev):
     # on an aliased phase.  Five back-to-back calls on one workspace must leave the status word
     # clear, and sampled rows match the oracle.
     import dataclasses
+    force_tile_rows(rows)
     cfg = dataclasses.replace(synth.CONFIGS["qwen25vl_7b"], B=64)
     c = synth.flat_case(cfg, with_lm_head=False, lengths=np.full(64, 32, np.int32))
     desc = jev.make_attn_desc(64, cfg.Lp, cfg.Hq, cfg.Hkv, cfg.d, c.T, jev.JEV_BF16, cfg.theta)

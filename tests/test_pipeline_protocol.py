@@ -413,6 +413,20 @@ def a_softmax(segs, i):
     yield ("final",)
 
 
+def _wait_problem(bars, name, op):
+    """A parity wait that would stall (its barrier has completed two phases past
+    the awaited one) or pass early (the phase before the awaited one is still
+    pending), else None."""
+    if not op or op[0] != "wait":
+        return None
+    done = bars[op[1]].phase
+    if done > op[2] + 1:
+        return f"{name} waits for phase {op[2]} of {op[1]}, which has completed {done}"
+    if done < op[2] and (done & 1) != (op[2] & 1):
+        return f"{name} would pass its wait for phase {op[2]} of {op[1]} with only {done} completed"
+    return None
+
+
 def _async_run(threads, bars, group_of, seed, p_timeout):
     """Random interleaving of roles, in-flight TMA loads and the tensor-core
     queue, with at most one timeout; None when the CTA exits with nothing in
@@ -492,6 +506,12 @@ def _async_run(threads, bars, group_of, seed, p_timeout):
                 return f"TMEM freed and CTA exiting with {len(tma)} loads and {len(tc_queue)} tensor-core ops pending"
             advance(n)
         elif op[0] == "wait":
+            # once the CTA is winding down, an abortable wait that passes early
+            # is harmless (the segment's results are dropped); a drain wait is not
+            if ready(op) and not (op[3] and state["abort"]):
+                msg = _wait_problem(bars, n, op)
+                if msg:
+                    return msg
             advance(n, ready(op))
         else:  # sync / syncand / final: release the whole group together
             members = group_of(op)

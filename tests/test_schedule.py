@@ -80,15 +80,28 @@ SHAPES = [  # (B, T, Lp, Hq, Hkv)
 ]
 
 
+@pytest.fixture
+def tile_rows():
+    """Forces the rows per tensor-core work tile for the test's plans (0: the
+    plan chooses) and restores the automatic choice afterwards."""
+    def force(rows):
+        jev.jev_debug_set_tc_tile_rows(rows)
+    yield force
+    jev.jev_debug_set_tc_tile_rows(0)
+
+
 @pytest.mark.parametrize("shape", SHAPES)
 @pytest.mark.parametrize("num_splits", [0, 1, 2, 3, 7])
 @pytest.mark.parametrize("sms", [148, 132, 7, 1])
-def test_schedule_covers_every_unit_once(shape, num_splits, sms):
+@pytest.mark.parametrize("rows", [0, 128, 256])
+def test_schedule_covers_every_unit_once(shape, num_splits, sms, rows, tile_rows):
     B, T, Lp, Hq, Hkv = shape
+    tile_rows(rows)
     desc = jev.make_attn_desc(B, Lp, Hq, Hkv, 128, T, jev.JEV_BF16, num_splits=num_splits)
     p = jev.jev_prefix_suffix_attn_plan(desc, kernel=1, num_sms=sms)
     assert p["kernel"] == 1
-    assert p["n_tiles"] == -(-T * (Hq // Hkv) // 256) * Hkv
+    assert p["tile_rows"] == (rows or p["tile_rows"]) and p["tile_rows"] in (128, 256)
+    assert p["n_tiles"] == -(-T * (Hq // Hkv) // p["tile_rows"]) * Hkv
     assert p["units_per_tile"] == -(-Lp // 128) + 1
     if num_splits == 1:
         assert p["split"] == 0 and p["n_ctas"] <= sms
@@ -97,13 +110,31 @@ def test_schedule_covers_every_unit_once(shape, num_splits, sms):
     _check(p)
 
 
+def test_tile_rows_choice():
+    """256-row work tiles (the two-Q-tile kernel) when they fill at least one
+    wave of CTAs, else 128-row tiles (the one-Q-tile kernel); 0 for the
+    CUDA-core plan."""
+    def rows(B, Lp, Hq, Hkv, T, sms=148, kernel=1):
+        return jev.jev_prefix_suffix_attn_plan(jev.make_attn_desc(B, Lp, Hq, Hkv, 128, T, jev.JEV_BF16), kernel,
+                                               sms)["tile_rows"]
+    assert rows(128, 4096, 28, 4, 3202) == 256     # 352 tiles of 256 rows
+    assert rows(32, 2048, 28, 4, 707) == 128       # 80 tiles of 256 rows on 148 SMs
+    assert rows(32, 2048, 28, 4, 707, sms=80) == 256
+    assert rows(32, 2048, 28, 4, 707, sms=81) == 128
+    assert rows(8, 1024, 12, 2, 128) == 128
+    assert rows(8, 1024, 12, 2, 128, kernel=0) == 0
+    with pytest.raises(jev.JevError):
+        jev.jev_debug_set_tc_tile_rows(64)
+
+
 def test_auto_schedule_choices():
     # fewer tiles than SMs and a long prefix: every tile is spread over several CTAs
     p = jev.jev_prefix_suffix_attn_plan(jev.make_attn_desc(8, 1024, 12, 2, 128, 138, jev.JEV_BF16), 1, 148)
+    assert p["tile_rows"] == 128
     assert p["full_waves"] == 0 and p["split"] == 1 and p["n_ctas"] > p["n_tiles"]
     # 352 tiles on 148 SMs: two whole waves, only the 56 tail tiles are shared
     p = jev.jev_prefix_suffix_attn_plan(jev.make_attn_desc(128, 4096, 28, 4, 128, 3072, jev.JEV_BF16), 1, 148)
-    assert p["n_tiles"] == 336 or p["n_tiles"] == 352
+    assert p["tile_rows"] == 256 and (p["n_tiles"] == 336 or p["n_tiles"] == 352)
     assert p["full_waves"] == 2 and p["tail0"] == 296 and p["n_ctas"] == 148
     # as many tiles as SMs: one whole tile each, nothing to merge
     p = jev.jev_prefix_suffix_attn_plan(jev.make_attn_desc(1, 512, 4, 4, 128, 9472, jev.JEV_BF16), 1, 148)
