@@ -105,7 +105,7 @@ struct Shared {
 
 template <int D, bool TREE>
 __global__ void __launch_bounds__(kThreads, 1)
-    attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kp,
+    attn_tc1_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kp,
                    const __grid_constant__ CUtensorMap tm_vp, const __grid_constant__ CUtensorMap tm_ks,
                    const __grid_constant__ CUtensorMap tm_vs, const AttnArgs a) {
   using C = Cfg<D>;
@@ -649,7 +649,7 @@ template <int D, bool TREE>
 cudaError_t launch_dt1(const AttnArgs& a, cudaStream_t s) {
   static bool attr = false;
   if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<D, TREE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(attn_tc1_kernel<D, TREE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          Cfg<D>::kSmem);
     if (e != cudaSuccess) return e;
     attr = true;
@@ -666,7 +666,7 @@ cudaError_t launch_dt1(const AttnArgs& a, cudaStream_t s) {
   cfg.stream = s;
   cfg.attrs = pdl;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, attn_tc_kernel<D, TREE>, mq, mkp, mvp, mks, mvs, a);
+  return cudaLaunchKernelEx(&cfg, attn_tc1_kernel<D, TREE>, mq, mkp, mvp, mks, mvs, a);
 }
 
 }  // namespace

@@ -371,7 +371,8 @@ def traffic_of(kernel: str, workload: str, src_files):
 
 
 KERNEL_SRC = {
-    "attn_tc": ["attention_cascade_b200/csrc/attn_tc.cu", "attention_cascade_b200/csrc/common.cuh",
+    "attn_tc": ["attention_cascade_b200/csrc/attn_tc.cu", "attention_cascade_b200/csrc/attn_tc1.cu",
+                "attention_cascade_b200/csrc/attn_tc_common.cuh", "attention_cascade_b200/csrc/common.cuh",
                 "attention_cascade_b200/csrc/tc_ptx.cuh", "attention_cascade_b200/csrc/kernels.h"],
     "attn_simt": ["attention_cascade_b200/csrc/attn_simt.cu", "attention_cascade_b200/csrc/common.cuh"],
 }
