@@ -139,9 +139,9 @@ bool use_tc(const jev_attn_desc* d) {
 // Work plan.  Tensor-core kernel: work tiles of tile_rows stacked rows of one
 // kv group, each with P = ceil(Lp/128) + 1 units (prefix key tiles + the
 // suffix window).  256-row tiles run on the two-Q-tile kernel, which is the
-// faster per unit once there are several waves of tiles; 128-row tiles on the
-// one-Q-tile kernel, chosen when 256-row tiles would not fill one wave of
-// CTAs (twice the tiles, so fewer of them are split and merged).  n_ctas persistent CTAs first take full_waves rounds of whole
+// faster per unit; 128-row tiles on the one-Q-tile kernel, chosen when
+// 256-row tiles would fill less than two thirds of a wave of CTAs (twice the
+// tiles, so fewer of them are split and merged).  n_ctas persistent CTAs first take full_waves rounds of whole
 // tiles; the remaining tail tiles' units are spread evenly over tail_ctas of
 // them, so a tail tile may be split across CTAs and merged afterwards.
 // num_splits: 1 -> no tile split (one CTA per tile up to one per SM),
@@ -189,6 +189,64 @@ double tc_schedule_us(int P, int d, int full_waves, long long U, int tail_ctas, 
   return worst;
 }
 
+// The tensor-core schedule for work tiles of `rows` stacked rows: fills p's
+// tile fields and returns the cost model's estimate (microseconds).
+double tc_plan(Plan& p, const jev_attn_desc* d, int rows, int sms) {
+  const int ktiles = (d->Lp + 127) / 128;
+  p.tile_rows = rows;
+  p.n_mt = (p.M + rows - 1) / rows;
+  p.n_tiles = p.n_mt * d->Hkv;
+  p.n_pre = ktiles;
+  p.P = ktiles + 1;
+  const int s = d->num_splits;
+  // whole tiles only: full_waves rounds over min(n_tiles, sms) CTAs, the
+  // rest one tile to each of the first tail_ctas CTAs
+  auto no_split = [&] {
+    p.n_ctas = std::max(1, std::min(p.n_tiles, sms));
+    p.full_waves = p.n_tiles / p.n_ctas;
+    p.tail0 = p.full_waves * p.n_ctas;
+    p.tail_ctas = std::max(1, p.n_tiles - p.tail0);
+    p.U = (long long)(p.n_tiles - p.tail0) * p.P;
+  };
+  double best = 0.0;
+  if (s == 1 || p.n_tiles == 0) {
+    no_split();
+    best = tc_schedule_us(p.P, d->d, p.full_waves, p.U, p.tail_ctas, rows);
+  } else if (s > 1) {
+    const long long U = (long long)p.n_tiles * p.P;
+    p.full_waves = 0;
+    p.tail0 = 0;
+    p.U = U;
+    p.n_ctas = p.tail_ctas = (int)std::max(1LL, std::min((long long)p.n_tiles * s, U));
+    best = tc_schedule_us(p.P, d->d, 0, U, p.tail_ctas, rows);
+  } else {
+    no_split();
+    best = tc_schedule_us(p.P, d->d, p.full_waves, p.U, p.tail_ctas, rows);
+    // Spread the tail (every tile when there are fewer tiles than SMs)
+    // over more CTAs, up to one per SM; keep the cheapest estimate.
+    const int fw = p.n_tiles >= sms ? p.n_tiles / sms : 0;
+    const int r = p.n_tiles - fw * sms;
+    const long long U = (long long)r * p.P;
+    // a tile spread over many CTAs costs a long merge; keep it within 64 segments
+    const long long t_max = std::min<long long>({(long long)sms, U, (long long)std::max(1, r) * 64});
+    for (long long t = std::max(1, r); r > 0 && t <= t_max; ++t) {
+      const double e = tc_schedule_us(p.P, d->d, fw, U, (int)t, rows);
+      if (e < best * 0.98) {
+        best = e;
+        p.full_waves = fw;
+        p.tail0 = fw * sms;
+        p.U = U;
+        p.tail_ctas = (int)t;
+        p.n_ctas = fw > 0 ? sms : (int)t;
+      }
+    }
+  }
+  p.split = false;
+  for (int c = 1; c < p.tail_ctas && p.U > 0 && !p.split; ++c)
+    if (((long long)c * p.U / p.tail_ctas) % p.P != 0) p.split = true;
+  return best;
+}
+
 // kernel: -1 as the device chooses, 0 CUDA-core, 1 tensor-core; sms <= 0: the device's count
 Plan compute_plan(const jev_attn_desc* d, int T, int kernel, int sms_hint) {
   Plan p{};
@@ -197,57 +255,16 @@ Plan compute_plan(const jev_attn_desc* d, int T, int kernel, int sms_hint) {
   const int ktiles = (d->Lp + 127) / 128;
   p.tc = kernel < 0 ? use_tc(d) : kernel == 1;
   if (p.tc) {
-    const int sms0 = std::max(1, sms_hint > 0 ? sms_hint : num_sms());
-    const int forced_rows = g_tile_rows.load();
-    p.tile_rows = forced_rows ? forced_rows : ((p.M + 255) / 256 * d->Hkv < sms0 ? 128 : 256);
-    p.n_mt = (p.M + p.tile_rows - 1) / p.tile_rows;
-    p.n_tiles = p.n_mt * d->Hkv;
-    p.n_pre = ktiles;
-    p.P = ktiles + 1;
-    const int s = d->num_splits;
     const int sms = std::max(1, sms_hint > 0 ? sms_hint : num_sms());
-    // whole tiles only: full_waves rounds over min(n_tiles, sms) CTAs, the
-    // rest one tile to each of the first tail_ctas CTAs
-    auto no_split = [&] {
-      p.n_ctas = std::max(1, std::min(p.n_tiles, sms));
-      p.full_waves = p.n_tiles / p.n_ctas;
-      p.tail0 = p.full_waves * p.n_ctas;
-      p.tail_ctas = std::max(1, p.n_tiles - p.tail0);
-      p.U = (long long)(p.n_tiles - p.tail0) * p.P;
-    };
-    if (s == 1 || p.n_tiles == 0) {
-      no_split();
-    } else if (s > 1) {
-      const long long U = (long long)p.n_tiles * p.P;
-      p.full_waves = 0;
-      p.tail0 = 0;
-      p.U = U;
-      p.n_ctas = p.tail_ctas = (int)std::max(1LL, std::min((long long)p.n_tiles * s, U));
-    } else {
-      no_split();
-      double best = tc_schedule_us(p.P, d->d, p.full_waves, p.U, p.tail_ctas, p.tile_rows);
-      // Spread the tail (every tile when there are fewer tiles than SMs)
-      // over more CTAs, up to one per SM; keep the cheapest estimate.
-      const int fw = p.n_tiles >= sms ? p.n_tiles / sms : 0;
-      const int r = p.n_tiles - fw * sms;
-      const long long U = (long long)r * p.P;
-      // a tile spread over many CTAs costs a long merge; keep it within 64 segments
-      const long long t_max = std::min<long long>({(long long)sms, U, (long long)std::max(1, r) * 64});
-      for (long long t = std::max(1, r); r > 0 && t <= t_max; ++t) {
-        const double e = tc_schedule_us(p.P, d->d, fw, U, (int)t, p.tile_rows);
-        if (e < best * 0.98) {
-          best = e;
-          p.full_waves = fw;
-          p.tail0 = fw * sms;
-          p.U = U;
-          p.tail_ctas = (int)t;
-          p.n_ctas = fw > 0 ? sms : (int)t;
-        }
-      }
-    }
-    p.split = false;
-    for (int c = 1; c < p.tail_ctas && p.U > 0 && !p.split; ++c)
-      if (((long long)c * p.U / p.tail_ctas) % p.P != 0) p.split = true;
+    // 128-row tiles (the one-Q-tile kernel) when 256-row tiles would fill
+    // less than two thirds of a wave of CTAs.  Timed on B200 with both forced
+    // (attention call, 28 / 4 heads, d = 128): 128-row tiles win at 0.49-0.57
+    // of a wave of 256-row tiles (by 2-22%), tie at 0.65, and lose at 0.92
+    // and from 1.2 waves on (by 5-17%), where the two-Q-tile kernel's lower
+    // cost per row outweighs the split and merge it saves.
+    const int forced_rows = g_tile_rows.load();
+    const int tiles256 = (p.M + 255) / 256 * d->Hkv;
+    tc_plan(p, d, forced_rows ? forced_rows : (3 * tiles256 < 2 * sms ? 128 : 256), sms);
     p.S = 1;
     p.split_len = std::max(1, ktiles) * 128;
     return p;
