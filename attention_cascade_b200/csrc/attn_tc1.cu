@@ -66,11 +66,14 @@ constexpr int kMmaWarp = kSoftWarps + 1;
 constexpr int kQCols = kBN / 4;  // score columns per softmax thread
 constexpr float kLazy = 8.0f;    // log2 headroom before the running max moves
 // Share of softmax exponentials computed on the FMA pipe (every kPolyEvery-th
-// score pair, as one packed f32x2 polynomial; 0 = none).
-#ifndef JEV_POLY_EVERY
-#define JEV_POLY_EVERY 8
+// score pair, as one packed f32x2 polynomial; 0 = none).  Measured on B200,
+// attention call alone: every 16th pair (one of a thread's 16 per key tile)
+// is about 1 us faster than every 8th at the 7B and tree workloads, every
+// 4th about 0.5-1 us slower.
+#ifndef JEV_POLY_EVERY1
+#define JEV_POLY_EVERY1 16
 #endif
-constexpr int kPolyEvery = JEV_POLY_EVERY;
+constexpr int kPolyEvery = JEV_POLY_EVERY1;
 static_assert(kBM == 128, "one TMEM lane per row");
 
 template <int D>
