@@ -140,8 +140,8 @@ bool use_tc(const jev_attn_desc* d) {
 // kv group, each with P = ceil(Lp/128) + 1 units (prefix key tiles + the
 // suffix window).  256-row tiles run on the two-Q-tile kernel, which is the
 // faster per unit; 128-row tiles on the one-Q-tile kernel, chosen when
-// 256-row tiles would fill less than two thirds of a wave of CTAs (twice the
-// tiles, so fewer of them are split and merged).  n_ctas persistent CTAs first take full_waves rounds of whole
+// 256-row tiles would leave little work per CTA (twice the tiles, so fewer of
+// them are split and merged; the rule is at the choice below).  n_ctas persistent CTAs first take full_waves rounds of whole
 // tiles; the remaining tail tiles' units are spread evenly over tail_ctas of
 // them, so a tail tile may be split across CTAs and merged afterwards.
 // num_splits: 1 -> no tile split (one CTA per tile up to one per SM),
@@ -256,15 +256,18 @@ Plan compute_plan(const jev_attn_desc* d, int T, int kernel, int sms_hint) {
   p.tc = kernel < 0 ? use_tc(d) : kernel == 1;
   if (p.tc) {
     const int sms = std::max(1, sms_hint > 0 ? sms_hint : num_sms());
-    // 128-row tiles (the one-Q-tile kernel) when 256-row tiles would fill
-    // less than two thirds of a wave of CTAs.  Timed on B200 with both forced
-    // (attention call, 28 / 4 heads, d = 128): 128-row tiles win at 0.49-0.57
-    // of a wave of 256-row tiles (by 2-22%), tie at 0.65, and lose at 0.92
-    // and from 1.2 waves on (by 5-17%), where the two-Q-tile kernel's lower
-    // cost per row outweighs the split and merge it saves.
+    // 128-row tiles (the one-Q-tile kernel) when 256-row tiles would not fill
+    // a wave of CTAs and their units, spread over the CTAs, come to fewer than
+    // 20 a CTA: there the per-segment costs and the merge weigh most, and the
+    // finer tiles save them; with more work per CTA the two-Q-tile kernel's
+    // lower cost per row wins.  Timed on B200 with both forced (attention
+    // call, 28 / 4 heads, d = 128; 256-row tiles x units per tile / SMs):
+    // 128-row tiles win at 8.3-11.5 units a CTA (by 2-22%), tie at 21.4, and
+    // lose at 59.7 (Lp 8192, 136 tiles) and whenever there is a whole wave.
     const int forced_rows = g_tile_rows.load();
-    const int tiles256 = (p.M + 255) / 256 * d->Hkv;
-    tc_plan(p, d, forced_rows ? forced_rows : (3 * tiles256 < 2 * sms ? 128 : 256), sms);
+    const long long tiles256 = (long long)((p.M + 255) / 256) * d->Hkv;
+    const long long units256 = tiles256 * (ktiles + 1);
+    tc_plan(p, d, forced_rows ? forced_rows : (tiles256 < sms && units256 < 20LL * sms ? 128 : 256), sms);
     p.S = 1;
     p.split_len = std::max(1, ktiles) * 128;
     return p;

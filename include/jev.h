@@ -106,10 +106,10 @@ size_t jev_prefix_suffix_attn_workspace(const jev_attn_desc* desc);
  * tail0 .. n_tiles-1 are spread evenly over CTAs 0 .. tail_ctas-1, CTA c
  * owning [c*tail_units/tail_ctas, (c+1)*tail_units/tail_ctas); split != 0
  * when some tile is shared by several CTAs and a merge kernel combines it.
- * tile_rows is 256 (a kernel with two 128-row Q tiles a CTA) when 256-row
- * tiles fill at least two thirds of a wave of num_sms CTAs, else 128 (a
- * kernel with one Q tile a CTA, for twice as many tiles); 0 for the CUDA-core
- * plan.
+ * tile_rows is 128 (a kernel with one Q tile a CTA, for twice as many
+ * tiles) when 256-row tiles would be fewer than num_sms and their units fewer
+ * than 20 x num_sms, else 256 (a kernel with two 128-row Q tiles a CTA); 0
+ * for the CUDA-core plan.
  * CUDA-core kernel (kernel == 0): simt_splits prefix splits of split_len
  * keys (a multiple of 32).  Returns the descriptor's error (as jev_prefix_suffix_attn would) or
  * JEV_ERR_INVALID_ARG for a NULL `plan` or a kernel outside -1 .. 1.

@@ -111,17 +111,19 @@ def test_schedule_covers_every_unit_once(shape, num_splits, sms, rows, tile_rows
 
 
 def test_tile_rows_choice():
-    """256-row work tiles (the two-Q-tile kernel) when they fill at least two
-    thirds of a wave of CTAs, else 128-row tiles (the one-Q-tile kernel); 0
-    for the CUDA-core plan."""
+    """128-row work tiles (the one-Q-tile kernel) when 256-row tiles would be
+    fewer than the SMs and their units fewer than 20 a CTA, else 256-row tiles
+    (the two-Q-tile kernel); 0 for the CUDA-core plan."""
     def rows(B, Lp, Hq, Hkv, T, sms=148, kernel=1):
         return jev.jev_prefix_suffix_attn_plan(jev.make_attn_desc(B, Lp, Hq, Hkv, 128, T, jev.JEV_BF16), kernel,
                                                sms)["tile_rows"]
     assert rows(128, 4096, 28, 4, 3202) == 256     # 352 tiles of 256 rows
     assert rows(32, 2048, 28, 4, 707) == 128       # 80 tiles of 256 rows on 148 SMs
-    assert rows(32, 2048, 28, 4, 707, sms=120) == 256  # 80 tiles: two thirds of 120
-    assert rows(32, 2048, 28, 4, 707, sms=121) == 128
-    assert rows(48, 8192, 28, 4, 1233) == 256      # 136 tiles: 0.92 of a wave
+    assert rows(32, 2048, 28, 4, 707, sms=80) == 256   # 80 tiles: a whole wave of 80 SMs
+    assert rows(32, 2048, 28, 4, 707, sms=81) == 128   # 1360 units < 20 x 81
+    assert rows(32, 2048, 28, 4, 707, sms=68) == 256   # 1360 units = 20 x 68, and a wave
+    assert rows(48, 8192, 28, 4, 1233) == 256      # 136 tiles of 65 units: 59.7 units a CTA
+    assert rows(80, 2048, 28, 4, 896) == 128       # 100 tiles of 17 units: 11.5 a CTA
     assert rows(8, 1024, 12, 2, 128) == 128
     assert rows(8, 1024, 12, 2, 128, kernel=0) == 0
     with pytest.raises(jev.JevError):
