@@ -186,12 +186,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ahead of V: the MMA thread needs K(x + 1) before it consumes V(x).
     // The whole warp runs this loop (its values stay warp-uniform); one
     // elected lane issues each load.
-    long long kn = 0, vn = 0;  // K and V tiles whose loads this warp has issued
+    // Key-tile counters are 32-bit: a CTA's tiles stay far below 2^32, and the
+    // stage and phase arithmetic (division by the 3 K stages) then costs a few
+    // instructions in warps that share their sub-partition with four busy
+    // softmax warps.
+    uint32_t kn = 0, vn = 0;  // K and V tiles whose loads this warp has issued
     int q_armed = 0;           // Q tiles loaded
     int k = 0;
     bool ok = true;
     if (lane == 0) tma_prefetch_desc(&tm_q);
-    auto load_tile = [&](bool is_k, long long x, const Segment& sg, long long J, bool pre_only) -> bool {
+    auto load_tile = [&](bool is_k, uint32_t x, const Segment& sg, uint32_t J, bool pre_only) -> bool {
       const int ns = is_k ? C::kNK : C::kNV;
       const int st = (int)(x % ns);
       const uint32_t full = (is_k ? B.k_full : B.v_full) + 8 * st;
@@ -228,7 +232,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     pdl_wait();
-    long long J = 0;
+    uint32_t J = 0;
     SegIter it{0, u_begin, u_end};
     int sw, sua, sub;
     bool stail;
@@ -274,11 +278,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       // whose empty-wait gave up was not issued and is not counted: the loop
       // above advances kn / vn only past issued loads.)
       for (int st = 0; st < C::kNK; ++st) {
-        const long long uses = kn > st ? (kn - st + C::kNK - 1) / C::kNK : 0;
+        const uint32_t uses = kn > (uint32_t)st ? (kn - st + C::kNK - 1) / C::kNK : 0;
         if (uses > 0) drain_bar(B.k_full + 8 * st, (uint32_t)((uses - 1) & 1), a.status);
       }
       for (int st = 0; st < C::kNV; ++st) {
-        const long long uses = vn > st ? (vn - st + C::kNV - 1) / C::kNV : 0;
+        const uint32_t uses = vn > (uint32_t)st ? (vn - st + C::kNV - 1) / C::kNV : 0;
         if (uses > 0) drain_bar(B.v_full + 8 * st, (uint32_t)((uses - 1) & 1), a.status);
       }
       if (q_armed > 0) drain_bar(B.q_full, (uint32_t)((q_armed - 1) & 1), a.status);
@@ -296,7 +300,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint64_t dv0 = smem_desc_sw128(sbase + C::kOffV, C::kBlk, 1024);
     // S(x) = Q K(x)^T into score buffer x % 2; its commits release the buffer
     // to the softmax and the K stage to the producer
-    auto issue_s = [&](long long x) {
+    auto issue_s = [&](uint32_t x) {
       const int st = (int)(x % C::kNK), buf = (int)(x & 1);
       const uint64_t ka = dk0 + (uint32_t)((st * C::kKVBytes) >> 4);
 #pragma unroll
@@ -309,7 +313,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_commit_w(B.k_empty + 8 * st);
     };
     // O (+)= P(x) V(x), P read from TMEM where the softmax threads packed it
-    auto issue_pv = [&](long long x, bool acc) {
+    auto issue_pv = [&](uint32_t x, bool acc) {
       const int st = (int)(x % C::kNV), buf = (int)(x & 1);
       const uint64_t va = dv0 + (uint32_t)((st * C::kKVBytes) >> 4);
 #pragma unroll
@@ -319,7 +323,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_commit_w(B.pv_done);
       mma_commit_w(B.v_empty + 8 * st);
     };
-    long long J = 0;
+    uint32_t J = 0;
     int k = 0;
     bool ok = true;
     pdl_wait();
@@ -341,7 +345,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = __shfl_sync(0xffffffffu, probe_wait(B.probe, abort, a.status, a.wait_cycles), 0);
       }
       for (int j = 0; ok && j < n; ++j) {
-        const long long JJ = J + j, JJ1 = JJ + 1;
+        const uint32_t JJ = J + j, JJ1 = JJ + 1;
         // the next tile's scores first: the tensor core computes them while
         // the softmax threads work on this tile
         if (j + 1 < n) {
@@ -392,7 +396,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t s_addr0 = tmem + c_base + lane_off;  // + buffer * kBN: this quarter's scores, then its packed P
     const uint32_t o_addr = tmem + C::kOCol + cq * kQD + lane_off;
     const float sl2 = a.scale_log2;
-    long long J = 0;
+    uint32_t J = 0;
     int k = 0;
     bool ok = true;
     pdl_wait();
@@ -436,7 +440,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // that every thread of the row group meets the same named barriers, and
       // the threads agree on the outcome at the epilogue's reducing barrier.
       for (int j = 0; j < sg.n; ++j) {
-        const long long JJ = J + j;
+        const uint32_t JJ = J + j;
         const int buf = (int)(JJ & 1);
         if (!wait_bar(B.s_full + 8 * buf, (uint32_t)((JJ >> 1) & 1), abort, a.status, a.wait_cycles)) ok = false;
         fence_after_sync();
