@@ -23,9 +23,10 @@
 //               the S/P rows (TMEM lanes 0-127), and the matching halves of O
 //   warps 8-15  Q tile 1, same split
 //   warp 16     TMA producer (Q once per segment, then K/V through a ring of stages)
-//   warp 17     TMEM allocator and tcgen05.mma issuer (one thread)
+//   warp 17     TMEM allocator and tcgen05.mma issuer (the loop runs warp-wide;
+//               an elected lane issues each MMA and commit)
 // TMEM (512 columns): S0/P0 [0,128), S1/P1 [128,256), O0 at 256, O1 at 256+D.
-// Per key tile j the MMA thread issues S_i = Q_i K_j^T (SS form), and after
+// Per key tile j the MMA warp issues S_i = Q_i K_j^T (SS form), and after
 // both halves of tile i have written P_i (bf16, aliasing S_i) it issues
 // O_i += P_i V_j with P_i read from TMEM (TS form); tile 0's softmax overlaps
 // tile 1's MMAs and the other way round.  The two halves of a row exchange

@@ -25,9 +25,10 @@
 //               lanes) and score columns 32(w / 4) .. +31 of each key tile, and
 //               output columns (D / 4)(w / 4) .. of O: four threads per row
 //   warp 16     TMA producer (Q once per segment; K and V through two rings)
-//   warp 17     TMEM allocator and tcgen05.mma issuer (one thread)
+//   warp 17     TMEM allocator and tcgen05.mma issuer (the loop runs warp-wide;
+//               an elected lane issues each MMA and commit)
 // TMEM (512 columns): score buffers S0 [0,128) and S1 [128,256), O at 256.
-// Key tile j's scores go to buffer j % 2.  The MMA thread issues S(j+1) =
+// Key tile j's scores go to buffer j % 2.  The MMA warp issues S(j+1) =
 // Q K(j+1)^T (SS form) before it waits for the softmax of tile j, then
 // O += P(j) V(j) (TS form, P(j) bf16 in TMEM, aliasing S(j)), so the softmax
 // of tile j+1 starts as soon as tile j's is done while the tensor core runs
@@ -183,7 +184,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------------------------------------------------------- TMA producer
     // Key tiles are numbered over the CTA's whole run (x); tile x goes to K
     // stage x % kNK and V stage x % kNV.  Inside a segment K runs one tile
-    // ahead of V: the MMA thread needs K(x + 1) before it consumes V(x).
+    // ahead of V: the MMA warp needs K(x + 1) before it consumes V(x).
     // The whole warp runs this loop (its values stay warp-uniform); one
     // elected lane issues each load.
     // Key-tile counters are 32-bit: a CTA's tiles stay far below 2^32, and the
