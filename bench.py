@@ -40,13 +40,52 @@ L2_BYTES = 126 * 1024 * 1024
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
-def peaks():
-    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+def _peak_number(v):
+    """A peak figure as a float: a plain number, or a record holding one under
+    "value", "median" or "mean"; None otherwise."""
+    if isinstance(v, bool):
+        return None
+    if isinstance(v, (int, float)):
+        return float(v) if v > 0 else None
+    if isinstance(v, dict):
+        for k in ("value", "median", "mean"):
+            if k in v:
+                return _peak_number(v[k])
+    return None
+
+
+def peaks(path=None):
+    """Roofline denominators: the measured HBM copy bandwidth (GB/s) and bf16
+    GEMM throughput (TFLOP/s, burst and sustained) of this machine's B200s
+    from MEASURED_PEAKS.json at the repository root, each figure found at the
+    top level or one object down; any figure the file lacks (or no file) takes
+    the fallback value, and the source says which."""
+    p = path or os.path.join(ROOT, "MEASURED_PEAKS.json")
+    d = {}
     if os.path.exists(p):
-        with open(p) as f:
-            d = json.load(f)
-        return d, "measured"
-    return dict(FALLBACK_PEAKS), "fallback"
+        try:
+            with open(p) as f:
+                d = json.load(f)
+        except (OSError, ValueError):
+            d = {}
+    if not isinstance(d, dict):
+        d = {}
+    out, found = dict(FALLBACK_PEAKS), []
+    for key in FALLBACK_PEAKS:
+        v = _peak_number(d.get(key))
+        if v is None:
+            for sub in d.values():
+                if isinstance(sub, dict) and _peak_number(sub.get(key)) is not None:
+                    v = _peak_number(sub.get(key))
+                    break
+        if v is not None:
+            out[key] = v
+            found.append(key)
+    if len(found) == len(FALLBACK_PEAKS):
+        return out, "measured"
+    if found:
+        return out, "measured (" + ", ".join(found) + "), fallback for the rest"
+    return out, "fallback"
 
 
 def host_cores() -> int:

@@ -70,3 +70,27 @@ def test_reference_arm_prints_only_on_rank_0(monkeypatch):
     with redirect_stdout(buf):
         bench.reference_arm(Args, "qwen2vl_2b")
     assert buf.getvalue() == ""
+
+
+def test_peaks_read_flat_nested_partial_and_missing_files(tmp_path):
+    """The roofline denominators come from the measured-peaks file whatever
+    its shape (figures at the top level, one object down, or as records with
+    a value); figures it lacks, and a missing or unreadable file, take the
+    fallback values, and the source says which."""
+    import json
+    sys.path.insert(0, ROOT)
+    import bench
+    p = tmp_path / "peaks.json"
+    p.write_text(json.dumps({"hbm_gbs": 7000.5, "bf16_tflops": 1650.6, "bf16_tflops_sustained": 1354.2}))
+    pk, src = bench.peaks(str(p))
+    assert src == "measured" and pk == {"hbm_gbs": 7000.5, "bf16_tflops": 1650.6, "bf16_tflops_sustained": 1354.2}
+    p.write_text(json.dumps({"gpu": {"hbm_gbs": {"value": 7001}, "bf16_tflops": 1600}, "clocks": [1965]}))
+    pk, src = bench.peaks(str(p))
+    assert pk["hbm_gbs"] == 7001.0 and pk["bf16_tflops"] == 1600.0
+    assert pk["bf16_tflops_sustained"] == bench.FALLBACK_PEAKS["bf16_tflops_sustained"]
+    assert src.startswith("measured (hbm_gbs, bf16_tflops)") and "fallback" in src
+    p.write_text("{not json")
+    assert bench.peaks(str(p)) == (bench.FALLBACK_PEAKS, "fallback")
+    assert bench.peaks(str(tmp_path / "absent.json")) == (bench.FALLBACK_PEAKS, "fallback")
+    p.write_text(json.dumps({"hbm_gbs": 0, "bf16_tflops": True}))
+    assert bench.peaks(str(p)) == (bench.FALLBACK_PEAKS, "fallback")
