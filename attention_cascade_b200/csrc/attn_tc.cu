@@ -266,7 +266,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Shared-memory descriptors are formed once; an operand's descriptor is a
     // base plus its byte offset >> 4 in the address field (every operand lies
     // below 256 KB of shared memory, so the 14-bit field never carries), so
-    // the one issuing thread spends a couple of instructions per MMA.
+    // each MMA costs the warp's loop a couple of instructions.
     const uint64_t dq0 = smem_desc_sw128(sbase, 16, 1024);
     const uint64_t dk0 = smem_desc_sw128(sbase + C::kOffK, 16, 1024);
     const uint64_t dv0 = smem_desc_sw128(sbase + C::kOffV, C::kBlk, 1024);
