@@ -22,7 +22,7 @@ from __future__ import annotations
 import ctypes as C
 import os
 import subprocess
-from typing import Optional, Sequence
+from typing import Optional
 
 import numpy as np
 

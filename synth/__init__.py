@@ -25,7 +25,7 @@ patterns; fp32 tensors are returned as ``float32``.
 from __future__ import annotations
 
 from dataclasses import dataclass, field
-from typing import Dict, List, Optional
+from typing import List, Optional
 
 import numpy as np
 

@@ -5,7 +5,6 @@ at the same time, and every result equals, bit for bit, the same call run
 alone."""
 import threading
 
-import numpy as np
 import pytest
 import torch
 

@@ -17,7 +17,7 @@ import torch
 
 import oracle
 import synth
-from gpu_helpers import NEAR_TIE, TOL, check_attn, check_readout, compact_lm_head, dev, host_f64
+from gpu_helpers import TOL, check_attn, check_readout, compact_lm_head, dev, host_f64
 
 pytestmark = pytest.mark.gpu
 

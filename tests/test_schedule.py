@@ -6,7 +6,6 @@ units) and which partial slot it writes, and how the merge kernel finds the
 segments of a split tile.  Every (tile, unit) must be computed exactly once,
 every split tile merged from exactly the slots its CTAs wrote, and no slot
 may fall outside the workspace's two partial rows per CTA."""
-import itertools
 
 import numpy as np
 
