@@ -26,6 +26,7 @@ The full-vocabulary LSE kernel (vocab_lse.cu: TMA ring, MMA warp, statistics
 threads releasing the TMEM tile) is modelled the same way at the end.
 """
 import random
+import sys
 
 import pytest
 
@@ -192,6 +193,20 @@ PATTERNS = [[17, 9], [17, 8, 1], [3, 1, 2], [1, 1, 1, 1], [2, 1, 1, 3], [4, 1, 4
 def test_protocol_has_no_stall_or_aliased_wait(segs, prefetch):
     for seed in range(150):
         msg = run(segs, early_release=False, seed=seed, prefetch=prefetch)
+        assert msg is None, f"seed {seed}: {msg}"
+
+
+@pytest.mark.parametrize("segs", PATTERNS, ids=["-".join(map(str, p)) for p in PATTERNS])
+def test_protocol_with_the_d64_ring(segs, monkeypatch):
+    # at d = 64 the kernel keeps 4 K/V stages: a deeper ring, the same protocol,
+    # on the normal path and on the timeout path
+    monkeypatch.setattr(sys.modules[__name__], "NS", 4)
+    for prefetch in (False, True):
+        for seed in range(60):
+            msg = run(segs, early_release=False, seed=seed, prefetch=prefetch)
+            assert msg is None, f"seed {seed}: {msg}"
+    for seed in range(60):
+        msg = run_abort(segs, drain=True, seed=seed)
         assert msg is None, f"seed {seed}: {msg}"
 
 

@@ -37,6 +37,8 @@ the two-Q-tile kernel's model (test_pipeline_protocol.py).
 """
 import random
 
+import sys
+
 import pytest
 
 from test_pipeline_protocol import Bar, _async_run, _wait_problem
@@ -228,6 +230,24 @@ PATTERNS = [[17, 9], [17, 8, 1], [3, 1, 2], [1, 1, 1, 1], [2, 1, 1, 3], [4, 1, 4
 def test_protocol_has_no_stall_or_aliased_wait(segs, prefetch):
     for seed in range(150):
         msg = run(segs, early_release=False, seed=seed, prefetch=prefetch)
+        assert msg is None, f"seed {seed}: {msg}"
+
+
+@pytest.mark.parametrize("segs", PATTERNS, ids=["-".join(map(str, p)) for p in PATTERNS])
+def test_protocol_with_the_d64_rings(segs, monkeypatch):
+    # at d = 64 the kernel keeps 6 K and 5 V stages: deeper rings, the same protocol,
+    # on the normal path and on the timeout path
+    monkeypatch.setattr(sys.modules[__name__], "NK", 6)
+    monkeypatch.setattr(sys.modules[__name__], "NV", 5)
+    for prefetch in (False, True):
+        for seed in range(60):
+            msg = run(segs, early_release=False, seed=seed, prefetch=prefetch)
+            assert msg is None, f"seed {seed}: {msg}"
+        order = list(_loads(segs, prefetch))
+        assert [x for kind, x in order if kind == "k"] == list(range(sum(segs)))
+        assert [x for kind, x in order if kind == "v"] == list(range(sum(segs)))
+    for seed in range(60):
+        msg = run_abort(segs, drain=True, seed=seed)
         assert msg is None, f"seed {seed}: {msg}"
 
 
